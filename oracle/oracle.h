@@ -1,0 +1,124 @@
+/*
+ * oracle.h -- plain single-threaded CPU oracle for the ternary routed-expert
+ * MoE hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link,
+ * load or call this code; only the test suite, the package smoke check and the
+ * benchmark's timed CPU-baseline leg use it.  It shares no source, header,
+ * table or constant with the CUDA library under bit_moe_b200/.
+ *
+ * What it computes, and where each piece comes from:
+ *   - routed-expert weights are ternary values (Parallax 8B kappa article,
+ *     section "Что именно доступно") kept compressed in blocks and multiplied
+ *     against int8-quantized activations (Parakon Runtime README, section
+ *     "How it works"); the block format itself is not printed on any page, so
+ *     it is fixed here as: 256 weights per block, absmean scale rounded to
+ *     fp16, five base-3 digits per byte (52 bytes per block);
+ *   - int8 activations carry one fp32 scale per 32 values (pxq_llama README,
+ *     section "PXQ vs MXFP4": one scale fixup per 32-value block);
+ *   - all top-k experts of a token are evaluated, none dropped
+ *     (llama-modchip page, "Key highlights");
+ *   - the expert FFN is gate/up with a SiLU unary, then down (pxq_llama README,
+ *     "Updates -- 2026-07-28", the up_gate_unary item).
+ * Every other detail is a reading of those passages; each function below says
+ * which.
+ *
+ * Floating point: sums that define a result are taken in fp64; where a float
+ * decides an integer (a scale rounded to fp16, an int8 code, a top-k order)
+ * the decision is taken in the precision stated at that function, which is
+ * the precision the method fixes.  Built with -ffp-contract=off.
+ */
+#ifndef BITMOE_ORACLE_H
+#define BITMOE_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Format constants (see orc_quantize_weights). */
+#define ORC_BLOCK 256       /* weights per ternary block                 */
+#define ORC_BLOCK_WORDS 13  /* 32-bit words of packed digits per block   */
+#define ORC_PANEL 32        /* rows interleaved word by word in storage  */
+#define ORC_QBLOCK 32       /* activations per int8 block                */
+
+/* ---- IEEE binary16 ---------------------------------------------------- */
+/* Round a double to the nearest binary16, ties to even; overflow gives inf. */
+uint16_t orc_f16_from_f64(double x);
+/* Exact widening of a binary16 bit pattern to float. */
+float orc_f16_to_f32(uint16_t h);
+
+/* ---- base-3 byte -------------------------------------------------------- */
+/* Five digits t[0..4] in {0,1,2}, t[0] most significant: v = sum t_i 3^(4-i),
+ * stored as the fixed-point fraction u = ceil(v * 256 / 243).              */
+uint8_t orc_trit_byte_encode(const int t[5]);
+/* Inverse of the above by plain integer arithmetic: v = floor(u*243/256),
+ * then repeated division by 3.  Returns -1 if u encodes no valid v.        */
+int orc_trit_byte_decode(uint8_t u, int t[5]);
+
+/* ---- weight storage ----------------------------------------------------- */
+int64_t orc_trit_words(int64_t rows, int64_t k);   /* rows*(k/256)*13 */
+int64_t orc_scale_count(int64_t rows, int64_t k);  /* rows*(k/256)    */
+/* Index of packed word w (0..12) of block b of row r. */
+int64_t orc_word_index(int64_t k, int64_t r, int64_t b, int w);
+/* Index of the fp16 scale of block b of row r. */
+int64_t orc_scale_index(int64_t k, int64_t r, int64_t b);
+
+/* Quantize w [rows][k] (row-major fp32) to ternary blocks.  Returns 0, or -1
+ * when rows % 32 or k % 256 is nonzero.                                    */
+int orc_quantize_weights(const float* w, int64_t rows, int64_t k,
+                         uint32_t* trits, uint16_t* scales);
+/* Expand rows [row0, row0+nrows) to q [nrows][k] in {-1,0,1} and the fp32
+ * value of each block scale s [nrows][k/256].  Returns 0, or -1 on a bad
+ * shape or an undecodable byte.                                            */
+int orc_unpack_weights(const uint32_t* trits, const uint16_t* scales,
+                       int64_t rows, int64_t k, int64_t row0, int64_t nrows,
+                       int8_t* q, float* s);
+
+/* ---- activations ---------------------------------------------------------- */
+/* x [ntok][k] -> xq [ntok][k] int8, xd [ntok][k/32] fp32.  Returns -1 if
+ * k % 32 != 0.                                                             */
+int orc_quant_act_q8(const float* x, int64_t ntok, int64_t k, int8_t* xq,
+                     float* xd);
+
+/* ---- block sums and mat-vec ----------------------------------------------- */
+/* isum [rows][k/32] = per-32-block int32 dot products of q rows with xq.   */
+void orc_blocksums(const int8_t* q, int64_t rows, int64_t k, const int8_t* xq,
+                   int32_t* isum);
+/* out[r] = sum_b s[r][b] * sum_{j in b} xd[j] * isum[r][j], in fp64.       */
+void orc_matvec(const int8_t* q, const float* s, int64_t rows, int64_t k,
+                const int8_t* xq, const float* xd, double* out);
+
+/* ---- router ------------------------------------------------------------------ */
+/* logits [ntok][E] in fp32, in the fixed evaluation order described at the
+ * definition.  Returns -1 if hidden % 32 != 0.                             */
+int orc_router_logits(const float* x, const float* wr, int64_t ntok,
+                      int64_t hidden, int64_t n_experts, float* logits);
+/* top-k experts by logit (descending, ties to the lower id) and their
+ * softmax weights renormalised over the k selected, in fp64.              */
+int orc_route_topk(const float* x, const float* wr, int64_t ntok,
+                   int64_t hidden, int64_t n_experts, int64_t top_k,
+                   int32_t* idx, double* wts);
+
+/* ---- expert FFN ------------------------------------------------------------- */
+typedef struct {
+  int64_t hidden, ffn, n_experts, top_k;
+  const uint32_t* gate_trits; const uint16_t* gate_scales; /* rows E*ffn, k hidden */
+  const uint32_t* up_trits;   const uint16_t* up_scales;   /* rows E*ffn, k hidden */
+  const uint32_t* down_trits; const uint16_t* down_scales; /* rows E*hidden, k ffn */
+} orc_layer;
+
+/* y [ntok][hidden] (fp64) = sum over slots j (in slot order) of
+ * wts[t][j] * FFN_{idx[t][j]}(x_t).  Optional (may be NULL) debug outputs,
+ * each [ntok][top_k][...]: g and u (fp64, [ffn]), aq (int8, [ffn]) and
+ * ad (fp32, [ffn/32]).  Returns 0, -1 on a bad shape, -2 on an expert id
+ * out of range.                                                           */
+int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
+                   const float* xd, const int32_t* idx, const float* wts,
+                   double* y, double* g_out, double* u_out, int8_t* aq_out,
+                   float* ad_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
