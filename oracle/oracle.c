@@ -194,7 +194,8 @@ int orc_unpack_weights(const uint32_t* trits, const uint16_t* scales,
    "How it works"; pxq_llama README "PXQ vs MXFP4").  Reading of the rounding:
      amax = max |x| over the block, d = amax / 127 (IEEE fp32 division),
      q = clamp(rint(x / d), -127, 127) with IEEE fp32 division and ties to
-     even; a block with amax = 0 gets d = 0 and q = 0.                     */
+     even; a block whose d is 0 (amax = 0, or amax/127 underflowing to 0)
+     gets q = 0.                                                           */
 int orc_quant_act_q8(const float* x, int64_t ntok, int64_t k, int8_t* xq,
                      float* xd) {
   if (k <= 0 || k % ORC_QBLOCK) return -1;
@@ -211,7 +212,7 @@ int orc_quant_act_q8(const float* x, int64_t ntok, int64_t k, int8_t* xq,
       float d = amax / 127.0f;
       xd[t * nq + j] = d;
       for (int i = 0; i < ORC_QBLOCK; ++i) {
-        if (amax == 0.0f) {
+        if (d == 0.0f) { /* amax = 0, or amax/127 below the smallest subnormal */
           qb[i] = 0;
           continue;
         }

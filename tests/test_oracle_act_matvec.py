@@ -44,6 +44,11 @@ def test_q8_ties_to_even_and_zero_block(orc):
     assert xd[0, 0] == 1.0 and xd[0, 1] == 0.0
     assert list(xq[0, 1:7]) == [2, 4, -2, -4, 0, 126]
     assert not xq[0, 32:].any()
+    # amax/127 underflows to 0: the block is treated as the zero block
+    x2 = np.zeros((1, 32), np.float32)
+    x2[0, 3] = np.float32(1e-44)
+    xq2, xd2 = orc.quant_act_q8(x2)
+    assert xd2[0, 0] == 0.0 and not xq2.any()
 
 
 def test_q8_scale_invariance(orc):
