@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Benchmark of the ternary routed-expert MoE hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl bitmoe|reference]
+
+A step is one pass of the whole hot path -- int8 activation quantization,
+router top-k, fused gate+up mat-vec with SwiGLU/requant, down mat-vec with
+the top-k combine -- for one batch of tokens through one MoE layer.  Steps
+rotate through a stack of layers (and a pool of inputs) whose bytes touched
+per rotation exceed twice the L2 size, so every step reads its weights from
+HBM, as a decode through consecutive layers does.  The K timed steps are
+replayed from CUDA graphs; one JSON line is printed by rank 0.
+
+With N > 1 (torchrun), every rank runs an independent replica on its own GPU
+(weak scaling, no collective on the data path); the timed region is bracketed
+by barriers and the max over ranks is reported.
+
+--impl reference times the CPU oracle (single-threaded C) on the host, each
+step being a bounded sample of the same workload (see `run_reference`).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed-expert decode tok/s per MoE layer; achieved HBM GB/s vs 8 TB/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="30b",
+                    help="tiny | 30b | 30b-b16 | large | large-b8 | 30b-prefill")
+    ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------------- bytes
+def matrix_bytes(rows, k):
+    """Packed bytes of a ternary matrix: 52 B of digits + 2 B of scale per 256."""
+    return rows * (k // 256) * 54
+
+
+def kernel_bytes(wl, unique_experts):
+    """Algorithmic bytes per launch of each kernel for one step (each byte
+    counted once: weights of the unique routed experts, activations in, results
+    out)."""
+    T, H, F, E, K = wl.ntok, wl.hidden, wl.ffn, wl.n_experts, wl.top_k
+    pairs = T * K
+    return {
+        "quant_act_q8": T * H * 4 + T * H + T * H // 32 * 4,
+        "router_logits": E * H * 4 + T * H * 4 + T * E * 4,
+        "topk_softmax": T * E * 4 + pairs * 8,
+        "group": pairs * 4 * 3,
+        "gateup": unique_experts * 2 * matrix_bytes(F, H) + T * H + T * H // 32 * 4
+        + pairs * F + pairs * F // 32 * 4 + pairs * 8,
+        "down": unique_experts * matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4
+        + pairs * H * 4 * 2 + T * H * 4 + pairs * 8,
+    }
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every `period` s
+    on a background thread (started before, stopped after the timed region)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_dev, period=0.002):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report what is known
+            self.err = repr(e)
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": getattr(self, "err", "no samples")}
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(s)}
+
+
+# --------------------------------------------------------------------------- traffic
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_moe_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The CPU oracle on the host cores, timed as the step of this workload.
+
+    Each step is a bounded sample of one step of the workload: the oracle's
+    activation quantization and router for one token plus the expert FFN of
+    one of that token's top-k slots (a 1/top_k share of the token's expert
+    work), so K steps stay within minutes.  The rate is reported in tokens/s
+    by counting each step as 1/top_k token."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    import synthetic
+    wl = synthetic.WORKLOADS[args.workload]
+    H, F, K = wl.hidden, wl.ffn, wl.top_k
+    wr = synthetic.router(wl, 0).numpy()
+    n_tok = 8
+    x = synthetic.activations(wl, 0, ntok=n_tok).numpy()
+    idx, wts = oracle.route_topk(x, wr, K)
+    experts = sorted(set(int(e) for e in idx.ravel()))
+    remap = {e: i for i, e in enumerate(experts)}
+    wg = np.concatenate([synthetic.expert_matrix(wl, 0, "gate", e).numpy() for e in experts])
+    wu = np.concatenate([synthetic.expert_matrix(wl, 0, "up", e).numpy() for e in experts])
+    wd = np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in experts])
+    layer = oracle.Layer.from_float(H, F, len(experts), 1, wg, wu, wd)
+
+    def step(j):
+        t, slot = (j // K) % n_tok, j % K
+        xt = x[t:t + 1]
+        xq, xd = oracle.quant_act_q8(xt)
+        i2, w2 = oracle.route_topk(xt, wr, K)
+        e = remap[int(i2[0, slot])]
+        oracle.expert_ffn(layer, xq, xd, np.array([[e]], np.int32),
+                          w2[:, slot:slot + 1].astype(np.float32))
+
+    for j in range(args.warmup):
+        step(j)
+    t0 = time.perf_counter()
+    for j in range(args.steps):
+        step(args.warmup + j)
+    dt = time.perf_counter() - t0
+    value = args.steps / K / dt
+    sample = ("each step: oracle act quant + router for 1 token of %s and the expert FFN of one of "
+              "its %d slots (counted as 1/%d token)" % (wl.describe(), K, K))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl, None),
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+def workload_config(wl, layers):
+    c = {"workload": wl.describe(), "hidden": wl.hidden, "expert_ffn": wl.ffn,
+         "experts": wl.n_experts, "top_k": wl.top_k, "tokens_per_step": wl.ntok,
+         "weights": "ternary absmean 256-blocks (52 B base-3 + fp16 scale), N(0,%g)" % wl.w_std,
+         "activations": "x ~ N(0,1) fp32, int8 32-blocks"}
+    if layers is not None:
+        c["layer_stack"] = layers
+        c["l2"] = "inputs larger than L2: %d-layer stack rotated per step" % layers
+    return c
+
+
+def stack_size(wl, step_bytes):
+    need = int(math.ceil(2 * L2_BYTES / max(step_bytes, 1)))
+    return max(wl.layers, min(need, 64))
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    """The oracle as it stands, single-threaded, on a bounded sample of steps of
+    this workload: consecutive batches of tokens (decode batches of the
+    workload's size; 8-token chunks for prefill) until about `budget_s` of CPU
+    time.  Packing the routed experts' weights is set-up and not timed."""
+    import numpy as np
+    import oracle
+    import synthetic
+    H, F, K = wl.hidden, wl.ffn, wl.top_k
+    chunk = wl.ntok if wl.ntok <= 64 else 8
+    wr = synthetic.router(wl, 0).numpy()
+    x = synthetic.activations(wl, 0, ntok=64).numpy()
+    n, tot = 0, 0.0
+    while tot < budget_s and n + chunk <= 64:
+        toks = x[n:n + chunk]
+        idx, _ = oracle.route_topk(toks, wr, K)
+        e_used = sorted(set(int(e) for e in idx.ravel()))
+        layer = oracle.Layer.from_float(
+            H, F, len(e_used), K,
+            np.concatenate([synthetic.expert_matrix(wl, 0, "gate", e).numpy() for e in e_used]),
+            np.concatenate([synthetic.expert_matrix(wl, 0, "up", e).numpy() for e in e_used]),
+            np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in e_used]))
+        remap = np.full(wl.n_experts, -1, np.int32)
+        remap[e_used] = np.arange(len(e_used))
+        t0 = time.perf_counter()
+        xq, xd = oracle.quant_act_q8(toks)
+        i2, w2 = oracle.route_topk(toks, wr, K)
+        oracle.expert_ffn(layer, xq, xd, remap[i2], w2.astype(np.float32))
+        tot += time.perf_counter() - t0
+        n += chunk
+    return {"value": n / tot, "unit": "tok/s", "cores": 1, "kind": "oracle",
+            "sample": "%d tokens in batches of %d of %s (layer 0), oracle single-threaded, "
+                      "weight packing untimed" % (n, chunk, wl.describe())}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    rank, world, local = dist_env()
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import bit_moe_b200 as B
+    import synthetic
+    from bit_moe_b200 import build
+    from bit_moe_b200.layers import quantize_layer
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    wl = synthetic.WORKLOADS[args.workload]
+    T, H, K = wl.ntok, wl.hidden, wl.top_k
+    dev = torch.device("cuda", local)
+    seed_off = 1000 * rank  # each replica draws its own layers and inputs
+
+    # ---- layer stack and inputs, resident in HBM
+    per_step_guess = (min(wl.n_experts, T * K) * wl.expert_bytes) + wl.n_experts * H * 4
+    L = stack_size(wl, per_step_guess)
+    layers, routers = [], []
+    for l in range(L):
+        fn = lambda role, e, l=l: synthetic.expert_matrix(wl, seed_off + l, role, e, dev)  # noqa: E731
+        layers.append(quantize_layer(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, fn))
+        routers.append(synthetic.router(wl, seed_off + l, dev))
+    NX = 64
+    xs = [synthetic.activations(wl, seed_off + j, device=dev) for j in range(NX)]
+    ws = B.Workspace.for_layer(layers[0], T)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step(j):
+        B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
+
+    # routing of every (layer, input) combination a step uses: unique experts
+    uniq = []
+    for j in range(min(L * NX, 256)):
+        idx, _ = B.moe_route_topk(xs[j % NX], routers[j % L], K)
+        uniq.append(len(set(idx.flatten().tolist())))
+    unique_experts = sum(uniq) / len(uniq)
+
+    # ---- warm-up (eager), then capture the step sequence as CUDA graphs
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize()
+    status = B.moe_check_status(ws)
+    if status != 0:
+        raise SystemExit("device status %d after warm-up" % status)
+    G = min(args.steps, 4 * L)
+    stream = torch.cuda.Stream(device=dev)
+
+    def capture(n_steps, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            step(first)  # make sure the stream has run the path once
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(n_steps):
+                    step(first + j)
+        return g
+
+    g_main = capture(G, args.warmup)
+    rem = args.steps % G
+    g_rem = capture(rem, args.warmup) if rem else None
+    reps = args.steps // G
+    launches_per_step = None
+    c0 = B.moe_launch_count()
+    step(0)
+    launches_per_step = B.moe_launch_count() - c0
+    torch.cuda.synchronize()
+    g_main.replay()  # untimed warm replay
+    torch.cuda.synchronize()
+
+    # ---- timed region
+    sampler = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g_main.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = B.moe_check_status(ws)
+    if status != 0:
+        raise SystemExit("device status %d after the timed region" % status)
+    tokens = world * T * args.steps
+    value = tokens / (ms / 1e3)
+
+    # ---- per-kernel times: the same steps as a traced graph (events after each kernel)
+    n_tr = min(G, 2 * L)
+    tr = B.KernelTrace(capacity=n_tr * launches_per_step + 8)
+    gt = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        stream.synchronize()
+        with torch.cuda.graph(gt, stream=stream):
+            with tr:
+                for j in range(n_tr):
+                    step(args.warmup + j)
+    per_kernel = {}
+    for _ in range(5):
+        gt.replay()
+        torch.cuda.synchronize()
+        for name, v in tr.durations().items():
+            per_kernel.setdefault(name, []).extend(v)
+    kb = kernel_bytes(wl, unique_experts)
+    total_ms = sum(sum(v) for v in per_kernel.values())
+    shares = {n: {"avg_us": 1e3 * sum(v) / len(v), "share": sum(v) / total_ms,
+                  "launches": len(v)} for n, v in per_kernel.items()}
+    dom = max(shares, key=lambda n: shares[n]["share"])
+    peak, peak_kind = measured_peaks()
+    avg_s = shares[dom]["avg_us"] / 1e6
+    achieved = kb.get(dom, 0) / avg_s / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": kb.get(dom, 0),
+                "traffic": ncu_traffic(dom, wl.describe())}
+    step_bytes = sum(kb[n] for n in kb if n in shares)
+    step_gbs = step_bytes / (ms / 1e3 / args.steps) / 1e9
+
+    # ---- end to end: the host-buffer entry point, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = min(args.steps, 2000)
+        xh = [xs[j % NX].cpu().pin_memory() for j in range(min(NX, n_e2e))]
+        yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
+        with torch.cuda.stream(stream):
+            for j in range(5):
+                B.moe_forward_host(layers[j % L], routers[j % L], xh[j % len(xh)], yh, ws, stream=stream)
+            stream.synchronize()
+            if world > 1:
+                dist.barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for j in range(n_e2e):
+                B.moe_forward_host(layers[j % L], routers[j % L], xh[j % len(xh)], yh, ws, stream=stream)
+            a1.record(stream)
+            stream.synchronize()
+        e_ms = a0.elapsed_time(a1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * T * n_e2e / (e_ms / 1e3), "unit": "tok/s",
+               "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4,
+               "steps": n_e2e, "api": "moe_forward_host"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
+            "data": "synthetic", "config": workload_config(wl, L),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary(),
+            "step_hbm_gbs": step_gbs, "unique_experts_per_step": unique_experts,
+            "kernels": shares,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del g_main, g_rem, gt
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,385 @@
+// api.cu -- the extern "C" entry points of libbitmoe: argument validation,
+// workspace layout, and the launch sequence of each call.
+#include <cstring>
+
+#include "bitmoe.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "quant.cuh"
+#include "router.cuh"
+
+namespace bitmoe {
+
+static thread_local char g_last_error[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+static thread_local int64_t g_launches = 0;
+static thread_local cudaEvent_t* g_trace_events = nullptr;
+static thread_local int g_trace_cap = 0;
+static thread_local int g_trace_n = 0;
+static thread_local int g_trace_ids[4096];
+
+void note_launch(int kernel_id, cudaStream_t stream) {
+  ++g_launches;
+  if (g_trace_events && g_trace_n < g_trace_cap && g_trace_n < 4096) {
+    cudaEventRecord(g_trace_events[g_trace_n], stream);
+    g_trace_ids[g_trace_n++] = kernel_id;
+  }
+}
+
+int check_launch(const char* what) {
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+  return MOE_OK;
+}
+
+int check_device() {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(MOE_ERR_DEVICE, "device %d is sm_%d%d; libbitmoe runs on sm_100 (B200) only", dev,
+                major, minor);
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- workspace
+struct WsLayout {
+  size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0, xs = 0, ys = 0;
+  GroupWs grp;
+  size_t total = 0;
+};
+
+static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
+  WsLayout L;
+  size_t off = kWsHeaderBytes;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.logits = take(sizeof(float) * T * static_cast<size_t>(E));
+  L.xq = take(static_cast<size_t>(T) * H);
+  L.xd = take(sizeof(float) * T * static_cast<size_t>(H / kQBlock));
+  L.idx = take(sizeof(int32_t) * T * static_cast<size_t>(K));
+  L.wts = take(sizeof(float) * T * static_cast<size_t>(K));
+  L.aq = take(static_cast<size_t>(T) * K * F);
+  L.ad = take(sizeof(float) * T * static_cast<size_t>(K) * (F / kQBlock));
+  L.ye = take(sizeof(float) * T * static_cast<size_t>(K) * H);
+  L.cnt = take(sizeof(int32_t) * T * static_cast<size_t>(H / kPanel));
+  L.xs = take(sizeof(float) * T * static_cast<size_t>(H));
+  L.ys = take(sizeof(float) * T * static_cast<size_t>(H));
+  off = group_ws_layout(E, T * K, off, &L.grp);
+  (void)prefill;
+  L.total = off;
+  return L;
+}
+
+static int check_layer(const moe_layer* L) {
+  if (!L) return fail(MOE_ERR_INVALID_ARG, "layer is NULL");
+  const int H = L->hidden, F = L->ffn, E = L->n_experts, K = L->top_k;
+  if (H <= 0 || F <= 0 || E <= 0 || K <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "layer sizes must be positive (hidden %d ffn %d E %d k %d)", H, F,
+                E, K);
+  if (K > E) return fail(MOE_ERR_INVALID_ARG, "top_k %d > n_experts %d", K, E);
+  if (H % kBlock || F % kBlock)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "hidden %d and ffn %d must be multiples of 256", H, F);
+  if (H > kMaxHidden || F > kMaxFfn || E > kMaxExperts || K > kMaxTopK)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                "limits: hidden <= %d, ffn <= %d, n_experts <= %d, top_k <= %d", kMaxHidden, kMaxFfn,
+                kMaxExperts, kMaxTopK);
+  const moe_tmat* m[3] = {&L->gate, &L->up, &L->down};
+  const char* names[3] = {"gate", "up", "down"};
+  for (int i = 0; i < 3; ++i) {
+    const int rows = i < 2 ? E * F : E * H, k = i < 2 ? H : F;
+    if (m[i]->rows != rows || m[i]->k != k)
+      return fail(MOE_ERR_INVALID_ARG, "%s is [%d][%d], expected [%d][%d]", names[i], m[i]->rows,
+                  m[i]->k, rows, k);
+    if (!m[i]->trits || !m[i]->scales) return fail(MOE_ERR_INVALID_ARG, "%s has a NULL pointer", names[i]);
+    if (!aligned16(m[i]->trits) || !aligned16(m[i]->scales))
+      return fail(MOE_ERR_ALIGNMENT, "%s pointers must be 16-byte aligned", names[i]);
+  }
+  return MOE_OK;
+}
+
+template <typename... Ps>
+static int check_ptrs(const char* what, Ps... ps) {
+  const void* arr[] = {static_cast<const void*>(ps)...};
+  for (const void* p : arr) {
+    if (!p) return fail(MOE_ERR_INVALID_ARG, "%s: NULL pointer argument", what);
+    if (!aligned16(p)) return fail(MOE_ERR_ALIGNMENT, "%s: pointers must be 16-byte aligned", what);
+  }
+  return MOE_OK;
+}
+
+static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, const float* xd,
+                                const int32_t* idx, const float* wts, float* y, void* ws,
+                                const WsLayout& W) {
+  DecodeParams P;
+  P.hidden = L->hidden; P.ffn = L->ffn; P.n_experts = L->n_experts; P.top_k = L->top_k;
+  P.ntok = ntok;
+  P.gate_trits = L->gate.trits; P.gate_scales = L->gate.scales;
+  P.up_trits = L->up.trits;     P.up_scales = L->up.scales;
+  P.down_trits = L->down.trits; P.down_scales = L->down.scales;
+  P.xq = xq; P.xd = xd; P.idx = idx; P.wts = wts; P.y = y;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  P.aq = reinterpret_cast<int8_t*>(base + W.aq);
+  P.ad = reinterpret_cast<float*>(base + W.ad);
+  P.ye = reinterpret_cast<float*>(base + W.ye);
+  P.cnt = reinterpret_cast<int32_t*>(base + W.cnt);
+  P.status = &reinterpret_cast<WsHeader*>(ws)->status;
+  P.direct = ntok == 1;
+  P.items = reinterpret_cast<const Item*>(base + W.grp.items);
+  P.n_items = reinterpret_cast<const int32_t*>(base + W.grp.n_items);
+  P.pairs = reinterpret_cast<const int32_t*>(base + W.grp.pairs);
+  P.group_scratch = reinterpret_cast<int32_t*>(base + W.grp.scratch);
+  return P;
+}
+
+// Decode: one token runs the slots directly; more tokens are grouped by expert.
+static int launch_decode(const DecodeParams& P, cudaStream_t stream) {
+  if (!P.direct) {
+    int rc = launch_group(P, stream);
+    if (rc) return rc;
+  }
+  return launch_ffn(P, stream);
+}
+
+}  // namespace bitmoe
+
+using namespace bitmoe;
+
+extern "C" {
+
+size_t moe_trit_words(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(k / kBlock) * kBlockWords;
+}
+
+size_t moe_scale_count(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(k / kBlock);
+}
+
+size_t moe_workspace_bytes(const moe_layer* L, int32_t ntok, int32_t prefill) {
+  if (check_layer(L) != MOE_OK || ntok <= 0) return 0;
+  return ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill != 0).total;
+}
+
+size_t moe_route_workspace_bytes(int32_t ntok, int32_t n_experts) {
+  if (ntok <= 0 || n_experts <= 0) return 0;
+  return kWsHeaderBytes + align_up(sizeof(float) * static_cast<size_t>(ntok) * n_experts, 256);
+}
+
+int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ws || ws_bytes < kWsHeaderBytes) return fail(MOE_ERR_INVALID_ARG, "workspace too small or NULL");
+  if (!aligned16(ws)) return fail(MOE_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  int rc = check_device();
+  if (rc) return rc;
+  cudaError_t err = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(err));
+  return MOE_OK;
+}
+
+int moe_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits, uint16_t* scales,
+                         moe_stream_t stream) {
+  int rc = check_ptrs("quantize_weights", w, trits, scales);
+  if (rc) return rc;
+  if (rows <= 0 || k <= 0) return fail(MOE_ERR_INVALID_ARG, "quantize_weights: rows, k must be > 0");
+  if (rows % kPanel || k % kBlock)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quantize_weights: rows %% 32 and k %% 256 must be 0");
+  if ((rc = check_device())) return rc;
+  return launch_quantize_weights(w, rows, k, trits, scales, static_cast<cudaStream_t>(stream));
+}
+
+int moe_quant_act_q8(const float* x, int32_t ntok, int32_t k, int8_t* xq, float* xd,
+                     moe_stream_t stream) {
+  int rc = check_ptrs("quant_act_q8", x, xq, xd);
+  if (rc) return rc;
+  if (ntok <= 0 || k <= 0) return fail(MOE_ERR_INVALID_ARG, "quant_act_q8: ntok, k must be > 0");
+  if (k % kQBlock || k > 65536 || ntok > (1 << 24))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quant_act_q8: k %% 32 == 0, k <= 65536, ntok <= 2^24");
+  if ((rc = check_device())) return rc;
+  return launch_quant_act_q8(x, ntok, k, xq, xd, static_cast<cudaStream_t>(stream));
+}
+
+int moe_route_topk(const float* x, const float* w_router, int32_t ntok, int32_t hidden,
+                   int32_t n_experts, int32_t top_k, int32_t* idx, float* wts, void* ws,
+                   size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_ptrs("route_topk", x, w_router, idx, wts, ws);
+  if (rc) return rc;
+  if (ntok <= 0 || hidden <= 0 || n_experts <= 0 || top_k <= 0 || top_k > n_experts)
+    return fail(MOE_ERR_INVALID_ARG, "route_topk: need positive sizes and top_k <= n_experts");
+  if (hidden % kBlock || hidden > kMaxHidden || n_experts > kMaxExperts || top_k > kMaxTopK ||
+      ntok > 65536)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "route_topk: shape outside the documented limits");
+  if (ws_bytes < moe_route_workspace_bytes(ntok, n_experts))
+    return fail(MOE_ERR_WORKSPACE, "route_topk: workspace %zu < %zu bytes", ws_bytes,
+                moe_route_workspace_bytes(ntok, n_experts));
+  if ((rc = check_device())) return rc;
+  float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kWsHeaderBytes);
+  return launch_route_topk(x, w_router, ntok, hidden, n_experts, top_k, idx, wts, logits,
+                           static_cast<cudaStream_t>(stream));
+}
+
+static int ffn_common(const char* what, const moe_layer* L, int32_t ntok, const int8_t* xq,
+                      const float* xd, const int32_t* idx, const float* wts, float* y, void* ws,
+                      size_t ws_bytes, bool prefill, WsLayout* W) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if ((rc = check_ptrs(what, xq, xd, idx, wts, y, ws))) return rc;
+  if (ntok <= 0) return fail(MOE_ERR_INVALID_ARG, "%s: ntok must be > 0", what);
+  if (!prefill && ntok > kMaxDecodeTokens)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: decode takes at most %d tokens", what, kMaxDecodeTokens);
+  if (prefill && ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: ntok <= 65536", what);
+  *W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
+  if (ws_bytes < W->total)
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace %zu < %zu bytes", what, ws_bytes, W->total);
+  return check_device();
+}
+
+int moe_expert_ffn_decode(const moe_layer* L, int32_t ntok, const int8_t* xq, const float* xd,
+                          const int32_t* idx, const float* wts, float* y, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  WsLayout W;
+  int rc = ffn_common("expert_ffn_decode", L, ntok, xq, xd, idx, wts, y, ws, ws_bytes, false, &W);
+  if (rc) return rc;
+  DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
+  return launch_decode(P, static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_ffn_prefill(const moe_layer* L, int32_t ntok, const int8_t* xq, const float* xd,
+                           const int32_t* idx, const float* wts, float* y, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  WsLayout W;
+  int rc = ffn_common("expert_ffn_prefill", L, ntok, xq, xd, idx, wts, y, ws, ws_bytes, true, &W);
+  if (rc) return rc;
+  DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
+  return launch_prefill(P, static_cast<cudaStream_t>(stream));
+}
+
+int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const float* x, float* y,
+                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if ((rc = check_ptrs("forward", w_router, x, y, ws))) return rc;
+  if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: 1 <= ntok <= 65536");
+  const bool prefill = ntok > kMaxDecodeTokens;
+  WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
+  if (ws_bytes < W.total) return fail(MOE_ERR_WORKSPACE, "forward: workspace %zu < %zu bytes", ws_bytes, W.total);
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  int8_t* xq = reinterpret_cast<int8_t*>(base + W.xq);
+  float* xd = reinterpret_cast<float*>(base + W.xd);
+  int32_t* idx = reinterpret_cast<int32_t*>(base + W.idx);
+  float* wts = reinterpret_cast<float*>(base + W.wts);
+  float* logits = reinterpret_cast<float*>(base + W.logits);
+  if ((rc = launch_quant_act_q8(x, ntok, L->hidden, xq, xd, s))) return rc;
+  if ((rc = launch_route_topk(x, w_router, ntok, L->hidden, L->n_experts, L->top_k, idx, wts, logits, s)))
+    return rc;
+  DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
+  if (prefill) return launch_prefill(P, s);
+  return launch_decode(P, s);
+}
+
+int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, const float* x_host,
+                     float* y_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if (!x_host || !y_host) return fail(MOE_ERR_INVALID_ARG, "forward_host: NULL host buffer");
+  if ((rc = check_ptrs("forward_host", w_router, ws))) return rc;
+  if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward_host: 1 <= ntok <= 65536");
+  const bool prefill = ntok > kMaxDecodeTokens;
+  WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
+  if (ws_bytes < W.total)
+    return fail(MOE_ERR_WORKSPACE, "forward_host: workspace %zu < %zu bytes", ws_bytes, W.total);
+  if ((rc = check_device())) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  float* xs = reinterpret_cast<float*>(base + W.xs);
+  float* ys = reinterpret_cast<float*>(base + W.ys);
+  const size_t bytes = sizeof(float) * static_cast<size_t>(ntok) * L->hidden;
+  cudaError_t err = cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, s);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy in: %s", cudaGetErrorString(err));
+  if ((rc = moe_forward(L, w_router, ntok, xs, ys, ws, ws_bytes, stream))) return rc;
+  err = cudaMemcpyAsync(y_host, ys, bytes, cudaMemcpyDeviceToHost, s);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy out: %s", cudaGetErrorString(err));
+  return MOE_OK;
+}
+
+int moe_check_status(void* ws, moe_stream_t stream) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "check_status: NULL workspace");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t status = 0;
+  cudaError_t err = cudaMemcpyAsync(&status, ws, sizeof(status), cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, sizeof(int32_t), s);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "check_status: %s", cudaGetErrorString(err));
+  if (status) set_error("device reported status %d", status);
+  return status;
+}
+
+const char* moe_last_error(void) { return g_last_error; }
+
+int64_t moe_launch_count(void) { return g_launches; }
+
+int moe_trace_begin(void* const* events, int32_t capacity) {
+  if (!events || capacity <= 0) return fail(MOE_ERR_INVALID_ARG, "trace_begin: no events");
+  g_trace_events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+  g_trace_cap = capacity;
+  g_trace_n = 0;
+  return MOE_OK;
+}
+
+int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
+  const int n = g_trace_n;
+  if (kernel_ids)
+    for (int i = 0; i < n && i < capacity; ++i) kernel_ids[i] = g_trace_ids[i];
+  g_trace_events = nullptr;
+  g_trace_cap = 0;
+  g_trace_n = 0;
+  return n;
+}
+
+const char* moe_kernel_name(int32_t id) {
+  static const char* names[MOE_K_COUNT] = {
+      "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down"};
+  return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
+}
+
+int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const float* xd, float* out,
+                     int32_t* isum, moe_stream_t stream) {
+  if (!m) return fail(MOE_ERR_INVALID_ARG, "debug_matvec: NULL matrix");
+  int rc = check_ptrs("debug_matvec", m->trits, m->scales, xq, xd, out);
+  if (rc) return rc;
+  if (isum && !aligned16(isum)) return fail(MOE_ERR_ALIGNMENT, "debug_matvec: isum not aligned");
+  if (ntok <= 0 || ntok > kMaxDecodeTokens || m->rows <= 0 || m->k <= 0)
+    return fail(MOE_ERR_INVALID_ARG, "debug_matvec: bad sizes");
+  if (m->rows % kPanel || m->k % kBlock || m->k > kMaxHidden)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "debug_matvec: rows %% 32, k %% 256, k <= %d", kMaxHidden);
+  if ((rc = check_device())) return rc;
+  return launch_debug_matvec(m, ntok, xq, xd, out, isum, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// common.cuh -- shared host/device helpers of libbitmoe (sm_100a only).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "bitmoe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ != 1000)
+#error "libbitmoe is written for sm_100a only"
+#endif
+
+namespace bitmoe {
+
+constexpr int kBlock = 256;      // weights per ternary block
+constexpr int kBlockWords = 13;  // packed uint32 words per block
+constexpr int kPanel = 32;       // rows per interleaved panel
+constexpr int kQBlock = 32;      // activations per int8 block
+constexpr int kSubPerBlock = kBlock / kQBlock;  // 8 activation blocks per weight block
+
+constexpr int kMaxHidden = 16384;
+constexpr int kMaxFfn = 8192;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxDecodeTokens = 64;
+constexpr int kMaxDynSmem = 227 * 1024;  // opt-in dynamic shared memory per CTA
+
+// Workspace header: the first 256 bytes hold the device status word.
+struct WsHeader {
+  int32_t status;    // first error code seen by a kernel (0 = ok)
+  int32_t pad[63];
+};
+constexpr size_t kWsHeaderBytes = sizeof(WsHeader);
+
+// ---------------------------------------------------------------- host errors
+void set_error(const char* fmt, ...);
+int fail(int code, const char* fmt, ...);
+int check_launch(const char* what);
+int check_device();
+
+// Called after every kernel launch: counts it and, while tracing, records an
+// event on its stream.
+void note_launch(int kernel_id, cudaStream_t stream);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- device helpers
+__device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
+  atomicCAS(status, 0, code);
+}
+
+// fp64 -> binary16, round to nearest even, in one conversion.
+__device__ __forceinline__ uint16_t f64_to_f16_rn(double x) {
+  uint16_t h;
+  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(h) : "d"(x));
+  return h;
+}
+
+__device__ __forceinline__ float f16_bits_to_f32(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// Streaming 32-bit load that does not allocate in L1 (weights are read once).
+__device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+  return v;
+}
+
+}  // namespace bitmoe

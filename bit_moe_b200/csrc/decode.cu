@@ -1,0 +1,382 @@
+// decode.cu -- expert FFN on CUDA cores: fused gate+up mat-vec with a SwiGLU
+// and int8 requantization epilogue, then the down mat-vec with the weighted
+// top-k combine (sm_100a).
+//
+// Parakon Runtime README, "How it works": decode uses fused mat-vec kernels
+// that read the quantized blocks directly from VRAM and accumulate against
+// int8-quantized activations.  pxq_llama README, "Updates -- 2026-07-28": gate
+// and up are computed together with the SiLU unary; "What's PXQ?": gate/up
+// fusion, K-split decode and a grouped-MoE path.
+//
+// Work is cut into items: up to kChunk (token, slot) pairs routed to the same
+// expert.  With one token every slot is its own item (direct mode); with more
+// tokens a grouping pass collects the pairs of each expert so that the
+// expert's weights stream from HBM once per step and every decoded digit word
+// serves all pairs of the item.
+#include <cub/block/block_scan.cuh>
+
+#include "bitmoe.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "ternary_dot.cuh"
+
+namespace bitmoe {
+
+size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G) {
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  G->items = take(sizeof(Item) * static_cast<size_t>(npairs));
+  G->n_items = take(sizeof(int32_t));
+  G->pairs = take(sizeof(int32_t) * static_cast<size_t>(npairs));
+  G->scratch = take(sizeof(int32_t) * 2 * static_cast<size_t>(E + 1));
+  return off;
+}
+
+// ---------------------------------------------------------------------------
+// Grouping (S6): count the pairs of each expert, scan, cut each expert's pairs
+// into items of at most kChunk, and scatter the pair ids.  Ids outside
+// [0, E) form one extra group with expert -1 (their outputs are zero).
+// One CTA of 1024 threads.
+// ---------------------------------------------------------------------------
+constexpr int kGroupThreads = 1024;
+
+__global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
+  using Scan = cub::BlockScan<int, kGroupThreads>;
+  __shared__ typename Scan::TempStorage scan_tmp;
+  __shared__ int cnt[kMaxExperts + 1];
+  __shared__ int off[kMaxExperts + 1];
+  __shared__ int fill[kMaxExperts + 1];
+  const int E = P.n_experts, npairs = P.ntok * P.top_k, tid = threadIdx.x;
+  for (int e = tid; e <= E; e += kGroupThreads) { cnt[e] = 0; fill[e] = 0; }
+  __syncthreads();
+  for (int p = tid; p < npairs; p += kGroupThreads) {
+    int e = P.idx[p];
+    if (e < 0 || e >= E) { record_status(P.status, MOE_ERR_BAD_INDEX); e = E; }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  // groups 0..E handled two per thread (E + 1 <= 2 * kGroupThreads)
+  int c[2], ic[2], o[2], io[2];
+  for (int r = 0; r < 2; ++r) {
+    const int e = 2 * tid + r;
+    c[r] = e <= E ? cnt[e] : 0;
+    ic[r] = (c[r] + kChunk - 1) / kChunk;
+  }
+  int tot_c = 0, tot_i = 0;
+  Scan(scan_tmp).ExclusiveSum(c[0] + c[1], o[0], tot_c);
+  __syncthreads();
+  Scan(scan_tmp).ExclusiveSum(ic[0] + ic[1], io[0], tot_i);
+  o[1] = o[0] + c[0];
+  io[1] = io[0] + ic[0];
+  Item* items = const_cast<Item*>(P.items);
+  for (int r = 0; r < 2; ++r) {
+    const int e = 2 * tid + r;
+    if (e > E) continue;
+    off[e] = o[r];
+    for (int i = 0; i < ic[r]; ++i) {
+      Item it;
+      it.expert = e == E ? -1 : e;
+      it.start = o[r] + i * kChunk;
+      it.count = min(kChunk, c[r] - i * kChunk);
+      it.pad = 0;
+      items[io[r] + i] = it;
+    }
+  }
+  if (tid == 0) *const_cast<int32_t*>(P.n_items) = tot_i;
+  __syncthreads();
+  int32_t* pairs = const_cast<int32_t*>(P.pairs);
+  for (int p = tid; p < npairs; p += kGroupThreads) {
+    int e = P.idx[p];
+    if (e < 0 || e >= E) e = E;
+    pairs[off[e] + atomicAdd(&fill[e], 1)] = p;
+  }
+}
+
+// Fetch work item `it`; returns false when there is none.
+__device__ __forceinline__ bool fetch_item(const DecodeParams& P, int it, Item& item) {
+  if (P.direct) {
+    if (it >= P.ntok * P.top_k) return false;
+    const int e = P.idx[it];
+    item.expert = (e >= 0 && e < P.n_experts) ? e : -1;
+    item.start = it;
+    item.count = 1;
+    return true;
+  }
+  if (it >= *P.n_items) return false;
+  item = P.items[it];
+  return true;
+}
+
+__device__ __forceinline__ int item_pair(const DecodeParams& P, const Item& item, int n) {
+  return P.direct ? item.start + n : P.pairs[item.start + n];
+}
+
+// ---------------------------------------------------------------------------
+// S3 + S4: gate and up of one item for one 32-row panel of the ffn dimension.
+// The 8 warps split the 256-blocks of the hidden dimension; the per-warp
+// partial rows are summed in warp order; warp n then applies SwiGLU to pair
+// n's 32 rows and requantizes them (one 32-block of a) to int8.
+// grid: (ffn/32, items), block: kGateUpWarps*32.
+// ---------------------------------------------------------------------------
+template <int NT>
+__device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& item, int panel,
+                                           unsigned char* smem) {
+  const int H = P.hidden, F = P.ffn;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int* q4 = reinterpret_cast<int*>(smem);
+  float* d = reinterpret_cast<float*>(q4 + (H / 4) * NT);
+  int* as = reinterpret_cast<int*>(d + (H / kQBlock) * NT);
+  float* red = reinterpret_cast<float*>(as + (H / kQBlock) * NT);  // [2][warps][NT][32]
+  for (int n = 0; n < NT; ++n) {
+    if (n < item.count) {
+      const int t = item_pair(P, item, n) / P.top_k;
+      stage_act<NT>(P.xq + static_cast<size_t>(t) * H, P.xd + static_cast<size_t>(t) * (H / kQBlock),
+                    H, n, q4, d, as, threadIdx.x, blockDim.x);
+    } else {
+      zero_act<NT>(H, n, q4, d, as, threadIdx.x, blockDim.x);
+    }
+  }
+  __syncthreads();
+  const int nb = H / kBlock;
+  const size_t pb0 = (static_cast<size_t>(item.expert) * (F / kPanel) + panel) * nb;
+  const uint32_t* const tw[2] = {P.gate_trits + pb0 * kBlockWords * kPanel + lane,
+                                 P.up_trits + pb0 * kBlockWords * kPanel + lane};
+  const uint16_t* const ts[2] = {P.gate_scales + pb0 * kPanel + lane, P.up_scales + pb0 * kPanel + lane};
+  float out[2][NT];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) out[m][n] = 0.f;
+  panel_dot<2, NT>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, out);
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) red[((m * kGateUpWarps + warp) * NT + n) * 32 + lane] = out[m][n];
+  __syncthreads();
+  if (warp < item.count) {
+    const int n = warp;
+    float g = 0.f, u = 0.f;
+    for (int w = 0; w < kGateUpWarps; ++w) {
+      g = __fadd_rn(g, red[((0 * kGateUpWarps + w) * NT + n) * 32 + lane]);
+      u = __fadd_rn(u, red[((1 * kGateUpWarps + w) * NT + n) * 32 + lane]);
+    }
+    const float a = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
+    const float amax = warp_max(fabsf(a));
+    const float dd = __fdiv_rn(amax, 127.f);
+    int q = 0;
+    if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
+    const int pair = item_pair(P, item, n);
+    P.aq[static_cast<size_t>(pair) * F + panel * kPanel + lane] = static_cast<int8_t>(q);
+    if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + panel] = dd;
+  }
+}
+
+template <int NTMAX>
+__global__ void __launch_bounds__(kGateUpWarps * 32) k_gateup(DecodeParams P) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  Item item;
+  if (!fetch_item(P, blockIdx.y, item)) return;
+  const int panel = blockIdx.x;
+  if (item.expert < 0) {
+    if (threadIdx.x == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < item.count) {
+      const int pair = item_pair(P, item, warp);
+      P.aq[static_cast<size_t>(pair) * P.ffn + panel * kPanel + lane] = 0;
+      if (lane == 0) P.ad[static_cast<size_t>(pair) * (P.ffn / kQBlock) + panel] = 0.f;
+    }
+    return;
+  }
+  if constexpr (NTMAX == 1) {
+    gateup_run<1>(P, item, panel, smem);
+  } else {
+    if (item.count <= 1) gateup_run<1>(P, item, panel, smem);
+    else if (item.count <= 2) gateup_run<2>(P, item, panel, smem);
+    else if (item.count <= 4) gateup_run<4>(P, item, panel, smem);
+    else gateup_run<8>(P, item, panel, smem);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// S5: down mat-vec of one item for kDownWarps 32-row panels of the hidden
+// dimension (one panel per warp), written per pair to ye; the CTA that
+// completes the last of a token's top_k slots for a panel combines
+// y[t] = sum_j wts[t][j] * ye[t][j] over the slots in order.
+// grid: (hidden/32/kDownWarps, items), block: kDownWarps*32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void arrive_and_combine(const DecodeParams& P, int pair, int panel,
+                                                   int lane) {
+  const int K = P.top_k, H = P.hidden;
+  const int t = pair / K;
+  int32_t* c = P.cnt + static_cast<size_t>(t) * (H / kPanel) + panel;
+  int old = 0;
+  if (lane == 0) old = atomicAdd(c, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old == K - 1) {
+    __threadfence();
+    float y = 0.f;
+    const float* ye = P.ye + static_cast<size_t>(t) * K * H + panel * kPanel + lane;
+    for (int j = 0; j < K; ++j)
+      y = __fmaf_rn(__ldcg(P.wts + static_cast<size_t>(t) * K + j), __ldcg(ye + static_cast<size_t>(j) * H), y);
+    P.y[static_cast<size_t>(t) * H + panel * kPanel + lane] = y;
+    if (lane == 0) atomicExch(c, 0);
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item, int pgroup,
+                                         unsigned char* smem) {
+  const int H = P.hidden, F = P.ffn;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int* q4 = reinterpret_cast<int*>(smem);
+  float* d = reinterpret_cast<float*>(q4 + (F / 4) * NT);
+  int* as = reinterpret_cast<int*>(d + (F / kQBlock) * NT);
+  for (int n = 0; n < NT; ++n) {
+    if (n < item.count) {
+      const int pair = item_pair(P, item, n);
+      stage_act<NT>(P.aq + static_cast<size_t>(pair) * F, P.ad + static_cast<size_t>(pair) * (F / kQBlock),
+                    F, n, q4, d, as, threadIdx.x, blockDim.x);
+    } else {
+      zero_act<NT>(F, n, q4, d, as, threadIdx.x, blockDim.x);
+    }
+  }
+  __syncthreads();
+  const int panel = pgroup * kDownWarps + warp;
+  const int nb = F / kBlock;
+  const size_t pb0 = (static_cast<size_t>(item.expert) * (H / kPanel) + panel) * nb;
+  const uint32_t* const tw[1] = {P.down_trits + pb0 * kBlockWords * kPanel + lane};
+  const uint16_t* const ts[1] = {P.down_scales + pb0 * kPanel + lane};
+  float out[1][NT];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) out[0][n] = 0.f;
+  panel_dot<1, NT>(tw, ts, 0, nb, 1, q4, d, as, out);
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+    if (n < item.count)
+      P.ye[static_cast<size_t>(item_pair(P, item, n)) * H + panel * kPanel + lane] = out[0][n];
+  __threadfence();
+  __syncwarp();
+  for (int n = 0; n < item.count; ++n) arrive_and_combine(P, item_pair(P, item, n), panel, lane);
+}
+
+template <int NTMAX>
+__global__ void __launch_bounds__(kDownWarps * 32) k_down(DecodeParams P) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  Item item;
+  if (!fetch_item(P, blockIdx.y, item)) return;
+  const int pgroup = blockIdx.x;
+  if (item.expert < 0) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int panel = pgroup * kDownWarps + warp;
+    for (int n = 0; n < item.count; ++n)
+      P.ye[static_cast<size_t>(item_pair(P, item, n)) * P.hidden + panel * kPanel + lane] = 0.f;
+    __threadfence();
+    __syncwarp();
+    for (int n = 0; n < item.count; ++n) arrive_and_combine(P, item_pair(P, item, n), panel, lane);
+    return;
+  }
+  if constexpr (NTMAX == 1) {
+    down_run<1>(P, item, pgroup, smem);
+  } else {
+    if (item.count <= 1) down_run<1>(P, item, pgroup, smem);
+    else if (item.count <= 2) down_run<2>(P, item, pgroup, smem);
+    else if (item.count <= 4) down_run<4>(P, item, pgroup, smem);
+    else down_run<8>(P, item, pgroup, smem);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Test hook: the mat-vec core on one matrix, with the exact block sums.
+// grid: (rows/32, ntok), block: kGateUpWarps*32; warps split the blocks.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kGateUpWarps * 32)
+    k_debug_matvec(const uint32_t* __restrict__ trits, const uint16_t* __restrict__ scales, int rows,
+                   int k, const int8_t* __restrict__ xq, const float* __restrict__ xd,
+                   float* __restrict__ out, int32_t* __restrict__ isum) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* q4 = reinterpret_cast<int*>(smem);
+  float* d = reinterpret_cast<float*>(q4 + k / 4);
+  int* as = reinterpret_cast<int*>(d + k / kQBlock);
+  float* red = reinterpret_cast<float*>(as + k / kQBlock);
+  const int panel = blockIdx.x, t = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  stage_act<1>(xq + static_cast<size_t>(t) * k, xd + static_cast<size_t>(t) * (k / kQBlock), k, 0, q4,
+               d, as, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int nb = k / kBlock;
+  const int r = panel * kPanel + lane;
+  const size_t pb0 = static_cast<size_t>(panel) * nb;
+  const uint32_t* const tw[1] = {trits + pb0 * kBlockWords * kPanel + lane};
+  const uint16_t* const ts[1] = {scales + pb0 * kPanel + lane};
+  float o[1][1] = {{0.f}};
+  int32_t* isum_row = isum ? isum + (static_cast<size_t>(t) * rows + r) * (k / kQBlock) : nullptr;
+  panel_dot<1, 1>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, o, isum_row, 0);
+  red[warp * 32 + lane] = o[0][0];
+  __syncthreads();
+  if (warp == 0) {
+    float acc = 0.f;
+    for (int w = 0; w < kGateUpWarps; ++w) acc = __fadd_rn(acc, red[w * 32 + lane]);
+    out[static_cast<size_t>(t) * rows + r] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+// Raise a kernel's dynamic shared-memory limit to the most any launch uses,
+// once per device (so no attribute call happens inside a stream capture).
+template <typename K>
+static void allow_smem(K kernel) {
+  constexpr int kMaxDev = 64;
+  static bool done[kMaxDev] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < kMaxDev && done[dev]) return;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  if (dev >= 0 && dev < kMaxDev) done[dev] = true;
+}
+
+int launch_group(const DecodeParams& P, cudaStream_t stream) {
+  k_group<<<1, kGroupThreads, 0, stream>>>(P);
+  note_launch(MOE_K_GROUP, stream);
+  return check_launch("group");
+}
+
+int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
+  const int npairs = P.ntok * P.top_k;
+  if (P.direct) {
+    const size_t s1 = ActSmem<1>::bytes(P.hidden) + 2 * kGateUpWarps * 1 * 32 * 4;
+    const size_t s2 = ActSmem<1>::bytes(P.ffn);
+    allow_smem(k_gateup<1>);
+    allow_smem(k_down<1>);
+    k_gateup<1><<<dim3(P.ffn / kPanel, npairs), kGateUpWarps * 32, s1, stream>>>(P);
+    note_launch(MOE_K_GATEUP, stream);
+    k_down<1><<<dim3(P.hidden / kPanel / kDownWarps, npairs), kDownWarps * 32, s2, stream>>>(P);
+    note_launch(MOE_K_DOWN, stream);
+  } else {
+    const size_t s1 = ActSmem<kChunk>::bytes(P.hidden) + 2 * kGateUpWarps * kChunk * 32 * 4;
+    const size_t s2 = ActSmem<kChunk>::bytes(P.ffn);
+    allow_smem(k_gateup<kChunk>);
+    allow_smem(k_down<kChunk>);
+    k_gateup<kChunk><<<dim3(P.ffn / kPanel, npairs), kGateUpWarps * 32, s1, stream>>>(P);
+    note_launch(MOE_K_GATEUP, stream);
+    k_down<kChunk><<<dim3(P.hidden / kPanel / kDownWarps, npairs), kDownWarps * 32, s2, stream>>>(P);
+    note_launch(MOE_K_DOWN, stream);
+  }
+  return check_launch("expert_ffn");
+}
+
+int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const float* xd, float* out,
+                        int32_t* isum, cudaStream_t stream) {
+  const size_t s = ActSmem<1>::bytes(m->k) + kGateUpWarps * 32 * 4;
+  allow_smem(k_debug_matvec);
+  k_debug_matvec<<<dim3(m->rows / kPanel, ntok), kGateUpWarps * 32, s, stream>>>(
+      m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
+  note_launch(MOE_K_DEBUG_MATVEC, stream);
+  return check_launch("debug_matvec");
+}
+
+}  // namespace bitmoe

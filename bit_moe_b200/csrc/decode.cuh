@@ -1,0 +1,51 @@
+// decode.cuh -- parameters and launchers of the expert-FFN mat-vec kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace bitmoe {
+
+constexpr int kGateUpWarps = 8;  // warps of a gate/up CTA; they split the hidden blocks
+constexpr int kDownWarps = 4;    // warps (= 32-row panels) of a down CTA
+constexpr int kChunk = 8;        // most (token, slot) pairs sharing one weight decode
+
+// A work item: up to kChunk (token, slot) pairs routed to one expert.
+struct Item {
+  int expert;  // -1: pairs whose expert id was out of range
+  int start;   // first entry in the pair list
+  int count;   // 1..kChunk
+  int pad;
+};
+
+struct DecodeParams {
+  int hidden, ffn, n_experts, top_k, ntok;
+  const uint32_t* gate_trits; const uint16_t* gate_scales;
+  const uint32_t* up_trits;   const uint16_t* up_scales;
+  const uint32_t* down_trits; const uint16_t* down_scales;
+  const int8_t* xq; const float* xd;     // [ntok][hidden], [ntok][hidden/32]
+  const int32_t* idx; const float* wts;  // [ntok][top_k]
+  int8_t* aq; float* ad;                 // [ntok*top_k][ffn], [ntok*top_k][ffn/32]
+  float* ye;                             // [ntok*top_k][hidden] per-pair down outputs
+  int32_t* cnt;                          // [ntok][hidden/32] arrival counters (kept at 0)
+  float* y;                              // [ntok][hidden]
+  int32_t* status;
+  // grouped mode (ntok > 1): items and the pair list, built on the device
+  int direct;                            // 1: item i is pair i (ntok == 1)
+  const Item* items;                     // [ntok*top_k + n_experts]
+  const int32_t* n_items;
+  const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert
+  int32_t* group_scratch;                // [2*(n_experts+1)] counters for the grouping
+};
+
+// Bytes of workspace the grouped mode needs after `off`; writes the offsets.
+struct GroupWs {
+  size_t items = 0, n_items = 0, pairs = 0, scratch = 0;
+};
+size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G);
+
+int launch_group(const DecodeParams& P, cudaStream_t stream);
+int launch_ffn(const DecodeParams& P, cudaStream_t stream);
+int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const float* xd, float* out,
+                        int32_t* isum, cudaStream_t stream);
+
+}  // namespace bitmoe

@@ -1,0 +1,121 @@
+// quant.cu -- S0 ternary weight quantization and S1 int8 activation
+// quantization (sm_100a).
+#include "bitmoe.h"
+#include "common.cuh"
+#include "quant.cuh"
+
+namespace bitmoe {
+
+constexpr int kQuantWarps = 4;
+constexpr int kTileStride = kBlock + 1;  // padded row of the staged tile
+
+// ---------------------------------------------------------------------------
+// S0 (Parallax 8B kappa article, "Что именно доступно": ternary routed-expert
+// weights).  One warp per (panel, block): the 32 rows x 256 weights are staged
+// in shared memory with coalesced loads, then lane r quantizes row r of the
+// panel: s = fp16_rn(sum |w| in fp64, ascending k / 256), q = sign(w) where
+// |w| >= s/2.  The digits are packed five per byte as ceil(v*256/243) and the
+// 13 words of each row are written 128 contiguous bytes per warp store.
+// Every lane does the same sequence of operations for its block whatever the
+// grid, so the output does not depend on the launch configuration.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQuantWarps * 32)
+    k_quantize_weights(const float* __restrict__ w, int64_t n_items, int k,
+                       uint32_t* __restrict__ trits, uint16_t* __restrict__ scales) {
+  extern __shared__ __align__(16) float tile_all[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float* tile = tile_all + warp * kPanel * kTileStride;
+  const int nb = k / kBlock;
+  for (int64_t item = static_cast<int64_t>(blockIdx.x) * kQuantWarps + warp; item < n_items;
+       item += static_cast<int64_t>(gridDim.x) * kQuantWarps) {
+    const int64_t p = item / nb;
+    const int b = static_cast<int>(item % nb);
+    for (int r = 0; r < kPanel; ++r) {
+      const float4* src =
+          reinterpret_cast<const float4*>(w + (p * kPanel + r) * static_cast<int64_t>(k) + b * kBlock);
+      const float4 v0 = src[lane], v1 = src[lane + 32];
+      float* dst = tile + r * kTileStride;
+      dst[4 * lane + 0] = v0.x; dst[4 * lane + 1] = v0.y;
+      dst[4 * lane + 2] = v0.z; dst[4 * lane + 3] = v0.w;
+      dst[128 + 4 * lane + 0] = v1.x; dst[128 + 4 * lane + 1] = v1.y;
+      dst[128 + 4 * lane + 2] = v1.z; dst[128 + 4 * lane + 3] = v1.w;
+    }
+    __syncwarp();
+    const float* row = tile + lane * kTileStride;
+    double sum = 0.0;
+    for (int kk = 0; kk < kBlock; ++kk) sum = __dadd_rn(sum, fabs(static_cast<double>(row[kk])));
+    const uint16_t s = f64_to_f16_rn(sum * (1.0 / 256.0));
+    const float half = 0.5f * f16_bits_to_f32(s);
+    scales[item * kPanel + lane] = s;
+#pragma unroll 1
+    for (int j = 0; j < kBlockWords; ++j) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int l = 0; l < 4; ++l) {
+        int v = 0;
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+          const int kk = 20 * j + 4 * i + l;
+          int t = 1;  // pad digit: weight 0
+          if (kk < kBlock) {
+            const float x = row[kk];
+            if (fabsf(x) >= half && x != 0.f) t = x > 0.f ? 2 : 0;
+          }
+          v = 3 * v + t;
+        }
+        const uint32_t u = static_cast<uint32_t>((v * 256 + 242) / 243);
+        word |= u << (8 * l);
+      }
+      trits[(item * kBlockWords + j) * kPanel + lane] = word;
+    }
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// S1 (Parakon Runtime README, "How it works"; pxq_llama README, "PXQ vs MXFP4":
+// one scale per 32 values).  One warp per 32-value block: d = amax/127 and
+// q = clamp(rint(x/d), -127, 127) with IEEE divisions; d = 0 gives q = 0.
+// ---------------------------------------------------------------------------
+__global__ void k_quant_act_q8(const float* __restrict__ x, int64_t nblk, int8_t* __restrict__ xq,
+                               float* __restrict__ xd) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t blk = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       blk < nblk; blk += warps) {
+    const float v = x[blk * kQBlock + lane];
+    const float amax = warp_max(fabsf(v));
+    const float d = __fdiv_rn(amax, 127.f);
+    int q = 0;
+    if (d != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(v, d))));
+    xq[blk * kQBlock + lane] = static_cast<int8_t>(q);
+    if (lane == 0) xd[blk] = d;
+  }
+}
+
+int launch_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,
+                            uint16_t* scales, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(kQuantWarps) * kPanel * kTileStride * sizeof(float);
+  cudaFuncSetAttribute(k_quantize_weights, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(smem));
+  const int64_t n_items = rows / kPanel * (k / kBlock);
+  int64_t grid = (n_items + kQuantWarps - 1) / kQuantWarps;
+  if (grid > 148 * 16) grid = 148 * 16;
+  k_quantize_weights<<<static_cast<unsigned>(grid), kQuantWarps * 32, smem, stream>>>(
+      w, n_items, static_cast<int>(k), trits, scales);
+  note_launch(MOE_K_QUANTIZE_WEIGHTS, stream);
+  return check_launch("quantize_weights");
+}
+
+int launch_quant_act_q8(const float* x, int64_t ntok, int k, int8_t* xq, float* xd,
+                        cudaStream_t stream) {
+  const int64_t nblk = ntok * (k / kQBlock);
+  const int warps_per_cta = 8;
+  int64_t grid = (nblk + warps_per_cta - 1) / warps_per_cta;
+  if (grid > 148 * 8) grid = 148 * 8;
+  k_quant_act_q8<<<static_cast<unsigned>(grid), warps_per_cta * 32, 0, stream>>>(x, nblk, xq, xd);
+  note_launch(MOE_K_QUANT_ACT, stream);
+  return check_launch("quant_act_q8");
+}
+
+}  // namespace bitmoe

@@ -1,0 +1,93 @@
+// router.cu -- S2: router logits in a fixed fp32 order and top-k softmax
+// (sm_100a).
+//
+// llama-modchip page, "Key highlights": every top-k expert of a token is
+// evaluated, with no dropping.  The routing decision is an integer result
+// taken on fp32 logits, so the evaluation order of each logit is fixed: 32
+// partial sums (lane l accumulates fused multiply-adds over k = l, l+32, ...
+// ascending) followed by xor-butterfly additions at distances 16, 8, 4, 2, 1.
+#include "bitmoe.h"
+#include "common.cuh"
+#include "router.cuh"
+
+namespace bitmoe {
+
+// One warp per (token, expert) logit.  The router matrix rows are read once per
+// token by one warp each (coalesced 128-byte loads); many warps run per SM.
+__global__ void k_router_logits(const float* __restrict__ x, const float* __restrict__ wr, int ntok,
+                                int H, int E, float* __restrict__ logits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t total = static_cast<int64_t>(ntok) * E;
+  for (int64_t pair = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       pair < total; pair += nw) {
+    const int t = static_cast<int>(pair / E), e = static_cast<int>(pair % E);
+    const float* xr = x + static_cast<int64_t>(t) * H;
+    const float* wrow = wr + static_cast<int64_t>(e) * H;
+    float p = 0.f;
+#pragma unroll 8
+    for (int k = lane; k < H; k += 32) p = __fmaf_rn(__ldg(wrow + k), __ldg(xr + k), p);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, m));
+    if (lane == 0) logits[pair] = p;
+  }
+}
+
+// One warp per token: top-k by (logit descending, id ascending), then
+// w_i = exp(l_i - l_0) / sum_j exp(l_j - l_0) in fp32, summed in rank order.
+__global__ void k_topk_softmax(const float* __restrict__ logits, int ntok, int E, int K,
+                               int32_t* __restrict__ idx, float* __restrict__ wts) {
+  __shared__ float sel_v[4][kMaxTopK];
+  __shared__ int sel_e[4][kMaxTopK];
+  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const int t = blockIdx.x * 4 + wl;
+  if (t >= ntok) return;
+  const float* lg = logits + static_cast<int64_t>(t) * E;
+  uint32_t used = 0;  // bit i: element lane + 32*i already chosen
+  for (int r = 0; r < K; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+    for (int i = 0; i * 32 + lane < E; ++i) {
+      if (used & (1u << i)) continue;
+      const int e = i * 32 + lane;
+      const float v = lg[e];
+      if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, m);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, m);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if ((be & 31) == lane) used |= 1u << (be >> 5);
+    if (lane == 0) { sel_v[wl][r] = bv; sel_e[wl][r] = be; }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    const float l0 = sel_v[wl][0];
+    float ex[kMaxTopK];
+    float den = 0.f;
+    for (int r = 0; r < K; ++r) {
+      ex[r] = expf(__fsub_rn(sel_v[wl][r], l0));
+      den = __fadd_rn(den, ex[r]);
+    }
+    for (int r = 0; r < K; ++r) {
+      idx[static_cast<int64_t>(t) * K + r] = sel_e[wl][r];
+      wts[static_cast<int64_t>(t) * K + r] = __fdiv_rn(ex[r], den);
+    }
+  }
+}
+
+int launch_route_topk(const float* x, const float* wr, int ntok, int H, int E, int K, int32_t* idx,
+                      float* wts, float* logits, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(ntok) * E;
+  int64_t grid = (total + 7) / 8;
+  if (grid > 148 * 16) grid = 148 * 16;
+  k_router_logits<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, wr, ntok, H, E, logits);
+  note_launch(MOE_K_ROUTER_LOGITS, stream);
+  k_topk_softmax<<<(ntok + 3) / 4, 128, 0, stream>>>(logits, ntok, E, K, idx, wts);
+  note_launch(MOE_K_TOPK, stream);
+  return check_launch("route_topk");
+}
+
+}  // namespace bitmoe

@@ -1,0 +1,27 @@
+"""Packing a whole MoE layer: every expert's fp32 matrices quantized in place
+into one ternary matrix per role (through moe_quantize_weights)."""
+import torch
+
+from . import MoELayer, TernaryMatrix, moe_quantize_weights, scale_count, trit_words
+
+
+def _expert_view(mat, e, rows_per_expert, k):
+    tw, sc = trit_words(rows_per_expert, k), scale_count(rows_per_expert, k)
+    return TernaryMatrix(rows_per_expert, k, mat.trits[e * tw:(e + 1) * tw],
+                         mat.scales[e * sc:(e + 1) * sc])
+
+
+def quantize_layer(hidden, ffn, n_experts, top_k, expert_fn, device="cuda", stream=None):
+    """expert_fn(role, e) -> fp32 CUDA tensor, [ffn][hidden] for "gate"/"up"
+    and [hidden][ffn] for "down".  Experts are quantized one at a time, so the
+    fp32 weights of only one expert are alive at once."""
+    gate = TernaryMatrix.empty(n_experts * ffn, hidden, device)
+    up = TernaryMatrix.empty(n_experts * ffn, hidden, device)
+    down = TernaryMatrix.empty(n_experts * hidden, ffn, device)
+    for e in range(n_experts):
+        for role, mat, rows, k in (("gate", gate, ffn, hidden), ("up", up, ffn, hidden),
+                                   ("down", down, hidden, ffn)):
+            w = expert_fn(role, e)
+            assert w.shape == (rows, k) and w.dtype == torch.float32
+            moe_quantize_weights(w.contiguous(), out=_expert_view(mat, e, rows, k), stream=stream)
+    return MoELayer(hidden, ffn, n_experts, top_k, gate, up, down)

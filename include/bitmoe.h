@@ -1,0 +1,203 @@
+/*
+ * bitmoe.h -- C ABI of libbitmoe.so, the sm_100a (B200) hot path of MoE
+ * routed-expert inference with ternary weights kept compressed in HBM.
+ *
+ * What the library computes (each entry point cites the passage it follows):
+ *   routed-expert weights are ternary (Parallax 8B kappa article, section
+ *   "Что именно доступно"), stay compressed in GPU memory and are never
+ *   expanded to fp16; decode runs fused mat-vecs that read the quantized
+ *   blocks directly and accumulate against int8-quantized activations; large
+ *   batches run a GEMM path (Parakon Runtime README, section "How it works").
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers unless the name ends in _host.  The
+ *     caller allocates and owns every buffer; the library allocates nothing,
+ *     frees nothing, and keeps no state between calls other than a
+ *     thread-local last-error string (moe_last_error).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronize, except moe_check_status.
+ *   - Arguments are validated on the host before any launch: a bad argument
+ *     returns a negative moe_status and launches nothing.  Problems only the
+ *     device can see (an expert id out of range) are recorded in the status
+ *     word at the start of the workspace and reported by moe_check_status;
+ *     the kernels never trap or abort.
+ *   - Device pointers must be 16-byte aligned.  Inputs are assumed finite.
+ *   - The current CUDA device must be a B200 (sm_100); the library is built
+ *     for sm_100a only and has no other code path.
+ *
+ * Storage format of a ternary matrix W [rows][k] (rows % 32 == 0,
+ * k % 256 == 0).  The pages fix no byte layout; this one is chosen for the
+ * decode kernels:
+ *   - blocks of 256 consecutive weights of a row; scale s = fp16(absmean),
+ *     weight q = sign(w) if |w| >= s/2 else 0 (see moe_quantize_weights);
+ *   - 13 little-endian uint32 words per block: byte lane l (0..3) of word j
+ *     (0..12) holds the five base-3 digits t = q + 1 of weights
+ *     k = 20j + 4i + l, i = 0..4, as u = ceil(v * 256 / 243) with
+ *     v = sum_i t_i 3^(4-i); the last word's fifth digit is a pad (t = 1);
+ *   - rows are grouped in panels of 32 whose words interleave row by row:
+ *     word j of block b of row r is trits[((r/32 * nb + b) * 13 + j) * 32 + r%32]
+ *     with nb = k/256; the fp16 scale of block b of row r is
+ *     scales[(r/32 * nb + b) * 32 + r%32].
+ * That is 52 bytes of digits plus a 2-byte scale per 256 weights (1.6875
+ * bits per weight).
+ */
+#ifndef BITMOE_H
+#define BITMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* moe_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,       /* null pointer, non-positive size, k > E ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = -2, /* outside the documented shape limits        */
+  MOE_ERR_ALIGNMENT = -3,         /* a device pointer not 16-byte aligned       */
+  MOE_ERR_WORKSPACE = -4,         /* workspace smaller than moe_workspace_bytes */
+  MOE_ERR_CUDA = -5,              /* a CUDA runtime error (see moe_last_error)  */
+  MOE_ERR_TIMEOUT = -6,           /* a bounded device-side wait ran out         */
+  MOE_ERR_BAD_INDEX = -7,         /* an expert id outside [0, n_experts)        */
+  MOE_ERR_DEVICE = -8             /* the current device is not sm_100           */
+} moe_status;
+
+/* One ternary matrix in the storage format above. */
+typedef struct {
+  int32_t rows;          /* multiple of 32                          */
+  int32_t k;             /* multiple of 256                         */
+  const uint32_t* trits; /* moe_trit_words(rows, k) words, device   */
+  const uint16_t* scales;/* moe_scale_count(rows, k) fp16, device   */
+} moe_tmat;
+
+/* One MoE layer.  Expert e owns rows [e*ffn, (e+1)*ffn) of gate and up
+ * (k = hidden) and rows [e*hidden, (e+1)*hidden) of down (k = ffn).
+ * Limits: hidden and ffn multiples of 256, hidden <= 16384, ffn <= 8192,
+ * 1 <= top_k <= min(n_experts, 32), n_experts <= 1024.                      */
+typedef struct {
+  int32_t hidden, ffn, n_experts, top_k;
+  moe_tmat gate, up, down;
+} moe_layer;
+
+/* ---- sizes ------------------------------------------------------------ */
+size_t moe_trit_words(int64_t rows, int64_t k);  /* rows*(k/256)*13 */
+size_t moe_scale_count(int64_t rows, int64_t k); /* rows*(k/256)    */
+/* Bytes of workspace a decode (prefill = 0) or prefill (prefill = 1) call
+ * of `ntok` tokens, or moe_forward, needs.  0 on invalid arguments.        */
+size_t moe_workspace_bytes(const moe_layer* layer, int32_t ntok, int32_t prefill);
+/* Zero a workspace (status word and counters).  Every workspace must be
+ * initialised once before its first use; calls leave it reusable.         */
+int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- S0: weight quantization (offline; Parallax 8B kappa article,
+ *      "Что именно доступно": ternary routed-expert weights) ------------
+ * w [rows][k] fp32 row-major -> trits, scales in the storage format.  Per
+ * 256-block: s = fp16 round-to-nearest-even of (sum |w| in fp64, ascending
+ * k) / 256; q = sign(w) where |w| >= 0.5*s (in fp32), else 0.  The output
+ * bytes do not depend on the launch configuration.                        */
+int moe_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,
+                         uint16_t* scales, moe_stream_t stream);
+
+/* ---- S1: activation quantization (Parakon Runtime README, "How it works":
+ *      int8-quantized activations; pxq_llama README, "PXQ vs MXFP4": one
+ *      scale per 32-value block) ------------------------------------------
+ * x [ntok][k] fp32 -> xq [ntok][k] int8, xd [ntok][k/32] fp32 with, per 32
+ * values, d = amax/127 and q = clamp(rint(x/d), -127, 127) (IEEE division,
+ * ties to even; a block whose d is 0 gets q = 0).  k % 32 == 0,
+ * k <= 65536, ntok <= 2^24.                                               */
+int moe_quant_act_q8(const float* x, int32_t ntok, int32_t k, int8_t* xq, float* xd,
+                     moe_stream_t stream);
+
+/* ---- S2: router (llama-modchip page, "Key highlights": every top-k expert
+ *      is evaluated, none dropped) ---------------------------------------
+ * logits = w_router [E][hidden] . x_t in fp32 in a fixed order (32 partial
+ * sums over k = l mod 32 ascending with fused multiply-adds, then pairwise
+ * rounds at distances 16, 8, 4, 2, 1); idx [ntok][top_k] = experts by
+ * descending logit, ties to the lower id; wts [ntok][top_k] = softmax over
+ * the selected logits (the full softmax renormalised over the top-k).
+ * ntok <= 65536, hidden % 256 == 0, hidden <= 16384, n_experts <= 1024,
+ * top_k <= min(n_experts, 32).                                            */
+int moe_route_topk(const float* x, const float* w_router, int32_t ntok, int32_t hidden,
+                   int32_t n_experts, int32_t top_k, int32_t* idx, float* wts, void* ws,
+                   size_t ws_bytes, moe_stream_t stream);
+/* Workspace bytes moe_route_topk needs (it keeps the [ntok][E] logits there). */
+size_t moe_route_workspace_bytes(int32_t ntok, int32_t n_experts);
+
+/* ---- S3-S5: expert FFN, decode (Parakon Runtime README, "How it works":
+ *      fused mat-vecs over the compressed blocks against int8 activations;
+ *      pxq_llama README, "Updates -- 2026-07-28": gate/up with the SiLU
+ *      unary) --------------------------------------------------------------
+ * For each token t and slot j (e = idx[t][j]):
+ *   g = Wg_e . x^_t, u = Wu_e . x^_t; a = g / (1 + exp(-g)) * u (fp32);
+ *   (aq, ad) = q8(a) in 32-blocks; y_t = sum_j wts[t][j] * (Wd_e . a^)
+ * summed over the slots in order.  y [ntok][hidden] fp32 is overwritten.
+ * 1 <= ntok <= 64.  An id outside [0, E) sets MOE_ERR_BAD_INDEX in the
+ * workspace status and its slot contributes nothing.                      */
+int moe_expert_ffn_decode(const moe_layer* layer, int32_t ntok, const int8_t* xq,
+                          const float* xd, const int32_t* idx, const float* wts, float* y,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- S7: expert FFN, prefill (Parakon Runtime README, "How it works":
+ *      large batches take a GEMM path over the quantized tiles) -----------
+ * Same result as moe_expert_ffn_decode for any ntok >= 1 (up to rounding
+ * order), computed by grouping the (token, slot) pairs by expert and running
+ * an int8 tensor-core grouped GEMM.  ntok <= 65536.                       */
+int moe_expert_ffn_prefill(const moe_layer* layer, int32_t ntok, const int8_t* xq,
+                           const float* xd, const int32_t* idx, const float* wts, float* y,
+                           void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---- the whole step ------------------------------------------------------
+ * S1 + S2 + (S3-S5 or S7): y [ntok][hidden] = MoE(x [ntok][hidden]).  Uses
+ * the decode path for ntok <= 64 and the prefill path above.  x and y are
+ * device pointers; the quantized x, the routing and the intermediates live
+ * in the workspace.                                                        */
+int moe_forward(const moe_layer* layer, const float* w_router, int32_t ntok, const float* x,
+                float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
+/* The same with x and y in HOST memory (pinned for asynchronous copies):
+ * copies x in, runs moe_forward, copies y out, all on `stream`.  The host
+ * buffers must stay valid until the stream reaches the end of the call.   */
+int moe_forward_host(const moe_layer* layer, const float* w_router, int32_t ntok,
+                     const float* x_host, float* y_host, void* ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+/* ---- status ------------------------------------------------------------- */
+/* Synchronizes `stream`, returns the status recorded in the workspace by
+ * the device (MOE_OK or a negative moe_status) and clears it.             */
+int moe_check_status(void* ws, moe_stream_t stream);
+/* Message of the last failing call on this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* ---- tracing --------------------------------------------------------------
+ * Kernel ids reported by the tracing calls below. */
+typedef enum {
+  MOE_K_QUANTIZE_WEIGHTS = 0, MOE_K_QUANT_ACT = 1, MOE_K_ROUTER_LOGITS = 2, MOE_K_TOPK = 3,
+  MOE_K_GROUP = 4, MOE_K_GATEUP = 5, MOE_K_DOWN = 6, MOE_K_DEBUG_MATVEC = 7,
+  MOE_K_PREFILL_GATEUP = 8, MOE_K_PREFILL_DOWN = 9, MOE_K_COUNT = 10
+} moe_kernel_id;
+/* Number of kernels this thread has launched through the library so far. */
+int64_t moe_launch_count(void);
+/* Start tracing on this thread: after each kernel it launches, the library
+ * records events[n] (caller-created cudaEvent_t handles, timing enabled) on
+ * the kernel's stream and notes the kernel id, until `capacity` events are
+ * used.  moe_trace_end stops tracing, copies the ids of the recorded events
+ * into kernel_ids and returns how many were recorded.                     */
+int moe_trace_begin(void* const* events, int32_t capacity);
+int moe_trace_end(int32_t* kernel_ids, int32_t capacity);
+/* Name of a kernel id ("" if out of range). */
+const char* moe_kernel_name(int32_t id);
+
+/* ---- test hook ------------------------------------------------------------
+ * The decode kernels' mat-vec on one matrix: for tokens t < ntok and rows r
+ * of m, out[t][r] = sum_b s[r][b] * sum_{j in b} xd[t][j] * isum[t][r][j]
+ * (fp32), and, if isum != NULL, the exact int32 block sums
+ * isum[t][r][j] = sum_{k in block j} q[r][k] * xq[t][k].  ntok <= 64.    */
+int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const float* xd,
+                     float* out, int32_t* isum, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITMOE_H */

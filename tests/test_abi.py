@@ -1,0 +1,54 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point that include/bitmoe.h declares, and rejects bad arguments on the host
+before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib():
+    from bit_moe_b200 import build
+    build.build()
+    import bit_moe_b200
+    return bit_moe_b200, bit_moe_b200.lib()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "bitmoe.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_and_binding_agree():
+    import bit_moe_b200
+    assert set(declared_functions()) == set(bit_moe_b200.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    _, L = _lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_host_side_validation_without_device():
+    B, L = _lib()
+    # null pointers are rejected before any device call
+    rc = L.moe_quant_act_q8(None, 1, 256, None, None, None)
+    assert rc == -1
+    assert b"NULL" in L.moe_last_error()
+    # shape limits
+    assert L.moe_trit_words(64, 512) == 64 * 2 * 13
+    assert L.moe_scale_count(64, 512) == 128
+    assert L.moe_route_workspace_bytes(0, 8) == 0
+    lay = B.moe_layer(256, 512, 8, 9, B.moe_tmat(), B.moe_tmat(), B.moe_tmat())
+    assert L.moe_workspace_bytes(ctypes.byref(lay), 1, 0) == 0   # top_k > E
+    lay = B.moe_layer(300, 512, 8, 2, B.moe_tmat(), B.moe_tmat(), B.moe_tmat())
+    assert L.moe_workspace_bytes(ctypes.byref(lay), 1, 0) == 0   # hidden % 256
+    rc = L.moe_check_status(None, None)
+    assert rc == -1
