@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layers in the rotated stack (default: enough to exceed 2x L2)")
     return ap.parse_args()
 
 
@@ -319,7 +321,7 @@ def main():
 
     # ---- layer stack and inputs, resident in HBM
     per_step_guess = (min(wl.n_experts, T * K) * wl.expert_bytes) + wl.n_experts * H * 4
-    L = stack_size(wl, per_step_guess)
+    L = args.layers if args.layers > 0 else stack_size(wl, per_step_guess)
     layers, routers = [], []
     for l in range(L):
         fn = lambda role, e, l=l: synthetic.expert_matrix(wl, seed_off + l, role, e, dev)  # noqa: E731
@@ -401,20 +403,19 @@ def main():
     tokens = world * T * args.steps
     value = tokens / (ms / 1e3)
 
-    # ---- per-kernel times: the same steps as a traced graph (events after each kernel)
+    # ---- per-kernel times: the same steps launched eagerly behind a spin
+    # kernel (so the host has queued them all before the GPU starts them and
+    # they run back to back), with an event after every library kernel
     n_tr = min(G, 2 * L)
-    tr = B.KernelTrace(capacity=n_tr * launches_per_step + 8)
-    gt = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        stream.synchronize()
-        with torch.cuda.graph(gt, stream=stream):
+    per_kernel = {}
+    for _ in range(3):
+        tr = B.KernelTrace(capacity=n_tr * launches_per_step + 8)
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(int(4e7))
             with tr:
                 for j in range(n_tr):
                     step(args.warmup + j)
-    per_kernel = {}
-    for _ in range(5):
-        gt.replay()
-        torch.cuda.synchronize()
+            stream.synchronize()
         for name, v in tr.durations().items():
             per_kernel.setdefault(name, []).extend(v)
     kb = kernel_bytes(wl, unique_experts)
@@ -477,7 +478,7 @@ def main():
         }
         print(json.dumps(line), flush=True)
     if world > 1:
-        del g_main, g_rem, gt
+        del g_main, g_rem
         dist.barrier()
         dist.destroy_process_group()
 

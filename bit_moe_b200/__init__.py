@@ -297,6 +297,9 @@ class KernelTrace:
 
     def __init__(self, capacity=4096):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(capacity)]
+        for e in self.events:  # torch creates the CUDA event on first record
+            e.record()
+        torch.cuda.current_stream().synchronize()
         self.handles = (ctypes.c_void_p * capacity)(*[e.cuda_event for e in self.events])
         self.start = torch.cuda.Event(enable_timing=True)
         self.n = 0

@@ -326,16 +326,22 @@ __global__ void __launch_bounds__(kGateUpWarps * 32)
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-// Raise a kernel's dynamic shared-memory limit to the most any launch uses,
-// once per device (so no attribute call happens inside a stream capture).
-template <typename K>
-static void allow_smem(K kernel) {
+// Raise the dynamic shared-memory limit of every kernel in this file to the
+// opt-in maximum, once per device (so no attribute call happens inside a
+// stream capture).
+static void init_kernel_attrs() {
   constexpr int kMaxDev = 64;
   static bool done[kMaxDev] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < kMaxDev && done[dev]) return;
-  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  const void* kernels[] = {reinterpret_cast<const void*>(&k_gateup<1>),
+                           reinterpret_cast<const void*>(&k_gateup<kChunk>),
+                           reinterpret_cast<const void*>(&k_down<1>),
+                           reinterpret_cast<const void*>(&k_down<kChunk>),
+                           reinterpret_cast<const void*>(&k_debug_matvec)};
+  for (const void* k : kernels)
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
   if (dev >= 0 && dev < kMaxDev) done[dev] = true;
 }
 
@@ -346,12 +352,11 @@ int launch_group(const DecodeParams& P, cudaStream_t stream) {
 }
 
 int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
+  init_kernel_attrs();
   const int npairs = P.ntok * P.top_k;
   if (P.direct) {
     const size_t s1 = ActSmem<1>::bytes(P.hidden) + 2 * kGateUpWarps * 1 * 32 * 4;
     const size_t s2 = ActSmem<1>::bytes(P.ffn);
-    allow_smem(k_gateup<1>);
-    allow_smem(k_down<1>);
     k_gateup<1><<<dim3(P.ffn / kPanel, npairs), kGateUpWarps * 32, s1, stream>>>(P);
     note_launch(MOE_K_GATEUP, stream);
     k_down<1><<<dim3(P.hidden / kPanel / kDownWarps, npairs), kDownWarps * 32, s2, stream>>>(P);
@@ -359,8 +364,6 @@ int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
   } else {
     const size_t s1 = ActSmem<kChunk>::bytes(P.hidden) + 2 * kGateUpWarps * kChunk * 32 * 4;
     const size_t s2 = ActSmem<kChunk>::bytes(P.ffn);
-    allow_smem(k_gateup<kChunk>);
-    allow_smem(k_down<kChunk>);
     k_gateup<kChunk><<<dim3(P.ffn / kPanel, npairs), kGateUpWarps * 32, s1, stream>>>(P);
     note_launch(MOE_K_GATEUP, stream);
     k_down<kChunk><<<dim3(P.hidden / kPanel / kDownWarps, npairs), kDownWarps * 32, s2, stream>>>(P);
@@ -371,8 +374,8 @@ int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
 
 int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const float* xd, float* out,
                         int32_t* isum, cudaStream_t stream) {
+  init_kernel_attrs();
   const size_t s = ActSmem<1>::bytes(m->k) + kGateUpWarps * 32 * 4;
-  allow_smem(k_debug_matvec);
   k_debug_matvec<<<dim3(m->rows / kPanel, ntok), kGateUpWarps * 32, s, stream>>>(
       m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
   note_launch(MOE_K_DEBUG_MATVEC, stream);
