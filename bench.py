@@ -336,13 +336,6 @@ def main():
     def step(j):
         B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
 
-    # routing of every (layer, input) combination a step uses: unique experts
-    uniq = []
-    for j in range(min(L * NX, 256)):
-        idx, _ = B.moe_route_topk(xs[j % NX], routers[j % L], K)
-        uniq.append(len(set(idx.flatten().tolist())))
-    unique_experts = sum(uniq) / len(uniq)
-
     # ---- warm-up (eager), then capture the step sequence as CUDA graphs
     for j in range(args.warmup):
         step(j)
@@ -418,6 +411,12 @@ def main():
             stream.synchronize()
         for name, v in tr.durations().items():
             per_kernel.setdefault(name, []).extend(v)
+    # routing of the (layer, input) combinations the steps use: unique experts
+    uniq = []
+    for j in range(min(L * NX, 256)):
+        idx, _ = B.moe_route_topk(xs[j % NX], routers[j % L], K)
+        uniq.append(len(set(idx.flatten().tolist())))
+    unique_experts = sum(uniq) / len(uniq)
     kb = kernel_bytes(wl, unique_experts)
     total_ms = sum(sum(v) for v in per_kernel.values())
     shares = {n: {"avg_us": 1e3 * sum(v) / len(v), "share": sum(v) / total_ms,
