@@ -33,7 +33,7 @@ EXPORTS = (
     "moe_quantize_weights", "moe_quant_act_q8", "moe_route_topk", "moe_route_workspace_bytes",
     "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_forward", "moe_forward_host",
     "moe_check_status", "moe_last_error", "moe_debug_matvec", "moe_launch_count",
-    "moe_trace_begin", "moe_trace_end", "moe_kernel_name",
+    "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
 )
 
 
@@ -86,6 +86,7 @@ def lib():
             "moe_trace_begin": (ctypes.c_int, [p, i32]),
             "moe_trace_end": (ctypes.c_int, [p, i32]),
             "moe_kernel_name": (ctypes.c_char_p, [i32]),
+            "moe_expert_ffn_decode_static": (ctypes.c_int, [p, i32, p, p, p, p, p, p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -233,6 +234,20 @@ def _ffn(fn, layer, xq, xd, idx, wts, ws, y, stream):
 
 def moe_expert_ffn_decode(layer, xq, xd, idx, wts, ws, y=None, stream=None):
     return _ffn(lib().moe_expert_ffn_decode, layer, xq, xd, idx, wts, ws, y, stream)
+
+
+def moe_expert_ffn_decode_static(layer, xq, xd, idx, wts, y=None, stream=None):
+    """Decode FFN for callers that cannot allocate device memory: no workspace
+    argument; the library's own fixed 4 MiB device scratch is used instead
+    (see include/bitmoe.h for its limits)."""
+    ntok = xq.shape[0]
+    if y is None:
+        y = torch.empty((ntok, layer.hidden), dtype=torch.float32, device=xq.device)
+    _check(lib().moe_expert_ffn_decode_static(
+        layer.c_ref(), ntok, _dev(xq, torch.int8, "xq"), _dev(xd, torch.float32, "xd"),
+        _dev(idx, torch.int32, "idx"), _dev(wts, torch.float32, "wts"),
+        _dev(y, torch.float32, "y"), _stream(stream)))
+    return y
 
 
 def moe_expert_ffn_prefill(layer, xq, xd, idx, wts, ws, y=None, stream=None):

@@ -140,6 +140,28 @@ int moe_expert_ffn_decode(const moe_layer* layer, int32_t ntok, const int8_t* xq
                           const float* xd, const int32_t* idx, const float* wts, float* y,
                           void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* ---- decode without a caller workspace ---------------------------------------
+ * No counterpart on the pages this library follows: an addition for callers
+ * that cannot allocate device memory at call time (a plug-in whose host
+ * application owns every device allocation, a serving loop that must never
+ * enter the CUDA allocator, code held to a device-memory budget fixed at
+ * start-up).  Same computation and arguments as moe_expert_ffn_decode, minus
+ * the workspace: the scratch is a 4 MiB array inside this library, reserved
+ * on every GPU that loads the library and held until the process exits.
+ *   - A call that needs more scratch than that
+ *     (moe_workspace_bytes(layer, ntok, 0) > 4 MiB) returns
+ *     MOE_ERR_WORKSPACE and launches nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call clears and reuses the same array, so two calls whose work
+ *     can overlap on the GPU (other streams, other host threads) race; keep
+ *     them ordered on one stream.
+ *   - Expert ids outside [0, E) contribute nothing and are not reported.
+ *   - It allocates and frees nothing.                                      */
+int moe_expert_ffn_decode_static(const moe_layer* layer, int32_t ntok, const int8_t* xq,
+                                 const float* xd, const int32_t* idx, const float* wts, float* y,
+                                 moe_stream_t stream);
+
 /* ---- S7: expert FFN, prefill (Parakon Runtime README, "How it works":
  *      large batches take a GEMM path over the quantized tiles) -----------
  * Same result as moe_expert_ffn_decode for any ntok >= 1 (up to rounding
