@@ -80,6 +80,7 @@ def kernel_bytes(wl, unique_experts):
     T, H, F, E, K = wl.ntok, wl.hidden, wl.ffn, wl.n_experts, wl.top_k
     pairs = T * K
     return {
+        "route": E * H * 4 + T * H * 4 + T * H + T * H // 32 * 4 + T * E * 4 + pairs * 8,
         "quant_act_q8": T * H * 4 + T * H + T * H // 32 * 4,
         "router_logits": E * H * 4 + T * H * 4 + T * E * 4,
         "topk_softmax": T * E * 4 + pairs * 8,

@@ -5,6 +5,7 @@
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode2.cuh"
 #include "prefill.cuh"
 #include "quant.cuh"
 #include "router.cuh"
@@ -154,13 +155,45 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   return P;
 }
 
-// Decode: one token runs the slots directly; more tokens are grouped by expert.
-static int launch_decode(const DecodeParams& P, cudaStream_t stream) {
+static int sm_count() {
+  constexpr int kMaxDev = 64;
+  static int cache[kMaxDev] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < kMaxDev && cache[dev]) return cache[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev >= 0 && dev < kMaxDev) cache[dev] = n;
+  return n;
+}
+
+static Decode2Params make_d2(const DecodeParams& P, void* ws, const WsLayout& W) {
+  Decode2Params D;
+  D.P = P;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  D.route_cnt = reinterpret_cast<uint32_t*>(&reinterpret_cast<WsHeader*>(ws)->pad[0]);
+  D.logits = reinterpret_cast<float*>(base + W.logits);
+  D.x = nullptr;
+  D.wr = nullptr;
+  D.route_warps = 0;
+  D.route_tc = 0;
+  D.n_sm = sm_count();
+  return D;
+}
+
+// Decode from quantized activations and routing.  One token: the persistent
+// cp.async mat-vec kernels over the slots directly.  More tokens: grouped by
+// expert, then the grouped mat-vec kernels that decode each weight once for
+// all the tokens of a group.
+static int launch_decode(const DecodeParams& P, void* ws, const WsLayout& W, cudaStream_t stream) {
   if (!P.direct) {
     int rc = launch_group(P, stream);
     if (rc) return rc;
+    return launch_ffn(P, stream);
   }
-  return launch_ffn(P, stream);
+  Decode2Params D = make_d2(P, ws, W);
+  return launch_decode2(D, false, stream);
 }
 
 }  // namespace bitmoe
@@ -263,7 +296,7 @@ int moe_expert_ffn_decode(const moe_layer* L, int32_t ntok, const int8_t* xq, co
   int rc = ffn_common("expert_ffn_decode", L, ntok, xq, xd, idx, wts, y, ws, ws_bytes, false, &W);
   if (rc) return rc;
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
-  return launch_decode(P, static_cast<cudaStream_t>(stream));
+  return launch_decode(P, ws, W, static_cast<cudaStream_t>(stream));
 }
 
 int moe_expert_ffn_prefill(const moe_layer* L, int32_t ntok, const int8_t* xq, const float* xd,
@@ -293,12 +326,19 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   int32_t* idx = reinterpret_cast<int32_t*>(base + W.idx);
   float* wts = reinterpret_cast<float*>(base + W.wts);
   float* logits = reinterpret_cast<float*>(base + W.logits);
-  if ((rc = launch_quant_act_q8(x, ntok, L->hidden, xq, xd, s))) return rc;
-  if ((rc = launch_route_topk(x, w_router, ntok, L->hidden, L->n_experts, L->top_k, idx, wts, logits, s)))
-    return rc;
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
-  if (prefill) return launch_prefill(P, s);
-  return launch_decode(P, s);
+  if (ntok > 1) {
+    if ((rc = launch_quant_act_q8(x, ntok, L->hidden, xq, xd, s))) return rc;
+    if ((rc = launch_route_topk(x, w_router, ntok, L->hidden, L->n_experts, L->top_k, idx, wts, logits, s)))
+      return rc;
+    return prefill ? launch_prefill(P, s) : launch_decode(P, ws, W, s);
+  }
+  // one token: act quant, router and top-k in one kernel, then the gate/up
+  // and down kernels, chained with programmatic dependent launch
+  Decode2Params D = make_d2(P, ws, W);
+  D.x = x;
+  D.wr = w_router;
+  return launch_decode2(D, true, s);
 }
 
 int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, const float* x_host,
@@ -364,7 +404,7 @@ int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
 const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
-      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down"};
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 
