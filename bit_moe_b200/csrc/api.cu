@@ -152,6 +152,7 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   P.n_items = reinterpret_cast<const int32_t*>(base + W.grp.n_items);
   P.pairs = reinterpret_cast<const int32_t*>(base + W.grp.pairs);
   P.group_scratch = reinterpret_cast<int32_t*>(base + W.grp.scratch);
+  P.group_chunk = kChunk;
   return P;
 }
 
@@ -404,7 +405,7 @@ int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
 const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
-      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route"};
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
   for (int r = 0; r < 2; ++r) {
     const int e = 2 * tid + r;
     c[r] = e <= E ? cnt[e] : 0;
-    ic[r] = (c[r] + kChunk - 1) / kChunk;
+    ic[r] = (c[r] + P.group_chunk - 1) / P.group_chunk;
   }
   int tot_c = 0, tot_i = 0;
   Scan(scan_tmp).ExclusiveSum(c[0] + c[1], o[0], tot_c);
@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
     for (int i = 0; i < ic[r]; ++i) {
       Item it;
       it.expert = e == E ? -1 : e;
-      it.start = o[r] + i * kChunk;
-      it.count = min(kChunk, c[r] - i * kChunk);
+      it.start = o[r] + i * P.group_chunk;
+      it.count = min(P.group_chunk, c[r] - i * P.group_chunk);
       it.pad = 0;
       items[io[r] + i] = it;
     }
@@ -352,6 +352,7 @@ int launch_group(const DecodeParams& P, cudaStream_t stream) {
 }
 
 int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
+  if (!P.direct && P.group_chunk != kChunk) return fail(MOE_ERR_INVALID_ARG, "expert_ffn: items of %d pairs", P.group_chunk);
   init_kernel_attrs();
   const int npairs = P.ntok * P.top_k;
   if (P.direct) {

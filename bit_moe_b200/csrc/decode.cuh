@@ -35,6 +35,7 @@ struct DecodeParams {
   const int32_t* n_items;
   const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert
   int32_t* group_scratch;                // [2*(n_experts+1)] counters for the grouping
+  int group_chunk;                       // most pairs per item (kChunk for decode)
 };
 
 // Bytes of workspace the grouped mode needs after `off`; writes the offsets.
