@@ -334,11 +334,17 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
       return rc;
     return prefill ? launch_prefill(P, s) : launch_decode(P, ws, W, s);
   }
-  // one token: act quant, router and top-k in one kernel, then the gate/up
-  // and down kernels, chained with programmatic dependent launch
+  // one token: the whole step in one cooperative kernel where the shape
+  // allows it; otherwise act quant, router and top-k in one kernel, then the
+  // gate/up and down kernels, chained with programmatic dependent launch
   Decode2Params D = make_d2(P, ws, W);
   D.x = x;
   D.wr = w_router;
+  size_t smem1 = 0;
+  if (step1_supported(P, D.n_sm, &smem1)) {
+    WsHeader* hd = reinterpret_cast<WsHeader*>(ws);
+    return launch_step1(D, reinterpret_cast<uint32_t*>(&hd->pad[3]), reinterpret_cast<uint32_t*>(&hd->pad[5]), s);
+  }
   return launch_decode2(D, true, s);
 }
 
@@ -405,7 +411,7 @@ int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
 const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
-      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine"};
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

@@ -33,4 +33,8 @@ struct Decode2Params {
 
 int launch_decode2(Decode2Params& D, bool with_route, cudaStream_t stream);
 
+// The whole one-token step in one cooperative kernel (step1.cu).
+bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem);
+int launch_step1(const Decode2Params& D, uint32_t* bar_count, uint32_t* bar_gen, cudaStream_t stream);
+
 }  // namespace bitmoe
