@@ -79,7 +79,16 @@ def kernel_bytes(wl, unique_experts):
     out)."""
     T, H, F, E, K = wl.ntok, wl.hidden, wl.ffn, wl.n_experts, wl.top_k
     pairs = T * K
+    weights = unique_experts * 3 * matrix_bytes(F, H)
     return {
+        # the whole one-token step in one kernel: router, x, the routed
+        # experts' packed weights, the int8 intermediates and y
+        "step1": E * H * 4 + T * H * 4 + weights + 2 * (pairs * F + pairs * F // 32 * 4)
+        + T * H + T * H // 32 * 4 + T * E * 4 + pairs * 8 + T * H * 4,
+        "prefill_gateup": unique_experts * 2 * matrix_bytes(F, H) + T * H + T * H // 32 * 4
+        + pairs * F + pairs * F // 32 * 4,
+        "prefill_down": unique_experts * matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4 + pairs * H * 4,
+        "combine": pairs * H * 4 + T * H * 4 + pairs * 4,
         "route": E * H * 4 + T * H * 4 + T * H + T * H // 32 * 4 + T * E * 4 + pairs * 8,
         "quant_act_q8": T * H * 4 + T * H + T * H // 32 * 4,
         "router_logits": E * H * 4 + T * H * 4 + T * E * 4,
@@ -240,6 +249,23 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- our arm
+def max_over_ranks(ms, world, device=None):
+    """The slowest rank's time (ms): the job is done when every replica is."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(tokens_per_rank, world, ms):
+    """Whole-job throughput: the tokens every rank processed over the slowest
+    rank's time."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 def workload_config(wl, layers):
     c = {"workload": wl.describe(), "hidden": wl.hidden, "expert_ffn": wl.ffn,
          "experts": wl.n_experts, "top_k": wl.top_k, "tokens_per_step": wl.ntok,
@@ -386,16 +412,11 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     status = B.moe_check_status(ws)
     if status != 0:
         raise SystemExit("device status %d after the timed region" % status)
-    tokens = world * T * args.steps
-    value = tokens / (ms / 1e3)
+    value = job_rate(T * args.steps, world, ms)
 
     # ---- per-kernel times: the same steps launched eagerly behind a spin
     # kernel (so the host has queued them all before the GPU starts them and
@@ -451,12 +472,8 @@ def main():
                 B.moe_forward_host(layers[j % L], routers[j % L], xh[j % len(xh)], yh, ws, stream=stream)
             a1.record(stream)
             stream.synchronize()
-        e_ms = a0.elapsed_time(a1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * T * n_e2e / (e_ms / 1e3), "unit": "tok/s",
+        e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev)
+        e2e = {"value": job_rate(T * n_e2e, world, e_ms), "unit": "tok/s",
                "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4,
                "steps": n_e2e, "api": "moe_forward_host"}
 
