@@ -36,6 +36,10 @@ struct DecodeParams {
   const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert
   int32_t* group_scratch;                // [2*(n_experts+1)] counters for the grouping
   int group_chunk;                       // most pairs per item (kChunk for decode)
+  // prefill only: the activation codes split for the e4m3 tensor-core path
+  // (code = 16*hi + lo, both parts exact in e4m3) and the code sums per 32-block
+  uint8_t* xh; uint8_t* xl; int32_t* xsum;   // [ntok][hidden], [ntok][hidden/32]
+  uint8_t* aqh; uint8_t* aql; int32_t* asum; // [ntok*top_k][ffn], [ntok*top_k][ffn/32]
 };
 
 // Bytes of workspace the grouped mode needs after `off`; writes the offsets.

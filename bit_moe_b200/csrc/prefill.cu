@@ -6,21 +6,29 @@
 //
 // The (token, slot) pairs are grouped by expert and cut into tiles of up to
 // kPN pairs.  A tile of the grouped GEMM is 128 weight rows x kPN pairs:
-//   - A (128 x 32 per MMA): the weights' base-3 digits t = q + 1 as u8,
-//     decoded in registers from the packed blocks (one thread per row) and
-//     written straight into tensor memory with tcgen05.st -- the expanded
-//     weights never exist in HBM or shared memory;
-//   - B (32 x kPN): the pairs' int8 activation codes, gathered with cp.async
-//     into the K-major core-matrix layout of shared memory;
-//   - one tcgen05.mma kind::i8 per 32-value sub-block into its own int32 TMEM
-//     accumulator (the activation scale changes every 32 values), read back
-//     with tcgen05.ld and scaled in fp32 exactly like the decode kernels:
-//     sum over sub-blocks of d * (sum t*a - sum a), then the fp16 weight
-//     scale per 256-block.
+//   - A (128 x 32 per MMA): the weights' base-3 digits t = q + 1 in {0,1,2},
+//     decoded in registers from the packed blocks and written straight into
+//     tensor memory with tcgen05.st.  Read as e4m3, the bytes 0, 1, 2 are the
+//     subnormals 0, 2^-9, 2^-8, i.e. exactly t * 2^-9, so the decoded digits
+//     need no conversion at all;
+//   - B (32 x kPN): each int8 activation code a = 16*h + l is split into two
+//     e4m3 operands, 16*h (h in [-8, 7]) and l (in [0, 15]), both exact; two
+//     MMAs accumulate t*16h and t*l into the same fp32 accumulator, which then
+//     holds 2^-9 * sum(t*a) exactly (every partial sum is a multiple of 2^-9
+//     below 2^4);
+//   - one fp32 TMEM accumulator per 32-value sub-block (the activation scale
+//     changes every 32 values); the epilogue forms sum(q*a) = 512*D - sum(a)
+//     and scales it in fp32 exactly like the decode kernels: sum over
+//     sub-blocks of d * sum(q*a), then the fp16 weight scale per 256-block.
+// Two warps share each TMEM lane quadrant: both hold the same 32 rows, one
+// decodes the first 32 digit columns and fixes up the first half of the
+// pairs, the other the rest.
 // Gate/up tiles hold 64 gate rows and the 64 matching up rows, so SwiGLU and
-// the int8 requantization of a run in the epilogue; down tiles write each
-// pair's rows, and a last pass combines the top_k slots of every token in
-// slot order.
+// the requantization run in the epilogue (writing the split codes of the down
+// input); down tiles write each pair's rows, and a last pass combines the
+// top_k slots of every token in slot order.
+#include <cuda_fp8.h>
+
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -31,7 +39,8 @@ namespace bitmoe {
 
 constexpr int kPN = 32;          // pairs per tile (MMA N)
 constexpr int kPM = 128;         // weight rows per tile (MMA M)
-constexpr int kPThreads = 128;   // one thread per row
+constexpr int kPThreads = 256;   // two warps per TMEM lane quadrant
+constexpr int kPHalf = kPN / 2;  // pairs fixed up by one warp of a quadrant
 constexpr int kTmemCols = 256;   // A: columns [0, 64); D: [64, 64 + 4 * kPN)
 constexpr int kADcol = 0;
 constexpr int kDcol = 64;
@@ -41,10 +50,11 @@ struct PrefillSmem {
   int abort;
   uint64_t bar;
   int pairs[kPN];
-  alignas(128) unsigned char B[kSubPerBlock * kPN * 32];  // activation codes, MMA layout
-  float d[kSubPerBlock][kPN];                              // activation scales
-  int as[kSubPerBlock][kPN];                               // sums of the codes
-  float xch[64][kPN + 1];                                  // gate results for the up rows
+  alignas(128) unsigned char Bh[2][kSubPerBlock * kPN * 32];  // 16*h parts, MMA layout, 2 blocks
+  alignas(128) unsigned char Bl[2][kSubPerBlock * kPN * 32];  // l parts
+  alignas(16) float d[kSubPerBlock][kPN];                      // activation scales of the block
+  alignas(16) float na[kSubPerBlock][kPN];                     // minus the code sums
+  float xch[64][kPN + 1];                                      // gate results for the up rows
 };
 
 // Byte offset of activation code (pair n, k in [0, 32)) of sub-block s in B:
@@ -54,16 +64,65 @@ __device__ __forceinline__ int b_off(int s, int n, int k) {
   return s * (kPN * 32) + (n >> 3) * 256 + (k >> 4) * 128 + (n & 7) * 16 + (k & 15);
 }
 
+// e4m3 bytes of the two parts of an activation code q = 16*h + l.
+__device__ __forceinline__ void code_split(int q, uint8_t& hi, uint8_t& lo) {
+  const int h = q >> 4;  // floor(q / 16), in [-8, 7]
+  const int l = q & 15;
+  hi = static_cast<uint8_t>(__nv_cvt_float_to_fp8(static_cast<float>(h * 16), __NV_SATFINITE, __NV_E4M3));
+  lo = static_cast<uint8_t>(__nv_cvt_float_to_fp8(static_cast<float>(l), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Split codes and per-32-block code sums of the gate/up input: one warp per
+// 32-block.
+__global__ void k_prefill_prep(DecodeParams P) {
+  const int64_t nblk = static_cast<int64_t>(P.ntok) * (P.hidden / kQBlock);
+  const int lane = threadIdx.x & 31;
+  for (int64_t blk = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; blk < nblk;
+       blk += static_cast<int64_t>(gridDim.x) * blockDim.x / 32) {
+    const int q = P.xq[blk * kQBlock + lane];
+    uint8_t hi, lo;
+    code_split(q, hi, lo);
+    P.xh[blk * kQBlock + lane] = hi;
+    P.xl[blk * kQBlock + lane] = lo;
+    const int sum = __reduce_add_sync(0xffffffffu, q);
+    if (lane == 0) P.xsum[blk] = sum;
+  }
+}
+
+// Digit words [32*kHalf, 32*kHalf + 32) of one packed block (digit word
+// 5*j + i holds level i of the four bytes of packed word j): each 16-bit lane
+// keeps u * 3^i, whose high byte H_i grows by one base-3 digit per level and
+// t_i = H_(i+1) - 3*H_i.  `w` holds packed words [6*kHalf, 6*kHalf + 7).
+template <int kHalf>
+__device__ __forceinline__ void decode_half(const uint32_t (&w)[7], uint32_t (&dg)[32]) {
+#pragma unroll
+  for (int jj = 0; jj < 7; ++jj) {
+    const int j = 6 * kHalf + jj;
+    uint32_t lo = w[jj] & 0x00FF00FFu, hi = (w[jj] >> 8) & 0x00FF00FFu, hp = 0u;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      if (j == kBlockWords - 1 && i == 4) break;
+      lo *= 3u;
+      hi *= 3u;
+      const uint32_t hn = __byte_perm(lo, hi, 0x7351);
+      const int c = 5 * j + i - 32 * kHalf;
+      if (c >= 0 && c < 32) dg[c] = hn - 3u * hp;
+      hp = hn;
+    }
+  }
+}
+
 template <bool kGU>
-__global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
+__global__ void __launch_bounds__(kPThreads, 2) k_prefill_mma(DecodeParams P) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
   const int H = P.hidden, F = P.ffn, K = P.top_k;
   const int kdim = kGU ? H : F;               // reduction length
   const int nb = kdim / kBlock;
   const int m_tiles = kGU ? F / 64 : H / kPM;
-  const uint32_t idesc = idesc_i8(kPM, kPN);
+  const uint32_t idesc = idesc_e4m3(kPM, kPN);
 
   if (warp == 0) {
     tmem_alloc(&S.tmem_base, kTmemCols);
@@ -78,7 +137,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
-  const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lane quadrant
+  const uint32_t tlane = tbase + (static_cast<uint32_t>(quad * 32) << 16);  // this warp's lane quadrant
   uint32_t phase = 0;
 
   const int n_tiles = *P.n_items * m_tiles;
@@ -92,11 +151,16 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       for (int n = 0; n < it.count; ++n) {
         const int pair = S.pairs[n];
         if (kGU) {
-          for (int r = tid; r < 64; r += kPThreads) {
-            P.aq[static_cast<size_t>(pair) * F + 64 * mt + r] = 0;
-            if ((r & 31) == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + (64 * mt + r) / kQBlock] = 0.f;
+          if (tid < 64) {
+            const size_t f = static_cast<size_t>(pair) * F + 64 * mt + tid;
+            P.aqh[f] = 0;
+            P.aql[f] = 0;
+            if ((tid & 31) == 0) {
+              P.ad[static_cast<size_t>(pair) * (F / kQBlock) + (64 * mt + tid) / kQBlock] = 0.f;
+              P.asum[static_cast<size_t>(pair) * (F / kQBlock) + (64 * mt + tid) / kQBlock] = 0;
+            }
           }
-        } else {
+        } else if (tid < kPM) {
           P.ye[static_cast<size_t>(pair) * H + kPM * mt + tid] = 0.f;
         }
       }
@@ -108,93 +172,102 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
     const uint16_t* scales;
     size_t panel;
     if (kGU) {
-      const bool up = warp >= 2;
+      const bool up = quad >= 2;
       trits = up ? P.up_trits : P.gate_trits;
       scales = up ? P.up_scales : P.gate_scales;
-      panel = (static_cast<size_t>(it.expert) * F + 64 * mt) / kPanel + (warp & 1);
+      panel = (static_cast<size_t>(it.expert) * F + 64 * mt) / kPanel + (quad & 1);
     } else {
       trits = P.down_trits;
       scales = P.down_scales;
-      panel = (static_cast<size_t>(it.expert) * H + kPM * mt) / kPanel + warp;
+      panel = (static_cast<size_t>(it.expert) * H + kPM * mt) / kPanel + quad;
     }
-    float y[kPN];
+    float y[kPHalf];
 #pragma unroll
-    for (int n = 0; n < kPN; ++n) y[n] = 0.f;
+    for (int n = 0; n < kPHalf; ++n) y[n] = 0.f;
 
-    for (int b = 0; b < nb; ++b) {
-      // ---- B: gather the pairs' codes of block b (zeros for empty slots)
-      for (int c = tid; c < kPN * 16; c += kPThreads) {
-        const int n = c >> 4, kc = c & 15;
-        unsigned char* dst = S.B + b_off(kc >> 1, n, (kc & 1) * 16);
+    // Gather block b's split codes of the tile's pairs into B[buf] (zeros for
+    // empty pair slots); one commit group per block.
+    auto gather = [&](int b, int buf) {
+#pragma unroll
+      for (int i = 0; i < (2 * kPN * 16) / kPThreads; ++i) {
+        const int c = tid + i * kPThreads;
+        const int part = c / (kPN * 16), n = (c / 16) % kPN, kc = c & 15;
+        unsigned char* dst = (part ? S.Bl[buf] : S.Bh[buf]) + b_off(kc >> 1, n, (kc & 1) * 16);
         const int pair = S.pairs[n];
         if (pair >= 0) {
-          const int8_t* row = kGU ? P.xq + static_cast<size_t>(pair / K) * H : P.aq + static_cast<size_t>(pair) * F;
+          const uint8_t* src = kGU ? (part ? P.xl : P.xh) + static_cast<size_t>(pair / K) * H
+                                   : (part ? P.aql : P.aqh) + static_cast<size_t>(pair) * F;
           asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
-                       "l"(row + b * kBlock + kc * 16)
+                       "l"(src + b * kBlock + kc * 16)
                        : "memory");
         } else {
           *reinterpret_cast<int4*>(dst) = make_int4(0, 0, 0, 0);
         }
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
-      // ---- A: decode this row's block into 64 digit words (groups of 4)
+    };
+    uint32_t wn[7];
+    uint16_t sn;
+    auto load_w = [&](int b) {
       const size_t pb = panel * nb + b;
-      uint32_t w[kBlockWords];
 #pragma unroll
-      for (int j = 0; j < kBlockWords; ++j) w[j] = ld_stream_u32(trits + (pb * kBlockWords + j) * kPanel + lane);
-      const float sw = f16_bits_to_f32(scales[pb * kPanel + lane]);
-      uint32_t digits[64];
+      for (int j = 0; j < 7; ++j)
+        wn[j] = ld_stream_u32(trits + (pb * kBlockWords + 6 * half + j) * kPanel + lane);
+      sn = scales[pb * kPanel + lane];
+    };
+    gather(0, 0);
+    load_w(0);
+    for (int b = 0; b < nb; ++b) {
+      const int buf = b & 1;
+      uint32_t w[7];
 #pragma unroll
-      for (int j = 0; j < kBlockWords; ++j) {
-        uint32_t lo = w[j] & 0x00FF00FFu, hi = (w[j] >> 8) & 0x00FF00FFu, hp = 0u;
-#pragma unroll
-        for (int i = 0; i < 5; ++i) {
-          if (j == kBlockWords - 1 && i == 4) break;
-          lo *= 3u;
-          hi *= 3u;
-          const uint32_t hn = __byte_perm(lo, hi, 0x7351);
-          digits[5 * j + i] = hn - 3u * hp;
-          hp = hn;
-        }
+      for (int j = 0; j < 7; ++j) w[j] = wn[j];
+      const float sw = f16_bits_to_f32(sn);
+      // prefetch block b+1 while this block is decoded, multiplied and scaled
+      if (b + 1 < nb) {
+        gather(b + 1, buf ^ 1);
+        load_w(b + 1);
       }
-      tmem_st64(tlane + kADcol, digits);
+      // ---- A: this warp's 32 digit columns of the rows' block
+      {
+        uint32_t dg[32];
+        if (half == 0) decode_half<0>(w, dg);
+        else decode_half<1>(w, dg);
+        tmem_st32(tlane + kADcol + 32 * half, dg);
+      }
       // ---- scales and code sums of block b
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      __syncthreads();
-      for (int q = tid; q < kSubPerBlock * kPN; q += kPThreads) {
-        const int s = q / kPN, n = q % kPN;
+      if (b + 1 < nb) asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else asm volatile("cp.async.wait_group 0;" ::: "memory");
+      {
+        const int s = tid >> 5, n = tid & 31;  // kPThreads == kSubPerBlock * kPN
         const int pair = S.pairs[n];
-        float dv = 0.f;
-        int sum = 0;
+        float dv = 0.f, av = 0.f;
         if (pair >= 0) {
-          dv = kGU ? P.xd[static_cast<size_t>(pair / K) * (H / kQBlock) + b * kSubPerBlock + s]
-                   : P.ad[static_cast<size_t>(pair) * (F / kQBlock) + b * kSubPerBlock + s];
-          const int4 lo4 = *reinterpret_cast<const int4*>(S.B + b_off(s, n, 0));
-          const int4 hi4 = *reinterpret_cast<const int4*>(S.B + b_off(s, n, 16));
-          sum = __dp4a(lo4.x, 0x01010101, sum); sum = __dp4a(lo4.y, 0x01010101, sum);
-          sum = __dp4a(lo4.z, 0x01010101, sum); sum = __dp4a(lo4.w, 0x01010101, sum);
-          sum = __dp4a(hi4.x, 0x01010101, sum); sum = __dp4a(hi4.y, 0x01010101, sum);
-          sum = __dp4a(hi4.z, 0x01010101, sum); sum = __dp4a(hi4.w, 0x01010101, sum);
+          const size_t q = kGU ? static_cast<size_t>(pair / K) * (H / kQBlock) + b * kSubPerBlock + s
+                               : static_cast<size_t>(pair) * (F / kQBlock) + b * kSubPerBlock + s;
+          dv = kGU ? P.xd[q] : P.ad[q];
+          av = static_cast<float>(kGU ? P.xsum[q] : P.asum[q]);
         }
         S.d[s][n] = dv;
-        S.as[s][n] = sum;
+        S.na[s][n] = -av;
       }
       tc_wait_st();
       fence_proxy_async_shared();
       tc_fence_before();
       __syncthreads();
-      float inner[kPN];
+      float inner[kPHalf];
 #pragma unroll
-      for (int n = 0; n < kPN; ++n) inner[n] = 0.f;
+      for (int n = 0; n < kPHalf; ++n) inner[n] = 0.f;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int h4 = 0; h4 < 2; ++h4) {
         if (tid == 0 && !*reinterpret_cast<volatile int*>(&S.abort)) {
           tc_fence_after();
 #pragma unroll
           for (int s4 = 0; s4 < 4; ++s4) {
-            const int s = 4 * half + s4;
-            mma_i8_ts(tbase + kDcol + s4 * kPN, tbase + kADcol + 8 * s,
-                      smem_desc(smem_u32(S.B + s * (kPN * 32)), 128, 256), idesc, false);
+            const int s = 4 * h4 + s4;
+            const uint32_t dcol = tbase + kDcol + s4 * kPN, acol = tbase + kADcol + 8 * s;
+            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.Bh[buf] + s * (kPN * 32)), 128, 256), idesc, false);
+            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.Bl[buf] + s * (kPN * 32)), 128, 256), idesc, true);
           }
           mma_commit(&S.bar);
         }
@@ -206,50 +279,69 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         tc_fence_after();
 #pragma unroll
         for (int s4 = 0; s4 < 4; ++s4) {
-          const int s = 4 * half + s4;
-          uint32_t v[32];
-          tmem_ld32(tlane + kDcol + s4 * kPN, v);
+          const int s = 4 * h4 + s4;
+          uint32_t v[16];
+          tmem_ld16(tlane + kDcol + s4 * kPN + kPHalf * half, v);
           tc_wait_ld();
+          const float4* dp = reinterpret_cast<const float4*>(&S.d[s][kPHalf * half]);
+          const float4* ap = reinterpret_cast<const float4*>(&S.na[s][kPHalf * half]);
 #pragma unroll
-          for (int n = 0; n < kPN; ++n)
-            inner[n] = __fmaf_rn(S.d[s][n], static_cast<float>(static_cast<int>(v[n]) - S.as[s][n]), inner[n]);
+          for (int n4 = 0; n4 < kPHalf / 4; ++n4) {
+            const float4 dd = dp[n4], aa = ap[n4];
+            const float dv[4] = {dd.x, dd.y, dd.z, dd.w}, av[4] = {aa.x, aa.y, aa.z, aa.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int n = 4 * n4 + e;
+              // 512 * D - sum(a) = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
+              const float qa = __fmaf_rn(__uint_as_float(v[n]), 512.f, av[e]);
+              inner[n] = __fmaf_rn(dv[e], qa, inner[n]);
+            }
+          }
         }
         tc_fence_before();
         __syncthreads();
       }
 #pragma unroll
-      for (int n = 0; n < kPN; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
+      for (int n = 0; n < kPHalf; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
     }
 
-    // ---- epilogue
+    // ---- epilogue (this warp: rows 32*quad + lane, pairs kPHalf*half + n)
+    const int n0 = kPHalf * half;
     if (kGU) {
-      if (warp < 2) {
+      if (quad < 2) {
 #pragma unroll
-        for (int n = 0; n < kPN; ++n) S.xch[tid][n] = y[n];
+        for (int n = 0; n < kPHalf; ++n) S.xch[32 * quad + lane][n0 + n] = y[n];
       }
       __syncthreads();
-      if (warp >= 2) {
-        const int r = tid - 64;               // f offset within the tile
+      if (quad >= 2) {
+        const int r = 32 * (quad - 2) + lane;  // f offset within the tile
         const int f = 64 * mt + r;
 #pragma unroll
-        for (int n = 0; n < kPN; ++n) {
-          if (n >= it.count) break;
-          const float g = S.xch[r][n];
+        for (int n = 0; n < kPHalf; ++n) {
+          if (n0 + n >= it.count) break;
+          const float g = S.xch[r][n0 + n];
           const float a = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
           const float amax = warp_max(fabsf(a));
           const float dd = __fdiv_rn(amax, 127.f);
           int q = 0;
           if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
-          const int pair = S.pairs[n];
-          P.aq[static_cast<size_t>(pair) * F + f] = static_cast<int8_t>(q);
-          if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + f / kQBlock] = dd;
+          const int pair = S.pairs[n0 + n];
+          uint8_t hi, lo;
+          code_split(q, hi, lo);
+          P.aqh[static_cast<size_t>(pair) * F + f] = hi;
+          P.aql[static_cast<size_t>(pair) * F + f] = lo;
+          const int sum = __reduce_add_sync(0xffffffffu, q);
+          if (lane == 0) {
+            P.ad[static_cast<size_t>(pair) * (F / kQBlock) + f / kQBlock] = dd;
+            P.asum[static_cast<size_t>(pair) * (F / kQBlock) + f / kQBlock] = sum;
+          }
         }
       }
     } else {
-      const int h = kPM * mt + tid;
+      const int h = kPM * mt + 32 * quad + lane;
 #pragma unroll
-      for (int n = 0; n < kPN; ++n)
-        if (n < it.count) P.ye[static_cast<size_t>(S.pairs[n]) * H + h] = y[n];
+      for (int n = 0; n < kPHalf; ++n)
+        if (n0 + n < it.count) P.ye[static_cast<size_t>(S.pairs[n0 + n]) * H + h] = y[n];
     }
     __syncthreads();
   }
@@ -294,6 +386,8 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = prefill_smem();
+  k_prefill_prep<<<2 * n_sm, 256, 0, stream>>>(P);
+  note_launch(MOE_K_PREFILL_PREP, stream);
   k_prefill_mma<true><<<2 * n_sm, kPThreads, smem, stream>>>(P);
   note_launch(MOE_K_PREFILL_GATEUP, stream);
   k_prefill_mma<false><<<2 * n_sm, kPThreads, smem, stream>>>(P);
