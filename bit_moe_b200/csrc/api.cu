@@ -2,6 +2,8 @@
 // workspace layout, and the launch sequence of each call.
 #include <cstring>
 
+#include <algorithm>
+
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode.cuh"
@@ -64,8 +66,9 @@ int check_device() {
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
-  size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0, xs = 0, ys = 0;
-  size_t xh = 0, xl = 0, xsum = 0, aqh = 0, aql = 0, asum = 0;  // prefill only
+  size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0, asum = 0;
+  size_t xs = 0, ys = 0;  // device copies of x and y for the host-buffer entry point
+  size_t xh = 0, xl = 0, xsum = 0, aqh = 0, aql = 0;  // prefill only
   GroupWs grp;
   size_t total = 0;
 };
@@ -78,7 +81,8 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
     off = align_up(off + bytes, 256);
     return o;
   };
-  L.logits = take(sizeof(float) * T * static_cast<size_t>(E));
+  // fp32 [T][E], or for the one-token step E tagged logits one 128-byte line apart
+  L.logits = take(std::max(sizeof(float) * T * static_cast<size_t>(E), static_cast<size_t>(128) * E));
   L.xq = take(static_cast<size_t>(T) * H);
   L.xd = take(sizeof(float) * T * static_cast<size_t>(H / kQBlock));
   L.idx = take(sizeof(int32_t) * T * static_cast<size_t>(K));
@@ -87,6 +91,7 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
   L.ad = take(sizeof(float) * T * static_cast<size_t>(K) * (F / kQBlock));
   L.ye = take(sizeof(float) * T * static_cast<size_t>(K) * H);
   L.cnt = take(sizeof(int32_t) * T * static_cast<size_t>(H / kPanel));
+  L.asum = take(sizeof(int32_t) * T * static_cast<size_t>(K) * (F / kQBlock));
   L.xs = take(sizeof(float) * T * static_cast<size_t>(H));
   L.ys = take(sizeof(float) * T * static_cast<size_t>(H));
   off = group_ws_layout(E, T * K, off, &L.grp);
@@ -96,7 +101,6 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
     L.xsum = take(sizeof(int32_t) * T * static_cast<size_t>(H / kQBlock));
     L.aqh = take(static_cast<size_t>(T) * K * F);
     L.aql = take(static_cast<size_t>(T) * K * F);
-    L.asum = take(sizeof(int32_t) * T * static_cast<size_t>(K) * (F / kQBlock));
   }
   L.total = off;
   return L;
@@ -167,7 +171,7 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   P.xsum = pf ? reinterpret_cast<int32_t*>(base + W.xsum) : nullptr;
   P.aqh = pf ? base + W.aqh : nullptr;
   P.aql = pf ? base + W.aql : nullptr;
-  P.asum = pf ? reinterpret_cast<int32_t*>(base + W.asum) : nullptr;
+  P.asum = reinterpret_cast<int32_t*>(base + W.asum);
   return P;
 }
 
@@ -358,7 +362,8 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   size_t smem1 = 0;
   if (step1_supported(P, D.n_sm, &smem1)) {
     WsHeader* hd = reinterpret_cast<WsHeader*>(ws);
-    return launch_step1(D, reinterpret_cast<uint32_t*>(&hd->pad[3]), reinterpret_cast<uint32_t*>(&hd->pad[5]), s);
+    return launch_step1(D, reinterpret_cast<unsigned long long*>(&hd->pad[3]),
+                        reinterpret_cast<uint32_t*>(&hd->pad[8]), s);
   }
   return launch_decode2(D, true, s);
 }

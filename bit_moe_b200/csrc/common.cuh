@@ -33,7 +33,8 @@ constexpr int kMaxDynSmem = 227 * 1024;  // opt-in dynamic shared memory per CTA
 // Workspace header: the first 256 bytes hold the device status word.
 struct WsHeader {
   int32_t status;    // first error code seen by a kernel (0 = ok)
-  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit grid barrier tickets
+  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit one-token step tickets;
+                     // pad[8..23]: two sets of slot counters of the one-token step
 };
 static_assert(offsetof(WsHeader, pad) + 3 * sizeof(int32_t) == 16, "8-byte aligned ticket counter");
 constexpr size_t kWsHeaderBytes = sizeof(WsHeader);

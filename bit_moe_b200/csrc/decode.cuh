@@ -39,7 +39,8 @@ struct DecodeParams {
   // prefill only: the activation codes split for the e4m3 tensor-core path
   // (code = 16*hi + lo, both parts exact in e4m3) and the code sums per 32-block
   uint8_t* xh; uint8_t* xl; int32_t* xsum;   // [ntok][hidden], [ntok][hidden/32]
-  uint8_t* aqh; uint8_t* aql; int32_t* asum; // [ntok*top_k][ffn], [ntok*top_k][ffn/32]
+  uint8_t* aqh; uint8_t* aql;                // [ntok*top_k][ffn]
+  int32_t* asum;                             // [ntok*top_k][ffn/32] code sums of a^ (prefill, one-token step)
 };
 
 // Bytes of workspace the grouped mode needs after `off`; writes the offsets.

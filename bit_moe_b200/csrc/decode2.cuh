@@ -35,6 +35,8 @@ int launch_decode2(Decode2Params& D, bool with_route, cudaStream_t stream);
 
 // The whole one-token step in one cooperative kernel (step1.cu).
 bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem);
-int launch_step1(const Decode2Params& D, uint32_t* bar_count, uint32_t* bar_gen, cudaStream_t stream);
+// `ticket`: a 64-bit counter that only grows; `slot_cnt`: top_k counters; the
+// logits area of D must hold 8 bytes per expert (tagged logits).
+int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* slot_cnt, cudaStream_t stream);
 
 }  // namespace bitmoe

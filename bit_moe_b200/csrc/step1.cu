@@ -4,19 +4,23 @@
 //
 // A one-token step moves a few megabytes: it is bound by latency, not by
 // bandwidth, so the step's three dependent phases run inside one cooperative
-// launch (every CTA resident) separated by two grid barriers:
+// launch (every CTA resident), handing data over through L2 with tagged
+// values and counters instead of grid-wide barriers:
 //   A. every CTA quantizes x to int8 32-blocks in its shared memory (the same
-//      result everywhere) and computes the fixed-order router logits of its
-//      share of the experts;                                     -- barrier --
-//   B. every CTA takes the top-k of the E logits itself (ties to the lower
-//      id, so every CTA agrees), starts the bulk copies of the down-projection
-//      weights it will need (its 32-row panel of hidden for each selected
-//      expert) into shared memory, and computes its share of the gate/up
-//      units (32-row panels of ffn, hidden blocks split over the warps),
-//      writing the requantized SwiGLU codes;                    -- barrier --
-//   C. each CTA with a panel of hidden finishes it: warp j multiplies slot j's
-//      codes with the prefetched down weights, and the slots are summed in
-//      order (no atomics).
+//      result everywhere) and publishes the fixed-order router logits of its
+//      share of the experts, each tagged with the launch's generation;
+//   B. every CTA polls the E tagged logits until all carry this launch's tag,
+//      takes the top-k itself (ties to the lower id, so every CTA agrees;
+//      every logit is ranked against all others in parallel), starts the bulk
+//      copies of the down-projection weights it will need (its 32-row panel
+//      of hidden for each selected expert) into shared memory, and computes
+//      its share of the gate/up units (32-row panels of ffn, hidden blocks
+//      split over the warps), writing the requantized SwiGLU codes and
+//      counting each finished unit on its slot's counter;
+//   C. each CTA with a panel of hidden waits for the k slot counters to reach
+//      the number of ffn panels, then warp j multiplies slot j's codes with the
+//      prefetched down weights, and the slots are summed in order (no atomics
+//      on data).
 // Parakon Runtime README, "How it works" (fused decode mat-vecs on the packed
 // blocks, int8 activations); llama-modchip page, "Key highlights" (all top-k
 // experts evaluated); pxq_llama README, "Updates -- 2026-07-28" (gate/up with
@@ -30,19 +34,26 @@
 namespace bitmoe {
 
 constexpr int kS1MaxH = 4096, kS1MaxF = 2048, kS1MaxK = 8;
-constexpr uint32_t kSpinLimit = 1u << 24;
+constexpr uint32_t kSpinLimit = 1u << 22;  // polls before a wait gives up (seconds)
+constexpr int kS1MaxE = kNC * 32;          // experts: one per thread of the CTA
+// One 128-byte line per tagged logit, so that the CTAs polling the logits
+// spread their loads over many L2 lines instead of queueing on a few.
+constexpr int kTagStride = 16;
+constexpr int kS1KeyBytes = kS1MaxE * 4;
+static_assert(kNC * kS1MaxK <= kNC * 32, "top-k candidates: one per thread");
 
 struct Step1Params {
   Decode2Params D;
-  uint32_t* bar_count;  // 64-bit grid barrier ticket counter (only grows)
-  uint32_t* bar_gen;    // unused
+  unsigned long long* ticket;  // launch ticket counter (only grows): generation = ticket / CTAs
+  unsigned long long* tagged;  // [E][kTagStride] logits as (generation + 1) << 32 | fp32 bits
+  uint32_t* slot_cnt;          // [top_k] finished gate/up units per slot (zeroed each launch)
 };
 
 struct Step1Layout {
   size_t ring, pref, xq4, xd, xas, lg, sel, red, flag, xf, act, total;
 };
 
-// Shared-memory plan of one CTA (x fp32 and the down activations alias the
+// Shared-memory plan of one CTA (the down activations alias the
 // gate/up ring; the router rows alias the down prefetch area).
 __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) {
   Step1Layout L{};
@@ -55,9 +66,9 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
   const size_t ring = static_cast<size_t>(kNC) * ring_depth<1>() * Slot<2, 1, true>::bytes;
   const size_t xf = static_cast<size_t>(H) * 4;
   const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
-  L.ring = take(ring > xf ? (ring > act ? ring : act) : (xf > act ? xf : act));
-  L.xf = L.ring;
+  L.ring = take(ring > act ? ring : act);
   L.act = L.ring;
+  L.xf = take(xf);
   const size_t pref = static_cast<size_t>(K) * (F / kBlock) * kMatBytes;
   const size_t rows = static_cast<size_t>(2) * H * 4;  // at most two router rows per CTA
   L.pref = take(pref > rows ? pref : rows);
@@ -72,45 +83,14 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
   return L;
 }
 
-// Grid barrier in two halves (all CTAs are resident: cooperative launch), so
-// that a CTA can work between announcing its arrival and waiting for the
-// others.  grid_arrive returns the generation to wait on; grid_wait is
-// bounded and returns false, with MOE_ERR_TIMEOUT recorded, if the other CTAs
-// did not arrive.
-__device__ __forceinline__ uint64_t grid_arrive(const Step1Params& S) {
-  __syncthreads();
-  uint64_t target = 0;
-  if (threadIdx.x == 0) {
-    __threadfence();
-    // tickets of one barrier round are consecutive: every CTA arrives at round
-    // r before any CTA leaves it, so round r owns tickets [r*C, (r+1)*C)
-    const unsigned long long t = atomicAdd(reinterpret_cast<unsigned long long*>(S.bar_count), 1ull);
-    target = (t / gridDim.x + 1) * gridDim.x;
-  }
-  return target;
+// Bounded polls of values another CTA publishes.
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
-
-__device__ __forceinline__ bool grid_wait(const Step1Params& S, uint64_t target, volatile int* abort) {
-  if (threadIdx.x == 0 && !*abort) {
-    uint32_t polls = 0;
-    for (;;) {
-      uint64_t v;
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(S.bar_count) : "memory");
-      if (v >= target) break;
-      if (++polls > kSpinLimit) {
-        record_status(S.D.P.status, MOE_ERR_TIMEOUT);
-        *abort = 1;
-        break;
-      }
-    }
-    __threadfence();
-  }
-  __syncthreads();
-  return !*abort;
-}
-
-__device__ __forceinline__ bool grid_sync(const Step1Params& S, volatile int* abort) {
-  return grid_wait(S, grid_arrive(S), abort);
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // Order-preserving map of an fp32 value to uint32 (larger value, larger key).
@@ -138,10 +118,20 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   float* sel_w = reinterpret_cast<float*>(smem + L.sel + kMaxTopK * 4);
   float* xf = reinterpret_cast<float*>(smem + L.xf);
   float* rows = reinterpret_cast<float*>(smem + L.pref);
+  uint32_t* sgen = reinterpret_cast<uint32_t*>(smem + L.flag + 32);
   if (tid == 0) {
     *abort = 0;
     mbar_init(pbar, K);
     fence_mbar_init();
+    // every CTA takes one ticket per launch, so the tickets of a launch are
+    // [g*C, (g+1)*C) and ticket / C is the same generation g in every CTA;
+    // the logits of this launch carry the tag g + 1
+    const uint32_t g = static_cast<uint32_t>(atomicAdd(S1.ticket, 1ull) / static_cast<unsigned long long>(C));
+    *sgen = g + 1u;
+    // slot counters: launch g counts on set g & 1 and clears the other set
+    // for launch g + 1 (which starts after this launch has ended)
+    if (c == 0)
+      for (int j = 0; j < kS1MaxK; ++j) S1.slot_cnt[((g + 1u) & 1u) * kS1MaxK + j] = 0u;
   }
 
   // ---------------- phase A: x, int8 x^, logits of this CTA's experts
@@ -155,71 +145,106 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   cp_commit();
   cp_wait<0>();
   __syncthreads();
-  if (warp < e1 - e0) {
+  const int nrows = e1 - e0;
+  const uint32_t tag = *sgen;
+  const uint32_t* gk = reinterpret_cast<const uint32_t*>(smem + L.red);  // [E] keys of the logits
+  if (warp < nrows) {
     const float* wrow = rows + static_cast<size_t>(warp) * H;
     float p = 0.f;
 #pragma unroll 16
     for (int k = lane; k < H; k += 32) p = __fmaf_rn(wrow[k], xf[k], p);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, m));
-    if (lane == 0) D.logits[e0 + warp] = p;
+    // the tagged value is all a reader needs: no ordering with other data
+    if (lane == 0) st_relaxed_u64(S1.tagged + static_cast<size_t>(e0 + warp) * kTagStride, (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(p));
   }
-  const uint64_t gen1 = grid_arrive(S1);
-  for (int blk = warp; blk < H / kQBlock; blk += kNC) {
-    const float v = xf[blk * kQBlock + lane];
-    const float amax = warp_max(fabsf(v));
-    const float d = __fdiv_rn(amax, 127.f);
-    int q = 0;
-    if (d != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(v, d))));
-    reinterpret_cast<int8_t*>(sq4)[blk * kQBlock + lane] = static_cast<int8_t>(q);
-    if (lane == 0) sxd[blk] = d;
-    if (c == 0) {
-      const_cast<int8_t*>(P.xq)[blk * kQBlock + lane] = static_cast<int8_t>(q);
-      if (lane == 0) const_cast<float*>(P.xd)[blk] = d;
+  if (warp == 0) {
+    // ---------------- phase B: poll the E logits of this launch (all loads of
+    // a round in flight at once), while the other warps quantize x
+    constexpr int kPer = kS1MaxE / 32;
+    unsigned long long v[kPer];
+    uint32_t ready = 0, need = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (lane + 32 * i < E) need |= 1u << i;
+    for (uint32_t polls = 0; ready != need; ++polls) {
+      if (polls > kSpinLimit) break;
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if ((need & ~ready) & (1u << i)) v[i] = ld_relaxed_u64(S1.tagged + static_cast<size_t>(lane + 32 * i) * kTagStride);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      if (need & (1u << i)) {
+        const float l = __uint_as_float(static_cast<uint32_t>(v[i]));
+        lg[lane + 32 * i] = l;
+        reinterpret_cast<uint32_t*>(smem + L.red)[lane + 32 * i] = f32_key(l);
+      }
+    }
+    if (!__all_sync(0xffffffffu, ready == need) && lane == 0) {
+      record_status(P.status, MOE_ERR_TIMEOUT);
+      *abort = 1;
     }
   }
   __syncthreads();
-  for (int i = tid; i < H / kQBlock; i += blockDim.x) {
-    int sum = 0;
+  if (*abort) return;
+  {
+    // the K largest logits, larger first, equal logits by lower id.  An entry
+    // outranks another if its key is larger or the keys are equal and its id
+    // lower.  Warp w ranks entries [32w, 32w + 32) among themselves and keeps
+    // its K best; then warp 0 takes the K best candidates, one per round: the
+    // largest key over the warp, then the lowest id holding it.
+    uint32_t* ck = reinterpret_cast<uint32_t*>(smem + L.red + kS1KeyBytes);  // [kNC][kS1MaxK] keys
+    int* ci = reinterpret_cast<int*>(ck + kNC * kS1MaxK);                    // [kNC][kS1MaxK] ids
+    constexpr int kNone = 0x7fffffff;
+    if (lane < kS1MaxK) { ck[warp * kS1MaxK + lane] = 0u; ci[warp * kS1MaxK + lane] = kNone; }
+    __syncwarp();
+    const int e = 32 * warp + lane;
+    if (32 * warp < E) {
+      const uint32_t ke = e < E ? gk[e] : 0u;
+      int r = 0;
 #pragma unroll
-    for (int j = 0; j < kQBlock / 4; ++j) sum = __dp4a(sq4[i * 8 + j], 0x01010101, sum);
-    sxas[i] = sum;
-  }
-  if (!grid_wait(S1, gen1, abort)) return;
-
-  // ---------------- phase B: top-k (every CTA), down prefetch, gate/up
-  if (warp == 0) {
-    for (int e = lane; e < E; e += 32) lg[e] = __ldcg(D.logits + e);
-    __syncwarp();
-    // the K largest logits, larger first, equal logits by lower id: per round
-    // the largest key over the warp, then the lowest id holding it
-    uint32_t used = 0;
-    for (int r = 0; r < K; ++r) {
-      uint32_t bk = 0;
-      int be = 0x7fffffff;
-      for (int i = 0; i * 32 + lane < E; ++i) {
-        if (used & (1u << i)) continue;
-        const uint32_t k = f32_key(lg[i * 32 + lane]);
-        if (k > bk) { bk = k; be = i * 32 + lane; }  // ascending ids: keep the first
+      for (int o = 0; o < 32; ++o) {
+        const uint32_t ko = __shfl_sync(0xffffffffu, ke, o);
+        r += (32 * warp + o < E) && (ko > ke || (ko == ke && o < lane));
       }
-      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-      const int we = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == wk ? static_cast<uint32_t>(be) : 0xffffffffu));
-      if ((we & 31) == lane) used |= 1u << (we >> 5);
-      if (lane == 0) { sel_e[r] = we; sel_w[r] = lg[we]; }
+      if (e < E && r < K) { ck[warp * kS1MaxK + r] = ke; ci[warp * kS1MaxK + r] = e; }
     }
-    __syncwarp();
-    if (lane == 0) {
-      const float l0 = sel_w[0];
-      float den = 0.f;
-      for (int r = 0; r < K; ++r) {
-        sel_w[r] = expf(__fsub_rn(sel_w[r], l0));
-        den = __fadd_rn(den, sel_w[r]);
+    __syncthreads();
+    if (tid < kNC * kS1MaxK) {
+      // rank of each candidate among all candidates
+      const uint32_t kt = ck[tid];
+      const int it = ci[tid];
+      if (it != kNone) {
+        int r = 0;
+#pragma unroll 8
+        for (int o = 0; o < kNC * kS1MaxK; ++o) {
+          const int io = ci[o];
+          const uint32_t ko = ck[o];
+          r += io != kNone && (ko > kt || (ko == kt && io < it));
+        }
+        if (r < K) sel_e[r] = it;
       }
-      for (int r = 0; r < K; ++r) {
-        sel_w[r] = __fdiv_rn(sel_w[r], den);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int my_e = lane < K ? sel_e[lane] : 0;
+      const float my_l = lg[my_e];
+      // softmax over the selected, renormalised: exp(l - l_0) / sum, summed in slot order
+      const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
+      const float ex = lane < K ? expf(__fsub_rn(my_l, l0)) : 0.f;
+      float den = 0.f;
+      for (int r = 0; r < K; ++r) den = __fadd_rn(den, __shfl_sync(0xffffffffu, ex, r));
+      if (lane < K) {
+        const float w = __fdiv_rn(ex, den);
+        sel_e[lane] = my_e;
+        sel_w[lane] = w;
         if (c == 0) {
-          const_cast<int32_t*>(P.idx)[r] = sel_e[r];
-          const_cast<float*>(P.wts)[r] = sel_w[r];
+          const_cast<int32_t*>(P.idx)[lane] = my_e;
+          const_cast<float*>(P.wts)[lane] = w;
         }
       }
     }
@@ -269,6 +294,46 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     };
 #pragma unroll
     for (int k = 0; k < SW; ++k) issue_next(k);
+    {
+      // x -> int8 32-blocks while the first weight blocks are in flight, kU
+      // blocks per warp at a time so that the reductions and divisions of
+      // independent blocks overlap
+      constexpr int kU = 8;
+      const int nblk = H / kQBlock;
+      for (int b0 = warp; b0 < nblk; b0 += kNC * kU) {
+        float xv[kU], am[kU];
+#pragma unroll
+        for (int i = 0; i < kU; ++i) {
+          const int blk = b0 + i * kNC;
+          xv[i] = blk < nblk ? xf[blk * kQBlock + lane] : 0.f;
+          am[i] = fabsf(xv[i]);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+          for (int i = 0; i < kU; ++i) am[i] = fmaxf(am[i], __shfl_xor_sync(0xffffffffu, am[i], m));
+#pragma unroll
+        for (int i = 0; i < kU; ++i) {
+          const int blk = b0 + i * kNC;
+          if (blk < nblk) {
+            const float d = __fdiv_rn(am[i], 127.f);
+            int q = 0;
+            if (d != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(xv[i], d))));
+            reinterpret_cast<int8_t*>(sq4)[blk * kQBlock + lane] = static_cast<int8_t>(q);
+            const int qs = __reduce_add_sync(0xffffffffu, q);
+            if (lane == 0) {
+              sxd[blk] = d;
+              sxas[blk] = qs;
+            }
+            if (c == 0) {
+              const_cast<int8_t*>(P.xq)[blk * kQBlock + lane] = static_cast<int8_t>(q);
+              if (lane == 0) const_cast<float*>(P.xd)[blk] = d;
+            }
+          }
+        }
+      }
+      __syncthreads();
+    }
     int s = 0, ui = 0;
     for (int64_t u = u0; u < u1; ++u, ++ui) {
       const int j = static_cast<int>(u / panels), p = static_cast<int>(u % panels);
@@ -298,32 +363,55 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
         int q = 0;
         if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
         P.aq[static_cast<size_t>(j) * F + p * kPanel + lane] = static_cast<int8_t>(q);
-        if (lane == 0) P.ad[static_cast<size_t>(j) * (F / kQBlock) + p] = dd;
+        const int qs = __reduce_add_sync(0xffffffffu, q);
+        if (lane == 0) {
+          P.ad[static_cast<size_t>(j) * (F / kQBlock) + p] = dd;
+          P.asum[static_cast<size_t>(j) * (F / kQBlock) + p] = qs;
+        }
       }
     }
     cp_wait<0>();
+    // publish this CTA's units: their codes and scales, then the slot counts
+    __syncthreads();
+    if (tid == 0 && u0 < u1) {
+      __threadfence();
+      uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
+      for (int j = static_cast<int>(u0 / panels); j <= static_cast<int>((u1 - 1) / panels); ++j) {
+        const int64_t lo = u0 > static_cast<int64_t>(j) * panels ? u0 : static_cast<int64_t>(j) * panels;
+        const int64_t hi = u1 < static_cast<int64_t>(j + 1) * panels ? u1 : static_cast<int64_t>(j + 1) * panels;
+        atomicAdd(cnt + j, static_cast<uint32_t>(hi - lo));
+      }
+    }
   }
-  const bool synced = grid_sync(S1, abort);
 
   // ---------------- phase C: this CTA's panel of hidden, all slots
   if (has_panel) {
     // the prefetch must land before this CTA reads it or exits
     bool ok = mbar_wait(pbar, 0);
     if (!ok) record_status(P.status, MOE_ERR_TIMEOUT);
-    if (synced && ok) {
+    // every gate/up unit of every slot has been published
+    if (tid < K) {
+      const uint32_t need = static_cast<uint32_t>(F / kPanel);
+      const uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
+      for (uint32_t polls = 0; ld_acquire_gpu(cnt + tid) < need; ++polls) {
+        if (polls > kSpinLimit) {
+          record_status(P.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    if (!*abort && ok) {
       int* aq4 = reinterpret_cast<int*>(smem + L.act);                       // [K][F/4]
       float* ad = reinterpret_cast<float*>(aq4 + K * (F / 4));                 // [K][F/32]
       int* aas = reinterpret_cast<int*>(ad + K * (F / kQBlock));              // [K][F/32]
       float* part = reinterpret_cast<float*>(smem + L.red);                  // [K][32]
       for (int q = tid; q < K * (F / 4); q += blockDim.x)
         aq4[q] = __ldcg(reinterpret_cast<const int*>(P.aq) + q);
-      for (int q = tid; q < K * (F / kQBlock); q += blockDim.x) ad[q] = __ldcg(P.ad + q);
-      __syncthreads();
       for (int q = tid; q < K * (F / kQBlock); q += blockDim.x) {
-        int sum = 0;
-#pragma unroll
-        for (int j = 0; j < kQBlock / 4; ++j) sum = __dp4a(aq4[q * 8 + j], 0x01010101, sum);
-        aas[q] = sum;
+        ad[q] = __ldcg(P.ad + q);
+        aas[q] = __ldcg(P.asum + q);
       }
       __syncthreads();
       for (int j = warp; j < K; j += kNC) {
@@ -352,12 +440,13 @@ bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem) {
   if (P.ntok != 1 || P.hidden > kS1MaxH || P.ffn > kS1MaxF || P.top_k > kS1MaxK) return false;
   if (P.hidden / kPanel > n_sm) return false;
   if (P.n_experts > 2 * n_sm) return false;  // at most two router rows per CTA
+  if (P.n_experts > kS1MaxE) return false;
   const Step1Layout L = step1_layout(P.hidden, P.ffn, P.n_experts, P.top_k);
   *smem = L.total;
   return L.total <= static_cast<size_t>(kMaxDynSmem);
 }
 
-int launch_step1(const Decode2Params& D, uint32_t* bar_count, uint32_t* bar_gen, cudaStream_t stream) {
+int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* slot_cnt, cudaStream_t stream) {
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -367,7 +456,7 @@ int launch_step1(const Decode2Params& D, uint32_t* bar_count, uint32_t* bar_gen,
   }
   size_t smem = 0;
   if (!step1_supported(D.P, D.n_sm, &smem)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "step1: unsupported shape");
-  Step1Params S{D, bar_count, bar_gen};
+  Step1Params S{D, ticket, reinterpret_cast<unsigned long long*>(D.logits), slot_cnt};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(D.n_sm);
   cfg.blockDim = dim3(kNC * 32);
