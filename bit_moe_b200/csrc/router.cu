@@ -8,6 +8,7 @@
 // ascending) followed by xor-butterfly additions at distances 16, 8, 4, 2, 1.
 #include "bitmoe.h"
 #include "common.cuh"
+#include "ptx.cuh"
 #include "router.cuh"
 
 namespace bitmoe {
@@ -30,6 +31,88 @@ __global__ void k_router_logits(const float* __restrict__ x, const float* __rest
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, m));
     if (lane == 0) logits[pair] = p;
+  }
+}
+
+// Many tokens: a CTA computes a 16-token x 16-expert tile of logits.  The
+// evaluation order is the same as above: the chain of lane l (k = l, l+32, ...
+// ascending) is kept by lane l of a warp for each (token, expert) pair of the
+// warp's 8 x 4 micro-tile, and the 32 chains are combined by the same xor
+// butterfly.  x and router rows are staged through shared memory in 256-wide
+// chunks (double-buffered cp.async), so each row is read from L2 once per tile
+// instead of once per logit.
+constexpr int kRtT = 16, kRtE = 16, kRtKC = 256;
+constexpr int kRtMT = 8, kRtME = 4;  // micro-tile per lane: tokens x experts
+
+__global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __restrict__ x,
+                                                             const float* __restrict__ wr, int ntok, int H,
+                                                             int E, float* __restrict__ logits) {
+  extern __shared__ __align__(16) float rsm[];
+  float* xs = rsm;                        // [2][kRtT][kRtKC]
+  float* ws = rsm + 2 * kRtT * kRtKC;     // [2][kRtE][kRtKC]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+  const int wt = (warp >> 2) * kRtMT;     // warp's first token in the tile (2 x 4 warp grid)
+  const int we = (warp & 3) * kRtME;      // warp's first expert in the tile
+  const int nchunk = H / kRtKC;
+  auto stage = [&](int ch, int buf) {
+    // (kRtT + kRtE) rows x 256 floats = 2048 chunks of 16 bytes, 8 per thread
+    for (int c = tid; c < (kRtT + kRtE) * (kRtKC / 4); c += 256) {
+      const int row = c / (kRtKC / 4), q = c % (kRtKC / 4);
+      const bool isx = row < kRtT;
+      const int r = isx ? row : row - kRtT;
+      const int g = isx ? t0 + r : e0 + r;
+      float* dst = (isx ? xs + (buf * kRtT + r) * kRtKC : ws + (buf * kRtE + r) * kRtKC) + q * 4;
+      if (g < (isx ? ntok : E)) {
+        const float* src = (isx ? x : wr) + static_cast<int64_t>(g) * H + ch * kRtKC + q * 4;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+      } else {
+        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  float acc[kRtMT][kRtME];
+#pragma unroll
+  for (int i = 0; i < kRtMT; ++i)
+#pragma unroll
+    for (int j = 0; j < kRtME; ++j) acc[i][j] = 0.f;
+  stage(0, 0);
+  for (int ch = 0; ch < nchunk; ++ch) {
+    const int buf = ch & 1;
+    if (ch + 1 < nchunk) {
+      stage(ch + 1, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const float* xb = xs + (buf * kRtT + wt) * kRtKC;
+    const float* wb = ws + (buf * kRtE + we) * kRtKC;
+#pragma unroll 2
+    for (int k = lane; k < kRtKC; k += 32) {
+      float xv[kRtMT], wv[kRtME];
+#pragma unroll
+      for (int i = 0; i < kRtMT; ++i) xv[i] = xb[i * kRtKC + k];
+#pragma unroll
+      for (int j = 0; j < kRtME; ++j) wv[j] = wb[j * kRtKC + k];
+#pragma unroll
+      for (int i = 0; i < kRtMT; ++i)
+#pragma unroll
+        for (int j = 0; j < kRtME; ++j) acc[i][j] = __fmaf_rn(wv[j], xv[i], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < kRtMT; ++i) {
+#pragma unroll
+    for (int j = 0; j < kRtME; ++j) {
+      float p = acc[i][j];
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, m));
+      const int t = t0 + wt + i, e = e0 + we + j;
+      if (lane == 0 && t < ntok && e < E) logits[static_cast<int64_t>(t) * E + e] = p;
+    }
   }
 }
 
@@ -80,10 +163,23 @@ __global__ void k_topk_softmax(const float* __restrict__ logits, int ntok, int E
 
 int launch_route_topk(const float* x, const float* wr, int ntok, int H, int E, int K, int32_t* idx,
                       float* wts, float* logits, cudaStream_t stream) {
-  const int64_t total = static_cast<int64_t>(ntok) * E;
-  int64_t grid = (total + 7) / 8;
-  if (grid > 148 * 16) grid = 148 * 16;
-  k_router_logits<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, wr, ntok, H, E, logits);
+  if (ntok >= kRtT && H % kRtKC == 0) {
+    const size_t smem = sizeof(float) * 2 * (kRtT + kRtE) * kRtKC;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+      cudaFuncSetAttribute(k_router_logits_tiled, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      attr_done[dev] = true;
+    }
+    const dim3 grid((ntok + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
+    k_router_logits_tiled<<<grid, 256, smem, stream>>>(x, wr, ntok, H, E, logits);
+  } else {
+    const int64_t total = static_cast<int64_t>(ntok) * E;
+    int64_t grid = (total + 7) / 8;
+    if (grid > 148 * 16) grid = 148 * 16;
+    k_router_logits<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, wr, ntok, H, E, logits);
+  }
   note_launch(MOE_K_ROUTER_LOGITS, stream);
   k_topk_softmax<<<(ntok + 3) / 4, 128, 0, stream>>>(logits, ntok, E, K, idx, wts);
   note_launch(MOE_K_TOPK, stream);
