@@ -39,7 +39,6 @@ constexpr int kS1MaxE = kNC * 32;          // experts: one per thread of the CTA
 // One 128-byte line per tagged logit, so that the CTAs polling the logits
 // spread their loads over many L2 lines instead of queueing on a few.
 constexpr int kTagStride = 16;
-constexpr int kS1KeyBytes = kS1MaxE * 4;
 static_assert(kNC * kS1MaxK <= kNC * 32, "top-k candidates: one per thread");
 
 struct Step1Params {
@@ -147,7 +146,6 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   __syncthreads();
   const int nrows = e1 - e0;
   const uint32_t tag = *sgen;
-  const uint32_t* gk = reinterpret_cast<const uint32_t*>(smem + L.red);  // [E] keys of the logits
   if (warp < nrows) {
     const float* wrow = rows + static_cast<size_t>(warp) * H;
     float p = 0.f;
@@ -160,8 +158,10 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   }
   if (warp == 0) {
     // ---------------- phase B: poll the E logits of this launch (all loads of
-    // a round in flight at once), while the other warps quantize x
+    // a round in flight at once), then the top-k, while the other warps
+    // quantize x
     constexpr int kPer = kS1MaxE / 32;
+    constexpr int kNone = 0x7fffffff;
     unsigned long long v[kPer];
     uint32_t ready = 0, need = 0;
 #pragma unroll
@@ -176,63 +176,39 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
       for (int i = 0; i < kPer; ++i)
         if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
     }
+    if (!__all_sync(0xffffffffu, ready == need)) {
+      if (lane == 0) {
+        record_status(P.status, MOE_ERR_TIMEOUT);
+        *abort = 1;
+      }
+    } else {
+      // the K largest logits, larger first, equal logits by lower id: per
+      // round the largest key over the warp, then the lowest id holding it
+      // (a lane's own entries are in ascending id order, so it keeps the first
+      // of equal keys)
+      uint32_t key[kPer];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      if (need & (1u << i)) {
-        const float l = __uint_as_float(static_cast<uint32_t>(v[i]));
-        lg[lane + 32 * i] = l;
-        reinterpret_cast<uint32_t*>(smem + L.red)[lane + 32 * i] = f32_key(l);
-      }
-    }
-    if (!__all_sync(0xffffffffu, ready == need) && lane == 0) {
-      record_status(P.status, MOE_ERR_TIMEOUT);
-      *abort = 1;
-    }
-  }
-  __syncthreads();
-  if (*abort) return;
-  {
-    // the K largest logits, larger first, equal logits by lower id.  An entry
-    // outranks another if its key is larger or the keys are equal and its id
-    // lower.  Warp w ranks entries [32w, 32w + 32) among themselves and keeps
-    // its K best; then warp 0 takes the K best candidates, one per round: the
-    // largest key over the warp, then the lowest id holding it.
-    uint32_t* ck = reinterpret_cast<uint32_t*>(smem + L.red + kS1KeyBytes);  // [kNC][kS1MaxK] keys
-    int* ci = reinterpret_cast<int*>(ck + kNC * kS1MaxK);                    // [kNC][kS1MaxK] ids
-    constexpr int kNone = 0x7fffffff;
-    if (lane < kS1MaxK) { ck[warp * kS1MaxK + lane] = 0u; ci[warp * kS1MaxK + lane] = kNone; }
-    __syncwarp();
-    const int e = 32 * warp + lane;
-    if (32 * warp < E) {
-      const uint32_t ke = e < E ? gk[e] : 0u;
-      int r = 0;
+      for (int i = 0; i < kPer; ++i) key[i] = f32_key(__uint_as_float(static_cast<uint32_t>(v[i])));
+      uint32_t avail = need;
+      int my_e = 0;
+      float my_l = 0.f;
+#pragma unroll 1
+      for (int r = 0; r < K; ++r) {
+        uint32_t bk = 0u;
+        int bi = kNone;
 #pragma unroll
-      for (int o = 0; o < 32; ++o) {
-        const uint32_t ko = __shfl_sync(0xffffffffu, ke, o);
-        r += (32 * warp + o < E) && (ko > ke || (ko == ke && o < lane));
+        for (int i = 0; i < kPer; ++i)
+          if (((avail >> i) & 1u) && (bi == kNone || key[i] > bk)) { bk = key[i]; bi = lane + 32 * i; }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const int wi = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == wk ? static_cast<uint32_t>(bi) : 0xffffffffu));
+        if ((wi & 31) == lane) avail &= ~(1u << (wi >> 5));
+        if (lane == r) my_e = wi;
       }
-      if (e < E && r < K) { ck[warp * kS1MaxK + r] = ke; ci[warp * kS1MaxK + r] = e; }
-    }
-    __syncthreads();
-    if (tid < kNC * kS1MaxK) {
-      // rank of each candidate among all candidates
-      const uint32_t kt = ck[tid];
-      const int it = ci[tid];
-      if (it != kNone) {
-        int r = 0;
-#pragma unroll 8
-        for (int o = 0; o < kNC * kS1MaxK; ++o) {
-          const int io = ci[o];
-          const uint32_t ko = ck[o];
-          r += io != kNone && (ko > kt || (ko == kt && io < it));
-        }
-        if (r < K) sel_e[r] = it;
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const int my_e = lane < K ? sel_e[lane] : 0;
-      const float my_l = lg[my_e];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i)
+        if (lane + 32 * i < E) lg[lane + 32 * i] = __uint_as_float(static_cast<uint32_t>(v[i]));
+      __syncwarp();
+      if (lane < K) my_l = lg[my_e];
       // softmax over the selected, renormalised: exp(l - l_0) / sum, summed in slot order
       const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
       const float ex = lane < K ? expf(__fsub_rn(my_l, l0)) : 0.f;
@@ -248,8 +224,46 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
         }
       }
     }
+  } else {
+    // x -> int8 32-blocks, kU blocks per warp at a time so that the
+    // reductions and divisions of independent blocks overlap
+    constexpr int kU = 8;
+    const int nblk = H / kQBlock, nqw = kNC - 1;
+    for (int b0 = warp - 1; b0 < nblk; b0 += nqw * kU) {
+      float xv[kU], am[kU];
+#pragma unroll
+      for (int i = 0; i < kU; ++i) {
+        const int blk = b0 + i * nqw;
+        xv[i] = blk < nblk ? xf[blk * kQBlock + lane] : 0.f;
+        am[i] = fabsf(xv[i]);
+      }
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+        for (int i = 0; i < kU; ++i) am[i] = fmaxf(am[i], __shfl_xor_sync(0xffffffffu, am[i], m));
+#pragma unroll
+      for (int i = 0; i < kU; ++i) {
+        const int blk = b0 + i * nqw;
+        if (blk < nblk) {
+          const float d = __fdiv_rn(am[i], 127.f);
+          int q = 0;
+          if (d != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(xv[i], d))));
+          reinterpret_cast<int8_t*>(sq4)[blk * kQBlock + lane] = static_cast<int8_t>(q);
+          const int qs = __reduce_add_sync(0xffffffffu, q);
+          if (lane == 0) {
+            sxd[blk] = d;
+            sxas[blk] = qs;
+          }
+          if (c == 0) {
+            const_cast<int8_t*>(P.xq)[blk * kQBlock + lane] = static_cast<int8_t>(q);
+            if (lane == 0) const_cast<float*>(P.xd)[blk] = d;
+          }
+        }
+      }
+    }
   }
   __syncthreads();
+  if (*abort) return;
   // down prefetch: this CTA's panel of hidden for every slot (one issuing
   // thread per slot: the panel's blocks are contiguous, one copy for the
   // digits and one for the scales)
@@ -292,48 +306,8 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
       }
       cp_commit();
     };
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < SW; ++k) issue_next(k);
-    {
-      // x -> int8 32-blocks while the first weight blocks are in flight, kU
-      // blocks per warp at a time so that the reductions and divisions of
-      // independent blocks overlap
-      constexpr int kU = 8;
-      const int nblk = H / kQBlock;
-      for (int b0 = warp; b0 < nblk; b0 += kNC * kU) {
-        float xv[kU], am[kU];
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-          const int blk = b0 + i * kNC;
-          xv[i] = blk < nblk ? xf[blk * kQBlock + lane] : 0.f;
-          am[i] = fabsf(xv[i]);
-        }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1)
-#pragma unroll
-          for (int i = 0; i < kU; ++i) am[i] = fmaxf(am[i], __shfl_xor_sync(0xffffffffu, am[i], m));
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-          const int blk = b0 + i * kNC;
-          if (blk < nblk) {
-            const float d = __fdiv_rn(am[i], 127.f);
-            int q = 0;
-            if (d != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(xv[i], d))));
-            reinterpret_cast<int8_t*>(sq4)[blk * kQBlock + lane] = static_cast<int8_t>(q);
-            const int qs = __reduce_add_sync(0xffffffffu, q);
-            if (lane == 0) {
-              sxd[blk] = d;
-              sxas[blk] = qs;
-            }
-            if (c == 0) {
-              const_cast<int8_t*>(P.xq)[blk * kQBlock + lane] = static_cast<int8_t>(q);
-              if (lane == 0) const_cast<float*>(P.xd)[blk] = d;
-            }
-          }
-        }
-      }
-      __syncthreads();
-    }
     int s = 0, ui = 0;
     for (int64_t u = u0; u < u1; ++u, ++ui) {
       const int j = static_cast<int>(u / panels), p = static_cast<int>(u % panels);
