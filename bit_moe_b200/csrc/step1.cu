@@ -39,7 +39,7 @@ constexpr int kS1MaxE = kNC * 32;          // experts: one per thread of the CTA
 // One 128-byte line per tagged logit, so that the CTAs polling the logits
 // spread their loads over many L2 lines instead of queueing on a few.
 constexpr int kTagStride = 16;
-static_assert(kNC * kS1MaxK <= kNC * 32, "top-k candidates: one per thread");
+static_assert(kS1MaxK <= kNC, "phase C: one warp per slot");
 
 struct Step1Params {
   Decode2Params D;
@@ -287,15 +287,24 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     constexpr int SW = ring_depth<1>();
     const int panels = F / kPanel;
     const int64_t U = static_cast<int64_t>(K) * panels;
-    int64_t u0, u1;
-    cta_range(U, c, C, u0, u1);
+    // this CTA's units: unit c in the first round, then in each later round
+    // the unit counted from the round's end, so that the extra units fall on
+    // the highest CTA ids (those without a panel of hidden) and the slots of
+    // the first round are complete first
+    auto unit_of = [&](int r) -> int64_t {
+      return r == 0 ? static_cast<int64_t>(c) : static_cast<int64_t>(r) * C + (C - 1 - c);
+    };
+    int nmine = 0;
+    while (unit_of(nmine) < U) ++nmine;
     unsigned char* myring = smem + L.ring + static_cast<size_t>(warp) * SW * SL::bytes;
     float* red = reinterpret_cast<float*>(smem + L.red);
-    int64_t iu = u0;
+    uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
+    int im = 0;
     int ib = warp;
     auto issue_next = [&](int slot) {
-      while (iu < u1 && ib >= nbH) { ++iu; ib = warp; }
-      if (iu < u1) {
+      while (im < nmine && ib >= nbH) { ++im; ib = warp; }
+      if (im < nmine) {
+        const int64_t iu = unit_of(im);
         Group G;
         G.expert = sel_e[iu / panels];
         G.count = 1;
@@ -308,8 +317,9 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     };
 #pragma unroll 1
     for (int k = 0; k < SW; ++k) issue_next(k);
-    int s = 0, ui = 0;
-    for (int64_t u = u0; u < u1; ++u, ++ui) {
+    int s = 0;
+    for (int ui = 0; ui < nmine; ++ui) {
+      const int64_t u = unit_of(ui);
       const int j = static_cast<int>(u / panels), p = static_cast<int>(u % panels);
       float part[2][1] = {{0.f}, {0.f}};
       for (int b = warp; b < nbH; b += kNC, ++s) {
@@ -342,20 +352,15 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
           P.ad[static_cast<size_t>(j) * (F / kQBlock) + p] = dd;
           P.asum[static_cast<size_t>(j) * (F / kQBlock) + p] = qs;
         }
+        __syncwarp();
+        if (lane == 0) {  // publish the unit: its codes, scale and sum, then the count
+          __threadfence();
+          atomicAdd(cnt + j, 1u);
+        }
       }
     }
     cp_wait<0>();
-    // publish this CTA's units: their codes and scales, then the slot counts
     __syncthreads();
-    if (tid == 0 && u0 < u1) {
-      __threadfence();
-      uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
-      for (int j = static_cast<int>(u0 / panels); j <= static_cast<int>((u1 - 1) / panels); ++j) {
-        const int64_t lo = u0 > static_cast<int64_t>(j) * panels ? u0 : static_cast<int64_t>(j) * panels;
-        const int64_t hi = u1 < static_cast<int64_t>(j + 1) * panels ? u1 : static_cast<int64_t>(j + 1) * panels;
-        atomicAdd(cnt + j, static_cast<uint32_t>(hi - lo));
-      }
-    }
   }
 
   // ---------------- phase C: this CTA's panel of hidden, all slots
@@ -363,32 +368,37 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     // the prefetch must land before this CTA reads it or exits
     bool ok = mbar_wait(pbar, 0);
     if (!ok) record_status(P.status, MOE_ERR_TIMEOUT);
-    // every gate/up unit of every slot has been published
-    if (tid < K) {
+    // warp j takes slot j as soon as the slot's gate/up units are published
+    // (slots of the first round of units complete first); the slots are
+    // combined in order once all are done
+    int* aq4 = reinterpret_cast<int*>(smem + L.act);                       // [K][F/4]
+    float* ad = reinterpret_cast<float*>(aq4 + K * (F / 4));                 // [K][F/32]
+    int* aas = reinterpret_cast<int*>(ad + K * (F / kQBlock));              // [K][F/32]
+    float* part = reinterpret_cast<float*>(smem + L.red);                  // [K][32]
+    if (warp < K && ok) {
+      const int j = warp;
       const uint32_t need = static_cast<uint32_t>(F / kPanel);
       const uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
-      for (uint32_t polls = 0; ld_acquire_gpu(cnt + tid) < need; ++polls) {
-        if (polls > kSpinLimit) {
-          record_status(P.status, MOE_ERR_TIMEOUT);
-          *abort = 1;
-          break;
+      bool ready = true;
+      if (lane == 0) {
+        for (uint32_t polls = 0; ld_acquire_gpu(cnt + j) < need; ++polls) {
+          if (polls > kSpinLimit) {
+            ready = false;
+            record_status(P.status, MOE_ERR_TIMEOUT);
+            *abort = 1;
+            break;
+          }
         }
       }
-    }
-    __syncthreads();
-    if (!*abort && ok) {
-      int* aq4 = reinterpret_cast<int*>(smem + L.act);                       // [K][F/4]
-      float* ad = reinterpret_cast<float*>(aq4 + K * (F / 4));                 // [K][F/32]
-      int* aas = reinterpret_cast<int*>(ad + K * (F / kQBlock));              // [K][F/32]
-      float* part = reinterpret_cast<float*>(smem + L.red);                  // [K][32]
-      for (int q = tid; q < K * (F / 4); q += blockDim.x)
-        aq4[q] = __ldcg(reinterpret_cast<const int*>(P.aq) + q);
-      for (int q = tid; q < K * (F / kQBlock); q += blockDim.x) {
-        ad[q] = __ldcg(P.ad + q);
-        aas[q] = __ldcg(P.asum + q);
-      }
-      __syncthreads();
-      for (int j = warp; j < K; j += kNC) {
+      ready = __shfl_sync(0xffffffffu, ready, 0);
+      if (ready) {
+        for (int q = lane; q < F / 4; q += 32)
+          aq4[j * (F / 4) + q] = __ldcg(reinterpret_cast<const int*>(P.aq + static_cast<size_t>(j) * F) + q);
+        for (int q = lane; q < F / kQBlock; q += 32) {
+          ad[j * (F / kQBlock) + q] = __ldcg(P.ad + static_cast<size_t>(j) * (F / kQBlock) + q);
+          aas[j * (F / kQBlock) + q] = __ldcg(P.asum + static_cast<size_t>(j) * (F / kQBlock) + q);
+        }
+        __syncwarp();
         float acc[1][1] = {{0.f}};
         const unsigned char* wj = pref + j * pref_slot;
         for (int b = 0; b < nbF; ++b) {
@@ -400,12 +410,12 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
         }
         part[j * 32 + lane] = acc[0][0];
       }
-      __syncthreads();
-      if (warp == 0) {
-        float y = 0.f;
-        for (int j = 0; j < K; ++j) y = __fmaf_rn(sel_w[j], part[j * 32 + lane], y);
-        P.y[panelH * kPanel + lane] = y;
-      }
+    }
+    __syncthreads();
+    if (!*abort && ok && warp == 0) {
+      float y = 0.f;
+      for (int j = 0; j < K; ++j) y = __fmaf_rn(sel_w[j], part[j * 32 + lane], y);
+      P.y[panelH * kPanel + lane] = y;
     }
   }
 }
