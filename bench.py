@@ -88,7 +88,7 @@ def kernel_bytes(wl, unique_experts):
         "prefill_gateup": unique_experts * 2 * matrix_bytes(F, H) + T * H + T * H // 32 * 4
         + pairs * F + pairs * F // 32 * 4,
         "prefill_down": unique_experts * matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4 + pairs * H * 4,
-        "prefill_prep": T * H + T * H // 32 * 4 + 2 * T * H + T * H // 32 * 4,
+        "prefill_gather": pairs * H + pairs * H // 32 * 4,
         "combine": pairs * H * 4 + T * H * 4 + pairs * 4,
         "route": E * H * 4 + T * H * 4 + T * H + T * H // 32 * 4 + T * E * 4 + pairs * 8,
         "quant_act_q8": T * H * 4 + T * H + T * H // 32 * 4,

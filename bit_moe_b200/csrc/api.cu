@@ -68,7 +68,7 @@ int check_device() {
 struct WsLayout {
   size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0, asum = 0;
   size_t xs = 0, ys = 0;  // device copies of x and y for the host-buffer entry point
-  size_t xh = 0, xl = 0, xsum = 0, aqh = 0, aql = 0;  // prefill only
+  size_t bgu = 0, bdn = 0;  // prefill only
   GroupWs grp;
   size_t total = 0;
 };
@@ -96,11 +96,10 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
   L.ys = take(sizeof(float) * T * static_cast<size_t>(H));
   off = group_ws_layout(E, T * K, off, &L.grp);
   if (prefill) {
-    L.xh = take(static_cast<size_t>(T) * H);
-    L.xl = take(static_cast<size_t>(T) * H);
-    L.xsum = take(sizeof(int32_t) * T * static_cast<size_t>(H / kQBlock));
-    L.aqh = take(static_cast<size_t>(T) * K * F);
-    L.aql = take(static_cast<size_t>(T) * K * F);
+    // groups of at most 32 pairs: at most T*K/32 full ones plus one partial per expert
+    const size_t groups = static_cast<size_t>(T) * K / 32 + E + 1;
+    L.bgu = take(groups * (H / kBlock) * prefill_block_bytes());
+    L.bdn = take(groups * (F / kBlock) * prefill_block_bytes());
   }
   L.total = off;
   return L;
@@ -165,12 +164,9 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   P.pairs = reinterpret_cast<const int32_t*>(base + W.grp.pairs);
   P.group_scratch = reinterpret_cast<int32_t*>(base + W.grp.scratch);
   P.group_chunk = kChunk;
-  const bool pf = W.xh != 0;
-  P.xh = pf ? base + W.xh : nullptr;
-  P.xl = pf ? base + W.xl : nullptr;
-  P.xsum = pf ? reinterpret_cast<int32_t*>(base + W.xsum) : nullptr;
-  P.aqh = pf ? base + W.aqh : nullptr;
-  P.aql = pf ? base + W.aql : nullptr;
+  const bool pf = W.bgu != 0;
+  P.bgu = pf ? base + W.bgu : nullptr;
+  P.bdn = pf ? base + W.bdn : nullptr;
   P.asum = reinterpret_cast<int32_t*>(base + W.asum);
   return P;
 }
@@ -431,7 +427,7 @@ int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
 const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
-      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_prep"};
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

@@ -36,11 +36,11 @@ struct DecodeParams {
   const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert
   int32_t* group_scratch;                // [2*(n_experts+1)] counters for the grouping
   int group_chunk;                       // most pairs per item (kChunk for decode)
-  // prefill only: the activation codes split for the e4m3 tensor-core path
-  // (code = 16*hi + lo, both parts exact in e4m3) and the code sums per 32-block
-  uint8_t* xh; uint8_t* xl; int32_t* xsum;   // [ntok][hidden], [ntok][hidden/32]
-  uint8_t* aqh; uint8_t* aql;                // [ntok*top_k][ffn]
-  int32_t* asum;                             // [ntok*top_k][ffn/32] code sums of a^ (prefill, one-token step)
+  // prefill only: the activation blocks of every 32-pair group, laid out as
+  // the tensor-core kernel's shared-memory stages, for gate/up and for down
+  unsigned char* bgu;                        // [groups][hidden/256] blocks
+  unsigned char* bdn;                        // [groups][ffn/256] blocks
+  int32_t* asum;                             // [ntok*top_k][ffn/32] code sums of a^ (one-token step)
 };
 
 // Bytes of workspace the grouped mode needs after `off`; writes the offsets.

@@ -20,13 +20,19 @@
 //     changes every 32 values); the epilogue forms sum(q*a) = 512*D - sum(a)
 //     and scales it in fp32 exactly like the decode kernels: sum over
 //     sub-blocks of d * sum(q*a), then the fp16 weight scale per 256-block.
-// Two warps share each TMEM lane quadrant: both hold the same 32 rows, one
-// decodes the first 32 digit columns and fixes up the first half of the
-// pairs, the other the rest.
+// The activations of a tile are laid out once per (group, 256-block) in HBM
+// exactly as shared memory holds them (split codes in the MMA's core-matrix
+// layout, then the scales and code sums of the 32 pairs): for gate/up by a
+// gather pass over x^, for down by the gate/up epilogue itself.  One bulk copy
+// (TMA) then brings each block's 18 KB into a shared-memory stage.
+// The kernel is persistent (one CTA per SM) and warp-specialized: decode
+// warps write the digits of block i while the MMAs of block i-1 run and the
+// fixup warps drain the accumulators of earlier half blocks; mbarriers pass
+// each stage along (digits: 2 TMEM stages, activations: 3 shared-memory
+// stages, accumulators: 2 TMEM stages of half a block).
 // Gate/up tiles hold 64 gate rows and the 64 matching up rows, so SwiGLU and
-// the requantization run in the epilogue (writing the split codes of the down
-// input); down tiles write each pair's rows, and a last pass combines the
-// top_k slots of every token in slot order.
+// the requantization run in the epilogue; down tiles write each pair's rows,
+// and a last pass combines the top_k slots of every token in slot order.
 #include <cuda_fp8.h>
 
 #include "bitmoe.h"
@@ -37,24 +43,43 @@
 
 namespace bitmoe {
 
-constexpr int kPN = 32;          // pairs per tile (MMA N)
-constexpr int kPM = 128;         // weight rows per tile (MMA M)
-constexpr int kPThreads = 256;   // two warps per TMEM lane quadrant
-constexpr int kPHalf = kPN / 2;  // pairs fixed up by one warp of a quadrant
-constexpr int kTmemCols = 256;   // A: columns [0, 64); D: [64, 64 + 4 * kPN)
-constexpr int kADcol = 0;
-constexpr int kDcol = 64;
+constexpr int kPN = 32;           // pairs per tile (MMA N)
+constexpr int kPM = 128;          // weight rows per tile (MMA M)
+// Warp roles of a CTA (one CTA per SM, persistent over the tiles):
+constexpr int kWDec = 0;          // warps 0-3: decode the digits into TMEM (thread = row)
+constexpr int kWFix = 4;          // warps 4-11: accumulator fixup and epilogue (thread = row,
+constexpr int kFixWarps = 8;      //   warp 4 + 4f + q: rows of quadrant q, pairs [16f, 16f + 16))
+constexpr int kWGat = 12;         // warp 12: lane 0 brings the activation blocks in (bulk copies)
+constexpr int kWMma = 13;         // warp 13: lane 0 issues the MMAs
+constexpr int kPThreads = 14 * 32;
+constexpr int kAStages = 2;       // digit stages in TMEM, 64 columns each
+constexpr int kBStages = 3;       // code / scale stages in shared memory
+constexpr int kDStages = 2;       // accumulator stages: half a block, 4 sub-blocks x kPN columns
+constexpr int kTmemCols = 512;
+constexpr int kAcol = 0;          // A stage a: columns [64a, 64a + 64)
+constexpr int kDcol = 128;        // D stage d: columns [128 + 128d, 256 + 128d)
+
+// One 256-wide block of a tile's activations, identical in HBM and in shared
+// memory: the split codes in the MMA layout, then per pair the 8 sub-block
+// scales and code sums.
+struct BStage {
+  unsigned char hi[kSubPerBlock * kPN * 32];  // 16*h parts
+  unsigned char lo[kSubPerBlock * kPN * 32];  // l parts
+  float d[kPN][kSubPerBlock];                 // activation scales
+  float sa[kPN][kSubPerBlock];                // code sums
+};
+constexpr int kBTile = static_cast<int>(sizeof(BStage));
+static_assert(kBTile % 128 == 0, "bulk copies of whole stages");
 
 struct PrefillSmem {
+  uint64_t a_full[kAStages], a_empty[kAStages];
+  uint64_t b_full[kBStages], b_empty[kBStages], s_empty[kBStages];
+  uint64_t d_full[kDStages], d_empty[kDStages];
+  uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  uint64_t bar;
-  int pairs[kPN];
-  alignas(128) unsigned char Bh[2][kSubPerBlock * kPN * 32];  // 16*h parts, MMA layout, 2 blocks
-  alignas(128) unsigned char Bl[2][kSubPerBlock * kPN * 32];  // l parts
-  alignas(16) float d[kSubPerBlock][kPN];                      // activation scales of the block
-  alignas(16) float na[kSubPerBlock][kPN];                     // minus the code sums
-  float xch[64][kPN + 1];                                      // gate results for the up rows
+  alignas(128) BStage st[kBStages];
+  float xch[64][kPN + 1];  // gate results for the up rows
 };
 
 // Byte offset of activation code (pair n, k in [0, 32)) of sub-block s in B:
@@ -72,33 +97,54 @@ __device__ __forceinline__ void code_split(int q, uint8_t& hi, uint8_t& lo) {
   lo = static_cast<uint8_t>(__nv_cvt_float_to_fp8(static_cast<float>(l), __NV_SATFINITE, __NV_E4M3));
 }
 
-// Split codes and per-32-block code sums of the gate/up input: one warp per
-// 32-block.
-__global__ void k_prefill_prep(DecodeParams P) {
-  const int64_t nblk = static_cast<int64_t>(P.ntok) * (P.hidden / kQBlock);
-  const int lane = threadIdx.x & 31;
-  for (int64_t blk = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; blk < nblk;
-       blk += static_cast<int64_t>(gridDim.x) * blockDim.x / 32) {
-    const int q = P.xq[blk * kQBlock + lane];
-    uint8_t hi, lo;
-    code_split(q, hi, lo);
-    P.xh[blk * kQBlock + lane] = hi;
-    P.xl[blk * kQBlock + lane] = lo;
-    const int sum = __reduce_add_sync(0xffffffffu, q);
-    if (lane == 0) P.xsum[blk] = sum;
+// The gate/up activation blocks of every group: thread (n, s) of a CTA
+// splits the 32 codes of sub-block s of pair n's token and adds them up.
+__global__ void __launch_bounds__(256) k_prefill_gather(DecodeParams P) {
+  const int H = P.hidden, K = P.top_k, nb = H / kBlock;
+  const int64_t work = static_cast<int64_t>(*P.n_items) * nb;
+  const int n = threadIdx.x >> 3, s = threadIdx.x & 7;
+  for (int64_t w = blockIdx.x; w < work; w += gridDim.x) {
+    const Item it = P.items[w / nb];
+    const int b = static_cast<int>(w % nb);
+    BStage* dst = reinterpret_cast<BStage*>(P.bgu) + w;
+    const int pair = n < it.count ? P.pairs[it.start + n] : -1;
+    int4 c[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
+    float d = 0.f;
+    if (pair >= 0) {
+      const int8_t* src = P.xq + static_cast<size_t>(pair / K) * H + b * kBlock + s * kQBlock;
+      c[0] = *reinterpret_cast<const int4*>(src);
+      c[1] = *reinterpret_cast<const int4*>(src + 16);
+      d = P.xd[static_cast<size_t>(pair / K) * (H / kQBlock) + b * kSubPerBlock + s];
+    }
+    int sum = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int8_t* q = reinterpret_cast<const int8_t*>(&c[h]);
+      int4 hv, lv;
+      uint8_t* hb = reinterpret_cast<uint8_t*>(&hv);
+      uint8_t* lb = reinterpret_cast<uint8_t*>(&lv);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        code_split(q[k], hb[k], lb[k]);
+        sum += q[k];
+      }
+      *reinterpret_cast<int4*>(dst->hi + b_off(s, n, 16 * h)) = hv;
+      *reinterpret_cast<int4*>(dst->lo + b_off(s, n, 16 * h)) = lv;
+    }
+    dst->d[n][s] = d;
+    dst->sa[n][s] = static_cast<float>(sum);
   }
 }
 
 // Digit words [32*kHalf, 32*kHalf + 32) of one packed block (digit word
 // 5*j + i holds level i of the four bytes of packed word j): each 16-bit lane
 // keeps u * 3^i, whose high byte H_i grows by one base-3 digit per level and
-// t_i = H_(i+1) - 3*H_i.  `w` holds packed words [6*kHalf, 6*kHalf + 7).
+// t_i = H_(i+1) - 3*H_i.  Packed word 6 feeds both halves.
 template <int kHalf>
-__device__ __forceinline__ void decode_half(const uint32_t (&w)[7], uint32_t (&dg)[32]) {
+__device__ __forceinline__ void decode_half(const uint32_t (&w)[kBlockWords], uint32_t (&dg)[32]) {
 #pragma unroll
-  for (int jj = 0; jj < 7; ++jj) {
-    const int j = 6 * kHalf + jj;
-    uint32_t lo = w[jj] & 0x00FF00FFu, hi = (w[jj] >> 8) & 0x00FF00FFu, hp = 0u;
+  for (int j = 6 * kHalf; j < 6 * kHalf + 7; ++j) {
+    uint32_t lo = w[j] & 0x00FF00FFu, hi = (w[j] >> 8) & 0x00FF00FFu, hp = 0u;
 #pragma unroll
     for (int i = 0; i < 5; ++i) {
       if (j == kBlockWords - 1 && i == 4) break;
@@ -112,24 +158,99 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[7], uint32_t (&d
   }
 }
 
+// Tile t of the grouped GEMM: item (expert, pairs) and 128-row tile index.
+struct TileInfo {
+  Item it;
+  int mt;
+};
+__device__ __forceinline__ TileInfo tile_info(const DecodeParams& P, int t, int m_tiles) {
+  TileInfo T;
+  T.it = P.items[t / m_tiles];
+  T.mt = t % m_tiles;
+  return T;
+}
+
+// The row of this thread in a tile (quadrant q, lane): matrix and panel.
 template <bool kGU>
-__global__ void __launch_bounds__(kPThreads, 2) k_prefill_mma(DecodeParams P) {
+__device__ __forceinline__ void tile_row(const DecodeParams& P, const TileInfo& T, int q, const uint32_t*& trits,
+                                         const uint16_t*& scales, size_t& panel) {
+  if (kGU) {
+    const bool up = q >= 2;
+    trits = up ? P.up_trits : P.gate_trits;
+    scales = up ? P.up_scales : P.gate_scales;
+    panel = (static_cast<size_t>(T.it.expert) * P.ffn + 64 * T.mt) / kPanel + (q & 1);
+  } else {
+    trits = P.down_trits;
+    scales = P.down_scales;
+    panel = (static_cast<size_t>(T.it.expert) * P.hidden + kPM * T.mt) / kPanel + q;
+  }
+}
+
+// The gate/up epilogue's output for pairs [n0, n0 + 16) at ffn row f of a
+// tile: each lane (32 consecutive f, one 32-block) requantizes the SwiGLU
+// values a[] (absent pairs and bad groups: zeros) and writes the split codes,
+// scale and code sum into the down input's activation block of the group.
+__device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, int item, int r, int n0,
+                                                 const float* a, int count, int my_pair, int lane) {
+  const int F = P.ffn;
+  const int f = 64 * mt + r;
+  const int bf = f / kBlock, sub = (f % kBlock) / kQBlock;
+  BStage* dst = reinterpret_cast<BStage*>(P.bdn) + static_cast<size_t>(item) * (F / kBlock) + bf;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    const int np = n0 + n;
+    float dd = 0.f;
+    int qq = 0;
+    if (a != nullptr && np < count) {
+      const float amax = warp_max(fabsf(a[n]));
+      dd = __fdiv_rn(amax, 127.f);
+      if (dd != 0.f) qq = max(-127, min(127, __float2int_rn(__fdiv_rn(a[n], dd))));
+    }
+    uint8_t hi, lo;
+    code_split(qq, hi, lo);
+    dst->hi[b_off(sub, np, lane)] = hi;
+    dst->lo[b_off(sub, np, lane)] = lo;
+    const int sum = __reduce_add_sync(0xffffffffu, qq);
+    if (lane == 0) {
+      dst->d[np][sub] = dd;
+      dst->sa[np][sub] = static_cast<float>(sum);
+    }
+  }
+  (void)my_pair;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, PrefillSmem& S, int32_t* status) {
+  if (*reinterpret_cast<volatile int*>(&S.abort)) return false;
+  if (mbar_wait(bar, parity)) return true;
+  *reinterpret_cast<volatile int*>(&S.abort) = 1;
+  record_status(status, MOE_ERR_TIMEOUT);
+  return false;
+}
+
+template <bool kGU>
+__global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quad = warp & 3, half = warp >> 2;
-  const int H = P.hidden, F = P.ffn, K = P.top_k;
+  const int H = P.hidden, F = P.ffn;
   const int kdim = kGU ? H : F;               // reduction length
   const int nb = kdim / kBlock;
   const int m_tiles = kGU ? F / 64 : H / kPM;
-  const uint32_t idesc = idesc_e4m3(kPM, kPN);
+  const int n_tiles = *P.n_items * m_tiles;
 
   if (warp == 0) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&S.bar, 1);
+    for (int i = 0; i < kAStages; ++i) { mbar_init(&S.a_full[i], 4); mbar_init(&S.a_empty[i], 1); }
+    for (int i = 0; i < kBStages; ++i) {
+      mbar_init(&S.b_full[i], 1);
+      mbar_init(&S.b_empty[i], 1);
+      mbar_init(&S.s_empty[i], kFixWarps);
+    }
+    for (int i = 0; i < kDStages; ++i) { mbar_init(&S.d_full[i], 1); mbar_init(&S.d_empty[i], kFixWarps); }
+    mbar_init(&S.mma_done, 1);
     fence_mbar_init();
     S.abort = 0;
   }
@@ -137,213 +258,218 @@ __global__ void __launch_bounds__(kPThreads, 2) k_prefill_mma(DecodeParams P) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
-  const uint32_t tlane = tbase + (static_cast<uint32_t>(quad * 32) << 16);  // this warp's lane quadrant
-  uint32_t phase = 0;
 
-  const int n_tiles = *P.n_items * m_tiles;
-  for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const Item it = P.items[tile / m_tiles];
-    const int mt = tile % m_tiles;
-    if (tid < kPN) S.pairs[tid] = tid < it.count ? P.pairs[it.start + tid] : -1;
-    __syncthreads();
-    if (it.expert < 0) {  // ids out of range: their outputs are zero
-      if (tid == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
-      for (int n = 0; n < it.count; ++n) {
-        const int pair = S.pairs[n];
-        if (kGU) {
-          if (tid < 64) {
-            const size_t f = static_cast<size_t>(pair) * F + 64 * mt + tid;
-            P.aqh[f] = 0;
-            P.aql[f] = 0;
-            if ((tid & 31) == 0) {
-              P.ad[static_cast<size_t>(pair) * (F / kQBlock) + (64 * mt + tid) / kQBlock] = 0.f;
-              P.asum[static_cast<size_t>(pair) * (F / kQBlock) + (64 * mt + tid) / kQBlock] = 0;
-            }
-          }
-        } else if (tid < kPM) {
-          P.ye[static_cast<size_t>(pair) * H + kPM * mt + tid] = 0.f;
-        }
-      }
-      __syncthreads();
-      continue;
-    }
-    // this thread's weight row: matrix, panel and row within the panel
-    const uint32_t* trits;
-    const uint16_t* scales;
-    size_t panel;
-    if (kGU) {
-      const bool up = quad >= 2;
-      trits = up ? P.up_trits : P.gate_trits;
-      scales = up ? P.up_scales : P.gate_scales;
-      panel = (static_cast<size_t>(it.expert) * F + 64 * mt) / kPanel + (quad & 1);
-    } else {
-      trits = P.down_trits;
-      scales = P.down_scales;
-      panel = (static_cast<size_t>(it.expert) * H + kPM * mt) / kPanel + quad;
-    }
-    float y[kPHalf];
-#pragma unroll
-    for (int n = 0; n < kPHalf; ++n) y[n] = 0.f;
-
-    // Gather block b's split codes of the tile's pairs into B[buf] (zeros for
-    // empty pair slots); one commit group per block.
-    auto gather = [&](int b, int buf) {
-#pragma unroll
-      for (int i = 0; i < (2 * kPN * 16) / kPThreads; ++i) {
-        const int c = tid + i * kPThreads;
-        const int part = c / (kPN * 16), n = (c / 16) % kPN, kc = c & 15;
-        unsigned char* dst = (part ? S.Bl[buf] : S.Bh[buf]) + b_off(kc >> 1, n, (kc & 1) * 16);
-        const int pair = S.pairs[n];
-        if (pair >= 0) {
-          const uint8_t* src = kGU ? (part ? P.xl : P.xh) + static_cast<size_t>(pair / K) * H
-                                   : (part ? P.aql : P.aqh) + static_cast<size_t>(pair) * F;
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
-                       "l"(src + b * kBlock + kc * 16)
-                       : "memory");
-        } else {
-          *reinterpret_cast<int4*>(dst) = make_int4(0, 0, 0, 0);
-        }
-      }
-      asm volatile("cp.async.commit_group;" ::: "memory");
+  if (warp >= kWDec && warp < kWFix) {
+    // ------------------------------------------------ decode: digits -> TMEM
+    const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    // the CTA's sequence of (tile, block): the next one's words are loaded
+    // while the current one is decoded
+    int t = blockIdx.x, b = 0;
+    auto skip_bad = [&]() {
+      while (t < n_tiles && P.items[t / m_tiles].expert < 0) t += gridDim.x;
     };
-    uint32_t wn[7];
-    uint16_t sn;
-    auto load_w = [&](int b) {
-      const size_t pb = panel * nb + b;
+    auto load = [&](int tt, int bb, uint32_t (&w)[kBlockWords]) {
+      const TileInfo T = tile_info(P, tt, m_tiles);
+      const uint32_t* trits;
+      const uint16_t* scales;
+      size_t panel;
+      tile_row<kGU>(P, T, warp, trits, scales, panel);
+      const size_t pb = panel * nb + bb;
 #pragma unroll
-      for (int j = 0; j < 7; ++j)
-        wn[j] = ld_stream_u32(trits + (pb * kBlockWords + 6 * half + j) * kPanel + lane);
-      sn = scales[pb * kPanel + lane];
+      for (int j = 0; j < kBlockWords; ++j) w[j] = ld_stream_u32(trits + (pb * kBlockWords + j) * kPanel + lane);
     };
-    gather(0, 0);
-    load_w(0);
-    for (int b = 0; b < nb; ++b) {
-      const int buf = b & 1;
-      uint32_t w[7];
+    skip_bad();
+    uint32_t wn[kBlockWords];
+    if (t < n_tiles) load(t, 0, wn);
+    for (uint32_t i = 0; t < n_tiles; ++i) {
+      uint32_t w[kBlockWords];
 #pragma unroll
-      for (int j = 0; j < 7; ++j) w[j] = wn[j];
-      const float sw = f16_bits_to_f32(sn);
-      // prefetch block b+1 while this block is decoded, multiplied and scaled
-      if (b + 1 < nb) {
-        gather(b + 1, buf ^ 1);
-        load_w(b + 1);
+      for (int j = 0; j < kBlockWords; ++j) w[j] = wn[j];
+      // advance to the next (tile, block) and start its loads
+      int tn = t, bn = b + 1;
+      if (bn == nb) {
+        bn = 0;
+        tn += gridDim.x;
+        while (tn < n_tiles && P.items[tn / m_tiles].expert < 0) tn += gridDim.x;
       }
-      // ---- A: this warp's 32 digit columns of the rows' block
+      if (tn < n_tiles) load(tn, bn, wn);
+      const int a = i % kAStages;
+      if (!wait_or_abort(&S.a_empty[a], ((i / kAStages) & 1u) ^ 1u, S, P.status)) break;
       {
         uint32_t dg[32];
-        if (half == 0) decode_half<0>(w, dg);
-        else decode_half<1>(w, dg);
-        tmem_st32(tlane + kADcol + 32 * half, dg);
+        decode_half<0>(w, dg);
+        tmem_st32(tlane + kAcol + 64 * a, dg);
       }
-      // ---- scales and code sums of block b
-      if (b + 1 < nb) asm volatile("cp.async.wait_group 1;" ::: "memory");
-      else asm volatile("cp.async.wait_group 0;" ::: "memory");
       {
-        const int s = tid >> 5, n = tid & 31;  // kPThreads == kSubPerBlock * kPN
-        const int pair = S.pairs[n];
-        float dv = 0.f, av = 0.f;
-        if (pair >= 0) {
-          const size_t q = kGU ? static_cast<size_t>(pair / K) * (H / kQBlock) + b * kSubPerBlock + s
-                               : static_cast<size_t>(pair) * (F / kQBlock) + b * kSubPerBlock + s;
-          dv = kGU ? P.xd[q] : P.ad[q];
-          av = static_cast<float>(kGU ? P.xsum[q] : P.asum[q]);
-        }
-        S.d[s][n] = dv;
-        S.na[s][n] = -av;
+        uint32_t dg[32];
+        decode_half<1>(w, dg);
+        tmem_st32(tlane + kAcol + 64 * a + 32, dg);
       }
       tc_wait_st();
-      fence_proxy_async_shared();
       tc_fence_before();
-      __syncthreads();
-      float inner[kPHalf];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a_full[a]);
+      t = tn;
+      b = bn;
+    }
+  } else if (warp < kWGat) {
+    // ------------------------------------------------ fixup and epilogue
+    const int q = (warp - kWFix) & 3, f16 = (warp - kWFix) >> 2;  // lane quadrant, pair half
+    const uint32_t tlane = tbase + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+      const TileInfo T = tile_info(P, t, m_tiles);
+      const int my_pair = lane < T.it.count ? P.pairs[T.it.start + lane] : -1;
+      if (T.it.expert < 0) {  // ids out of range: their outputs are zero
+        if (warp == kWFix && lane == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
+        if (kGU) {
+          if (q >= 2) write_down_codes(P, T.mt, t / m_tiles, 32 * (q - 2) + lane, 16 * f16, nullptr, 0, my_pair, lane);
+        } else {
+          for (int n = 16 * f16; n < 16 * f16 + 16; ++n) {
+            const int pair = __shfl_sync(0xffffffffu, my_pair, n);
+            if (n < T.it.count) P.ye[static_cast<size_t>(pair) * H + kPM * T.mt + 32 * q + lane] = 0.f;
+          }
+        }
+        continue;
+      }
+      const uint32_t* trits;
+      const uint16_t* scales;
+      size_t panel;
+      tile_row<kGU>(P, T, q, trits, scales, panel);
+      float y[16];
 #pragma unroll
-      for (int n = 0; n < kPHalf; ++n) inner[n] = 0.f;
+      for (int n = 0; n < 16; ++n) y[n] = 0.f;
+      uint16_t sn = scales[(panel * nb) * kPanel + lane];
+      bool ok = true;
+      for (int b = 0; b < nb && ok; ++b, ++i) {
+        const float sw = f16_bits_to_f32(sn);
+        if (b + 1 < nb) sn = scales[(panel * nb + b + 1) * kPanel + lane];
+        const int bs = i % kBStages;
+        if (!wait_or_abort(&S.b_full[bs], (i / kBStages) & 1u, S, P.status)) { ok = false; break; }
+        float inner[16];
 #pragma unroll
-      for (int h4 = 0; h4 < 2; ++h4) {
-        if (tid == 0 && !*reinterpret_cast<volatile int*>(&S.abort)) {
+        for (int n = 0; n < 16; ++n) inner[n] = 0.f;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t j2 = 2 * i + h;
+          const int ds = j2 % kDStages;
+          if (!wait_or_abort(&S.d_full[ds], (j2 / kDStages) & 1u, S, P.status)) { ok = false; break; }
+          tc_fence_after();
+          // 4 sub-blocks x this warp's 16 pairs of the half block
+          uint32_t v[4][16];
+#pragma unroll
+          for (int s4 = 0; s4 < 4; ++s4) tmem_ld16(tlane + kDcol + 128 * ds + 32 * s4 + 16 * f16, v[s4]);
+          tc_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.d_empty[ds]);
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            const int np = 16 * f16 + n;
+            const float4 d4 = *reinterpret_cast<const float4*>(&S.st[bs].d[np][4 * h]);
+            const float4 a4 = *reinterpret_cast<const float4*>(&S.st[bs].sa[np][4 * h]);
+            const float dv[4] = {d4.x, d4.y, d4.z, d4.w}, av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+              // 512 * D - sum(a) = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
+              const float qa = __fmaf_rn(__uint_as_float(v[s4][n]), 512.f, -av[s4]);
+              inner[n] = __fmaf_rn(dv[s4], qa, inner[n]);
+            }
+          }
+        }
+        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.s_empty[bs]);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
+      }
+      if (!ok) break;
+      // ---- epilogue (rows 32*q + lane, pairs [16*f16, 16*f16 + 16))
+      if (kGU) {
+        if (q < 2) {
+#pragma unroll
+          for (int n = 0; n < 16; ++n) S.xch[32 * q + lane][16 * f16 + n] = y[n];
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (q >= 2) {
+          const int r = 32 * (q - 2) + lane;  // f offset within the tile
+          float a[16];
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            const float g = S.xch[r][16 * f16 + n];
+            a[n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
+          }
+          write_down_codes(P, T.mt, t / m_tiles, r, 16 * f16, a, T.it.count, my_pair, lane);
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+      } else {
+        const int hrow = kPM * T.mt + 32 * q + lane;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          const int np = 16 * f16 + n;
+          const int pair = __shfl_sync(0xffffffffu, my_pair, np);
+          if (np < T.it.count) P.ye[static_cast<size_t>(pair) * H + hrow] = y[n];
+        }
+      }
+    }
+  } else if (warp == kWGat && lane == 0) {
+    // ------------------------------------------------ activation blocks: one bulk copy each
+    const unsigned char* src = kGU ? P.bgu : P.bdn;
+    const uint64_t pol = policy_evict_last();  // each block serves all the group's row tiles
+    uint32_t i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+      const int item = t / m_tiles;
+      if (P.items[item].expert < 0) continue;
+      bool ok = true;
+      for (int b = 0; b < nb; ++b, ++i) {
+        const int bs = i % kBStages;
+        const uint32_t par = ((i / kBStages) & 1u) ^ 1u;
+        if (!wait_or_abort(&S.b_empty[bs], par, S, P.status) || !wait_or_abort(&S.s_empty[bs], par, S, P.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&S.b_full[bs], kBTile);
+        bulk_g2s(&S.st[bs], src + (static_cast<size_t>(item) * nb + b) * kBTile, kBTile, &S.b_full[bs], pol);
+      }
+      if (!ok) break;
+    }
+  } else if (warp == kWMma && lane == 0) {
+    // ------------------------------------------------ MMA issue
+    const uint32_t idesc = idesc_e4m3(kPM, kPN);
+    uint32_t i = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      if (P.items[t / m_tiles].expert < 0) continue;
+      for (int b = 0; b < nb; ++b, ++i) {
+        const int a = i % kAStages, bs = i % kBStages;
+        if (!wait_or_abort(&S.a_full[a], (i / kAStages) & 1u, S, P.status) ||
+            !wait_or_abort(&S.b_full[bs], (i / kBStages) & 1u, S, P.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t j2 = 2 * i + h;
+          const int ds = j2 % kDStages;
+          if (!wait_or_abort(&S.d_empty[ds], ((j2 / kDStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int s4 = 0; s4 < 4; ++s4) {
-            const int s = 4 * h4 + s4;
-            const uint32_t dcol = tbase + kDcol + s4 * kPN, acol = tbase + kADcol + 8 * s;
-            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.Bh[buf] + s * (kPN * 32)), 128, 256), idesc, false);
-            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.Bl[buf] + s * (kPN * 32)), 128, 256), idesc, true);
+            const int s = 4 * h + s4;
+            const uint32_t dcol = tbase + kDcol + 128 * ds + 32 * s4, acol = tbase + kAcol + 64 * a + 8 * s;
+            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.st[bs].hi + s * (kPN * 32)), 128, 256), idesc, false);
+            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.st[bs].lo + s * (kPN * 32)), 128, 256), idesc, true);
           }
-          mma_commit(&S.bar);
+          mma_commit(&S.d_full[ds]);
         }
-        if (!*reinterpret_cast<volatile int*>(&S.abort) && !mbar_wait(&S.bar, phase & 1)) {
-          S.abort = 1;
-          record_status(P.status, MOE_ERR_TIMEOUT);
-        }
-        ++phase;
-        tc_fence_after();
-#pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-          const int s = 4 * h4 + s4;
-          uint32_t v[16];
-          tmem_ld16(tlane + kDcol + s4 * kPN + kPHalf * half, v);
-          tc_wait_ld();
-          const float4* dp = reinterpret_cast<const float4*>(&S.d[s][kPHalf * half]);
-          const float4* ap = reinterpret_cast<const float4*>(&S.na[s][kPHalf * half]);
-#pragma unroll
-          for (int n4 = 0; n4 < kPHalf / 4; ++n4) {
-            const float4 dd = dp[n4], aa = ap[n4];
-            const float dv[4] = {dd.x, dd.y, dd.z, dd.w}, av[4] = {aa.x, aa.y, aa.z, aa.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int n = 4 * n4 + e;
-              // 512 * D - sum(a) = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
-              const float qa = __fmaf_rn(__uint_as_float(v[n]), 512.f, av[e]);
-              inner[n] = __fmaf_rn(dv[e], qa, inner[n]);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncthreads();
+        if (!ok) break;
+        mma_commit(&S.a_empty[a]);
+        mma_commit(&S.b_empty[bs]);
       }
-#pragma unroll
-      for (int n = 0; n < kPHalf; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
     }
-
-    // ---- epilogue (this warp: rows 32*quad + lane, pairs kPHalf*half + n)
-    const int n0 = kPHalf * half;
-    if (kGU) {
-      if (quad < 2) {
-#pragma unroll
-        for (int n = 0; n < kPHalf; ++n) S.xch[32 * quad + lane][n0 + n] = y[n];
-      }
-      __syncthreads();
-      if (quad >= 2) {
-        const int r = 32 * (quad - 2) + lane;  // f offset within the tile
-        const int f = 64 * mt + r;
-#pragma unroll
-        for (int n = 0; n < kPHalf; ++n) {
-          if (n0 + n >= it.count) break;
-          const float g = S.xch[r][n0 + n];
-          const float a = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
-          const float amax = warp_max(fabsf(a));
-          const float dd = __fdiv_rn(amax, 127.f);
-          int q = 0;
-          if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
-          const int pair = S.pairs[n0 + n];
-          uint8_t hi, lo;
-          code_split(q, hi, lo);
-          P.aqh[static_cast<size_t>(pair) * F + f] = hi;
-          P.aql[static_cast<size_t>(pair) * F + f] = lo;
-          const int sum = __reduce_add_sync(0xffffffffu, q);
-          if (lane == 0) {
-            P.ad[static_cast<size_t>(pair) * (F / kQBlock) + f / kQBlock] = dd;
-            P.asum[static_cast<size_t>(pair) * (F / kQBlock) + f / kQBlock] = sum;
-          }
-        }
-      }
-    } else {
-      const int h = kPM * mt + 32 * quad + lane;
-#pragma unroll
-      for (int n = 0; n < kPHalf; ++n)
-        if (n0 + n < it.count) P.ye[static_cast<size_t>(S.pairs[n0 + n]) * H + h] = y[n];
-    }
-    __syncthreads();
+    // every MMA has completed before the columns are released
+    mma_commit(&S.mma_done);
+    if (!mbar_wait(&S.mma_done, 0)) record_status(P.status, MOE_ERR_TIMEOUT);
   }
   tc_fence_before();
   __syncthreads();
@@ -364,10 +490,13 @@ __global__ void k_combine(DecodeParams P) {
 }
 
 static size_t prefill_smem() {
-  // at least 80 KB so that no more than two CTAs (2 x 256 TMEM columns) share an SM
+  // more than half of the SM's shared memory, so that one CTA (holding all 512
+  // TMEM columns) runs per SM
   const size_t s = sizeof(PrefillSmem) + 1024;
-  return s < 80 * 1024 ? 80 * 1024 : s;
+  return s < 120 * 1024 ? 120 * 1024 : s;
 }
+
+size_t prefill_block_bytes() { return kBTile; }
 
 int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   DecodeParams P = P0;
@@ -386,11 +515,11 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = prefill_smem();
-  k_prefill_prep<<<2 * n_sm, 256, 0, stream>>>(P);
-  note_launch(MOE_K_PREFILL_PREP, stream);
-  k_prefill_mma<true><<<2 * n_sm, kPThreads, smem, stream>>>(P);
+  k_prefill_gather<<<4 * n_sm, 256, 0, stream>>>(P);
+  note_launch(MOE_K_PREFILL_GATHER, stream);
+  k_prefill_mma<true><<<n_sm, kPThreads, smem, stream>>>(P);
   note_launch(MOE_K_PREFILL_GATEUP, stream);
-  k_prefill_mma<false><<<2 * n_sm, kPThreads, smem, stream>>>(P);
+  k_prefill_mma<false><<<n_sm, kPThreads, smem, stream>>>(P);
   note_launch(MOE_K_PREFILL_DOWN, stream);
   k_combine<<<4 * n_sm, 256, 0, stream>>>(P);
   note_launch(MOE_K_COMBINE, stream);

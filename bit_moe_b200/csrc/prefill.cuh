@@ -3,4 +3,6 @@
 #include "decode.cuh"
 namespace bitmoe {
 int launch_prefill(const DecodeParams& P, cudaStream_t stream);
+// Bytes of one activation block of a 32-pair group (split codes, scales, sums).
+size_t prefill_block_bytes();
 }  // namespace bitmoe
