@@ -47,26 +47,29 @@ constexpr int kPN = 32;           // pairs per tile (MMA N)
 constexpr int kPM = 128;          // weight rows per tile (MMA M)
 // Warp roles of a CTA (one CTA per SM, persistent over the tiles):
 constexpr int kWDec = 0;          // warps 0-3: decode the digits into TMEM (thread = row)
-constexpr int kWFix = 4;          // warps 4-11: accumulator fixup and epilogue (thread = row,
-constexpr int kFixWarps = 8;      //   warp 4 + 4f + q: rows of quadrant q, pairs [16f, 16f + 16))
-constexpr int kWGat = 12;         // warp 12: lane 0 brings the activation blocks in (bulk copies)
-constexpr int kWMma = 13;         // warp 13: lane 0 issues the MMAs
-constexpr int kPThreads = 14 * 32;
+constexpr int kWFix = 4;          // warps 4-19: accumulator fixup and epilogue (thread = row,
+constexpr int kFixWarps = 16;     //   warp 4 + 4f + q: rows of quadrant q, pairs [8f, 8f + 8))
+constexpr int kFixPairs = kPN / (kFixWarps / 4);
+constexpr int kWGat = 20;         // warp 20: lane 0 brings the activation blocks in (bulk copies)
+constexpr int kWMma = 21;         // warp 21: lane 0 issues the MMAs
+constexpr int kPThreads = 22 * 32;
 constexpr int kAStages = 2;       // digit stages in TMEM, 64 columns each
 constexpr int kBStages = 3;       // code / scale stages in shared memory
-constexpr int kDStages = 2;       // accumulator stages: half a block, 4 sub-blocks x kPN columns
+constexpr int kQSub = 4;          // sub-blocks per accumulator stage (half a block)
+constexpr int kDStages = 3;       // accumulator stages in flight
 constexpr int kTmemCols = 512;
 constexpr int kAcol = 0;          // A stage a: columns [64a, 64a + 64)
-constexpr int kDcol = 128;        // D stage d: columns [128 + 128d, 256 + 128d)
+constexpr int kDSub = kPN;        // D columns per sub-block: one fp32 accumulator per pair
+constexpr int kDcol = 128;        // D stage d: columns [128 + kQSub*kDSub*d, 128 + kQSub*kDSub*(d+1))
+static_assert(kDcol + kDStages * kQSub * kDSub <= 512, "tensor memory columns");
 
 // One 256-wide block of a tile's activations, identical in HBM and in shared
-// memory: the split codes in the MMA layout, then per pair the 8 sub-block
-// scales and code sums.
+// memory: the split codes in the MMA layout, then per sub-block the 32 pairs'
+// scales and code sums (negated).
 struct BStage {
-  unsigned char hi[kSubPerBlock * kPN * 32];  // 16*h parts
-  unsigned char lo[kSubPerBlock * kPN * 32];  // l parts
-  float d[kPN][kSubPerBlock];                 // activation scales
-  float sa[kPN][kSubPerBlock];                // code sums
+  unsigned char codes[2][kSubPerBlock * kPN * 32];  // 16*h parts, then l parts, MMA layout
+  float d[kSubPerBlock][kPN];                        // activation scales
+  float nsa[kSubPerBlock][kPN];                      // minus the code sums
 };
 constexpr int kBTile = static_cast<int>(sizeof(BStage));
 static_assert(kBTile % 128 == 0, "bulk copies of whole stages");
@@ -82,9 +85,9 @@ struct PrefillSmem {
   float xch[64][kPN + 1];  // gate results for the up rows
 };
 
-// Byte offset of activation code (pair n, k in [0, 32)) of sub-block s in B:
-// 8-row x 16-byte core matrices, the two 16-byte halves of K 128 bytes apart,
-// consecutive 8-pair groups 256 bytes apart.
+// Byte offset of activation code (pair n, k in [0, 32)) of sub-block s in one
+// part's B operand: 8-row x 16-byte core matrices, the two 16-byte halves of K
+// 128 bytes apart, consecutive 8-pair groups 256 bytes apart.
 __device__ __forceinline__ int b_off(int s, int n, int k) {
   return s * (kPN * 32) + (n >> 3) * 256 + (k >> 4) * 128 + (n & 7) * 16 + (k & 15);
 }
@@ -128,11 +131,11 @@ __global__ void __launch_bounds__(256) k_prefill_gather(DecodeParams P) {
         code_split(q[k], hb[k], lb[k]);
         sum += q[k];
       }
-      *reinterpret_cast<int4*>(dst->hi + b_off(s, n, 16 * h)) = hv;
-      *reinterpret_cast<int4*>(dst->lo + b_off(s, n, 16 * h)) = lv;
+      *reinterpret_cast<int4*>(dst->codes[0] + b_off(s, n, 16 * h)) = hv;
+      *reinterpret_cast<int4*>(dst->codes[1] + b_off(s, n, 16 * h)) = lv;
     }
-    dst->d[n][s] = d;
-    dst->sa[n][s] = static_cast<float>(sum);
+    dst->d[s][n] = d;
+    dst->nsa[s][n] = -static_cast<float>(sum);
   }
 }
 
@@ -156,6 +159,16 @@ __device__ __forceinline__ void decode_half(const uint32_t (&w)[kBlockWords], ui
       hp = hn;
     }
   }
+}
+
+// Two independent fp32 fused multiply-adds, round to nearest each, in one
+// packed instruction: (r0, r1) = (a0*b0 + c0, a1*b1 + c1).
+__device__ __forceinline__ void fma2(float& r0, float& r1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
 // Tile t of the grouped GEMM: item (expert, pairs) and 128-row tile index.
@@ -186,18 +199,18 @@ __device__ __forceinline__ void tile_row(const DecodeParams& P, const TileInfo& 
   }
 }
 
-// The gate/up epilogue's output for pairs [n0, n0 + 16) at ffn row f of a
+// The gate/up epilogue's output for pairs [n0, n0 + kFixPairs) at ffn row f of a
 // tile: each lane (32 consecutive f, one 32-block) requantizes the SwiGLU
 // values a[] (absent pairs and bad groups: zeros) and writes the split codes,
 // scale and code sum into the down input's activation block of the group.
 __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, int item, int r, int n0,
-                                                 const float* a, int count, int my_pair, int lane) {
+                                                 const float* a, int count, int lane) {
   const int F = P.ffn;
   const int f = 64 * mt + r;
   const int bf = f / kBlock, sub = (f % kBlock) / kQBlock;
   BStage* dst = reinterpret_cast<BStage*>(P.bdn) + static_cast<size_t>(item) * (F / kBlock) + bf;
 #pragma unroll
-  for (int n = 0; n < 16; ++n) {
+  for (int n = 0; n < kFixPairs; ++n) {
     const int np = n0 + n;
     float dd = 0.f;
     int qq = 0;
@@ -208,20 +221,19 @@ __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, 
     }
     uint8_t hi, lo;
     code_split(qq, hi, lo);
-    dst->hi[b_off(sub, np, lane)] = hi;
-    dst->lo[b_off(sub, np, lane)] = lo;
+    dst->codes[0][b_off(sub, np, lane)] = hi;
+    dst->codes[1][b_off(sub, np, lane)] = lo;
     const int sum = __reduce_add_sync(0xffffffffu, qq);
     if (lane == 0) {
-      dst->d[np][sub] = dd;
-      dst->sa[np][sub] = static_cast<float>(sum);
+      dst->d[sub][np] = dd;
+      dst->nsa[sub][np] = -static_cast<float>(sum);
     }
   }
-  (void)my_pair;
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, PrefillSmem& S, int32_t* status) {
   if (*reinterpret_cast<volatile int*>(&S.abort)) return false;
-  if (mbar_wait(bar, parity)) return true;
+  if (mbar_wait_sleep(bar, parity)) return true;
   *reinterpret_cast<volatile int*>(&S.abort) = 1;
   record_status(status, MOE_ERR_TIMEOUT);
   return false;
@@ -314,7 +326,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
     }
   } else if (warp < kWGat) {
     // ------------------------------------------------ fixup and epilogue
-    const int q = (warp - kWFix) & 3, f16 = (warp - kWFix) >> 2;  // lane quadrant, pair half
+    const int q = (warp - kWFix) & 3, f16 = (warp - kWFix) >> 2;  // lane quadrant, pair group
     const uint32_t tlane = tbase + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
@@ -323,9 +335,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       if (T.it.expert < 0) {  // ids out of range: their outputs are zero
         if (warp == kWFix && lane == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
         if (kGU) {
-          if (q >= 2) write_down_codes(P, T.mt, t / m_tiles, 32 * (q - 2) + lane, 16 * f16, nullptr, 0, my_pair, lane);
+          if (q >= 2) write_down_codes(P, T.mt, t / m_tiles, 32 * (q - 2) + lane, kFixPairs * f16, nullptr, 0, lane);
         } else {
-          for (int n = 16 * f16; n < 16 * f16 + 16; ++n) {
+          for (int n = kFixPairs * f16; n < kFixPairs * f16 + kFixPairs; ++n) {
             const int pair = __shfl_sync(0xffffffffu, my_pair, n);
             if (n < T.it.count) P.ye[static_cast<size_t>(pair) * H + kPM * T.mt + 32 * q + lane] = 0.f;
           }
@@ -336,9 +348,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       const uint16_t* scales;
       size_t panel;
       tile_row<kGU>(P, T, q, trits, scales, panel);
-      float y[16];
+      float y[kFixPairs];
 #pragma unroll
-      for (int n = 0; n < 16; ++n) y[n] = 0.f;
+      for (int n = 0; n < kFixPairs; ++n) y[n] = 0.f;
       uint16_t sn = scales[(panel * nb) * kPanel + lane];
       bool ok = true;
       for (int b = 0; b < nb && ok; ++b, ++i) {
@@ -346,34 +358,39 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         if (b + 1 < nb) sn = scales[(panel * nb + b + 1) * kPanel + lane];
         const int bs = i % kBStages;
         if (!wait_or_abort(&S.b_full[bs], (i / kBStages) & 1u, S, P.status)) { ok = false; break; }
-        float inner[16];
+        float inner[kFixPairs];
 #pragma unroll
-        for (int n = 0; n < 16; ++n) inner[n] = 0.f;
+        for (int n = 0; n < kFixPairs; ++n) inner[n] = 0.f;
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t j2 = 2 * i + h;
+        for (int h = 0; h < kSubPerBlock / kQSub; ++h) {
+          const uint32_t j2 = (kSubPerBlock / kQSub) * i + h;
           const int ds = j2 % kDStages;
           if (!wait_or_abort(&S.d_full[ds], (j2 / kDStages) & 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
-          // 4 sub-blocks x this warp's 16 pairs of the half block
-          uint32_t v[4][16];
+          // kQSub sub-blocks x this warp's pairs
+          uint32_t v[kQSub][kFixPairs];
 #pragma unroll
-          for (int s4 = 0; s4 < 4; ++s4) tmem_ld16(tlane + kDcol + 128 * ds + 32 * s4 + 16 * f16, v[s4]);
+          for (int s2 = 0; s2 < kQSub; ++s2)
+            tmem_ld8(tlane + kDcol + kQSub * kDSub * ds + kDSub * s2 + kFixPairs * f16, v[s2]);
           tc_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.d_empty[ds]);
 #pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            const int np = 16 * f16 + n;
-            const float4 d4 = *reinterpret_cast<const float4*>(&S.st[bs].d[np][4 * h]);
-            const float4 a4 = *reinterpret_cast<const float4*>(&S.st[bs].sa[np][4 * h]);
-            const float dv[4] = {d4.x, d4.y, d4.z, d4.w}, av[4] = {a4.x, a4.y, a4.z, a4.w};
+          for (int s2 = 0; s2 < kQSub; ++s2) {
+            const int s = kQSub * h + s2;
+            const float4* dp = reinterpret_cast<const float4*>(&S.st[bs].d[s][kFixPairs * f16]);
+            const float4* ap = reinterpret_cast<const float4*>(&S.st[bs].nsa[s][kFixPairs * f16]);
 #pragma unroll
-            for (int s4 = 0; s4 < 4; ++s4) {
+            for (int n4 = 0; n4 < kFixPairs / 4; ++n4) {
+              const float4 dd = dp[n4], aa = ap[n4];
               // 512 * D - sum(a) = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
-              const float qa = __fmaf_rn(__uint_as_float(v[s4][n]), 512.f, -av[s4]);
-              inner[n] = __fmaf_rn(dv[s4], qa, inner[n]);
+              const uint32_t* vv = &v[s2][4 * n4];
+              float q0, q1, q2, q3;
+              fma2(q0, q1, __uint_as_float(vv[0]), __uint_as_float(vv[1]), 512.f, 512.f, aa.x, aa.y);
+              fma2(q2, q3, __uint_as_float(vv[2]), __uint_as_float(vv[3]), 512.f, 512.f, aa.z, aa.w);
+              fma2(inner[4 * n4], inner[4 * n4 + 1], dd.x, dd.y, q0, q1, inner[4 * n4], inner[4 * n4 + 1]);
+              fma2(inner[4 * n4 + 2], inner[4 * n4 + 3], dd.z, dd.w, q2, q3, inner[4 * n4 + 2], inner[4 * n4 + 3]);
             }
           }
         }
@@ -381,32 +398,32 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.s_empty[bs]);
 #pragma unroll
-        for (int n = 0; n < 16; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
+        for (int n = 0; n < kFixPairs; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
       }
       if (!ok) break;
-      // ---- epilogue (rows 32*q + lane, pairs [16*f16, 16*f16 + 16))
+      // ---- epilogue (rows 32*q + lane, pairs [kFixPairs*f16, kFixPairs*f16 + kFixPairs))
       if (kGU) {
         if (q < 2) {
 #pragma unroll
-          for (int n = 0; n < 16; ++n) S.xch[32 * q + lane][16 * f16 + n] = y[n];
+          for (int n = 0; n < kFixPairs; ++n) S.xch[32 * q + lane][kFixPairs * f16 + n] = y[n];
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(kFixWarps * 32) : "memory");
         if (q >= 2) {
           const int r = 32 * (q - 2) + lane;  // f offset within the tile
-          float a[16];
+          float a[kFixPairs];
 #pragma unroll
-          for (int n = 0; n < 16; ++n) {
-            const float g = S.xch[r][16 * f16 + n];
+          for (int n = 0; n < kFixPairs; ++n) {
+            const float g = S.xch[r][kFixPairs * f16 + n];
             a[n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
           }
-          write_down_codes(P, T.mt, t / m_tiles, r, 16 * f16, a, T.it.count, my_pair, lane);
+          write_down_codes(P, T.mt, t / m_tiles, r, kFixPairs * f16, a, T.it.count, lane);
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(kFixWarps * 32) : "memory");
       } else {
         const int hrow = kPM * T.mt + 32 * q + lane;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          const int np = 16 * f16 + n;
+        for (int n = 0; n < kFixPairs; ++n) {
+          const int np = kFixPairs * f16 + n;
           const int pair = __shfl_sync(0xffffffffu, my_pair, np);
           if (np < T.it.count) P.ye[static_cast<size_t>(pair) * H + hrow] = y[n];
         }
@@ -448,17 +465,21 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
           break;
         }
         tc_fence_after();
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t j2 = 2 * i + h;
+        const uint64_t bdesc0 = smem_desc(smem_u32(S.st[bs].codes[0]), 128, 256);
+        const uint64_t bdesc1 = smem_desc(smem_u32(S.st[bs].codes[1]), 128, 256);
+        for (int h = 0; h < kSubPerBlock / kQSub; ++h) {
+          const uint32_t j2 = (kSubPerBlock / kQSub) * i + h;
           const int ds = j2 % kDStages;
           if (!wait_or_abort(&S.d_empty[ds], ((j2 / kDStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
-          for (int s4 = 0; s4 < 4; ++s4) {
-            const int s = 4 * h + s4;
-            const uint32_t dcol = tbase + kDcol + 128 * ds + 32 * s4, acol = tbase + kAcol + 64 * a + 8 * s;
-            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.st[bs].hi + s * (kPN * 32)), 128, 256), idesc, false);
-            mma_f8_ts(dcol, acol, smem_desc(smem_u32(S.st[bs].lo + s * (kPN * 32)), 128, 256), idesc, true);
+          for (int s2 = 0; s2 < kQSub; ++s2) {
+            const int s = kQSub * h + s2;
+            // start address field (bits 0-13, address >> 4) advanced by the sub-block's offset
+            const uint64_t off = static_cast<uint64_t>((s * kPN * 32) >> 4);
+            const uint32_t dcol = tbase + kDcol + kQSub * kDSub * ds + kDSub * s2, acol = tbase + kAcol + 64 * a + 8 * s;
+            mma_f8_ts(dcol, acol, bdesc0 + off, idesc, false);
+            mma_f8_ts(dcol, acol, bdesc1 + off, idesc, true);
           }
           mma_commit(&S.d_full[ds]);
         }

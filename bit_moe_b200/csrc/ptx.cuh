@@ -44,6 +44,25 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Wait for the phase with the given parity to complete, the thread suspended
+// in the barrier between checks (each check gives up after a hint of 20 us,
+// so that a waiting warp takes no issue slots from the working ones).
+// Returns false after about 2^17 checks (seconds).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t i = 0; i < (1u << 17); ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity), "r"(20000u)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false if the
 // poll budget ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
