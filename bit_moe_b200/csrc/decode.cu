@@ -44,6 +44,7 @@ size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G) {
 constexpr int kGroupThreads = 1024;
 
 __global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
+  pdl_enter();
   using Scan = cub::BlockScan<int, kGroupThreads>;
   __shared__ typename Scan::TempStorage scan_tmp;
   __shared__ int cnt[kMaxExperts + 1];
@@ -176,6 +177,7 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
 
 template <int NTMAX>
 __global__ void __launch_bounds__(kGateUpWarps * 32) k_gateup(DecodeParams P) {
+  pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
   Item item;
   if (!fetch_item(P, blockIdx.y, item)) return;
@@ -264,6 +266,7 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
 
 template <int NTMAX>
 __global__ void __launch_bounds__(kDownWarps * 32) k_down(DecodeParams P) {
+  pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
   Item item;
   if (!fetch_item(P, blockIdx.y, item)) return;
@@ -346,7 +349,7 @@ static void init_kernel_attrs() {
 }
 
 int launch_group(const DecodeParams& P, cudaStream_t stream) {
-  k_group<<<1, kGroupThreads, 0, stream>>>(P);
+  launch_k(k_group, dim3(1), dim3(kGroupThreads), 0, stream, P);
   note_launch(MOE_K_GROUP, stream);
   return check_launch("group");
 }
@@ -358,16 +361,16 @@ int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
   if (P.direct) {
     const size_t s1 = ActSmem<1>::bytes(P.hidden) + 2 * kGateUpWarps * 1 * 32 * 4;
     const size_t s2 = ActSmem<1>::bytes(P.ffn);
-    k_gateup<1><<<dim3(P.ffn / kPanel, npairs), kGateUpWarps * 32, s1, stream>>>(P);
+    launch_k(k_gateup<1>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
     note_launch(MOE_K_GATEUP, stream);
-    k_down<1><<<dim3(P.hidden / kPanel / kDownWarps, npairs), kDownWarps * 32, s2, stream>>>(P);
+    launch_k(k_down<1>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
     note_launch(MOE_K_DOWN, stream);
   } else {
     const size_t s1 = ActSmem<kChunk>::bytes(P.hidden) + 2 * kGateUpWarps * kChunk * 32 * 4;
     const size_t s2 = ActSmem<kChunk>::bytes(P.ffn);
-    k_gateup<kChunk><<<dim3(P.ffn / kPanel, npairs), kGateUpWarps * 32, s1, stream>>>(P);
+    launch_k(k_gateup<kChunk>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
     note_launch(MOE_K_GATEUP, stream);
-    k_down<kChunk><<<dim3(P.hidden / kPanel / kDownWarps, npairs), kDownWarps * 32, s2, stream>>>(P);
+    launch_k(k_down<kChunk>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
     note_launch(MOE_K_DOWN, stream);
   }
   return check_launch("expert_ffn");

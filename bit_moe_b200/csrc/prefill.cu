@@ -103,6 +103,7 @@ __device__ __forceinline__ void code_split(int q, uint8_t& hi, uint8_t& lo) {
 // The gate/up activation blocks of every group: thread (n, s) of a CTA
 // splits the 32 codes of sub-block s of pair n's token and adds them up.
 __global__ void __launch_bounds__(256) k_prefill_gather(DecodeParams P) {
+  pdl_enter();
   const int H = P.hidden, K = P.top_k, nb = H / kBlock;
   const int64_t work = static_cast<int64_t>(*P.n_items) * nb;
   const int n = threadIdx.x >> 3, s = threadIdx.x & 7;
@@ -241,6 +242,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Pr
 
 template <bool kGU>
 __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
+  pdl_enter();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -499,6 +501,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
 
 // y[t] = sum_j wts[t][j] * ye[t][j], slots in order.
 __global__ void k_combine(DecodeParams P) {
+  pdl_enter();
   const int H = P.hidden, K = P.top_k;
   const int64_t total = static_cast<int64_t>(P.ntok) * H;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -536,13 +539,13 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = prefill_smem();
-  k_prefill_gather<<<4 * n_sm, 256, 0, stream>>>(P);
+  launch_k(k_prefill_gather, dim3(4 * n_sm), dim3(256), 0, stream, P);
   note_launch(MOE_K_PREFILL_GATHER, stream);
-  k_prefill_mma<true><<<n_sm, kPThreads, smem, stream>>>(P);
+  launch_k(k_prefill_mma<true>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
   note_launch(MOE_K_PREFILL_GATEUP, stream);
-  k_prefill_mma<false><<<n_sm, kPThreads, smem, stream>>>(P);
+  launch_k(k_prefill_mma<false>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
   note_launch(MOE_K_PREFILL_DOWN, stream);
-  k_combine<<<4 * n_sm, 256, 0, stream>>>(P);
+  launch_k(k_combine, dim3(4 * n_sm), dim3(256), 0, stream, P);
   note_launch(MOE_K_COMBINE, stream);
   return check_launch("expert_ffn_prefill");
 }

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
 // ---------------------------------------------------------------------------
 __global__ void k_quant_act_q8(const float* __restrict__ x, int64_t nblk, int8_t* __restrict__ xq,
                                float* __restrict__ xd) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t blk = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -113,7 +114,7 @@ int launch_quant_act_q8(const float* x, int64_t ntok, int k, int8_t* xq, float* 
   const int warps_per_cta = 8;
   int64_t grid = (nblk + warps_per_cta - 1) / warps_per_cta;
   if (grid > 148 * 8) grid = 148 * 8;
-  k_quant_act_q8<<<static_cast<unsigned>(grid), warps_per_cta * 32, 0, stream>>>(x, nblk, xq, xd);
+  launch_k(k_quant_act_q8, dim3(static_cast<unsigned>(grid)), dim3(warps_per_cta * 32), 0, stream, x, nblk, xq, xd);
   note_launch(MOE_K_QUANT_ACT, stream);
   return check_launch("quant_act_q8");
 }

@@ -17,6 +17,7 @@ namespace bitmoe {
 // token by one warp each (coalesced 128-byte loads); many warps run per SM.
 __global__ void k_router_logits(const float* __restrict__ x, const float* __restrict__ wr, int ntok,
                                 int H, int E, float* __restrict__ logits) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int64_t total = static_cast<int64_t>(ntok) * E;
@@ -34,26 +35,33 @@ __global__ void k_router_logits(const float* __restrict__ x, const float* __rest
   }
 }
 
-// Many tokens: a CTA computes a 16-token x 16-expert tile of logits.  The
+// Many tokens: a CTA computes a tile of 16 tokens x 16 experts (4 experts
+// when there are few tokens, so that more CTAs share the work).  The
 // evaluation order is the same as above: the chain of lane l (k = l, l+32, ...
 // ascending) is kept by lane l of a warp for each (token, expert) pair of the
-// warp's 8 x 4 micro-tile, and the 32 chains are combined by the same xor
+// warp's micro-tile, and the 32 chains are combined by the same xor
 // butterfly.  x and router rows are staged through shared memory in 256-wide
 // chunks (double-buffered cp.async), so each row is read from L2 once per tile
 // instead of once per logit.
-constexpr int kRtT = 16, kRtE = 16, kRtKC = 256;
-constexpr int kRtMT = 8, kRtME = 4;  // micro-tile per lane: tokens x experts
+constexpr int kRtT = 16, kRtKC = 256;
 
+// kWE warps along the experts (8 / kWE along the tokens); a lane holds a
+// micro-tile of kMT tokens x kME experts: the CTA tile is 16 tokens x
+// kWE*kME experts.
+template <int kWE, int kMT, int kME>
 __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __restrict__ x,
                                                              const float* __restrict__ wr, int ntok, int H,
                                                              int E, float* __restrict__ logits) {
+  pdl_enter();
+  constexpr int kRtMT = kMT, kRtME = kME, kRtE = kWE * kME;
+  static_assert((8 / kWE) * kMT == kRtT, "16 tokens per tile");
   extern __shared__ __align__(16) float rsm[];
   float* xs = rsm;                        // [2][kRtT][kRtKC]
   float* ws = rsm + 2 * kRtT * kRtKC;     // [2][kRtE][kRtKC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
-  const int wt = (warp >> 2) * kRtMT;     // warp's first token in the tile (2 x 4 warp grid)
-  const int we = (warp & 3) * kRtME;      // warp's first expert in the tile
+  const int wt = (warp / kWE) * kRtMT;    // warp's first token in the tile
+  const int we = (warp % kWE) * kRtME;    // warp's first expert in the tile
   const int nchunk = H / kRtKC;
   auto stage = [&](int ch, int buf) {
     // (kRtT + kRtE) rows x 256 floats = 2048 chunks of 16 bytes, 8 per thread
@@ -120,12 +128,16 @@ __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __rest
 // w_i = exp(l_i - l_0) / sum_j exp(l_j - l_0) in fp32, summed in rank order.
 __global__ void k_topk_softmax(const float* __restrict__ logits, int ntok, int E, int K,
                                int32_t* __restrict__ idx, float* __restrict__ wts) {
+  pdl_enter();
   __shared__ float sel_v[4][kMaxTopK];
   __shared__ int sel_e[4][kMaxTopK];
+  __shared__ float lgs[4][kMaxExperts];  // the token's logits, read from L2 once
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
   const int t = blockIdx.x * 4 + wl;
   if (t >= ntok) return;
-  const float* lg = logits + static_cast<int64_t>(t) * E;
+  for (int e = lane; e < E; e += 32) lgs[wl][e] = logits[static_cast<int64_t>(t) * E + e];
+  __syncwarp();
+  const float* lg = lgs[wl];
   uint32_t used = 0;  // bit i: element lane + 32*i already chosen
   for (int r = 0; r < K; ++r) {
     float bv = -INFINITY;
@@ -161,27 +173,43 @@ __global__ void k_topk_softmax(const float* __restrict__ logits, int ntok, int E
   }
 }
 
-int launch_route_topk(const float* x, const float* wr, int ntok, int H, int E, int K, int32_t* idx,
-                      float* wts, float* logits, cudaStream_t stream) {
-  if (ntok >= kRtT && H % kRtKC == 0) {
-    const size_t smem = sizeof(float) * 2 * (kRtT + kRtE) * kRtKC;
-    static bool attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-      cudaFuncSetAttribute(k_router_logits_tiled, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      attr_done[dev] = true;
-    }
-    const dim3 grid((ntok + kRtT - 1) / kRtT, (E + kRtE - 1) / kRtE);
-    k_router_logits_tiled<<<grid, 256, smem, stream>>>(x, wr, ntok, H, E, logits);
-  } else {
+template <int kWE, int kMT, int kME>
+static void launch_tiled(const float* x, const float* wr, int ntok, int H, int E, float* logits,
+                         cudaStream_t stream) {
+  auto kern = k_router_logits_tiled<kWE, kMT, kME>;
+  const size_t smem = sizeof(float) * 2 * (kRtT + kWE * kME) * kRtKC;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    attr_done[dev] = true;
+  }
+  const dim3 grid((ntok + kRtT - 1) / kRtT, (E + kWE * kME - 1) / (kWE * kME));
+  launch_k(kern, grid, dim3(256), smem, stream, x, wr, ntok, H, E, logits);
+}
+
+int launch_router_logits(const float* x, const float* wr, int ntok, int H, int E, float* logits,
+                         cudaStream_t stream) {
+  if (H % kRtKC != 0) {
     const int64_t total = static_cast<int64_t>(ntok) * E;
     int64_t grid = (total + 7) / 8;
     if (grid > 148 * 16) grid = 148 * 16;
-    k_router_logits<<<static_cast<unsigned>(grid), 256, 0, stream>>>(x, wr, ntok, H, E, logits);
+    launch_k(k_router_logits, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, wr, ntok, H, E, logits);
+  } else if (ntok >= 4 * kRtT) {
+    launch_tiled<4, 8, 4>(x, wr, ntok, H, E, logits, stream);  // 16 x 16 tiles
+  } else {
+    launch_tiled<2, 4, 2>(x, wr, ntok, H, E, logits, stream);  // 16 x 4 tiles
   }
   note_launch(MOE_K_ROUTER_LOGITS, stream);
-  k_topk_softmax<<<(ntok + 3) / 4, 128, 0, stream>>>(logits, ntok, E, K, idx, wts);
+  return check_launch("router_logits");
+}
+
+int launch_route_topk(const float* x, const float* wr, int ntok, int H, int E, int K, int32_t* idx,
+                      float* wts, float* logits, cudaStream_t stream) {
+  int rc = launch_router_logits(x, wr, ntok, H, E, logits, stream);
+  if (rc) return rc;
+  launch_k(k_topk_softmax, dim3((ntok + 3) / 4), dim3(128), 0, stream, logits, ntok, E, K, idx, wts);
   note_launch(MOE_K_TOPK, stream);
   return check_launch("route_topk");
 }
