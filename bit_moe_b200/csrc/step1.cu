@@ -127,10 +127,6 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     // the logits of this launch carry the tag g + 1
     const uint32_t g = static_cast<uint32_t>(atomicAdd(S1.ticket, 1ull) / static_cast<unsigned long long>(C));
     *sgen = g + 1u;
-    // slot counters: launch g counts on set g & 1 and clears the other set
-    // for launch g + 1 (which starts after this launch has ended)
-    if (c == 0)
-      for (int j = 0; j < kS1MaxK; ++j) S1.slot_cnt[((g + 1u) & 1u) * kS1MaxK + j] = 0u;
   }
 
   // ---------------- phase A: x, int8 x^, logits of this CTA's experts
@@ -144,6 +140,9 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   cp_commit();
   cp_wait<0>();
   __syncthreads();
+  // the next step's kernel may start launching (its CTAs start as this
+  // launch's CTAs leave their SMs); every CTA of this launch holds its ticket
+  pdl_launch_dependents();
   const int nrows = e1 - e0;
   const uint32_t tag = *sgen;
   if (warp < nrows) {
@@ -264,23 +263,13 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   }
   __syncthreads();
   if (*abort) return;
-  // down prefetch: this CTA's panel of hidden for every slot (one issuing
-  // thread per slot: the panel's blocks are contiguous, one copy for the
-  // digits and one for the scales)
+  // down prefetch (issued after the first gate/up copies): this CTA's panel
+  // of hidden for every slot, one issuing thread per slot (the panel's blocks
+  // are contiguous: one copy for the digits and one for the scales)
   const int panelH = c;  // C >= hidden/32: at most one panel per CTA
   const bool has_panel = panelH < H / kPanel;
   unsigned char* pref = smem + L.pref;
   const size_t pref_slot = static_cast<size_t>(nbF) * kMatBytes;
-  if (has_panel && tid < K) {
-    const int j = tid;
-    const size_t pb0 = (static_cast<size_t>(sel_e[j]) * (H / kPanel) + panelH) * nbF;
-    unsigned char* dst = pref + j * pref_slot;
-    const uint32_t tb = static_cast<uint32_t>(nbF) * kBlockWords * kPanel * 4;
-    const uint32_t sb = static_cast<uint32_t>(nbF) * kPanel * 2;
-    mbar_arrive_expect_tx(pbar, tb + sb);
-    bulk_g2s(dst, P.down_trits + pb0 * kBlockWords * kPanel, tb, pbar, policy_evict_first());
-    bulk_g2s(dst + tb, P.down_scales + pb0 * kPanel, sb, pbar, policy_evict_first());
-  }
   // gate/up: units (slot, 32-row panel of ffn); blocks of hidden split by warp
   {
     using SL = Slot<2, 1, true>;
@@ -317,6 +306,23 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     };
 #pragma unroll 1
     for (int k = 0; k < SW; ++k) issue_next(k);
+    // the previous step's kernel has completed before this one writes the
+    // codes, scales and counters that kernel may still read; launch g counts
+    // on slot counter set g & 1 and clears set (g + 1) & 1 for launch g + 1
+    pdl_wait();
+    if (c == 0 && tid == 0)
+      for (int j = 0; j < kS1MaxK; ++j) S1.slot_cnt[(*sgen & 1u) * kS1MaxK + j] = 0u;
+    // then the down panels, which are needed only after the gate/up phase
+    if (has_panel && tid < K) {
+      const int j = tid;
+      const size_t pb0 = (static_cast<size_t>(sel_e[j]) * (H / kPanel) + panelH) * nbF;
+      unsigned char* dst = pref + j * pref_slot;
+      const uint32_t tb = static_cast<uint32_t>(nbF) * kBlockWords * kPanel * 4;
+      const uint32_t sb = static_cast<uint32_t>(nbF) * kPanel * 2;
+      mbar_arrive_expect_tx(pbar, tb + sb);
+      bulk_g2s(dst, P.down_trits + pb0 * kBlockWords * kPanel, tb, pbar, policy_evict_first());
+      bulk_g2s(dst + tb, P.down_scales + pb0 * kPanel, sb, pbar, policy_evict_first());
+    }
     int s = 0;
     for (int ui = 0; ui < nmine; ++ui) {
       const int64_t u = unit_of(ui);
@@ -446,12 +452,27 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* s
   cfg.blockDim = dim3(kNC * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  // cooperative (every CTA resident), and a programmatic dependent launch so
+  // that consecutive steps overlap (phase A of one step with the tail of the
+  // previous); without the latter where the runtime refuses the combination
+  static int pdl_ok[64] = {};  // 0 unknown, 1 yes, -1 no
+  const int di = dev >= 0 && dev < 64 ? dev : 0;
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_ok[di] >= 0 ? 2 : 1;
   cudaError_t err = cudaLaunchKernelEx(&cfg, k_step1, S);
+  if (err != cudaSuccess && cfg.numAttrs == 2 && pdl_ok[di] == 0) {
+    cudaGetLastError();
+    pdl_ok[di] = -1;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, k_step1, S);
+  } else if (err == cudaSuccess && cfg.numAttrs == 2) {
+    pdl_ok[di] = 1;
+  }
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "step1: %s", cudaGetErrorString(err));
   note_launch(MOE_K_STEP1, stream);
   return check_launch("step1");
