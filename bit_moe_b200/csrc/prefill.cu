@@ -499,17 +499,27 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   if (warp == 0) tmem_dealloc(tbase, kTmemCols);
 }
 
-// y[t] = sum_j wts[t][j] * ye[t][j], slots in order.
+// y[t] = sum_j wts[t][j] * ye[t][j], slots in order; four h per thread
+// (16-byte loads and stores; hidden is a multiple of 256).
 __global__ void k_combine(DecodeParams P) {
   pdl_enter();
-  const int H = P.hidden, K = P.top_k;
-  const int64_t total = static_cast<int64_t>(P.ntok) * H;
+  const int H = P.hidden, K = P.top_k, H4 = H / 4;
+  const int64_t total = static_cast<int64_t>(P.ntok) * H4;
+  const float4* ye = reinterpret_cast<const float4*>(P.ye);
+  float4* y = reinterpret_cast<float4*>(P.y);
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / H, h = i % H;
-    float y = 0.f;
-    for (int j = 0; j < K; ++j) y = __fmaf_rn(P.wts[t * K + j], P.ye[(t * K + j) * H + h], y);
-    P.y[i] = y;
+    const int64_t t = i / H4, h4 = i % H4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < K; ++j) {
+      const float w = P.wts[t * K + j];
+      const float4 v = __ldcs(ye + (t * K + j) * H4 + h4);
+      acc.x = __fmaf_rn(w, v.x, acc.x);
+      acc.y = __fmaf_rn(w, v.y, acc.y);
+      acc.z = __fmaf_rn(w, v.z, acc.z);
+      acc.w = __fmaf_rn(w, v.w, acc.w);
+    }
+    y[i] = acc;
   }
 }
 
