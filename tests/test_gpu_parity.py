@@ -260,6 +260,86 @@ def test_prefill_equals_decode():
     assert rel_err_rms(yp, yd) <= 1e-4
 
 
+@pytest.mark.parametrize("ntok", [1, 3, 65, 97])
+def test_prefill_tiny_ragged_all_tokens(orc, ntok):
+    """The tensor-core GEMM on the tiny layer: groups of 1..32 pairs with
+    ragged tails, every output compared with the oracle."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"]
+    layer, fn = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 21, ntok=ntok, device="cuda")
+    xq, xd = B.moe_quant_act_q8(x)
+    idx, wts = B.moe_route_topk(x, wr, wl.top_k)
+    ws = B.Workspace.for_layer(layer, ntok, prefill=True)
+    y = B.moe_expert_ffn_prefill(layer, xq, xd, idx, wts, ws).cpu().numpy()
+    assert B.moe_check_status(ws) == 0
+    olayer, remap = oracle_layer(orc, wl, fn)
+    ref = orc.expert_ffn(olayer, xq.cpu().numpy(), xd.cpu().numpy(), idx.cpu().numpy(),
+                         wts.cpu().numpy())
+    assert rel_err_rms(y, ref) <= LAYER_TOL
+
+
+def test_prefill_bad_expert_ids():
+    """Ids out of range in the prefill GEMM: status set, their slots add
+    nothing, the other slots equal the decode path's."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"]
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    ntok = 70
+    x = synthetic.activations(wl, 22, ntok=ntok, device="cuda")
+    xq, xd = B.moe_quant_act_q8(x)
+    idx, wts = B.moe_route_topk(x, wr, wl.top_k)
+    bad = idx.clone()
+    bad[::7, 1] = 1000
+    ws = B.Workspace.for_layer(layer, ntok, prefill=True)
+    yp = B.moe_expert_ffn_prefill(layer, xq, xd, bad, wts, ws).cpu().numpy()
+    assert B.moe_check_status(ws) == -7
+    ok_idx = bad.clone()
+    ok_w = wts.clone()
+    ok_idx[::7, 1] = 0
+    ok_w[::7, 1] = 0.0
+    yr = B.moe_expert_ffn_prefill(layer, xq, xd, ok_idx, ok_w, ws).cpu().numpy()
+    assert B.moe_check_status(ws) == 0
+    assert rel_err_rms(yp, yr) <= 1e-6
+
+
+def test_forward_decode_prefill_boundary(orc):
+    """64 tokens take the grouped decode kernels, 65 the prefill GEMM; both
+    match the oracle on sampled tokens."""
+    B = bm()
+    wl = synthetic.WORKLOADS["30b"]
+    layer, fn = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    for ntok in (64, 65):
+        x = synthetic.activations(wl, 23, ntok=ntok, device="cuda")
+        y, _ = _run_forward(B, layer, wr, x)
+        rows = np.array([0, ntok // 2, ntok - 1])
+        ref, _ = _oracle_tokens(orc, wl, fn, wr.cpu().numpy(), x.cpu().numpy(), rows)
+        assert rel_err_rms(y[rows], ref) <= LAYER_TOL
+
+
+def test_workspace_reused_across_shapes():
+    """One workspace serves the one-token step of two layer shapes in turn
+    (its tickets, tagged logits and slot counters carry over), with the same
+    results as fresh workspaces."""
+    B = bm()
+    out = {}
+    for name in ("tiny", "30b"):
+        wl = synthetic.WORKLOADS[name]
+        layer, _ = gpu_layer(wl)
+        out[name] = (layer, synthetic.router(wl, 0, "cuda"), synthetic.activations(wl, 24, ntok=1, device="cuda"))
+    big = B.Workspace.for_layer(out["30b"][0], 1)
+    fresh = {n: B.moe_forward(l, r, x, B.Workspace.for_layer(l, 1)).cpu().numpy() for n, (l, r, x) in out.items()}
+    for rep in range(3):
+        for n in ("tiny", "30b", "tiny"):
+            l, r, x = out[n]
+            y = B.moe_forward(l, r, x, big).cpu().numpy()
+            assert B.moe_check_status(big) == 0
+            assert np.array_equal(y, fresh[n])
+
+
 def test_forward_host_equals_device():
     B = bm()
     wl = synthetic.WORKLOADS["30b"]
