@@ -212,6 +212,37 @@ static int launch_decode(const DecodeParams& P, void* ws, const WsLayout& W, cud
   return launch_decode2(D, false, stream);
 }
 
+// ---------------------------------------------------------------- small host copies
+constexpr size_t kSmallHostCopy = 64 * 1024;
+
+// The device address of page-locked host memory, or null if the GPU cannot
+// address it (pageable memory).
+static void* host_device_view(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+  return a.devicePointer;
+}
+
+// dst[i] = src[i] for `bytes` (a multiple of 16, both 16-byte aligned).
+__global__ void __launch_bounds__(512) k_copy16(int4* __restrict__ dst, const int4* __restrict__ src, size_t n16) {
+  pdl_enter();
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
+}
+
+static int launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+  const size_t n16 = bytes / 16;
+  const unsigned grid = static_cast<unsigned>((n16 + 511) / 512 < 8 ? (n16 + 511) / 512 : 8);
+  launch_k(k_copy16, dim3(grid), dim3(512), 0, s, static_cast<int4*>(dst), static_cast<const int4*>(src), n16);
+  note_launch(MOE_K_COPY, s);
+  return check_launch("forward_host: copy");
+}
+
 }  // namespace bitmoe
 
 using namespace bitmoe;
@@ -381,9 +412,22 @@ int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, co
   float* xs = reinterpret_cast<float*>(base + W.xs);
   float* ys = reinterpret_cast<float*>(base + W.ys);
   const size_t bytes = sizeof(float) * static_cast<size_t>(ntok) * L->hidden;
-  cudaError_t err = cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, s);
-  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy in: %s", cudaGetErrorString(err));
+  // A few kilobytes from page-locked memory the GPU can address: one CTA
+  // copies them with loads over the bus (about a microsecond, and chained to
+  // the step by programmatic dependent launch) instead of a DMA copy, whose
+  // setup costs several microseconds.  Larger or pageable buffers: DMA copies.
+  const void* xd = host_device_view(x_host);
+  void* yd = host_device_view(y_host);
+  const bool small = bytes <= kSmallHostCopy && xd && yd && aligned16(xd) && aligned16(yd);
+  cudaError_t err = cudaSuccess;
+  if (small) {
+    if ((rc = launch_copy16(xs, xd, bytes, s))) return rc;
+  } else {
+    err = cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, s);
+    if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy in: %s", cudaGetErrorString(err));
+  }
   if ((rc = moe_forward(L, w_router, ntok, xs, ys, ws, ws_bytes, stream))) return rc;
+  if (small) return launch_copy16(yd, ys, bytes, s);
   err = cudaMemcpyAsync(y_host, ys, bytes, cudaMemcpyDeviceToHost, s);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy out: %s", cudaGetErrorString(err));
   return MOE_OK;
@@ -427,7 +471,7 @@ int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
 const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
-      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather"};
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather", "copy"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

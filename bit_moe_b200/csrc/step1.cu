@@ -129,6 +129,10 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     *sgen = g + 1u;
   }
 
+  // launched as a programmatic dependent: everything the kernels before it
+  // wrote (x among them) is visible only past this wait
+  pdl_wait();
+
   // ---------------- phase A: x, int8 x^, logits of this CTA's experts
   const int e0 = static_cast<int>(static_cast<int64_t>(E) * c / C);
   const int e1 = static_cast<int>(static_cast<int64_t>(E) * (c + 1) / C);
@@ -140,8 +144,9 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   cp_commit();
   cp_wait<0>();
   __syncthreads();
-  // the next step's kernel may start launching (its CTAs start as this
-  // launch's CTAs leave their SMs); every CTA of this launch holds its ticket
+  // the next kernel may start launching (its CTAs become resident as this
+  // launch's CTAs leave their SMs, then wait in pdl_wait for this launch to
+  // complete); every CTA of this launch holds its ticket by now
   pdl_launch_dependents();
   const int nrows = e1 - e0;
   const uint32_t tag = *sgen;
@@ -306,10 +311,8 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     };
 #pragma unroll 1
     for (int k = 0; k < SW; ++k) issue_next(k);
-    // the previous step's kernel has completed before this one writes the
-    // codes, scales and counters that kernel may still read; launch g counts
-    // on slot counter set g & 1 and clears set (g + 1) & 1 for launch g + 1
-    pdl_wait();
+    // launch g counts on slot counter set g & 1 and clears set (g + 1) & 1
+    // for launch g + 1 (the previous launch has completed: see pdl_wait)
     if (c == 0 && tid == 0)
       for (int j = 0; j < kS1MaxK; ++j) S1.slot_cnt[(*sgen & 1u) * kS1MaxK + j] = 0u;
     // then the down panels, which are needed only after the gate/up phase

@@ -179,8 +179,10 @@ int moe_expert_ffn_prefill(const moe_layer* layer, int32_t ntok, const int8_t* x
 int moe_forward(const moe_layer* layer, const float* w_router, int32_t ntok, const float* x,
                 float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
 /* The same with x and y in HOST memory (pinned for asynchronous copies):
- * copies x in, runs moe_forward, copies y out, all on `stream`.  The host
- * buffers must stay valid until the stream reaches the end of the call.   */
+ * copies x in, runs moe_forward, copies y out, all on `stream`.  Up to 64 KB
+ * of page-locked x and y are moved by a small kernel that addresses them
+ * over the bus; larger or pageable buffers by DMA copies.  The host buffers
+ * must stay valid until the stream reaches the end of the call.           */
 int moe_forward_host(const moe_layer* layer, const float* w_router, int32_t ntok,
                      const float* x_host, float* y_host, void* ws, size_t ws_bytes,
                      moe_stream_t stream);
@@ -198,7 +200,7 @@ typedef enum {
   MOE_K_QUANTIZE_WEIGHTS = 0, MOE_K_QUANT_ACT = 1, MOE_K_ROUTER_LOGITS = 2, MOE_K_TOPK = 3,
   MOE_K_GROUP = 4, MOE_K_GATEUP = 5, MOE_K_DOWN = 6, MOE_K_DEBUG_MATVEC = 7,
   MOE_K_PREFILL_GATEUP = 8, MOE_K_PREFILL_DOWN = 9, MOE_K_ROUTE = 10, MOE_K_COMBINE = 11,
-  MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COUNT = 14
+  MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COPY = 14, MOE_K_COUNT = 15
 } moe_kernel_id;
 /* Number of kernels this thread has launched through the library so far. */
 int64_t moe_launch_count(void);

@@ -320,6 +320,35 @@ def test_forward_decode_prefill_boundary(orc):
         assert rel_err_rms(y[rows], ref) <= LAYER_TOL
 
 
+@pytest.mark.parametrize("ntok", [1, 2, 70])
+def test_chained_layers_no_sync(ntok):
+    """Layer outputs fed straight into the next call on the same stream (the
+    kernels overlap their launches): the same results as with a
+    synchronization between the calls, through device and host buffers."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"]
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 25, ntok=ntok, device="cuda")
+    ws = B.Workspace.for_layer(layer, ntok)
+    ref = [x]
+    for _ in range(4):
+        ref.append(B.moe_forward(layer, wr, ref[-1], ws).clone())
+        torch.cuda.synchronize()
+    ys = [x]
+    for _ in range(4):
+        ys.append(B.moe_forward(layer, wr, ys[-1], ws))
+    torch.cuda.synchronize()
+    for a, b in zip(ys[1:], ref[1:]):
+        assert torch.equal(a, b)
+    hx = [x.cpu().pin_memory()] + [torch.empty_like(x, device="cpu").pin_memory() for _ in range(4)]
+    for i in range(4):
+        B.moe_forward_host(layer, wr, hx[i], hx[i + 1], ws)
+        torch.cuda.synchronize()  # the host buffer of one call is the input of the next
+        assert torch.equal(hx[i + 1], ref[i + 1].cpu())
+    assert B.moe_check_status(ws) == 0
+
+
 def test_workspace_reused_across_shapes():
     """One workspace serves the one-token step of two layer shapes in turn
     (its tickets, tagged logits and slot counters carry over), with the same
