@@ -96,8 +96,8 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
   L.ys = take(sizeof(float) * T * static_cast<size_t>(H));
   off = group_ws_layout(E, T * K, off, &L.grp);
   if (prefill) {
-    // groups of at most 32 pairs: at most T*K/32 full ones plus one partial per expert
-    const size_t groups = static_cast<size_t>(T) * K / 32 + E + 1;
+    // groups of at most G pairs: at most T*K/G full ones plus one partial per expert
+    const size_t groups = static_cast<size_t>(T) * K / prefill_group_pairs() + E + 1;
     L.bgu = take(groups * (H / kBlock) * prefill_block_bytes());
     L.bdn = take(groups * (F / kBlock) * prefill_block_bytes());
   }

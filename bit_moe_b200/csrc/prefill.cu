@@ -22,7 +22,7 @@
 //     sub-blocks of d * sum(q*a), then the fp16 weight scale per 256-block.
 // The activations of a tile are laid out once per (group, 256-block) in HBM
 // exactly as shared memory holds them (split codes in the MMA's core-matrix
-// layout, then the scales and code sums of the 32 pairs): for gate/up by a
+// layout, then the scales and code sums of the group's pairs): for gate/up by a
 // gather pass over x^, for down by the gate/up epilogue itself.  One bulk copy
 // (TMA) then brings each block's 18 KB into a shared-memory stage.
 // The kernel is persistent (one CTA per SM) and warp-specialized: decode
@@ -43,7 +43,7 @@
 
 namespace bitmoe {
 
-constexpr int kPN = 32;           // pairs per tile (MMA N)
+constexpr int kPN = 64;           // pairs per tile (MMA N)
 constexpr int kPM = 128;          // weight rows per tile (MMA M)
 // Warp roles of a CTA (one CTA per SM, persistent over the tiles):
 constexpr int kWDec = 0;          // warps 0-3: decode the digits into TMEM (thread = row)
@@ -55,7 +55,7 @@ constexpr int kWMma = 21;         // warp 21: lane 0 issues the MMAs
 constexpr int kPThreads = 22 * 32;
 constexpr int kAStages = 2;       // digit stages in TMEM, 64 columns each
 constexpr int kBStages = 3;       // code / scale stages in shared memory
-constexpr int kQSub = 4;          // sub-blocks per accumulator stage (half a block)
+constexpr int kQSub = 2;          // sub-blocks per accumulator stage (a quarter of a block)
 constexpr int kDStages = 3;       // accumulator stages in flight
 constexpr int kTmemCols = 512;
 constexpr int kAcol = 0;          // A stage a: columns [64a, 64a + 64)
@@ -64,7 +64,7 @@ constexpr int kDcol = 128;        // D stage d: columns [128 + kQSub*kDSub*d, 12
 static_assert(kDcol + kDStages * kQSub * kDSub <= 512, "tensor memory columns");
 
 // One 256-wide block of a tile's activations, identical in HBM and in shared
-// memory: the split codes in the MMA layout, then per sub-block the 32 pairs'
+// memory: the split codes in the MMA layout, then per sub-block the pairs'
 // scales and code sums (negated).
 struct BStage {
   unsigned char codes[2][kSubPerBlock * kPN * 32];  // 16*h parts, then l parts, MMA layout
@@ -102,7 +102,7 @@ __device__ __forceinline__ void code_split(int q, uint8_t& hi, uint8_t& lo) {
 
 // The gate/up activation blocks of every group: thread (n, s) of a CTA
 // splits the 32 codes of sub-block s of pair n's token and adds them up.
-__global__ void __launch_bounds__(256) k_prefill_gather(DecodeParams P) {
+__global__ void __launch_bounds__(kPN * kSubPerBlock) k_prefill_gather(DecodeParams P) {
   pdl_enter();
   const int H = P.hidden, K = P.top_k, nb = H / kBlock;
   const int64_t work = static_cast<int64_t>(*P.n_items) * nb;
@@ -333,14 +333,17 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
     uint32_t i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
       const TileInfo T = tile_info(P, t, m_tiles);
-      const int my_pair = lane < T.it.count ? P.pairs[T.it.start + lane] : -1;
+      // pair n of the tile: lane n & 31 of mp[n >> 5]
+      const int mp0 = lane < T.it.count ? P.pairs[T.it.start + lane] : -1;
+      const int mp1 = lane + 32 < T.it.count ? P.pairs[T.it.start + lane + 32] : -1;
+      auto pair_at = [&](int n) { return __shfl_sync(0xffffffffu, n < 32 ? mp0 : mp1, n & 31); };
       if (T.it.expert < 0) {  // ids out of range: their outputs are zero
         if (warp == kWFix && lane == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
         if (kGU) {
           if (q >= 2) write_down_codes(P, T.mt, t / m_tiles, 32 * (q - 2) + lane, kFixPairs * f16, nullptr, 0, lane);
         } else {
           for (int n = kFixPairs * f16; n < kFixPairs * f16 + kFixPairs; ++n) {
-            const int pair = __shfl_sync(0xffffffffu, my_pair, n);
+            const int pair = pair_at(n);
             if (n < T.it.count) P.ye[static_cast<size_t>(pair) * H + kPM * T.mt + 32 * q + lane] = 0.f;
           }
         }
@@ -369,17 +372,18 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
           const int ds = j2 % kDStages;
           if (!wait_or_abort(&S.d_full[ds], (j2 / kDStages) & 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
-          // kQSub sub-blocks x this warp's pairs
-          uint32_t v[kQSub][kFixPairs];
-#pragma unroll
-          for (int s2 = 0; s2 < kQSub; ++s2)
-            tmem_ld8(tlane + kDcol + kQSub * kDSub * ds + kDSub * s2 + kFixPairs * f16, v[s2]);
-          tc_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&S.d_empty[ds]);
+          // kQSub sub-blocks x this warp's pairs, one sub-block at a time; the
+          // stage goes back to the MMA once the last one is in registers
 #pragma unroll
           for (int s2 = 0; s2 < kQSub; ++s2) {
+            uint32_t v[kFixPairs];
+            tmem_ld16(tlane + kDcol + kQSub * kDSub * ds + kDSub * s2 + kFixPairs * f16, v);
+            tc_wait_ld();
+            if (s2 == kQSub - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&S.d_empty[ds]);
+            }
             const int s = kQSub * h + s2;
             const float4* dp = reinterpret_cast<const float4*>(&S.st[bs].d[s][kFixPairs * f16]);
             const float4* ap = reinterpret_cast<const float4*>(&S.st[bs].nsa[s][kFixPairs * f16]);
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
             for (int n4 = 0; n4 < kFixPairs / 4; ++n4) {
               const float4 dd = dp[n4], aa = ap[n4];
               // 512 * D - sum(a) = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
-              const uint32_t* vv = &v[s2][4 * n4];
+              const uint32_t* vv = &v[4 * n4];
               float q0, q1, q2, q3;
               fma2(q0, q1, __uint_as_float(vv[0]), __uint_as_float(vv[1]), 512.f, 512.f, aa.x, aa.y);
               fma2(q2, q3, __uint_as_float(vv[2]), __uint_as_float(vv[3]), 512.f, 512.f, aa.z, aa.w);
@@ -426,7 +430,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
 #pragma unroll
         for (int n = 0; n < kFixPairs; ++n) {
           const int np = kFixPairs * f16 + n;
-          const int pair = __shfl_sync(0xffffffffu, my_pair, np);
+          const int pair = pair_at(np);
           if (np < T.it.count) P.ye[static_cast<size_t>(pair) * H + hrow] = y[n];
         }
       }
@@ -531,6 +535,7 @@ static size_t prefill_smem() {
 }
 
 size_t prefill_block_bytes() { return kBTile; }
+int prefill_group_pairs() { return kPN; }
 
 int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   DecodeParams P = P0;
@@ -549,7 +554,7 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = prefill_smem();
-  launch_k(k_prefill_gather, dim3(4 * n_sm), dim3(256), 0, stream, P);
+  launch_k(k_prefill_gather, dim3(4 * n_sm), dim3(kPN * kSubPerBlock), 0, stream, P);
   note_launch(MOE_K_PREFILL_GATHER, stream);
   launch_k(k_prefill_mma<true>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
   note_launch(MOE_K_PREFILL_GATEUP, stream);

@@ -5,4 +5,6 @@ namespace bitmoe {
 int launch_prefill(const DecodeParams& P, cudaStream_t stream);
 // Bytes of one activation block of a 32-pair group (split codes, scales, sums).
 size_t prefill_block_bytes();
+// Most (token, slot) pairs in one group of the prefill GEMM.
+int prefill_group_pairs();
 }  // namespace bitmoe
