@@ -35,7 +35,12 @@ namespace bitmoe {
 
 constexpr int kS1MaxH = 4096, kS1MaxF = 2048, kS1MaxK = 8;
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls before a wait gives up (seconds)
-constexpr int kS1MaxE = kNC * 32;          // experts: one per thread of the CTA
+// Two gate/up streams of kNC warps per CTA: each stream computes one unit at a
+// time with the block split and summation order of the grouped decode kernels,
+// and the two streams of an SM run different units side by side.
+constexpr int kS1Streams = 2;
+constexpr int kS1Warps = kS1Streams * kNC;
+constexpr int kS1MaxE = kNC * 32;          // experts: one per lane of the polling warp's kPer rounds
 // One 128-byte line per tagged logit, so that the CTAs polling the logits
 // spread their loads over many L2 lines instead of queueing on a few.
 constexpr int kTagStride = 16;
@@ -50,36 +55,56 @@ struct Step1Params {
 
 struct Step1Layout {
   size_t ring, pref, xq4, xd, xas, lg, sel, red, flag, xf, act, total;
+  int sw;  // ring slots per warp
 };
 
-// Shared-memory plan of one CTA (the down activations alias the
-// gate/up ring; the router rows alias the down prefetch area).
+// Shared-memory plan of one CTA.  x in fp32, the logits and the down
+// activations alias the gate/up ring (which is used only between them); the
+// router rows alias the down prefetch area.  Three ring slots per warp where
+// they fit, else two.
 __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) {
   Step1Layout L{};
-  size_t off = 0;
-  auto take = [&](size_t bytes) {
-    const size_t o = off;
-    off = (off + bytes + 127) / 128 * 128;
-    return o;
-  };
-  const size_t ring = static_cast<size_t>(kNC) * ring_depth<1>() * Slot<2, 1, true>::bytes;
-  const size_t xf = static_cast<size_t>(H) * 4;
-  const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
-  L.ring = take(ring > act ? ring : act);
-  L.act = L.ring;
-  L.xf = take(xf);
-  const size_t pref = static_cast<size_t>(K) * (F / kBlock) * kMatBytes;
-  const size_t rows = static_cast<size_t>(2) * H * 4;  // at most two router rows per CTA
-  L.pref = take(pref > rows ? pref : rows);
-  L.xq4 = take(static_cast<size_t>(H));
-  L.xd = take(static_cast<size_t>(H / kQBlock) * 4);
-  L.xas = take(static_cast<size_t>(H / kQBlock) * 4);
-  L.lg = take(static_cast<size_t>(E) * 4);
-  L.sel = take(2 * kMaxTopK * 4);
-  L.red = take(2 * 2 * kNC * 32 * 4);
-  L.flag = take(64);
-  L.total = off;
+  for (int sw = 3; sw >= 2; --sw) {
+    L = Step1Layout{};
+    L.sw = sw;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+      const size_t o = off;
+      off = (off + bytes + 127) / 128 * 128;
+      return o;
+    };
+    size_t ring = static_cast<size_t>(kS1Warps) * sw * Slot<2, 1, true>::bytes;
+    const size_t xf = static_cast<size_t>(H) * 4 + static_cast<size_t>(E) * 4;
+    const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
+    if (ring < xf) ring = xf;
+    if (ring < act) ring = act;
+    L.ring = take(ring);
+    L.act = L.ring;
+    L.xf = L.ring;
+    L.lg = L.ring + static_cast<size_t>(H) * 4;
+    const size_t pref = static_cast<size_t>(K) * (F / kBlock) * kMatBytes;
+    const size_t rows = static_cast<size_t>(2) * H * 4;  // at most two router rows per CTA
+    L.pref = take(pref > rows ? pref : rows);
+    L.xq4 = take(static_cast<size_t>(H));
+    L.xd = take(static_cast<size_t>(H / kQBlock) * 4);
+    L.xas = take(static_cast<size_t>(H / kQBlock) * 4);
+    L.sel = take(2 * kMaxTopK * 4);
+    L.red = take(static_cast<size_t>(kS1Streams) * 2 * kNC * 32 * 4);
+    L.flag = take(64);
+    L.total = off;
+    if (L.total <= static_cast<size_t>(kMaxDynSmem)) break;
+  }
   return L;
+}
+
+// Named barriers of gate/up stream h (kNC warps each): the unit's partial
+// sums are written (all warps sync), and read by the epilogue warp (it
+// arrives, the other warps sync before they overwrite them).
+__device__ __forceinline__ void stream_bar_sync(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kNC * 32) : "memory");
+}
+__device__ __forceinline__ void stream_bar_arrive(int id) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kNC * 32) : "memory");
 }
 
 // Bounded polls of values another CTA publishes.
@@ -98,7 +123,7 @@ __device__ __forceinline__ uint32_t f32_key(float v) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
+__global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const Decode2Params& D = S1.D;
   const DecodeParams& P = D.P;
@@ -232,7 +257,7 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     // x -> int8 32-blocks, kU blocks per warp at a time so that the
     // reductions and divisions of independent blocks overlap
     constexpr int kU = 8;
-    const int nblk = H / kQBlock, nqw = kNC - 1;
+    const int nblk = H / kQBlock, nqw = kS1Warps - 1;
     for (int b0 = warp - 1; b0 < nblk; b0 += nqw * kU) {
       float xv[kU], am[kU];
 #pragma unroll
@@ -275,30 +300,35 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
   const bool has_panel = panelH < H / kPanel;
   unsigned char* pref = smem + L.pref;
   const size_t pref_slot = static_cast<size_t>(nbF) * kMatBytes;
-  // gate/up: units (slot, 32-row panel of ffn); blocks of hidden split by warp
+  // gate/up: units (slot, 32-row panel of ffn); stream h of this CTA takes
+  // every other unit of the CTA's list, the blocks of hidden of a unit split
+  // over the stream's warps
   {
     using SL = Slot<2, 1, true>;
-    constexpr int SW = ring_depth<1>();
+    const int SW = L.sw;
     const int panels = F / kPanel;
     const int64_t U = static_cast<int64_t>(K) * panels;
-    // this CTA's units: unit c in the first round, then in each later round
-    // the unit counted from the round's end, so that the extra units fall on
-    // the highest CTA ids (those without a panel of hidden) and the slots of
-    // the first round are complete first
-    auto unit_of = [&](int r) -> int64_t {
-      return r == 0 ? static_cast<int64_t>(c) : static_cast<int64_t>(r) * C + (C - 1 - c);
+    const int h = warp / kNC, w8 = warp % kNC;
+    // this CTA's units: unit c first, then in each later round the unit
+    // counted from the round's end, so that the extra units fall on the
+    // highest CTA ids (those without a panel of hidden) and the slots of the
+    // first round are complete first; stream h takes rounds h, h+2, ...
+    auto unit_of = [&](int q) -> int64_t {
+      return q == 0 ? static_cast<int64_t>(c) : static_cast<int64_t>(q) * C + (C - 1 - c);
     };
     int nmine = 0;
-    while (unit_of(nmine) < U) ++nmine;
+    while (unit_of(kS1Streams * nmine + h) < U) ++nmine;
+    auto my_unit = [&](int i) { return unit_of(kS1Streams * i + h); };
     unsigned char* myring = smem + L.ring + static_cast<size_t>(warp) * SW * SL::bytes;
-    float* red = reinterpret_cast<float*>(smem + L.red);
+    float* rb = reinterpret_cast<float*>(smem + L.red) + h * (2 * kNC * 32);
+    const int bar_done = 1 + h, bar_free = 1 + kS1Streams + h;
     uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
     int im = 0;
-    int ib = warp;
+    int ib = w8;
     auto issue_next = [&](int slot) {
-      while (im < nmine && ib >= nbH) { ++im; ib = warp; }
+      while (im < nmine && ib >= nbH) { ++im; ib = w8; }
       if (im < nmine) {
-        const int64_t iu = unit_of(im);
+        const int64_t iu = my_unit(im);
         Group G;
         G.expert = sel_e[iu / panels];
         G.count = 1;
@@ -328,28 +358,30 @@ __global__ void __launch_bounds__(kNC * 32, 1) k_step1(Step1Params S1) {
     }
     int s = 0;
     for (int ui = 0; ui < nmine; ++ui) {
-      const int64_t u = unit_of(ui);
+      const int64_t u = my_unit(ui);
       const int j = static_cast<int>(u / panels), p = static_cast<int>(u % panels);
       float part[2][1] = {{0.f}, {0.f}};
-      for (int b = warp; b < nbH; b += kNC, ++s) {
-        cp_wait<SW - 1>();
+      for (int b = w8; b < nbH; b += kNC, ++s) {
+        if (SW == 3) cp_wait<2>(); else cp_wait<1>();
         __syncwarp();
         block_dot<2, 1, 1>(myring + (s % SW) * SL::bytes, sq4 + b * (kBlock / 4), 0, sxd + b * kSubPerBlock,
                            sxas + b * kSubPerBlock, 0, lane, part);
         __syncwarp();
         issue_next(s % SW);
       }
-      float* rb = red + (ui & 1) * (2 * kNC * 32);
-      rb[(0 * kNC + warp) * 32 + lane] = part[0][0];
-      rb[(1 * kNC + warp) * 32 + lane] = part[1][0];
-      __syncthreads();
-      if (warp == 0) {
+      // the epilogue warp has read the previous unit's sums
+      if (ui > 0 && w8 != 0) stream_bar_sync(bar_free);
+      rb[(0 * kNC + w8) * 32 + lane] = part[0][0];
+      rb[(1 * kNC + w8) * 32 + lane] = part[1][0];
+      stream_bar_sync(bar_done);
+      if (w8 == 0) {
         float g = 0.f, uu = 0.f;
         const int nw = nbH < kNC ? nbH : kNC;
         for (int v = 0; v < nw; ++v) {
           g = __fadd_rn(g, rb[(0 * kNC + v) * 32 + lane]);
           uu = __fadd_rn(uu, rb[(1 * kNC + v) * 32 + lane]);
         }
+        if (ui + 1 < nmine) stream_bar_arrive(bar_free);
         const float a = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), uu);
         const float amax = warp_max(fabsf(a));
         const float dd = __fdiv_rn(amax, 127.f);
@@ -452,7 +484,7 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* s
   Step1Params S{D, ticket, reinterpret_cast<unsigned long long*>(D.logits), slot_cnt};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(D.n_sm);
-  cfg.blockDim = dim3(kNC * 32);
+  cfg.blockDim = dim3(kS1Warps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   // cooperative (every CTA resident), and a programmatic dependent launch so
