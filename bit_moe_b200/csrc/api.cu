@@ -66,7 +66,8 @@ int check_device() {
 
 // ---------------------------------------------------------------- workspace
 struct WsLayout {
-  size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0, asum = 0;
+  size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0;
+  size_t units = 0;       // tagged gate/up unit outputs of the one-token step
   size_t xs = 0, ys = 0;  // device copies of x and y for the host-buffer entry point
   size_t bgu = 0, bdn = 0;  // prefill only
   GroupWs grp;
@@ -91,7 +92,7 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
   L.ad = take(sizeof(float) * T * static_cast<size_t>(K) * (F / kQBlock));
   L.ye = take(sizeof(float) * T * static_cast<size_t>(K) * H);
   L.cnt = take(sizeof(int32_t) * T * static_cast<size_t>(H / kPanel));
-  L.asum = take(sizeof(int32_t) * T * static_cast<size_t>(K) * (F / kQBlock));
+  L.units = take(sizeof(unsigned long long) * K * static_cast<size_t>(F / kPanel) * (kPanel / 4 + 2));
   L.xs = take(sizeof(float) * T * static_cast<size_t>(H));
   L.ys = take(sizeof(float) * T * static_cast<size_t>(H));
   off = group_ws_layout(E, T * K, off, &L.grp);
@@ -167,7 +168,6 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   const bool pf = W.bgu != 0;
   P.bgu = pf ? base + W.bgu : nullptr;
   P.bdn = pf ? base + W.bdn : nullptr;
-  P.asum = reinterpret_cast<int32_t*>(base + W.asum);
   return P;
 }
 
@@ -374,6 +374,14 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   float* wts = reinterpret_cast<float*>(base + W.wts);
   float* logits = reinterpret_cast<float*>(base + W.logits);
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
+  if (ntok > 1 && !prefill && router_quant_small_ok(ntok, L->hidden)) {
+    // few tokens: router logits with the activation quantization, then the
+    // top-k with the grouping, then the grouped mat-vecs
+    if ((rc = launch_router_quant_small(x, w_router, ntok, L->hidden, L->n_experts, logits, xq, xd, s)))
+      return rc;
+    if ((rc = launch_topk_group(P, logits, wts, s))) return rc;
+    return launch_ffn(P, s);
+  }
   if (ntok > 1) {
     if ((rc = launch_quant_act_q8(x, ntok, L->hidden, xq, xd, s))) return rc;
     if ((rc = launch_route_topk(x, w_router, ntok, L->hidden, L->n_experts, L->top_k, idx, wts, logits, s)))
@@ -390,7 +398,7 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   if (step1_supported(P, D.n_sm, &smem1)) {
     WsHeader* hd = reinterpret_cast<WsHeader*>(ws);
     return launch_step1(D, reinterpret_cast<unsigned long long*>(&hd->pad[3]),
-                        reinterpret_cast<uint32_t*>(&hd->pad[8]), s);
+                        reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(ws) + W.units), s);
   }
   return launch_decode2(D, true, s);
 }
@@ -471,7 +479,8 @@ int moe_trace_end(int32_t* kernel_ids, int32_t capacity) {
 const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
-      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather", "copy"};
+      "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather", "copy",
+      "router_quant", "topk_group"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

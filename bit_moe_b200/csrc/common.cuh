@@ -33,8 +33,7 @@ constexpr int kMaxDynSmem = 227 * 1024;  // opt-in dynamic shared memory per CTA
 // Workspace header: the first 256 bytes hold the device status word.
 struct WsHeader {
   int32_t status;    // first error code seen by a kernel (0 = ok)
-  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit one-token step tickets;
-                     // pad[8..23]: two sets of slot counters of the one-token step
+  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit one-token step tickets
 };
 static_assert(offsetof(WsHeader, pad) + 3 * sizeof(int32_t) == 16, "8-byte aligned ticket counter");
 constexpr size_t kWsHeaderBytes = sizeof(WsHeader);
@@ -105,6 +104,16 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
   return v;
+}
+
+// Order-preserving map of an fp32 value to uint32 (larger value, larger key;
+// -0 ranks as +0), and back (-0 comes back as +0).
+__device__ __forceinline__ uint32_t f32_key(float v) {
+  const uint32_t b = __float_as_uint(v == 0.f ? 0.f : v);  // -0 ranks as +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float f32_unkey(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 }  // namespace bitmoe

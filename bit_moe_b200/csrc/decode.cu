@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "ternary_dot.cuh"
+#include "topk.cuh"
 
 namespace bitmoe {
 
@@ -43,8 +44,7 @@ size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G) {
 // ---------------------------------------------------------------------------
 constexpr int kGroupThreads = 1024;
 
-__global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
-  pdl_enter();
+__device__ __forceinline__ void group_body(const DecodeParams& P) {
   using Scan = cub::BlockScan<int, kGroupThreads>;
   __shared__ typename Scan::TempStorage scan_tmp;
   __shared__ int cnt[kMaxExperts + 1];
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
   for (int e = tid; e <= E; e += kGroupThreads) { cnt[e] = 0; fill[e] = 0; }
   __syncthreads();
   for (int p = tid; p < npairs; p += kGroupThreads) {
-    int e = P.idx[p];
+    int e = __ldcg(P.idx + p);
     if (e < 0 || e >= E) { record_status(P.status, MOE_ERR_BAD_INDEX); e = E; }
     atomicAdd(&cnt[e], 1);
   }
@@ -90,10 +90,47 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
   __syncthreads();
   int32_t* pairs = const_cast<int32_t*>(P.pairs);
   for (int p = tid; p < npairs; p += kGroupThreads) {
-    int e = P.idx[p];
+    int e = __ldcg(P.idx + p);
     if (e < 0 || e >= E) e = E;
     pairs[off[e] + atomicAdd(&fill[e], 1)] = p;
   }
+}
+
+__global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
+  pdl_enter();
+  group_body(P);
+}
+
+// Up to kGroupThreads/32 tokens: warp t takes token t's top-k and softmax
+// (warp_topk_softmax, as k_topk_softmax), then the CTA groups the pairs.
+template <int kPer>
+__global__ void __launch_bounds__(kGroupThreads) k_topk_group(DecodeParams P, const float* __restrict__ logits,
+                                                              float* __restrict__ wts) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31, t = threadIdx.x >> 5;
+  const int E = P.n_experts, K = P.top_k;
+  if (t < P.ntok) {
+    uint32_t key[kPer];
+    uint32_t need = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = 0u;
+      if (e < E) {
+        key[i] = f32_key(logits[static_cast<int64_t>(t) * E + e]);
+        need |= 1u << i;
+      }
+    }
+    int my_e;
+    float w;
+    warp_topk_softmax<kPer>(key, need, K, lane, my_e, w);
+    if (lane < K) {
+      const_cast<int32_t*>(P.idx)[static_cast<int64_t>(t) * K + lane] = my_e;
+      wts[static_cast<int64_t>(t) * K + lane] = w;
+    }
+  }
+  __syncthreads();
+  group_body(P);
 }
 
 // Fetch work item `it`; returns false when there is none.
@@ -352,6 +389,16 @@ int launch_group(const DecodeParams& P, cudaStream_t stream) {
   launch_k(k_group, dim3(1), dim3(kGroupThreads), 0, stream, P);
   note_launch(MOE_K_GROUP, stream);
   return check_launch("group");
+}
+
+int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cudaStream_t stream) {
+  if (P.ntok > kGroupThreads / 32) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "topk_group: more than %d tokens", kGroupThreads / 32);
+  const int E = P.n_experts;
+  if (E <= 128) launch_k(k_topk_group<4>, dim3(1), dim3(kGroupThreads), 0, stream, P, logits, wts);
+  else if (E <= 256) launch_k(k_topk_group<8>, dim3(1), dim3(kGroupThreads), 0, stream, P, logits, wts);
+  else launch_k(k_topk_group<32>, dim3(1), dim3(kGroupThreads), 0, stream, P, logits, wts);
+  note_launch(MOE_K_TOPK_GROUP, stream);
+  return check_launch("topk_group");
 }
 
 int launch_ffn(const DecodeParams& P, cudaStream_t stream) {

@@ -40,7 +40,6 @@ struct DecodeParams {
   // the tensor-core kernel's shared-memory stages, for gate/up and for down
   unsigned char* bgu;                        // [groups][hidden/256] blocks
   unsigned char* bdn;                        // [groups][ffn/256] blocks
-  int32_t* asum;                             // [ntok*top_k][ffn/32] code sums of a^ (one-token step)
 };
 
 // Bytes of workspace the grouped mode needs after `off`; writes the offsets.
@@ -50,6 +49,9 @@ struct GroupWs {
 size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G);
 
 int launch_group(const DecodeParams& P, cudaStream_t stream);
+// Top-k softmax of P.ntok <= 32 tokens' logits ([ntok][E] fp32) into P.idx
+// and wts, then the grouping of launch_group, in one single-CTA kernel.
+int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cudaStream_t stream);
 int launch_ffn(const DecodeParams& P, cudaStream_t stream);
 int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const float* xd, float* out,
                         int32_t* isum, cudaStream_t stream);

@@ -35,8 +35,10 @@ int launch_decode2(Decode2Params& D, bool with_route, cudaStream_t stream);
 
 // The whole one-token step in one cooperative kernel (step1.cu).
 bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem);
-// `ticket`: a 64-bit counter that only grows; `slot_cnt`: top_k counters; the
-// logits area of D must hold 8 bytes per expert (tagged logits).
-int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* slot_cnt, cudaStream_t stream);
+// `ticket`: a 64-bit counter that only grows; `units`: top_k * (ffn / 32) * 10
+// 8-byte words for the tagged gate/up unit outputs; the logits area of D must
+// hold 128 bytes per expert (tagged logits).
+int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned long long* units,
+                 cudaStream_t stream);
 
 }  // namespace bitmoe

@@ -134,13 +134,16 @@ __device__ __forceinline__ void issue_item(unsigned char* dst, const DecodeParam
 // Decode of one block: NM matrices (words and scales at wsrc) against NT
 // activation vectors (codes q4[n*qs + g], scales ds[n*dsn + s], block sums
 // as[n*dsn + s], or computed here from the codes when as is null).
-// part[m][n] += s_w[m] * sum_s d[n][s] * isum[m][n][s].
+// part[m][n] += s_w[m] * sum_s d[n][s] * isum[m][n][s]; with kInner, part
+// receives the block's inner sum sum_s d[n][s] * isum[m][n][s] itself and
+// sc_out[m] the weight scale s_w[m], so that a caller can apply the scales of
+// blocks computed by different warps in the same order.
 // ---------------------------------------------------------------------------
-template <int NM, int NT, int NTMAX>
+template <int NM, int NT, int NTMAX, bool kInner = false>
 __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc, const int* __restrict__ q4,
                                           int qs, const float* __restrict__ ds, const int* __restrict__ as,
                                           int dsn, int lane, float (&part)[NM][NTMAX],
-                                          int scale_off = kBlockWords * kPanel * 4) {
+                                          int scale_off = kBlockWords * kPanel * 4, float* sc_out = nullptr) {
   int s2[NT];
   if (as == nullptr) {
     // sums of the codes per 32-block: lane l adds words 2l, 2l+1 (sub-block
@@ -212,9 +215,14 @@ __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc
     }
   }
 #pragma unroll
-  for (int m = 0; m < NM; ++m)
+  for (int m = 0; m < NM; ++m) {
 #pragma unroll
-    for (int n = 0; n < NT; ++n) part[m][n] = __fmaf_rn(sc[m], inner[m][n], part[m][n]);
+    for (int n = 0; n < NT; ++n) {
+      if constexpr (kInner) part[m][n] = inner[m][n];
+      else part[m][n] = __fmaf_rn(sc[m], inner[m][n], part[m][n]);
+    }
+    if constexpr (kInner) sc_out[m] = sc[m];
+  }
 }
 
 // Dispatch on the number of pairs of the item (1, 2, 4 or 8 vectors).

@@ -83,15 +83,8 @@ __global__ void k_quant_act_q8(const float* __restrict__ x, int64_t nblk, int8_t
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t blk = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       blk < nblk; blk += warps) {
-    const float v = x[blk * kQBlock + lane];
-    const float amax = warp_max(fabsf(v));
-    const float d = __fdiv_rn(amax, 127.f);
-    int q = 0;
-    if (d != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(v, d))));
-    xq[blk * kQBlock + lane] = static_cast<int8_t>(q);
-    if (lane == 0) xd[blk] = d;
-  }
+       blk < nblk; blk += warps)
+    quant_act_block(x, blk, lane, xq, xd);
 }
 
 int launch_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,

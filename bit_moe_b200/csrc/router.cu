@@ -9,7 +9,9 @@
 #include "bitmoe.h"
 #include "common.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 #include "router.cuh"
+#include "topk.cuh"
 
 namespace bitmoe {
 
@@ -44,35 +46,41 @@ __global__ void k_router_logits(const float* __restrict__ x, const float* __rest
 // chunks (double-buffered cp.async), so each row is read from L2 once per tile
 // instead of once per logit.
 constexpr int kRtT = 16, kRtKC = 256;
+// Few tokens: the tiles have little arithmetic per chunk, so the chunks are
+// 1024 wide (two stages of 80 KB) to cut the number of copy round trips.
+constexpr int kRtKCWide = 1024;
 
 // kWE warps along the experts (8 / kWE along the tokens); a lane holds a
 // micro-tile of kMT tokens x kME experts: the CTA tile is 16 tokens x
 // kWE*kME experts.
-template <int kWE, int kMT, int kME>
+// With xq non-null the CTAs also quantize x to int8 32-blocks, the blocks
+// dealt round-robin over all warps of the grid (as k_quant_act_q8 does).
+template <int kWE, int kMT, int kME, int kKC>
 __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __restrict__ x,
                                                              const float* __restrict__ wr, int ntok, int H,
-                                                             int E, float* __restrict__ logits) {
+                                                             int E, float* __restrict__ logits,
+                                                             int8_t* __restrict__ xq, float* __restrict__ xd) {
   pdl_enter();
   constexpr int kRtMT = kMT, kRtME = kME, kRtE = kWE * kME;
   static_assert((8 / kWE) * kMT == kRtT, "16 tokens per tile");
   extern __shared__ __align__(16) float rsm[];
-  float* xs = rsm;                        // [2][kRtT][kRtKC]
-  float* ws = rsm + 2 * kRtT * kRtKC;     // [2][kRtE][kRtKC]
+  float* xs = rsm;                        // [2][kRtT][kKC]
+  float* ws = rsm + 2 * kRtT * kKC;     // [2][kRtE][kKC]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
   const int wt = (warp / kWE) * kRtMT;    // warp's first token in the tile
   const int we = (warp % kWE) * kRtME;    // warp's first expert in the tile
-  const int nchunk = H / kRtKC;
+  const int nchunk = H / kKC;
   auto stage = [&](int ch, int buf) {
     // (kRtT + kRtE) rows x 256 floats = 2048 chunks of 16 bytes, 8 per thread
-    for (int c = tid; c < (kRtT + kRtE) * (kRtKC / 4); c += 256) {
-      const int row = c / (kRtKC / 4), q = c % (kRtKC / 4);
+    for (int c = tid; c < (kRtT + kRtE) * (kKC / 4); c += 256) {
+      const int row = c / (kKC / 4), q = c % (kKC / 4);
       const bool isx = row < kRtT;
       const int r = isx ? row : row - kRtT;
       const int g = isx ? t0 + r : e0 + r;
-      float* dst = (isx ? xs + (buf * kRtT + r) * kRtKC : ws + (buf * kRtE + r) * kRtKC) + q * 4;
+      float* dst = (isx ? xs + (buf * kRtT + r) * kKC : ws + (buf * kRtE + r) * kKC) + q * 4;
       if (g < (isx ? ntok : E)) {
-        const float* src = (isx ? x : wr) + static_cast<int64_t>(g) * H + ch * kRtKC + q * 4;
+        const float* src = (isx ? x : wr) + static_cast<int64_t>(g) * H + ch * kKC + q * 4;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
       } else {
         *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -86,6 +94,13 @@ __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __rest
 #pragma unroll
     for (int j = 0; j < kRtME; ++j) acc[i][j] = 0.f;
   stage(0, 0);
+  if (xq) {
+    const int64_t nblk = static_cast<int64_t>(ntok) * (H / kQBlock);
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * gridDim.y * 8;
+    for (int64_t blk = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * 8 + warp; blk < nblk;
+         blk += nwarps)
+      quant_act_block(x, blk, lane, xq, xd);
+  }
   for (int ch = 0; ch < nchunk; ++ch) {
     const int buf = ch & 1;
     if (ch + 1 < nchunk) {
@@ -95,15 +110,15 @@ __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __rest
       asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
-    const float* xb = xs + (buf * kRtT + wt) * kRtKC;
-    const float* wb = ws + (buf * kRtE + we) * kRtKC;
+    const float* xb = xs + (buf * kRtT + wt) * kKC;
+    const float* wb = ws + (buf * kRtE + we) * kKC;
 #pragma unroll 2
-    for (int k = lane; k < kRtKC; k += 32) {
+    for (int k = lane; k < kKC; k += 32) {
       float xv[kRtMT], wv[kRtME];
 #pragma unroll
-      for (int i = 0; i < kRtMT; ++i) xv[i] = xb[i * kRtKC + k];
+      for (int i = 0; i < kRtMT; ++i) xv[i] = xb[i * kKC + k];
 #pragma unroll
-      for (int j = 0; j < kRtME; ++j) wv[j] = wb[j * kRtKC + k];
+      for (int j = 0; j < kRtME; ++j) wv[j] = wb[j * kKC + k];
 #pragma unroll
       for (int i = 0; i < kRtMT; ++i)
 #pragma unroll
@@ -124,60 +139,41 @@ __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __rest
   }
 }
 
-// One warp per token: top-k by (logit descending, id ascending), then
-// w_i = exp(l_i - l_0) / sum_j exp(l_j - l_0) in fp32, summed in rank order.
+
+// One warp per token: the token's logits in registers (kPer per lane), then
+// the top-k and the softmax of warp_topk_softmax.
+template <int kPer>
 __global__ void k_topk_softmax(const float* __restrict__ logits, int ntok, int E, int K,
                                int32_t* __restrict__ idx, float* __restrict__ wts) {
   pdl_enter();
-  __shared__ float sel_v[4][kMaxTopK];
-  __shared__ int sel_e[4][kMaxTopK];
-  __shared__ float lgs[4][kMaxExperts];  // the token's logits, read from L2 once
-  const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-  const int t = blockIdx.x * 4 + wl;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= ntok) return;
-  for (int e = lane; e < E; e += 32) lgs[wl][e] = logits[static_cast<int64_t>(t) * E + e];
-  __syncwarp();
-  const float* lg = lgs[wl];
-  uint32_t used = 0;  // bit i: element lane + 32*i already chosen
-  for (int r = 0; r < K; ++r) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-    for (int i = 0; i * 32 + lane < E; ++i) {
-      if (used & (1u << i)) continue;
-      const int e = i * 32 + lane;
-      const float v = lg[e];
-      if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
-    }
+  uint32_t key[kPer];
+  uint32_t need = 0;
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, m);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, m);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = 0u;
+    if (e < E) {
+      key[i] = f32_key(logits[static_cast<int64_t>(t) * E + e]);
+      need |= 1u << i;
     }
-    if ((be & 31) == lane) used |= 1u << (be >> 5);
-    if (lane == 0) { sel_v[wl][r] = bv; sel_e[wl][r] = be; }
   }
-  __syncwarp();
-  if (lane == 0) {
-    const float l0 = sel_v[wl][0];
-    float ex[kMaxTopK];
-    float den = 0.f;
-    for (int r = 0; r < K; ++r) {
-      ex[r] = expf(__fsub_rn(sel_v[wl][r], l0));
-      den = __fadd_rn(den, ex[r]);
-    }
-    for (int r = 0; r < K; ++r) {
-      idx[static_cast<int64_t>(t) * K + r] = sel_e[wl][r];
-      wts[static_cast<int64_t>(t) * K + r] = __fdiv_rn(ex[r], den);
-    }
+  int my_e;
+  float w;
+  warp_topk_softmax<kPer>(key, need, K, lane, my_e, w);
+  if (lane < K) {
+    idx[static_cast<int64_t>(t) * K + lane] = my_e;
+    wts[static_cast<int64_t>(t) * K + lane] = w;
   }
 }
 
-template <int kWE, int kMT, int kME>
+template <int kWE, int kMT, int kME, int kKC = kRtKC>
 static void launch_tiled(const float* x, const float* wr, int ntok, int H, int E, float* logits,
-                         cudaStream_t stream) {
-  auto kern = k_router_logits_tiled<kWE, kMT, kME>;
-  const size_t smem = sizeof(float) * 2 * (kRtT + kWE * kME) * kRtKC;
+                         cudaStream_t stream, int8_t* xq = nullptr, float* xd = nullptr) {
+  auto kern = k_router_logits_tiled<kWE, kMT, kME, kKC>;
+  const size_t smem = sizeof(float) * 2 * (kRtT + kWE * kME) * kKC;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -186,7 +182,7 @@ static void launch_tiled(const float* x, const float* wr, int ntok, int H, int E
     attr_done[dev] = true;
   }
   const dim3 grid((ntok + kRtT - 1) / kRtT, (E + kWE * kME - 1) / (kWE * kME));
-  launch_k(kern, grid, dim3(256), smem, stream, x, wr, ntok, H, E, logits);
+  launch_k(kern, grid, dim3(256), smem, stream, x, wr, ntok, H, E, logits, xq, xd);
 }
 
 int launch_router_logits(const float* x, const float* wr, int ntok, int H, int E, float* logits,
@@ -198,6 +194,8 @@ int launch_router_logits(const float* x, const float* wr, int ntok, int H, int E
     launch_k(k_router_logits, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, wr, ntok, H, E, logits);
   } else if (ntok >= 4 * kRtT) {
     launch_tiled<4, 8, 4>(x, wr, ntok, H, E, logits, stream);  // 16 x 16 tiles
+  } else if (H % kRtKCWide == 0) {
+    launch_tiled<2, 4, 2, kRtKCWide>(x, wr, ntok, H, E, logits, stream);  // 16 x 4 tiles, wide chunks
   } else {
     launch_tiled<2, 4, 2>(x, wr, ntok, H, E, logits, stream);  // 16 x 4 tiles
   }
@@ -209,9 +207,28 @@ int launch_route_topk(const float* x, const float* wr, int ntok, int H, int E, i
                       float* wts, float* logits, cudaStream_t stream) {
   int rc = launch_router_logits(x, wr, ntok, H, E, logits, stream);
   if (rc) return rc;
-  launch_k(k_topk_softmax, dim3((ntok + 3) / 4), dim3(128), 0, stream, logits, ntok, E, K, idx, wts);
+  const dim3 grid((ntok + 3) / 4), block(128);
+  if (E <= 128)
+    launch_k(k_topk_softmax<4>, grid, block, 0, stream, logits, ntok, E, K, idx, wts);
+  else if (E <= 256)
+    launch_k(k_topk_softmax<8>, grid, block, 0, stream, logits, ntok, E, K, idx, wts);
+  else
+    launch_k(k_topk_softmax<32>, grid, block, 0, stream, logits, ntok, E, K, idx, wts);
   note_launch(MOE_K_TOPK, stream);
   return check_launch("route_topk");
+}
+
+bool router_quant_small_ok(int ntok, int H) { return ntok <= 32 && H % kRtKC == 0; }
+
+int launch_router_quant_small(const float* x, const float* wr, int ntok, int H, int E, float* logits,
+                              int8_t* xq, float* xd, cudaStream_t stream) {
+  if (!router_quant_small_ok(ntok, H)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "router_quant: shape");
+  if (H % kRtKCWide == 0)
+    launch_tiled<2, 4, 2, kRtKCWide>(x, wr, ntok, H, E, logits, stream, xq, xd);  // 16 x 4 tiles, wide chunks
+  else
+    launch_tiled<2, 4, 2>(x, wr, ntok, H, E, logits, stream, xq, xd);
+  note_launch(MOE_K_ROUTER_QUANT, stream);
+  return check_launch("router_quant");
 }
 
 }  // namespace bitmoe

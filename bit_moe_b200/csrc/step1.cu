@@ -30,6 +30,7 @@
 #include "decode2.cuh"
 #include "matvec.cuh"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace bitmoe {
 
@@ -46,15 +47,20 @@ constexpr int kS1MaxE = kNC * 32;          // experts: one per lane of the polli
 constexpr int kTagStride = 16;
 static_assert(kS1MaxK <= kNC, "phase C: one warp per slot");
 
+// One finished gate/up unit (slot j, 32-row panel p of ffn) is published as
+// kUnitWords tagged words: its 32 int8 codes four to a word, the fp32 scale
+// and the int32 code sum.
+constexpr int kUnitWords = kPanel / 4 + 2;
+
 struct Step1Params {
   Decode2Params D;
   unsigned long long* ticket;  // launch ticket counter (only grows): generation = ticket / CTAs
   unsigned long long* tagged;  // [E][kTagStride] logits as (generation + 1) << 32 | fp32 bits
-  uint32_t* slot_cnt;          // [top_k] finished gate/up units per slot (zeroed each launch)
+  unsigned long long* units;   // [top_k][ffn/32][kUnitWords] unit outputs, tagged the same way
 };
 
 struct Step1Layout {
-  size_t ring, pref, xq4, xd, xas, lg, sel, red, flag, xf, act, total;
+  size_t ring, pref, xq4, xd, xas, sel, red, flag, rbar, xf, act, inner, total;
   int sw;  // ring slots per warp
 };
 
@@ -74,14 +80,15 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
       return o;
     };
     size_t ring = static_cast<size_t>(kS1Warps) * sw * Slot<2, 1, true>::bytes;
-    const size_t xf = static_cast<size_t>(H) * 4 + static_cast<size_t>(E) * 4;
+    const size_t xf = static_cast<size_t>(H) * 4;
     const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
+    const size_t inner = static_cast<size_t>(2) * K * (F / kBlock) * kPanel * 4;
     if (ring < xf) ring = xf;
-    if (ring < act) ring = act;
+    if (ring < act + inner) ring = act + inner;
     L.ring = take(ring);
     L.act = L.ring;
+    L.inner = L.ring + act;
     L.xf = L.ring;
-    L.lg = L.ring + static_cast<size_t>(H) * 4;
     const size_t pref = static_cast<size_t>(K) * (F / kBlock) * kMatBytes;
     const size_t rows = static_cast<size_t>(2) * H * 4;  // at most two router rows per CTA
     L.pref = take(pref > rows ? pref : rows);
@@ -91,6 +98,7 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
     L.sel = take(2 * kMaxTopK * 4);
     L.red = take(static_cast<size_t>(kS1Streams) * 2 * kNC * 32 * 4);
     L.flag = take(64);
+    L.rbar = take(static_cast<size_t>(kS1Warps) * 3 * 8);
     L.total = off;
     if (L.total <= static_cast<size_t>(kMaxDynSmem)) break;
   }
@@ -117,12 +125,6 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Order-preserving map of an fp32 value to uint32 (larger value, larger key).
-__device__ __forceinline__ uint32_t f32_key(float v) {
-  const uint32_t b = __float_as_uint(v == 0.f ? 0.f : v);  // -0 ranks as +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
 __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const Decode2Params& D = S1.D;
@@ -137,15 +139,16 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   int* sq4 = reinterpret_cast<int*>(smem + L.xq4);
   float* sxd = reinterpret_cast<float*>(smem + L.xd);
   int* sxas = reinterpret_cast<int*>(smem + L.xas);
-  float* lg = reinterpret_cast<float*>(smem + L.lg);
   int* sel_e = reinterpret_cast<int*>(smem + L.sel);
   float* sel_w = reinterpret_cast<float*>(smem + L.sel + kMaxTopK * 4);
   float* xf = reinterpret_cast<float*>(smem + L.xf);
   float* rows = reinterpret_cast<float*>(smem + L.pref);
   uint32_t* sgen = reinterpret_cast<uint32_t*>(smem + L.flag + 32);
+  uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + L.rbar);  // [warp][ring slot]
   if (tid == 0) {
     *abort = 0;
     mbar_init(pbar, K);
+    for (int i = 0; i < kS1Warps * L.sw; ++i) mbar_init(rbar + i, 1);
     fence_mbar_init();
     // every CTA takes one ticket per launch, so the tickets of a launch are
     // [g*C, (g+1)*C) and ticket / C is the same generation g in every CTA;
@@ -154,18 +157,22 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     *sgen = g + 1u;
   }
 
+  // ---------------- phase A: x, int8 x^, logits of this CTA's experts
+  // The router rows are caller data that no kernel of this library writes,
+  // so their copy starts before the dependency wait below.
+  const int e0 = static_cast<int>(static_cast<int64_t>(E) * c / C);
+  const int e1 = static_cast<int>(static_cast<int64_t>(E) * (c + 1) / C);
+  for (int q = tid; q < (e1 - e0) * H * 4 / 16; q += blockDim.x)
+    cp16(reinterpret_cast<unsigned char*>(rows) + q * 16,
+         reinterpret_cast<const unsigned char*>(D.wr + static_cast<size_t>(e0) * H) + q * 16);
+  cp_commit();
+
   // launched as a programmatic dependent: everything the kernels before it
   // wrote (x among them) is visible only past this wait
   pdl_wait();
 
-  // ---------------- phase A: x, int8 x^, logits of this CTA's experts
-  const int e0 = static_cast<int>(static_cast<int64_t>(E) * c / C);
-  const int e1 = static_cast<int>(static_cast<int64_t>(E) * (c + 1) / C);
   for (int q = tid; q < H * 4 / 16; q += blockDim.x)
     cp16(reinterpret_cast<unsigned char*>(xf) + q * 16, reinterpret_cast<const unsigned char*>(D.x) + q * 16);
-  for (int q = tid; q < (e1 - e0) * H * 4 / 16; q += blockDim.x)
-    cp16(reinterpret_cast<unsigned char*>(rows) + q * 16,
-         reinterpret_cast<const unsigned char*>(D.wr + static_cast<size_t>(e0) * H) + q * 16);
   cp_commit();
   cp_wait<0>();
   __syncthreads();
@@ -190,7 +197,6 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     // a round in flight at once), then the top-k, while the other warps
     // quantize x
     constexpr int kPer = kS1MaxE / 32;
-    constexpr int kNone = 0x7fffffff;
     unsigned long long v[kPer];
     uint32_t ready = 0, need = 0;
 #pragma unroll
@@ -211,40 +217,14 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         *abort = 1;
       }
     } else {
-      // the K largest logits, larger first, equal logits by lower id: per
-      // round the largest key over the warp, then the lowest id holding it
-      // (a lane's own entries are in ascending id order, so it keeps the first
-      // of equal keys)
+      // the top-k and the renormalised softmax over it
       uint32_t key[kPer];
 #pragma unroll
       for (int i = 0; i < kPer; ++i) key[i] = f32_key(__uint_as_float(static_cast<uint32_t>(v[i])));
-      uint32_t avail = need;
-      int my_e = 0;
-      float my_l = 0.f;
-#pragma unroll 1
-      for (int r = 0; r < K; ++r) {
-        uint32_t bk = 0u;
-        int bi = kNone;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i)
-          if (((avail >> i) & 1u) && (bi == kNone || key[i] > bk)) { bk = key[i]; bi = lane + 32 * i; }
-        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-        const int wi = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == wk ? static_cast<uint32_t>(bi) : 0xffffffffu));
-        if ((wi & 31) == lane) avail &= ~(1u << (wi >> 5));
-        if (lane == r) my_e = wi;
-      }
-#pragma unroll
-      for (int i = 0; i < kPer; ++i)
-        if (lane + 32 * i < E) lg[lane + 32 * i] = __uint_as_float(static_cast<uint32_t>(v[i]));
-      __syncwarp();
-      if (lane < K) my_l = lg[my_e];
-      // softmax over the selected, renormalised: exp(l - l_0) / sum, summed in slot order
-      const float l0 = __shfl_sync(0xffffffffu, my_l, 0);
-      const float ex = lane < K ? expf(__fsub_rn(my_l, l0)) : 0.f;
-      float den = 0.f;
-      for (int r = 0; r < K; ++r) den = __fadd_rn(den, __shfl_sync(0xffffffffu, ex, r));
+      int my_e;
+      float w;
+      warp_topk_softmax<kPer>(key, need, K, lane, my_e, w);
       if (lane < K) {
-        const float w = __fdiv_rn(ex, den);
         sel_e[lane] = my_e;
         sel_w[lane] = w;
         if (c == 0) {
@@ -322,32 +302,41 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     unsigned char* myring = smem + L.ring + static_cast<size_t>(warp) * SW * SL::bytes;
     float* rb = reinterpret_cast<float*>(smem + L.red) + h * (2 * kNC * 32);
     const int bar_done = 1 + h, bar_free = 1 + kS1Streams + h;
-    uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
+    const unsigned long long tag64 = static_cast<unsigned long long>(*sgen) << 32;
     int im = 0;
     int ib = w8;
+    // ring slot k of a warp is filled by bulk copies issued by its lane 0
+    // and completes on the slot's mbarrier
+    const uint64_t pol = policy_evict_first();
+    uint64_t* mybar = rbar + warp * SW;
     auto issue_next = [&](int slot) {
       while (im < nmine && ib >= nbH) { ++im; ib = w8; }
       if (im < nmine) {
-        const int64_t iu = my_unit(im);
-        Group G;
-        G.expert = sel_e[iu / panels];
-        G.count = 1;
-        G.start = static_cast<int>(iu / panels);
-        ActSrc<1> A{};
-        issue_item<2, 1, true>(myring + slot * SL::bytes, P, G, A, static_cast<int>(iu % panels), ib, lane);
+        if (lane == 0) {
+          const int64_t iu = my_unit(im);
+          const int e = sel_e[iu / panels];
+          unsigned char* dst = myring + slot * SL::bytes;
+          if (e >= 0 && e < E) {
+            const size_t pb = (static_cast<size_t>(e) * panels + static_cast<size_t>(iu % panels)) * nbH + ib;
+            const uint32_t tb = kBlockWords * kPanel * 4, sb = kPanel * 2;
+            mbar_arrive_expect_tx(mybar + slot, 2 * (tb + sb));
+            bulk_g2s(dst, P.gate_trits + pb * kBlockWords * kPanel, tb, mybar + slot, pol);
+            bulk_g2s(dst + tb, P.gate_scales + pb * kPanel, sb, mybar + slot, pol);
+            bulk_g2s(dst + kMatBytes, P.up_trits + pb * kBlockWords * kPanel, tb, mybar + slot, pol);
+            bulk_g2s(dst + kMatBytes + tb, P.up_scales + pb * kPanel, sb, mybar + slot, pol);
+          } else {
+            mbar_arrive(mybar + slot);
+          }
+        }
         ib += kNC;
       }
-      cp_commit();
     };
 #pragma unroll 1
     for (int k = 0; k < SW; ++k) issue_next(k);
-    // launch g counts on slot counter set g & 1 and clears set (g + 1) & 1
-    // for launch g + 1 (the previous launch has completed: see pdl_wait)
-    if (c == 0 && tid == 0)
-      for (int j = 0; j < kS1MaxK; ++j) S1.slot_cnt[(*sgen & 1u) * kS1MaxK + j] = 0u;
-    // then the down panels, which are needed only after the gate/up phase
-    if (has_panel && tid < K) {
-      const int j = tid;
+    // then the down panels, which are needed only after the gate/up phase:
+    // lane 0 of warp j issues slot j's
+    if (has_panel && lane == 0 && warp < K) {
+      const int j = warp;
       const size_t pb0 = (static_cast<size_t>(sel_e[j]) * (H / kPanel) + panelH) * nbF;
       unsigned char* dst = pref + j * pref_slot;
       const uint32_t tb = static_cast<uint32_t>(nbF) * kBlockWords * kPanel * 4;
@@ -362,12 +351,15 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       const int j = static_cast<int>(u / panels), p = static_cast<int>(u % panels);
       float part[2][1] = {{0.f}, {0.f}};
       for (int b = w8; b < nbH; b += kNC, ++s) {
-        if (SW == 3) cp_wait<2>(); else cp_wait<1>();
-        __syncwarp();
-        block_dot<2, 1, 1>(myring + (s % SW) * SL::bytes, sq4 + b * (kBlock / 4), 0, sxd + b * kSubPerBlock,
+        const int slot = s % SW;
+        if (!mbar_wait_sleep(mybar + slot, static_cast<uint32_t>(s / SW) & 1u) && lane == 0) {
+          record_status(P.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+        }
+        block_dot<2, 1, 1>(myring + slot * SL::bytes, sq4 + b * (kBlock / 4), 0, sxd + b * kSubPerBlock,
                            sxas + b * kSubPerBlock, 0, lane, part);
         __syncwarp();
-        issue_next(s % SW);
+        issue_next(slot);
       }
       // the epilogue warp has read the previous unit's sums
       if (ui > 0 && w8 != 0) stream_bar_sync(bar_free);
@@ -387,75 +379,106 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         const float dd = __fdiv_rn(amax, 127.f);
         int q = 0;
         if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
-        P.aq[static_cast<size_t>(j) * F + p * kPanel + lane] = static_cast<int8_t>(q);
         const int qs = __reduce_add_sync(0xffffffffu, q);
-        if (lane == 0) {
-          P.ad[static_cast<size_t>(j) * (F / kQBlock) + p] = dd;
-          P.asum[static_cast<size_t>(j) * (F / kQBlock) + p] = qs;
-        }
-        __syncwarp();
-        if (lane == 0) {  // publish the unit: its codes, scale and sum, then the count
-          __threadfence();
-          atomicAdd(cnt + j, 1u);
-        }
+        // publish the unit: lane i < 8 the codes of rows 4i..4i+3, lane 8
+        // the scale, lane 9 the code sum, each word tagged with the launch
+        const uint32_t qb = static_cast<uint32_t>(q) & 0xffu;
+        const uint32_t w4 = qb | (__shfl_down_sync(0xffffffffu, qb, 1) << 8) |
+                            (__shfl_down_sync(0xffffffffu, qb, 2) << 16) |
+                            (__shfl_down_sync(0xffffffffu, qb, 3) << 24);
+        const uint32_t cw = __shfl_sync(0xffffffffu, w4, (4 * lane) & 31);
+        const uint32_t payload = lane < kPanel / 4 ? cw
+                                 : lane == kPanel / 4 ? __float_as_uint(dd) : static_cast<uint32_t>(qs);
+        if (lane < kUnitWords)
+          st_relaxed_u64(S1.units + (static_cast<size_t>(j) * panels + p) * kUnitWords + lane, tag64 | payload);
       }
     }
-    cp_wait<0>();
+    // every copy issued was consumed above: none is in flight here
     __syncthreads();
   }
 
   // ---------------- phase C: this CTA's panel of hidden, all slots
   if (has_panel) {
     // the prefetch must land before this CTA reads it or exits
-    bool ok = mbar_wait(pbar, 0);
+    bool ok = mbar_wait_sleep(pbar, 0);
     if (!ok) record_status(P.status, MOE_ERR_TIMEOUT);
-    // warp j takes slot j as soon as the slot's gate/up units are published
-    // (slots of the first round of units complete first); the slots are
-    // combined in order once all are done
+    // warp w takes slot w % kNC, the first (w < kNC) or second half of its
+    // blocks of ffn, as soon as the units of those blocks are published; each
+    // block's inner sum and weight scale go to shared memory, and one warp
+    // applies the scales and combines the slots in the order of the grouped
+    // down kernel
+    const int panels = F / kPanel;
     int* aq4 = reinterpret_cast<int*>(smem + L.act);                       // [K][F/4]
     float* ad = reinterpret_cast<float*>(aq4 + K * (F / 4));                 // [K][F/32]
     int* aas = reinterpret_cast<int*>(ad + K * (F / kQBlock));              // [K][F/32]
-    float* part = reinterpret_cast<float*>(smem + L.red);                  // [K][32]
-    if (warp < K && ok) {
-      const int j = warp;
-      const uint32_t need = static_cast<uint32_t>(F / kPanel);
-      const uint32_t* cnt = S1.slot_cnt + ((*sgen - 1u) & 1u) * kS1MaxK;
-      bool ready = true;
-      if (lane == 0) {
-        for (uint32_t polls = 0; ld_acquire_gpu(cnt + j) < need; ++polls) {
-          if (polls > kSpinLimit) {
-            ready = false;
-            record_status(P.status, MOE_ERR_TIMEOUT);
-            *abort = 1;
-            break;
+    float* sinner = reinterpret_cast<float*>(smem + L.inner);               // [K][nbF][32]
+    float* sscale = sinner + K * nbF * kPanel;                              // [K][nbF][32]
+    const int j = warp % kNC, half = warp / kNC;
+    const int nb0 = (nbF + 1) / 2;
+    const int bb = half ? nb0 : 0, be = half ? nbF : nb0;
+    if (j < K && ok && bb < be) {
+      // the tagged words of panels [8*bb, 8*be) of slot j, all loads of a
+      // round in flight at once
+      constexpr int kPerC = (kS1MaxF / kBlock + 1) / 2 * (kBlock / kPanel) * kUnitWords / 32;
+      const int nw = (be - bb) * (kBlock / kPanel) * kUnitWords;
+      const unsigned long long* src =
+          S1.units + (static_cast<size_t>(j) * panels + bb * (kBlock / kPanel)) * kUnitWords;
+      const uint32_t tag = *sgen;
+      unsigned long long v[kPerC];
+      uint32_t ready = 0, need = 0;
+#pragma unroll
+      for (int i = 0; i < kPerC; ++i)
+        if (lane + 32 * i < nw) need |= 1u << i;
+      for (uint32_t polls = 0; ready != need; ++polls) {
+        if (polls > kSpinLimit) break;
+#pragma unroll
+        for (int i = 0; i < kPerC; ++i)
+          if ((need & ~ready) & (1u << i)) v[i] = ld_relaxed_u64(src + lane + 32 * i);
+#pragma unroll
+        for (int i = 0; i < kPerC; ++i)
+          if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+      }
+      if (!__all_sync(0xffffffffu, ready == need)) {
+        if (lane == 0) {
+          record_status(P.status, MOE_ERR_TIMEOUT);
+          *abort = 1;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kPerC; ++i) {
+          const int w = lane + 32 * i;
+          if (w < nw) {
+            const int pl = bb * (kBlock / kPanel) + w / kUnitWords, k = w % kUnitWords;
+            const uint32_t x32 = static_cast<uint32_t>(v[i]);
+            if (k < kPanel / 4) aq4[j * (F / 4) + pl * (kPanel / 4) + k] = static_cast<int>(x32);
+            else if (k == kPanel / 4) ad[j * (F / kQBlock) + pl] = __uint_as_float(x32);
+            else aas[j * (F / kQBlock) + pl] = static_cast<int>(x32);
           }
         }
-      }
-      ready = __shfl_sync(0xffffffffu, ready, 0);
-      if (ready) {
-        for (int q = lane; q < F / 4; q += 32)
-          aq4[j * (F / 4) + q] = __ldcg(reinterpret_cast<const int*>(P.aq + static_cast<size_t>(j) * F) + q);
-        for (int q = lane; q < F / kQBlock; q += 32) {
-          ad[j * (F / kQBlock) + q] = __ldcg(P.ad + static_cast<size_t>(j) * (F / kQBlock) + q);
-          aas[j * (F / kQBlock) + q] = __ldcg(P.asum + static_cast<size_t>(j) * (F / kQBlock) + q);
-        }
         __syncwarp();
-        float acc[1][1] = {{0.f}};
         const unsigned char* wj = pref + j * pref_slot;
-        for (int b = 0; b < nbF; ++b) {
+        for (int b = bb; b < be; ++b) {
           const int scale_off = nbF * kBlockWords * kPanel * 4 + b * kPanel * 2 - b * kBlockWords * kPanel * 4;
-          block_dot<1, 1, 1>(wj + static_cast<size_t>(b) * kBlockWords * kPanel * 4,
-                             aq4 + j * (F / 4) + b * (kBlock / 4), 0,
-                             ad + j * (F / kQBlock) + b * kSubPerBlock, aas + j * (F / kQBlock) + b * kSubPerBlock,
-                             0, lane, acc, scale_off);
+          float inner[1][1];
+          float sc[1];
+          block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kBlockWords * kPanel * 4,
+                                   aq4 + j * (F / 4) + b * (kBlock / 4), 0,
+                                   ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                   aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
+          sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
+          sscale[(j * nbF + b) * kPanel + lane] = sc[0];
         }
-        part[j * 32 + lane] = acc[0][0];
       }
     }
     __syncthreads();
     if (!*abort && ok && warp == 0) {
       float y = 0.f;
-      for (int j = 0; j < K; ++j) y = __fmaf_rn(sel_w[j], part[j * 32 + lane], y);
+      for (int jj = 0; jj < K; ++jj) {
+        float part = 0.f;
+        for (int b = 0; b < nbF; ++b)
+          part = __fmaf_rn(sscale[(jj * nbF + b) * kPanel + lane], sinner[(jj * nbF + b) * kPanel + lane], part);
+        y = __fmaf_rn(sel_w[jj], part, y);
+      }
       P.y[panelH * kPanel + lane] = y;
     }
   }
@@ -471,7 +494,8 @@ bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem) {
   return L.total <= static_cast<size_t>(kMaxDynSmem);
 }
 
-int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* slot_cnt, cudaStream_t stream) {
+int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned long long* units,
+                 cudaStream_t stream) {
   static bool done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -481,7 +505,7 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, uint32_t* s
   }
   size_t smem = 0;
   if (!step1_supported(D.P, D.n_sm, &smem)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "step1: unsupported shape");
-  Step1Params S{D, ticket, reinterpret_cast<unsigned long long*>(D.logits), slot_cnt};
+  Step1Params S{D, ticket, reinterpret_cast<unsigned long long*>(D.logits), units};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(D.n_sm);
   cfg.blockDim = dim3(kS1Warps * 32);

@@ -200,7 +200,8 @@ typedef enum {
   MOE_K_QUANTIZE_WEIGHTS = 0, MOE_K_QUANT_ACT = 1, MOE_K_ROUTER_LOGITS = 2, MOE_K_TOPK = 3,
   MOE_K_GROUP = 4, MOE_K_GATEUP = 5, MOE_K_DOWN = 6, MOE_K_DEBUG_MATVEC = 7,
   MOE_K_PREFILL_GATEUP = 8, MOE_K_PREFILL_DOWN = 9, MOE_K_ROUTE = 10, MOE_K_COMBINE = 11,
-  MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COPY = 14, MOE_K_COUNT = 15
+  MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COPY = 14, MOE_K_ROUTER_QUANT = 15,
+  MOE_K_TOPK_GROUP = 16, MOE_K_COUNT = 17
 } moe_kernel_id;
 /* Number of kernels this thread has launched through the library so far. */
 int64_t moe_launch_count(void);
