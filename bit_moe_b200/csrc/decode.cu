@@ -212,8 +212,11 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
   }
 }
 
+// Four CTAs per SM (at most 64 registers a thread): the items of a decode
+// batch are mostly single pairs, whose path needs few registers; the rare
+// 8-pair path spills a little.
 template <int NTMAX>
-__global__ void __launch_bounds__(kGateUpWarps * 32) k_gateup(DecodeParams P) {
+__global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
   Item item;
