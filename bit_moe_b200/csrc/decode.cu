@@ -304,8 +304,10 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
   for (int n = 0; n < item.count; ++n) arrive_and_combine(P, item_pair(P, item, n), panel, lane);
 }
 
+// Eight CTAs per SM (at most 64 registers a thread, which leaves room for the
+// prefetched next block of weight words in panel_dot).
 template <int NTMAX>
-__global__ void __launch_bounds__(kDownWarps * 32) k_down(DecodeParams P) {
+__global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
   Item item;

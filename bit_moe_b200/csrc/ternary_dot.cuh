@@ -76,15 +76,45 @@ __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
                                           const float* __restrict__ d,
                                           const int* __restrict__ as, float (&out)[NM][NT],
                                           int32_t* isum_out = nullptr, size_t isum_stride = 0) {
+  // one matrix: the next block's words are loaded while this one decodes
+  uint32_t wn[NM][kBlockWords];
+  uint16_t sn[NM];
+  if (NM == 1 && b_begin < b_end) {
+#pragma unroll
+    for (int m = 0; m < NM; ++m) {
+      const uint32_t* src = tw[m] + static_cast<size_t>(b_begin) * kBlockWords * kPanel;
+#pragma unroll
+      for (int j = 0; j < kBlockWords; ++j) wn[m][j] = ld_stream_u32(src + j * kPanel);
+      sn[m] = ts[m][static_cast<size_t>(b_begin) * kPanel];
+    }
+  }
   for (int b = b_begin; b < b_end; b += b_step) {
     uint32_t w[NM][kBlockWords];
     float sc[NM];
+    if constexpr (NM == 1) {
 #pragma unroll
-    for (int m = 0; m < NM; ++m) {
-      const uint32_t* src = tw[m] + static_cast<size_t>(b) * kBlockWords * kPanel;
+      for (int m = 0; m < NM; ++m) {
 #pragma unroll
-      for (int j = 0; j < kBlockWords; ++j) w[m][j] = ld_stream_u32(src + j * kPanel);
-      sc[m] = f16_bits_to_f32(ts[m][static_cast<size_t>(b) * kPanel]);
+        for (int j = 0; j < kBlockWords; ++j) w[m][j] = wn[m][j];
+        sc[m] = f16_bits_to_f32(sn[m]);
+      }
+      if (b + b_step < b_end) {
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+          const uint32_t* src = tw[m] + static_cast<size_t>(b + b_step) * kBlockWords * kPanel;
+#pragma unroll
+          for (int j = 0; j < kBlockWords; ++j) wn[m][j] = ld_stream_u32(src + j * kPanel);
+          sn[m] = ts[m][static_cast<size_t>(b + b_step) * kPanel];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const uint32_t* src = tw[m] + static_cast<size_t>(b) * kBlockWords * kPanel;
+#pragma unroll
+        for (int j = 0; j < kBlockWords; ++j) w[m][j] = ld_stream_u32(src + j * kPanel);
+        sc[m] = f16_bits_to_f32(ts[m][static_cast<size_t>(b) * kPanel]);
+      }
     }
     int acc[NM][NT];
     float inner[NM][NT];
