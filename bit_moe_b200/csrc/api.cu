@@ -420,10 +420,11 @@ int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, co
   float* xs = reinterpret_cast<float*>(base + W.xs);
   float* ys = reinterpret_cast<float*>(base + W.ys);
   const size_t bytes = sizeof(float) * static_cast<size_t>(ntok) * L->hidden;
-  // A few kilobytes from page-locked memory the GPU can address: one CTA
-  // copies them with loads over the bus (about a microsecond, and chained to
+  // A few kilobytes of page-locked memory the GPU can address: one CTA
+  // copies x in with loads over the bus (about a microsecond, and chained to
   // the step by programmatic dependent launch) instead of a DMA copy, whose
-  // setup costs several microseconds.  Larger or pageable buffers: DMA copies.
+  // setup costs several microseconds, and the step's kernels store y straight
+  // into the host buffer.  Larger or pageable buffers: DMA copies.
   const void* xd = host_device_view(x_host);
   void* yd = host_device_view(y_host);
   const bool small = bytes <= kSmallHostCopy && xd && yd && aligned16(xd) && aligned16(yd);
@@ -434,8 +435,8 @@ int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, co
     err = cudaMemcpyAsync(xs, x_host, bytes, cudaMemcpyHostToDevice, s);
     if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy in: %s", cudaGetErrorString(err));
   }
+  if (small) return moe_forward(L, w_router, ntok, xs, static_cast<float*>(yd), ws, ws_bytes, stream);
   if ((rc = moe_forward(L, w_router, ntok, xs, ys, ws, ws_bytes, stream))) return rc;
-  if (small) return launch_copy16(yd, ys, bytes, s);
   err = cudaMemcpyAsync(y_host, ys, bytes, cudaMemcpyDeviceToHost, s);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "forward_host: copy out: %s", cudaGetErrorString(err));
   return MOE_OK;

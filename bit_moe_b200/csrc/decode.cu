@@ -101,15 +101,16 @@ __global__ void __launch_bounds__(kGroupThreads) k_group(DecodeParams P) {
   group_body(P);
 }
 
-// Up to kGroupThreads/32 tokens: warp t takes token t's top-k and softmax
-// (warp_topk_softmax, as k_topk_softmax), then the CTA groups the pairs.
+// Up to kMaxDecodeTokens tokens: warp w takes the top-k and softmax of tokens
+// w, w + 32, ... (warp_topk_softmax, as k_topk_softmax), then the CTA groups
+// the pairs.
 template <int kPer>
 __global__ void __launch_bounds__(kGroupThreads) k_topk_group(DecodeParams P, const float* __restrict__ logits,
                                                               float* __restrict__ wts) {
   pdl_enter();
-  const int lane = threadIdx.x & 31, t = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int E = P.n_experts, K = P.top_k;
-  if (t < P.ntok) {
+  for (int t = threadIdx.x >> 5; t < P.ntok; t += kGroupThreads / 32) {
     uint32_t key[kPer];
     uint32_t need = 0;
 #pragma unroll
@@ -397,7 +398,7 @@ int launch_group(const DecodeParams& P, cudaStream_t stream) {
 }
 
 int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cudaStream_t stream) {
-  if (P.ntok > kGroupThreads / 32) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "topk_group: more than %d tokens", kGroupThreads / 32);
+  if (P.ntok > kMaxDecodeTokens) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "topk_group: more than %d tokens", kMaxDecodeTokens);
   const int E = P.n_experts;
   if (E <= 128) launch_k(k_topk_group<4>, dim3(1), dim3(kGroupThreads), 0, stream, P, logits, wts);
   else if (E <= 256) launch_k(k_topk_group<8>, dim3(1), dim3(kGroupThreads), 0, stream, P, logits, wts);

@@ -49,7 +49,7 @@ struct GroupWs {
 size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G);
 
 int launch_group(const DecodeParams& P, cudaStream_t stream);
-// Top-k softmax of P.ntok <= 32 tokens' logits ([ntok][E] fp32) into P.idx
+// Top-k softmax of P.ntok <= 64 tokens' logits ([ntok][E] fp32) into P.idx
 // and wts, then the grouping of launch_group, in one single-CTA kernel.
 int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cudaStream_t stream);
 int launch_ffn(const DecodeParams& P, cudaStream_t stream);

@@ -218,7 +218,7 @@ int launch_route_topk(const float* x, const float* wr, int ntok, int H, int E, i
   return check_launch("route_topk");
 }
 
-bool router_quant_small_ok(int ntok, int H) { return ntok <= 32 && H % kRtKC == 0; }
+bool router_quant_small_ok(int ntok, int H) { return ntok <= kMaxDecodeTokens && H % kRtKC == 0; }
 
 int launch_router_quant_small(const float* x, const float* wr, int ntok, int H, int E, float* logits,
                               int8_t* xq, float* xd, cudaStream_t stream) {

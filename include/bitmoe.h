@@ -180,9 +180,10 @@ int moe_forward(const moe_layer* layer, const float* w_router, int32_t ntok, con
                 float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
 /* The same with x and y in HOST memory (pinned for asynchronous copies):
  * copies x in, runs moe_forward, copies y out, all on `stream`.  Up to 64 KB
- * of page-locked x and y are moved by a small kernel that addresses them
- * over the bus; larger or pageable buffers by DMA copies.  The host buffers
- * must stay valid until the stream reaches the end of the call.           */
+ * of page-locked x is moved in by a small kernel that addresses it over the
+ * bus, and the step's kernels store y straight into page-locked y of that
+ * size; larger or pageable buffers go by DMA copies.  The host buffers must
+ * stay valid until the stream reaches the end of the call.                */
 int moe_forward_host(const moe_layer* layer, const float* w_router, int32_t ntok,
                      const float* x_host, float* y_host, void* ws, size_t ws_bytes,
                      moe_stream_t stream);
