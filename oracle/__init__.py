@@ -46,6 +46,14 @@ def lib():
         L.orc_scale_index.argtypes = [i64, i64, i64]
         L.orc_quantize_weights.restype = ctypes.c_int
         L.orc_quantize_weights.argtypes = [p, i64, i64, p, p]
+        L.orc_sign_words.restype = i64
+        L.orc_sign_words.argtypes = [i64, i64]
+        L.orc_sign_word_index.restype = i64
+        L.orc_sign_word_index.argtypes = [i64, i64, i64, ctypes.c_int]
+        L.orc_quantize_weights_sign.restype = ctypes.c_int
+        L.orc_quantize_weights_sign.argtypes = [p, i64, i64, p, p]
+        L.orc_unpack_weights_sign.restype = ctypes.c_int
+        L.orc_unpack_weights_sign.argtypes = [p, p, i64, i64, i64, i64, p, p]
         L.orc_unpack_weights.restype = ctypes.c_int
         L.orc_unpack_weights.argtypes = [p, p, i64, i64, i64, i64, p, p]
         L.orc_quant_act_q8.restype = ctypes.c_int
@@ -71,7 +79,11 @@ class OrcLayer(ctypes.Structure):
         ("gate_trits", ctypes.c_void_p), ("gate_scales", ctypes.c_void_p),
         ("up_trits", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
         ("down_trits", ctypes.c_void_p), ("down_scales", ctypes.c_void_p),
+        ("format", ctypes.c_int64),
     ]
+
+
+FORMATS = {"ternary": 0, "sign": 1}
 
 
 def _c(a, dtype):
@@ -151,6 +163,39 @@ def unpack_weights(trits, scales, rows, k, row0=0, nrows=None):
     return q, s
 
 
+# ---------------------------------------------------------------- 1-bit sign codes
+def sign_words(rows, k):
+    return int(lib().orc_sign_words(rows, k))
+
+
+def sign_word_index(k, r, b, w):
+    return int(lib().orc_sign_word_index(k, r, b, w))
+
+
+def quantize_weights_sign(w):
+    """w [rows][k] fp32 -> (codes uint32 [rows*(k/256)*8], scales uint16 [rows*(k/256)])."""
+    w = _c(w, np.float32)
+    rows, k = w.shape
+    codes = np.zeros(sign_words(rows, k), dtype=np.uint32)
+    scales = np.zeros(scale_count(rows, k), dtype=np.uint16)
+    if lib().orc_quantize_weights_sign(_ptr(w), rows, k, _ptr(codes), _ptr(scales)):
+        raise ValueError("orc_quantize_weights_sign: bad shape %r" % (w.shape,))
+    return codes, scales
+
+
+def unpack_weights_sign(codes, scales, rows, k, row0=0, nrows=None):
+    """-> (q int8 [nrows][k] in {-1, +1}, s float32 [nrows][k/256])."""
+    if nrows is None:
+        nrows = rows - row0
+    codes = _c(codes, np.uint32)
+    scales = _c(scales, np.uint16)
+    q = np.zeros((nrows, k), dtype=np.int8)
+    s = np.zeros((nrows, k // BLOCK), dtype=np.float32)
+    if lib().orc_unpack_weights_sign(_ptr(codes), _ptr(scales), rows, k, row0, nrows, _ptr(q), _ptr(s)):
+        raise ValueError("orc_unpack_weights_sign failed")
+    return q, s
+
+
 # ---------------------------------------------------------------- activations
 def quant_act_q8(x):
     """x [ntok][k] fp32 -> (xq int8 [ntok][k], xd fp32 [ntok][k/32])."""
@@ -219,33 +264,37 @@ def route_topk(x, wr, top_k):
 
 # ---------------------------------------------------------------- layer
 class Layer:
-    """A packed MoE layer in the storage format of orc_quantize_weights.
+    """A packed MoE layer in the storage format of orc_quantize_weights
+    (fmt "ternary") or orc_quantize_weights_sign (fmt "sign").
 
     gate/up: rows E*ffn, k hidden; down: rows E*hidden, k ffn.  Expert e owns
     rows [e*ffn, (e+1)*ffn) of gate/up and [e*hidden, (e+1)*hidden) of down.
     """
 
-    def __init__(self, hidden, ffn, n_experts, top_k, gate, up, down):
+    def __init__(self, hidden, ffn, n_experts, top_k, gate, up, down, fmt="ternary"):
         self.hidden, self.ffn, self.n_experts, self.top_k = hidden, ffn, n_experts, top_k
+        self.fmt = fmt
         self.gate = (_c(gate[0], np.uint32), _c(gate[1], np.uint16))
         self.up = (_c(up[0], np.uint32), _c(up[1], np.uint16))
         self.down = (_c(down[0], np.uint32), _c(down[1], np.uint16))
-        assert self.gate[0].size == trit_words(n_experts * ffn, hidden)
-        assert self.up[0].size == trit_words(n_experts * ffn, hidden)
-        assert self.down[0].size == trit_words(n_experts * hidden, ffn)
+        words = sign_words if fmt == "sign" else trit_words
+        assert self.gate[0].size == words(n_experts * ffn, hidden)
+        assert self.up[0].size == words(n_experts * ffn, hidden)
+        assert self.down[0].size == words(n_experts * hidden, ffn)
 
     @classmethod
-    def from_float(cls, hidden, ffn, n_experts, top_k, wg, wu, wd):
+    def from_float(cls, hidden, ffn, n_experts, top_k, wg, wu, wd, fmt="ternary"):
         """wg, wu [E*ffn][hidden], wd [E*hidden][ffn] fp32."""
-        return cls(hidden, ffn, n_experts, top_k,
-                   quantize_weights(wg), quantize_weights(wu), quantize_weights(wd))
+        quant = quantize_weights_sign if fmt == "sign" else quantize_weights
+        return cls(hidden, ffn, n_experts, top_k, quant(wg), quant(wu), quant(wd), fmt=fmt)
 
     def c_struct(self, top_k=None):
         return OrcLayer(self.hidden, self.ffn, self.n_experts,
                         self.top_k if top_k is None else top_k,
                         _ptr(self.gate[0]).value, _ptr(self.gate[1]).value,
                         _ptr(self.up[0]).value, _ptr(self.up[1]).value,
-                        _ptr(self.down[0]).value, _ptr(self.down[1]).value)
+                        _ptr(self.down[0]).value, _ptr(self.down[1]).value,
+                        FORMATS[self.fmt])
 
 
 def expert_ffn(layer, xq, xd, idx, wts, debug=False):

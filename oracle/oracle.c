@@ -188,6 +188,76 @@ int orc_unpack_weights(const uint32_t* trits, const uint16_t* scales,
 }
 
 /* ======================================================================== */
+/* 1-bit sign codes                                                          */
+/* ======================================================================== */
+/* The PXQ1 tier of the pxq_llama README ("What's PXQ?": 1-bit sign codes
+   times scales), read with this build's block and scale: per 256-weight
+   block s = fp16_RNE(sum|w| / 256) as for the ternary format (for codes of
+   +-1 this mean is also the scale of least squared error), q = -1 where
+   w < 0 and +1 otherwise.  Storage: 8 words per block, word j holding the
+   32 weights of activation block j, weight 32j + 4i + l in bit 8l + i (so
+   that the bits of four consecutive weights sit in the four bytes of a word
+   at the same position), a set bit meaning +1; words and scales interleaved
+   over 32-row panels exactly as the ternary words and scales.            */
+int64_t orc_sign_words(int64_t rows, int64_t k) {
+  return rows * (k / ORC_BLOCK) * ORC_SIGN_WORDS;
+}
+int64_t orc_sign_word_index(int64_t k, int64_t r, int64_t b, int w) {
+  int64_t nb = k / ORC_BLOCK;
+  int64_t p = r / ORC_PANEL;
+  return ((p * nb + b) * ORC_SIGN_WORDS + w) * ORC_PANEL + (r % ORC_PANEL);
+}
+
+int orc_quantize_weights_sign(const float* w, int64_t rows, int64_t k,
+                              uint32_t* codes, uint16_t* scales) {
+  if (rows <= 0 || k <= 0 || rows % ORC_PANEL || k % ORC_BLOCK) return -1;
+  int64_t nb = k / ORC_BLOCK;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* wb = w + r * k + b * ORC_BLOCK;
+      double sum = 0.0;
+      for (int kk = 0; kk < ORC_BLOCK; ++kk) sum += fabs((double)wb[kk]);
+      scales[orc_scale_index(k, r, b)] = orc_f16_from_f64(sum / 256.0);
+      for (int j = 0; j < ORC_SIGN_WORDS; ++j) {
+        uint32_t word = 0;
+        for (int i = 0; i < 8; ++i) {
+          for (int l = 0; l < 4; ++l) {
+            int kk = 32 * j + 4 * i + l;
+            if (!(wb[kk] < 0.0f)) word |= 1u << (8 * l + i);
+          }
+        }
+        codes[orc_sign_word_index(k, r, b, j)] = word;
+      }
+    }
+  }
+  return 0;
+}
+
+int orc_unpack_weights_sign(const uint32_t* codes, const uint16_t* scales,
+                            int64_t rows, int64_t k, int64_t row0,
+                            int64_t nrows, int8_t* q, float* s) {
+  if (rows <= 0 || k <= 0 || rows % ORC_PANEL || k % ORC_BLOCK) return -1;
+  if (row0 < 0 || nrows < 0 || row0 + nrows > rows) return -1;
+  int64_t nb = k / ORC_BLOCK;
+  for (int64_t rr = 0; rr < nrows; ++rr) {
+    int64_t r = row0 + rr;
+    for (int64_t b = 0; b < nb; ++b) {
+      if (s) s[rr * nb + b] = orc_f16_to_f32(scales[orc_scale_index(k, r, b)]);
+      for (int j = 0; j < ORC_SIGN_WORDS; ++j) {
+        uint32_t word = codes[orc_sign_word_index(k, r, b, j)];
+        for (int i = 0; i < 8; ++i) {
+          for (int l = 0; l < 4; ++l) {
+            int kk = 32 * j + 4 * i + l;
+            q[rr * k + b * ORC_BLOCK + kk] = (int8_t)(((word >> (8 * l + i)) & 1u) ? 1 : -1);
+          }
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+/* ======================================================================== */
 /* activation quantization                                                   */
 /* ======================================================================== */
 /* int8 activations with one fp32 scale per 32 values (Parakon Runtime README
@@ -355,6 +425,7 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
                    float* ad_out) {
   int64_t H = L->hidden, F = L->ffn, E = L->n_experts, K = L->top_k;
   if (H <= 0 || F <= 0 || E <= 0 || K < 1 || K > E) return -1;
+  if (L->format != ORC_FORMAT_TERNARY && L->format != ORC_FORMAT_SIGN) return -1;
   if (H % ORC_BLOCK || F % ORC_BLOCK || F % ORC_PANEL || H % ORC_PANEL) return -1;
   for (int64_t i = 0; i < ntok * K; ++i)
     if (idx[i] < 0 || idx[i] >= E) return -2;
@@ -378,9 +449,11 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
     int used = 0;
     for (int64_t i = 0; i < ntok * K; ++i) used |= (idx[i] == e);
     if (!used) continue;
-    if (orc_unpack_weights(L->gate_trits, L->gate_scales, E * F, H, e * F, F, qg, sg) ||
-        orc_unpack_weights(L->up_trits, L->up_scales, E * F, H, e * F, F, qu, su) ||
-        orc_unpack_weights(L->down_trits, L->down_scales, E * H, F, e * H, H, qd, sd)) {
+    int (*unpack)(const uint32_t*, const uint16_t*, int64_t, int64_t, int64_t, int64_t, int8_t*, float*) =
+        L->format == ORC_FORMAT_SIGN ? orc_unpack_weights_sign : orc_unpack_weights;
+    if (unpack(L->gate_trits, L->gate_scales, E * F, H, e * F, F, qg, sg) ||
+        unpack(L->up_trits, L->up_scales, E * F, H, e * F, F, qu, su) ||
+        unpack(L->down_trits, L->down_scales, E * H, F, e * H, H, qd, sd)) {
       rc = -1;
       break;
     }

@@ -75,6 +75,27 @@ int orc_unpack_weights(const uint32_t* trits, const uint16_t* scales,
                        int64_t rows, int64_t k, int64_t row0, int64_t nrows,
                        int8_t* q, float* s);
 
+/* ---- 1-bit sign codes -------------------------------------------------- */
+/* The 1-bit tier of the pxq_llama README ("What's PXQ?", the PXQ1 row: sign
+ * codes times scales).  Reading: the same 256-weight blocks, 32-row panels
+ * and fp16 absmean scale as the ternary format; q = -1 where w < 0, else +1;
+ * one bit per weight in ORC_SIGN_WORDS 32-bit words per block: word j holds
+ * weights 32j .. 32j+31, weight 32j + 4i + l in bit 8l + i, a set bit
+ * meaning +1.  34 bytes per block (1.0625 bits per weight).                */
+#define ORC_SIGN_WORDS 8
+int64_t orc_sign_words(int64_t rows, int64_t k);   /* rows*(k/256)*8 */
+/* Index of code word w (0..7) of block b of row r. */
+int64_t orc_sign_word_index(int64_t k, int64_t r, int64_t b, int w);
+/* Quantize w [rows][k] to sign codes; scales as orc_quantize_weights.
+ * Returns 0, or -1 when rows % 32 or k % 256 is nonzero.                  */
+int orc_quantize_weights_sign(const float* w, int64_t rows, int64_t k,
+                              uint32_t* codes, uint16_t* scales);
+/* Expand rows [row0, row0+nrows) to q [nrows][k] in {-1,+1} and the block
+ * scales s [nrows][k/256].  Returns 0, or -1 on a bad shape.              */
+int orc_unpack_weights_sign(const uint32_t* codes, const uint16_t* scales,
+                            int64_t rows, int64_t k, int64_t row0,
+                            int64_t nrows, int8_t* q, float* s);
+
 /* ---- activations ---------------------------------------------------------- */
 /* x [ntok][k] -> xq [ntok][k] int8, xd [ntok][k/32] fp32.  Returns -1 if
  * k % 32 != 0.                                                             */
@@ -106,7 +127,11 @@ typedef struct {
   const uint32_t* gate_trits; const uint16_t* gate_scales; /* rows E*ffn, k hidden */
   const uint32_t* up_trits;   const uint16_t* up_scales;   /* rows E*ffn, k hidden */
   const uint32_t* down_trits; const uint16_t* down_scales; /* rows E*hidden, k ffn */
+  int64_t format; /* ORC_FORMAT_TERNARY, or ORC_FORMAT_SIGN (the *_trits
+                     pointers then hold sign code words)                  */
 } orc_layer;
+#define ORC_FORMAT_TERNARY 0
+#define ORC_FORMAT_SIGN 1
 
 /* y [ntok][hidden] (fp64) = sum over slots j (in slot order) of
  * wts[t][j] * FFN_{idx[t][j]}(x_t).  Optional (may be NULL) debug outputs,

@@ -90,9 +90,11 @@ def _tiny(orc, H=256, F=512, E=4, K=2, seed=5, std=0.05):
     return (wg, wu, wd, wr, x)
 
 
-def _dense_mixture(orc, layer, wr, x):
+def _dense_mixture(orc, layer, wr, x, unpack=None):
     """Independent dense evaluation of a layer that routes to every expert:
-    y = sum_e softmax(logits)_e * Wd_e (q8(silu(Wg_e x^) * Wu_e x^))^."""
+    y = sum_e softmax(logits)_e * Wd_e (q8(silu(Wg_e x^) * Wu_e x^))^.
+    `unpack` expands a packed matrix (the ternary unpacking by default)."""
+    unpack = orc.unpack_weights if unpack is None else unpack
     H, F, E = layer.hidden, layer.ffn, layer.n_experts
     xq, xd = orc.quant_act_q8(x)
     lg = orc.router_logits(x, wr).astype(np.float64)
@@ -100,7 +102,7 @@ def _dense_mixture(orc, layer, wr, x):
     xdeq = xq.astype(np.float64) * np.repeat(xd.astype(np.float64), 32, axis=1)
 
     def deq(mat, rows, k, e):
-        q, s = orc.unpack_weights(mat[0], mat[1], E * rows, k, e * rows, rows)
+        q, s = unpack(mat[0], mat[1], E * rows, k, e * rows, rows)
         return q.astype(np.float64) * np.repeat(s.astype(np.float64), 256, axis=1)
 
     y = np.zeros((x.shape[0], H))
