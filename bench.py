@@ -41,7 +41,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="30b",
-                    help="tiny | 30b | 30b-b16 | large | large-b8 | 30b-prefill")
+                    help="tiny | 30b | 30b-b16 | large | large-b8 | 30b-prefill | 30b-sign | large-sign-b8")
     ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -68,9 +68,10 @@ def measured_peaks():
 
 
 # --------------------------------------------------------------------------- bytes
-def matrix_bytes(rows, k):
-    """Packed bytes of a ternary matrix: 52 B of digits + 2 B of scale per 256."""
-    return rows * (k // 256) * 54
+def matrix_bytes(rows, k, block_bytes=54):
+    """Packed bytes of a matrix: per 256 weights 52 B of base-3 digits (or 32 B
+    of sign bits) + 2 B of scale."""
+    return rows * (k // 256) * block_bytes
 
 
 def kernel_bytes(wl, unique_experts):
@@ -79,7 +80,8 @@ def kernel_bytes(wl, unique_experts):
     out)."""
     T, H, F, E, K = wl.ntok, wl.hidden, wl.ffn, wl.n_experts, wl.top_k
     pairs = T * K
-    weights = unique_experts * 3 * matrix_bytes(F, H)
+    bb = wl.block_bytes
+    weights = unique_experts * 3 * matrix_bytes(F, H, bb)
     return {
         # the whole one-token step in one kernel: router, x, the routed
         # experts' packed weights, the int8 intermediates and y
@@ -97,9 +99,9 @@ def kernel_bytes(wl, unique_experts):
         "router_quant": E * H * 4 + T * H * 4 + T * E * 4 + T * H + T * H // 32 * 4,
         "topk_group": T * E * 4 + pairs * 8 + pairs * 4 * 3,
         "group": pairs * 4 * 3,
-        "gateup": unique_experts * 2 * matrix_bytes(F, H) + T * H + T * H // 32 * 4
+        "gateup": unique_experts * 2 * matrix_bytes(F, H, bb) + T * H + T * H // 32 * 4
         + pairs * F + pairs * F // 32 * 4 + pairs * 8,
-        "down": unique_experts * matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4
+        "down": unique_experts * matrix_bytes(H, F, bb) + pairs * F + pairs * F // 32 * 4
         + pairs * H * 4 * 2 + T * H * 4 + pairs * 8,
     }
 
@@ -219,7 +221,7 @@ def run_reference(args):
     wg = np.concatenate([synthetic.expert_matrix(wl, 0, "gate", e).numpy() for e in experts])
     wu = np.concatenate([synthetic.expert_matrix(wl, 0, "up", e).numpy() for e in experts])
     wd = np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in experts])
-    layer = oracle.Layer.from_float(H, F, len(experts), 1, wg, wu, wd)
+    layer = oracle.Layer.from_float(H, F, len(experts), 1, wg, wu, wd, fmt=wl.fmt)
 
     def step(j):
         t, slot = (j // K) % n_tok, j % K
@@ -272,7 +274,9 @@ def job_rate(tokens_per_rank, world, ms):
 def workload_config(wl, layers):
     c = {"workload": wl.describe(), "hidden": wl.hidden, "expert_ffn": wl.ffn,
          "experts": wl.n_experts, "top_k": wl.top_k, "tokens_per_step": wl.ntok,
-         "weights": "ternary absmean 256-blocks (52 B base-3 + fp16 scale), N(0,%g)" % wl.w_std,
+         "weights": ("1-bit sign codes, 256-blocks (32 B of signs + fp16 absmean scale), N(0,%g)"
+                     if wl.fmt == "sign" else
+                     "ternary absmean 256-blocks (52 B base-3 + fp16 scale), N(0,%g)") % wl.w_std,
          "activations": "x ~ N(0,1) fp32, int8 32-blocks"}
     if layers is not None:
         c["layer_stack"] = layers
@@ -306,7 +310,8 @@ def cpu_baseline(wl, budget_s=12.0):
             H, F, len(e_used), K,
             np.concatenate([synthetic.expert_matrix(wl, 0, "gate", e).numpy() for e in e_used]),
             np.concatenate([synthetic.expert_matrix(wl, 0, "up", e).numpy() for e in e_used]),
-            np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in e_used]))
+            np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in e_used]),
+            fmt=wl.fmt)
         remap = np.full(wl.n_experts, -1, np.int32)
         remap[e_used] = np.arange(len(e_used))
         t0 = time.perf_counter()
@@ -355,7 +360,7 @@ def main():
     layers, routers = [], []
     for l in range(L):
         fn = lambda role, e, l=l: synthetic.expert_matrix(wl, seed_off + l, role, e, dev)  # noqa: E731
-        layers.append(quantize_layer(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, fn))
+        layers.append(quantize_layer(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, fn, fmt=wl.fmt))
         routers.append(synthetic.router(wl, seed_off + l, dev))
     NX = 64
     xs = [synthetic.activations(wl, seed_off + j, device=dev) for j in range(NX)]

@@ -29,11 +29,12 @@ STATUS = {
 
 # every symbol include/bitmoe.h declares
 EXPORTS = (
-    "moe_trit_words", "moe_scale_count", "moe_workspace_bytes", "moe_workspace_init",
-    "moe_quantize_weights", "moe_quant_act_q8", "moe_route_topk", "moe_route_workspace_bytes",
+    "moe_trit_words", "moe_sign_words", "moe_scale_count", "moe_workspace_bytes", "moe_workspace_init",
+    "moe_quantize_weights", "moe_quantize_weights_sign", "moe_quant_act_q8", "moe_route_topk", "moe_route_workspace_bytes",
     "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_forward", "moe_forward_host",
     "moe_check_status", "moe_last_error", "moe_debug_matvec", "moe_launch_count",
     "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
+    "moe_sign_words", "moe_quantize_weights_sign",
 )
 
 
@@ -45,7 +46,11 @@ class MoEError(RuntimeError):
 
 class moe_tmat(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("trits", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+                ("trits", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("format", ctypes.c_int32)]
+
+
+FORMATS = {"ternary": 0, "sign": 1}   # moe_format
 
 
 class moe_layer(ctypes.Structure):
@@ -68,10 +73,12 @@ def lib():
         p, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         sig = {
             "moe_trit_words": (sz, [i64, i64]),
+            "moe_sign_words": (sz, [i64, i64]),
             "moe_scale_count": (sz, [i64, i64]),
             "moe_workspace_bytes": (sz, [p, i32, i32]),
             "moe_workspace_init": (ctypes.c_int, [p, sz, p]),
             "moe_quantize_weights": (ctypes.c_int, [p, i64, i64, p, p, p]),
+            "moe_quantize_weights_sign": (ctypes.c_int, [p, i64, i64, p, p, p]),
             "moe_quant_act_q8": (ctypes.c_int, [p, i32, i32, p, p, p]),
             "moe_route_topk": (ctypes.c_int, [p, p, i32, i32, i32, i32, p, p, p, sz, p]),
             "moe_route_workspace_bytes": (sz, [i32, i32]),
@@ -121,25 +128,34 @@ def trit_words(rows, k):
     return int(lib().moe_trit_words(rows, k))
 
 
+def sign_words(rows, k):
+    return int(lib().moe_sign_words(rows, k))
+
+
+def packed_words(rows, k, fmt="ternary"):
+    return sign_words(rows, k) if fmt == "sign" else trit_words(rows, k)
+
+
 def scale_count(rows, k):
     return int(lib().moe_scale_count(rows, k))
 
 
 # ---------------------------------------------------------------- weights
 class TernaryMatrix:
-    """Packed ternary matrix: trits (int32 view of the uint32 words) and
-    scales (int16 view of the fp16 bits), in the storage format of bitmoe.h."""
+    """Packed matrix: trits (int32 view of the uint32 words: base-3 digits,
+    or 1-bit sign codes when fmt is "sign") and scales (int16 view of the fp16
+    bits), in the storage formats of bitmoe.h."""
 
-    def __init__(self, rows, k, trits, scales):
-        self.rows, self.k, self.trits, self.scales = rows, k, trits, scales
+    def __init__(self, rows, k, trits, scales, fmt="ternary"):
+        self.rows, self.k, self.trits, self.scales, self.fmt = rows, k, trits, scales, fmt
 
     @classmethod
-    def empty(cls, rows, k, device="cuda"):
-        return cls(rows, k, torch.empty(trit_words(rows, k), dtype=torch.int32, device=device),
-                   torch.empty(scale_count(rows, k), dtype=torch.int16, device=device))
+    def empty(cls, rows, k, device="cuda", fmt="ternary"):
+        return cls(rows, k, torch.empty(packed_words(rows, k, fmt), dtype=torch.int32, device=device),
+                   torch.empty(scale_count(rows, k), dtype=torch.int16, device=device), fmt)
 
     def c_struct(self):
-        return moe_tmat(self.rows, self.k, self.trits.data_ptr(), self.scales.data_ptr())
+        return moe_tmat(self.rows, self.k, self.trits.data_ptr(), self.scales.data_ptr(), FORMATS[self.fmt])
 
     @property
     def nbytes(self):
@@ -153,6 +169,16 @@ def moe_quantize_weights(w, out=None, stream=None):
     _check(lib().moe_quantize_weights(_dev(w, torch.float32, "w"), rows, k,
                                       ctypes.c_void_p(m.trits.data_ptr()),
                                       ctypes.c_void_p(m.scales.data_ptr()), _stream(stream)))
+    return m
+
+
+def moe_quantize_weights_sign(w, out=None, stream=None):
+    """w [rows][k] fp32 CUDA -> 1-bit sign-code TernaryMatrix (fmt "sign")."""
+    rows, k = w.shape
+    m = TernaryMatrix.empty(rows, k, w.device, fmt="sign") if out is None else out
+    _check(lib().moe_quantize_weights_sign(_dev(w, torch.float32, "w"), rows, k,
+                                           ctypes.c_void_p(m.trits.data_ptr()),
+                                           ctypes.c_void_p(m.scales.data_ptr()), _stream(stream)))
     return m
 
 

@@ -121,6 +121,10 @@ static int check_layer(const moe_layer* L) {
                 kMaxExperts, kMaxTopK);
   const moe_tmat* m[3] = {&L->gate, &L->up, &L->down};
   const char* names[3] = {"gate", "up", "down"};
+  if (L->gate.format != MOE_FORMAT_TERNARY && L->gate.format != MOE_FORMAT_SIGN)
+    return fail(MOE_ERR_INVALID_ARG, "unknown weight format %d", L->gate.format);
+  if (L->up.format != L->gate.format || L->down.format != L->gate.format)
+    return fail(MOE_ERR_INVALID_ARG, "gate, up and down must share one weight format");
   for (int i = 0; i < 3; ++i) {
     const int rows = i < 2 ? E * F : E * H, k = i < 2 ? H : F;
     if (m[i]->rows != rows || m[i]->k != k)
@@ -160,6 +164,7 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   P.cnt = reinterpret_cast<int32_t*>(base + W.cnt);
   P.status = &reinterpret_cast<WsHeader*>(ws)->status;
   P.direct = ntok == 1;
+  P.format = L->gate.format;
   P.items = reinterpret_cast<const Item*>(base + W.grp.items);
   P.n_items = reinterpret_cast<const int32_t*>(base + W.grp.n_items);
   P.pairs = reinterpret_cast<const int32_t*>(base + W.grp.pairs);
@@ -208,6 +213,8 @@ static int launch_decode(const DecodeParams& P, void* ws, const WsLayout& W, cud
     if (rc) return rc;
     return launch_ffn(P, stream);
   }
+  // sign codes: the grouped kernels in direct mode (item i = slot i)
+  if (P.format == MOE_FORMAT_SIGN) return launch_ffn(P, stream);
   Decode2Params D = make_d2(P, ws, W);
   return launch_decode2(D, false, stream);
 }
@@ -249,6 +256,11 @@ using namespace bitmoe;
 
 extern "C" {
 
+size_t moe_sign_words(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(k / kBlock) * kSignWords;
+}
+
 size_t moe_trit_words(int64_t rows, int64_t k) {
   if (rows <= 0 || k <= 0) return 0;
   return static_cast<size_t>(rows) * static_cast<size_t>(k / kBlock) * kBlockWords;
@@ -288,6 +300,17 @@ int moe_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trit
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quantize_weights: rows %% 32 and k %% 256 must be 0");
   if ((rc = check_device())) return rc;
   return launch_quantize_weights(w, rows, k, trits, scales, static_cast<cudaStream_t>(stream));
+}
+
+int moe_quantize_weights_sign(const float* w, int64_t rows, int64_t k, uint32_t* codes, uint16_t* scales,
+                              moe_stream_t stream) {
+  int rc = check_ptrs("quantize_weights_sign", w, codes, scales);
+  if (rc) return rc;
+  if (rows <= 0 || k <= 0) return fail(MOE_ERR_INVALID_ARG, "quantize_weights_sign: rows, k must be > 0");
+  if (rows % kPanel || k % kBlock)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quantize_weights_sign: rows %% 32 and k %% 256 must be 0");
+  if ((rc = check_device())) return rc;
+  return launch_quantize_weights(w, rows, k, codes, scales, static_cast<cudaStream_t>(stream), true);
 }
 
 int moe_quant_act_q8(const float* x, int32_t ntok, int32_t k, int8_t* xq, float* xd,
@@ -351,6 +374,8 @@ int moe_expert_ffn_prefill(const moe_layer* L, int32_t ntok, const int8_t* xq, c
                            moe_stream_t stream) {
   WsLayout W;
   int rc = ffn_common("expert_ffn_prefill", L, ntok, xq, xd, idx, wts, y, ws, ws_bytes, true, &W);
+  if (!rc && L->gate.format != MOE_FORMAT_TERNARY)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "expert_ffn_prefill: ternary layers only");
   if (rc) return rc;
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
   return launch_prefill(P, static_cast<cudaStream_t>(stream));
@@ -363,6 +388,9 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   if ((rc = check_ptrs("forward", w_router, x, y, ws))) return rc;
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
+  const bool sign = L->gate.format == MOE_FORMAT_SIGN;
+  if (sign && prefill)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: sign-code layers take at most %d tokens", kMaxDecodeTokens);
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total) return fail(MOE_ERR_WORKSPACE, "forward: workspace %zu < %zu bytes", ws_bytes, W.total);
   if ((rc = check_device())) return rc;
@@ -374,15 +402,16 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   float* wts = reinterpret_cast<float*>(base + W.wts);
   float* logits = reinterpret_cast<float*>(base + W.logits);
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
-  if (ntok > 1 && !prefill && router_quant_small_ok(ntok, L->hidden)) {
-    // few tokens: router logits with the activation quantization, then the
-    // top-k with the grouping, then the grouped mat-vecs
+  if ((ntok > 1 || sign) && !prefill && router_quant_small_ok(ntok, L->hidden)) {
+    // few tokens (and one token of a sign-code layer): router logits with
+    // the activation quantization, then the top-k with the grouping, then
+    // the grouped mat-vecs
     if ((rc = launch_router_quant_small(x, w_router, ntok, L->hidden, L->n_experts, logits, xq, xd, s)))
       return rc;
     if ((rc = launch_topk_group(P, logits, wts, s))) return rc;
     return launch_ffn(P, s);
   }
-  if (ntok > 1) {
+  if (ntok > 1 || sign) {
     if ((rc = launch_quant_act_q8(x, ntok, L->hidden, xq, xd, s))) return rc;
     if ((rc = launch_route_topk(x, w_router, ntok, L->hidden, L->n_experts, L->top_k, idx, wts, logits, s)))
       return rc;
@@ -495,6 +524,8 @@ int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const fl
     return fail(MOE_ERR_INVALID_ARG, "debug_matvec: bad sizes");
   if (m->rows % kPanel || m->k % kBlock || m->k > kMaxHidden)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "debug_matvec: rows %% 32, k %% 256, k <= %d", kMaxHidden);
+  if (m->format != MOE_FORMAT_TERNARY && m->format != MOE_FORMAT_SIGN)
+    return fail(MOE_ERR_INVALID_ARG, "debug_matvec: unknown weight format %d", m->format);
   if ((rc = check_device())) return rc;
   return launch_debug_matvec(m, ntok, xq, xd, out, isum, static_cast<cudaStream_t>(stream));
 }

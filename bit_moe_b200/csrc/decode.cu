@@ -160,9 +160,10 @@ __device__ __forceinline__ int item_pair(const DecodeParams& P, const Item& item
 // n's 32 rows and requantizes them (one 32-block of a) to int8.
 // grid: (ffn/32, items), block: kGateUpWarps*32.
 // ---------------------------------------------------------------------------
-template <int NT>
+template <int NT, bool kSign>
 __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& item, int panel,
                                            unsigned char* smem) {
+  constexpr int kWords = WordsPerBlock<kSign>::value;
   const int H = P.hidden, F = P.ffn;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int* q4 = reinterpret_cast<int*>(smem);
@@ -181,15 +182,15 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
   __syncthreads();
   const int nb = H / kBlock;
   const size_t pb0 = (static_cast<size_t>(item.expert) * (F / kPanel) + panel) * nb;
-  const uint32_t* const tw[2] = {P.gate_trits + pb0 * kBlockWords * kPanel + lane,
-                                 P.up_trits + pb0 * kBlockWords * kPanel + lane};
+  const uint32_t* const tw[2] = {P.gate_trits + pb0 * kWords * kPanel + lane,
+                                 P.up_trits + pb0 * kWords * kPanel + lane};
   const uint16_t* const ts[2] = {P.gate_scales + pb0 * kPanel + lane, P.up_scales + pb0 * kPanel + lane};
   float out[2][NT];
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
     for (int n = 0; n < NT; ++n) out[m][n] = 0.f;
-  panel_dot<2, NT>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, out);
+  panel_dot<2, NT, kSign>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, out);
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -216,7 +217,7 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
 // Four CTAs per SM (at most 64 registers a thread): the items of a decode
 // batch are mostly single pairs, whose path needs few registers; the rare
 // 8-pair path spills a little.
-template <int NTMAX>
+template <int NTMAX, bool kSign>
 __global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
@@ -234,12 +235,12 @@ __global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P)
     return;
   }
   if constexpr (NTMAX == 1) {
-    gateup_run<1>(P, item, panel, smem);
+    gateup_run<1, kSign>(P, item, panel, smem);
   } else {
-    if (item.count <= 1) gateup_run<1>(P, item, panel, smem);
-    else if (item.count <= 2) gateup_run<2>(P, item, panel, smem);
-    else if (item.count <= 4) gateup_run<4>(P, item, panel, smem);
-    else gateup_run<8>(P, item, panel, smem);
+    if (item.count <= 1) gateup_run<1, kSign>(P, item, panel, smem);
+    else if (item.count <= 2) gateup_run<2, kSign>(P, item, panel, smem);
+    else if (item.count <= 4) gateup_run<4, kSign>(P, item, panel, smem);
+    else gateup_run<8, kSign>(P, item, panel, smem);
   }
 }
 
@@ -269,9 +270,10 @@ __device__ __forceinline__ void arrive_and_combine(const DecodeParams& P, int pa
   }
 }
 
-template <int NT>
+template <int NT, bool kSign>
 __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item, int pgroup,
                                          unsigned char* smem) {
+  constexpr int kWords = WordsPerBlock<kSign>::value;
   const int H = P.hidden, F = P.ffn;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int* q4 = reinterpret_cast<int*>(smem);
@@ -290,12 +292,12 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
   const int panel = pgroup * kDownWarps + warp;
   const int nb = F / kBlock;
   const size_t pb0 = (static_cast<size_t>(item.expert) * (H / kPanel) + panel) * nb;
-  const uint32_t* const tw[1] = {P.down_trits + pb0 * kBlockWords * kPanel + lane};
+  const uint32_t* const tw[1] = {P.down_trits + pb0 * kWords * kPanel + lane};
   const uint16_t* const ts[1] = {P.down_scales + pb0 * kPanel + lane};
   float out[1][NT];
 #pragma unroll
   for (int n = 0; n < NT; ++n) out[0][n] = 0.f;
-  panel_dot<1, NT>(tw, ts, 0, nb, 1, q4, d, as, out);
+  panel_dot<1, NT, kSign>(tw, ts, 0, nb, 1, q4, d, as, out);
 #pragma unroll
   for (int n = 0; n < NT; ++n)
     if (n < item.count)
@@ -307,7 +309,7 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
 
 // Eight CTAs per SM (at most 64 registers a thread, which leaves room for the
 // prefetched next block of weight words in panel_dot).
-template <int NTMAX>
+template <int NTMAX, bool kSign>
 __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
@@ -325,12 +327,12 @@ __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
     return;
   }
   if constexpr (NTMAX == 1) {
-    down_run<1>(P, item, pgroup, smem);
+    down_run<1, kSign>(P, item, pgroup, smem);
   } else {
-    if (item.count <= 1) down_run<1>(P, item, pgroup, smem);
-    else if (item.count <= 2) down_run<2>(P, item, pgroup, smem);
-    else if (item.count <= 4) down_run<4>(P, item, pgroup, smem);
-    else down_run<8>(P, item, pgroup, smem);
+    if (item.count <= 1) down_run<1, kSign>(P, item, pgroup, smem);
+    else if (item.count <= 2) down_run<2, kSign>(P, item, pgroup, smem);
+    else if (item.count <= 4) down_run<4, kSign>(P, item, pgroup, smem);
+    else down_run<8, kSign>(P, item, pgroup, smem);
   }
 }
 
@@ -338,6 +340,7 @@ __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
 // Test hook: the mat-vec core on one matrix, with the exact block sums.
 // grid: (rows/32, ntok), block: kGateUpWarps*32; warps split the blocks.
 // ---------------------------------------------------------------------------
+template <bool kSign>
 __global__ void __launch_bounds__(kGateUpWarps * 32)
     k_debug_matvec(const uint32_t* __restrict__ trits, const uint16_t* __restrict__ scales, int rows,
                    int k, const int8_t* __restrict__ xq, const float* __restrict__ xd,
@@ -355,11 +358,11 @@ __global__ void __launch_bounds__(kGateUpWarps * 32)
   const int nb = k / kBlock;
   const int r = panel * kPanel + lane;
   const size_t pb0 = static_cast<size_t>(panel) * nb;
-  const uint32_t* const tw[1] = {trits + pb0 * kBlockWords * kPanel + lane};
+  const uint32_t* const tw[1] = {trits + pb0 * WordsPerBlock<kSign>::value * kPanel + lane};
   const uint16_t* const ts[1] = {scales + pb0 * kPanel + lane};
   float o[1][1] = {{0.f}};
   int32_t* isum_row = isum ? isum + (static_cast<size_t>(t) * rows + r) * (k / kQBlock) : nullptr;
-  panel_dot<1, 1>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, o, isum_row, 0);
+  panel_dot<1, 1, kSign>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, o, isum_row, 0);
   red[warp * 32 + lane] = o[0][0];
   __syncthreads();
   if (warp == 0) {
@@ -381,11 +384,16 @@ static void init_kernel_attrs() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < kMaxDev && done[dev]) return;
-  const void* kernels[] = {reinterpret_cast<const void*>(&k_gateup<1>),
-                           reinterpret_cast<const void*>(&k_gateup<kChunk>),
-                           reinterpret_cast<const void*>(&k_down<1>),
-                           reinterpret_cast<const void*>(&k_down<kChunk>),
-                           reinterpret_cast<const void*>(&k_debug_matvec)};
+  const void* kernels[] = {reinterpret_cast<const void*>(&k_gateup<1, false>),
+                           reinterpret_cast<const void*>(&k_gateup<kChunk, false>),
+                           reinterpret_cast<const void*>(&k_down<1, false>),
+                           reinterpret_cast<const void*>(&k_down<kChunk, false>),
+                           reinterpret_cast<const void*>(&k_gateup<1, true>),
+                           reinterpret_cast<const void*>(&k_gateup<kChunk, true>),
+                           reinterpret_cast<const void*>(&k_down<1, true>),
+                           reinterpret_cast<const void*>(&k_down<kChunk, true>),
+                           reinterpret_cast<const void*>(&k_debug_matvec<false>),
+                           reinterpret_cast<const void*>(&k_debug_matvec<true>)};
   for (const void* k : kernels)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
   if (dev >= 0 && dev < kMaxDev) done[dev] = true;
@@ -407,25 +415,32 @@ int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cu
   return check_launch("topk_group");
 }
 
-int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
-  if (!P.direct && P.group_chunk != kChunk) return fail(MOE_ERR_INVALID_ARG, "expert_ffn: items of %d pairs", P.group_chunk);
-  init_kernel_attrs();
+template <bool kSign>
+static void launch_ffn_fmt(const DecodeParams& P, cudaStream_t stream) {
   const int npairs = P.ntok * P.top_k;
   if (P.direct) {
     const size_t s1 = ActSmem<1>::bytes(P.hidden) + 2 * kGateUpWarps * 1 * 32 * 4;
     const size_t s2 = ActSmem<1>::bytes(P.ffn);
-    launch_k(k_gateup<1>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
+    launch_k(k_gateup<1, kSign>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
     note_launch(MOE_K_GATEUP, stream);
-    launch_k(k_down<1>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
+    launch_k(k_down<1, kSign>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
     note_launch(MOE_K_DOWN, stream);
   } else {
     const size_t s1 = ActSmem<kChunk>::bytes(P.hidden) + 2 * kGateUpWarps * kChunk * 32 * 4;
     const size_t s2 = ActSmem<kChunk>::bytes(P.ffn);
-    launch_k(k_gateup<kChunk>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
+    launch_k(k_gateup<kChunk, kSign>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
     note_launch(MOE_K_GATEUP, stream);
-    launch_k(k_down<kChunk>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
+    launch_k(k_down<kChunk, kSign>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream,
+             P);
     note_launch(MOE_K_DOWN, stream);
   }
+}
+
+int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
+  if (!P.direct && P.group_chunk != kChunk) return fail(MOE_ERR_INVALID_ARG, "expert_ffn: items of %d pairs", P.group_chunk);
+  init_kernel_attrs();
+  if (P.format == MOE_FORMAT_SIGN) launch_ffn_fmt<true>(P, stream);
+  else launch_ffn_fmt<false>(P, stream);
   return check_launch("expert_ffn");
 }
 
@@ -433,8 +448,11 @@ int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const flo
                         int32_t* isum, cudaStream_t stream) {
   init_kernel_attrs();
   const size_t s = ActSmem<1>::bytes(m->k) + kGateUpWarps * 32 * 4;
-  k_debug_matvec<<<dim3(m->rows / kPanel, ntok), kGateUpWarps * 32, s, stream>>>(
-      m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
+  const dim3 grid(m->rows / kPanel, ntok);
+  if (m->format == MOE_FORMAT_SIGN)
+    k_debug_matvec<true><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
+  else
+    k_debug_matvec<false><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
   note_launch(MOE_K_DEBUG_MATVEC, stream);
   return check_launch("debug_matvec");
 }

@@ -31,6 +31,7 @@ struct DecodeParams {
   int32_t* status;
   // grouped mode (ntok > 1): items and the pair list, built on the device
   int direct;                            // 1: item i is pair i (ntok == 1)
+  int format;                            // MOE_FORMAT_TERNARY or MOE_FORMAT_SIGN
   const Item* items;                     // [ntok*top_k + n_experts]
   const int32_t* n_items;
   const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert

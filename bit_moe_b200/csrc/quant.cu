@@ -18,7 +18,11 @@ constexpr int kTileStride = kBlock + 1;  // padded row of the staged tile
 // 13 words of each row are written 128 contiguous bytes per warp store.
 // Every lane does the same sequence of operations for its block whatever the
 // grid, so the output does not depend on the launch configuration.
+// With kSign the same scale is kept and the codes are 1-bit signs (pxq_llama
+// README, "What's PXQ?": the PXQ1 tier): q = -1 where w < 0, else +1, bit
+// 8l + i of word j set for q = +1 at weight 32j + 4i + l.
 // ---------------------------------------------------------------------------
+template <bool kSign>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     k_quantize_weights(const float* __restrict__ w, int64_t n_items, int k,
                        uint32_t* __restrict__ trits, uint16_t* __restrict__ scales) {
@@ -47,26 +51,39 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     const uint16_t s = f64_to_f16_rn(sum * (1.0 / 256.0));
     const float half = 0.5f * f16_bits_to_f32(s);
     scales[item * kPanel + lane] = s;
+    if constexpr (kSign) {
 #pragma unroll 1
-    for (int j = 0; j < kBlockWords; ++j) {
-      uint32_t word = 0;
+      for (int j = 0; j < kSignWords; ++j) {
+        uint32_t word = 0;
 #pragma unroll
-      for (int l = 0; l < 4; ++l) {
-        int v = 0;
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int i = 0; i < 5; ++i) {
-          const int kk = 20 * j + 4 * i + l;
-          int t = 1;  // pad digit: weight 0
-          if (kk < kBlock) {
-            const float x = row[kk];
-            if (fabsf(x) >= half && x != 0.f) t = x > 0.f ? 2 : 0;
-          }
-          v = 3 * v + t;
-        }
-        const uint32_t u = static_cast<uint32_t>((v * 256 + 242) / 243);
-        word |= u << (8 * l);
+          for (int l = 0; l < 4; ++l)
+            if (!(row[32 * j + 4 * i + l] < 0.f)) word |= 1u << (8 * l + i);
+        trits[(item * kSignWords + j) * kPanel + lane] = word;
       }
-      trits[(item * kBlockWords + j) * kPanel + lane] = word;
+    } else {
+#pragma unroll 1
+      for (int j = 0; j < kBlockWords; ++j) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+          int v = 0;
+#pragma unroll
+          for (int i = 0; i < 5; ++i) {
+            const int kk = 20 * j + 4 * i + l;
+            int t = 1;  // pad digit: weight 0
+            if (kk < kBlock) {
+              const float x = row[kk];
+              if (fabsf(x) >= half && x != 0.f) t = x > 0.f ? 2 : 0;
+            }
+            v = 3 * v + t;
+          }
+          const uint32_t u = static_cast<uint32_t>((v * 256 + 242) / 243);
+          word |= u << (8 * l);
+        }
+        trits[(item * kBlockWords + j) * kPanel + lane] = word;
+      }
     }
     __syncwarp();
   }
@@ -88,14 +105,14 @@ __global__ void k_quant_act_q8(const float* __restrict__ x, int64_t nblk, int8_t
 }
 
 int launch_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,
-                            uint16_t* scales, cudaStream_t stream) {
+                            uint16_t* scales, cudaStream_t stream, bool sign) {
   const size_t smem = static_cast<size_t>(kQuantWarps) * kPanel * kTileStride * sizeof(float);
-  cudaFuncSetAttribute(k_quantize_weights, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(smem));
+  auto kern = sign ? k_quantize_weights<true> : k_quantize_weights<false>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   const int64_t n_items = rows / kPanel * (k / kBlock);
   int64_t grid = (n_items + kQuantWarps - 1) / kQuantWarps;
   if (grid > 148 * 16) grid = 148 * 16;
-  k_quantize_weights<<<static_cast<unsigned>(grid), kQuantWarps * 32, smem, stream>>>(
+  kern<<<static_cast<unsigned>(grid), kQuantWarps * 32, smem, stream>>>(
       w, n_items, static_cast<int>(k), trits, scales);
   note_launch(MOE_K_QUANTIZE_WEIGHTS, stream);
   return check_launch("quantize_weights");

@@ -2,8 +2,9 @@
 #pragma once
 #include "common.cuh"
 namespace bitmoe {
+// sign: 1-bit sign codes (MOE_FORMAT_SIGN) instead of ternary digits.
 int launch_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,
-                            uint16_t* scales, cudaStream_t stream);
+                            uint16_t* scales, cudaStream_t stream, bool sign = false);
 int launch_quant_act_q8(const float* x, int64_t ntok, int k, int8_t* xq, float* xd,
                         cudaStream_t stream);
 

@@ -26,6 +26,13 @@
 // accumulated in fp32 (sub-blocks in order), and the fp16 weight scale is
 // applied once per 256-block.
 //
+// 1-bit sign codes (kSign; pxq_llama README, "What's PXQ?": the PXQ1 tier of
+// sign codes times scales): 8 words per block, word j covering activation
+// block j, weight 32j + 4i + l in bit 8l + i.  For group i of a word the
+// digit word t = (w >> i) & 0x01010101 holds the bits of weights 4i..4i+3 in
+// its four bytes, dp4a gives sum t*a, and with q = 2t - 1 the block sum is
+// sum q*a = 2 * sum t*a - sum a.
+//
 // Shared-memory activation layout for NT vectors over a k-long dimension:
 //   q4  [k/4][NT]  int32, four int8 codes each (token-minor, so the NT words
 //                  of one group load as NT/4 128-bit broadcasts)
@@ -69,50 +76,56 @@ __device__ __forceinline__ void load_group(const int* __restrict__ q4, int g, in
 //   ts[m]: scales of matrix m at (panel, block 0), offset by lane
 // If isum_out is not null (NM == 1), the exact block sums of the lane's row
 // are stored at isum_out[n * isum_stride + s] for every global sub-block s.
-template <int NM, int NT>
+template <int kSign>
+struct WordsPerBlock {
+  static constexpr int value = kSign ? kSignWords : kBlockWords;
+};
+
+template <int NM, int NT, bool kSign = false>
 __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
                                           const uint16_t* const (&ts)[NM], int b_begin, int b_end,
                                           int b_step, const int* __restrict__ q4,
                                           const float* __restrict__ d,
                                           const int* __restrict__ as, float (&out)[NM][NT],
                                           int32_t* isum_out = nullptr, size_t isum_stride = 0) {
+  constexpr int kWords = WordsPerBlock<kSign>::value;
   // one matrix: the next block's words are loaded while this one decodes
-  uint32_t wn[NM][kBlockWords];
+  uint32_t wn[NM][WordsPerBlock<kSign>::value];
   uint16_t sn[NM];
   if (NM == 1 && b_begin < b_end) {
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
-      const uint32_t* src = tw[m] + static_cast<size_t>(b_begin) * kBlockWords * kPanel;
+      const uint32_t* src = tw[m] + static_cast<size_t>(b_begin) * kWords * kPanel;
 #pragma unroll
-      for (int j = 0; j < kBlockWords; ++j) wn[m][j] = ld_stream_u32(src + j * kPanel);
+      for (int j = 0; j < kWords; ++j) wn[m][j] = ld_stream_u32(src + j * kPanel);
       sn[m] = ts[m][static_cast<size_t>(b_begin) * kPanel];
     }
   }
   for (int b = b_begin; b < b_end; b += b_step) {
-    uint32_t w[NM][kBlockWords];
+    uint32_t w[NM][WordsPerBlock<kSign>::value];
     float sc[NM];
     if constexpr (NM == 1) {
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
 #pragma unroll
-        for (int j = 0; j < kBlockWords; ++j) w[m][j] = wn[m][j];
+        for (int j = 0; j < kWords; ++j) w[m][j] = wn[m][j];
         sc[m] = f16_bits_to_f32(sn[m]);
       }
       if (b + b_step < b_end) {
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-          const uint32_t* src = tw[m] + static_cast<size_t>(b + b_step) * kBlockWords * kPanel;
+          const uint32_t* src = tw[m] + static_cast<size_t>(b + b_step) * kWords * kPanel;
 #pragma unroll
-          for (int j = 0; j < kBlockWords; ++j) wn[m][j] = ld_stream_u32(src + j * kPanel);
+          for (int j = 0; j < kWords; ++j) wn[m][j] = ld_stream_u32(src + j * kPanel);
           sn[m] = ts[m][static_cast<size_t>(b + b_step) * kPanel];
         }
       }
     } else {
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
-        const uint32_t* src = tw[m] + static_cast<size_t>(b) * kBlockWords * kPanel;
+        const uint32_t* src = tw[m] + static_cast<size_t>(b) * kWords * kPanel;
 #pragma unroll
-        for (int j = 0; j < kBlockWords; ++j) w[m][j] = ld_stream_u32(src + j * kPanel);
+        for (int j = 0; j < kWords; ++j) w[m][j] = ld_stream_u32(src + j * kPanel);
         sc[m] = f16_bits_to_f32(ts[m][static_cast<size_t>(b) * kPanel]);
       }
     }
@@ -123,43 +136,73 @@ __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
 #pragma unroll
       for (int n = 0; n < NT; ++n) { acc[m][n] = 0; inner[m][n] = 0.f; }
     const int* qb = q4 + b * (kBlock / 4) * NT;
+    if constexpr (kSign) {
 #pragma unroll
-    for (int j = 0; j < kBlockWords; ++j) {
-      uint32_t lo[NM], hi[NM], hp[NM];
+      for (int j = 0; j < kSignWords; ++j) {  // word j = activation block j of the block
 #pragma unroll
-      for (int m = 0; m < NM; ++m) {
-        lo[m] = w[m][j] & 0x00FF00FFu;
-        hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
-        hp[m] = 0u;
+        for (int i = 0; i < 8; ++i) {
+          int a[NT];
+          load_group<NT>(qb, 8 * j + i, a);
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+            const int t = static_cast<int>((w[m][j] >> i) & 0x01010101u);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) acc[m][n] = __dp4a(t, a[n], acc[m][n]);
+          }
+        }
+        const int s = b * kSubPerBlock + j;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const float dn = d[s * NT + n];
+          const int an = as[s * NT + n];
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+            const int isum = 2 * acc[m][n] - an;
+            inner[m][n] = __fmaf_rn(dn, static_cast<float>(isum), inner[m][n]);
+            acc[m][n] = 0;
+            if (NM == 1 && isum_out) isum_out[n * isum_stride + s] = isum;
+          }
+        }
       }
+    } else {
 #pragma unroll
-      for (int i = 0; i < 5; ++i) {
-        if (j == kBlockWords - 1 && i == 4) break;  // pad digit of the last word
-        const int g = 5 * j + i;                    // group of 4 weights, 0..63
-        int a[NT];
-        load_group<NT>(qb, g, a);
+      for (int j = 0; j < kBlockWords; ++j) {
+        uint32_t lo[NM], hi[NM], hp[NM];
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-          lo[m] *= 3u;
-          hi[m] *= 3u;
-          const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
-          const int t = static_cast<int>(hn - 3u * hp[m]);
-          hp[m] = hn;
-#pragma unroll
-          for (int n = 0; n < NT; ++n) acc[m][n] = __dp4a(t, a[n], acc[m][n]);
+          lo[m] = w[m][j] & 0x00FF00FFu;
+          hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
+          hp[m] = 0u;
         }
-        if ((g & 7) == 7) {  // a 32-weight sub-block is complete
-          const int s = b * kSubPerBlock + (g >> 3);
 #pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const float dn = d[s * NT + n];
-            const int an = as[s * NT + n];
+        for (int i = 0; i < 5; ++i) {
+          if (j == kBlockWords - 1 && i == 4) break;  // pad digit of the last word
+          const int g = 5 * j + i;                    // group of 4 weights, 0..63
+          int a[NT];
+          load_group<NT>(qb, g, a);
 #pragma unroll
-            for (int m = 0; m < NM; ++m) {
-              const int isum = acc[m][n] - an;
-              inner[m][n] = __fmaf_rn(dn, static_cast<float>(isum), inner[m][n]);
-              acc[m][n] = 0;
-              if (NM == 1 && isum_out) isum_out[n * isum_stride + s] = isum;
+          for (int m = 0; m < NM; ++m) {
+            lo[m] *= 3u;
+            hi[m] *= 3u;
+            const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
+            const int t = static_cast<int>(hn - 3u * hp[m]);
+            hp[m] = hn;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) acc[m][n] = __dp4a(t, a[n], acc[m][n]);
+          }
+          if ((g & 7) == 7) {  // a 32-weight sub-block is complete
+            const int s = b * kSubPerBlock + (g >> 3);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              const float dn = d[s * NT + n];
+              const int an = as[s * NT + n];
+#pragma unroll
+              for (int m = 0; m < NM; ++m) {
+                const int isum = acc[m][n] - an;
+                inner[m][n] = __fmaf_rn(dn, static_cast<float>(isum), inner[m][n]);
+                acc[m][n] = 0;
+                if (NM == 1 && isum_out) isum_out[n * isum_stride + s] = isum;
+              }
             }
           }
         }

@@ -40,6 +40,15 @@
  *     scales[(r/32 * nb + b) * 32 + r%32].
  * That is 52 bytes of digits plus a 2-byte scale per 256 weights (1.6875
  * bits per weight).
+ *
+ * Storage format of a 1-bit sign-code matrix (MOE_FORMAT_SIGN; the 1-bit
+ * tier of the pxq_llama README, "What's PXQ?": sign codes times scales).
+ * The same blocks, fp16 absmean scales and 32-row panels; q = -1 where
+ * w < 0, else +1; 8 uint32 words per block, word j holding weights
+ * 32j .. 32j+31 of the block, weight 32j + 4i + l in bit 8l + i (i = 0..7,
+ * l = 0..3), a set bit meaning +1; word j of block b of row r is
+ * codes[((r/32 * nb + b) * 8 + j) * 32 + r%32].  34 bytes per 256 weights
+ * (1.0625 bits per weight).
  */
 #ifndef BITMOE_H
 #define BITMOE_H
@@ -65,18 +74,27 @@ typedef enum {
   MOE_ERR_DEVICE = -8             /* the current device is not sm_100           */
 } moe_status;
 
-/* One ternary matrix in the storage format above. */
+/* Weight formats. */
+typedef enum { MOE_FORMAT_TERNARY = 0, MOE_FORMAT_SIGN = 1 } moe_format;
+
+/* One packed matrix in one of the storage formats above. */
 typedef struct {
   int32_t rows;          /* multiple of 32                          */
   int32_t k;             /* multiple of 256                         */
-  const uint32_t* trits; /* moe_trit_words(rows, k) words, device   */
+  const uint32_t* trits; /* the packed words, device: moe_trit_words(rows, k)
+                            base-3 words, or moe_sign_words(rows, k) sign
+                            words for MOE_FORMAT_SIGN                */
   const uint16_t* scales;/* moe_scale_count(rows, k) fp16, device   */
+  int32_t format;        /* a moe_format                             */
 } moe_tmat;
 
 /* One MoE layer.  Expert e owns rows [e*ffn, (e+1)*ffn) of gate and up
- * (k = hidden) and rows [e*hidden, (e+1)*hidden) of down (k = ffn).
- * Limits: hidden and ffn multiples of 256, hidden <= 16384, ffn <= 8192,
- * 1 <= top_k <= min(n_experts, 32), n_experts <= 1024.                      */
+ * (k = hidden) and rows [e*hidden, (e+1)*hidden) of down (k = ffn).  The
+ * three matrices share one format.  Limits: hidden and ffn multiples of 256,
+ * hidden <= 16384, ffn <= 8192, 1 <= top_k <= min(n_experts, 32),
+ * n_experts <= 1024.  Sign-code layers run the decode path only: up to 64
+ * tokens per call (moe_expert_ffn_prefill, and moe_forward of more than 64
+ * tokens, return MOE_ERR_UNSUPPORTED_SHAPE for them).                      */
 typedef struct {
   int32_t hidden, ffn, n_experts, top_k;
   moe_tmat gate, up, down;
@@ -84,6 +102,7 @@ typedef struct {
 
 /* ---- sizes ------------------------------------------------------------ */
 size_t moe_trit_words(int64_t rows, int64_t k);  /* rows*(k/256)*13 */
+size_t moe_sign_words(int64_t rows, int64_t k);  /* rows*(k/256)*8  */
 size_t moe_scale_count(int64_t rows, int64_t k); /* rows*(k/256)    */
 /* Bytes of workspace a decode (prefill = 0) or prefill (prefill = 1) call
  * of `ntok` tokens, or moe_forward, needs.  0 on invalid arguments.        */
@@ -100,6 +119,10 @@ int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);
  * bytes do not depend on the launch configuration.                        */
 int moe_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,
                          uint16_t* scales, moe_stream_t stream);
+/* The same to 1-bit sign codes (MOE_FORMAT_SIGN): the same scales; q = -1
+ * where w < 0, else +1 (see the storage format above).                    */
+int moe_quantize_weights_sign(const float* w, int64_t rows, int64_t k, uint32_t* codes,
+                              uint16_t* scales, moe_stream_t stream);
 
 /* ---- S1: activation quantization (Parakon Runtime README, "How it works":
  *      int8-quantized activations; pxq_llama README, "PXQ vs MXFP4": one

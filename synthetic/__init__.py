@@ -38,17 +38,25 @@ class Workload:
     layers: int = 1          # layers in the stack the benchmark rotates through
     prefill: bool = False
     seed: int = 0
+    fmt: str = "ternary"     # packed weight format: "ternary" or "sign" (1-bit sign codes)
 
     def with_(self, **kw):
         return replace(self, **kw)
 
     @property
+    def block_bytes(self):
+        """Packed bytes per 256 weights: 52 B of base-3 digits or 32 B of sign
+        bits, plus the 2-byte scale."""
+        return 34 if self.fmt == "sign" else 54
+
+    @property
     def expert_bytes(self):
-        """Packed bytes of one expert's gate+up+down (54 B per 256 weights)."""
-        return 3 * self.hidden * self.ffn // 256 * 54
+        """Packed bytes of one expert's gate+up+down."""
+        return 3 * self.hidden * self.ffn // 256 * self.block_bytes
 
     def describe(self):
-        return "%s-t%d%s" % (self.name, self.ntok, "-prefill" if self.prefill else "")
+        return "%s%s-t%d%s" % (self.name, "-sign" if self.fmt == "sign" else "", self.ntok,
+                               "-prefill" if self.prefill else "")
 
 
 WORKLOADS = {
@@ -61,6 +69,11 @@ WORKLOADS = {
     # large layer, decode of 1 token (and 8 with ntok=8), 5-layer stack
     "large": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 1, 0.015, layers=5, seed=3),
     "large-b8": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 8, 0.015, layers=5, seed=3),
+    # the same layers with 1-bit sign codes instead of ternary digits
+    "30b-sign": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 1, 0.02, layers=4, seed=5,
+                         fmt="sign"),
+    "large-sign-b8": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 8, 0.015, layers=5,
+                              seed=6, fmt="sign"),
     # prefill of 2048 tokens through the 30B-class layer
     "30b-prefill": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 2048, 0.02,
                             layers=1, prefill=True, seed=4),

@@ -22,14 +22,14 @@ def bm():
     return bit_moe_b200
 
 
-def gpu_layer(wl, layer=0):
+def gpu_layer(wl, layer=0, fmt="ternary"):
     """(device MoELayer, fp32 generator) for workload `wl`, weights drawn on cuda."""
     from bit_moe_b200.layers import quantize_layer
     fn = lambda role, e: synthetic.expert_matrix(wl, layer, role, e, "cuda")  # noqa: E731
-    return quantize_layer(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, fn), fn
+    return quantize_layer(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, fn, fmt=fmt), fn
 
 
-def oracle_layer(orc, wl, fn, experts=None):
+def oracle_layer(orc, wl, fn, experts=None, fmt="ternary"):
     """Oracle layer with the same fp32 weights (copied from the device), holding
     only `experts` (all if None) renumbered 0..n-1.  Returns (layer, remap)
     with remap[e] the compact id of expert e (-1 if absent)."""
@@ -45,7 +45,7 @@ def oracle_layer(orc, wl, fn, experts=None):
         wg[i * F:(i + 1) * F] = fn("gate", e).cpu().numpy()
         wu[i * F:(i + 1) * F] = fn("up", e).cpu().numpy()
         wd[i * H:(i + 1) * H] = fn("down", e).cpu().numpy()
-    return orc.Layer.from_float(H, F, n, wl.top_k, wg, wu, wd), remap
+    return orc.Layer.from_float(H, F, n, wl.top_k, wg, wu, wd, fmt=fmt), remap
 
 
 def rel_err_rms(y, ref):
