@@ -51,11 +51,12 @@ def test_sign_matvec_blocksums_and_outputs(orc, rows, k, ntok):
 
 def test_sign_matvec_extreme_codes(orc):
     """Activations at +-127 and weights all negative or all positive: the
-    block sums reach +-32*127 exactly."""
+    block sums are bit-exact and reach +-32*127 where the codes agree."""
     B = bm()
     rows, k = 32, 512
     w = np.where(np.arange(rows)[:, None] % 2 == 0, 1.0, -1.0).astype(np.float32) * np.ones((1, k), np.float32)
-    x = np.where(np.arange(k) % 3 == 0, 1.0, -1.0).astype(np.float32)[None, :]
+    # the first 256 activations all +1 (codes +127), the rest a +-1 pattern
+    x = np.where((np.arange(k) < 256) | (np.arange(k) % 3 == 0), 1.0, -1.0).astype(np.float32)[None, :]
     m = B.moe_quantize_weights_sign(torch.from_numpy(w).cuda())
     xq, xd = orc.quant_act_q8(x)
     _, isum = B.moe_debug_matvec(m, torch.from_numpy(xq).cuda(), torch.from_numpy(xd).cuda())
