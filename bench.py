@@ -23,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import sys
 import threading
 import time
@@ -171,12 +172,20 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- traffic
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/', re.S)
+
+
 def kernel_source_hash():
+    """Hash of the kernel sources' code: comments dropped and runs of white
+    space collapsed, so that counters taken on a source stay attributed to it
+    when only its comments change."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_moe_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        code = _CODE_TOKENS.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
+        h.update(name.encode() + b"\0" + " ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -4,22 +4,23 @@
 //
 // A one-token step moves a few megabytes: it is bound by latency, not by
 // bandwidth, so the step's three dependent phases run inside one cooperative
-// launch (every CTA resident), handing data over through L2 with tagged
-// values and counters instead of grid-wide barriers:
+// launch (every CTA resident), handing data over through L2 as values tagged
+// with the launch's generation instead of grid-wide barriers:
 //   A. every CTA quantizes x to int8 32-blocks in its shared memory (the same
 //      result everywhere) and publishes the fixed-order router logits of its
-//      share of the experts, each tagged with the launch's generation;
+//      share of the experts, each tagged;
 //   B. every CTA polls the E tagged logits until all carry this launch's tag,
-//      takes the top-k itself (ties to the lower id, so every CTA agrees;
-//      every logit is ranked against all others in parallel), starts the bulk
-//      copies of the down-projection weights it will need (its 32-row panel
-//      of hidden for each selected expert) into shared memory, and computes
-//      its share of the gate/up units (32-row panels of ffn, hidden blocks
-//      split over the warps), writing the requantized SwiGLU codes and
-//      counting each finished unit on its slot's counter;
-//   C. each CTA with a panel of hidden waits for the k slot counters to reach
-//      the number of ffn panels, then warp j multiplies slot j's codes with the
-//      prefetched down weights, and the slots are summed in order (no atomics
+//      takes the top-k itself (ties to the lower id, so every CTA agrees),
+//      starts the bulk copies of the down-projection weights it will need (its
+//      32-row panel of hidden for each selected expert) into shared memory,
+//      and computes its share of the gate/up units (32-row panels of ffn) in
+//      two streams of 8 warps, the hidden blocks of a unit split over a
+//      stream's warps; each finished unit publishes its requantized SwiGLU
+//      codes, scale and code sum as tagged words;
+//   C. each CTA with a panel of hidden splits every slot's ffn blocks over two
+//      warps, which start as soon as the units of their blocks carry this
+//      launch's tag, multiply them with the prefetched down weights, and one
+//      warp applies the block scales and sums the slots in order (no atomics
 //      on data).
 // Parakon Runtime README, "How it works" (fused decode mat-vecs on the packed
 // blocks, int8 activations); llama-modchip page, "Key highlights" (all top-k
