@@ -320,6 +320,24 @@ def test_forward_decode_prefill_boundary(orc):
         assert rel_err_rms(y[rows], ref) <= LAYER_TOL
 
 
+@pytest.mark.parametrize("n_experts,top_k", [(300, 2), (64, 10)])
+def test_forward_one_token_outside_fused_step(orc, n_experts, top_k):
+    """One token of a layer the fused one-token kernel does not take (more than
+    256 experts, or top-k above 8) runs the chained kernels (router with the
+    activation quantization and top-k, gate/up, down); it matches the oracle
+    and equals the same token inside a 3-token batch bitwise."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"].with_(n_experts=n_experts, top_k=top_k, seed=40 + top_k)
+    layer, fn = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 41, ntok=3, device="cuda")
+    y1, _ = _run_forward(B, layer, wr, x[:1].contiguous())
+    ref, _ = _oracle_tokens(orc, wl, fn, wr.cpu().numpy(), x[:1].cpu().numpy(), np.array([0]))
+    assert rel_err_rms(y1, ref) <= LAYER_TOL
+    y3, _ = _run_forward(B, layer, wr, x)
+    assert np.array_equal(y1[0], y3[0])
+
+
 @pytest.mark.parametrize("ntok", [1, 2, 70])
 def test_chained_layers_no_sync(ntok):
     """Layer outputs fed straight into the next call on the same stream (the
