@@ -52,3 +52,28 @@ def test_host_side_validation_without_device():
     assert L.moe_workspace_bytes(ctypes.byref(lay), 1, 0) == 0   # hidden % 256
     rc = L.moe_check_status(None, None)
     assert rc == -1
+
+
+def test_sign_format_host_side_without_device():
+    B, L = _lib()
+    assert L.moe_sign_words(64, 512) == 64 * 2 * 8
+    assert L.moe_sign_words(0, 512) == 0
+    # argument checks of the sign-code quantizer come before any device call
+    rc = L.moe_quantize_weights_sign(None, 32, 256, None, None, None)
+    assert rc == -1 and b"NULL" in L.moe_last_error()
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
+    assert L.moe_quantize_weights_sign(p, 31, 256, p, p, None) == -2     # rows % 32
+    assert L.moe_quantize_weights_sign(p, 32, 200, p, p, None) == -2     # k % 256
+    # a layer whose matrices mix formats, or name an unknown one, is rejected
+    def tm(rows, k, fmt):
+        return B.moe_tmat(rows, k, p.value, p.value, fmt)
+    mixed = B.moe_layer(256, 256, 2, 1, tm(512, 256, 1), tm(512, 256, 1), tm(512, 256, 0))
+    x = ctypes.c_void_p(p.value)
+    rc = L.moe_forward(ctypes.byref(mixed), x, 1, x, x, x, 1 << 30, None)
+    assert rc == -1 and b"format" in L.moe_last_error()
+    bad = B.moe_layer(256, 256, 2, 1, tm(512, 256, 7), tm(512, 256, 7), tm(512, 256, 7))
+    rc = L.moe_forward(ctypes.byref(bad), x, 1, x, x, x, 1 << 30, None)
+    assert rc == -1 and b"format" in L.moe_last_error()
+    # the binding's struct matches the header's field order
+    assert [f[0] for f in B.moe_tmat._fields_] == ["rows", "k", "trits", "scales", "format"]
