@@ -54,6 +54,16 @@ def lib():
         L.orc_quantize_weights_sign.argtypes = [p, i64, i64, p, p]
         L.orc_unpack_weights_sign.restype = ctypes.c_int
         L.orc_unpack_weights_sign.argtypes = [p, p, i64, i64, i64, i64, p, p]
+        L.orc_e16_code_words.restype = i64
+        L.orc_e16_code_words.argtypes = [i64, i64]
+        L.orc_e16_code_index.restype = i64
+        L.orc_e16_code_index.argtypes = [i64, i64, i64, ctypes.c_int]
+        L.orc_quantize_weights_e16.restype = ctypes.c_int
+        L.orc_quantize_weights_e16.argtypes = [p, i64, i64, p, p, p]
+        L.orc_unpack_weights_e16.restype = ctypes.c_int
+        L.orc_unpack_weights_e16.argtypes = [p, p, p, i64, i64, i64, i64, p, p]
+        L.orc_matvec_e16.restype = None
+        L.orc_matvec_e16.argtypes = [p, p, i64, i64, p, p, p]
         L.orc_unpack_weights.restype = ctypes.c_int
         L.orc_unpack_weights.argtypes = [p, p, i64, i64, i64, i64, p, p]
         L.orc_quant_act_q8.restype = ctypes.c_int
@@ -80,10 +90,12 @@ class OrcLayer(ctypes.Structure):
         ("up_trits", ctypes.c_void_p), ("up_scales", ctypes.c_void_p),
         ("down_trits", ctypes.c_void_p), ("down_scales", ctypes.c_void_p),
         ("format", ctypes.c_int64),
+        ("gate_codes", ctypes.c_void_p), ("up_codes", ctypes.c_void_p),
+        ("down_codes", ctypes.c_void_p),
     ]
 
 
-FORMATS = {"ternary": 0, "sign": 1}
+FORMATS = {"ternary": 0, "sign": 1, "e16": 2}
 
 
 def _c(a, dtype):
@@ -196,6 +208,51 @@ def unpack_weights_sign(codes, scales, rows, k, row0=0, nrows=None):
     return q, s
 
 
+# ---------------------------------------------------------------- two-level scales (E16)
+def e16_code_words(rows, k):
+    return int(lib().orc_e16_code_words(rows, k))
+
+
+def e16_code_index(k, r, b, u):
+    return int(lib().orc_e16_code_index(k, r, b, u))
+
+
+def quantize_weights_e16(w):
+    """w [rows][k] fp32 -> (trits uint32 [rows*(k/256)*13], codes uint32
+    [rows*(k/256)*2], anchors uint16 [rows])."""
+    w = _c(w, np.float32)
+    rows, k = w.shape
+    trits = np.zeros(trit_words(rows, k), dtype=np.uint32)
+    codes = np.zeros(e16_code_words(rows, k), dtype=np.uint32)
+    anchors = np.zeros(rows, dtype=np.uint16)
+    if lib().orc_quantize_weights_e16(_ptr(w), rows, k, _ptr(trits), _ptr(codes), _ptr(anchors)):
+        raise ValueError("orc_quantize_weights_e16: bad shape %r" % (w.shape,))
+    return trits, codes, anchors
+
+
+def unpack_weights_e16(trits, codes, anchors, rows, k, row0=0, nrows=None):
+    """-> (q int8 [nrows][k], s16 float32 [nrows][k/16])."""
+    if nrows is None:
+        nrows = rows - row0
+    trits, codes, anchors = _c(trits, np.uint32), _c(codes, np.uint32), _c(anchors, np.uint16)
+    q = np.zeros((nrows, k), dtype=np.int8)
+    s16 = np.zeros((nrows, k // 16), dtype=np.float32)
+    if lib().orc_unpack_weights_e16(_ptr(trits), _ptr(codes), _ptr(anchors), rows, k, row0, nrows,
+                                    _ptr(q), _ptr(s16)):
+        raise ValueError("orc_unpack_weights_e16 failed")
+    return q, s16
+
+
+def matvec_e16(q, s16, xq, xd):
+    """fp64 [rows]: sum_j xd_j * sum_{16-blocks h of j} s16[h] * sum_{k in h} q*xq."""
+    q = _c(q, np.int8)
+    s16 = _c(s16, np.float32)
+    rows, k = q.shape
+    out = np.zeros(rows, dtype=np.float64)
+    lib().orc_matvec_e16(_ptr(q), _ptr(s16), rows, k, _ptr(_c(xq, np.int8)), _ptr(_c(xd, np.float32)), _ptr(out))
+    return out
+
+
 # ---------------------------------------------------------------- activations
 def quant_act_q8(x):
     """x [ntok][k] fp32 -> (xq int8 [ntok][k], xd fp32 [ntok][k/32])."""
@@ -274,9 +331,11 @@ class Layer:
     def __init__(self, hidden, ffn, n_experts, top_k, gate, up, down, fmt="ternary"):
         self.hidden, self.ffn, self.n_experts, self.top_k = hidden, ffn, n_experts, top_k
         self.fmt = fmt
-        self.gate = (_c(gate[0], np.uint32), _c(gate[1], np.uint16))
-        self.up = (_c(up[0], np.uint32), _c(up[1], np.uint16))
-        self.down = (_c(down[0], np.uint32), _c(down[1], np.uint16))
+        if fmt == "e16":  # (trits, codes, anchors): kept as (trits, anchors, codes)
+            gate, up, down = [(m[0], m[2], m[1]) for m in (gate, up, down)]
+        self.gate = (_c(gate[0], np.uint32), _c(gate[1], np.uint16)) + tuple(_c(m, np.uint32) for m in gate[2:])
+        self.up = (_c(up[0], np.uint32), _c(up[1], np.uint16)) + tuple(_c(m, np.uint32) for m in up[2:])
+        self.down = (_c(down[0], np.uint32), _c(down[1], np.uint16)) + tuple(_c(m, np.uint32) for m in down[2:])
         words = sign_words if fmt == "sign" else trit_words
         assert self.gate[0].size == words(n_experts * ffn, hidden)
         assert self.up[0].size == words(n_experts * ffn, hidden)
@@ -285,7 +344,7 @@ class Layer:
     @classmethod
     def from_float(cls, hidden, ffn, n_experts, top_k, wg, wu, wd, fmt="ternary"):
         """wg, wu [E*ffn][hidden], wd [E*hidden][ffn] fp32."""
-        quant = quantize_weights_sign if fmt == "sign" else quantize_weights
+        quant = {"sign": quantize_weights_sign, "e16": quantize_weights_e16}.get(fmt, quantize_weights)
         return cls(hidden, ffn, n_experts, top_k, quant(wg), quant(wu), quant(wd), fmt=fmt)
 
     def c_struct(self, top_k=None):
@@ -294,7 +353,8 @@ class Layer:
                         _ptr(self.gate[0]).value, _ptr(self.gate[1]).value,
                         _ptr(self.up[0]).value, _ptr(self.up[1]).value,
                         _ptr(self.down[0]).value, _ptr(self.down[1]).value,
-                        FORMATS[self.fmt])
+                        FORMATS[self.fmt],
+                        *[(_ptr(m[2]).value if len(m) > 2 else None) for m in (self.gate, self.up, self.down)])
 
 
 def expert_ffn(layer, xq, xd, idx, wts, debug=False):

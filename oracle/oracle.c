@@ -258,6 +258,123 @@ int orc_unpack_weights_sign(const uint32_t* codes, const uint16_t* scales,
 }
 
 /* ======================================================================== */
+/* two-level scales (E16)                                                    */
+/* ======================================================================== */
+/* The E16-row scales of the pxq_llama README ("What's PXQ?"), read onto the
+   ternary digits (see oracle.h): one fp16 anchor per row, a 4-bit code per
+   16-weight block, s_h = A * (c_h + 1) / 16.                              */
+int64_t orc_e16_code_words(int64_t rows, int64_t k) {
+  return rows * (k / ORC_BLOCK) * ORC_E16_WORDS;
+}
+int64_t orc_e16_code_index(int64_t k, int64_t r, int64_t b, int u) {
+  int64_t nb = k / ORC_BLOCK;
+  int64_t p = r / ORC_PANEL;
+  return ((p * nb + b) * ORC_E16_WORDS + u) * ORC_PANEL + (r % ORC_PANEL);
+}
+
+static double mean_abs16(const float* w) {
+  double sum = 0.0;
+  for (int i = 0; i < 16; ++i) sum += fabs((double)w[i]);
+  return sum / 16.0;
+}
+
+int orc_quantize_weights_e16(const float* w, int64_t rows, int64_t k,
+                             uint32_t* trits, uint32_t* codes,
+                             uint16_t* anchors) {
+  if (rows <= 0 || k <= 0 || rows % ORC_PANEL || k % ORC_BLOCK) return -1;
+  int64_t nb = k / ORC_BLOCK;
+  int8_t q[256];
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* wr = w + r * k;
+    double mmax = 0.0;
+    for (int64_t h = 0; h < k / 16; ++h) {
+      double m = mean_abs16(wr + 16 * h);
+      if (m > mmax) mmax = m;
+    }
+    uint16_t ah = orc_f16_from_f64(mmax);
+    anchors[r] = ah;
+    double a = (double)orc_f16_to_f32(ah);
+    for (int64_t b = 0; b < nb; ++b) {
+      uint32_t cw[ORC_E16_WORDS] = {0, 0};
+      for (int h = 0; h < 16; ++h) {
+        const float* wb = wr + b * ORC_BLOCK + 16 * h;
+        int c = 0;
+        if (a > 0.0) {
+          double t = rint(16.0 * mean_abs16(wb) / a) - 1.0;
+          c = t < 0.0 ? 0 : (t > 15.0 ? 15 : (int)t);
+        }
+        cw[h / 8] |= (uint32_t)c << (4 * (h % 8));
+        float half = 0.5f * (float)(a * (c + 1) / 16.0);
+        for (int i = 0; i < 16; ++i) {
+          float x = wb[i];
+          q[16 * h + i] = (fabsf(x) >= half && x != 0.0f) ? (int8_t)(x > 0.0f ? 1 : -1) : 0;
+        }
+      }
+      for (int u = 0; u < ORC_E16_WORDS; ++u) codes[orc_e16_code_index(k, r, b, u)] = cw[u];
+      for (int wd = 0; wd < ORC_BLOCK_WORDS; ++wd) {
+        uint32_t word = 0;
+        for (int l = 0; l < 4; ++l) {
+          int t[5];
+          for (int i = 0; i < 5; ++i) {
+            int kk = 20 * wd + 4 * i + l;
+            t[i] = (kk < ORC_BLOCK) ? q[kk] + 1 : 1;
+          }
+          word |= (uint32_t)orc_trit_byte_encode(t) << (8 * l);
+        }
+        trits[orc_word_index(k, r, b, wd)] = word;
+      }
+    }
+  }
+  return 0;
+}
+
+int orc_unpack_weights_e16(const uint32_t* trits, const uint32_t* codes,
+                           const uint16_t* anchors, int64_t rows, int64_t k,
+                           int64_t row0, int64_t nrows, int8_t* q,
+                           float* s16) {
+  if (rows <= 0 || k <= 0 || rows % ORC_PANEL || k % ORC_BLOCK) return -1;
+  if (row0 < 0 || nrows < 0 || row0 + nrows > rows) return -1;
+  int64_t nb = k / ORC_BLOCK;
+  /* the digits are those of the ternary format; the scales come from the
+     anchor and the codes */
+  if (orc_unpack_weights(trits, NULL, rows, k, row0, nrows, q, NULL)) return -1;
+  for (int64_t rr = 0; rr < nrows; ++rr) {
+    int64_t r = row0 + rr;
+    double a = (double)orc_f16_to_f32(anchors[r]);
+    for (int64_t b = 0; b < nb; ++b) {
+      for (int h = 0; h < 16; ++h) {
+        uint32_t cw = codes[orc_e16_code_index(k, r, b, h / 8)];
+        int c = (int)((cw >> (4 * (h % 8))) & 15u);
+        s16[rr * (k / 16) + b * 16 + h] = (float)(a * (c + 1) / 16.0);
+      }
+    }
+  }
+  return 0;
+}
+
+void orc_matvec_e16(const int8_t* q, const float* s16, int64_t rows,
+                    int64_t k, const int8_t* xq, const float* xd,
+                    double* out) {
+  for (int64_t r = 0; r < rows; ++r) {
+    double acc = 0.0;
+    for (int64_t j = 0; j < k / ORC_QBLOCK; ++j) {
+      double inner = 0.0;
+      for (int half = 0; half < 2; ++half) {
+        int64_t h = 2 * j + half;
+        int32_t isum = 0;
+        for (int i = 0; i < 16; ++i) {
+          int64_t kk = 16 * h + i;
+          isum += (int32_t)q[r * k + kk] * (int32_t)xq[kk];
+        }
+        inner += (double)s16[r * (k / 16) + h] * (double)isum;
+      }
+      acc += (double)xd[j] * inner;
+    }
+    out[r] = acc;
+  }
+}
+
+/* ======================================================================== */
 /* activation quantization                                                   */
 /* ======================================================================== */
 /* int8 activations with one fp32 scale per 32 values (Parakon Runtime README
@@ -425,7 +542,8 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
                    float* ad_out) {
   int64_t H = L->hidden, F = L->ffn, E = L->n_experts, K = L->top_k;
   if (H <= 0 || F <= 0 || E <= 0 || K < 1 || K > E) return -1;
-  if (L->format != ORC_FORMAT_TERNARY && L->format != ORC_FORMAT_SIGN) return -1;
+  if (L->format != ORC_FORMAT_TERNARY && L->format != ORC_FORMAT_SIGN && L->format != ORC_FORMAT_E16)
+    return -1;
   if (H % ORC_BLOCK || F % ORC_BLOCK || F % ORC_PANEL || H % ORC_PANEL) return -1;
   for (int64_t i = 0; i < ntok * K; ++i)
     if (idx[i] < 0 || idx[i] >= E) return -2;
@@ -434,9 +552,11 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
   int8_t* qg = (int8_t*)malloc((size_t)(F * H));
   int8_t* qu = (int8_t*)malloc((size_t)(F * H));
   int8_t* qd = (int8_t*)malloc((size_t)(H * F));
-  float* sg = (float*)malloc(sizeof(float) * (size_t)(F * nbH));
-  float* su = (float*)malloc(sizeof(float) * (size_t)(F * nbH));
-  float* sd = (float*)malloc(sizeof(float) * (size_t)(H * nbF));
+  /* block scales: one per 256 weights, or one per 16 (ORC_FORMAT_E16) */
+  const int64_t per = L->format == ORC_FORMAT_E16 ? ORC_BLOCK / 16 : 1;
+  float* sg = (float*)malloc(sizeof(float) * (size_t)(F * nbH * per));
+  float* su = (float*)malloc(sizeof(float) * (size_t)(F * nbH * per));
+  float* sd = (float*)malloc(sizeof(float) * (size_t)(H * nbF * per));
   double* g = (double*)malloc(sizeof(double) * (size_t)F);
   double* u = (double*)malloc(sizeof(double) * (size_t)F);
   float* a = (float*)malloc(sizeof(float) * (size_t)F);
@@ -449,11 +569,19 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
     int used = 0;
     for (int64_t i = 0; i < ntok * K; ++i) used |= (idx[i] == e);
     if (!used) continue;
-    int (*unpack)(const uint32_t*, const uint16_t*, int64_t, int64_t, int64_t, int64_t, int8_t*, float*) =
-        L->format == ORC_FORMAT_SIGN ? orc_unpack_weights_sign : orc_unpack_weights;
-    if (unpack(L->gate_trits, L->gate_scales, E * F, H, e * F, F, qg, sg) ||
-        unpack(L->up_trits, L->up_scales, E * F, H, e * F, F, qu, su) ||
-        unpack(L->down_trits, L->down_scales, E * H, F, e * H, H, qd, sd)) {
+    int bad;
+    if (L->format == ORC_FORMAT_E16) {
+      bad = orc_unpack_weights_e16(L->gate_trits, L->gate_codes, L->gate_scales, E * F, H, e * F, F, qg, sg) ||
+            orc_unpack_weights_e16(L->up_trits, L->up_codes, L->up_scales, E * F, H, e * F, F, qu, su) ||
+            orc_unpack_weights_e16(L->down_trits, L->down_codes, L->down_scales, E * H, F, e * H, H, qd, sd);
+    } else {
+      int (*unpack)(const uint32_t*, const uint16_t*, int64_t, int64_t, int64_t, int64_t, int8_t*, float*) =
+          L->format == ORC_FORMAT_SIGN ? orc_unpack_weights_sign : orc_unpack_weights;
+      bad = unpack(L->gate_trits, L->gate_scales, E * F, H, e * F, F, qg, sg) ||
+            unpack(L->up_trits, L->up_scales, E * F, H, e * F, F, qu, su) ||
+            unpack(L->down_trits, L->down_scales, E * H, F, e * H, H, qd, sd);
+    }
+    if (bad) {
       rc = -1;
       break;
     }
@@ -462,11 +590,13 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
         if (idx[t * K + j] != e) continue;
         const int8_t* xt = xq + t * H;
         const float* dt = xd + t * (H / ORC_QBLOCK);
-        orc_matvec(qg, sg, F, H, xt, dt, g);
-        orc_matvec(qu, su, F, H, xt, dt, u);
+        void (*matvec)(const int8_t*, const float*, int64_t, int64_t, const int8_t*, const float*, double*) =
+            L->format == ORC_FORMAT_E16 ? orc_matvec_e16 : orc_matvec;
+        matvec(qg, sg, F, H, xt, dt, g);
+        matvec(qu, su, F, H, xt, dt, u);
         for (int64_t f = 0; f < F; ++f) a[f] = (float)(g[f] / (1.0 + exp(-g[f])) * u[f]);
         orc_quant_act_q8(a, 1, F, aq, ad);
-        orc_matvec(qd, sd, H, F, aq, ad, ye + (t * K + j) * H);
+        matvec(qd, sd, H, F, aq, ad, ye + (t * K + j) * H);
         int64_t o = t * K + j;
         if (g_out) memcpy(g_out + o * F, g, sizeof(double) * (size_t)F);
         if (u_out) memcpy(u_out + o * F, u, sizeof(double) * (size_t)F);

@@ -96,6 +96,40 @@ int orc_unpack_weights_sign(const uint32_t* codes, const uint16_t* scales,
                             int64_t rows, int64_t k, int64_t row0,
                             int64_t nrows, int8_t* q, float* s);
 
+/* ---- two-level scales (E16) ------------------------------------------------ */
+/* The E16-row scales of the pxq_llama README ("What's PXQ?": a per-row fp16
+ * anchor plus a 4-bit sub-scale per 16-element block), read onto the
+ * ternary digits: per row A = fp16_RNE(max over its 16-weight blocks of
+ * mean|w|, fp64); per 16-weight block h a code c_h in 0..15 with scale
+ * s_h = A * (c_h + 1) / 16, c_h = clamp(rint(16 * m_h / A) - 1, 0, 15)
+ * (m_h the block's mean|w| in fp64, A as a double; c_h = 0 when A = 0);
+ * q = sign(w) where |w| >= s_h / 2 in fp32, else 0.  Storage: the base-3
+ * words of the ternary format (orc_word_index), ORC_E16_WORDS words of
+ * codes per 256 weights (word u of block b holds 16-blocks 8u..8u+7, block
+ * 8u + v in bits 4v..4v+3; interleaved over 32-row panels like the digits)
+ * and one fp16 anchor per row.                                            */
+#define ORC_E16_WORDS 2
+int64_t orc_e16_code_words(int64_t rows, int64_t k);  /* rows*(k/256)*2 */
+/* Index of code word u (0..1) of block b of row r. */
+int64_t orc_e16_code_index(int64_t k, int64_t r, int64_t b, int u);
+/* Quantize w [rows][k]: trits [orc_trit_words], codes [orc_e16_code_words],
+ * anchors [rows].  Returns 0, or -1 when rows % 32 or k % 256 is nonzero. */
+int orc_quantize_weights_e16(const float* w, int64_t rows, int64_t k,
+                             uint32_t* trits, uint32_t* codes,
+                             uint16_t* anchors);
+/* Expand rows [row0, row0+nrows) to q [nrows][k] in {-1,0,1} and the fp32
+ * scale of every 16-weight block s16 [nrows][k/16] (A * (c+1) / 16, exact
+ * in fp32).  Returns 0, or -1 on a bad shape or an undecodable byte.     */
+int orc_unpack_weights_e16(const uint32_t* trits, const uint32_t* codes,
+                           const uint16_t* anchors, int64_t rows, int64_t k,
+                           int64_t row0, int64_t nrows, int8_t* q,
+                           float* s16);
+/* out[r] = sum_j xd[j] * sum_{16-blocks h in activation block j}
+ *          s16[r][h] * sum_{k in h} q[r][k] * xq[k], in fp64.             */
+void orc_matvec_e16(const int8_t* q, const float* s16, int64_t rows,
+                    int64_t k, const int8_t* xq, const float* xd,
+                    double* out);
+
 /* ---- activations ---------------------------------------------------------- */
 /* x [ntok][k] -> xq [ntok][k] int8, xd [ntok][k/32] fp32.  Returns -1 if
  * k % 32 != 0.                                                             */
@@ -127,11 +161,16 @@ typedef struct {
   const uint32_t* gate_trits; const uint16_t* gate_scales; /* rows E*ffn, k hidden */
   const uint32_t* up_trits;   const uint16_t* up_scales;   /* rows E*ffn, k hidden */
   const uint32_t* down_trits; const uint16_t* down_scales; /* rows E*hidden, k ffn */
-  int64_t format; /* ORC_FORMAT_TERNARY, or ORC_FORMAT_SIGN (the *_trits
-                     pointers then hold sign code words)                  */
+  int64_t format; /* ORC_FORMAT_TERNARY, ORC_FORMAT_SIGN (the *_trits
+                     pointers then hold sign code words) or ORC_FORMAT_E16
+                     (the *_scales pointers then hold the per-row anchors)  */
+  const uint32_t* gate_codes; /* ORC_FORMAT_E16: the 4-bit sub-scale words */
+  const uint32_t* up_codes;
+  const uint32_t* down_codes;
 } orc_layer;
 #define ORC_FORMAT_TERNARY 0
 #define ORC_FORMAT_SIGN 1
+#define ORC_FORMAT_E16 2
 
 /* y [ntok][hidden] (fp64) = sum over slots j (in slot order) of
  * wts[t][j] * FFN_{idx[t][j]}(x_t).  Optional (may be NULL) debug outputs,
