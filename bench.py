@@ -42,7 +42,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="30b",
-                    help="tiny | 30b | 30b-b16 | large | large-b8 | 30b-prefill | 30b-sign | large-sign-b8")
+                    help="tiny | 30b | 30b-b16 | large | large-b8 | 30b-prefill | 30b-sign | large-sign-b8 | "
+                         "30b-e16 | large-e16-b8")
     ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -81,8 +82,7 @@ def kernel_bytes(wl, unique_experts):
     out)."""
     T, H, F, E, K = wl.ntok, wl.hidden, wl.ffn, wl.n_experts, wl.top_k
     pairs = T * K
-    bb = wl.block_bytes
-    weights = unique_experts * 3 * matrix_bytes(F, H, bb)
+    weights = unique_experts * wl.expert_bytes
     return {
         # the whole one-token step in one kernel: router, x, the routed
         # experts' packed weights, the int8 intermediates and y
@@ -100,9 +100,9 @@ def kernel_bytes(wl, unique_experts):
         "router_quant": E * H * 4 + T * H * 4 + T * E * 4 + T * H + T * H // 32 * 4,
         "topk_group": T * E * 4 + pairs * 8 + pairs * 4 * 3,
         "group": pairs * 4 * 3,
-        "gateup": unique_experts * 2 * matrix_bytes(F, H, bb) + T * H + T * H // 32 * 4
+        "gateup": unique_experts * 2 * wl.matrix_bytes(F, H) + T * H + T * H // 32 * 4
         + pairs * F + pairs * F // 32 * 4 + pairs * 8,
-        "down": unique_experts * matrix_bytes(H, F, bb) + pairs * F + pairs * F // 32 * 4
+        "down": unique_experts * wl.matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4
         + pairs * H * 4 * 2 + T * H * 4 + pairs * 8,
     }
 
@@ -283,9 +283,10 @@ def job_rate(tokens_per_rank, world, ms):
 def workload_config(wl, layers):
     c = {"workload": wl.describe(), "hidden": wl.hidden, "expert_ffn": wl.ffn,
          "experts": wl.n_experts, "top_k": wl.top_k, "tokens_per_step": wl.ntok,
-         "weights": ("1-bit sign codes, 256-blocks (32 B of signs + fp16 absmean scale), N(0,%g)"
-                     if wl.fmt == "sign" else
-                     "ternary absmean 256-blocks (52 B base-3 + fp16 scale), N(0,%g)") % wl.w_std,
+         "weights": {"sign": "1-bit sign codes, 256-blocks (32 B of signs + fp16 absmean scale), N(0,%g)",
+                     "e16": "ternary digits with two-level scales (fp16 anchor per row, 4-bit sub-scale "
+                            "per 16 weights), N(0,%g)"}.get(
+                         wl.fmt, "ternary absmean 256-blocks (52 B base-3 + fp16 scale), N(0,%g)") % wl.w_std,
          "activations": "x ~ N(0,1) fp32, int8 32-blocks"}
     if layers is not None:
         c["layer_stack"] = layers

@@ -34,7 +34,7 @@ EXPORTS = (
     "moe_expert_ffn_decode", "moe_expert_ffn_prefill", "moe_forward", "moe_forward_host",
     "moe_check_status", "moe_last_error", "moe_debug_matvec", "moe_launch_count",
     "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
-    "moe_sign_words", "moe_quantize_weights_sign",
+    "moe_sign_words", "moe_quantize_weights_sign", "moe_e16_code_words", "moe_quantize_weights_e16",
 )
 
 
@@ -47,10 +47,10 @@ class MoEError(RuntimeError):
 class moe_tmat(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("trits", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("format", ctypes.c_int32)]
+                ("format", ctypes.c_int32), ("codes", ctypes.c_void_p)]
 
 
-FORMATS = {"ternary": 0, "sign": 1}   # moe_format
+FORMATS = {"ternary": 0, "sign": 1, "e16": 2}   # moe_format
 
 
 class moe_layer(ctypes.Structure):
@@ -74,11 +74,13 @@ def lib():
         sig = {
             "moe_trit_words": (sz, [i64, i64]),
             "moe_sign_words": (sz, [i64, i64]),
+            "moe_e16_code_words": (sz, [i64, i64]),
             "moe_scale_count": (sz, [i64, i64]),
             "moe_workspace_bytes": (sz, [p, i32, i32]),
             "moe_workspace_init": (ctypes.c_int, [p, sz, p]),
             "moe_quantize_weights": (ctypes.c_int, [p, i64, i64, p, p, p]),
             "moe_quantize_weights_sign": (ctypes.c_int, [p, i64, i64, p, p, p]),
+            "moe_quantize_weights_e16": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
             "moe_quant_act_q8": (ctypes.c_int, [p, i32, i32, p, p, p]),
             "moe_route_topk": (ctypes.c_int, [p, p, i32, i32, i32, i32, p, p, p, sz, p]),
             "moe_route_workspace_bytes": (sz, [i32, i32]),
@@ -132,8 +134,17 @@ def sign_words(rows, k):
     return int(lib().moe_sign_words(rows, k))
 
 
+def e16_code_words(rows, k):
+    return int(lib().moe_e16_code_words(rows, k))
+
+
 def packed_words(rows, k, fmt="ternary"):
     return sign_words(rows, k) if fmt == "sign" else trit_words(rows, k)
+
+
+def scale_words(rows, k, fmt="ternary"):
+    """fp16 values in a matrix's `scales`: one per block, or one anchor per row (e16)."""
+    return rows if fmt == "e16" else scale_count(rows, k)
 
 
 def scale_count(rows, k):
@@ -143,23 +154,30 @@ def scale_count(rows, k):
 # ---------------------------------------------------------------- weights
 class TernaryMatrix:
     """Packed matrix: trits (int32 view of the uint32 words: base-3 digits,
-    or 1-bit sign codes when fmt is "sign") and scales (int16 view of the fp16
-    bits), in the storage formats of bitmoe.h."""
+    or 1-bit sign codes when fmt is "sign"), scales (int16 view of the fp16
+    bits: block scales, or per-row anchors when fmt is "e16") and, for "e16",
+    codes (int32 view of the 4-bit sub-scale words), in the storage formats of
+    bitmoe.h."""
 
-    def __init__(self, rows, k, trits, scales, fmt="ternary"):
+    def __init__(self, rows, k, trits, scales, fmt="ternary", codes=None):
         self.rows, self.k, self.trits, self.scales, self.fmt = rows, k, trits, scales, fmt
+        self.codes = codes
 
     @classmethod
     def empty(cls, rows, k, device="cuda", fmt="ternary"):
+        codes = (torch.empty(e16_code_words(rows, k), dtype=torch.int32, device=device)
+                 if fmt == "e16" else None)
         return cls(rows, k, torch.empty(packed_words(rows, k, fmt), dtype=torch.int32, device=device),
-                   torch.empty(scale_count(rows, k), dtype=torch.int16, device=device), fmt)
+                   torch.empty(scale_words(rows, k, fmt), dtype=torch.int16, device=device), fmt, codes)
 
     def c_struct(self):
-        return moe_tmat(self.rows, self.k, self.trits.data_ptr(), self.scales.data_ptr(), FORMATS[self.fmt])
+        return moe_tmat(self.rows, self.k, self.trits.data_ptr(), self.scales.data_ptr(), FORMATS[self.fmt],
+                        self.codes.data_ptr() if self.codes is not None else None)
 
     @property
     def nbytes(self):
-        return self.trits.numel() * 4 + self.scales.numel() * 2
+        n = self.trits.numel() * 4 + self.scales.numel() * 2
+        return n + (self.codes.numel() * 4 if self.codes is not None else 0)
 
 
 def moe_quantize_weights(w, out=None, stream=None):
@@ -179,6 +197,18 @@ def moe_quantize_weights_sign(w, out=None, stream=None):
     _check(lib().moe_quantize_weights_sign(_dev(w, torch.float32, "w"), rows, k,
                                            ctypes.c_void_p(m.trits.data_ptr()),
                                            ctypes.c_void_p(m.scales.data_ptr()), _stream(stream)))
+    return m
+
+
+def moe_quantize_weights_e16(w, out=None, stream=None):
+    """w [rows][k] fp32 CUDA -> ternary digits with two-level scales
+    (TernaryMatrix, fmt "e16": per-row anchors in `scales`, sub-scale codes)."""
+    rows, k = w.shape
+    m = TernaryMatrix.empty(rows, k, w.device, fmt="e16") if out is None else out
+    _check(lib().moe_quantize_weights_e16(_dev(w, torch.float32, "w"), rows, k,
+                                          ctypes.c_void_p(m.trits.data_ptr()),
+                                          ctypes.c_void_p(m.codes.data_ptr()),
+                                          ctypes.c_void_p(m.scales.data_ptr()), _stream(stream)))
     return m
 
 

@@ -121,7 +121,7 @@ static int check_layer(const moe_layer* L) {
                 kMaxExperts, kMaxTopK);
   const moe_tmat* m[3] = {&L->gate, &L->up, &L->down};
   const char* names[3] = {"gate", "up", "down"};
-  if (L->gate.format != MOE_FORMAT_TERNARY && L->gate.format != MOE_FORMAT_SIGN)
+  if (L->gate.format != MOE_FORMAT_TERNARY && L->gate.format != MOE_FORMAT_SIGN && L->gate.format != MOE_FORMAT_E16)
     return fail(MOE_ERR_INVALID_ARG, "unknown weight format %d", L->gate.format);
   if (L->up.format != L->gate.format || L->down.format != L->gate.format)
     return fail(MOE_ERR_INVALID_ARG, "gate, up and down must share one weight format");
@@ -133,6 +133,10 @@ static int check_layer(const moe_layer* L) {
     if (!m[i]->trits || !m[i]->scales) return fail(MOE_ERR_INVALID_ARG, "%s has a NULL pointer", names[i]);
     if (!aligned16(m[i]->trits) || !aligned16(m[i]->scales))
       return fail(MOE_ERR_ALIGNMENT, "%s pointers must be 16-byte aligned", names[i]);
+    if (m[i]->format == MOE_FORMAT_E16) {
+      if (!m[i]->codes) return fail(MOE_ERR_INVALID_ARG, "%s has no sub-scale codes", names[i]);
+      if (!aligned16(m[i]->codes)) return fail(MOE_ERR_ALIGNMENT, "%s codes must be 16-byte aligned", names[i]);
+    }
   }
   return MOE_OK;
 }
@@ -165,6 +169,9 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
   P.status = &reinterpret_cast<WsHeader*>(ws)->status;
   P.direct = ntok == 1;
   P.format = L->gate.format;
+  P.gate_codes = L->gate.codes;
+  P.up_codes = L->up.codes;
+  P.down_codes = L->down.codes;
   P.items = reinterpret_cast<const Item*>(base + W.grp.items);
   P.n_items = reinterpret_cast<const int32_t*>(base + W.grp.n_items);
   P.pairs = reinterpret_cast<const int32_t*>(base + W.grp.pairs);
@@ -213,8 +220,9 @@ static int launch_decode(const DecodeParams& P, void* ws, const WsLayout& W, cud
     if (rc) return rc;
     return launch_ffn(P, stream);
   }
-  // sign codes: the grouped kernels in direct mode (item i = slot i)
-  if (P.format == MOE_FORMAT_SIGN) return launch_ffn(P, stream);
+  // sign codes and two-level scales: the grouped kernels in direct mode
+  // (item i = slot i)
+  if (P.format != MOE_FORMAT_TERNARY) return launch_ffn(P, stream);
   Decode2Params D = make_d2(P, ws, W);
   return launch_decode2(D, false, stream);
 }
@@ -255,6 +263,11 @@ static int launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t 
 using namespace bitmoe;
 
 extern "C" {
+
+size_t moe_e16_code_words(int64_t rows, int64_t k) {
+  if (rows <= 0 || k <= 0) return 0;
+  return static_cast<size_t>(rows) * static_cast<size_t>(k / kBlock) * kE16Words;
+}
 
 size_t moe_sign_words(int64_t rows, int64_t k) {
   if (rows <= 0 || k <= 0) return 0;
@@ -311,6 +324,17 @@ int moe_quantize_weights_sign(const float* w, int64_t rows, int64_t k, uint32_t*
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quantize_weights_sign: rows %% 32 and k %% 256 must be 0");
   if ((rc = check_device())) return rc;
   return launch_quantize_weights(w, rows, k, codes, scales, static_cast<cudaStream_t>(stream), true);
+}
+
+int moe_quantize_weights_e16(const float* w, int64_t rows, int64_t k, uint32_t* trits, uint32_t* codes,
+                             uint16_t* anchors, moe_stream_t stream) {
+  int rc = check_ptrs("quantize_weights_e16", w, trits, codes, anchors);
+  if (rc) return rc;
+  if (rows <= 0 || k <= 0) return fail(MOE_ERR_INVALID_ARG, "quantize_weights_e16: rows, k must be > 0");
+  if (rows % kPanel || k % kBlock)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quantize_weights_e16: rows %% 32 and k %% 256 must be 0");
+  if ((rc = check_device())) return rc;
+  return launch_quantize_weights_e16(w, rows, k, trits, codes, anchors, static_cast<cudaStream_t>(stream));
 }
 
 int moe_quant_act_q8(const float* x, int32_t ntok, int32_t k, int8_t* xq, float* xd,
@@ -388,9 +412,10 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   if ((rc = check_ptrs("forward", w_router, x, y, ws))) return rc;
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
-  const bool sign = L->gate.format == MOE_FORMAT_SIGN;
+  const bool sign = L->gate.format != MOE_FORMAT_TERNARY;  // sign codes or two-level scales
   if (sign && prefill)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: sign-code layers take at most %d tokens", kMaxDecodeTokens);
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: sign-code and E16 layers take at most %d tokens",
+                kMaxDecodeTokens);
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total) return fail(MOE_ERR_WORKSPACE, "forward: workspace %zu < %zu bytes", ws_bytes, W.total);
   if ((rc = check_device())) return rc;
@@ -403,7 +428,7 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   float* logits = reinterpret_cast<float*>(base + W.logits);
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
   if ((ntok > 1 || sign) && !prefill && router_quant_small_ok(ntok, L->hidden)) {
-    // few tokens (and one token of a sign-code layer): router logits with
+    // few tokens (and one token of a sign-code or E16 layer): router logits with
     // the activation quantization, then the top-k with the grouping, then
     // the grouped mat-vecs
     if ((rc = launch_router_quant_small(x, w_router, ntok, L->hidden, L->n_experts, logits, xq, xd, s)))
@@ -524,8 +549,10 @@ int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const fl
     return fail(MOE_ERR_INVALID_ARG, "debug_matvec: bad sizes");
   if (m->rows % kPanel || m->k % kBlock || m->k > kMaxHidden)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "debug_matvec: rows %% 32, k %% 256, k <= %d", kMaxHidden);
-  if (m->format != MOE_FORMAT_TERNARY && m->format != MOE_FORMAT_SIGN)
+  if (m->format != MOE_FORMAT_TERNARY && m->format != MOE_FORMAT_SIGN && m->format != MOE_FORMAT_E16)
     return fail(MOE_ERR_INVALID_ARG, "debug_matvec: unknown weight format %d", m->format);
+  if (m->format == MOE_FORMAT_E16 && (!m->codes || !aligned16(m->codes)))
+    return fail(MOE_ERR_INVALID_ARG, "debug_matvec: E16 codes missing or not 16-byte aligned");
   if ((rc = check_device())) return rc;
   return launch_debug_matvec(m, ntok, xq, xd, out, isum, static_cast<cudaStream_t>(stream));
 }

@@ -20,6 +20,7 @@ namespace bitmoe {
 constexpr int kBlock = 256;      // weights per ternary block
 constexpr int kBlockWords = 13;  // packed uint32 words per block
 constexpr int kSignWords = 8;    // uint32 words per block of 1-bit sign codes
+constexpr int kE16Words = 2;     // uint32 words of 4-bit sub-scale codes per block (two-level scales)
 constexpr int kPanel = 32;       // rows per interleaved panel
 constexpr int kQBlock = 32;      // activations per int8 block
 constexpr int kSubPerBlock = kBlock / kQBlock;  // 8 activation blocks per weight block

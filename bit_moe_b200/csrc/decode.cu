@@ -160,10 +160,10 @@ __device__ __forceinline__ int item_pair(const DecodeParams& P, const Item& item
 // n's 32 rows and requantizes them (one 32-block of a) to int8.
 // grid: (ffn/32, items), block: kGateUpWarps*32.
 // ---------------------------------------------------------------------------
-template <int NT, bool kSign>
+template <int NT, int kFmt>
 __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& item, int panel,
                                            unsigned char* smem) {
-  constexpr int kWords = WordsPerBlock<kSign>::value;
+  constexpr int kWords = WordsPerBlock<kFmt == MOE_FORMAT_SIGN>::value;
   const int H = P.hidden, F = P.ffn;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int* q4 = reinterpret_cast<int*>(smem);
@@ -190,7 +190,16 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
   for (int m = 0; m < 2; ++m)
 #pragma unroll
     for (int n = 0; n < NT; ++n) out[m][n] = 0.f;
-  panel_dot<2, NT, kSign>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, out);
+  if constexpr (kFmt == MOE_FORMAT_E16) {
+    // per-row fp16 anchors, 4-bit sub-scale codes per 16 weights
+    const size_t row = static_cast<size_t>(item.expert) * F + panel * kPanel + lane;
+    const uint32_t* const tc[2] = {P.gate_codes + pb0 * kE16Words * kPanel + lane,
+                                   P.up_codes + pb0 * kE16Words * kPanel + lane};
+    const float a16[2] = {f16_bits_to_f32(P.gate_scales[row]) * 0.0625f, f16_bits_to_f32(P.up_scales[row]) * 0.0625f};
+    panel_dot_e16<2, NT>(tw, tc, a16, warp, nb, kGateUpWarps, q4, d, out);
+  } else {
+    panel_dot<2, NT, kFmt == MOE_FORMAT_SIGN>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, out);
+  }
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -217,7 +226,7 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
 // Four CTAs per SM (at most 64 registers a thread): the items of a decode
 // batch are mostly single pairs, whose path needs few registers; the rare
 // 8-pair path spills a little.
-template <int NTMAX, bool kSign>
+template <int NTMAX, int kFmt>
 __global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
@@ -235,12 +244,12 @@ __global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P)
     return;
   }
   if constexpr (NTMAX == 1) {
-    gateup_run<1, kSign>(P, item, panel, smem);
+    gateup_run<1, kFmt>(P, item, panel, smem);
   } else {
-    if (item.count <= 1) gateup_run<1, kSign>(P, item, panel, smem);
-    else if (item.count <= 2) gateup_run<2, kSign>(P, item, panel, smem);
-    else if (item.count <= 4) gateup_run<4, kSign>(P, item, panel, smem);
-    else gateup_run<8, kSign>(P, item, panel, smem);
+    if (item.count <= 1) gateup_run<1, kFmt>(P, item, panel, smem);
+    else if (item.count <= 2) gateup_run<2, kFmt>(P, item, panel, smem);
+    else if (item.count <= 4) gateup_run<4, kFmt>(P, item, panel, smem);
+    else gateup_run<8, kFmt>(P, item, panel, smem);
   }
 }
 
@@ -270,10 +279,10 @@ __device__ __forceinline__ void arrive_and_combine(const DecodeParams& P, int pa
   }
 }
 
-template <int NT, bool kSign>
+template <int NT, int kFmt>
 __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item, int pgroup,
                                          unsigned char* smem) {
-  constexpr int kWords = WordsPerBlock<kSign>::value;
+  constexpr int kWords = WordsPerBlock<kFmt == MOE_FORMAT_SIGN>::value;
   const int H = P.hidden, F = P.ffn;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int* q4 = reinterpret_cast<int*>(smem);
@@ -297,7 +306,14 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
   float out[1][NT];
 #pragma unroll
   for (int n = 0; n < NT; ++n) out[0][n] = 0.f;
-  panel_dot<1, NT, kSign>(tw, ts, 0, nb, 1, q4, d, as, out);
+  if constexpr (kFmt == MOE_FORMAT_E16) {
+    const size_t row = static_cast<size_t>(item.expert) * H + panel * kPanel + lane;
+    const uint32_t* const tc[1] = {P.down_codes + pb0 * kE16Words * kPanel + lane};
+    const float a16[1] = {f16_bits_to_f32(P.down_scales[row]) * 0.0625f};
+    panel_dot_e16<1, NT>(tw, tc, a16, 0, nb, 1, q4, d, out);
+  } else {
+    panel_dot<1, NT, kFmt == MOE_FORMAT_SIGN>(tw, ts, 0, nb, 1, q4, d, as, out);
+  }
 #pragma unroll
   for (int n = 0; n < NT; ++n)
     if (n < item.count)
@@ -309,7 +325,7 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
 
 // Eight CTAs per SM (at most 64 registers a thread, which leaves room for the
 // prefetched next block of weight words in panel_dot).
-template <int NTMAX, bool kSign>
+template <int NTMAX, int kFmt>
 __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char smem[];
@@ -327,12 +343,12 @@ __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
     return;
   }
   if constexpr (NTMAX == 1) {
-    down_run<1, kSign>(P, item, pgroup, smem);
+    down_run<1, kFmt>(P, item, pgroup, smem);
   } else {
-    if (item.count <= 1) down_run<1, kSign>(P, item, pgroup, smem);
-    else if (item.count <= 2) down_run<2, kSign>(P, item, pgroup, smem);
-    else if (item.count <= 4) down_run<4, kSign>(P, item, pgroup, smem);
-    else down_run<8, kSign>(P, item, pgroup, smem);
+    if (item.count <= 1) down_run<1, kFmt>(P, item, pgroup, smem);
+    else if (item.count <= 2) down_run<2, kFmt>(P, item, pgroup, smem);
+    else if (item.count <= 4) down_run<4, kFmt>(P, item, pgroup, smem);
+    else down_run<8, kFmt>(P, item, pgroup, smem);
   }
 }
 
@@ -340,11 +356,11 @@ __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
 // Test hook: the mat-vec core on one matrix, with the exact block sums.
 // grid: (rows/32, ntok), block: kGateUpWarps*32; warps split the blocks.
 // ---------------------------------------------------------------------------
-template <bool kSign>
+template <int kFmt>
 __global__ void __launch_bounds__(kGateUpWarps * 32)
-    k_debug_matvec(const uint32_t* __restrict__ trits, const uint16_t* __restrict__ scales, int rows,
-                   int k, const int8_t* __restrict__ xq, const float* __restrict__ xd,
-                   float* __restrict__ out, int32_t* __restrict__ isum) {
+    k_debug_matvec(const uint32_t* __restrict__ trits, const uint16_t* __restrict__ scales,
+                   const uint32_t* __restrict__ codes, int rows, int k, const int8_t* __restrict__ xq,
+                   const float* __restrict__ xd, float* __restrict__ out, int32_t* __restrict__ isum) {
   extern __shared__ __align__(16) unsigned char smem[];
   int* q4 = reinterpret_cast<int*>(smem);
   float* d = reinterpret_cast<float*>(q4 + k / 4);
@@ -358,11 +374,17 @@ __global__ void __launch_bounds__(kGateUpWarps * 32)
   const int nb = k / kBlock;
   const int r = panel * kPanel + lane;
   const size_t pb0 = static_cast<size_t>(panel) * nb;
-  const uint32_t* const tw[1] = {trits + pb0 * WordsPerBlock<kSign>::value * kPanel + lane};
+  const uint32_t* const tw[1] = {trits + pb0 * WordsPerBlock<kFmt == MOE_FORMAT_SIGN>::value * kPanel + lane};
   const uint16_t* const ts[1] = {scales + pb0 * kPanel + lane};
   float o[1][1] = {{0.f}};
   int32_t* isum_row = isum ? isum + (static_cast<size_t>(t) * rows + r) * (k / kQBlock) : nullptr;
-  panel_dot<1, 1, kSign>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, o, isum_row, 0);
+  if constexpr (kFmt == MOE_FORMAT_E16) {
+    const uint32_t* const tc[1] = {codes + pb0 * kE16Words * kPanel + lane};
+    const float a16[1] = {f16_bits_to_f32(scales[r]) * 0.0625f};
+    panel_dot_e16<1, 1>(tw, tc, a16, warp, nb, kGateUpWarps, q4, d, o, isum_row, 0);
+  } else {
+    panel_dot<1, 1, kFmt == MOE_FORMAT_SIGN>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, o, isum_row, 0);
+  }
   red[warp * 32 + lane] = o[0][0];
   __syncthreads();
   if (warp == 0) {
@@ -384,16 +406,15 @@ static void init_kernel_attrs() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < kMaxDev && done[dev]) return;
-  const void* kernels[] = {reinterpret_cast<const void*>(&k_gateup<1, false>),
-                           reinterpret_cast<const void*>(&k_gateup<kChunk, false>),
-                           reinterpret_cast<const void*>(&k_down<1, false>),
-                           reinterpret_cast<const void*>(&k_down<kChunk, false>),
-                           reinterpret_cast<const void*>(&k_gateup<1, true>),
-                           reinterpret_cast<const void*>(&k_gateup<kChunk, true>),
-                           reinterpret_cast<const void*>(&k_down<1, true>),
-                           reinterpret_cast<const void*>(&k_down<kChunk, true>),
-                           reinterpret_cast<const void*>(&k_debug_matvec<false>),
-                           reinterpret_cast<const void*>(&k_debug_matvec<true>)};
+  const void* kernels[] = {
+      reinterpret_cast<const void*>(&k_gateup<1, 0>),     reinterpret_cast<const void*>(&k_gateup<kChunk, 0>),
+      reinterpret_cast<const void*>(&k_down<1, 0>),       reinterpret_cast<const void*>(&k_down<kChunk, 0>),
+      reinterpret_cast<const void*>(&k_gateup<1, 1>),     reinterpret_cast<const void*>(&k_gateup<kChunk, 1>),
+      reinterpret_cast<const void*>(&k_down<1, 1>),       reinterpret_cast<const void*>(&k_down<kChunk, 1>),
+      reinterpret_cast<const void*>(&k_gateup<1, 2>),     reinterpret_cast<const void*>(&k_gateup<kChunk, 2>),
+      reinterpret_cast<const void*>(&k_down<1, 2>),       reinterpret_cast<const void*>(&k_down<kChunk, 2>),
+      reinterpret_cast<const void*>(&k_debug_matvec<0>),  reinterpret_cast<const void*>(&k_debug_matvec<1>),
+      reinterpret_cast<const void*>(&k_debug_matvec<2>)};
   for (const void* k : kernels)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
   if (dev >= 0 && dev < kMaxDev) done[dev] = true;
@@ -415,22 +436,22 @@ int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cu
   return check_launch("topk_group");
 }
 
-template <bool kSign>
+template <int kFmt>
 static void launch_ffn_fmt(const DecodeParams& P, cudaStream_t stream) {
   const int npairs = P.ntok * P.top_k;
   if (P.direct) {
     const size_t s1 = ActSmem<1>::bytes(P.hidden) + 2 * kGateUpWarps * 1 * 32 * 4;
     const size_t s2 = ActSmem<1>::bytes(P.ffn);
-    launch_k(k_gateup<1, kSign>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
+    launch_k(k_gateup<1, kFmt>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
     note_launch(MOE_K_GATEUP, stream);
-    launch_k(k_down<1, kSign>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
+    launch_k(k_down<1, kFmt>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream, P);
     note_launch(MOE_K_DOWN, stream);
   } else {
     const size_t s1 = ActSmem<kChunk>::bytes(P.hidden) + 2 * kGateUpWarps * kChunk * 32 * 4;
     const size_t s2 = ActSmem<kChunk>::bytes(P.ffn);
-    launch_k(k_gateup<kChunk, kSign>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
+    launch_k(k_gateup<kChunk, kFmt>, dim3(P.ffn / kPanel, npairs), dim3(kGateUpWarps * 32), s1, stream, P);
     note_launch(MOE_K_GATEUP, stream);
-    launch_k(k_down<kChunk, kSign>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream,
+    launch_k(k_down<kChunk, kFmt>, dim3(P.hidden / kPanel / kDownWarps, npairs), dim3(kDownWarps * 32), s2, stream,
              P);
     note_launch(MOE_K_DOWN, stream);
   }
@@ -439,8 +460,9 @@ static void launch_ffn_fmt(const DecodeParams& P, cudaStream_t stream) {
 int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
   if (!P.direct && P.group_chunk != kChunk) return fail(MOE_ERR_INVALID_ARG, "expert_ffn: items of %d pairs", P.group_chunk);
   init_kernel_attrs();
-  if (P.format == MOE_FORMAT_SIGN) launch_ffn_fmt<true>(P, stream);
-  else launch_ffn_fmt<false>(P, stream);
+  if (P.format == MOE_FORMAT_SIGN) launch_ffn_fmt<MOE_FORMAT_SIGN>(P, stream);
+  else if (P.format == MOE_FORMAT_E16) launch_ffn_fmt<MOE_FORMAT_E16>(P, stream);
+  else launch_ffn_fmt<MOE_FORMAT_TERNARY>(P, stream);
   return check_launch("expert_ffn");
 }
 
@@ -450,9 +472,14 @@ int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const flo
   const size_t s = ActSmem<1>::bytes(m->k) + kGateUpWarps * 32 * 4;
   const dim3 grid(m->rows / kPanel, ntok);
   if (m->format == MOE_FORMAT_SIGN)
-    k_debug_matvec<true><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
+    k_debug_matvec<1><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, nullptr, m->rows, m->k, xq, xd,
+                                                             out, isum);
+  else if (m->format == MOE_FORMAT_E16)
+    k_debug_matvec<2><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, m->codes, m->rows, m->k, xq, xd,
+                                                             out, isum);
   else
-    k_debug_matvec<false><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, m->rows, m->k, xq, xd, out, isum);
+    k_debug_matvec<0><<<grid, kGateUpWarps * 32, s, stream>>>(m->trits, m->scales, nullptr, m->rows, m->k, xq, xd,
+                                                             out, isum);
   note_launch(MOE_K_DEBUG_MATVEC, stream);
   return check_launch("debug_matvec");
 }

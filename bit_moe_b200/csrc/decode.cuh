@@ -31,7 +31,10 @@ struct DecodeParams {
   int32_t* status;
   // grouped mode (ntok > 1): items and the pair list, built on the device
   int direct;                            // 1: item i is pair i (ntok == 1)
-  int format;                            // MOE_FORMAT_TERNARY or MOE_FORMAT_SIGN
+  int format;                            // MOE_FORMAT_TERNARY, _SIGN or _E16
+  const uint32_t* gate_codes;            // MOE_FORMAT_E16: 4-bit sub-scale words (the
+  const uint32_t* up_codes;              // *_scales pointers then hold per-row anchors)
+  const uint32_t* down_codes;
   const Item* items;                     // [ntok*top_k + n_experts]
   const int32_t* n_items;
   const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert

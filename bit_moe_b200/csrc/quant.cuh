@@ -5,6 +5,10 @@ namespace bitmoe {
 // sign: 1-bit sign codes (MOE_FORMAT_SIGN) instead of ternary digits.
 int launch_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trits,
                             uint16_t* scales, cudaStream_t stream, bool sign = false);
+// Two-level scales (MOE_FORMAT_E16): the per-row anchors, then the digits
+// and the 4-bit sub-scale codes.
+int launch_quantize_weights_e16(const float* w, int64_t rows, int64_t k, uint32_t* trits, uint32_t* codes,
+                                uint16_t* anchors, cudaStream_t stream);
 int launch_quant_act_q8(const float* x, int64_t ntok, int k, int8_t* xq, float* xd,
                         cudaStream_t stream);
 

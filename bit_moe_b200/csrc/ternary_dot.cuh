@@ -215,6 +215,111 @@ __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
   }
 }
 
+// Two-level (E16) scales (pxq_llama README, "What's PXQ?": a per-row fp16
+// anchor A plus a 4-bit sub-scale per 16-element block): the ternary digits
+// of panel_dot, and per 16-weight block h a code c_h with scale
+// A * (c_h + 1) / 16.  Per 16-block the exact sum q.a = t.a - sum a is
+// weighted by c_h + 1 (the activations' 16-sums come from dp4a against
+// 0x01010101), per 32-block the weighted integer sum is scaled by the
+// activation scale, and A / 16 (a16[m], exact) is applied once at the end.
+//   tw[m]: digit words of matrix m at (panel, block 0), offset by lane
+//   tc[m]: code words at (panel, block 0), offset by lane (kE16Words a block)
+// If isum_out is not null (NM == 1), the weighted block sums
+// sum_h (c_h + 1) * sum_{k in h} q * xq of every 32-block s are stored at
+// isum_out[n * isum_stride + s].
+template <int NM, int NT>
+__device__ __forceinline__ void panel_dot_e16(const uint32_t* const (&tw)[NM], const uint32_t* const (&tc)[NM],
+                                              const float (&a16)[NM], int b_begin, int b_end, int b_step,
+                                              const int* __restrict__ q4, const float* __restrict__ d,
+                                              float (&out)[NM][NT], int32_t* isum_out = nullptr,
+                                              size_t isum_stride = 0) {
+  float tot[NM][NT];
+#pragma unroll
+  for (int m = 0; m < NM; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) tot[m][n] = 0.f;
+  for (int b = b_begin; b < b_end; b += b_step) {
+    uint32_t w[NM][kBlockWords];
+    uint32_t cw[NM][kE16Words];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) {
+      const uint32_t* src = tw[m] + static_cast<size_t>(b) * kBlockWords * kPanel;
+#pragma unroll
+      for (int j = 0; j < kBlockWords; ++j) w[m][j] = ld_stream_u32(src + j * kPanel);
+#pragma unroll
+      for (int u = 0; u < kE16Words; ++u) cw[m][u] = ld_stream_u32(tc[m] + (static_cast<size_t>(b) * kE16Words + u) * kPanel);
+    }
+    int acc[NM][NT], accw[NM][NT], as16[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      as16[n] = 0;
+#pragma unroll
+      for (int m = 0; m < NM; ++m) { acc[m][n] = 0; accw[m][n] = 0; }
+    }
+    const int* qb = q4 + b * (kBlock / 4) * NT;
+#pragma unroll
+    for (int j = 0; j < kBlockWords; ++j) {
+      uint32_t lo[NM], hi[NM], hp[NM];
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        lo[m] = w[m][j] & 0x00FF00FFu;
+        hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
+        hp[m] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        if (j == kBlockWords - 1 && i == 4) break;  // pad digit of the last word
+        const int g = 5 * j + i;                    // group of 4 weights, 0..63
+        int a[NT];
+        load_group<NT>(qb, g, a);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) as16[n] = __dp4a(a[n], 0x01010101, as16[n]);
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+          lo[m] *= 3u;
+          hi[m] *= 3u;
+          const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
+          const int t = static_cast<int>(hn - 3u * hp[m]);
+          hp[m] = hn;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) acc[m][n] = __dp4a(t, a[n], acc[m][n]);
+        }
+        if ((g & 3) == 3) {  // a 16-weight block h = g / 4 is complete
+          const int h = g >> 2;
+#pragma unroll
+          for (int m = 0; m < NM; ++m) {
+            const int cm = static_cast<int>((cw[m][h >> 3] >> (4 * (h & 7))) & 15u) + 1;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              accw[m][n] += cm * (acc[m][n] - as16[n]);
+              acc[m][n] = 0;
+            }
+          }
+#pragma unroll
+          for (int n = 0; n < NT; ++n) as16[n] = 0;
+        }
+        if ((g & 7) == 7) {  // a 32-weight activation block is complete
+          const int s = b * kSubPerBlock + (g >> 3);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const float dn = d[s * NT + n];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+              tot[m][n] = __fmaf_rn(dn, static_cast<float>(accw[m][n]), tot[m][n]);
+              if (NM == 1 && isum_out) isum_out[n * isum_stride + s] = accw[m][n];
+              accw[m][n] = 0;
+            }
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NM; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) out[m][n] = __fmaf_rn(a16[m], tot[m][n], out[m][n]);
+}
+
 // Stage activation vector n (k int8 codes with k/32 scales) into the
 // token-minor shared layout; threads [tid0, tid0+nthr) take part.  The block
 // sums are computed here from the codes.

@@ -49,6 +49,17 @@
  * l = 0..3), a set bit meaning +1; word j of block b of row r is
  * codes[((r/32 * nb + b) * 8 + j) * 32 + r%32].  34 bytes per 256 weights
  * (1.0625 bits per weight).
+ *
+ * Two-level scales (MOE_FORMAT_E16; pxq_llama README, "What's PXQ?": a
+ * per-row fp16 anchor plus a 4-bit sub-scale per 16-element block): the
+ * ternary digits above, with per row an fp16 anchor A (in `scales`, one per
+ * row) and per 16-weight block h a 4-bit code c_h (in `codes`: word u of
+ * block b of row r is codes[((r/32 * nb + b) * 2 + u) * 32 + r%32], block
+ * 8u + v in bits 4v..4v+3), the block's scale being A * (c_h + 1) / 16.
+ * Quantization (moe_quantize_weights_e16): A = fp16(max over the row's
+ * 16-blocks of mean|w|), c_h = clamp(rint(16 * mean_h / A) - 1, 0, 15),
+ * q = sign(w) where |w| >= s_h / 2, else 0.  60 bytes per 256 weights plus
+ * 2 bytes per row.
  */
 #ifndef BITMOE_H
 #define BITMOE_H
@@ -75,7 +86,7 @@ typedef enum {
 } moe_status;
 
 /* Weight formats. */
-typedef enum { MOE_FORMAT_TERNARY = 0, MOE_FORMAT_SIGN = 1 } moe_format;
+typedef enum { MOE_FORMAT_TERNARY = 0, MOE_FORMAT_SIGN = 1, MOE_FORMAT_E16 = 2 } moe_format;
 
 /* One packed matrix in one of the storage formats above. */
 typedef struct {
@@ -84,17 +95,20 @@ typedef struct {
   const uint32_t* trits; /* the packed words, device: moe_trit_words(rows, k)
                             base-3 words, or moe_sign_words(rows, k) sign
                             words for MOE_FORMAT_SIGN                */
-  const uint16_t* scales;/* moe_scale_count(rows, k) fp16, device   */
+  const uint16_t* scales;/* moe_scale_count(rows, k) fp16, device, or
+                            one fp16 anchor per row for MOE_FORMAT_E16 */
   int32_t format;        /* a moe_format                             */
+  const uint32_t* codes; /* MOE_FORMAT_E16: moe_e16_code_words(rows, k)
+                            sub-scale words, device; else unused      */
 } moe_tmat;
 
 /* One MoE layer.  Expert e owns rows [e*ffn, (e+1)*ffn) of gate and up
  * (k = hidden) and rows [e*hidden, (e+1)*hidden) of down (k = ffn).  The
  * three matrices share one format.  Limits: hidden and ffn multiples of 256,
  * hidden <= 16384, ffn <= 8192, 1 <= top_k <= min(n_experts, 32),
- * n_experts <= 1024.  Sign-code layers run the decode path only: up to 64
- * tokens per call (moe_expert_ffn_prefill, and moe_forward of more than 64
- * tokens, return MOE_ERR_UNSUPPORTED_SHAPE for them).                      */
+ * n_experts <= 1024.  Sign-code and E16 layers run the decode path only: up
+ * to 64 tokens per call (moe_expert_ffn_prefill, and moe_forward of more than
+ * 64 tokens, return MOE_ERR_UNSUPPORTED_SHAPE for them).                   */
 typedef struct {
   int32_t hidden, ffn, n_experts, top_k;
   moe_tmat gate, up, down;
@@ -103,6 +117,7 @@ typedef struct {
 /* ---- sizes ------------------------------------------------------------ */
 size_t moe_trit_words(int64_t rows, int64_t k);  /* rows*(k/256)*13 */
 size_t moe_sign_words(int64_t rows, int64_t k);  /* rows*(k/256)*8  */
+size_t moe_e16_code_words(int64_t rows, int64_t k); /* rows*(k/256)*2 */
 size_t moe_scale_count(int64_t rows, int64_t k); /* rows*(k/256)    */
 /* Bytes of workspace a decode (prefill = 0) or prefill (prefill = 1) call
  * of `ntok` tokens, or moe_forward, needs.  0 on invalid arguments.        */
@@ -123,6 +138,11 @@ int moe_quantize_weights(const float* w, int64_t rows, int64_t k, uint32_t* trit
  * where w < 0, else +1 (see the storage format above).                    */
 int moe_quantize_weights_sign(const float* w, int64_t rows, int64_t k, uint32_t* codes,
                               uint16_t* scales, moe_stream_t stream);
+/* The same to ternary digits with two-level scales (MOE_FORMAT_E16): trits
+ * as moe_quantize_weights' (digits of the E16 quantization), codes
+ * [moe_e16_code_words(rows, k)], anchors [rows] fp16.                     */
+int moe_quantize_weights_e16(const float* w, int64_t rows, int64_t k, uint32_t* trits,
+                             uint32_t* codes, uint16_t* anchors, moe_stream_t stream);
 
 /* ---- S1: activation quantization (Parakon Runtime README, "How it works":
  *      int8-quantized activations; pxq_llama README, "PXQ vs MXFP4": one

@@ -38,7 +38,8 @@ class Workload:
     layers: int = 1          # layers in the stack the benchmark rotates through
     prefill: bool = False
     seed: int = 0
-    fmt: str = "ternary"     # packed weight format: "ternary" or "sign" (1-bit sign codes)
+    fmt: str = "ternary"     # packed weight format: "ternary", "sign" (1-bit sign codes) or
+                             # "e16" (ternary digits with two-level scales)
 
     def with_(self, **kw):
         return replace(self, **kw)
@@ -46,16 +47,21 @@ class Workload:
     @property
     def block_bytes(self):
         """Packed bytes per 256 weights: 52 B of base-3 digits or 32 B of sign
-        bits, plus the 2-byte scale."""
-        return 34 if self.fmt == "sign" else 54
+        bits, plus the 2-byte scale (e16: 8 bytes of 4-bit sub-scales instead,
+        the 2-byte anchor being per row)."""
+        return {"sign": 34, "e16": 60}.get(self.fmt, 54)
+
+    def matrix_bytes(self, rows, k):
+        """Packed bytes of a [rows][k] matrix in this workload's format."""
+        return rows * (k // 256) * self.block_bytes + (2 * rows if self.fmt == "e16" else 0)
 
     @property
     def expert_bytes(self):
         """Packed bytes of one expert's gate+up+down."""
-        return 3 * self.hidden * self.ffn // 256 * self.block_bytes
+        return 2 * self.matrix_bytes(self.ffn, self.hidden) + self.matrix_bytes(self.hidden, self.ffn)
 
     def describe(self):
-        return "%s%s-t%d%s" % (self.name, "-sign" if self.fmt == "sign" else "", self.ntok,
+        return "%s%s-t%d%s" % (self.name, "" if self.fmt == "ternary" else "-" + self.fmt, self.ntok,
                                "-prefill" if self.prefill else "")
 
 
@@ -74,6 +80,11 @@ WORKLOADS = {
                          fmt="sign"),
     "large-sign-b8": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 8, 0.015, layers=5,
                               seed=6, fmt="sign"),
+    # and with ternary digits under two-level (per-row anchor, per-16 sub-scale) scales
+    "30b-e16": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 1, 0.02, layers=4, seed=7,
+                        fmt="e16"),
+    "large-e16-b8": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 8, 0.015, layers=5,
+                             seed=8, fmt="e16"),
     # prefill of 2048 tokens through the 30B-class layer
     "30b-prefill": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 2048, 0.02,
                             layers=1, prefill=True, seed=4),

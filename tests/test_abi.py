@@ -76,4 +76,11 @@ def test_sign_format_host_side_without_device():
     rc = L.moe_forward(ctypes.byref(bad), x, 1, x, x, x, 1 << 30, None)
     assert rc == -1 and b"format" in L.moe_last_error()
     # the binding's struct matches the header's field order
-    assert [f[0] for f in B.moe_tmat._fields_] == ["rows", "k", "trits", "scales", "format"]
+    assert [f[0] for f in B.moe_tmat._fields_] == ["rows", "k", "trits", "scales", "format", "codes"]
+    assert L.moe_e16_code_words(64, 512) == 64 * 2 * 2
+    # a two-level-scale layer without its sub-scale codes is rejected
+    nocodes = B.moe_layer(256, 256, 2, 1, tm(512, 256, 2), tm(512, 256, 2), tm(512, 256, 2))
+    rc = L.moe_forward(ctypes.byref(nocodes), x, 1, x, x, x, 1 << 30, None)
+    assert rc == -1 and b"codes" in L.moe_last_error()
+    rc = L.moe_quantize_weights_e16(p, 32, 200, p, p, p, None)
+    assert rc == -2
