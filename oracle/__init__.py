@@ -64,6 +64,12 @@ def lib():
         L.orc_unpack_weights_e16.argtypes = [p, p, p, i64, i64, i64, i64, p, p]
         L.orc_matvec_e16.restype = None
         L.orc_matvec_e16.argtypes = [p, p, i64, i64, p, p, p]
+        L.orc_quantize_weights_q8.restype = ctypes.c_int
+        L.orc_quantize_weights_q8.argtypes = [p, i64, i64, p, p]
+        L.orc_matvec_q8.restype = None
+        L.orc_matvec_q8.argtypes = [p, p, i64, i64, p, p, p]
+        L.orc_shared_ffn.restype = ctypes.c_int
+        L.orc_shared_ffn.argtypes = [i64, i64, p, p, p, p, p, p, i64, p, p, p]
         L.orc_unpack_weights.restype = ctypes.c_int
         L.orc_unpack_weights.argtypes = [p, p, i64, i64, i64, i64, p, p]
         L.orc_quant_act_q8.restype = ctypes.c_int
@@ -253,6 +259,47 @@ def matvec_e16(q, s16, xq, xd):
     return out
 
 
+# ---------------------------------------------------------------- shared expert (q8 blocks)
+def quantize_weights_q8(w):
+    """w [rows][k] fp32 -> (q int8 [rows][k], d uint16 fp16 bits [rows][k/32])."""
+    w = _c(w, np.float32)
+    rows, k = w.shape
+    q = np.zeros((rows, k), dtype=np.int8)
+    d = np.zeros((rows, k // QBLOCK), dtype=np.uint16)
+    if lib().orc_quantize_weights_q8(_ptr(w), rows, k, _ptr(q), _ptr(d)):
+        raise ValueError("orc_quantize_weights_q8: bad shape %r" % (w.shape,))
+    return q, d
+
+
+def matvec_q8(q, d, xq, xd):
+    q, d = _c(q, np.int8), _c(d, np.uint16)
+    rows, k = q.shape
+    out = np.zeros(rows, dtype=np.float64)
+    lib().orc_matvec_q8(_ptr(q), _ptr(d), rows, k, _ptr(_c(xq, np.int8)), _ptr(_c(xd, np.float32)), _ptr(out))
+    return out
+
+
+class SharedExpert:
+    """The shared expert in q8 blocks: gate/up [ffn][hidden], down [hidden][ffn]."""
+
+    def __init__(self, hidden, ffn, wg, wu, wd):
+        self.hidden, self.ffn = hidden, ffn
+        self.gate, self.up, self.down = quantize_weights_q8(wg), quantize_weights_q8(wu), quantize_weights_q8(wd)
+
+    def add_to(self, y, xq, xd):
+        """y [ntok][hidden] fp64 += the shared expert's FFN of the tokens."""
+        xq, xd = _c(xq, np.int8), _c(xd, np.float32)
+        if xq.ndim == 1:
+            xq, xd = xq[None], xd[None]
+        y = np.ascontiguousarray(y, dtype=np.float64)
+        (gq, gd), (uq, ud), (dq, dd) = self.gate, self.up, self.down
+        rc = lib().orc_shared_ffn(self.hidden, self.ffn, _ptr(gq), _ptr(gd), _ptr(uq), _ptr(ud), _ptr(dq),
+                                  _ptr(dd), xq.shape[0], _ptr(xq), _ptr(xd), _ptr(y))
+        if rc:
+            raise ValueError("orc_shared_ffn: bad shape")
+        return y
+
+
 # ---------------------------------------------------------------- activations
 def quant_act_q8(x):
     """x [ntok][k] fp32 -> (xq int8 [ntok][k], xd fp32 [ntok][k/32])."""
@@ -388,8 +435,9 @@ def expert_ffn(layer, xq, xd, idx, wts, debug=False):
     return (y, dbg) if debug else y
 
 
-def moe_forward(layer, wr, x, debug=False):
-    """The whole decode step on the CPU: act quant, router, expert FFN.
+def moe_forward(layer, wr, x, debug=False, shared=None):
+    """The whole decode step on the CPU: act quant, router, expert FFN, and
+    the shared expert's FFN added when `shared` (a SharedExpert) is given.
 
     Returns y fp64 [ntok][hidden], idx, wts (fp64) and, with debug, the
     intermediates.
@@ -397,8 +445,11 @@ def moe_forward(layer, wr, x, debug=False):
     xq, xd = quant_act_q8(x)
     idx, wts = route_topk(x, wr, layer.top_k)
     out = expert_ffn(layer, xq, xd, idx, wts.astype(np.float32), debug=debug)
+    y = out[0] if debug else out
+    if shared is not None:
+        y = shared.add_to(y, xq, xd)
     if debug:
-        y, dbg = out
+        dbg = out[1]
         dbg.update(xq=xq, xd=xd)
         return y, idx, wts, dbg
-    return out, idx, wts
+    return y, idx, wts

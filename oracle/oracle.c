@@ -618,3 +618,80 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
   free(g); free(u); free(a); free(aq); free(ad); free(ye);
   return rc;
 }
+
+/* ======================================================================== */
+/* shared expert (8-bit blocks)                                              */
+/* ======================================================================== */
+/* The shared expert beside the routed ones stays at higher precision
+   (llama-modchip page, "The interesting bit"); read here as 8-bit blocks of
+   32 weights with an fp16 scale (see oracle.h).                           */
+int orc_quantize_weights_q8(const float* w, int64_t rows, int64_t k, int8_t* q,
+                            uint16_t* d) {
+  if (rows <= 0 || k <= 0 || k % ORC_QBLOCK) return -1;
+  int64_t nq = k / ORC_QBLOCK;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t j = 0; j < nq; ++j) {
+      const float* wb = w + r * k + j * ORC_QBLOCK;
+      double amax = 0.0;
+      for (int i = 0; i < ORC_QBLOCK; ++i) {
+        double a = fabs((double)wb[i]);
+        if (a > amax) amax = a;
+      }
+      uint16_t dh = orc_f16_from_f64(amax / 127.0);
+      d[r * nq + j] = dh;
+      float df = orc_f16_to_f32(dh);
+      for (int i = 0; i < ORC_QBLOCK; ++i) {
+        int8_t v = 0;
+        if (df != 0.0f) {
+          float t = rintf(wb[i] / df);
+          if (t > 127.0f) t = 127.0f;
+          if (t < -127.0f) t = -127.0f;
+          v = (int8_t)t;
+        }
+        q[r * k + j * ORC_QBLOCK + i] = v;
+      }
+    }
+  }
+  return 0;
+}
+
+void orc_matvec_q8(const int8_t* q, const uint16_t* d, int64_t rows, int64_t k,
+                   const int8_t* xq, const float* xd, double* out) {
+  int64_t nq = k / ORC_QBLOCK;
+  for (int64_t r = 0; r < rows; ++r) {
+    double acc = 0.0;
+    for (int64_t j = 0; j < nq; ++j) {
+      int32_t isum = 0;
+      for (int i = 0; i < ORC_QBLOCK; ++i)
+        isum += (int32_t)q[r * k + j * ORC_QBLOCK + i] * (int32_t)xq[j * ORC_QBLOCK + i];
+      acc += (double)orc_f16_to_f32(d[r * nq + j]) * (double)xd[j] * (double)isum;
+    }
+    out[r] = acc;
+  }
+}
+
+int orc_shared_ffn(int64_t hidden, int64_t ffn, const int8_t* gq, const uint16_t* gd,
+                   const int8_t* uq, const uint16_t* ud, const int8_t* dq,
+                   const uint16_t* dd, int64_t ntok, const int8_t* xq,
+                   const float* xd, double* y) {
+  int64_t H = hidden, F = ffn;
+  if (H <= 0 || F <= 0 || H % ORC_QBLOCK || F % ORC_QBLOCK) return -1;
+  double* g = (double*)malloc(sizeof(double) * (size_t)F);
+  double* u = (double*)malloc(sizeof(double) * (size_t)F);
+  float* a = (float*)malloc(sizeof(float) * (size_t)F);
+  int8_t* aq = (int8_t*)malloc((size_t)F);
+  float* ad = (float*)malloc(sizeof(float) * (size_t)(F / ORC_QBLOCK));
+  double* ys = (double*)malloc(sizeof(double) * (size_t)H);
+  for (int64_t t = 0; t < ntok; ++t) {
+    const int8_t* xt = xq + t * H;
+    const float* dt = xd + t * (H / ORC_QBLOCK);
+    orc_matvec_q8(gq, gd, F, H, xt, dt, g);
+    orc_matvec_q8(uq, ud, F, H, xt, dt, u);
+    for (int64_t f = 0; f < F; ++f) a[f] = (float)(g[f] / (1.0 + exp(-g[f])) * u[f]);
+    orc_quant_act_q8(a, 1, F, aq, ad);
+    orc_matvec_q8(dq, dd, H, F, aq, ad, ys);
+    for (int64_t h = 0; h < H; ++h) y[t * H + h] += ys[h];
+  }
+  free(g); free(u); free(a); free(aq); free(ad); free(ys);
+  return 0;
+}

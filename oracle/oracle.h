@@ -182,6 +182,30 @@ int orc_expert_ffn(const orc_layer* L, int64_t ntok, const int8_t* xq,
                    double* y, double* g_out, double* u_out, int8_t* aq_out,
                    float* ad_out);
 
+/* ---- shared expert ---------------------------------------------------------- */
+/* The shared expert kept at higher precision beside the low-bit routed
+ * experts (llama-modchip page, "The interesting bit": shared experts stay in
+ * 4/5-bit or float formats while the routed experts go to 1-bit).  Reading:
+ * 8-bit blocks of 32 weights (the Q8_0 layout of the pxq_llama tensor census,
+ * "Full census"): per block d = fp16_RNE(amax / 127, in fp64) and
+ * q = clamp(rint(w / d), -127, 127) (fp32 division by the fp16 value; a block
+ * whose d is 0 is all zeros); stored row-major: q [rows][k] int8,
+ * d [rows][k/32] fp16.  Its FFN output is added to every token's routed sum
+ * with weight 1.                                                           */
+int orc_quantize_weights_q8(const float* w, int64_t rows, int64_t k, int8_t* q,
+                            uint16_t* d);
+/* out[r] = sum_j d_w[r][j] * xd[j] * sum_{k in block j} q[r][k] * xq[k],
+ * in fp64.                                                                */
+void orc_matvec_q8(const int8_t* q, const uint16_t* d, int64_t rows, int64_t k,
+                   const int8_t* xq, const float* xd, double* out);
+/* y[t] += Wd_s . q8(silu(Wg_s . x^_t) * Wu_s . x^_t)^ for t < ntok (fp64),
+ * gate/up [ffn][hidden], down [hidden][ffn], all in the q8 block format.
+ * Returns 0, or -1 on a bad shape (hidden, ffn multiples of 32).          */
+int orc_shared_ffn(int64_t hidden, int64_t ffn, const int8_t* gq, const uint16_t* gd,
+                   const int8_t* uq, const uint16_t* ud, const int8_t* dq,
+                   const uint16_t* dd, int64_t ntok, const int8_t* xq,
+                   const float* xd, double* y);
+
 #ifdef __cplusplus
 }
 #endif
