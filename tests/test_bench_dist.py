@@ -45,3 +45,25 @@ def test_single_rank_is_local():
     import bench
     assert bench.max_over_ranks(7.0, 1) == 7.0
     assert bench.job_rate(10, 1, 5.0) == pytest.approx(2000.0)
+
+
+@pytest.mark.parametrize("workload", ["tiny", "30b-sign", "30b-e16"])
+def test_reference_arm_json_line(workload):
+    """`bench.py --impl reference` runs the oracle on the host and prints one
+    JSON line with the contract's keys, its cpu_baseline and e2e equal to the
+    line's own value."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--workload", workload, "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=600, check=True).stdout
+    line = json.loads(out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 1
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["workload"].startswith("moe-")
