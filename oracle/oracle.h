@@ -19,7 +19,11 @@
  *   - all top-k experts of a token are evaluated, none dropped
  *     (llama-modchip page, "Key highlights");
  *   - the expert FFN is gate/up with a SiLU unary, then down (pxq_llama README,
- *     "Updates -- 2026-07-28", the up_gate_unary item).
+ *     "Updates -- 2026-07-28", the up_gate_unary item);
+ *   - two more routed-weight formats of the pxq_llama README ("What's PXQ?"):
+ *     1-bit sign codes, and two-level (E16) scales on the ternary digits;
+ *   - a shared expert kept at higher precision beside the routed ones
+ *     (llama-modchip page, "The interesting bit"), in 8-bit blocks.
  * Every other detail is a reading of those passages; each function below says
  * which.
  *
