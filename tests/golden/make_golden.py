@@ -58,6 +58,41 @@ def main():
         json.dump(out, f, indent=1)
     print("wrote", path)
 
+    path = os.path.join(HERE, "tiny_layer_formats.json")
+    with open(path, "w") as f:
+        json.dump(formats_case(), f, indent=1)
+    print("wrote", path)
+
+
+def shared_expert(wl):
+    """A seeded shared expert of the tiny layer's width (ffn 256)."""
+    rng = np.random.default_rng(99)
+    fs = 256
+    return oracle.SharedExpert(wl.hidden, fs,
+                               (rng.standard_normal((fs, wl.hidden)) * 0.02).astype(np.float32),
+                               (rng.standard_normal((fs, wl.hidden)) * 0.02).astype(np.float32),
+                               (rng.standard_normal((wl.hidden, fs)) * 0.02).astype(np.float32))
+
+
+def formats_case():
+    """The tiny layer in the sign-code and E16 formats, and the ternary layer
+    with a shared expert: packed digests and outputs."""
+    wl, wg, wu, wd, wr, x = tiny_case()
+    out = {"what": "oracle outputs of the tiny layer of tiny_layer.json in the 1-bit sign-code and "
+                   "two-level (E16) formats, and of the ternary layer with a seeded 8-bit shared "
+                   "expert (ffn 256, weights N(0, 0.02) from numpy's default_rng(99))"}
+    for fmt in ("sign", "e16"):
+        layer = oracle.Layer.from_float(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, wg, wu, wd, fmt=fmt)
+        y, idx, _ = oracle.moe_forward(layer, wr, x)
+        out[fmt] = {"packed_sha256": digest(*layer.gate, *layer.up, *layer.down),
+                    "idx": idx.tolist(), "y": [[float(v) for v in row] for row in y]}
+    layer = oracle.Layer.from_float(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, wg, wu, wd)
+    sh = shared_expert(wl)
+    y, idx, _ = oracle.moe_forward(layer, wr, x, shared=sh)
+    out["shared"] = {"packed_sha256": digest(*sh.gate, *sh.up, *sh.down),
+                     "y": [[float(v) for v in row] for row in y]}
+    return out
+
 
 if __name__ == "__main__":
     main()

@@ -1,4 +1,5 @@
-"""The oracle reproduces its stored outputs (tests/golden/tiny_layer.json)."""
+"""The oracle reproduces its stored outputs (tests/golden/tiny_layer.json and
+tests/golden/tiny_layer_formats.json)."""
 import json
 import os
 import sys
@@ -26,3 +27,14 @@ def test_tiny_layer_golden(orc):
     assert idx.tolist() == gold["idx"]
     assert np.array_equal(wts, np.array(gold["wts"]))
     assert np.array_equal(y, np.array(gold["y"]))
+
+
+def test_tiny_layer_formats_golden(orc):
+    with open(os.path.join(HERE, "golden", "tiny_layer_formats.json")) as f:
+        gold = json.load(f)
+    got = make_golden.formats_case()
+    for key in ("sign", "e16", "shared"):
+        assert got[key]["packed_sha256"] == gold[key]["packed_sha256"], key
+        assert np.array_equal(np.array(got[key]["y"]), np.array(gold[key]["y"])), key
+    for key in ("sign", "e16"):
+        assert got[key]["idx"] == gold[key]["idx"]
