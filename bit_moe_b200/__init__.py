@@ -35,6 +35,7 @@ EXPORTS = (
     "moe_check_status", "moe_last_error", "moe_debug_matvec", "moe_launch_count",
     "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
     "moe_sign_words", "moe_quantize_weights_sign", "moe_e16_code_words", "moe_quantize_weights_e16",
+    "moe_quantize_weights_q8", "moe_shared_workspace_bytes", "moe_shared_ffn_add",
 )
 
 
@@ -51,6 +52,13 @@ class moe_tmat(ctypes.Structure):
 
 
 FORMATS = {"ternary": 0, "sign": 1, "e16": 2}   # moe_format
+
+
+class moe_shared(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("gate_q", ctypes.c_void_p), ("gate_d", ctypes.c_void_p),
+                ("up_q", ctypes.c_void_p), ("up_d", ctypes.c_void_p),
+                ("down_q", ctypes.c_void_p), ("down_d", ctypes.c_void_p)]
 
 
 class moe_layer(ctypes.Structure):
@@ -81,6 +89,9 @@ def lib():
             "moe_quantize_weights": (ctypes.c_int, [p, i64, i64, p, p, p]),
             "moe_quantize_weights_sign": (ctypes.c_int, [p, i64, i64, p, p, p]),
             "moe_quantize_weights_e16": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
+            "moe_quantize_weights_q8": (ctypes.c_int, [p, i64, i64, p, p, p]),
+            "moe_shared_workspace_bytes": (sz, [p, i32]),
+            "moe_shared_ffn_add": (ctypes.c_int, [p, i32, p, p, p, p, sz, p]),
             "moe_quant_act_q8": (ctypes.c_int, [p, i32, i32, p, p, p]),
             "moe_route_topk": (ctypes.c_int, [p, p, i32, i32, i32, i32, p, p, p, sz, p]),
             "moe_route_workspace_bytes": (sz, [i32, i32]),
@@ -210,6 +221,47 @@ def moe_quantize_weights_e16(w, out=None, stream=None):
                                           ctypes.c_void_p(m.codes.data_ptr()),
                                           ctypes.c_void_p(m.scales.data_ptr()), _stream(stream)))
     return m
+
+
+def moe_quantize_weights_q8(w, stream=None):
+    """w [rows][k] fp32 CUDA -> (q int8 [rows][k], d int16 view of fp16 [rows][k/32])."""
+    rows, k = w.shape
+    q = torch.empty((rows, k), dtype=torch.int8, device=w.device)
+    d = torch.empty((rows, k // QBLOCK), dtype=torch.int16, device=w.device)
+    _check(lib().moe_quantize_weights_q8(_dev(w, torch.float32, "w"), rows, k, ctypes.c_void_p(q.data_ptr()),
+                                         ctypes.c_void_p(d.data_ptr()), _stream(stream)))
+    return q, d
+
+
+class SharedExpert:
+    """The shared expert in 8-bit blocks (gate/up [ffn][hidden], down
+    [hidden][ffn]), quantized from fp32 CUDA tensors."""
+
+    def __init__(self, wg, wu, wd, stream=None):
+        self.ffn, self.hidden = wg.shape
+        self.gate = moe_quantize_weights_q8(wg.contiguous(), stream)
+        self.up = moe_quantize_weights_q8(wu.contiguous(), stream)
+        self.down = moe_quantize_weights_q8(wd.contiguous(), stream)
+        self._c = moe_shared(self.hidden, self.ffn, *[t.data_ptr() for m in (self.gate, self.up, self.down) for t in m])
+
+    def c_ref(self):
+        return ctypes.byref(self._c)
+
+    def workspace(self, ntok, device="cuda"):
+        n = lib().moe_shared_workspace_bytes(self.c_ref(), ntok)
+        if n == 0:
+            _check(-1)
+        return torch.empty(int(n), dtype=torch.uint8, device=device)
+
+    def add(self, xq, xd, y, ws=None, stream=None):
+        """y [ntok][hidden] += the shared expert's FFN of (xq, xd); returns y."""
+        ntok = xq.shape[0]
+        if ws is None:
+            ws = self.workspace(ntok, y.device)
+        _check(lib().moe_shared_ffn_add(self.c_ref(), ntok, _dev(xq, torch.int8, "xq"), _dev(xd, torch.float32, "xd"),
+                                        _dev(y, torch.float32, "y"), ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                        _stream(stream)))
+        return y
 
 
 class MoELayer:

@@ -9,6 +9,7 @@
 #include "decode.cuh"
 #include "decode2.cuh"
 #include "prefill.cuh"
+#include "shared.cuh"
 #include "quant.cuh"
 #include "router.cuh"
 
@@ -496,6 +497,42 @@ int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, co
   return MOE_OK;
 }
 
+static int check_shared(const char* what, const moe_shared* S) {
+  if (!S) return fail(MOE_ERR_INVALID_ARG, "%s: NULL shared expert", what);
+  if (S->hidden <= 0 || S->ffn <= 0) return fail(MOE_ERR_INVALID_ARG, "%s: sizes must be positive", what);
+  if (S->hidden % kBlock || S->ffn % kQBlock || S->hidden > kMaxHidden || S->ffn > kMaxFfn)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: hidden %% 256, ffn %% 32, hidden <= %d, ffn <= %d", what, kMaxHidden,
+                kMaxFfn);
+  return check_ptrs(what, S->gate_q, S->gate_d, S->up_q, S->up_d, S->down_q, S->down_d);
+}
+
+int moe_quantize_weights_q8(const float* w, int64_t rows, int64_t k, int8_t* q, uint16_t* d, moe_stream_t stream) {
+  int rc = check_ptrs("quantize_weights_q8", w, q, d);
+  if (rc) return rc;
+  if (rows <= 0 || k <= 0) return fail(MOE_ERR_INVALID_ARG, "quantize_weights_q8: rows, k must be > 0");
+  if (k % kQBlock) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "quantize_weights_q8: k %% 32 must be 0");
+  if ((rc = check_device())) return rc;
+  return launch_quantize_weights_q8(w, rows, k, q, d, static_cast<cudaStream_t>(stream));
+}
+
+size_t moe_shared_workspace_bytes(const moe_shared* S, int32_t ntok) {
+  if (!S || S->hidden <= 0 || S->ffn <= 0 || S->ffn % kQBlock || ntok <= 0 || ntok > 65536) return 0;
+  return shared_ws_bytes(S->hidden, S->ffn, ntok);
+}
+
+int moe_shared_ffn_add(const moe_shared* S, int32_t ntok, const int8_t* xq, const float* xd, float* y, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  int rc = check_shared("shared_ffn_add", S);
+  if (rc) return rc;
+  if ((rc = check_ptrs("shared_ffn_add", xq, xd, y, ws))) return rc;
+  if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "shared_ffn_add: 1 <= ntok <= 65536");
+  const size_t need = shared_ws_bytes(S->hidden, S->ffn, ntok);
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "shared_ffn_add: workspace %zu < %zu bytes", ws_bytes, need);
+  if ((rc = check_device())) return rc;
+  SharedParams P{S->hidden, S->ffn, S->gate_q, S->gate_d, S->up_q, S->up_d, S->down_q, S->down_d};
+  return launch_shared_ffn_add(P, ntok, xq, xd, y, ws, static_cast<cudaStream_t>(stream));
+}
+
 int moe_check_status(void* ws, moe_stream_t stream) {
   if (!ws) return fail(MOE_ERR_INVALID_ARG, "check_status: NULL workspace");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -535,7 +572,7 @@ const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
       "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather", "copy",
-      "router_quant", "topk_group"};
+      "router_quant", "topk_group", "shared"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

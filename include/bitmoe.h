@@ -231,6 +231,31 @@ int moe_forward_host(const moe_layer* layer, const float* w_router, int32_t ntok
                      const float* x_host, float* y_host, void* ws, size_t ws_bytes,
                      moe_stream_t stream);
 
+/* ---- shared expert (llama-modchip page, "The interesting bit": shared
+ *      experts stay at higher precision beside the low-bit routed experts) --
+ * An always-active FFN in 8-bit blocks of 32 weights: per block
+ * d = fp16_RNE(amax/127) (the division in fp64), q = clamp(rint(w/d), -127,
+ * 127) with an IEEE fp32 division by the fp16 value (a block whose d is 0 is
+ * all zeros); codes row-major int8 [rows][k], scales fp16 [rows][k/32].    */
+typedef struct {
+  int32_t hidden, ffn;       /* multiples of 256 and of 32                 */
+  const int8_t* gate_q;  const uint16_t* gate_d;   /* [ffn][hidden]       */
+  const int8_t* up_q;    const uint16_t* up_d;     /* [ffn][hidden]       */
+  const int8_t* down_q;  const uint16_t* down_d;   /* [hidden][ffn]       */
+} moe_shared;
+/* w [rows][k] fp32 -> q, d in the 8-bit block format (k % 32 == 0).        */
+int moe_quantize_weights_q8(const float* w, int64_t rows, int64_t k, int8_t* q, uint16_t* d,
+                            moe_stream_t stream);
+/* Workspace bytes of moe_shared_ffn_add for `ntok` tokens (0 on bad args). */
+size_t moe_shared_workspace_bytes(const moe_shared* shared, int32_t ntok);
+/* y [ntok][hidden] += Wd (q8(silu(Wg x^) * Wu x^))^ for the int8 activations
+ * xq [ntok][hidden], xd [ntok][hidden/32] (moe_quant_act_q8's output): the
+ * shared expert's output added to the routed experts' sum (call it after
+ * moe_expert_ffn_decode / moe_forward on the same stream).  ws is a separate
+ * scratch of moe_shared_workspace_bytes bytes.                             */
+int moe_shared_ffn_add(const moe_shared* shared, int32_t ntok, const int8_t* xq, const float* xd,
+                       float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ---- status ------------------------------------------------------------- */
 /* Synchronizes `stream`, returns the status recorded in the workspace by
  * the device (MOE_OK or a negative moe_status) and clears it.             */
@@ -245,7 +270,7 @@ typedef enum {
   MOE_K_GROUP = 4, MOE_K_GATEUP = 5, MOE_K_DOWN = 6, MOE_K_DEBUG_MATVEC = 7,
   MOE_K_PREFILL_GATEUP = 8, MOE_K_PREFILL_DOWN = 9, MOE_K_ROUTE = 10, MOE_K_COMBINE = 11,
   MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COPY = 14, MOE_K_ROUTER_QUANT = 15,
-  MOE_K_TOPK_GROUP = 16, MOE_K_COUNT = 17
+  MOE_K_TOPK_GROUP = 16, MOE_K_SHARED = 17, MOE_K_COUNT = 18
 } moe_kernel_id;
 /* Number of kernels this thread has launched through the library so far. */
 int64_t moe_launch_count(void);

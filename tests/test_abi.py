@@ -84,3 +84,17 @@ def test_sign_format_host_side_without_device():
     assert rc == -1 and b"codes" in L.moe_last_error()
     rc = L.moe_quantize_weights_e16(p, 32, 200, p, p, p, None)
     assert rc == -2
+
+
+def test_shared_expert_host_side_without_device():
+    B, L = _lib()
+    s = B.moe_shared(256, 512, None, None, None, None, None, None)
+    assert L.moe_shared_workspace_bytes(ctypes.byref(s), 4) > 0
+    assert L.moe_shared_workspace_bytes(ctypes.byref(s), 0) == 0
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
+    rc = L.moe_shared_ffn_add(ctypes.byref(s), 1, p, p, p, p, 1 << 20, None)
+    assert rc == -1 and b"NULL" in L.moe_last_error()
+    bad = B.moe_shared(300, 512, p.value, p.value, p.value, p.value, p.value, p.value)
+    assert L.moe_shared_ffn_add(ctypes.byref(bad), 1, p, p, p, p, 1 << 20, None) == -2
+    assert L.moe_quantize_weights_q8(p, 4, 48, p, p, None) == -2
