@@ -1,0 +1,40 @@
+"""Host-side pieces of the benchmark (CPU only): the byte accounting of the
+weight formats and the code hash that attributes DRAM counters to sources."""
+import os
+
+import bench
+import synthetic
+
+
+def test_block_bytes_and_expert_bytes():
+    wl = synthetic.WORKLOADS["30b"]
+    assert wl.block_bytes == 54 and wl.matrix_bytes(768, 2048) == 768 * 8 * 54
+    s = synthetic.WORKLOADS["30b-sign"]
+    assert s.block_bytes == 34 and s.matrix_bytes(768, 2048) == 768 * 8 * 34
+    e = synthetic.WORKLOADS["30b-e16"]
+    assert e.block_bytes == 60 and e.matrix_bytes(768, 2048) == 768 * 8 * 60 + 2 * 768
+    # one expert = gate + up ([ffn][hidden]) + down ([hidden][ffn])
+    assert wl.expert_bytes == 3 * 768 * 2048 // 256 * 54
+    assert e.expert_bytes == 2 * (768 * 8 * 60 + 2 * 768) + (2048 * 3 * 60 + 2 * 2048)
+
+
+def test_kernel_bytes_scale_with_unique_experts():
+    wl = synthetic.WORKLOADS["large-b8"]
+    a, b = bench.kernel_bytes(wl, 10.0), bench.kernel_bytes(wl, 20.0)
+    per_expert = 2 * wl.matrix_bytes(wl.ffn, wl.hidden)
+    assert b["gateup"] - a["gateup"] == 10 * per_expert
+    assert b["down"] - a["down"] == 10 * wl.matrix_bytes(wl.hidden, wl.ffn)
+
+
+def test_code_hash_ignores_comments(tmp_path, monkeypatch):
+    csrc = tmp_path / "bit_moe_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text('int a = 1; // one\n/* block */ const char* s = "x//y";\n')
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    (csrc / "k.cu").write_text('int a = 1;   // another comment\nconst char* s = "x//y";  /* c */\n')
+    assert bench.kernel_source_hash() == h0
+    (csrc / "k.cu").write_text('int a = 2; // one\n/* block */ const char* s = "x//y";\n')
+    assert bench.kernel_source_hash() != h0
+    (csrc / "k.cu").write_text('int a = 1; // one\n/* block */ const char* s = "x/ /y";\n')
+    assert bench.kernel_source_hash() != h0
