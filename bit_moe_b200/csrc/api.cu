@@ -466,6 +466,10 @@ int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, co
   if ((rc = check_ptrs("forward_host", w_router, ws))) return rc;
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward_host: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
+  // refused before the copy of x is launched, as moe_forward would refuse it
+  if (prefill && L->gate.format != MOE_FORMAT_TERNARY)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward_host: sign-code and E16 layers take at most %d tokens",
+                kMaxDecodeTokens);
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total)
     return fail(MOE_ERR_WORKSPACE, "forward_host: workspace %zu < %zu bytes", ws_bytes, W.total);

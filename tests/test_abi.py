@@ -98,3 +98,17 @@ def test_shared_expert_host_side_without_device():
     bad = B.moe_shared(300, 512, p.value, p.value, p.value, p.value, p.value, p.value)
     assert L.moe_shared_ffn_add(ctypes.byref(bad), 1, p, p, p, p, 1 << 20, None) == -2
     assert L.moe_quantize_weights_q8(p, 4, 48, p, p, None) == -2
+
+
+def test_forward_host_refuses_long_non_ternary_calls_before_any_launch():
+    B, L = _lib()
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
+
+    def tm(rows, k, fmt):
+        return B.moe_tmat(rows, k, p.value, p.value, fmt, p.value)
+    lay = B.moe_layer(256, 256, 2, 1, tm(512, 256, 1), tm(512, 256, 1), tm(512, 256, 1))
+    n0 = L.moe_launch_count()
+    rc = L.moe_forward_host(ctypes.byref(lay), p, 65, p, p, p, 1 << 30, None)
+    assert rc == -2 and b"64 tokens" in L.moe_last_error()
+    assert L.moe_launch_count() == n0
