@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points of libbitmoe: argument validation,
 // workspace layout, and the launch sequence of each call.
+#include <atomic>
 #include <cstring>
 
 #include <algorithm>
@@ -186,14 +187,17 @@ static DecodeParams make_params(const moe_layer* L, int ntok, const int8_t* xq, 
 
 static int sm_count() {
   constexpr int kMaxDev = 64;
-  static int cache[kMaxDev] = {};
+  static std::atomic<int> cache[kMaxDev];  // per device, written once (any thread)
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDev && cache[dev]) return cache[dev];
+  if (dev >= 0 && dev < kMaxDev) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   int n = 0;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   if (n <= 0) n = 148;
-  if (dev >= 0 && dev < kMaxDev) cache[dev] = n;
+  if (dev >= 0 && dev < kMaxDev) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

@@ -13,6 +13,7 @@
 // tokens a grouping pass collects the pairs of each expert so that the
 // expert's weights stream from HBM once per step and every decoded digit word
 // serves all pairs of the item.
+#include <atomic>
 #include <cub/block/block_scan.cuh>
 
 #include "bitmoe.h"
@@ -402,10 +403,10 @@ __global__ void __launch_bounds__(kGateUpWarps * 32)
 // stream capture).
 static void init_kernel_attrs() {
   constexpr int kMaxDev = 64;
-  static bool done[kMaxDev] = {};
+  static std::atomic<bool> done[kMaxDev];  // the attribute calls are idempotent
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDev && done[dev]) return;
+  if (dev >= 0 && dev < kMaxDev && done[dev].load(std::memory_order_relaxed)) return;
   const void* kernels[] = {
       reinterpret_cast<const void*>(&k_gateup<1, 0>),     reinterpret_cast<const void*>(&k_gateup<kChunk, 0>),
       reinterpret_cast<const void*>(&k_down<1, 0>),       reinterpret_cast<const void*>(&k_down<kChunk, 0>),
@@ -417,7 +418,7 @@ static void init_kernel_attrs() {
       reinterpret_cast<const void*>(&k_debug_matvec<2>)};
   for (const void* k : kernels)
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-  if (dev >= 0 && dev < kMaxDev) done[dev] = true;
+  if (dev >= 0 && dev < kMaxDev) done[dev].store(true, std::memory_order_relaxed);
 }
 
 int launch_group(const DecodeParams& P, cudaStream_t stream) {

@@ -23,6 +23,7 @@
 // blocks b = w, w + 8, ... of a row are accumulated by warp w and the eight
 // warp partials summed in warp order; down rows are accumulated block by block
 // in order.
+#include <atomic>
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode2.cuh"
@@ -466,17 +467,17 @@ static size_t down_smem(int F, int K) {
 
 static void init_attrs2() {
   constexpr int kMaxDev = 64;
-  static bool done[kMaxDev] = {};
+  static std::atomic<bool> done[kMaxDev];  // the attribute calls are idempotent
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDev && done[dev]) return;
+  if (dev >= 0 && dev < kMaxDev && done[dev].load(std::memory_order_relaxed)) return;
   const void* ks[] = {reinterpret_cast<const void*>(&k_gateup3<1, true>),
                       reinterpret_cast<const void*>(&k_gateup3<kChunk, false>),
                       reinterpret_cast<const void*>(&k_down3<1, true>),
                       reinterpret_cast<const void*>(&k_down3<kChunk, false>),
                       reinterpret_cast<const void*>(&k_route)};
   for (const void* k : ks) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-  if (dev >= 0 && dev < kMaxDev) done[dev] = true;
+  if (dev >= 0 && dev < kMaxDev) done[dev].store(true, std::memory_order_relaxed);
 }
 
 // CTAs per SM the occupancy calculator allows, at most 2.

@@ -6,6 +6,7 @@
 // taken on fp32 logits, so the evaluation order of each logit is fixed: 32
 // partial sums (lane l accumulates fused multiply-adds over k = l, l+32, ...
 // ascending) followed by xor-butterfly additions at distances 16, 8, 4, 2, 1.
+#include <atomic>
 #include "bitmoe.h"
 #include "common.cuh"
 #include "ptx.cuh"
@@ -174,12 +175,12 @@ static void launch_tiled(const float* x, const float* wr, int ntok, int H, int E
                          cudaStream_t stream, int8_t* xq = nullptr, float* xd = nullptr) {
   auto kern = k_router_logits_tiled<kWE, kMT, kME, kKC>;
   const size_t smem = sizeof(float) * 2 * (kRtT + kWE * kME) * kKC;
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[64];  // the attribute call is idempotent
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_done[dev].load(std::memory_order_relaxed)) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    attr_done[dev] = true;
+    attr_done[dev].store(true, std::memory_order_relaxed);
   }
   const dim3 grid((ntok + kRtT - 1) / kRtT, (E + kWE * kME - 1) / (kWE * kME));
   launch_k(kern, grid, dim3(256), smem, stream, x, wr, ntok, H, E, logits, xq, xd);

@@ -26,6 +26,7 @@
 // blocks, int8 activations); llama-modchip page, "Key highlights" (all top-k
 // experts evaluated); pxq_llama README, "Updates -- 2026-07-28" (gate/up with
 // the SiLU unary).  The numerics are those of the decode kernels.
+#include <atomic>
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode2.cuh"
@@ -497,12 +498,12 @@ bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem) {
 
 int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned long long* units,
                  cudaStream_t stream) {
-  static bool done[64] = {};
+  static std::atomic<bool> done[64];  // the attribute call is idempotent
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !done[dev]) {
+  if (dev >= 0 && dev < 64 && !done[dev].load(std::memory_order_relaxed)) {
     cudaFuncSetAttribute(k_step1, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_relaxed);
   }
   size_t smem = 0;
   if (!step1_supported(D.P, D.n_sm, &smem)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "step1: unsupported shape");
@@ -515,7 +516,7 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   // cooperative (every CTA resident), and a programmatic dependent launch so
   // that consecutive steps overlap (phase A of one step with the tail of the
   // previous); without the latter where the runtime refuses the combination
-  static int pdl_ok[64] = {};  // 0 unknown, 1 yes, -1 no
+  static std::atomic<int> pdl_ok[64];  // 0 unknown, 1 yes, -1 no (any thread may settle it)
   const int di = dev >= 0 && dev < 64 ? dev : 0;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
