@@ -33,6 +33,7 @@
 // Gate/up tiles hold 64 gate rows and the 64 matching up rows, so SwiGLU and
 // the requantization run in the epilogue; down tiles write each pair's rows,
 // and a last pass combines the top_k slots of every token in slot order.
+#include <atomic>
 #include <cuda_fp8.h>
 
 #include "bitmoe.h"
@@ -543,13 +544,13 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   P.group_chunk = kPN;
   int rc = launch_group(P, stream);
   if (rc) return rc;
-  static bool attrs_done[64] = {};
+  static std::atomic<bool> attrs_done[64];  // the attribute calls are idempotent
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attrs_done[dev]) {
+  if (dev >= 0 && dev < 64 && !attrs_done[dev].load(std::memory_order_relaxed)) {
     cudaFuncSetAttribute(k_prefill_mma<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     cudaFuncSetAttribute(k_prefill_mma<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    attrs_done[dev] = true;
+    attrs_done[dev].store(true, std::memory_order_relaxed);
   }
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
