@@ -40,7 +40,7 @@ struct DecodeParams {
   const int32_t* pairs;                  // [ntok*top_k] pair ids grouped by expert
   int32_t* group_scratch;                // [2*(n_experts+1)] counters for the grouping
   int group_chunk;                       // most pairs per item (kChunk for decode)
-  // prefill only: the activation blocks of every 32-pair group, laid out as
+  // prefill only: the activation blocks of every 64-pair group, laid out as
   // the tensor-core kernel's shared-memory stages, for gate/up and for down
   unsigned char* bgu;                        // [groups][hidden/256] blocks
   unsigned char* bdn;                        // [groups][ffn/256] blocks

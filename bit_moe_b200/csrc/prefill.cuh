@@ -3,7 +3,7 @@
 #include "decode.cuh"
 namespace bitmoe {
 int launch_prefill(const DecodeParams& P, cudaStream_t stream);
-// Bytes of one activation block of a 32-pair group (split codes, scales, sums).
+// Bytes of one activation block of a group of prefill_group_pairs() pairs (split codes, scales, sums).
 size_t prefill_block_bytes();
 // Most (token, slot) pairs in one group of the prefill GEMM.
 int prefill_group_pairs();
