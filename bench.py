@@ -41,12 +41,15 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="30b",
+    ap.add_argument("--workload", default="large",
                     help="tiny | 30b | 30b-b16 | large | large-b8 | 30b-prefill | 30b-sign | large-sign-b8 | "
                          "30b-e16 | large-e16-b8")
     ap.add_argument("--impl", default="bitmoe", choices=["bitmoe", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-suite", action="store_true",
+                    help="time only --workload (by default the large-layer run also times the large layer "
+                         "at 8 tokens, the 30B-class layer at 1 and 16 tokens and its 2048-token prefill)")
     ap.add_argument("--layers", type=int, default=0,
                     help="layers in the rotated stack (default: enough to exceed 2x L2)")
     return ap.parse_args()
@@ -204,6 +207,21 @@ def ncu_traffic(kernel, workload):
         return None
 
 
+def ncu_field(kernel, workload, field):
+    """Another figure of the committed ncu summary (e.g. the tensor-pipe
+    utilisation), under the same source-hash rule as ncu_traffic."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e[field])
+    except Exception:
+        return None
+
+
 # --------------------------------------------------------------------------- reference arm
 def run_reference(args):
     """The CPU oracle on the host cores, timed as the step of this workload.
@@ -241,22 +259,25 @@ def run_reference(args):
         oracle.expert_ffn(layer, xq, xd, np.array([[e]], np.int32),
                           w2[:, slot:slot + 1].astype(np.float32))
 
-    for j in range(args.warmup):
-        step(j)
-    t0 = time.perf_counter()
-    for j in range(args.steps):
-        step(args.warmup + j)
-    dt = time.perf_counter() - t0
+    with PinnedToOneCore() as pin:
+        for j in range(args.warmup):
+            step(j)
+        t0 = time.perf_counter()
+        for j in range(args.steps):
+            step(args.warmup + j)
+        dt = time.perf_counter() - t0
     value = args.steps / K / dt
     sample = ("each step: oracle act quant + router for 1 token of %s and the expert FFN of one of "
-              "its %d slots (counted as 1/%d token)" % (wl.describe(), K, K))
+              "its %d slots (counted as 1/%d token), single-threaded, pinned to one core"
+              % (wl.describe(), K, K))
+    nproc, model = host_cpu()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(wl, None),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "pinned_core": pin.core, "nproc": nproc, "cpu_model": model},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -299,80 +320,121 @@ def stack_size(wl, step_bytes):
     return max(wl.layers, min(need, 64))
 
 
-def cpu_baseline(wl, budget_s=12.0):
-    """The oracle as it stands, single-threaded, on a bounded sample of steps of
-    this workload: consecutive batches of tokens (decode batches of the
-    workload's size; 8-token chunks for prefill) until about `budget_s` of CPU
-    time.  Packing the routed experts' weights is set-up and not timed."""
+def host_cpu():
+    """(nproc, CPU model) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+class PinnedToOneCore:
+    """Pins this process to one core for the duration of a CPU measurement
+    (what `taskset -c <core>` does for a child), then restores the affinity."""
+
+    def __enter__(self):
+        self.saved = None
+        self.core = None
+        try:
+            self.saved = os.sched_getaffinity(0)
+            self.core = max(self.saved)
+            os.sched_setaffinity(0, {self.core})
+        except (AttributeError, OSError):
+            pass
+        return self
+
+    def __exit__(self, *a):
+        if self.saved is not None:
+            try:
+                os.sched_setaffinity(0, self.saved)
+            except OSError:
+                pass
+        return False
+
+
+def cpu_baseline(wl, repeats=3, n_tok=None):
+    """The oracle as it stands, single-threaded and pinned to one core, on a
+    bounded sample of this workload: the first `n_tok` tokens of the
+    workload's inputs in decode batches of the workload's size (8-token
+    chunks for prefill).  The routed experts' weights are packed once,
+    untimed; the sample is then timed `repeats` times and the median taken."""
     import numpy as np
     import oracle
     import synthetic
     H, F, K = wl.hidden, wl.ffn, wl.top_k
     chunk = wl.ntok if wl.ntok <= 64 else 8
+    if n_tok is None:
+        big = wl.hidden * wl.ffn >= 4096 * 2048
+        n_tok = chunk * (1 if chunk >= 8 else (2 if big else 4))
     wr = synthetic.router(wl, 0).numpy()
-    x = synthetic.activations(wl, 0, ntok=64).numpy()
-    n, tot = 0, 0.0
-    while tot < budget_s and n + chunk <= 64:
-        toks = x[n:n + chunk]
-        idx, _ = oracle.route_topk(toks, wr, K)
-        e_used = sorted(set(int(e) for e in idx.ravel()))
-        layer = oracle.Layer.from_float(
-            H, F, len(e_used), K,
-            np.concatenate([synthetic.expert_matrix(wl, 0, "gate", e).numpy() for e in e_used]),
-            np.concatenate([synthetic.expert_matrix(wl, 0, "up", e).numpy() for e in e_used]),
-            np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in e_used]),
-            fmt=wl.fmt)
-        remap = np.full(wl.n_experts, -1, np.int32)
-        remap[e_used] = np.arange(len(e_used))
+    x = synthetic.activations(wl, 0, ntok=max(n_tok, 1)).numpy()[:n_tok]
+    idx, _ = oracle.route_topk(x, wr, K)
+    e_used = sorted(set(int(e) for e in idx.ravel()))
+    layer = oracle.Layer.from_float(
+        H, F, len(e_used), K,
+        np.concatenate([synthetic.expert_matrix(wl, 0, "gate", e).numpy() for e in e_used]),
+        np.concatenate([synthetic.expert_matrix(wl, 0, "up", e).numpy() for e in e_used]),
+        np.concatenate([synthetic.expert_matrix(wl, 0, "down", e).numpy() for e in e_used]),
+        fmt=wl.fmt)
+    remap = np.full(wl.n_experts, -1, np.int32)
+    remap[e_used] = np.arange(len(e_used))
+
+    def sample():
         t0 = time.perf_counter()
-        xq, xd = oracle.quant_act_q8(toks)
-        i2, w2 = oracle.route_topk(toks, wr, K)
-        oracle.expert_ffn(layer, xq, xd, remap[i2], w2.astype(np.float32))
-        tot += time.perf_counter() - t0
-        n += chunk
-    return {"value": n / tot, "unit": "tok/s", "cores": 1, "kind": "oracle",
-            "sample": "%d tokens in batches of %d of %s (layer 0), oracle single-threaded, "
-                      "weight packing untimed" % (n, chunk, wl.describe())}
+        for n in range(0, n_tok, chunk):
+            toks = x[n:n + chunk]
+            xq, xd = oracle.quant_act_q8(toks)
+            i2, w2 = oracle.route_topk(toks, wr, K)
+            oracle.expert_ffn(layer, xq, xd, remap[i2], w2.astype(np.float32))
+        return time.perf_counter() - t0
+
+    with PinnedToOneCore() as pin:
+        times = [sample() for _ in range(repeats)]
+    med = sorted(times)[len(times) // 2]
+    nproc, model = host_cpu()
+    return {"value": n_tok / med, "unit": "tok/s", "cores": 1, "kind": "oracle",
+            "sample": "%d tokens in batches of %d of %s (layer 0), oracle single-threaded, pinned to one "
+                      "core, median of %d timings; weight packing untimed" % (n_tok, chunk, wl.describe(), repeats),
+            "times_s": times, "pinned_core": pin.core, "nproc": nproc, "cpu_model": model}
 
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        run_reference(args)
-        return
-    rank, world, local = dist_env()
+# --------------------------------------------------------------------------- one workload
+def routing_histogram(B, x, router, wl):
+    """Per-expert count of (token, slot) pairs of one step's routing."""
     import torch
-    import torch.distributed as dist
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    idx, _ = B.moe_route_topk(x, router, wl.top_k)
+    counts = torch.bincount(idx.flatten().long(), minlength=wl.n_experts).cpu().tolist()
+    used = [c for c in counts if c]
+    return {"counts": counts, "unique_experts": len(used), "max_pairs": max(used),
+            "mean_pairs_per_used_expert": sum(used) / len(used)}
 
-    import bit_moe_b200 as B
-    import synthetic
-    from bit_moe_b200 import build
+
+def build_stack(B, wl, n_layers, dev, seed_off):
     from bit_moe_b200.layers import quantize_layer
-    if rank == 0:
-        build.build()
-    if world > 1:
-        dist.barrier()
-    B.lib()
-
-    wl = synthetic.WORKLOADS[args.workload]
-    T, H, K = wl.ntok, wl.hidden, wl.top_k
-    dev = torch.device("cuda", local)
-    seed_off = 1000 * rank  # each replica draws its own layers and inputs
-
-    # ---- layer stack and inputs, resident in HBM
-    per_step_guess = (min(wl.n_experts, T * K) * wl.expert_bytes) + wl.n_experts * H * 4
-    L = args.layers if args.layers > 0 else stack_size(wl, per_step_guess)
+    import synthetic
     layers, routers = [], []
-    for l in range(L):
+    for l in range(n_layers):
         fn = lambda role, e, l=l: synthetic.expert_matrix(wl, seed_off + l, role, e, dev)  # noqa: E731
         layers.append(quantize_layer(wl.hidden, wl.ffn, wl.n_experts, wl.top_k, fn, fmt=wl.fmt))
         routers.append(synthetic.router(wl, seed_off + l, dev))
-    NX = 64
+    return layers, routers
+
+
+def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do_e2e=True):
+    """Warm-up, CUDA-graph capture and the timed region for one workload,
+    then its per-kernel times and roofline.  Returns the result dict."""
+    import torch
+    import torch.distributed as dist
+    import synthetic
+    T, H, K = wl.ntok, wl.hidden, wl.top_k
+    L = len(layers)
+    NX = 64 if T <= 64 else 4
     xs = [synthetic.activations(wl, seed_off + j, device=dev) for j in range(NX)]
     ws = B.Workspace.for_layer(layers[0], T)
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
@@ -381,14 +443,13 @@ def main():
     def step(j):
         B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
 
-    # ---- warm-up (eager), then capture the step sequence as CUDA graphs
-    for j in range(args.warmup):
+    for j in range(warmup):
         step(j)
     torch.cuda.synchronize()
     status = B.moe_check_status(ws)
     if status != 0:
         raise SystemExit("device status %d after warm-up" % status)
-    G = min(args.steps, 4 * L)
+    G = min(steps, 4 * L)
     stream = torch.cuda.Stream(device=dev)
 
     def capture(n_steps, first):
@@ -401,11 +462,10 @@ def main():
                     step(first + j)
         return g
 
-    g_main = capture(G, args.warmup)
-    rem = args.steps % G
-    g_rem = capture(rem, args.warmup) if rem else None
-    reps = args.steps // G
-    launches_per_step = None
+    g_main = capture(G, warmup)
+    rem = steps % G
+    g_rem = capture(rem, warmup) if rem else None
+    reps = steps // G
     c0 = B.moe_launch_count()
     step(0)
     launches_per_step = B.moe_launch_count() - c0
@@ -414,7 +474,7 @@ def main():
     torch.cuda.synchronize()
 
     # ---- timed region
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -434,12 +494,12 @@ def main():
     status = B.moe_check_status(ws)
     if status != 0:
         raise SystemExit("device status %d after the timed region" % status)
-    value = job_rate(T * args.steps, world, ms)
+    del g_main, g_rem
 
     # ---- per-kernel times: the same steps launched eagerly behind a spin
     # kernel (so the host has queued them all before the GPU starts them and
     # they run back to back), with an event after every library kernel
-    n_tr = min(G, 2 * L)
+    n_tr = min(G, 2 * L) if T <= 64 else min(G, 4)
     per_kernel = {}
     for _ in range(3):
         tr = B.KernelTrace(capacity=n_tr * launches_per_step + 8)
@@ -447,13 +507,13 @@ def main():
             torch.cuda._sleep(int(4e7))
             with tr:
                 for j in range(n_tr):
-                    step(args.warmup + j)
+                    step(warmup + j)
             stream.synchronize()
         for name, v in tr.durations().items():
             per_kernel.setdefault(name, []).extend(v)
     # routing of the (layer, input) combinations the steps use: unique experts
     uniq = []
-    for j in range(min(L * NX, 256)):
+    for j in range(min(L * NX, 256 if T <= 64 else 8)):
         idx, _ = B.moe_route_topk(xs[j % NX], routers[j % L], K)
         uniq.append(len(set(idx.flatten().tolist())))
     unique_experts = sum(uniq) / len(uniq)
@@ -470,15 +530,28 @@ def main():
                 "algorithmic_bytes_per_launch": kb.get(dom, 0),
                 "traffic": ncu_traffic(dom, wl.describe())}
     step_bytes = sum(kb[n] for n in kb if n in shares)
-    step_gbs = step_bytes / (ms / 1e3 / args.steps) / 1e9
+    step_s = ms / 1e3 / steps
+    res = {"workload": wl.describe(), "tokens_per_step": T, "steps": steps, "warmup": warmup,
+           "ms_per_step": ms / steps, "value": job_rate(T * steps, world, ms), "unit": "tok/s",
+           "layer_stack": L, "roofline": roofline, "step_hbm_gbs": step_bytes / step_s / 1e9,
+           "step_hbm_frac": step_bytes / step_s / 1e9 / peak,
+           "unique_experts_per_step": unique_experts, "kernels": shares,
+           "launches_per_step": launches_per_step, "clocks": sampler.summary()}
+    if wl.prefill:
+        macs = T * K * 3 * H * wl.ffn
+        gemm_s = sum(shares[n]["avg_us"] for n in ("prefill_gateup", "prefill_down") if n in shares) / 1e6
+        res["int8_tops"] = {"value": 2 * macs / gemm_s / 1e12 if gemm_s else None,
+                            "macs_per_step": macs, "kernels": ["prefill_gateup", "prefill_down"],
+                            "tensor_pipe_pct": ncu_field("prefill_gateup", wl.describe(), "tensor_pipe_pct")}
+    if T > 1:
+        res["routing_histogram"] = routing_histogram(B, xs[0], routers[0], wl)
 
     # ---- end to end: the host-buffer entry point, copies inside the timed region.
     # Every step copies its x in from pinned host memory and its y out to pinned
     # host memory on the stream; the steps are replayed from CUDA graphs of
     # moe_forward_host calls, as a serving loop would drive them.
-    e2e = None
-    if not args.no_e2e:
-        n_e2e = min(args.steps, 2000)
+    if do_e2e:
+        n_e2e = min(steps, 2000)
         xh = [xs[j % NX].cpu().pin_memory() for j in range(min(NX, n_e2e))]
         yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
 
@@ -513,29 +586,95 @@ def main():
             stream.synchronize()
         del ge_main, ge_rem
         e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev)
-        e2e = {"value": job_rate(T * n_e2e, world, e_ms), "unit": "tok/s",
-               "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4,
-               "steps": n_e2e, "api": "moe_forward_host", "launch": "CUDA graph replay"}
+        res["e2e"] = {"value": job_rate(T * n_e2e, world, e_ms), "unit": "tok/s",
+                      "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4,
+                      "steps": n_e2e, "api": "moe_forward_host", "launch": "CUDA graph replay"}
+    return res
+
+
+# the other configurations measured in the same run (single GPU): the large
+# layer at 8 tokens, the 30B-class layer at 1 and 16 tokens, and its
+# 2048-token prefill
+SUITE = ("large-b8", "30b", "30b-b16", "30b-prefill")
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    rank, world, local = dist_env()
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import bit_moe_b200 as B
+    import synthetic
+    from bit_moe_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    B.lib()
+
+    wl = synthetic.WORKLOADS[args.workload]
+    T, H, K = wl.ntok, wl.hidden, wl.top_k
+    dev = torch.device("cuda", local)
+    seed_off = 1000 * rank  # each replica draws its own layers and inputs
+
+    def stack_for(w):
+        per_step_guess = (min(w.n_experts, w.ntok * w.top_k) * w.expert_bytes) + w.n_experts * w.hidden * 4
+        return args.layers if args.layers > 0 else stack_size(w, per_step_guess)
+
+    # ---- headline workload: layer stack and inputs resident in HBM
+    L = stack_for(wl)
+    layers, routers = build_stack(B, wl, L, dev, seed_off)
+    head = run_workload(B, wl, layers, routers, args.steps, args.warmup, dev, world, seed_off,
+                        do_e2e=not args.no_e2e)
+
+    # ---- the other configurations (one GPU only): each on its own stack,
+    # the large layer's reused where the seeds agree
+    suite = []
+    if world == 1 and not args.no_suite and args.workload == "large":
+        held = wl  # the workload whose layer stack is built
+        for name in SUITE:
+            w = synthetic.WORKLOADS[name]
+            same = lambda a, b: (a.hidden, a.ffn, a.n_experts, a.seed, a.fmt) == (b.hidden, b.ffn, b.n_experts,  # noqa: E731
+                                                                                 b.seed, b.fmt)
+            if not same(w, held) or stack_for(w) > len(layers):
+                del layers, routers
+                torch.cuda.empty_cache()
+                layers, routers = build_stack(B, w, stack_for(w), dev, seed_off)
+                held = w
+            suite.append(run_workload(B, w, layers, routers, max(args.steps, 20), max(args.warmup, 3), dev,
+                                      world, seed_off, do_e2e=not args.no_e2e))
+    del layers, routers
+    torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(wl)
+        cpu = cpu_baseline(synthetic.WORKLOADS[args.workload])
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "metric": METRIC, "value": head["value"], "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
-            "data": "synthetic", "config": workload_config(wl, L),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": sampler.summary(),
-            "step_hbm_gbs": step_gbs, "unique_experts_per_step": unique_experts,
-            "kernels": shares,
+            "data": "synthetic", "config": workload_config(synthetic.WORKLOADS[args.workload], L),
+            "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": head.get("e2e"),
+            "gpu_launches": head["launches_per_step"] * args.steps,
+            "clocks": head["clocks"],
+            "step_hbm_gbs": head["step_hbm_gbs"], "step_hbm_frac": head["step_hbm_frac"],
+            "unique_experts_per_step": head["unique_experts_per_step"],
+            "kernels": head["kernels"],
+            "configs": suite,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
-        del g_main, g_rem
         dist.barrier()
         dist.destroy_process_group()
 

@@ -11,6 +11,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
@@ -40,15 +41,39 @@ def _stale():
 
 
 def build(force=False, verbose=False, extra=()):
+    """Compile every source to an object file (in parallel, one nvcc per
+    source) and link them into libbitmoe.so."""
     if not force and not _stale():
         return OUT
-    tmp = OUT + ".tmp.%d" % os.getpid()
-    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-           "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr", *extra, "-o", tmp, *sources()]
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.check_call(cmd)
-    os.replace(tmp, OUT)
+    tag = ".tmp.%d" % os.getpid()
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
+             "--expt-relaxed-constexpr", *extra]
+    srcs = sources()
+    objs = [os.path.join(CSRC, os.path.basename(s)[:-3] + tag + ".o") for s in srcs]
+
+    def compile_one(pair):
+        src, obj = pair
+        cmd = [nvcc_path(), *flags, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        return subprocess.run(cmd).returncode
+
+    try:
+        with ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+            rcs = list(ex.map(compile_one, zip(srcs, objs)))
+        bad = [s for s, rc in zip(srcs, rcs) if rc != 0]
+        if bad:
+            raise subprocess.CalledProcessError(1, "nvcc " + " ".join(os.path.basename(b) for b in bad))
+        tmp = OUT + tag
+        cmd = [nvcc_path(), *ARCH, "-shared", "-o", tmp, *objs]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.check_call(cmd)
+        os.replace(tmp, OUT)
+    finally:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
     return OUT
 
 

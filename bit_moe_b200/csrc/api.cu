@@ -263,6 +263,20 @@ static int launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t 
   return check_launch("forward_host: copy");
 }
 
+// The checks of moe_expert_ffn_decode that do not involve a workspace (layer,
+// pointers, token count, device), for entry points that bring their own
+// scratch and must validate a call before touching it.
+int check_decode_call(const char* what, const moe_layer* L, int32_t ntok, const int8_t* xq, const float* xd,
+                      const int32_t* idx, const float* wts, float* y) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if ((rc = check_ptrs(what, xq, xd, idx, wts, y))) return rc;
+  if (ntok <= 0) return fail(MOE_ERR_INVALID_ARG, "%s: ntok must be > 0", what);
+  if (ntok > kMaxDecodeTokens)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: decode takes at most %d tokens", what, kMaxDecodeTokens);
+  return check_device();
+}
+
 }  // namespace bitmoe
 
 using namespace bitmoe;

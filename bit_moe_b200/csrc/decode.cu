@@ -135,25 +135,6 @@ __global__ void __launch_bounds__(kGroupThreads) k_topk_group(DecodeParams P, co
   group_body(P);
 }
 
-// Fetch work item `it`; returns false when there is none.
-__device__ __forceinline__ bool fetch_item(const DecodeParams& P, int it, Item& item) {
-  if (P.direct) {
-    if (it >= P.ntok * P.top_k) return false;
-    const int e = P.idx[it];
-    item.expert = (e >= 0 && e < P.n_experts) ? e : -1;
-    item.start = it;
-    item.count = 1;
-    return true;
-  }
-  if (it >= *P.n_items) return false;
-  item = P.items[it];
-  return true;
-}
-
-__device__ __forceinline__ int item_pair(const DecodeParams& P, const Item& item, int n) {
-  return P.direct ? item.start + n : P.pairs[item.start + n];
-}
-
 // ---------------------------------------------------------------------------
 // S3 + S4: gate and up of one item for one 32-row panel of the ffn dimension.
 // The 8 warps split the 256-blocks of the hidden dimension; the per-warp
@@ -261,25 +242,6 @@ __global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P)
 // y[t] = sum_j wts[t][j] * ye[t][j] over the slots in order.
 // grid: (hidden/32/kDownWarps, items), block: kDownWarps*32.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void arrive_and_combine(const DecodeParams& P, int pair, int panel,
-                                                   int lane) {
-  const int K = P.top_k, H = P.hidden;
-  const int t = pair / K;
-  int32_t* c = P.cnt + static_cast<size_t>(t) * (H / kPanel) + panel;
-  int old = 0;
-  if (lane == 0) old = atomicAdd(c, 1);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (old == K - 1) {
-    __threadfence();
-    float y = 0.f;
-    const float* ye = P.ye + static_cast<size_t>(t) * K * H + panel * kPanel + lane;
-    for (int j = 0; j < K; ++j)
-      y = __fmaf_rn(__ldcg(P.wts + static_cast<size_t>(t) * K + j), __ldcg(ye + static_cast<size_t>(j) * H), y);
-    P.y[static_cast<size_t>(t) * H + panel * kPanel + lane] = y;
-    if (lane == 0) atomicExch(c, 0);
-  }
-}
-
 template <int NT, int kFmt>
 __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item, int pgroup,
                                          unsigned char* smem) {

@@ -46,11 +46,57 @@ struct DecodeParams {
   unsigned char* bdn;                        // [groups][ffn/256] blocks
 };
 
+// Fetch work item `it`; returns false when there is none.
+__device__ __forceinline__ bool fetch_item(const DecodeParams& P, int it, Item& item) {
+  if (P.direct) {
+    if (it >= P.ntok * P.top_k) return false;
+    const int e = P.idx[it];
+    item.expert = (e >= 0 && e < P.n_experts) ? e : -1;
+    item.start = it;
+    item.count = 1;
+    return true;
+  }
+  if (it >= *P.n_items) return false;
+  item = P.items[it];
+  return true;
+}
+
+__device__ __forceinline__ int item_pair(const DecodeParams& P, const Item& item, int n) {
+  return P.direct ? item.start + n : P.pairs[item.start + n];
+}
+
+// The CTA that completes the last of token t's top_k slots for 32-row panel
+// `panel` of hidden (counted in P.cnt, reset by that CTA) combines
+// y[t] = sum_j wts[t][j] * ye[t][j] over the slots in order; called by a
+// whole warp (lane = row of the panel) after its ye values are visible.
+__device__ __forceinline__ void arrive_and_combine(const DecodeParams& P, int pair, int panel,
+                                                   int lane) {
+  const int K = P.top_k, H = P.hidden;
+  const int t = pair / K;
+  int32_t* c = P.cnt + static_cast<size_t>(t) * (H / kPanel) + panel;
+  int old = 0;
+  if (lane == 0) old = atomicAdd(c, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old == K - 1) {
+    __threadfence();
+    float y = 0.f;
+    const float* ye = P.ye + static_cast<size_t>(t) * K * H + panel * kPanel + lane;
+    for (int j = 0; j < K; ++j)
+      y = __fmaf_rn(__ldcg(P.wts + static_cast<size_t>(t) * K + j), __ldcg(ye + static_cast<size_t>(j) * H), y);
+    P.y[static_cast<size_t>(t) * H + panel * kPanel + lane] = y;
+    if (lane == 0) atomicExch(c, 0);
+  }
+}
+
 // Bytes of workspace the grouped mode needs after `off`; writes the offsets.
 struct GroupWs {
   size_t items = 0, n_items = 0, pairs = 0, scratch = 0;
 };
 size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G);
+
+// Argument checks of a decode call that do not involve its workspace.
+int check_decode_call(const char* what, const moe_layer* L, int32_t ntok, const int8_t* xq, const float* xd,
+                      const int32_t* idx, const float* wts, float* y);
 
 int launch_group(const DecodeParams& P, cudaStream_t stream);
 // Top-k softmax of P.ntok <= 64 tokens' logits ([ntok][E] fp32) into P.idx

@@ -55,6 +55,10 @@ using namespace bitmoe;
 extern "C" int moe_expert_ffn_decode_static(const moe_layer* layer, int32_t ntok, const int8_t* xq,
                                             const float* xd, const int32_t* idx, const float* wts,
                                             float* y, moe_stream_t stream) {
+  // Every argument is checked before the shared array is touched, so a call
+  // that is refused leaves it (and any call still using it) alone.
+  int rc = check_decode_call("expert_ffn_decode_static", layer, ntok, xq, xd, idx, wts, y);
+  if (rc) return rc;
   const size_t need = moe_workspace_bytes(layer, ntok, 0);
   if (need == 0) return fail(MOE_ERR_INVALID_ARG, "expert_ffn_decode_static: invalid layer or ntok");
   if (need > kStaticScratchBytes)
@@ -63,11 +67,13 @@ extern "C" int moe_expert_ffn_decode_static(const moe_layer* layer, int32_t ntok
                 "holds %zu (use moe_expert_ffn_decode with a workspace)",
                 need, kStaticScratchBytes);
   void* scratch = nullptr;
-  int rc = static_scratch(&scratch);
+  rc = static_scratch(&scratch);
   if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The array keeps what the previous call left there.  Counters and the status
-  // word must start at zero: clear the whole region this call uses.
+  // word must start at zero: clear the whole region this call uses.  The
+  // status word is cleared by every call, so device-side reports (bad expert
+  // ids) cannot be read back through this entry point.
   cudaError_t err = cudaMemsetAsync(scratch, 0, need, s);
   if (err != cudaSuccess)
     return fail(MOE_ERR_CUDA, "expert_ffn_decode_static: clearing scratch: %s", cudaGetErrorString(err));

@@ -39,6 +39,7 @@
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "digits.cuh"
 #include "prefill.cuh"
 #include "tc.cuh"
 
@@ -138,28 +139,6 @@ __global__ void __launch_bounds__(kPN * kSubPerBlock) k_prefill_gather(DecodePar
     }
     dst->d[s][n] = d;
     dst->nsa[s][n] = -static_cast<float>(sum);
-  }
-}
-
-// Digit words [32*kHalf, 32*kHalf + 32) of one packed block (digit word
-// 5*j + i holds level i of the four bytes of packed word j): each 16-bit lane
-// keeps u * 3^i, whose high byte H_i grows by one base-3 digit per level and
-// t_i = H_(i+1) - 3*H_i.  Packed word 6 feeds both halves.
-template <int kHalf>
-__device__ __forceinline__ void decode_half(const uint32_t (&w)[kBlockWords], uint32_t (&dg)[32]) {
-#pragma unroll
-  for (int j = 6 * kHalf; j < 6 * kHalf + 7; ++j) {
-    uint32_t lo = w[j] & 0x00FF00FFu, hi = (w[j] >> 8) & 0x00FF00FFu, hp = 0u;
-#pragma unroll
-    for (int i = 0; i < 5; ++i) {
-      if (j == kBlockWords - 1 && i == 4) break;
-      lo *= 3u;
-      hi *= 3u;
-      const uint32_t hn = __byte_perm(lo, hi, 0x7351);
-      const int c = 5 * j + i - 32 * kHalf;
-      if (c >= 0 && c < 32) dg[c] = hn - 3u * hp;
-      hp = hn;
-    }
   }
 }
 
@@ -310,15 +289,14 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       if (tn < n_tiles) load(tn, bn, wn);
       const int a = i % kAStages;
       if (!wait_or_abort(&S.a_empty[a], ((i / kAStages) & 1u) ^ 1u, S, P.status)) break;
-      {
-        uint32_t dg[32];
-        decode_half<0>(w, dg);
-        tmem_st32(tlane + kAcol + 64 * a, dg);
-      }
-      {
-        uint32_t dg[32];
-        decode_half<1>(w, dg);
-        tmem_st32(tlane + kAcol + 64 * a + 32, dg);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w7[7], dg[32];
+#pragma unroll
+        for (int jj = 0; jj < 7; ++jj) w7[jj] = w[6 * h + jj];
+        if (h == 0) digit_half<0>(w7, dg);
+        else digit_half<1>(w7, dg);
+        tmem_st32(tlane + kAcol + 64 * a + 32 * h, dg);
       }
       tc_wait_st();
       tc_fence_before();

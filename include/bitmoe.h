@@ -199,7 +199,12 @@ int moe_expert_ffn_decode(const moe_layer* layer, int32_t ntok, const int8_t* xq
  *   - Every call clears and reuses the same array, so two calls whose work
  *     can overlap on the GPU (other streams, other host threads) race; keep
  *     them ordered on one stream.
- *   - Expert ids outside [0, E) contribute nothing and are not reported.
+ *   - Arguments are checked before the array is touched: a refused call
+ *     (NULL or misaligned pointer, bad sizes) clears nothing.
+ *   - No device-side status can be observed through this entry point: each
+ *     call clears the array's status word, and there is no workspace to pass
+ *     to moe_check_status.  Expert ids outside [0, E) contribute nothing and
+ *     are not reported.
  *   - It allocates and frees nothing.                                      */
 int moe_expert_ffn_decode_static(const moe_layer* layer, int32_t ntok, const int8_t* xq,
                                  const float* xd, const int32_t* idx, const float* wts, float* y,

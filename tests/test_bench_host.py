@@ -38,3 +38,16 @@ def test_code_hash_ignores_comments(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() != h0
     (csrc / "k.cu").write_text('int a = 1; // one\n/* block */ const char* s = "x/ /y";\n')
     assert bench.kernel_source_hash() != h0
+
+
+def test_cpu_baseline_reports_host_and_pinning():
+    """The oracle's timed CPU baseline on the tiny layer: pinned to one core
+    (the affinity is restored afterwards), median of 3 timings, and the host's
+    core count and CPU model stated."""
+    before = os.sched_getaffinity(0)
+    cb = bench.cpu_baseline(synthetic.WORKLOADS["tiny"], repeats=3, n_tok=2)
+    assert os.sched_getaffinity(0) == before
+    assert cb["cores"] == 1 and cb["kind"] == "oracle" and cb["unit"] == "tok/s"
+    assert len(cb["times_s"]) == 3 and cb["value"] == 2 / sorted(cb["times_s"])[1]
+    assert cb["pinned_core"] in before
+    assert cb["nproc"] >= 1 and isinstance(cb["cpu_model"], str)

@@ -217,3 +217,49 @@ def test_synthetic_inputs_are_deterministic():
     c = synthetic.expert_matrix(wl, 0, "gate", 4).numpy()
     assert np.array_equal(a, b) and not np.array_equal(a, c)
     assert abs(a.std() - 0.02) < 0.002
+
+
+def test_swiglu_against_fixed_values(orc):
+    """The activation between gate/up and down, pinned to literal values of
+    SiLU (a = g * sigmoid(g) * u; pxq_llama README, "Updates -- 2026-07-28":
+    the SiLU unary of the gate), so that a wrong activation shared with a
+    numpy restatement cannot pass.  One expert, top-1; single-nonzero weight
+    blocks and integer activation blocks with amax 127 make g and u exact:
+      - up: every row holds 4 at column 0 (scale 1/64), x[0] = 64, so u = 1;
+      - gate rows 32..35 hold 4 at their own column (scale 1/64), x = 127, 64,
+        -64, 0, so g = 1.984375, 1, -1, 0;
+      - gate rows 64, 65 hold 256 at their own column (scale 1), x = 127, -127,
+        so g = 127, -127 (the large-|g| limits);
+      - gate rows 0..31 are zero, so that activation block is all zeros.
+    The SwiGLU output is observed through its int8 requantization, within half
+    a quantization step of the literal values."""
+    H = F = 256
+    wg = np.zeros((F, H), np.float32)
+    for r in (32, 33, 34, 35):
+        wg[r, r] = 4.0
+    for r in (64, 65):
+        wg[r, r] = 256.0
+    wu = np.zeros((F, H), np.float32)
+    wu[:, 0] = 4.0
+    wd = np.zeros((H, F), np.float32)
+    layer = orc.Layer.from_float(H, F, 1, 1, wg, wu, wd)
+    x = np.zeros((1, H), np.float32)
+    x[0, 0], x[0, 1] = 64.0, 127.0
+    x[0, 32:36] = [127.0, 64.0, -64.0, 0.0]
+    x[0, 64], x[0, 65] = 127.0, -127.0
+    xq, xd = orc.quant_act_q8(x)
+    assert np.array_equal(xq[0].astype(np.float32) * np.repeat(xd[0], 32), x[0])  # exact inputs
+    _, dbg = orc.expert_ffn(layer, xq, xd, np.array([[0]], np.int32), np.ones((1, 1), np.float32), debug=True)
+    g, u, aq, ad = dbg["g"][0, 0], dbg["u"][0, 0], dbg["aq"][0, 0].astype(np.int64), dbg["ad"][0, 0]
+    assert np.all(u == 1.0)
+    assert list(g[32:36]) == [1.984375, 1.0, -1.0, 0.0] and list(g[64:66]) == [127.0, -127.0]
+    assert np.all(g[:32] == 0.0) and np.all(aq[:32] == 0) and ad[0] == 0.0
+    # block 1: amax = silu(1.984375) = 1.7445568667767222..., so ad = amax / 127
+    assert abs(float(ad[1]) * 127 - 1.7445568667767222) < 1e-6
+    step = float(ad[1])
+    assert aq[32] == 127
+    assert abs(aq[33] * step - 0.7310585786300049) <= step / 2    # silu(1)
+    assert abs(aq[34] * step - (-0.2689414213699951)) <= step / 2  # silu(-1)
+    assert aq[35] == 0                                              # silu(0) = 0
+    # block 2: silu(127) = 127 to fp32 precision, silu(-127) ~ -8.9e-54
+    assert float(ad[2]) == 1.0 and aq[64] == 127 and aq[65] == 0
