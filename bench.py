@@ -86,7 +86,7 @@ def kernel_bytes(wl, unique_experts):
     T, H, F, E, K = wl.ntok, wl.hidden, wl.ffn, wl.n_experts, wl.top_k
     pairs = T * K
     weights = unique_experts * wl.expert_bytes
-    return {
+    kb = {
         # the whole one-token step in one kernel: router, x, the routed
         # experts' packed weights, the int8 intermediates and y
         "step1": E * H * 4 + T * H * 4 + weights + 2 * (pairs * F + pairs * F // 32 * 4)
@@ -108,6 +108,9 @@ def kernel_bytes(wl, unique_experts):
         "down": unique_experts * wl.matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4
         + pairs * H * 4 * 2 + T * H * 4 + pairs * 8,
     }
+    # the tensor-core mat-vecs move the same bytes as the CUDA-core ones
+    kb["tc_gateup"], kb["tc_down"] = kb["gateup"], kb["down"]
+    return kb
 
 
 # --------------------------------------------------------------------------- clocks

@@ -36,6 +36,7 @@ EXPORTS = (
     "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
     "moe_sign_words", "moe_quantize_weights_sign", "moe_e16_code_words", "moe_quantize_weights_e16",
     "moe_quantize_weights_q8", "moe_shared_workspace_bytes", "moe_shared_ffn_add",
+    "moe_debug_ffn_blocksums", "moe_debug_wait_knob",
 )
 
 
@@ -107,6 +108,8 @@ def lib():
             "moe_trace_end": (ctypes.c_int, [p, i32]),
             "moe_kernel_name": (ctypes.c_char_p, [i32]),
             "moe_expert_ffn_decode_static": (ctypes.c_int, [p, i32, p, p, p, p, p, p]),
+            "moe_debug_ffn_blocksums": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, i32, p, p, p, p]),
+            "moe_debug_wait_knob": (ctypes.c_int, [p, sz, i32, i32, p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -401,6 +404,33 @@ def moe_debug_matvec(mat, xq, xd, want_isum=True, stream=None):
                                   ctypes.c_void_p(isum.data_ptr()) if isum is not None else None,
                                   _stream(stream)))
     return out, isum
+
+
+def moe_debug_ffn_blocksums(layer, xq, xd, idx, wts, ws, prefill=False, stream=None):
+    """The expert FFN through the tensor-core path (decode mat-vecs, or the
+    prefill GEMM with prefill=True) with its exact int32 block sums:
+    returns (y, isum_gu [pairs][2][ffn][hidden/32], isum_dn
+    [pairs][hidden][ffn/32], aq [pairs][ffn])."""
+    ntok = xq.shape[0]
+    K, H, F = idx.shape[1], layer.hidden, layer.ffn
+    dev = xq.device
+    y = torch.empty((ntok, H), dtype=torch.float32, device=dev)
+    gu = torch.zeros((ntok * K, 2, F, H // QBLOCK), dtype=torch.int32, device=dev)
+    dn = torch.zeros((ntok * K, H, F // QBLOCK), dtype=torch.int32, device=dev)
+    aq = torch.zeros((ntok * K, F), dtype=torch.int8, device=dev)
+    _check(lib().moe_debug_ffn_blocksums(
+        layer.c_ref(), ntok, _dev(xq, torch.int8, "xq"), _dev(xd, torch.float32, "xd"),
+        _dev(idx, torch.int32, "idx"), _dev(wts, torch.float32, "wts"), _dev(y, torch.float32, "y"),
+        ws.ptr(), ws.nbytes, int(bool(prefill)), ctypes.c_void_p(gu.data_ptr()),
+        ctypes.c_void_p(dn.data_ptr()), ctypes.c_void_p(aq.data_ptr()), _stream(stream)))
+    return y, gu, dn, aq
+
+
+def moe_debug_wait_knob(ws, mode, polls=0, stream=None):
+    """Test knob of the bounded device waits (see include/bitmoe.h): mode 1
+    makes the one-token step's logit poll run out, mode 2 the tensor-core
+    mat-vecs' mbarrier waits; 0 restores normal operation."""
+    _check(lib().moe_debug_wait_knob(ws.ptr(), ws.nbytes, int(mode), int(polls), _stream(stream)))
 
 
 # ---------------------------------------------------------------- tracing

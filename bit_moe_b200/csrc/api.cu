@@ -10,6 +10,7 @@
 #include "decode.cuh"
 #include "decode2.cuh"
 #include "prefill.cuh"
+#include "tcmv.cuh"
 #include "shared.cuh"
 #include "quant.cuh"
 #include "router.cuh"
@@ -263,6 +264,15 @@ static int launch_copy16(void* dst, const void* src, size_t bytes, cudaStream_t 
   return check_launch("forward_host: copy");
 }
 
+// One token of a ternary layer: the routing kernel and the tensor-core
+// mat-vecs, or the fused one-token step (chosen by layer size).
+#ifndef MOE_ONE_TOKEN_TC_MIN_HIDDEN
+#define MOE_ONE_TOKEN_TC_MIN_HIDDEN 1000000
+#endif
+static bool one_token_on_tensor_cores(const DecodeParams& P) {
+  return tc_ffn_supported(P) && P.hidden >= MOE_ONE_TOKEN_TC_MIN_HIDDEN;
+}
+
 // The checks of moe_expert_ffn_decode that do not involve a workspace (layer,
 // pointers, token count, device), for entry points that bring their own
 // scratch and must validate a call before touching it.
@@ -467,6 +477,11 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   Decode2Params D = make_d2(P, ws, W);
   D.x = x;
   D.wr = w_router;
+  if (one_token_on_tensor_cores(P)) {
+    // the routing kernel, then the tensor-core mat-vecs over the top_k slots
+    if ((rc = launch_route_only(D, s))) return rc;
+    return launch_ffn_tc(P, s);
+  }
   size_t smem1 = 0;
   if (step1_supported(P, D.n_sm, &smem1)) {
     WsHeader* hd = reinterpret_cast<WsHeader*>(ws);
@@ -594,7 +609,7 @@ const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
       "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather", "copy",
-      "router_quant", "topk_group", "shared"};
+      "router_quant", "topk_group", "shared", "tc_gateup", "tc_down"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 
@@ -614,6 +629,50 @@ int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const fl
     return fail(MOE_ERR_INVALID_ARG, "debug_matvec: E16 codes missing or not 16-byte aligned");
   if ((rc = check_device())) return rc;
   return launch_debug_matvec(m, ntok, xq, xd, out, isum, static_cast<cudaStream_t>(stream));
+}
+
+int moe_debug_ffn_blocksums(const moe_layer* L, int32_t ntok, const int8_t* xq, const float* xd,
+                            const int32_t* idx, const float* wts, float* y, void* ws, size_t ws_bytes,
+                            int32_t prefill, int32_t* isum_gu, int32_t* isum_dn, int8_t* aq,
+                            moe_stream_t stream) {
+  WsLayout W;
+  int rc = ffn_common("debug_ffn_blocksums", L, ntok, xq, xd, idx, wts, y, ws, ws_bytes, prefill != 0, &W);
+  if (rc) return rc;
+  if (!isum_gu || !isum_dn || !aligned16(isum_gu) || !aligned16(isum_dn))
+    return fail(MOE_ERR_INVALID_ARG, "debug_ffn_blocksums: isum_gu and isum_dn must be 16-byte aligned device arrays");
+  DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
+  P.dbg_isum_gu = isum_gu;
+  P.dbg_isum_dn = isum_dn;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prefill) {
+    if (!prefill_tc_supported(P))
+      return fail(MOE_ERR_UNSUPPORTED_SHAPE, "debug_ffn_blocksums: the prefill GEMM does not take this layer");
+    rc = launch_prefill(P, s);
+  } else {
+    if (!tc_ffn_supported(P))
+      return fail(MOE_ERR_UNSUPPORTED_SHAPE, "debug_ffn_blocksums: the tensor-core decode does not take this layer");
+    if (!P.direct && (rc = launch_group(P, s))) return rc;
+    if (!rc) rc = launch_ffn_tc(P, s);
+  }
+  if (rc || !aq) return rc;
+  const size_t bytes = static_cast<size_t>(ntok) * L->top_k * L->ffn;
+  cudaError_t err = cudaMemcpyAsync(aq, P.aq, bytes, cudaMemcpyDeviceToDevice, s);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "debug_ffn_blocksums: copy of aq: %s", cudaGetErrorString(err));
+  return MOE_OK;
+}
+
+int moe_debug_wait_knob(void* ws, size_t ws_bytes, int32_t mode, int32_t polls, moe_stream_t stream) {
+  if (!ws || ws_bytes < kWsHeaderBytes) return fail(MOE_ERR_INVALID_ARG, "debug_wait_knob: no workspace");
+  if (mode < 0 || mode > kKnobTcGather || polls < 0)
+    return fail(MOE_ERR_INVALID_ARG, "debug_wait_knob: mode %d, polls %d", mode, polls);
+  int rc = check_device();
+  if (rc) return rc;
+  const int32_t v[2] = {mode, polls};
+  cudaError_t err = cudaMemcpyAsync(static_cast<int32_t*>(ws) + kWsKnobMode, v, sizeof(v), cudaMemcpyHostToDevice,
+                                    static_cast<cudaStream_t>(stream));
+  if (err == cudaSuccess) err = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "debug_wait_knob: %s", cudaGetErrorString(err));
+  return MOE_OK;
 }
 
 }  // extern "C"

@@ -35,8 +35,17 @@ constexpr int kMaxDynSmem = 227 * 1024;  // opt-in dynamic shared memory per CTA
 // Workspace header: the first 256 bytes hold the device status word.
 struct WsHeader {
   int32_t status;    // first error code seen by a kernel (0 = ok)
-  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit one-token step tickets
+  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit one-token step tickets;
+                     // pad[8..9]: the wait test knob (below)
 };
+// Test knob of the bounded device waits (moe_debug_wait_knob; zero in every
+// fresh workspace): header word kWsKnobMode selects a wait that is made to run
+// out, word kWsKnobPolls (if nonzero) replaces the poll budget of the kernels
+// that read the knob.
+constexpr int kWsKnobMode = 9;   // word index in the header (pad[8])
+constexpr int kWsKnobPolls = 10; // pad[9]
+constexpr int kKnobStep1Tag = 1; // the one-token step polls for a logit tag that no CTA publishes
+constexpr int kKnobTcGather = 2; // the tensor-core mat-vecs' gather warp withholds its first arrival
 static_assert(offsetof(WsHeader, pad) + 3 * sizeof(int32_t) == 16, "8-byte aligned ticket counter");
 constexpr size_t kWsHeaderBytes = sizeof(WsHeader);
 

@@ -19,6 +19,7 @@
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "tcmv.cuh"
 #include "ternary_dot.cuh"
 #include "topk.cuh"
 
@@ -422,6 +423,8 @@ static void launch_ffn_fmt(const DecodeParams& P, cudaStream_t stream) {
 
 int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
   if (!P.direct && P.group_chunk != kChunk) return fail(MOE_ERR_INVALID_ARG, "expert_ffn: items of %d pairs", P.group_chunk);
+  // ternary layers of batches: the tensor-core mat-vecs
+  if (!P.direct && tc_ffn_supported(P)) return launch_ffn_tc(P, stream);
   init_kernel_attrs();
   if (P.format == MOE_FORMAT_SIGN) launch_ffn_fmt<MOE_FORMAT_SIGN>(P, stream);
   else if (P.format == MOE_FORMAT_E16) launch_ffn_fmt<MOE_FORMAT_E16>(P, stream);

@@ -44,6 +44,11 @@ struct DecodeParams {
   // the tensor-core kernel's shared-memory stages, for gate/up and for down
   unsigned char* bgu;                        // [groups][hidden/256] blocks
   unsigned char* bdn;                        // [groups][ffn/256] blocks
+  // test hook of the tensor-core mat-vecs (null otherwise): the exact block
+  // sums sum(q * a) of every pair, row and 32-block, gate/up as
+  // [pairs][2][ffn][hidden/32] and down as [pairs][hidden][ffn/32]
+  int32_t* dbg_isum_gu = nullptr;
+  int32_t* dbg_isum_dn = nullptr;
 };
 
 // Fetch work item `it`; returns false when there is none.

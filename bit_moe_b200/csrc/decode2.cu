@@ -507,6 +507,20 @@ static size_t route_smem_bytes(int H, int E, int W, int TC) {
   return a > b ? a : b;
 }
 
+int launch_route_only(Decode2Params& D, cudaStream_t stream) {
+  init_attrs2();
+  const DecodeParams& P = D.P;
+  int W, TC;
+  route_shape(P.hidden, P.n_experts, P.ntok, &W, &TC);
+  D.route_warps = W;
+  D.route_tc = TC;
+  dim3 grid((P.n_experts + W - 1) / W, (P.ntok + TC - 1) / TC);
+  cudaError_t err = launch_pdl(k_route, grid, dim3(W * 32), route_smem_bytes(P.hidden, P.n_experts, W, TC), stream, D);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "route: %s", cudaGetErrorString(err));
+  note_launch(MOE_K_ROUTE, stream);
+  return MOE_OK;
+}
+
 int launch_decode2(Decode2Params& D, bool with_route, cudaStream_t stream) {
   init_attrs2();
   const DecodeParams& P = D.P;

@@ -32,6 +32,9 @@ struct Decode2Params {
 };
 
 int launch_decode2(Decode2Params& D, bool with_route, cudaStream_t stream);
+// k_route alone (activation q8, router logits, top-k softmax into P.idx,
+// P.wts; grouping with more than one token), for the tensor-core mat-vecs.
+int launch_route_only(Decode2Params& D, cudaStream_t stream);
 
 // The whole one-token step in one cooperative kernel (step1.cu).
 bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem);

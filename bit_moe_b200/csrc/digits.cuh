@@ -19,17 +19,21 @@ namespace bitmoe {
 
 // Digit words [32*kHalf, 32*kHalf + 32) of one block from packed words
 // w[jj] = word 6*kHalf + jj, jj in [0, 7) (word 6 feeds both halves).
+// `three` must hold 3: a value the compiler cannot see, so that one of the two
+// lane multiplies of a level stays an integer multiply-add (FMA pipe) while
+// the other may become a shift-add (ALU pipe), and the two pipes share the
+// decode evenly.
 template <int kHalf>
-__device__ __forceinline__ void digit_half(const uint32_t (&w)[7], uint32_t (&dg)[32]) {
+__device__ __forceinline__ void digit_half(const uint32_t (&w)[7], uint32_t (&dg)[32], uint32_t three = 3u) {
 #pragma unroll
   for (int jj = 0; jj < 7; ++jj) {
     const int j = 6 * kHalf + jj;
-    uint32_t lo = w[jj] & 0x00FF00FFu, hi = (w[jj] >> 8) & 0x00FF00FFu, hp = 0u;
+    uint32_t lo = w[jj] & 0x00FF00FFu, hi = __byte_perm(w[jj], 0u, 0x4341), hp = 0u;
 #pragma unroll
     for (int i = 0; i < 5; ++i) {
       if (j == kBlockWords - 1 && i == 4) break;
       lo *= 3u;
-      hi *= 3u;
+      hi *= three;
       const uint32_t hn = __byte_perm(lo, hi, 0x7351);
       const int c = 5 * j + i - 32 * kHalf;
       if (c >= 0 && c < 32) dg[c] = hn - 3u * hp;

@@ -4,37 +4,35 @@
 // takes a GEMM path over the quantized tiles; pxq_llama README, "What's PXQ?":
 // a grouped-MoE GEMM, and "Updates -- 2026-07-19": an int8 prefill tile.
 //
-// The (token, slot) pairs are grouped by expert and cut into tiles of up to
-// kPN pairs.  A tile of the grouped GEMM is 128 weight rows x kPN pairs:
-//   - A (128 x 32 per MMA): the weights' base-3 digits t = q + 1 in {0,1,2},
-//     decoded in registers from the packed blocks and written straight into
-//     tensor memory with tcgen05.st.  Read as e4m3, the bytes 0, 1, 2 are the
-//     subnormals 0, 2^-9, 2^-8, i.e. exactly t * 2^-9, so the decoded digits
-//     need no conversion at all;
-//   - B (32 x kPN): each int8 activation code a = 16*h + l is split into two
-//     e4m3 operands, 16*h (h in [-8, 7]) and l (in [0, 15]), both exact; two
-//     MMAs accumulate t*16h and t*l into the same fp32 accumulator, which then
-//     holds 2^-9 * sum(t*a) exactly (every partial sum is a multiple of 2^-9
-//     below 2^4);
-//   - one fp32 TMEM accumulator per 32-value sub-block (the activation scale
-//     changes every 32 values); the epilogue forms sum(q*a) = 512*D - sum(a)
-//     and scales it in fp32 exactly like the decode kernels: sum over
-//     sub-blocks of d * sum(q*a), then the fp16 weight scale per 256-block.
+// The (token, slot) pairs are grouped by expert and cut into groups of up to
+// kPN = 128 pairs.  A tile of the grouped GEMM is 128 weight rows x one group,
+// one tcgen05.mma kind::i8 (M = 128, N = 128, K = 32) per 32-value sub-block:
+//   - A (tensor memory): the weights' base-3 digits t = q + 1 in {0, 1, 2} as
+//     u8, decoded in registers from the packed blocks (digits.cuh) and written
+//     straight into tensor memory -- the expanded weights exist nowhere else;
+//   - B (shared memory): the group's int8 activation codes as s8;
+//   - D (tensor memory): int32, exact.  Each accumulator stage starts at the
+//     integer 0x4B400000, so that after the MMA its bits read as the fp32
+//     value 12582912 + sum(t * a), exactly (|sum| < 2^13); one fp32
+//     subtraction of m = 12582912 + sum(a) then gives sum(q * a) exactly, and
+//     the fixup scales it as every decode kernel does: per block
+//     inner = sum_s fma(d_s, sum_s(q * a), inner), per row and pair
+//     y = fma(s_b, inner, y) over the blocks in order (y kept in tensor
+//     memory between blocks).
 // The activations of a tile are laid out once per (group, 256-block) in HBM
-// exactly as shared memory holds them (split codes in the MMA's core-matrix
-// layout, then the scales and code sums of the group's pairs): for gate/up by a
-// gather pass over x^, for down by the gate/up epilogue itself.  One bulk copy
-// (TMA) then brings each block's 18 KB into a shared-memory stage.
+// exactly as shared memory holds them (codes in the MMA's core-matrix layout,
+// then the scales and m of the group's pairs): for gate/up by a gather pass
+// over x^, for down by the gate/up epilogue itself.  One bulk copy (TMA) brings
+// each block's 40 KB into a shared-memory stage; the weights stream through
+// an 8-stage ring of bulk copies (one per 32-row panel and block).
 // The kernel is persistent (one CTA per SM) and warp-specialized: decode
 // warps write the digits of block i while the MMAs of block i-1 run and the
-// fixup warps drain the accumulators of earlier half blocks; mbarriers pass
-// each stage along (digits: 2 TMEM stages, activations: 3 shared-memory
-// stages, accumulators: 2 TMEM stages of half a block).
+// fixup warps drain the accumulators sub-block by sub-block; mbarriers pass
+// each stage along, and every wait is bounded.
 // Gate/up tiles hold 64 gate rows and the 64 matching up rows, so SwiGLU and
 // the requantization run in the epilogue; down tiles write each pair's rows,
 // and a last pass combines the top_k slots of every token in slot order.
 #include <atomic>
-#include <cuda_fp8.h>
 
 #include "bitmoe.h"
 #include "common.cuh"
@@ -45,65 +43,65 @@
 
 namespace bitmoe {
 
-constexpr int kPN = 64;           // pairs per tile (MMA N)
+constexpr int kPN = 128;          // pairs per group (MMA N)
 constexpr int kPM = 128;          // weight rows per tile (MMA M)
 // Warp roles of a CTA (one CTA per SM, persistent over the tiles):
 constexpr int kWDec = 0;          // warps 0-3: decode the digits into TMEM (thread = row)
 constexpr int kWFix = 4;          // warps 4-19: accumulator fixup and epilogue (thread = row,
-constexpr int kFixWarps = 16;     //   warp 4 + 4f + q: rows of quadrant q, pairs [8f, 8f + 8))
+constexpr int kFixWarps = 16;     //   warp 4 + 4f + q: rows of quadrant q, pairs [32f, 32f + 32))
 constexpr int kFixPairs = kPN / (kFixWarps / 4);
-constexpr int kWGat = 20;         // warp 20: lane 0 brings the activation blocks in (bulk copies)
-constexpr int kWMma = 21;         // warp 21: lane 0 issues the MMAs
-constexpr int kPThreads = 22 * 32;
+constexpr int kWCopyW = 20;       // warp 20: lane 0 brings the weight blocks in (bulk copies)
+constexpr int kWCopyB = 21;       // warp 21: lane 0 brings the activation blocks in (bulk copies)
+constexpr int kWMma = 22;         // warp 22: lane 0 issues the MMAs
+constexpr int kPThreads = 23 * 32;
+constexpr int kWStages = 8;       // weight ring: one block of the tile's 4 panels per stage
 constexpr int kAStages = 2;       // digit stages in TMEM, 64 columns each
-constexpr int kBStages = 3;       // code / scale stages in shared memory
-constexpr int kQSub = 2;          // sub-blocks per accumulator stage (a quarter of a block)
-constexpr int kDStages = 3;       // accumulator stages in flight
+constexpr int kBStages = 3;       // activation stages in shared memory
+constexpr int kDStages = 2;       // accumulator stages in TMEM: one sub-block (kPN columns) each
 constexpr int kTmemCols = 512;
 constexpr int kAcol = 0;          // A stage a: columns [64a, 64a + 64)
-constexpr int kDSub = kPN;        // D columns per sub-block: one fp32 accumulator per pair
-constexpr int kDcol = 128;        // D stage d: columns [128 + kQSub*kDSub*d, 128 + kQSub*kDSub*(d+1))
-static_assert(kDcol + kDStages * kQSub * kDSub <= 512, "tensor memory columns");
+constexpr int kDcol = 128;        // D stage d: columns [128 + kPN*d, 128 + kPN*(d+1))
+constexpr int kYcol = kDcol + kDStages * kPN;  // y of every (row, pair) between blocks
+static_assert(kYcol + kPN <= kTmemCols, "tensor memory columns");
+constexpr int kPanelBytes = kBlockWords * kPanel * 4;
+constexpr uint32_t kMagic = 0x4B400000u;  // bits of 12582912.0f
+constexpr float kMagicF = 12582912.0f;
 
-// One 256-wide block of a tile's activations, identical in HBM and in shared
-// memory: the split codes in the MMA layout, then per sub-block the pairs'
-// scales and code sums (negated).
+// One 256-wide block of a group's activations, identical in HBM and in shared
+// memory: the codes in the MMA layout, then per sub-block the pairs' scales
+// and m = 12582912 + sum of the codes.
 struct BStage {
-  unsigned char codes[2][kSubPerBlock * kPN * 32];  // 16*h parts, then l parts, MMA layout
-  float d[kSubPerBlock][kPN];                        // activation scales
-  float nsa[kSubPerBlock][kPN];                      // minus the code sums
+  unsigned char codes[kSubPerBlock * kPN * 32];
+  float d[kSubPerBlock][kPN];
+  float m[kSubPerBlock][kPN];
 };
 constexpr int kBTile = static_cast<int>(sizeof(BStage));
 static_assert(kBTile % 128 == 0, "bulk copies of whole stages");
 
 struct PrefillSmem {
+  uint64_t w_full[kWStages], w_empty[kWStages];
   uint64_t a_full[kAStages], a_empty[kAStages];
-  uint64_t b_full[kBStages], b_empty[kBStages], s_empty[kBStages];
+  uint64_t b_full[kBStages], b_empty[kBStages];
   uint64_t d_full[kDStages], d_empty[kDStages];
+  uint64_t fx_bar[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
+  alignas(128) uint32_t w[kWStages][4][kBlockWords * kPanel];  // packed words, [panel][word][row]
+  alignas(16) uint16_t wsc[kWStages][4][kPanel];                // fp16 block scales, [panel][row]
   alignas(128) BStage st[kBStages];
   float xch[64][kPN + 1];  // gate results for the up rows
 };
 
-// Byte offset of activation code (pair n, k in [0, 32)) of sub-block s in one
-// part's B operand: 8-row x 16-byte core matrices, the two 16-byte halves of K
-// 128 bytes apart, consecutive 8-pair groups 256 bytes apart.
+// Byte offset of activation code (pair n, k in [0, 32)) of sub-block s: 8-row
+// x 16-byte core matrices, the two 16-byte halves of K 128 bytes apart,
+// consecutive 8-pair groups 256 bytes apart.
 __device__ __forceinline__ int b_off(int s, int n, int k) {
   return s * (kPN * 32) + (n >> 3) * 256 + (k >> 4) * 128 + (n & 7) * 16 + (k & 15);
 }
 
-// e4m3 bytes of the two parts of an activation code q = 16*h + l.
-__device__ __forceinline__ void code_split(int q, uint8_t& hi, uint8_t& lo) {
-  const int h = q >> 4;  // floor(q / 16), in [-8, 7]
-  const int l = q & 15;
-  hi = static_cast<uint8_t>(__nv_cvt_float_to_fp8(static_cast<float>(h * 16), __NV_SATFINITE, __NV_E4M3));
-  lo = static_cast<uint8_t>(__nv_cvt_float_to_fp8(static_cast<float>(l), __NV_SATFINITE, __NV_E4M3));
-}
-
-// The gate/up activation blocks of every group: thread (n, s) of a CTA
-// splits the 32 codes of sub-block s of pair n's token and adds them up.
+// The gate/up activation blocks of every group: thread (n, s) of a CTA copies
+// the 32 codes of sub-block s of pair n's token and adds them up.
 __global__ void __launch_bounds__(kPN * kSubPerBlock) k_prefill_gather(DecodeParams P) {
   pdl_enter();
   const int H = P.hidden, K = P.top_k, nb = H / kBlock;
@@ -125,25 +123,19 @@ __global__ void __launch_bounds__(kPN * kSubPerBlock) k_prefill_gather(DecodePar
     int sum = 0;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int8_t* q = reinterpret_cast<const int8_t*>(&c[h]);
-      int4 hv, lv;
-      uint8_t* hb = reinterpret_cast<uint8_t*>(&hv);
-      uint8_t* lb = reinterpret_cast<uint8_t*>(&lv);
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        code_split(q[k], hb[k], lb[k]);
-        sum += q[k];
-      }
-      *reinterpret_cast<int4*>(dst->codes[0] + b_off(s, n, 16 * h)) = hv;
-      *reinterpret_cast<int4*>(dst->codes[1] + b_off(s, n, 16 * h)) = lv;
+      sum = __dp4a(c[h].x, 0x01010101, sum);
+      sum = __dp4a(c[h].y, 0x01010101, sum);
+      sum = __dp4a(c[h].z, 0x01010101, sum);
+      sum = __dp4a(c[h].w, 0x01010101, sum);
+      *reinterpret_cast<int4*>(dst->codes + b_off(s, n, 16 * h)) = c[h];
     }
     dst->d[s][n] = d;
-    dst->nsa[s][n] = -static_cast<float>(sum);
+    dst->m[s][n] = kMagicF + static_cast<float>(sum);
   }
 }
 
-// Two independent fp32 fused multiply-adds, round to nearest each, in one
-// packed instruction: (r0, r1) = (a0*b0 + c0, a1*b1 + c1).
+// Two independent fp32 operations, round to nearest each, in one packed
+// instruction: (r0, r1) = (a0*b0 + c0, a1*b1 + c1), and (a0 - b0, a1 - b1).
 __device__ __forceinline__ void fma2(float& r0, float& r1, float a0, float a1, float b0, float b1, float c0,
                                      float c1) {
   asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
@@ -151,64 +143,81 @@ __device__ __forceinline__ void fma2(float& r0, float& r1, float a0, float a1, f
       : "=f"(r0), "=f"(r1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
+__device__ __forceinline__ void sub2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Store the same 32-bit value into 32 consecutive columns of this thread's
+// TMEM lane.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
+      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
 
 // Tile t of the grouped GEMM: item (expert, pairs) and 128-row tile index.
 struct TileInfo {
   Item it;
-  int mt;
+  int item, mt;
 };
-__device__ __forceinline__ TileInfo tile_info(const DecodeParams& P, int t, int m_tiles) {
-  TileInfo T;
-  T.it = P.items[t / m_tiles];
+__device__ __forceinline__ bool tile_info(const DecodeParams& P, int t, int m_tiles, TileInfo& T) {
+  T.item = t / m_tiles;
+  if (T.item >= *P.n_items) return false;
+  T.it = P.items[T.item];
   T.mt = t % m_tiles;
-  return T;
+  return true;
 }
 
-// The row of this thread in a tile (quadrant q, lane): matrix and panel.
+// Panel p (0..3) of a tile: gate/up tiles are gate panels 2mt, 2mt+1 then up
+// panels 2mt, 2mt+1 of the expert; down tiles are panels 4mt..4mt+3.
 template <bool kGU>
-__device__ __forceinline__ void tile_row(const DecodeParams& P, const TileInfo& T, int q, const uint32_t*& trits,
-                                         const uint16_t*& scales, size_t& panel) {
-  if (kGU) {
-    const bool up = q >= 2;
-    trits = up ? P.up_trits : P.gate_trits;
-    scales = up ? P.up_scales : P.gate_scales;
-    panel = (static_cast<size_t>(T.it.expert) * P.ffn + 64 * T.mt) / kPanel + (q & 1);
-  } else {
-    trits = P.down_trits;
-    scales = P.down_scales;
-    panel = (static_cast<size_t>(T.it.expert) * P.hidden + kPM * T.mt) / kPanel + q;
-  }
+__device__ __forceinline__ size_t tile_panel_index(const DecodeParams& P, const TileInfo& T, int p) {
+  if (kGU) return static_cast<size_t>(T.it.expert) * (P.ffn / kPanel) + 2 * T.mt + (p & 1);
+  return static_cast<size_t>(T.it.expert) * (P.hidden / kPanel) + 4 * T.mt + p;
+}
+template <bool kGU>
+__device__ __forceinline__ const uint32_t* panel_trits(const DecodeParams& P, int p) {
+  return kGU ? (p < 2 ? P.gate_trits : P.up_trits) : P.down_trits;
+}
+template <bool kGU>
+__device__ __forceinline__ const uint16_t* panel_scales(const DecodeParams& P, int p) {
+  return kGU ? (p < 2 ? P.gate_scales : P.up_scales) : P.down_scales;
 }
 
 // The gate/up epilogue's output for pairs [n0, n0 + kFixPairs) at ffn row f of a
 // tile: each lane (32 consecutive f, one 32-block) requantizes the SwiGLU
-// values a[] (absent pairs and bad groups: zeros) and writes the split codes,
-// scale and code sum into the down input's activation block of the group.
+// values a[] (absent pairs and bad groups: zeros) and writes the codes, scale
+// and m into the down input's activation block of the group.
 __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, int item, int r, int n0,
-                                                 const float* a, int count, int lane) {
+                                                 const float* a, const Item& it, int lane) {
   const int F = P.ffn;
   const int f = 64 * mt + r;
   const int bf = f / kBlock, sub = (f % kBlock) / kQBlock;
   BStage* dst = reinterpret_cast<BStage*>(P.bdn) + static_cast<size_t>(item) * (F / kBlock) + bf;
-#pragma unroll
+#pragma unroll 4
   for (int n = 0; n < kFixPairs; ++n) {
     const int np = n0 + n;
     float dd = 0.f;
     int qq = 0;
-    if (a != nullptr && np < count) {
+    if (a != nullptr && np < it.count) {
       const float amax = warp_max(fabsf(a[n]));
       dd = __fdiv_rn(amax, 127.f);
       if (dd != 0.f) qq = max(-127, min(127, __float2int_rn(__fdiv_rn(a[n], dd))));
     }
-    uint8_t hi, lo;
-    code_split(qq, hi, lo);
-    dst->codes[0][b_off(sub, np, lane)] = hi;
-    dst->codes[1][b_off(sub, np, lane)] = lo;
+    dst->codes[b_off(sub, np, lane)] = static_cast<unsigned char>(static_cast<int8_t>(qq));
     const int sum = __reduce_add_sync(0xffffffffu, qq);
     if (lane == 0) {
       dst->d[sub][np] = dd;
-      dst->nsa[sub][np] = -static_cast<float>(sum);
+      dst->m[sub][np] = kMagicF + static_cast<float>(sum);
     }
+    if (P.dbg_isum_gu != nullptr && np < it.count)  // test hook: the SwiGLU codes
+      P.aq[static_cast<size_t>(P.pairs[it.start + np]) * F + f] = static_cast<int8_t>(qq);
   }
 }
 
@@ -230,20 +239,19 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   const int kdim = kGU ? H : F;               // reduction length
   const int nb = kdim / kBlock;
   const int m_tiles = kGU ? F / 64 : H / kPM;
-  const int n_tiles = *P.n_items * m_tiles;
 
   if (warp == 0) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
+    // a weight stage is free once the 4 decode warps have its words and the 16
+    // fixup warps its scales
+    for (int i = 0; i < kWStages; ++i) { mbar_init(&S.w_full[i], 1); mbar_init(&S.w_empty[i], 4 + kFixWarps); }
     for (int i = 0; i < kAStages; ++i) { mbar_init(&S.a_full[i], 4); mbar_init(&S.a_empty[i], 1); }
-    for (int i = 0; i < kBStages; ++i) {
-      mbar_init(&S.b_full[i], 1);
-      mbar_init(&S.b_empty[i], 1);
-      mbar_init(&S.s_empty[i], kFixWarps);
-    }
+    for (int i = 0; i < kBStages; ++i) { mbar_init(&S.b_full[i], 1); mbar_init(&S.b_empty[i], 1 + kFixWarps); }
     for (int i = 0; i < kDStages; ++i) { mbar_init(&S.d_full[i], 1); mbar_init(&S.d_empty[i], kFixWarps); }
+    for (int i = 0; i < 2; ++i) mbar_init(&S.fx_bar[i], kFixWarps);
     mbar_init(&S.mma_done, 1);
     fence_mbar_init();
     S.abort = 0;
@@ -252,220 +260,260 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
+  if (warp >= kWFix && warp < kWFix + kFixWarps) {
+    // every accumulator stage starts at the magic integer before the first MMA
+    const int q = (warp - kWFix) & 3, f = (warp - kWFix) >> 2;
+    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
+    for (int ds = 0; ds < kDStages; ++ds) tmem_fill32(tl + kDcol + kPN * ds + kFixPairs * f, kMagic);
+    tc_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp >= kWDec && warp < kWFix) {
     // ------------------------------------------------ decode: digits -> TMEM
     const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    // the CTA's sequence of (tile, block): the next one's words are loaded
-    // while the current one is decoded
-    int t = blockIdx.x, b = 0;
-    auto skip_bad = [&]() {
-      while (t < n_tiles && P.items[t / m_tiles].expert < 0) t += gridDim.x;
-    };
-    auto load = [&](int tt, int bb, uint32_t (&w)[kBlockWords]) {
-      const TileInfo T = tile_info(P, tt, m_tiles);
-      const uint32_t* trits;
-      const uint16_t* scales;
-      size_t panel;
-      tile_row<kGU>(P, T, warp, trits, scales, panel);
-      const size_t pb = panel * nb + bb;
+    uint32_t wi = 0;
+    TileInfo T;
+    for (int t = blockIdx.x; tile_info(P, t, m_tiles, T); t += gridDim.x) {
+      if (T.it.expert < 0) continue;
+      bool ok = true;
+      for (int b = 0; b < nb; ++b, ++wi) {
+        const int ws = wi % kWStages, a = wi % kAStages;
+        if (!wait_or_abort(&S.w_full[ws], (wi / kWStages) & 1u, S, P.status)) { ok = false; break; }
+        uint32_t w[kBlockWords];
 #pragma unroll
-      for (int j = 0; j < kBlockWords; ++j) w[j] = ld_stream_u32(trits + (pb * kBlockWords + j) * kPanel + lane);
-    };
-    skip_bad();
-    uint32_t wn[kBlockWords];
-    if (t < n_tiles) load(t, 0, wn);
-    for (uint32_t i = 0; t < n_tiles; ++i) {
-      uint32_t w[kBlockWords];
+        for (int j = 0; j < kBlockWords; ++j) w[j] = S.w[ws][warp][j * kPanel + lane];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.w_empty[ws]);
+        if (!wait_or_abort(&S.a_empty[a], ((wi / kAStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
 #pragma unroll
-      for (int j = 0; j < kBlockWords; ++j) w[j] = wn[j];
-      // advance to the next (tile, block) and start its loads
-      int tn = t, bn = b + 1;
-      if (bn == nb) {
-        bn = 0;
-        tn += gridDim.x;
-        while (tn < n_tiles && P.items[tn / m_tiles].expert < 0) tn += gridDim.x;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w7[7], dg[32];
+#pragma unroll
+          for (int jj = 0; jj < 7; ++jj) w7[jj] = w[6 * h + jj];
+          if (h == 0) digit_half<0>(w7, dg);
+          else digit_half<1>(w7, dg);
+          tmem_st32(tlane + kAcol + 64 * a + 32 * h, dg);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.a_full[a]);
       }
-      if (tn < n_tiles) load(tn, bn, wn);
-      const int a = i % kAStages;
-      if (!wait_or_abort(&S.a_empty[a], ((i / kAStages) & 1u) ^ 1u, S, P.status)) break;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t w7[7], dg[32];
-#pragma unroll
-        for (int jj = 0; jj < 7; ++jj) w7[jj] = w[6 * h + jj];
-        if (h == 0) digit_half<0>(w7, dg);
-        else digit_half<1>(w7, dg);
-        tmem_st32(tlane + kAcol + 64 * a + 32 * h, dg);
-      }
-      tc_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a_full[a]);
-      t = tn;
-      b = bn;
+      if (!ok) break;
     }
-  } else if (warp < kWGat) {
+  } else if (warp < kWFix + kFixWarps) {
     // ------------------------------------------------ fixup and epilogue
-    const int q = (warp - kWFix) & 3, f16 = (warp - kWFix) >> 2;  // lane quadrant, pair group
+    const int q = (warp - kWFix) & 3, f = (warp - kWFix) >> 2;  // lane quadrant, pair group
+    const int n0 = kFixPairs * f;
     const uint32_t tlane = tbase + (static_cast<uint32_t>(q * 32) << 16);
-    uint32_t i = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-      const TileInfo T = tile_info(P, t, m_tiles);
-      // pair n of the tile: lane n & 31 of mp[n >> 5]
-      const int mp0 = lane < T.it.count ? P.pairs[T.it.start + lane] : -1;
-      const int mp1 = lane + 32 < T.it.count ? P.pairs[T.it.start + lane + 32] : -1;
-      auto pair_at = [&](int n) { return __shfl_sync(0xffffffffu, n < 32 ? mp0 : mp1, n & 31); };
+    uint32_t bi = 0, si = 0, ep = 0;
+    TileInfo T;
+    for (int t = blockIdx.x; tile_info(P, t, m_tiles, T); t += gridDim.x) {
       if (T.it.expert < 0) {  // ids out of range: their outputs are zero
         if (warp == kWFix && lane == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
         if (kGU) {
-          if (q >= 2) write_down_codes(P, T.mt, t / m_tiles, 32 * (q - 2) + lane, kFixPairs * f16, nullptr, 0, lane);
+          if (q >= 2) write_down_codes(P, T.mt, T.item, 32 * (q - 2) + lane, n0, nullptr, T.it, lane);
         } else {
-          for (int n = kFixPairs * f16; n < kFixPairs * f16 + kFixPairs; ++n) {
-            const int pair = pair_at(n);
-            if (n < T.it.count) P.ye[static_cast<size_t>(pair) * H + kPM * T.mt + 32 * q + lane] = 0.f;
-          }
+          for (int n = n0; n < n0 + kFixPairs && n < T.it.count; ++n)
+            P.ye[static_cast<size_t>(P.pairs[T.it.start + n]) * H + kPM * T.mt + 32 * q + lane] = 0.f;
         }
         continue;
       }
-      const uint32_t* trits;
-      const uint16_t* scales;
-      size_t panel;
-      tile_row<kGU>(P, T, q, trits, scales, panel);
-      float y[kFixPairs];
-#pragma unroll
-      for (int n = 0; n < kFixPairs; ++n) y[n] = 0.f;
-      uint16_t sn = scales[(panel * nb) * kPanel + lane];
       bool ok = true;
-      for (int b = 0; b < nb && ok; ++b, ++i) {
-        const float sw = f16_bits_to_f32(sn);
-        if (b + 1 < nb) sn = scales[(panel * nb + b + 1) * kPanel + lane];
-        const int bs = i % kBStages;
-        if (!wait_or_abort(&S.b_full[bs], (i / kBStages) & 1u, S, P.status)) { ok = false; break; }
-        float inner[kFixPairs];
+      float inner[kFixPairs];  // per block the scaled sub-block sums, at the end y
+      for (int b = 0; b < nb && ok; ++b, ++bi) {
+        // the row's block scale from the weight stage of this block
+        const int ws = bi % kWStages;
+        if (!wait_or_abort(&S.w_full[ws], (bi / kWStages) & 1u, S, P.status)) { ok = false; break; }
+        const float sw = f16_bits_to_f32(S.wsc[ws][q][lane]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.w_empty[ws]);
+        const int bs = bi % kBStages;
+        if (!wait_or_abort(&S.b_full[bs], (bi / kBStages) & 1u, S, P.status)) { ok = false; break; }
 #pragma unroll
         for (int n = 0; n < kFixPairs; ++n) inner[n] = 0.f;
 #pragma unroll 1
-        for (int h = 0; h < kSubPerBlock / kQSub; ++h) {
-          const uint32_t j2 = (kSubPerBlock / kQSub) * i + h;
-          const int ds = j2 % kDStages;
-          if (!wait_or_abort(&S.d_full[ds], (j2 / kDStages) & 1u, S, P.status)) { ok = false; break; }
+        for (int s = 0; s < kSubPerBlock; ++s, ++si) {
+          const int ds = si % kDStages;
+          if (!wait_or_abort(&S.d_full[ds], (si / kDStages) & 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
-          // kQSub sub-blocks x this warp's pairs, one sub-block at a time; the
-          // stage goes back to the MMA once the last one is in registers
+          const uint32_t col = tlane + kDcol + kPN * ds + n0;
 #pragma unroll
-          for (int s2 = 0; s2 < kQSub; ++s2) {
-            uint32_t v[kFixPairs];
-            tmem_ld16(tlane + kDcol + kQSub * kDSub * ds + kDSub * s2 + kFixPairs * f16, v);
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t v[16];
+            tmem_ld16(col + 16 * hf, v);
             tc_wait_ld();
-            if (s2 == kQSub - 1) {
+            if (hf == 1) {
+              // the stage goes back to the MMA at the magic integer
+              tmem_fill32(col, kMagic);
+              tc_wait_st();
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&S.d_empty[ds]);
             }
-            const int s = kQSub * h + s2;
-            const float4* dp = reinterpret_cast<const float4*>(&S.st[bs].d[s][kFixPairs * f16]);
-            const float4* ap = reinterpret_cast<const float4*>(&S.st[bs].nsa[s][kFixPairs * f16]);
+            const float* dp = &S.st[bs].d[s][n0 + 16 * hf];
+            const float* mp = &S.st[bs].m[s][n0 + 16 * hf];
+            if ((kGU ? P.dbg_isum_gu : P.dbg_isum_dn) != nullptr) {  // test hook: the exact block sums
 #pragma unroll
-            for (int n4 = 0; n4 < kFixPairs / 4; ++n4) {
-              const float4 dd = dp[n4], aa = ap[n4];
-              // 512 * D - sum(a) = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
-              const uint32_t* vv = &v[4 * n4];
-              float q0, q1, q2, q3;
-              fma2(q0, q1, __uint_as_float(vv[0]), __uint_as_float(vv[1]), 512.f, 512.f, aa.x, aa.y);
-              fma2(q2, q3, __uint_as_float(vv[2]), __uint_as_float(vv[3]), 512.f, 512.f, aa.z, aa.w);
-              fma2(inner[4 * n4], inner[4 * n4 + 1], dd.x, dd.y, q0, q1, inner[4 * n4], inner[4 * n4 + 1]);
-              fma2(inner[4 * n4 + 2], inner[4 * n4 + 3], dd.z, dd.w, q2, q3, inner[4 * n4 + 2], inner[4 * n4 + 3]);
+              for (int e = 0; e < 16; ++e) {
+                const int np = n0 + 16 * hf + e;
+                if (np >= T.it.count) continue;
+                const int pair = P.pairs[T.it.start + np];
+                const int isum = static_cast<int>(__fsub_rn(__uint_as_float(v[e]), mp[e]));
+                const int sg = b * kSubPerBlock + s;
+                if (kGU) {
+                  const int fr = 64 * T.mt + 32 * (q & 1) + lane;
+                  P.dbg_isum_gu[((static_cast<size_t>(pair) * 2 + (q >> 1)) * F + fr) * (H / kQBlock) + sg] = isum;
+                } else {
+                  const int hr = kPM * T.mt + 32 * q + lane;
+                  P.dbg_isum_dn[(static_cast<size_t>(pair) * H + hr) * (F / kQBlock) + sg] = isum;
+                }
+              }
+            }
+#pragma unroll
+            for (int n4 = 0; n4 < 4; ++n4) {
+              const float4 dd = reinterpret_cast<const float4*>(dp)[n4];
+              const float4 mm = reinterpret_cast<const float4*>(mp)[n4];
+              const int nn = 16 * hf + 4 * n4;
+              // D - m = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
+              float i0, i1, i2, i3;
+              sub2(i0, i1, __uint_as_float(v[4 * n4]), __uint_as_float(v[4 * n4 + 1]), mm.x, mm.y);
+              sub2(i2, i3, __uint_as_float(v[4 * n4 + 2]), __uint_as_float(v[4 * n4 + 3]), mm.z, mm.w);
+              fma2(inner[nn], inner[nn + 1], dd.x, dd.y, i0, i1, inner[nn], inner[nn + 1]);
+              fma2(inner[nn + 2], inner[nn + 3], dd.z, dd.w, i2, i3, inner[nn + 2], inner[nn + 3]);
             }
           }
         }
         if (!ok) break;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.s_empty[bs]);
+        if (lane == 0) mbar_arrive(&S.b_empty[bs]);
+        // y = fma(sw, inner, y) over the blocks in order, y kept in TMEM
+        // between blocks (inner holds y from here on)
+        if (b == 0) {
 #pragma unroll
-        for (int n = 0; n < kFixPairs; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
+          for (int n = 0; n < kFixPairs; ++n) inner[n] = __fmaf_rn(sw, inner[n], 0.f);
+        } else {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t v[16];
+            tmem_ld16(tlane + kYcol + n0 + 16 * hf, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int n = 0; n < 16; ++n) inner[16 * hf + n] = __fmaf_rn(sw, inner[16 * hf + n], __uint_as_float(v[n]));
+          }
+        }
+        if (b + 1 < nb) {
+          uint32_t yb[kFixPairs];
+#pragma unroll
+          for (int n = 0; n < kFixPairs; ++n) yb[n] = __float_as_uint(inner[n]);
+          tmem_st32(tlane + kYcol + n0, yb);
+          tc_wait_st();
+        }
       }
       if (!ok) break;
-      // ---- epilogue (rows 32*q + lane, pairs [kFixPairs*f16, kFixPairs*f16 + kFixPairs))
+      // ---- epilogue (rows 32*q + lane, pairs [n0, n0 + kFixPairs))
       if (kGU) {
         if (q < 2) {
 #pragma unroll
-          for (int n = 0; n < kFixPairs; ++n) S.xch[32 * q + lane][kFixPairs * f16 + n] = y[n];
+          for (int n = 0; n < kFixPairs; ++n) S.xch[32 * q + lane][n0 + n] = inner[n];
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kFixWarps * 32) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.fx_bar[0]);
+        if (!wait_or_abort(&S.fx_bar[0], ep & 1u, S, P.status)) break;
         if (q >= 2) {
           const int r = 32 * (q - 2) + lane;  // f offset within the tile
           float a[kFixPairs];
 #pragma unroll
           for (int n = 0; n < kFixPairs; ++n) {
-            const float g = S.xch[r][kFixPairs * f16 + n];
-            a[n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
+            const float g = S.xch[r][n0 + n];
+            a[n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), inner[n]);
           }
-          write_down_codes(P, T.mt, t / m_tiles, r, kFixPairs * f16, a, T.it.count, lane);
+          write_down_codes(P, T.mt, T.item, r, n0, a, T.it, lane);
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kFixWarps * 32) : "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.fx_bar[1]);
+        if (!wait_or_abort(&S.fx_bar[1], ep & 1u, S, P.status)) break;
+        ++ep;
       } else {
         const int hrow = kPM * T.mt + 32 * q + lane;
+        for (int n = 0; n < kFixPairs && n0 + n < T.it.count; ++n)
+          P.ye[static_cast<size_t>(P.pairs[T.it.start + n0 + n]) * H + hrow] = inner[n];
+      }
+    }
+  } else if (warp == kWCopyW && lane == 0) {
+    // ------------------------------------------------ weight blocks: 4 bulk copies each
+    const uint64_t pol = policy_evict_first();
+    uint32_t wi = 0;
+    bool ok = true;
+    TileInfo T;
+    for (int t = blockIdx.x; ok && tile_info(P, t, m_tiles, T); t += gridDim.x) {
+      if (T.it.expert < 0) continue;
+      const uint32_t* src[4];
+      const uint16_t* ssrc[4];
 #pragma unroll
-        for (int n = 0; n < kFixPairs; ++n) {
-          const int np = kFixPairs * f16 + n;
-          const int pair = pair_at(np);
-          if (np < T.it.count) P.ye[static_cast<size_t>(pair) * H + hrow] = y[n];
+      for (int p = 0; p < 4; ++p) {
+        src[p] = panel_trits<kGU>(P, p) + tile_panel_index<kGU>(P, T, p) * nb * kBlockWords * kPanel;
+        ssrc[p] = panel_scales<kGU>(P, p) + tile_panel_index<kGU>(P, T, p) * nb * kPanel;
+      }
+      for (int b = 0; b < nb; ++b, ++wi) {
+        const int ws = wi % kWStages;
+        if (!wait_or_abort(&S.w_empty[ws], ((wi / kWStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&S.w_full[ws], 4 * (kPanelBytes + kPanel * 2));
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          bulk_g2s(S.w[ws][p], src[p] + static_cast<size_t>(b) * kBlockWords * kPanel, kPanelBytes, &S.w_full[ws],
+                   pol);
+          bulk_g2s(S.wsc[ws][p], ssrc[p] + static_cast<size_t>(b) * kPanel, kPanel * 2, &S.w_full[ws], pol);
         }
       }
     }
-  } else if (warp == kWGat && lane == 0) {
+    for (uint32_t k = wi > kWStages ? wi - kWStages : 0; k < wi; ++k)  // copies still in flight land
+      if (!mbar_wait(&S.w_full[k % kWStages], (k / kWStages) & 1u)) record_status(P.status, MOE_ERR_TIMEOUT);
+  } else if (warp == kWCopyB && lane == 0) {
     // ------------------------------------------------ activation blocks: one bulk copy each
     const unsigned char* src = kGU ? P.bgu : P.bdn;
     const uint64_t pol = policy_evict_last();  // each block serves all the group's row tiles
-    uint32_t i = 0;
-    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
-      const int item = t / m_tiles;
-      if (P.items[item].expert < 0) continue;
-      bool ok = true;
-      for (int b = 0; b < nb; ++b, ++i) {
-        const int bs = i % kBStages;
-        const uint32_t par = ((i / kBStages) & 1u) ^ 1u;
-        if (!wait_or_abort(&S.b_empty[bs], par, S, P.status) || !wait_or_abort(&S.s_empty[bs], par, S, P.status)) {
-          ok = false;
-          break;
-        }
+    uint32_t bi = 0;
+    bool ok = true;
+    TileInfo T;
+    for (int t = blockIdx.x; ok && tile_info(P, t, m_tiles, T); t += gridDim.x) {
+      if (T.it.expert < 0) continue;
+      for (int b = 0; b < nb; ++b, ++bi) {
+        const int bs = bi % kBStages;
+        if (!wait_or_abort(&S.b_empty[bs], ((bi / kBStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
         mbar_arrive_expect_tx(&S.b_full[bs], kBTile);
-        bulk_g2s(&S.st[bs], src + (static_cast<size_t>(item) * nb + b) * kBTile, kBTile, &S.b_full[bs], pol);
+        bulk_g2s(&S.st[bs], src + (static_cast<size_t>(T.item) * nb + b) * kBTile, kBTile, &S.b_full[bs], pol);
       }
-      if (!ok) break;
     }
+    for (uint32_t k = bi > kBStages ? bi - kBStages : 0; k < bi; ++k)
+      if (!mbar_wait(&S.b_full[k % kBStages], (k / kBStages) & 1u)) record_status(P.status, MOE_ERR_TIMEOUT);
   } else if (warp == kWMma && lane == 0) {
     // ------------------------------------------------ MMA issue
-    const uint32_t idesc = idesc_e4m3(kPM, kPN);
-    uint32_t i = 0;
+    const uint32_t idesc = idesc_i8(kPM, kPN);
+    uint32_t bi = 0, si = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-      if (P.items[t / m_tiles].expert < 0) continue;
-      for (int b = 0; b < nb; ++b, ++i) {
-        const int a = i % kAStages, bs = i % kBStages;
-        if (!wait_or_abort(&S.a_full[a], (i / kAStages) & 1u, S, P.status) ||
-            !wait_or_abort(&S.b_full[bs], (i / kBStages) & 1u, S, P.status)) {
+    TileInfo T;
+    for (int t = blockIdx.x; ok && tile_info(P, t, m_tiles, T); t += gridDim.x) {
+      if (T.it.expert < 0) continue;
+      for (int b = 0; b < nb; ++b, ++bi) {
+        const int a = bi % kAStages, bs = bi % kBStages;
+        if (!wait_or_abort(&S.a_full[a], (bi / kAStages) & 1u, S, P.status) ||
+            !wait_or_abort(&S.b_full[bs], (bi / kBStages) & 1u, S, P.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t bdesc0 = smem_desc(smem_u32(S.st[bs].codes[0]), 128, 256);
-        const uint64_t bdesc1 = smem_desc(smem_u32(S.st[bs].codes[1]), 128, 256);
-        for (int h = 0; h < kSubPerBlock / kQSub; ++h) {
-          const uint32_t j2 = (kSubPerBlock / kQSub) * i + h;
-          const int ds = j2 % kDStages;
-          if (!wait_or_abort(&S.d_empty[ds], ((j2 / kDStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
+        const uint64_t bdesc = smem_desc(smem_u32(S.st[bs].codes), 128, 256);
+        for (int s = 0; s < kSubPerBlock; ++s, ++si) {
+          const int ds = si % kDStages;
+          if (!wait_or_abort(&S.d_empty[ds], ((si / kDStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int s2 = 0; s2 < kQSub; ++s2) {
-            const int s = kQSub * h + s2;
-            // start address field (bits 0-13, address >> 4) advanced by the sub-block's offset
-            const uint64_t off = static_cast<uint64_t>((s * kPN * 32) >> 4);
-            const uint32_t dcol = tbase + kDcol + kQSub * kDSub * ds + kDSub * s2, acol = tbase + kAcol + 64 * a + 8 * s;
-            mma_f8_ts(dcol, acol, bdesc0 + off, idesc, false);
-            mma_f8_ts(dcol, acol, bdesc1 + off, idesc, true);
-          }
+          // the stage holds the magic integer: accumulate onto it
+          mma_i8_ts(tbase + kDcol + kPN * ds, tbase + kAcol + 64 * a + 8 * s,
+                    bdesc + static_cast<uint64_t>((s * kPN * 32) >> 4), idesc, true);
           mma_commit(&S.d_full[ds]);
         }
         if (!ok) break;
@@ -515,6 +563,7 @@ static size_t prefill_smem() {
 
 size_t prefill_block_bytes() { return kBTile; }
 int prefill_group_pairs() { return kPN; }
+bool prefill_tc_supported(const DecodeParams& P) { return P.format == MOE_FORMAT_TERNARY; }
 
 int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   DecodeParams P = P0;

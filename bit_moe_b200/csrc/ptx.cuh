@@ -47,10 +47,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 // Wait for the phase with the given parity to complete, the thread suspended
 // in the barrier between checks (each check gives up after a hint of 20 us,
 // so that a waiting warp takes no issue slots from the working ones).
-// Returns false after about 2^17 checks (seconds).
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+// Returns false after `checks` checks (by default 2^17: seconds).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t checks = 1u << 17) {
   const uint32_t a = smem_u32(bar);
-  for (uint32_t i = 0; i < (1u << 17); ++i) {
+  for (uint32_t i = 0; i < checks; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"

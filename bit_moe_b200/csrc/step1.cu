@@ -197,7 +197,12 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   if (warp == 0) {
     // ---------------- phase B: poll the E logits of this launch (all loads of
     // a round in flight at once), then the top-k, while the other warps
-    // quantize x
+    // quantize x.  (The wait test knob makes this poll wait for the next
+    // generation's tag, which no CTA of this launch publishes, with its own
+    // poll budget.)
+    const int32_t* knob = reinterpret_cast<const int32_t*>(P.status);
+    const uint32_t want = tag + (knob[kWsKnobMode] == kKnobStep1Tag ? 1u : 0u);
+    const uint32_t limit = knob[kWsKnobPolls] ? static_cast<uint32_t>(knob[kWsKnobPolls]) : kSpinLimit;
     constexpr int kPer = kS1MaxE / 32;
     unsigned long long v[kPer];
     uint32_t ready = 0, need = 0;
@@ -205,13 +210,13 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     for (int i = 0; i < kPer; ++i)
       if (lane + 32 * i < E) need |= 1u << i;
     for (uint32_t polls = 0; ready != need; ++polls) {
-      if (polls > kSpinLimit) break;
+      if (polls > limit) break;
 #pragma unroll
       for (int i = 0; i < kPer; ++i)
         if ((need & ~ready) & (1u << i)) v[i] = ld_relaxed_u64(S1.tagged + static_cast<size_t>(lane + 32 * i) * kTagStride);
 #pragma unroll
       for (int i = 0; i < kPer; ++i)
-        if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+        if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == want) ready |= 1u << i;
     }
     if (!__all_sync(0xffffffffu, ready == need)) {
       if (lane == 0) {

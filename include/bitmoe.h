@@ -275,7 +275,8 @@ typedef enum {
   MOE_K_GROUP = 4, MOE_K_GATEUP = 5, MOE_K_DOWN = 6, MOE_K_DEBUG_MATVEC = 7,
   MOE_K_PREFILL_GATEUP = 8, MOE_K_PREFILL_DOWN = 9, MOE_K_ROUTE = 10, MOE_K_COMBINE = 11,
   MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COPY = 14, MOE_K_ROUTER_QUANT = 15,
-  MOE_K_TOPK_GROUP = 16, MOE_K_SHARED = 17, MOE_K_COUNT = 18
+  MOE_K_TOPK_GROUP = 16, MOE_K_SHARED = 17, MOE_K_TC_GATEUP = 18, MOE_K_TC_DOWN = 19,
+  MOE_K_COUNT = 20
 } moe_kernel_id;
 /* Number of kernels this thread has launched through the library so far. */
 int64_t moe_launch_count(void);
@@ -296,6 +297,43 @@ const char* moe_kernel_name(int32_t id);
  * isum[t][r][j] = sum_{k in block j} q[r][k] * xq[t][k].  ntok <= 64.    */
 int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const float* xd,
                      float* out, int32_t* isum, moe_stream_t stream);
+
+/* The exact int32 block sums of the tensor-core paths (pxq_llama README,
+ * "PXQ vs MXFP4": one fixup per 32-value activation block; Parakon Runtime
+ * README, "How it works": int8 x quantized-block products).  Runs the expert
+ * FFN of moe_expert_ffn_decode (prefill == 0: the grouped tensor-core
+ * mat-vecs, any ntok <= 64, ternary layers with hidden and ffn <= 4096) or of
+ * moe_expert_ffn_prefill (prefill != 0: the grouped tensor-core GEMM) with
+ * the same arguments, and also writes, for every (token, slot) pair
+ * p = t * top_k + j, row and 32-value block s, the exact sum(q * a):
+ *   isum_gu [p][2][ffn][hidden/32]   gate (index 0) and up (index 1) rows
+ *                                    against the pair's token's codes xq;
+ *   isum_dn [p][hidden][ffn/32]      down rows against the pair's int8
+ *                                    SwiGLU codes;
+ *   aq      [p][ffn] (may be NULL)   those SwiGLU codes.
+ * Device arrays, 16-byte aligned; entries of pairs whose expert id is out of
+ * range are not written.  A layer the path does not take:
+ * MOE_ERR_UNSUPPORTED_SHAPE.                                                */
+/* Test knob of the bounded device waits (no page has a counterpart: every
+ * device wait of this library is bounded, and this lets a test make one run
+ * out on purpose and read the reported status).  Writes `mode` and `polls` into the
+ * workspace header (synchronizing `stream`); calls on that workspace then:
+ *   mode 0: run normally (a fresh workspace holds 0);
+ *   mode 1: the one-token step polls its router logits for a tag that no CTA
+ *           publishes, gives up after `polls` rounds, records MOE_ERR_TIMEOUT
+ *           and leaves before any weight copy is issued;
+ *   mode 2: the gather warp of the tensor-core mat-vecs withholds its first
+ *           arrival, so the MMA and fixup waits run out after `polls` checks
+ *           (each a suspended wait of at most ~20 us), record
+ *           MOE_ERR_TIMEOUT, drain the copies in flight and free tensor memory.
+ * polls == 0 keeps the kernels' default budgets.  Outputs of a call that
+ * timed out are undefined; the context stays usable.                       */
+int moe_debug_wait_knob(void* ws, size_t ws_bytes, int32_t mode, int32_t polls, moe_stream_t stream);
+
+int moe_debug_ffn_blocksums(const moe_layer* layer, int32_t ntok, const int8_t* xq, const float* xd,
+                            const int32_t* idx, const float* wts, float* y, void* ws, size_t ws_bytes,
+                            int32_t prefill, int32_t* isum_gu, int32_t* isum_dn, int8_t* aq,
+                            moe_stream_t stream);
 
 #ifdef __cplusplus
 }

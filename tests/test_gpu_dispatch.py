@@ -21,7 +21,7 @@ def _names(B, fn):
 
 @pytest.mark.parametrize("fmt,ntok,expect", [
     ("ternary", 1, ["step1"]),
-    ("ternary", 16, ["router_quant", "topk_group", "gateup", "down"]),
+    ("ternary", 16, ["router_quant", "topk_group", "tc_gateup", "tc_down"]),
     ("sign", 1, ["router_quant", "topk_group", "gateup", "down"]),
     ("e16", 3, ["router_quant", "topk_group", "gateup", "down"]),
 ])
@@ -59,7 +59,7 @@ def test_forward_outside_fused_step_and_decode_kernels():
     idx, wts = B.moe_route_topk(x, wr, wl.top_k)
     assert _names(B, lambda: B.moe_expert_ffn_decode(layer, xq[:1].contiguous(), xd[:1].contiguous(),
                                                      idx[:1].contiguous(), wts[:1].contiguous(), ws)) == ["gateup", "down"]
-    assert _names(B, lambda: B.moe_expert_ffn_decode(layer, xq, xd, idx, wts, ws)) == ["group", "gateup", "down"]
+    assert _names(B, lambda: B.moe_expert_ffn_decode(layer, xq, xd, idx, wts, ws)) == ["group", "tc_gateup", "tc_down"]
 
 
 def test_forward_host_kernels():

@@ -59,7 +59,7 @@ def test_e16_matvec_blocksums_and_outputs(orc, rows, k, ntok):
         assert elementwise_rel(out[t], orc.matvec_e16(q, s16, xq[t], xd[t])) <= MATVEC_TOL
 
 
-def _layer_parity(orc, wl, ntok, seed, rows):
+def _layer_parity(orc, wl, ntok, seed, rows, chunk=None):
     B = bm()
     layer, fn = gpu_layer(wl, fmt="e16")
     wr = synthetic.router(wl, 0, "cuda")
@@ -67,12 +67,16 @@ def _layer_parity(orc, wl, ntok, seed, rows):
     ws = B.Workspace.for_layer(layer, ntok)
     y = B.moe_forward(layer, wr, x, ws).cpu().numpy()
     assert B.moe_check_status(ws) == 0
-    xs = x.cpu().numpy()[rows]
-    oidx, owts = orc.route_topk(xs, wr.cpu().numpy(), wl.top_k)
-    olayer, remap = oracle_layer(orc, wl, fn, oidx, fmt="e16")
-    xq, xd = orc.quant_act_q8(xs)
-    ref = orc.expert_ffn(olayer, xq, xd, remap[oidx], owts.astype(np.float32))
-    return y[rows], ref
+    rows = np.asarray(rows)
+    chunk = len(rows) if chunk is None else chunk
+    refs = []
+    for c0 in range(0, len(rows), chunk):  # only a chunk's experts in fp32 at once
+        xs = x.cpu().numpy()[rows[c0:c0 + chunk]]
+        oidx, owts = orc.route_topk(xs, wr.cpu().numpy(), wl.top_k)
+        olayer, remap = oracle_layer(orc, wl, fn, oidx, fmt="e16")
+        xq, xd = orc.quant_act_q8(xs)
+        refs.append(orc.expert_ffn(olayer, xq, xd, remap[oidx], owts.astype(np.float32)))
+    return y[rows], np.concatenate(refs)
 
 
 @pytest.mark.parametrize("ntok", [1, 2, 8])
@@ -83,8 +87,17 @@ def test_e16_layer_tiny(orc, ntok):
 
 @pytest.mark.parametrize("ntok", [1, 16])
 def test_e16_layer_30b(orc, ntok):
-    rows = np.arange(ntok) if ntok <= 4 else np.array([0, 6, 15])
+    rows = np.arange(ntok)  # every token
     y, ref = _layer_parity(orc, synthetic.WORKLOADS["30b"], ntok, 52, rows)
+    assert rel_err_rms(y, ref) <= LAYER_TOL
+
+
+@pytest.mark.parametrize("ntok", [8])
+def test_e16_layer_large(orc, ntok):
+    """The large layer (hidden 4096, ffn 2048, 256 experts, top-8) at 8
+    tokens, the shape the benchmark times: every token, two at a time through
+    the oracle."""
+    y, ref = _layer_parity(orc, synthetic.WORKLOADS["large"], ntok, 54, np.arange(ntok), chunk=2)
     assert rel_err_rms(y, ref) <= LAYER_TOL
 
 

@@ -137,14 +137,21 @@ def _run_forward(B, layer, wr_dev, x_dev, prefill=None):
     return y.cpu().numpy(), ws
 
 
-def _oracle_tokens(orc, wl, fn, wr, x, rows):
-    """Oracle y for the tokens `rows` of x (routing by the oracle router)."""
-    xs = x[rows]
-    oidx, owts = orc.route_topk(xs, wr, wl.top_k)
-    olayer, remap = oracle_layer(orc, wl, fn, oidx)
-    xq, xd = orc.quant_act_q8(xs)
-    y = orc.expert_ffn(olayer, xq, xd, remap[oidx], owts.astype(np.float32))
-    return y, oidx
+def _oracle_tokens(orc, wl, fn, wr, x, rows, chunk=None):
+    """Oracle y for the tokens `rows` of x (routing by the oracle router), in
+    chunks of `chunk` tokens so that only their experts' fp32 weights are held
+    at once."""
+    rows = np.asarray(rows)
+    chunk = len(rows) if chunk is None else chunk
+    ys, ids = [], []
+    for c0 in range(0, len(rows), chunk):
+        xs = x[rows[c0:c0 + chunk]]
+        oidx, owts = orc.route_topk(xs, wr, wl.top_k)
+        olayer, remap = oracle_layer(orc, wl, fn, oidx)
+        xq, xd = orc.quant_act_q8(xs)
+        ys.append(orc.expert_ffn(olayer, xq, xd, remap[oidx], owts.astype(np.float32)))
+        ids.append(oidx)
+    return np.concatenate(ys), np.concatenate(ids)
 
 
 @pytest.mark.parametrize("ntok", [1, 2, 3, 8])
@@ -197,7 +204,7 @@ def test_layer_30b(orc, ntok):
     wr = synthetic.router(wl, 0, "cuda")
     x = synthetic.activations(wl, 1, ntok=ntok, device="cuda")
     y, _ = _run_forward(B, layer, wr, x)
-    rows = np.arange(ntok) if ntok <= 4 else np.array([0, 5, 11, 15])
+    rows = np.arange(ntok)  # every token
     ref, _ = _oracle_tokens(orc, wl, fn, wr.cpu().numpy(), x.cpu().numpy(), rows)
     assert rel_err_rms(y[rows], ref) <= LAYER_TOL
 
@@ -214,7 +221,20 @@ def test_layer_30b_prefill_sampled(orc):
     oidx, _ = orc.route_topk(x.cpu().numpy(), wr.cpu().numpy(), wl.top_k)
     assert np.array_equal(idx.cpu().numpy(), oidx)
     y, _ = _run_forward(B, layer, wr, x)
-    rows = np.array([0, 1, 777, 1500, 2047])
+    # tokens that reach every expert at least twice (so each expert's groups
+    # of the GEMM are sampled), plus the first and last token
+    counts = np.zeros(wl.n_experts, np.int64)
+    rows = [0, 2047]
+    for t in (0, 2047):
+        counts[oidx[t]] += 1
+    for t in range(1, 2047):
+        if np.any(counts[oidx[t]] < 2):
+            rows.append(t)
+            counts[oidx[t]] += 1
+        if counts.min() >= 2:
+            break
+    assert counts.min() >= 2
+    rows = np.array(sorted(rows))
     ref, _ = _oracle_tokens(orc, wl, fn, wr.cpu().numpy(), x.cpu().numpy(), rows)
     assert rel_err_rms(y[rows], ref) <= LAYER_TOL
 
@@ -227,8 +247,8 @@ def test_layer_large_sampled(orc, ntok):
     wr = synthetic.router(wl, 0, "cuda")
     x = synthetic.activations(wl, 2, ntok=ntok, device="cuda")
     y, _ = _run_forward(B, layer, wr, x)
-    rows = np.array([0]) if ntok == 1 else np.array([2, 7])
-    ref, _ = _oracle_tokens(orc, wl, fn, wr.cpu().numpy(), x.cpu().numpy(), rows)
+    rows = np.arange(ntok)  # every token, two at a time through the oracle
+    ref, _ = _oracle_tokens(orc, wl, fn, wr.cpu().numpy(), x.cpu().numpy(), rows, chunk=2)
     assert rel_err_rms(y[rows], ref) <= LAYER_TOL
 
 

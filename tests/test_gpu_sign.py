@@ -67,7 +67,7 @@ def test_sign_matvec_extreme_codes(orc):
     assert np.abs(isum.cpu().numpy()).max() == 32 * 127
 
 
-def _layer_parity(orc, wl, ntok, seed, rows):
+def _layer_parity(orc, wl, ntok, seed, rows, chunk=None):
     B = bm()
     layer, fn = gpu_layer(wl, fmt="sign")
     wr = synthetic.router(wl, 0, "cuda")
@@ -75,12 +75,16 @@ def _layer_parity(orc, wl, ntok, seed, rows):
     ws = B.Workspace.for_layer(layer, ntok)
     y = B.moe_forward(layer, wr, x, ws).cpu().numpy()
     assert B.moe_check_status(ws) == 0
-    xs = x.cpu().numpy()[rows]
-    oidx, owts = orc.route_topk(xs, wr.cpu().numpy(), wl.top_k)
-    olayer, remap = oracle_layer(orc, wl, fn, oidx, fmt="sign")
-    xq, xd = orc.quant_act_q8(xs)
-    ref = orc.expert_ffn(olayer, xq, xd, remap[oidx], owts.astype(np.float32))
-    return y[rows], ref
+    rows = np.asarray(rows)
+    chunk = len(rows) if chunk is None else chunk
+    refs = []
+    for c0 in range(0, len(rows), chunk):  # only a chunk's experts in fp32 at once
+        xs = x.cpu().numpy()[rows[c0:c0 + chunk]]
+        oidx, owts = orc.route_topk(xs, wr.cpu().numpy(), wl.top_k)
+        olayer, remap = oracle_layer(orc, wl, fn, oidx, fmt="sign")
+        xq, xd = orc.quant_act_q8(xs)
+        refs.append(orc.expert_ffn(olayer, xq, xd, remap[oidx], owts.astype(np.float32)))
+    return y[rows], np.concatenate(refs)
 
 
 @pytest.mark.parametrize("ntok", [1, 2, 8])
@@ -91,8 +95,17 @@ def test_sign_layer_tiny(orc, ntok):
 
 @pytest.mark.parametrize("ntok", [1, 16])
 def test_sign_layer_30b(orc, ntok):
-    rows = np.arange(ntok) if ntok <= 4 else np.array([0, 6, 15])
+    rows = np.arange(ntok)  # every token
     y, ref = _layer_parity(orc, synthetic.WORKLOADS["30b"], ntok, 32, rows)
+    assert rel_err_rms(y, ref) <= LAYER_TOL
+
+
+@pytest.mark.parametrize("ntok", [8])
+def test_sign_layer_large(orc, ntok):
+    """The large layer (hidden 4096, ffn 2048, 256 experts, top-8) at 8
+    tokens, the shape the benchmark times: every token, two at a time through
+    the oracle."""
+    y, ref = _layer_parity(orc, synthetic.WORKLOADS["large"], ntok, 34, np.arange(ntok), chunk=2)
     assert rel_err_rms(y, ref) <= LAYER_TOL
 
 
