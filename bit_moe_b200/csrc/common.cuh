@@ -104,6 +104,14 @@ __device__ __forceinline__ float f16_bits_to_f32(uint16_t h) {
   return __half2float(__ushort_as_half(h));
 }
 
+// The base-3 decode multiplies two registers of 16-bit lanes by 3 per digit
+// level.  Left to itself the compiler turns both into shift-adds on the ALU
+// pipe, which also carries the byte permutes; taking one factor from constant
+// memory (a value the compiler cannot fold) keeps that multiply an integer
+// multiply-add on the FMA pipe, and the two pipes share the decode.
+static __constant__ uint32_t g_three = 3u;
+__device__ __forceinline__ uint32_t mul3_fma(uint32_t x) { return x * g_three; }
+
 // Streaming 32-bit load that does not allocate in L1 (weights are read once).
 __device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t* p) {
   uint32_t v;

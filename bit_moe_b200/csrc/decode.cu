@@ -423,8 +423,10 @@ static void launch_ffn_fmt(const DecodeParams& P, cudaStream_t stream) {
 
 int launch_ffn(const DecodeParams& P, cudaStream_t stream) {
   if (!P.direct && P.group_chunk != kChunk) return fail(MOE_ERR_INVALID_ARG, "expert_ffn: items of %d pairs", P.group_chunk);
-  // ternary layers of batches: the tensor-core mat-vecs
-  if (!P.direct && tc_ffn_supported(P)) return launch_ffn_tc(P, stream);
+  // ternary layers of batches whose items hold many pairs: the tensor-core
+  // mat-vecs (a tcgen05.mma of N <= 64 costs the same as one of N = 16, so
+  // they pay only when the items are large)
+  if (!P.direct && tc_ffn_supported(P) && tc_ffn_preferred(P)) return launch_ffn_tc(P, stream);
   init_kernel_attrs();
   if (P.format == MOE_FORMAT_SIGN) launch_ffn_fmt<MOE_FORMAT_SIGN>(P, stream);
   else if (P.format == MOE_FORMAT_E16) launch_ffn_fmt<MOE_FORMAT_E16>(P, stream);

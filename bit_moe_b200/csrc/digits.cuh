@@ -19,25 +19,32 @@ namespace bitmoe {
 
 // Digit words [32*kHalf, 32*kHalf + 32) of one block from packed words
 // w[jj] = word 6*kHalf + jj, jj in [0, 7) (word 6 feeds both halves).
-// `three` must hold 3: a value the compiler cannot see, so that one of the two
-// lane multiplies of a level stays an integer multiply-add (FMA pipe) while
-// the other may become a shift-add (ALU pipe), and the two pipes share the
-// decode evenly.
+// One of the two lane multiplies of a level runs on the FMA pipe (mul3_fma).
 template <int kHalf>
-__device__ __forceinline__ void digit_half(const uint32_t (&w)[7], uint32_t (&dg)[32], uint32_t three = 3u) {
+__device__ __forceinline__ void digit_half(const uint32_t (&w)[7], uint32_t (&dg)[32]) {
+  // level-major: the 7 words' chains advance side by side (7 independent
+  // multiply chains per level), so one warp keeps its pipes busy
+  uint32_t lo[7], hi[7], hp[7];
 #pragma unroll
   for (int jj = 0; jj < 7; ++jj) {
-    const int j = 6 * kHalf + jj;
-    uint32_t lo = w[jj] & 0x00FF00FFu, hi = __byte_perm(w[jj], 0u, 0x4341), hp = 0u;
+    lo[jj] = w[jj] & 0x00FF00FFu;
+    hi[jj] = __byte_perm(w[jj], 0u, 0x4341);
+    hp[jj] = 0u;
+  }
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-      if (j == kBlockWords - 1 && i == 4) break;
-      lo *= 3u;
-      hi *= three;
-      const uint32_t hn = __byte_perm(lo, hi, 0x7351);
+  for (int i = 0; i < 5; ++i) {
+#pragma unroll
+    for (int jj = 0; jj < 7; ++jj) {
+      const int j = 6 * kHalf + jj;
       const int c = 5 * j + i - 32 * kHalf;
-      if (c >= 0 && c < 32) dg[c] = hn - 3u * hp;
-      hp = hn;
+      if (j == kBlockWords - 1 && i == 4) continue;  // the last word's pad digit
+      // levels past the half's last digit word are not needed
+      if (c >= 32) continue;
+      lo[jj] *= 3u;
+      hi[jj] = mul3_fma(hi[jj]);
+      const uint32_t hn = __byte_perm(lo[jj], hi[jj], 0x7351);
+      if (c >= 0) dg[c] = hn - 3u * hp[jj];
+      hp[jj] = hn;
     }
   }
 }

@@ -5,20 +5,22 @@
 // a grouped-MoE GEMM, and "Updates -- 2026-07-19": an int8 prefill tile.
 //
 // The (token, slot) pairs are grouped by expert and cut into groups of up to
-// kPN = 128 pairs.  A tile of the grouped GEMM is 128 weight rows x one group,
-// one tcgen05.mma kind::i8 (M = 128, N = 128, K = 32) per 32-value sub-block:
+// kPN = 64 pairs.  A tile of the grouped GEMM is 128 weight rows x one group,
+// one tcgen05.mma kind::i8 (M = 128, N = 64, K = 32) per 32-value sub-block:
 //   - A (tensor memory): the weights' base-3 digits t = q + 1 in {0, 1, 2} as
 //     u8, decoded in registers from the packed blocks (digits.cuh) and written
 //     straight into tensor memory -- the expanded weights exist nowhere else;
 //   - B (shared memory): the group's int8 activation codes as s8;
-//   - D (tensor memory): int32, exact.  Each accumulator stage starts at the
-//     integer 0x4B400000, so that after the MMA its bits read as the fp32
-//     value 12582912 + sum(t * a), exactly (|sum| < 2^13); one fp32
-//     subtraction of m = 12582912 + sum(a) then gives sum(q * a) exactly, and
-//     the fixup scales it as every decode kernel does: per block
+//   - D (tensor memory): int32, exact (|sum(t * a)| < 2^13).  The fixup adds
+//     the integer 0x4B400000 to each sum, so that its bits read as the fp32
+//     value 12582912 + sum(t * a) exactly; one fp32 subtraction of
+//     m = 12582912 + sum(a) then gives sum(q * a) exactly, and the fixup
+//     scales it as every decode kernel does: per block
 //     inner = sum_s fma(d_s, sum_s(q * a), inner), per row and pair
-//     y = fma(s_b, inner, y) over the blocks in order (y kept in tensor
-//     memory between blocks).
+//     y = fma(s_b, inner, y) over the blocks in order.
+// 64-pair groups keep a fixup warp's 16 pairs (inner, y and one sub-block's
+// sums) in registers; a tcgen05.mma of N = 64 costs the issue of one of N = 16
+// on B200, so the grouped GEMM is bound by the fixup, not the tensor cores.
 // The activations of a tile are laid out once per (group, 256-block) in HBM
 // exactly as shared memory holds them (codes in the MMA's core-matrix layout,
 // then the scales and m of the group's pairs): for gate/up by a gather pass
@@ -43,12 +45,12 @@
 
 namespace bitmoe {
 
-constexpr int kPN = 128;          // pairs per group (MMA N)
+constexpr int kPN = 64;           // pairs per group (MMA N)
 constexpr int kPM = 128;          // weight rows per tile (MMA M)
 // Warp roles of a CTA (one CTA per SM, persistent over the tiles):
 constexpr int kWDec = 0;          // warps 0-3: decode the digits into TMEM (thread = row)
 constexpr int kWFix = 4;          // warps 4-19: accumulator fixup and epilogue (thread = row,
-constexpr int kFixWarps = 16;     //   warp 4 + 4f + q: rows of quadrant q, pairs [32f, 32f + 32))
+constexpr int kFixWarps = 16;     //   warp 4 + 4f + q: rows of quadrant q, pairs [16f, 16f + 16))
 constexpr int kFixPairs = kPN / (kFixWarps / 4);
 constexpr int kWCopyW = 20;       // warp 20: lane 0 brings the weight blocks in (bulk copies)
 constexpr int kWCopyB = 21;       // warp 21: lane 0 brings the activation blocks in (bulk copies)
@@ -56,13 +58,14 @@ constexpr int kWMma = 22;         // warp 22: lane 0 issues the MMAs
 constexpr int kPThreads = 23 * 32;
 constexpr int kWStages = 8;       // weight ring: one block of the tile's 4 panels per stage
 constexpr int kAStages = 2;       // digit stages in TMEM, 64 columns each
-constexpr int kBStages = 3;       // activation stages in shared memory
-constexpr int kDStages = 2;       // accumulator stages in TMEM: one sub-block (kPN columns) each
+constexpr int kBStages = 4;       // activation stages in shared memory
+constexpr int kDSub = 2;          // sub-blocks per accumulator stage
+constexpr int kDStages = 3;       // accumulator stages in TMEM, kDSub * kPN columns each
 constexpr int kTmemCols = 512;
 constexpr int kAcol = 0;          // A stage a: columns [64a, 64a + 64)
-constexpr int kDcol = 128;        // D stage d: columns [128 + kPN*d, 128 + kPN*(d+1))
-constexpr int kYcol = kDcol + kDStages * kPN;  // y of every (row, pair) between blocks
-static_assert(kYcol + kPN <= kTmemCols, "tensor memory columns");
+constexpr int kDcol = 128;        // D stage d: columns [128 + kDSub*kPN*d, 128 + kDSub*kPN*(d+1))
+static_assert(kDcol + kDStages * kDSub * kPN <= kTmemCols, "tensor memory columns");
+static_assert(kSubPerBlock % kDSub == 0, "whole sub-blocks per stage");
 constexpr int kPanelBytes = kBlockWords * kPanel * 4;
 constexpr uint32_t kMagic = 0x4B400000u;  // bits of 12582912.0f
 constexpr float kMagicF = 12582912.0f;
@@ -150,17 +153,6 @@ __device__ __forceinline__ void sub2(float& r0, float& r1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// Store the same 32-bit value into 32 consecutive columns of this thread's
-// TMEM lane.
-__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
-      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
-      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-
 // Tile t of the grouped GEMM: item (expert, pairs) and 128-row tile index.
 struct TileInfo {
   Item it;
@@ -194,6 +186,7 @@ __device__ __forceinline__ const uint16_t* panel_scales(const DecodeParams& P, i
 // tile: each lane (32 consecutive f, one 32-block) requantizes the SwiGLU
 // values a[] (absent pairs and bad groups: zeros) and writes the codes, scale
 // and m into the down input's activation block of the group.
+template <bool kDbg>
 __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, int item, int r, int n0,
                                                  const float* a, const Item& it, int lane) {
   const int F = P.ffn;
@@ -216,7 +209,7 @@ __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, 
       dst->d[sub][np] = dd;
       dst->m[sub][np] = kMagicF + static_cast<float>(sum);
     }
-    if (P.dbg_isum_gu != nullptr && np < it.count)  // test hook: the SwiGLU codes
+    if (kDbg && np < it.count)  // test hook: the SwiGLU codes
       P.aq[static_cast<size_t>(P.pairs[it.start + np]) * F + f] = static_cast<int8_t>(qq);
   }
 }
@@ -229,7 +222,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Pr
   return false;
 }
 
-template <bool kGU>
+// kDbg: the test hook's instantiation, which also writes the exact block sums.
+template <bool kGU, bool kDbg>
 __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   pdl_enter();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -260,17 +254,6 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
-  if (warp >= kWFix && warp < kWFix + kFixWarps) {
-    // every accumulator stage starts at the magic integer before the first MMA
-    const int q = (warp - kWFix) & 3, f = (warp - kWFix) >> 2;
-    const uint32_t tl = tbase + (static_cast<uint32_t>(q * 32) << 16);
-    for (int ds = 0; ds < kDStages; ++ds) tmem_fill32(tl + kDcol + kPN * ds + kFixPairs * f, kMagic);
-    tc_wait_st();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
   if (warp >= kWDec && warp < kWFix) {
     // ------------------------------------------------ decode: digits -> TMEM
     const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);
@@ -315,7 +298,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       if (T.it.expert < 0) {  // ids out of range: their outputs are zero
         if (warp == kWFix && lane == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
         if (kGU) {
-          if (q >= 2) write_down_codes(P, T.mt, T.item, 32 * (q - 2) + lane, n0, nullptr, T.it, lane);
+          if (q >= 2) write_down_codes<kDbg>(P, T.mt, T.item, 32 * (q - 2) + lane, n0, nullptr, T.it, lane);
         } else {
           for (int n = n0; n < n0 + kFixPairs && n < T.it.count; ++n)
             P.ye[static_cast<size_t>(P.pairs[T.it.start + n]) * H + kPM * T.mt + 32 * q + lane] = 0.f;
@@ -323,7 +306,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         continue;
       }
       bool ok = true;
-      float inner[kFixPairs];  // per block the scaled sub-block sums, at the end y
+      float y[kFixPairs];
+#pragma unroll
+      for (int n = 0; n < kFixPairs; ++n) y[n] = 0.f;
       for (int b = 0; b < nb && ok; ++b, ++bi) {
         // the row's block scale from the weight stage of this block
         const int ws = bi % kWStages;
@@ -333,36 +318,34 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         if (lane == 0) mbar_arrive(&S.w_empty[ws]);
         const int bs = bi % kBStages;
         if (!wait_or_abort(&S.b_full[bs], (bi / kBStages) & 1u, S, P.status)) { ok = false; break; }
+        float inner[kFixPairs];
 #pragma unroll
         for (int n = 0; n < kFixPairs; ++n) inner[n] = 0.f;
 #pragma unroll 1
-        for (int s = 0; s < kSubPerBlock; ++s, ++si) {
+        for (int h = 0; h < kSubPerBlock / kDSub; ++h, ++si) {
           const int ds = si % kDStages;
           if (!wait_or_abort(&S.d_full[ds], (si / kDStages) & 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t col = tlane + kDcol + kPN * ds + n0;
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t v[16];
-            tmem_ld16(col + 16 * hf, v);
+          for (int s2 = 0; s2 < kDSub; ++s2) {
+            const int s = kDSub * h + s2;
+            uint32_t v[kFixPairs];
+            tmem_ld16(tlane + kDcol + kDSub * kPN * ds + kPN * s2 + n0, v);
             tc_wait_ld();
-            if (hf == 1) {
-              // the stage goes back to the MMA at the magic integer
-              tmem_fill32(col, kMagic);
-              tc_wait_st();
+            if (s2 == kDSub - 1) {  // the stage goes back to the MMA
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(&S.d_empty[ds]);
             }
-            const float* dp = &S.st[bs].d[s][n0 + 16 * hf];
-            const float* mp = &S.st[bs].m[s][n0 + 16 * hf];
-            if ((kGU ? P.dbg_isum_gu : P.dbg_isum_dn) != nullptr) {  // test hook: the exact block sums
+            const float* dp = &S.st[bs].d[s][n0];
+            const float* mp = &S.st[bs].m[s][n0];
+            if (kDbg) {  // test hook: the exact block sums
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int np = n0 + 16 * hf + e;
+              for (int e = 0; e < kFixPairs; ++e) {
+                const int np = n0 + e;
                 if (np >= T.it.count) continue;
                 const int pair = P.pairs[T.it.start + np];
-                const int isum = static_cast<int>(__fsub_rn(__uint_as_float(v[e]), mp[e]));
+                const int isum = static_cast<int>(__fsub_rn(__uint_as_float(v[e] + kMagic), mp[e]));
                 const int sg = b * kSubPerBlock + s;
                 if (kGU) {
                   const int fr = 64 * T.mt + 32 * (q & 1) + lane;
@@ -374,14 +357,15 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
               }
             }
 #pragma unroll
-            for (int n4 = 0; n4 < 4; ++n4) {
+            for (int n4 = 0; n4 < kFixPairs / 4; ++n4) {
               const float4 dd = reinterpret_cast<const float4*>(dp)[n4];
               const float4 mm = reinterpret_cast<const float4*>(mp)[n4];
-              const int nn = 16 * hf + 4 * n4;
-              // D - m = sum(q*a), exact; then d * sum(q*a) as in the decode kernels
+              const int nn = 4 * n4;
+              // (D + 0x4B400000) as fp32 minus m = sum(q*a), exact; then
+              // d * sum(q*a) as in the decode kernels
               float i0, i1, i2, i3;
-              sub2(i0, i1, __uint_as_float(v[4 * n4]), __uint_as_float(v[4 * n4 + 1]), mm.x, mm.y);
-              sub2(i2, i3, __uint_as_float(v[4 * n4 + 2]), __uint_as_float(v[4 * n4 + 3]), mm.z, mm.w);
+              sub2(i0, i1, __uint_as_float(v[nn] + kMagic), __uint_as_float(v[nn + 1] + kMagic), mm.x, mm.y);
+              sub2(i2, i3, __uint_as_float(v[nn + 2] + kMagic), __uint_as_float(v[nn + 3] + kMagic), mm.z, mm.w);
               fma2(inner[nn], inner[nn + 1], dd.x, dd.y, i0, i1, inner[nn], inner[nn + 1]);
               fma2(inner[nn + 2], inner[nn + 3], dd.z, dd.w, i2, i3, inner[nn + 2], inner[nn + 3]);
             }
@@ -390,48 +374,30 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         if (!ok) break;
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.b_empty[bs]);
-        // y = fma(sw, inner, y) over the blocks in order, y kept in TMEM
-        // between blocks (inner holds y from here on)
-        if (b == 0) {
+        // y = fma(sw, inner, y) over the blocks in order
 #pragma unroll
-          for (int n = 0; n < kFixPairs; ++n) inner[n] = __fmaf_rn(sw, inner[n], 0.f);
-        } else {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t v[16];
-            tmem_ld16(tlane + kYcol + n0 + 16 * hf, v);
-            tc_wait_ld();
-#pragma unroll
-            for (int n = 0; n < 16; ++n) inner[16 * hf + n] = __fmaf_rn(sw, inner[16 * hf + n], __uint_as_float(v[n]));
-          }
-        }
-        if (b + 1 < nb) {
-          uint32_t yb[kFixPairs];
-#pragma unroll
-          for (int n = 0; n < kFixPairs; ++n) yb[n] = __float_as_uint(inner[n]);
-          tmem_st32(tlane + kYcol + n0, yb);
-          tc_wait_st();
-        }
+        for (int n = 0; n < kFixPairs; ++n) y[n] = __fmaf_rn(sw, inner[n], y[n]);
       }
       if (!ok) break;
       // ---- epilogue (rows 32*q + lane, pairs [n0, n0 + kFixPairs))
       if (kGU) {
         if (q < 2) {
 #pragma unroll
-          for (int n = 0; n < kFixPairs; ++n) S.xch[32 * q + lane][n0 + n] = inner[n];
+          for (int n = 0; n < kFixPairs; ++n) S.xch[32 * q + lane][n0 + n] = y[n];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.fx_bar[0]);
         if (!wait_or_abort(&S.fx_bar[0], ep & 1u, S, P.status)) break;
         if (q >= 2) {
           const int r = 32 * (q - 2) + lane;  // f offset within the tile
-          float a[kFixPairs];
+          // the SwiGLU value replaces g in the exchange row (each entry is
+          // read and written by its own thread)
 #pragma unroll
           for (int n = 0; n < kFixPairs; ++n) {
             const float g = S.xch[r][n0 + n];
-            a[n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), inner[n]);
+            S.xch[r][n0 + n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
           }
-          write_down_codes(P, T.mt, T.item, r, n0, a, T.it, lane);
+          write_down_codes<kDbg>(P, T.mt, T.item, r, n0, &S.xch[r][n0], T.it, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.fx_bar[1]);
@@ -439,8 +405,9 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         ++ep;
       } else {
         const int hrow = kPM * T.mt + 32 * q + lane;
-        for (int n = 0; n < kFixPairs && n0 + n < T.it.count; ++n)
-          P.ye[static_cast<size_t>(P.pairs[T.it.start + n0 + n]) * H + hrow] = inner[n];
+#pragma unroll
+        for (int n = 0; n < kFixPairs; ++n)
+          if (n0 + n < T.it.count) P.ye[static_cast<size_t>(P.pairs[T.it.start + n0 + n]) * H + hrow] = y[n];
       }
     }
   } else if (warp == kWCopyW && lane == 0) {
@@ -507,13 +474,16 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         }
         tc_fence_after();
         const uint64_t bdesc = smem_desc(smem_u32(S.st[bs].codes), 128, 256);
-        for (int s = 0; s < kSubPerBlock; ++s, ++si) {
+        for (int h = 0; h < kSubPerBlock / kDSub; ++h, ++si) {
           const int ds = si % kDStages;
           if (!wait_or_abort(&S.d_empty[ds], ((si / kDStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
-          // the stage holds the magic integer: accumulate onto it
-          mma_i8_ts(tbase + kDcol + kPN * ds, tbase + kAcol + 64 * a + 8 * s,
-                    bdesc + static_cast<uint64_t>((s * kPN * 32) >> 4), idesc, true);
+#pragma unroll
+          for (int s2 = 0; s2 < kDSub; ++s2) {
+            const int s = kDSub * h + s2;
+            mma_i8_ts(tbase + kDcol + kDSub * kPN * ds + kPN * s2, tbase + kAcol + 64 * a + 8 * s,
+                      bdesc + static_cast<uint64_t>((s * kPN * 32) >> 4), idesc, false);
+          }
           mma_commit(&S.d_full[ds]);
         }
         if (!ok) break;
@@ -575,8 +545,10 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attrs_done[dev].load(std::memory_order_relaxed)) {
-    cudaFuncSetAttribute(k_prefill_mma<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_prefill_mma<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     attrs_done[dev].store(true, std::memory_order_relaxed);
   }
   int n_sm = 148;
@@ -584,9 +556,11 @@ int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   const size_t smem = prefill_smem();
   launch_k(k_prefill_gather, dim3(4 * n_sm), dim3(kPN * kSubPerBlock), 0, stream, P);
   note_launch(MOE_K_PREFILL_GATHER, stream);
-  launch_k(k_prefill_mma<true>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
+  const bool dbg = P.dbg_isum_gu != nullptr;
+  launch_k(dbg ? k_prefill_mma<true, true> : k_prefill_mma<true, false>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
   note_launch(MOE_K_PREFILL_GATEUP, stream);
-  launch_k(k_prefill_mma<false>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
+  launch_k(dbg ? k_prefill_mma<false, true> : k_prefill_mma<false, false>, dim3(n_sm), dim3(kPThreads), smem, stream,
+           P);
   note_launch(MOE_K_PREFILL_DOWN, stream);
   launch_k(k_combine, dim3(4 * n_sm), dim3(256), 0, stream, P);
   note_launch(MOE_K_COMBINE, stream);

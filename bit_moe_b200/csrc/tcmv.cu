@@ -211,7 +211,7 @@ __device__ __forceinline__ void tc_gather(const DecodeParams& P, TcSmem& S, int 
 // pairs (D columns n0 .. n0 + NC of each sub-block), the stage handed back
 // to the MMA, then per pair inner = sum_s fma(d_s, sum_s(t*a) - sum_s(a), inner)
 // and chain w = fma(s_b, inner, chain w).
-template <int NC, int kChains, bool kGU = (kChains == 8)>
+template <int NC, int kChains, bool kDbg, bool kGU = (kChains == 8)>
 __device__ __forceinline__ void fix_block(const DecodeParams& P, TcSmem& S, uint32_t dcol, int buf, int i, int n0,
                                           int nc, int w, float sw, float (&acc)[kChains][kTFixPairs],
                                           const TcUnit& U, int b, int q, int lane, uint64_t* d_empty) {
@@ -236,7 +236,7 @@ __device__ __forceinline__ void fix_block(const DecodeParams& P, TcSmem& S, uint
     for (int n = 0; n < NC; ++n) {
       const int isum = static_cast<int>(v[s][n]) - S.sa[buf][i][s][n0 + n];
       inner[n] = __fmaf_rn(S.dsc[buf][i][s][n0 + n], static_cast<float>(isum), inner[n]);
-      if (dbg != nullptr && n < nc) {  // test hook: the exact block sums
+      if (kDbg && n < nc) {  // test hook: the exact block sums
         const int pair = item_pair(P, U.it, n0 + n);
         const int sg = b * kSubPerBlock + s;
         if (kGU) {
@@ -257,8 +257,9 @@ __device__ __forceinline__ void fix_block(const DecodeParams& P, TcSmem& S, uint
     }
 }
 
-template <bool kGU>
-__global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n, uint32_t three) {
+// kDbg: the test hook's instantiation, which also writes the exact block sums.
+template <bool kGU, bool kDbg>
+__global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n) {
   pdl_enter();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   TcSmem& S = *reinterpret_cast<TcSmem*>(smem_raw);
@@ -312,8 +313,8 @@ __global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n,
         const int as = ai % kTAStages;
         if (!tc_wait(&S.a_empty[as], ((ai / kTAStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
         uint32_t dg[32];
-        if (hh == 0) digit_half<0>(w7, dg, three);
-        else digit_half<1>(w7, dg, three);
+        if (hh == 0) digit_half<0>(w7, dg);
+        else digit_half<1>(w7, dg);
         tmem_st32(tl + kTAcol + 64 * as + 32 * hh, dg);
         tc_wait_st();
         tc_fence_before();
@@ -374,9 +375,9 @@ __global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n,
         // only this warp's pairs of the item (a warp with none just passes the stage on)
         const uint32_t dcol = tl + kTDcol + kTDStageCols * ds + n0;
         const int w = kGU ? (b & 7) : 0;
-        if (nc >= 3) fix_block<4, kChains>(P, S, dcol, buf, i, n0, nc, w, sw, acc, U, b, q, lane, &S.d_empty[ds]);
-        else if (nc == 2) fix_block<2, kChains>(P, S, dcol, buf, i, n0, nc, w, sw, acc, U, b, q, lane, &S.d_empty[ds]);
-        else if (nc == 1) fix_block<1, kChains>(P, S, dcol, buf, i, n0, nc, w, sw, acc, U, b, q, lane, &S.d_empty[ds]);
+        if (nc >= 3) fix_block<4, kChains, kDbg>(P, S, dcol, buf, i, n0, nc, w, sw, acc, U, b, q, lane, &S.d_empty[ds]);
+        else if (nc == 2) fix_block<2, kChains, kDbg>(P, S, dcol, buf, i, n0, nc, w, sw, acc, U, b, q, lane, &S.d_empty[ds]);
+        else if (nc == 1) fix_block<1, kChains, kDbg>(P, S, dcol, buf, i, n0, nc, w, sw, acc, U, b, q, lane, &S.d_empty[ds]);
         else {
           tc_fence_before();
           __syncwarp();
@@ -537,22 +538,32 @@ bool tc_ffn_supported(const DecodeParams& P) {
          P.hidden % kTM == 0 && P.ffn % 64 == 0;
 }
 
+bool tc_ffn_preferred(const DecodeParams& P) {
+  // measured on B200: with 1-2 pairs per expert (the 8- and 16-token decode
+  // batches) the CUDA-core grouped kernels are faster; the tensor-core path
+  // is kept for the test hook until its decode warps keep the MMA fed
+  (void)P;
+  return false;
+}
+
 int launch_ffn_tc(const DecodeParams& P, cudaStream_t stream) {
   static std::atomic<bool> attrs_done[64];  // the attribute calls are idempotent
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attrs_done[dev].load(std::memory_order_relaxed)) {
-    cudaFuncSetAttribute(k_tcmv<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_tcmv<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_tcmv<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_tcmv<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_tcmv<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_tcmv<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     attrs_done[dev].store(true, std::memory_order_relaxed);
   }
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
   const size_t smem = tc_smem();
-  // the decode's multiplier 3 is passed as an argument (see digit_half)
-  launch_k(k_tcmv<true>, dim3(n_sm), dim3(kTThreads), smem, stream, P, 1, 3u);
+  const bool dbg = P.dbg_isum_gu != nullptr;
+  launch_k(dbg ? k_tcmv<true, true> : k_tcmv<true, false>, dim3(n_sm), dim3(kTThreads), smem, stream, P, 1);
   note_launch(MOE_K_TC_GATEUP, stream);
-  launch_k(k_tcmv<false>, dim3(n_sm), dim3(kTThreads), smem, stream, P, 1, 3u);
+  launch_k(dbg ? k_tcmv<false, true> : k_tcmv<false, false>, dim3(n_sm), dim3(kTThreads), smem, stream, P, 1);
   note_launch(MOE_K_TC_DOWN, stream);
   return check_launch("expert_ffn (tensor cores)");
 }

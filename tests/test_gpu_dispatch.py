@@ -21,7 +21,7 @@ def _names(B, fn):
 
 @pytest.mark.parametrize("fmt,ntok,expect", [
     ("ternary", 1, ["step1"]),
-    ("ternary", 16, ["router_quant", "topk_group", "tc_gateup", "tc_down"]),
+    ("ternary", 16, ["router_quant", "topk_group", "gateup", "down"]),
     ("sign", 1, ["router_quant", "topk_group", "gateup", "down"]),
     ("e16", 3, ["router_quant", "topk_group", "gateup", "down"]),
 ])
@@ -59,7 +59,24 @@ def test_forward_outside_fused_step_and_decode_kernels():
     idx, wts = B.moe_route_topk(x, wr, wl.top_k)
     assert _names(B, lambda: B.moe_expert_ffn_decode(layer, xq[:1].contiguous(), xd[:1].contiguous(),
                                                      idx[:1].contiguous(), wts[:1].contiguous(), ws)) == ["gateup", "down"]
-    assert _names(B, lambda: B.moe_expert_ffn_decode(layer, xq, xd, idx, wts, ws)) == ["group", "tc_gateup", "tc_down"]
+    assert _names(B, lambda: B.moe_expert_ffn_decode(layer, xq, xd, idx, wts, ws)) == ["group", "gateup", "down"]
+
+
+def test_blocksum_hook_kernels():
+    """The block-sum test hook runs the tensor-core kernels (decode: grouping
+    then the two mat-vecs; prefill: the grouped GEMM chain)."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"]
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    for ntok, prefill, expect in ((3, False, ["group", "tc_gateup", "tc_down"]),
+                                  (70, True, ["group", "prefill_gather", "prefill_gateup", "prefill_down",
+                                              "combine"])):
+        x = synthetic.activations(wl, 86, ntok=ntok, device="cuda")
+        xq, xd = B.moe_quant_act_q8(x)
+        idx, wts = B.moe_route_topk(x, wr, wl.top_k)
+        ws = B.Workspace.for_layer(layer, ntok, prefill=prefill)
+        assert _names(B, lambda: B.moe_debug_ffn_blocksums(layer, xq, xd, idx, wts, ws, prefill=prefill)) == expect
 
 
 def test_forward_host_kernels():

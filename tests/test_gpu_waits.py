@@ -26,29 +26,54 @@ def _names(B, fn):
     return [B.lib().moe_kernel_name(i).decode() for i in tr.ids]
 
 
-@pytest.mark.parametrize("name,ntok,mode,polls,kernels", [
-    ("30b", 1, 1, 2000, ["step1"]),                                        # tagged logit poll
-    ("30b-b16", 16, 2, 50, ["router_quant", "topk_group", "tc_gateup", "tc_down"]),  # mbarrier waits
-])
-def test_wait_runs_out_and_context_recovers(name, ntok, mode, polls, kernels):
+def test_step1_logit_poll_runs_out_and_context_recovers():
+    """The one-token step polls for a logit tag that no CTA publishes."""
     B = bm()
-    wl = synthetic.WORKLOADS[name]
+    wl = synthetic.WORKLOADS["30b"]
     layer, _ = gpu_layer(wl)
     wr = synthetic.router(wl, 0, "cuda")
-    x = synthetic.activations(wl, 90, ntok=ntok, device="cuda")
-    fresh = B.Workspace.for_layer(layer, ntok)
+    x = synthetic.activations(wl, 90, ntok=1, device="cuda")
+    fresh = B.Workspace.for_layer(layer, 1)
     y_ref = B.moe_forward(layer, wr, x, fresh).cpu().numpy()
     assert B.moe_check_status(fresh) == 0
 
-    ws = B.Workspace.for_layer(layer, ntok)
-    B.moe_debug_wait_knob(ws, mode, polls)
-    assert _names(B, lambda: B.moe_forward(layer, wr, x, ws)) == kernels
+    ws = B.Workspace.for_layer(layer, 1)
+    B.moe_debug_wait_knob(ws, 1, 2000)
+    assert _names(B, lambda: B.moe_forward(layer, wr, x, ws)) == ["step1"]
     assert B.moe_check_status(ws) == MOE_ERR_TIMEOUT
     assert B.moe_check_status(ws) == 0  # read and cleared
 
     B.moe_debug_wait_knob(ws, 0, 0)
     for _ in range(2):
         y = B.moe_forward(layer, wr, x, ws).cpu().numpy()
+        assert B.moe_check_status(ws) == 0
+        assert np.array_equal(y, y_ref)
+
+
+def test_tc_mbarrier_waits_run_out_and_context_recovers():
+    """The tensor-core mat-vecs' gather warp withholds its first arrival: the
+    MMA and fixup warps' mbarrier waits run out, the kernels drain their
+    copies, free tensor memory and report MOE_ERR_TIMEOUT."""
+    B = bm()
+    wl = synthetic.WORKLOADS["30b-b16"]
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 91, ntok=16, device="cuda")
+    xq, xd = B.moe_quant_act_q8(x)
+    idx, wts = B.moe_route_topk(x, wr, wl.top_k)
+    fresh = B.Workspace.for_layer(layer, 16, prefill=False)
+    y_ref = B.moe_debug_ffn_blocksums(layer, xq, xd, idx, wts, fresh)[0].cpu().numpy()
+    assert B.moe_check_status(fresh) == 0
+
+    ws = B.Workspace.for_layer(layer, 16, prefill=False)
+    B.moe_debug_wait_knob(ws, 2, 50)
+    names = _names(B, lambda: B.moe_debug_ffn_blocksums(layer, xq, xd, idx, wts, ws))
+    assert names == ["group", "tc_gateup", "tc_down"]
+    assert B.moe_check_status(ws) == MOE_ERR_TIMEOUT
+
+    B.moe_debug_wait_knob(ws, 0, 0)
+    for _ in range(2):
+        y = B.moe_debug_ffn_blocksums(layer, xq, xd, idx, wts, ws)[0].cpu().numpy()
         assert B.moe_check_status(ws) == 0
         assert np.array_equal(y, y_ref)
 
