@@ -110,6 +110,12 @@ def kernel_bytes(wl, unique_experts):
     }
     # the tensor-core mat-vecs move the same bytes as the CUDA-core ones
     kb["tc_gateup"], kb["tc_down"] = kb["gateup"], kb["down"]
+    if wl.shared_ffn:
+        # the shared expert's three kernels (gate/up, requantization, down with
+        # the add into y), per launch on average: 8-bit codes plus an fp16 scale
+        # per 32 weights, activations in and out
+        Fs = wl.shared_ffn
+        kb["shared"] = (3 * H * Fs * 34 // 32 + T * H * 2 + T * Fs * 6 + T * H * 8) / 3
     return kb
 
 
@@ -429,6 +435,13 @@ def build_stack(B, wl, n_layers, dev, seed_off):
     return layers, routers
 
 
+def build_shared(B, wl, n_layers, dev, seed_off):
+    """The shared expert of each layer of the stack (8-bit blocks)."""
+    import synthetic
+    return [B.SharedExpert(*[synthetic.shared_matrix(wl, seed_off + l, r, dev) for r in ("gate", "up", "down")])
+            for l in range(n_layers)]
+
+
 def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do_e2e=True):
     """Warm-up, CUDA-graph capture and the timed region for one workload,
     then its per-kernel times and roofline.  Returns the result dict."""
@@ -441,10 +454,22 @@ def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do
     xs = [synthetic.activations(wl, seed_off + j, device=dev) for j in range(NX)]
     ws = B.Workspace.for_layer(layers[0], T)
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
+    shared = build_shared(B, wl, L, dev, seed_off) if wl.shared_ffn else None
+    if shared:
+        sxq = torch.empty((T, H), dtype=torch.int8, device=dev)
+        sxd = torch.empty((T, H // 32), dtype=torch.float32, device=dev)
+        sws = shared[0].workspace(T, dev)
     torch.cuda.synchronize()
 
     def step(j):
         B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
+        if shared:
+            # the shared expert's FFN added to y: x^ again (the step's own copy
+            # stays inside the fused kernels), then the 8-bit gate/up, the
+            # requantization and the down mat-vec with the add
+            B.lib().moe_quant_act_q8(xs[j % NX].data_ptr(), T, H, sxq.data_ptr(), sxd.data_ptr(),
+                                     torch.cuda.current_stream().cuda_stream)
+            shared[j % L].add(sxq, sxd, y, ws=sws)
 
     for j in range(warmup):
         step(j)
@@ -553,7 +578,7 @@ def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do
     # Every step copies its x in from pinned host memory and its y out to pinned
     # host memory on the stream; the steps are replayed from CUDA graphs of
     # moe_forward_host calls, as a serving loop would drive them.
-    if do_e2e:
+    if do_e2e and not wl.shared_ffn:  # the host-buffer entry point has no shared expert
         n_e2e = min(steps, 2000)
         xh = [xs[j % NX].cpu().pin_memory() for j in range(min(NX, n_e2e))]
         yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
@@ -598,7 +623,7 @@ def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do
 # the other configurations measured in the same run (single GPU): the large
 # layer at 8 tokens, the 30B-class layer at 1 and 16 tokens, and its
 # 2048-token prefill
-SUITE = ("large-b8", "30b", "30b-b16", "30b-prefill")
+SUITE = ("large-b8", "30b", "30b-shared", "30b-b16", "30b-prefill")
 
 
 def main():

@@ -14,6 +14,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbitmoe.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libbitmoe_checked.so")  # -DMOE_CHECKED, for the tests
 
 BLOCK = 256
 BLOCK_WORDS = 13
@@ -24,7 +25,7 @@ MAX_DECODE_TOKENS = 64
 STATUS = {
     0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED_SHAPE",
     -3: "MOE_ERR_ALIGNMENT", -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA",
-    -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_BAD_INDEX", -8: "MOE_ERR_DEVICE",
+    -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_BAD_INDEX", -8: "MOE_ERR_DEVICE", -9: "MOE_ERR_BOUNDS",
 }
 
 # every symbol include/bitmoe.h declares
@@ -78,44 +79,51 @@ def lib():
         if not os.path.exists(LIB_PATH):
             raise RuntimeError("libbitmoe.so is not built (run `python -m bit_moe_b200.build`); "
                                "the ternary MoE path has no other implementation")
-        L = ctypes.CDLL(LIB_PATH)
-        p, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
-        sig = {
-            "moe_trit_words": (sz, [i64, i64]),
-            "moe_sign_words": (sz, [i64, i64]),
-            "moe_e16_code_words": (sz, [i64, i64]),
-            "moe_scale_count": (sz, [i64, i64]),
-            "moe_workspace_bytes": (sz, [p, i32, i32]),
-            "moe_workspace_init": (ctypes.c_int, [p, sz, p]),
-            "moe_quantize_weights": (ctypes.c_int, [p, i64, i64, p, p, p]),
-            "moe_quantize_weights_sign": (ctypes.c_int, [p, i64, i64, p, p, p]),
-            "moe_quantize_weights_e16": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
-            "moe_quantize_weights_q8": (ctypes.c_int, [p, i64, i64, p, p, p]),
-            "moe_shared_workspace_bytes": (sz, [p, i32]),
-            "moe_shared_ffn_add": (ctypes.c_int, [p, i32, p, p, p, p, sz, p]),
-            "moe_quant_act_q8": (ctypes.c_int, [p, i32, i32, p, p, p]),
-            "moe_route_topk": (ctypes.c_int, [p, p, i32, i32, i32, i32, p, p, p, sz, p]),
-            "moe_route_workspace_bytes": (sz, [i32, i32]),
-            "moe_expert_ffn_decode": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, p]),
-            "moe_expert_ffn_prefill": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, p]),
-            "moe_forward": (ctypes.c_int, [p, p, i32, p, p, p, sz, p]),
-            "moe_forward_host": (ctypes.c_int, [p, p, i32, p, p, p, sz, p]),
-            "moe_check_status": (ctypes.c_int, [p, p]),
-            "moe_last_error": (ctypes.c_char_p, []),
-            "moe_debug_matvec": (ctypes.c_int, [p, i32, p, p, p, p, p]),
-            "moe_launch_count": (i64, []),
-            "moe_trace_begin": (ctypes.c_int, [p, i32]),
-            "moe_trace_end": (ctypes.c_int, [p, i32]),
-            "moe_kernel_name": (ctypes.c_char_p, [i32]),
-            "moe_expert_ffn_decode_static": (ctypes.c_int, [p, i32, p, p, p, p, p, p]),
-            "moe_debug_ffn_blocksums": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, i32, p, p, p, p]),
-            "moe_debug_wait_knob": (ctypes.c_int, [p, sz, i32, i32, p]),
-        }
-        for name, (res, args) in sig.items():
-            fn = getattr(L, name)
-            fn.restype, fn.argtypes = res, args
-        _lib = L
+        _lib = load_library(LIB_PATH)
     return _lib
+
+
+def load_library(path):
+    """A ctypes handle of a build of the library at `path` (the normal build,
+    or the bounds-checked one that the tests load), with every entry point's
+    signature set."""
+    L = ctypes.CDLL(path)
+    p, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    sig = {
+        "moe_trit_words": (sz, [i64, i64]),
+        "moe_sign_words": (sz, [i64, i64]),
+        "moe_e16_code_words": (sz, [i64, i64]),
+        "moe_scale_count": (sz, [i64, i64]),
+        "moe_workspace_bytes": (sz, [p, i32, i32]),
+        "moe_workspace_init": (ctypes.c_int, [p, sz, p]),
+        "moe_quantize_weights": (ctypes.c_int, [p, i64, i64, p, p, p]),
+        "moe_quantize_weights_sign": (ctypes.c_int, [p, i64, i64, p, p, p]),
+        "moe_quantize_weights_e16": (ctypes.c_int, [p, i64, i64, p, p, p, p]),
+        "moe_quantize_weights_q8": (ctypes.c_int, [p, i64, i64, p, p, p]),
+        "moe_shared_workspace_bytes": (sz, [p, i32]),
+        "moe_shared_ffn_add": (ctypes.c_int, [p, i32, p, p, p, p, sz, p]),
+        "moe_quant_act_q8": (ctypes.c_int, [p, i32, i32, p, p, p]),
+        "moe_route_topk": (ctypes.c_int, [p, p, i32, i32, i32, i32, p, p, p, sz, p]),
+        "moe_route_workspace_bytes": (sz, [i32, i32]),
+        "moe_expert_ffn_decode": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, p]),
+        "moe_expert_ffn_prefill": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, p]),
+        "moe_forward": (ctypes.c_int, [p, p, i32, p, p, p, sz, p]),
+        "moe_forward_host": (ctypes.c_int, [p, p, i32, p, p, p, sz, p]),
+        "moe_check_status": (ctypes.c_int, [p, p]),
+        "moe_last_error": (ctypes.c_char_p, []),
+        "moe_debug_matvec": (ctypes.c_int, [p, i32, p, p, p, p, p]),
+        "moe_launch_count": (i64, []),
+        "moe_trace_begin": (ctypes.c_int, [p, i32]),
+        "moe_trace_end": (ctypes.c_int, [p, i32]),
+        "moe_kernel_name": (ctypes.c_char_p, [i32]),
+        "moe_expert_ffn_decode_static": (ctypes.c_int, [p, i32, p, p, p, p, p, p]),
+        "moe_debug_ffn_blocksums": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, i32, p, p, p, p]),
+        "moe_debug_wait_knob": (ctypes.c_int, [p, sz, i32, i32, p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype, fn.argtypes = res, args
+    return L
 
 
 def _check(rc):

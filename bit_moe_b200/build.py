@@ -32,20 +32,33 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale():
-    if not os.path.exists(OUT):
+def _stale(out=None):
+    out = OUT if out is None else out
+    if not os.path.exists(out):
         return True
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force=False, verbose=False, extra=()):
+CHECKED_OUT = os.path.join(HERE, "libbitmoe_checked.so")
+
+
+def build_checked(force=False, verbose=False):
+    """The bounds-checked build (-DMOE_CHECKED): every guarded index that
+    falls outside its buffer records MOE_ERR_BOUNDS and the access is skipped.
+    The tests load it beside the normal build (no memory checker runs on this
+    pool's GPUs)."""
+    return build(force=force, verbose=verbose, extra=("-DMOE_CHECKED",), out=CHECKED_OUT)
+
+
+def build(force=False, verbose=False, extra=(), out=None):
     """Compile every source to an object file (in parallel, one nvcc per
-    source) and link them into libbitmoe.so."""
-    if not force and not _stale():
-        return OUT
-    tag = ".tmp.%d" % os.getpid()
+    source) and link them into libbitmoe.so (or `out`)."""
+    out = OUT if out is None else out
+    if not force and not _stale(out):
+        return out
+    tag = ".tmp.%d.%d" % (os.getpid(), len(extra))
     flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
              "--expt-relaxed-constexpr", *extra]
     srcs = sources()
@@ -64,19 +77,21 @@ def build(force=False, verbose=False, extra=()):
         bad = [s for s, rc in zip(srcs, rcs) if rc != 0]
         if bad:
             raise subprocess.CalledProcessError(1, "nvcc " + " ".join(os.path.basename(b) for b in bad))
-        tmp = OUT + tag
+        tmp = out + tag
         cmd = [nvcc_path(), *ARCH, "-shared", "-o", tmp, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
-        os.replace(tmp, OUT)
+        os.replace(tmp, out)
     finally:
         for o in objs:
             if os.path.exists(o):
                 os.remove(o)
-    return OUT
+    return out
 
 
 if __name__ == "__main__":
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []
     print(build(force="--force" in sys.argv or bool(extra), verbose=True, extra=extra))
+    if "--checked" in sys.argv:
+        print(build_checked(force="--force" in sys.argv, verbose=True))

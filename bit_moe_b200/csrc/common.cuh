@@ -93,6 +93,18 @@ __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
   atomicCAS(status, 0, code);
 }
 
+// Bounds-checked build (compiled with -DMOE_CHECKED; the tests build it as
+// a separate library): MOE_IN(i, n) is true when 0 <= i < n; otherwise it
+// records MOE_ERR_BOUNDS in the status word and is false, so that the guarded
+// access is skipped.  In the normal build it is always true and costs nothing.
+#ifdef MOE_CHECKED
+#define MOE_IN(i, n, status) \
+  ((static_cast<unsigned long long>(i) < static_cast<unsigned long long>(n)) ? true \
+   : (record_status((status), MOE_ERR_BOUNDS), false))
+#else
+#define MOE_IN(i, n, status) true
+#endif
+
 // fp64 -> binary16, round to nearest even, in one conversion.
 __device__ __forceinline__ uint16_t f64_to_f16_rn(double x) {
   uint16_t h;
@@ -103,14 +115,6 @@ __device__ __forceinline__ uint16_t f64_to_f16_rn(double x) {
 __device__ __forceinline__ float f16_bits_to_f32(uint16_t h) {
   return __half2float(__ushort_as_half(h));
 }
-
-// The base-3 decode multiplies two registers of 16-bit lanes by 3 per digit
-// level.  Left to itself the compiler turns both into shift-adds on the ALU
-// pipe, which also carries the byte permutes; taking one factor from constant
-// memory (a value the compiler cannot fold) keeps that multiply an integer
-// multiply-add on the FMA pipe, and the two pipes share the decode.
-static __constant__ uint32_t g_three = 3u;
-__device__ __forceinline__ uint32_t mul3_fma(uint32_t x) { return x * g_three; }
 
 // Streaming 32-bit load that does not allocate in L1 (weights are read once).
 __device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t* p) {

@@ -201,8 +201,10 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
     int q = 0;
     if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
     const int pair = item_pair(P, item, n);
-    P.aq[static_cast<size_t>(pair) * F + panel * kPanel + lane] = static_cast<int8_t>(q);
-    if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + panel] = dd;
+    if (pair_ok(P, pair)) {
+      P.aq[static_cast<size_t>(pair) * F + panel * kPanel + lane] = static_cast<int8_t>(q);
+      if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + panel] = dd;
+    }
   }
 }
 
@@ -221,8 +223,10 @@ __global__ void __launch_bounds__(kGateUpWarps * 32, 4) k_gateup(DecodeParams P)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < item.count) {
       const int pair = item_pair(P, item, warp);
-      P.aq[static_cast<size_t>(pair) * P.ffn + panel * kPanel + lane] = 0;
-      if (lane == 0) P.ad[static_cast<size_t>(pair) * (P.ffn / kQBlock) + panel] = 0.f;
+      if (pair_ok(P, pair)) {
+        P.aq[static_cast<size_t>(pair) * P.ffn + panel * kPanel + lane] = 0;
+        if (lane == 0) P.ad[static_cast<size_t>(pair) * (P.ffn / kQBlock) + panel] = 0.f;
+      }
     }
     return;
   }
@@ -281,7 +285,8 @@ __device__ __forceinline__ void down_run(const DecodeParams& P, const Item& item
 #pragma unroll
   for (int n = 0; n < NT; ++n)
     if (n < item.count)
-      P.ye[static_cast<size_t>(item_pair(P, item, n)) * H + panel * kPanel + lane] = out[0][n];
+      if (pair_ok(P, item_pair(P, item, n)))
+        P.ye[static_cast<size_t>(item_pair(P, item, n)) * H + panel * kPanel + lane] = out[0][n];
   __threadfence();
   __syncwarp();
   for (int n = 0; n < item.count; ++n) arrive_and_combine(P, item_pair(P, item, n), panel, lane);
@@ -300,7 +305,8 @@ __global__ void __launch_bounds__(kDownWarps * 32, 8) k_down(DecodeParams P) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int panel = pgroup * kDownWarps + warp;
     for (int n = 0; n < item.count; ++n)
-      P.ye[static_cast<size_t>(item_pair(P, item, n)) * P.hidden + panel * kPanel + lane] = 0.f;
+      if (pair_ok(P, item_pair(P, item, n)))
+        P.ye[static_cast<size_t>(item_pair(P, item, n)) * P.hidden + panel * kPanel + lane] = 0.f;
     __threadfence();
     __syncwarp();
     for (int n = 0; n < item.count; ++n) arrive_and_combine(P, item_pair(P, item, n), panel, lane);

@@ -67,7 +67,13 @@ __device__ __forceinline__ bool fetch_item(const DecodeParams& P, int it, Item& 
 }
 
 __device__ __forceinline__ int item_pair(const DecodeParams& P, const Item& item, int n) {
+  if (!P.direct && !MOE_IN(item.start + n, P.ntok * P.top_k, P.status)) return 0;
   return P.direct ? item.start + n : P.pairs[item.start + n];
+}
+
+// Bounds-checked build: a (token, slot) pair id inside [0, ntok * top_k).
+__device__ __forceinline__ bool pair_ok(const DecodeParams& P, int pair) {
+  return MOE_IN(pair, P.ntok * P.top_k, P.status);
 }
 
 // The CTA that completes the last of token t's top_k slots for 32-row panel
@@ -78,6 +84,7 @@ __device__ __forceinline__ void arrive_and_combine(const DecodeParams& P, int pa
                                                    int lane) {
   const int K = P.top_k, H = P.hidden;
   const int t = pair / K;
+  if (!MOE_IN(t, P.ntok, P.status) || !MOE_IN(panel, H / kPanel, P.status)) return;
   int32_t* c = P.cnt + static_cast<size_t>(t) * (H / kPanel) + panel;
   int old = 0;
   if (lane == 0) old = atomicAdd(c, 1);

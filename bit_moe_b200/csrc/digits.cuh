@@ -19,7 +19,6 @@ namespace bitmoe {
 
 // Digit words [32*kHalf, 32*kHalf + 32) of one block from packed words
 // w[jj] = word 6*kHalf + jj, jj in [0, 7) (word 6 feeds both halves).
-// One of the two lane multiplies of a level runs on the FMA pipe (mul3_fma).
 template <int kHalf>
 __device__ __forceinline__ void digit_half(const uint32_t (&w)[7], uint32_t (&dg)[32]) {
   // level-major: the 7 words' chains advance side by side (7 independent
@@ -41,7 +40,7 @@ __device__ __forceinline__ void digit_half(const uint32_t (&w)[7], uint32_t (&dg
       // levels past the half's last digit word are not needed
       if (c >= 32) continue;
       lo[jj] *= 3u;
-      hi[jj] = mul3_fma(hi[jj]);
+      hi[jj] *= 3u;
       const uint32_t hn = __byte_perm(lo[jj], hi[jj], 0x7351);
       if (c >= 0) dg[c] = hn - 3u * hp[jj];
       hp[jj] = hn;

@@ -179,7 +179,7 @@ __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
       lo[m] = w[m][j] & 0x00FF00FFu;
-      hi[m] = __byte_perm(w[m][j], 0u, 0x4341);
+      hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
       hp[m] = 0u;
     }
 #pragma unroll
@@ -192,7 +192,7 @@ __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         lo[m] *= 3u;
-        hi[m] = mul3_fma(hi[m]);
+        hi[m] *= 3u;
         const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
         const int t = static_cast<int>(hn - 3u * hp[m]);
         hp[m] = hn;

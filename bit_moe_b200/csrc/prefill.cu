@@ -113,11 +113,12 @@ __global__ void __launch_bounds__(kPN * kSubPerBlock) k_prefill_gather(DecodePar
   for (int64_t w = blockIdx.x; w < work; w += gridDim.x) {
     const Item it = P.items[w / nb];
     const int b = static_cast<int>(w % nb);
+    if (!MOE_IN(w / nb, P.ntok * P.top_k / kPN + P.n_experts + 1, P.status)) continue;
     BStage* dst = reinterpret_cast<BStage*>(P.bgu) + w;
-    const int pair = n < it.count ? P.pairs[it.start + n] : -1;
+    const int pair = n < it.count && MOE_IN(it.start + n, P.ntok * P.top_k, P.status) ? P.pairs[it.start + n] : -1;
     int4 c[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
     float d = 0.f;
-    if (pair >= 0) {
+    if (pair >= 0 && pair_ok(P, pair)) {
       const int8_t* src = P.xq + static_cast<size_t>(pair / K) * H + b * kBlock + s * kQBlock;
       c[0] = *reinterpret_cast<const int4*>(src);
       c[1] = *reinterpret_cast<const int4*>(src + 16);
@@ -192,6 +193,7 @@ __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, 
   const int F = P.ffn;
   const int f = 64 * mt + r;
   const int bf = f / kBlock, sub = (f % kBlock) / kQBlock;
+  if (!MOE_IN(item, P.ntok * P.top_k / kPN + P.n_experts + 1, P.status) || !MOE_IN(bf, F / kBlock, P.status)) return;
   BStage* dst = reinterpret_cast<BStage*>(P.bdn) + static_cast<size_t>(item) * (F / kBlock) + bf;
 #pragma unroll 4
   for (int n = 0; n < kFixPairs; ++n) {
@@ -209,7 +211,7 @@ __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, 
       dst->d[sub][np] = dd;
       dst->m[sub][np] = kMagicF + static_cast<float>(sum);
     }
-    if (kDbg && np < it.count)  // test hook: the SwiGLU codes
+    if (kDbg && np < it.count && pair_ok(P, P.pairs[it.start + np]))  // test hook: the SwiGLU codes
       P.aq[static_cast<size_t>(P.pairs[it.start + np]) * F + f] = static_cast<int8_t>(qq);
   }
 }
@@ -301,7 +303,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
           if (q >= 2) write_down_codes<kDbg>(P, T.mt, T.item, 32 * (q - 2) + lane, n0, nullptr, T.it, lane);
         } else {
           for (int n = n0; n < n0 + kFixPairs && n < T.it.count; ++n)
-            P.ye[static_cast<size_t>(P.pairs[T.it.start + n]) * H + kPM * T.mt + 32 * q + lane] = 0.f;
+            if (pair_ok(P, P.pairs[T.it.start + n]))
+              P.ye[static_cast<size_t>(P.pairs[T.it.start + n]) * H + kPM * T.mt + 32 * q + lane] = 0.f;
         }
         continue;
       }
@@ -326,17 +329,19 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
           const int ds = si % kDStages;
           if (!wait_or_abort(&S.d_full[ds], (si / kDStages) & 1u, S, P.status)) { ok = false; break; }
           tc_fence_after();
+          // both sub-blocks' sums in one round trip to tensor memory, then
+          // the stage goes back to the MMA
+          uint32_t vv[kDSub][kFixPairs];
+#pragma unroll
+          for (int s2 = 0; s2 < kDSub; ++s2) tmem_ld16(tlane + kDcol + kDSub * kPN * ds + kPN * s2 + n0, vv[s2]);
+          tc_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.d_empty[ds]);
 #pragma unroll
           for (int s2 = 0; s2 < kDSub; ++s2) {
             const int s = kDSub * h + s2;
-            uint32_t v[kFixPairs];
-            tmem_ld16(tlane + kDcol + kDSub * kPN * ds + kPN * s2 + n0, v);
-            tc_wait_ld();
-            if (s2 == kDSub - 1) {  // the stage goes back to the MMA
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&S.d_empty[ds]);
-            }
+            const uint32_t (&v)[kFixPairs] = vv[s2];
             const float* dp = &S.st[bs].d[s][n0];
             const float* mp = &S.st[bs].m[s][n0];
             if (kDbg) {  // test hook: the exact block sums
@@ -407,7 +412,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
         const int hrow = kPM * T.mt + 32 * q + lane;
 #pragma unroll
         for (int n = 0; n < kFixPairs; ++n)
-          if (n0 + n < T.it.count) P.ye[static_cast<size_t>(P.pairs[T.it.start + n0 + n]) * H + hrow] = y[n];
+          if (n0 + n < T.it.count && pair_ok(P, P.pairs[T.it.start + n0 + n]))
+            P.ye[static_cast<size_t>(P.pairs[T.it.start + n0 + n]) * H + hrow] = y[n];
       }
     }
   } else if (warp == kWCopyW && lane == 0) {

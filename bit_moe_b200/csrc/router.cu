@@ -224,7 +224,11 @@ bool router_quant_small_ok(int ntok, int H) { return ntok <= kMaxDecodeTokens &&
 int launch_router_quant_small(const float* x, const float* wr, int ntok, int H, int E, float* logits,
                               int8_t* xq, float* xd, cudaStream_t stream) {
   if (!router_quant_small_ok(ntok, H)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "router_quant: shape");
-  if (H % kRtKCWide == 0)
+  if (H % kRtKCWide == 0 && ntok <= kRtT)
+    // one token tile: 16 x 2 tiles (all 8 warps along the tokens), so that
+    // E/2 CTAs share the router rows instead of E/8
+    launch_tiled<1, 2, 2, kRtKCWide>(x, wr, ntok, H, E, logits, stream, xq, xd);
+  else if (H % kRtKCWide == 0)
     launch_tiled<2, 4, 2, kRtKCWide>(x, wr, ntok, H, E, logits, stream, xq, xd);  // 16 x 4 tiles, wide chunks
   else
     launch_tiled<2, 4, 2>(x, wr, ntok, H, E, logits, stream, xq, xd);

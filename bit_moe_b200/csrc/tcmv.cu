@@ -338,13 +338,15 @@ __global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n)
           if (q >= 2) {
             for (int n = n0; n < n0 + kTFixPairs && n < U.it.count; ++n) {
               const int pair = item_pair(P, U.it, n);
+              if (!pair_ok(P, pair)) continue;
               P.aq[static_cast<size_t>(pair) * F + 64 * U.mt + 32 * (q - 2) + lane] = 0;
               if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + 2 * U.mt + (q - 2)] = 0.f;
             }
           }
         } else {
           for (int n = n0; n < n0 + kTFixPairs && n < U.it.count; ++n)
-            P.ye[static_cast<size_t>(item_pair(P, U.it, n)) * H + kTM * U.mt + 32 * q + lane] = 0.f;
+            if (pair_ok(P, item_pair(P, U.it, n)))
+              P.ye[static_cast<size_t>(item_pair(P, U.it, n)) * H + kTM * U.mt + 32 * q + lane] = 0.f;
           __threadfence();
           __syncwarp();
           for (int n = n0; n < n0 + kTFixPairs && n < U.it.count; ++n)
@@ -416,8 +418,10 @@ __global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n)
             int qq = 0;
             if (dd != 0.f) qq = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
             const int pair = item_pair(P, U.it, n0 + n);
-            P.aq[static_cast<size_t>(pair) * F + 64 * U.mt + rr] = static_cast<int8_t>(qq);
-            if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + 2 * U.mt + (q - 2)] = dd;
+            if (pair_ok(P, pair)) {
+              P.aq[static_cast<size_t>(pair) * F + 64 * U.mt + rr] = static_cast<int8_t>(qq);
+              if (lane == 0) P.ad[static_cast<size_t>(pair) * (F / kQBlock) + 2 * U.mt + (q - 2)] = dd;
+            }
           }
         }
         __syncwarp();
@@ -426,7 +430,8 @@ __global__ void __launch_bounds__(kTThreads, 1) k_tcmv(DecodeParams P, int ks_n)
       } else {
         const int hrow = kTM * U.mt + 32 * q + lane;
         for (int n = 0; n < kTFixPairs && n0 + n < U.it.count; ++n)
-          P.ye[static_cast<size_t>(item_pair(P, U.it, n0 + n)) * H + hrow] = acc[0][n];
+          if (pair_ok(P, item_pair(P, U.it, n0 + n)))
+            P.ye[static_cast<size_t>(item_pair(P, U.it, n0 + n)) * H + hrow] = acc[0][n];
         __threadfence();
         __syncwarp();
         for (int n = 0; n < kTFixPairs && n0 + n < U.it.count; ++n)

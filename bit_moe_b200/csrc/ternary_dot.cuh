@@ -171,7 +171,7 @@ __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
           lo[m] = w[m][j] & 0x00FF00FFu;
-          hi[m] = __byte_perm(w[m][j], 0u, 0x4341);
+          hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
           hp[m] = 0u;
         }
 #pragma unroll
@@ -183,7 +183,7 @@ __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
 #pragma unroll
           for (int m = 0; m < NM; ++m) {
             lo[m] *= 3u;
-            hi[m] = mul3_fma(hi[m]);
+            hi[m] *= 3u;
             const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
             const int t = static_cast<int>(hn - 3u * hp[m]);
             hp[m] = hn;
@@ -263,7 +263,7 @@ __device__ __forceinline__ void panel_dot_e16(const uint32_t* const (&tw)[NM], c
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         lo[m] = w[m][j] & 0x00FF00FFu;
-        hi[m] = __byte_perm(w[m][j], 0u, 0x4341);
+        hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
         hp[m] = 0u;
       }
 #pragma unroll
@@ -277,7 +277,7 @@ __device__ __forceinline__ void panel_dot_e16(const uint32_t* const (&tw)[NM], c
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
           lo[m] *= 3u;
-          hi[m] = mul3_fma(hi[m]);
+          hi[m] *= 3u;
           const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
           const int t = static_cast<int>(hn - 3u * hp[m]);
           hp[m] = hn;

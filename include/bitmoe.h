@@ -82,7 +82,10 @@ typedef enum {
   MOE_ERR_CUDA = -5,              /* a CUDA runtime error (see moe_last_error)  */
   MOE_ERR_TIMEOUT = -6,           /* a bounded device-side wait ran out         */
   MOE_ERR_BAD_INDEX = -7,         /* an expert id outside [0, n_experts)        */
-  MOE_ERR_DEVICE = -8             /* the current device is not sm_100           */
+  MOE_ERR_DEVICE = -8,            /* the current device is not sm_100           */
+  MOE_ERR_BOUNDS = -9             /* bounds-checked build only (MOE_CHECKED): a
+                                     kernel computed an index outside its buffer
+                                     and skipped the access                     */
 } moe_status;
 
 /* Weight formats. */

@@ -14,7 +14,8 @@ pages; weights are random-init, not trained):
   moe-h256-f512-e8-k2       tiny layer, weights N(0, 0.02)
   moe-h2048-f768-e128-k8    30B-class layer, weights N(0, 0.02)
   moe-h4096-f2048-e256-k8   large layer, weights N(0, 0.015), 5-layer stack
-Router weights N(0, 0.02); activations N(0, 1).
+Router weights N(0, 0.02); activations N(0, 1); a shared expert (where a
+workload has one) N(0, w_std) like the routed experts.
 """
 import hashlib
 from dataclasses import dataclass, replace
@@ -22,7 +23,8 @@ from dataclasses import dataclass, replace
 import numpy as np
 import torch
 
-ROLE_IDS = {"gate": 1, "up": 2, "down": 3, "router": 4, "x": 5}
+ROLE_IDS = {"gate": 1, "up": 2, "down": 3, "router": 4, "x": 5,
+            "shared_gate": 6, "shared_up": 7, "shared_down": 8}
 
 
 @dataclass(frozen=True)
@@ -40,6 +42,7 @@ class Workload:
     seed: int = 0
     fmt: str = "ternary"     # packed weight format: "ternary", "sign" (1-bit sign codes) or
                              # "e16" (ternary digits with two-level scales)
+    shared_ffn: int = 0      # >0: a shared expert of this ffn width in 8-bit blocks beside the routed ones
 
     def with_(self, **kw):
         return replace(self, **kw)
@@ -61,8 +64,9 @@ class Workload:
         return 2 * self.matrix_bytes(self.ffn, self.hidden) + self.matrix_bytes(self.hidden, self.ffn)
 
     def describe(self):
-        return "%s%s-t%d%s" % (self.name, "" if self.fmt == "ternary" else "-" + self.fmt, self.ntok,
-                               "-prefill" if self.prefill else "")
+        return "%s%s%s-t%d%s" % (self.name, "" if self.fmt == "ternary" else "-" + self.fmt,
+                                 "-shared%d" % self.shared_ffn if self.shared_ffn else "", self.ntok,
+                                 "-prefill" if self.prefill else "")
 
 
 WORKLOADS = {
@@ -85,6 +89,9 @@ WORKLOADS = {
                         fmt="e16"),
     "large-e16-b8": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 8, 0.015, layers=5,
                              seed=8, fmt="e16"),
+    # the 30B-class layer with a shared expert (ffn 768, 8-bit blocks) beside the routed ones
+    "30b-shared": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 1, 0.02, layers=4, seed=1,
+                           shared_ffn=768),
     # prefill of 2048 tokens through the 30B-class layer
     "30b-prefill": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 2048, 0.02,
                             layers=1, prefill=True, seed=4),
@@ -118,6 +125,13 @@ def expert_matrix(wl: Workload, layer: int, role: str, expert: int, device="cpu"
     """One expert's fp32 matrix: gate/up [ffn][hidden], down [hidden][ffn]."""
     rows, k = (wl.hidden, wl.ffn) if role == "down" else (wl.ffn, wl.hidden)
     return gaussian((wl.seed, layer, ROLE_IDS[role], expert), (rows, k), wl.w_std, device)
+
+
+def shared_matrix(wl: Workload, layer: int, role: str, device="cpu"):
+    """The shared expert's fp32 matrix: gate/up [shared_ffn][hidden], down
+    [hidden][shared_ffn]; role "gate", "up" or "down"."""
+    rows, k = (wl.hidden, wl.shared_ffn) if role == "down" else (wl.shared_ffn, wl.hidden)
+    return gaussian((wl.seed, layer, ROLE_IDS["shared_" + role], 0), (rows, k), wl.w_std, device)
 
 
 def router(wl: Workload, layer: int, device="cpu"):
