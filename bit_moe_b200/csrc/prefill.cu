@@ -93,7 +93,8 @@ struct PrefillSmem {
   alignas(128) uint32_t w[kWStages][4][kBlockWords * kPanel];  // packed words, [panel][word][row]
   alignas(16) uint16_t wsc[kWStages][4][kPanel];                // fp16 block scales, [panel][row]
   alignas(128) BStage st[kBStages];
-  float xch[64][kPN + 1];  // gate results for the up rows
+  alignas(128) unsigned char neg1[kPM * 32];  // A operand of all -1 (s8): D = -sum(a) before the digits' MMA
+  float xch[2][64][kPN + 1];  // the tile's gate and up results, [row][pair], for the epilogue
 };
 
 // Byte offset of activation code (pair n, k in [0, 32)) of sub-block s: 8-row
@@ -183,11 +184,11 @@ __device__ __forceinline__ const uint16_t* panel_scales(const DecodeParams& P, i
   return kGU ? (p < 2 ? P.gate_scales : P.up_scales) : P.down_scales;
 }
 
-// The gate/up epilogue's output for pairs [n0, n0 + kFixPairs) at ffn row f of a
+// The gate/up epilogue's output for pairs [n0, n0 + kNP) at ffn row f of a
 // tile: each lane (32 consecutive f, one 32-block) requantizes the SwiGLU
 // values a[] (absent pairs and bad groups: zeros) and writes the codes, scale
 // and m into the down input's activation block of the group.
-template <bool kDbg>
+template <bool kDbg, int kNP>
 __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, int item, int r, int n0,
                                                  const float* a, const Item& it, int lane) {
   const int F = P.ffn;
@@ -196,7 +197,7 @@ __device__ __forceinline__ void write_down_codes(const DecodeParams& P, int mt, 
   if (!MOE_IN(item, P.ntok * P.top_k / kPN + P.n_experts + 1, P.status) || !MOE_IN(bf, F / kBlock, P.status)) return;
   BStage* dst = reinterpret_cast<BStage*>(P.bdn) + static_cast<size_t>(item) * (F / kBlock) + bf;
 #pragma unroll 4
-  for (int n = 0; n < kFixPairs; ++n) {
+  for (int n = 0; n < kNP; ++n) {
     const int np = n0 + n;
     float dd = 0.f;
     int qq = 0;
@@ -256,6 +257,18 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = S.tmem_base;
+  for (int i = tid; i < kPM * 32 / 4; i += kPThreads) reinterpret_cast<uint32_t*>(S.neg1)[i] = 0xFFFFFFFFu;
+  fence_proxy_async_shared();  // read by the tensor cores
+  if (warp >= kWFix && warp < kWFix + kFixWarps) {
+    // every accumulator column starts out holding the offset 0x4B400000
+    const int q = (warp - kWFix) & 3, n0 = kFixPairs * ((warp - kWFix) >> 2);
+    for (int c = 0; c < kDStages * kDSub; ++c)
+      tmem_st16_fill(tbase + (static_cast<uint32_t>(q * 32) << 16) + kDcol + kPN * c + n0, kMagic);
+    tc_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   if (warp >= kWDec && warp < kWFix) {
     // ------------------------------------------------ decode: digits -> TMEM
     const uint32_t tlane = tbase + (static_cast<uint32_t>(warp * 32) << 16);
@@ -300,7 +313,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       if (T.it.expert < 0) {  // ids out of range: their outputs are zero
         if (warp == kWFix && lane == 0) record_status(P.status, MOE_ERR_BAD_INDEX);
         if (kGU) {
-          if (q >= 2) write_down_codes<kDbg>(P, T.mt, T.item, 32 * (q - 2) + lane, n0, nullptr, T.it, lane);
+          if (q >= 2) write_down_codes<kDbg, kFixPairs>(P, T.mt, T.item, 32 * (q - 2) + lane, n0, nullptr, T.it, lane);
         } else {
           for (int n = n0; n < n0 + kFixPairs && n < T.it.count; ++n)
             if (pair_ok(P, P.pairs[T.it.start + n]))
@@ -335,6 +348,10 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
 #pragma unroll
           for (int s2 = 0; s2 < kDSub; ++s2) tmem_ld16(tlane + kDcol + kDSub * kPN * ds + kPN * s2 + n0, vv[s2]);
           tc_wait_ld();
+          // the stage goes back holding the offset again
+#pragma unroll
+          for (int s2 = 0; s2 < kDSub; ++s2) tmem_st16_fill(tlane + kDcol + kDSub * kPN * ds + kPN * s2 + n0, kMagic);
+          tc_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.d_empty[ds]);
@@ -343,14 +360,13 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
             const int s = kDSub * h + s2;
             const uint32_t (&v)[kFixPairs] = vv[s2];
             const float* dp = &S.st[bs].d[s][n0];
-            const float* mp = &S.st[bs].m[s][n0];
             if (kDbg) {  // test hook: the exact block sums
 #pragma unroll
               for (int e = 0; e < kFixPairs; ++e) {
                 const int np = n0 + e;
                 if (np >= T.it.count) continue;
                 const int pair = P.pairs[T.it.start + np];
-                const int isum = static_cast<int>(__fsub_rn(__uint_as_float(v[e] + kMagic), mp[e]));
+                const int isum = static_cast<int>(__fsub_rn(__uint_as_float(v[e]), kMagicF));
                 const int sg = b * kSubPerBlock + s;
                 if (kGU) {
                   const int fr = 64 * T.mt + 32 * (q & 1) + lane;
@@ -364,13 +380,12 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
 #pragma unroll
             for (int n4 = 0; n4 < kFixPairs / 4; ++n4) {
               const float4 dd = reinterpret_cast<const float4*>(dp)[n4];
-              const float4 mm = reinterpret_cast<const float4*>(mp)[n4];
               const int nn = 4 * n4;
-              // (D + 0x4B400000) as fp32 minus m = sum(q*a), exact; then
-              // d * sum(q*a) as in the decode kernels
+              // D (0x4B400000 + sum(q*a)) as fp32 minus 12582912 = sum(q*a),
+              // exact; then d * sum(q*a) as in the decode kernels
               float i0, i1, i2, i3;
-              sub2(i0, i1, __uint_as_float(v[nn] + kMagic), __uint_as_float(v[nn + 1] + kMagic), mm.x, mm.y);
-              sub2(i2, i3, __uint_as_float(v[nn + 2] + kMagic), __uint_as_float(v[nn + 3] + kMagic), mm.z, mm.w);
+              sub2(i0, i1, __uint_as_float(v[nn]), __uint_as_float(v[nn + 1]), kMagicF, kMagicF);
+              sub2(i2, i3, __uint_as_float(v[nn + 2]), __uint_as_float(v[nn + 3]), kMagicF, kMagicF);
               fma2(inner[nn], inner[nn + 1], dd.x, dd.y, i0, i1, inner[nn], inner[nn + 1]);
               fma2(inner[nn + 2], inner[nn + 3], dd.z, dd.w, i2, i3, inner[nn + 2], inner[nn + 3]);
             }
@@ -386,23 +401,27 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       if (!ok) break;
       // ---- epilogue (rows 32*q + lane, pairs [n0, n0 + kFixPairs))
       if (kGU) {
-        if (q < 2) {
+        // gate rows (q < 2) and up rows (q >= 2) go to the exchange; then
+        // every fixup warp takes one 32-row block of f and 8 pairs: SwiGLU
+        // and the requantization of those (block, pair) columns
 #pragma unroll
-          for (int n = 0; n < kFixPairs; ++n) S.xch[32 * q + lane][n0 + n] = y[n];
-        }
+        for (int n = 0; n < kFixPairs; ++n) S.xch[q >> 1][32 * (q & 1) + lane][n0 + n] = y[n];
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.fx_bar[0]);
         if (!wait_or_abort(&S.fx_bar[0], ep & 1u, S, P.status)) break;
-        if (q >= 2) {
-          const int r = 32 * (q - 2) + lane;  // f offset within the tile
-          // the SwiGLU value replaces g in the exchange row (each entry is
-          // read and written by its own thread)
+        {
+          constexpr int kEpPairs = kPN * 2 / kFixWarps;  // 8 pairs per warp and row block
+          const int fw = warp - kWFix;
+          const int r = 32 * (fw & 1) + lane;            // f offset within the tile
+          const int e0 = kEpPairs * (fw >> 1);
+          // the SwiGLU value replaces g in the exchange (each entry is read
+          // and written by its own thread)
 #pragma unroll
-          for (int n = 0; n < kFixPairs; ++n) {
-            const float g = S.xch[r][n0 + n];
-            S.xch[r][n0 + n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), y[n]);
+          for (int n = 0; n < kEpPairs; ++n) {
+            const float g = S.xch[0][r][e0 + n];
+            S.xch[0][r][e0 + n] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), S.xch[1][r][e0 + n]);
           }
-          write_down_codes<kDbg>(P, T.mt, T.item, r, n0, &S.xch[r][n0], T.it, lane);
+          write_down_codes<kDbg, kEpPairs>(P, T.mt, T.item, r, e0, &S.xch[0][r][e0], T.it, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.fx_bar[1]);
@@ -466,6 +485,8 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   } else if (warp == kWMma && lane == 0) {
     // ------------------------------------------------ MMA issue
     const uint32_t idesc = idesc_i8(kPM, kPN);
+    const uint32_t idesc_neg = idesc_i8(kPM, kPN, true);
+    const uint64_t ndesc = smem_desc(smem_u32(S.neg1), 128, 256);
     uint32_t bi = 0, si = 0;
     bool ok = true;
     TileInfo T;
@@ -486,9 +507,12 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
           tc_fence_after();
 #pragma unroll
           for (int s2 = 0; s2 < kDSub; ++s2) {
+            // onto the offset: -sum(a) (all -1 A operand), then sum(t * a)
             const int s = kDSub * h + s2;
-            mma_i8_ts(tbase + kDcol + kDSub * kPN * ds + kPN * s2, tbase + kAcol + 64 * a + 8 * s,
-                      bdesc + static_cast<uint64_t>((s * kPN * 32) >> 4), idesc, false);
+            const uint32_t dcol = tbase + kDcol + kDSub * kPN * ds + kPN * s2;
+            const uint64_t bsub = bdesc + static_cast<uint64_t>((s * kPN * 32) >> 4);
+            mma_i8_ss(dcol, ndesc, bsub, idesc_neg, true);
+            mma_i8_ts(dcol, tbase + kAcol + 64 * a + 8 * s, bsub, idesc, true);
           }
           mma_commit(&S.d_full[ds]);
         }

@@ -136,6 +136,35 @@ __global__ void k_quant_act_q8(const float* __restrict__ x, int64_t nblk, int8_t
     quant_act_block(x, blk, lane, xq, xd);
 }
 
+// The same quantization, four 32-blocks per warp at a time: lane l holds
+// values 4l..4l+3 of the four blocks (one 16-byte load), the eight lanes of a
+// block reduce its amax, and each lane stores its four codes as one word.
+__global__ void k_quant_act_q8_x4(const float* __restrict__ x, int64_t ngroups, int8_t* __restrict__ xq,
+                                  float* __restrict__ xd) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups;
+       g += warps) {
+    const float4 v = reinterpret_cast<const float4*>(x + g * 4 * kQBlock)[lane];
+    float am = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+    for (int m = 1; m <= 4; m <<= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
+    const float d = __fdiv_rn(am, 127.f);
+    uint32_t packed = 0;
+    if (d != 0.f) {
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = max(-127, min(127, __float2int_rn(__fdiv_rn(vv[i], d))));
+        packed |= (static_cast<uint32_t>(q) & 0xffu) << (8 * i);
+      }
+    }
+    reinterpret_cast<uint32_t*>(xq + g * 4 * kQBlock)[lane] = packed;
+    if ((lane & 7) == 0) xd[g * 4 + (lane >> 3)] = d;
+  }
+}
+
 // Anchors of the two-level scales: one warp per row, lane l taking the
 // 16-weight blocks l, l+32, ...; A = fp16_RNE(max over the blocks of
 // mean|w|), each mean summed in fp64 in ascending order.
@@ -202,9 +231,16 @@ int launch_quant_act_q8(const float* x, int64_t ntok, int k, int8_t* xq, float* 
                         cudaStream_t stream) {
   const int64_t nblk = ntok * (k / kQBlock);
   const int warps_per_cta = 8;
-  int64_t grid = (nblk + warps_per_cta - 1) / warps_per_cta;
+  const bool vec = k % (4 * kQBlock) == 0 && reinterpret_cast<uintptr_t>(x) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(xq) % 4 == 0;
+  const int64_t units = vec ? nblk / 4 : nblk;
+  int64_t grid = (units + warps_per_cta - 1) / warps_per_cta;
   if (grid > 148 * 8) grid = 148 * 8;
-  launch_k(k_quant_act_q8, dim3(static_cast<unsigned>(grid)), dim3(warps_per_cta * 32), 0, stream, x, nblk, xq, xd);
+  if (vec)
+    launch_k(k_quant_act_q8_x4, dim3(static_cast<unsigned>(grid)), dim3(warps_per_cta * 32), 0, stream, x, units, xq,
+             xd);
+  else
+    launch_k(k_quant_act_q8, dim3(static_cast<unsigned>(grid)), dim3(warps_per_cta * 32), 0, stream, x, nblk, xq, xd);
   note_launch(MOE_K_QUANT_ACT, stream);
   return check_launch("quant_act_q8");
 }

@@ -193,6 +193,10 @@ int launch_router_logits(const float* x, const float* wr, int ntok, int H, int E
     int64_t grid = (total + 7) / 8;
     if (grid > 148 * 16) grid = 148 * 16;
     launch_k(k_router_logits, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, wr, ntok, H, E, logits);
+  } else if (ntok >= 4 * kRtT && E >= 64) {
+    // 16 tokens x 32 experts: an 8 x 8 micro-tile per lane, 16 shared-memory
+    // loads per 64 fused multiply-adds
+    launch_tiled<4, 8, 8>(x, wr, ntok, H, E, logits, stream);
   } else if (ntok >= 4 * kRtT) {
     launch_tiled<4, 8, 4>(x, wr, ntok, H, E, logits, stream);  // 16 x 16 tiles
   } else if (H % kRtKCWide == 0) {

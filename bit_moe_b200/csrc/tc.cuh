@@ -67,6 +67,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
       : "memory");
 }
 
+// Store the value c into 16 consecutive 32-bit columns of this thread's TMEM
+// lane, four columns per store (the stored registers must be consecutive, so
+// wider stores of one value would hold more registers).
+__device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t c) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%1,%1,%1};" ::"r"(taddr + 4 * i), "r"(c) : "memory");
+}
+
 // Load 1 or 2 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t (&v)[1]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v[0]) : "r"(taddr) : "memory");
@@ -118,11 +127,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 }
 
 // ---- MMA ----------------------------------------------------------------------
-// Instruction descriptor of tcgen05.mma kind::i8: D s32, A u8 (digits), B s8
-// (activation codes), both K-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+// Instruction descriptor of tcgen05.mma kind::i8: D s32, A u8 (digits; s8
+// with a_signed), B s8 (activation codes), both K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed = false) {
   return (2u << 4)                                // D format: s32
-         | (0u << 7)                              // A: unsigned 8-bit
+         | ((a_signed ? 1u : 0u) << 7)            // A: unsigned or signed 8-bit
          | (1u << 10)                             // B: signed 8-bit
          | (0u << 15) | (0u << 16)                // A, B K-major
          | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
@@ -162,6 +171,18 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc), "r"(z)
+      : "memory");
+}
+
+// D[tmem d] (+)= A[smem desc a] * B[smem desc b], kind::i8; issued by one thread.
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  const uint32_t z = 0u;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc), "r"(z)
       : "memory");
 }
 
