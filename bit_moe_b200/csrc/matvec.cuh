@@ -179,7 +179,7 @@ __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
       lo[m] = w[m][j] & 0x00FF00FFu;
-      hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
+      hi[m] = __byte_perm(w[m][j], 0u, 0x4341);  // bytes 1, 3 into 16-bit lanes
       hp[m] = 0u;
     }
 #pragma unroll

@@ -478,14 +478,19 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       }
     }
     __syncthreads();
+    // warp j applies slot j's block scales in order, then warp 0 combines
+    // the slots in order (the summation order of the grouped down kernel)
+    float* spart = reinterpret_cast<float*>(smem + L.red);  // [K][32]; the gate/up sums are done with it
+    if (!*abort && ok && warp < K) {
+      float part = 0.f;
+      for (int b = 0; b < nbF; ++b)
+        part = __fmaf_rn(sscale[(warp * nbF + b) * kPanel + lane], sinner[(warp * nbF + b) * kPanel + lane], part);
+      spart[warp * kPanel + lane] = part;
+    }
+    __syncthreads();
     if (!*abort && ok && warp == 0) {
       float y = 0.f;
-      for (int jj = 0; jj < K; ++jj) {
-        float part = 0.f;
-        for (int b = 0; b < nbF; ++b)
-          part = __fmaf_rn(sscale[(jj * nbF + b) * kPanel + lane], sinner[(jj * nbF + b) * kPanel + lane], part);
-        y = __fmaf_rn(sel_w[jj], part, y);
-      }
+      for (int jj = 0; jj < K; ++jj) y = __fmaf_rn(sel_w[jj], spart[jj * kPanel + lane], y);
       P.y[panelH * kPanel + lane] = y;
     }
   }

@@ -171,7 +171,7 @@ __device__ __forceinline__ void panel_dot(const uint32_t* const (&tw)[NM],
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
           lo[m] = w[m][j] & 0x00FF00FFu;
-          hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
+          hi[m] = __byte_perm(w[m][j], 0u, 0x4341);  // bytes 1, 3 into 16-bit lanes
           hp[m] = 0u;
         }
 #pragma unroll
@@ -263,7 +263,7 @@ __device__ __forceinline__ void panel_dot_e16(const uint32_t* const (&tw)[NM], c
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
         lo[m] = w[m][j] & 0x00FF00FFu;
-        hi[m] = (w[m][j] >> 8) & 0x00FF00FFu;
+        hi[m] = __byte_perm(w[m][j], 0u, 0x4341);  // bytes 1, 3 into 16-bit lanes
         hp[m] = 0u;
       }
 #pragma unroll
