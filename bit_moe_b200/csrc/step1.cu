@@ -108,8 +108,9 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
 }
 
 // Named barriers of gate/up stream h (kNC warps each): the unit's partial
-// sums are written (all warps sync), and read by the epilogue warp (it
-// arrives, the other warps sync before they overwrite them).
+// sums are written (the unit's epilogue warp syncs, the others arrive), and
+// read by the epilogue warp (it arrives, the other warps sync before they
+// overwrite them).
 __device__ __forceinline__ void stream_bar_sync(int id) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kNC * 32) : "memory");
 }
@@ -368,12 +369,18 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         __syncwarp();
         issue_next(slot);
       }
-      // the epilogue warp has read the previous unit's sums
-      if (ui > 0 && w8 != 0) stream_bar_sync(bar_free);
+      // unit ui's epilogue runs on warp ui % kNC of the stream, which waits
+      // for the stream's sums; the other warps leave theirs and go on with
+      // the next unit (before they overwrite the sums, the previous unit's
+      // epilogue warp has read them)
+      const int ep = ui % kNC, ep_prev = (ui + kNC - 1) % kNC;
+      if (ui > 0 && w8 != ep_prev) stream_bar_sync(bar_free);
       rb[(0 * kNC + w8) * 32 + lane] = part[0][0];
       rb[(1 * kNC + w8) * 32 + lane] = part[1][0];
-      stream_bar_sync(bar_done);
-      if (w8 == 0) {
+      if (w8 != ep) {
+        stream_bar_arrive(bar_done);
+      } else {
+        stream_bar_sync(bar_done);
         float g = 0.f, uu = 0.f;
         const int nw = nbH < kNC ? nbH : kNC;
         for (int v = 0; v < nw; ++v) {
