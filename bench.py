@@ -73,12 +73,6 @@ def measured_peaks():
 
 
 # --------------------------------------------------------------------------- bytes
-def matrix_bytes(rows, k, block_bytes=54):
-    """Packed bytes of a matrix: per 256 weights 52 B of base-3 digits (or 32 B
-    of sign bits) + 2 B of scale."""
-    return rows * (k // 256) * block_bytes
-
-
 def kernel_bytes(wl, unique_experts):
     """Algorithmic bytes per launch of each kernel for one step (each byte
     counted once: weights of the unique routed experts, activations in, results
@@ -91,9 +85,9 @@ def kernel_bytes(wl, unique_experts):
         # experts' packed weights, the int8 intermediates and y
         "step1": E * H * 4 + T * H * 4 + weights + 2 * (pairs * F + pairs * F // 32 * 4)
         + T * H + T * H // 32 * 4 + T * E * 4 + pairs * 8 + T * H * 4,
-        "prefill_gateup": unique_experts * 2 * matrix_bytes(F, H) + T * H + T * H // 32 * 4
+        "prefill_gateup": unique_experts * 2 * wl.matrix_bytes(F, H) + T * H + T * H // 32 * 4
         + pairs * F + pairs * F // 32 * 4,
-        "prefill_down": unique_experts * matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4 + pairs * H * 4,
+        "prefill_down": unique_experts * wl.matrix_bytes(H, F) + pairs * F + pairs * F // 32 * 4 + pairs * H * 4,
         "prefill_gather": pairs * H + pairs * H // 32 * 4,
         "combine": pairs * H * 4 + T * H * 4 + pairs * 4,
         "route": E * H * 4 + T * H * 4 + T * H + T * H // 32 * 4 + T * E * 4 + pairs * 8,

@@ -427,8 +427,6 @@ int moe_expert_ffn_prefill(const moe_layer* L, int32_t ntok, const int8_t* xq, c
                            moe_stream_t stream) {
   WsLayout W;
   int rc = ffn_common("expert_ffn_prefill", L, ntok, xq, xd, idx, wts, y, ws, ws_bytes, true, &W);
-  if (!rc && L->gate.format != MOE_FORMAT_TERNARY)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "expert_ffn_prefill: ternary layers only");
   if (rc) return rc;
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
   return launch_prefill(P, static_cast<cudaStream_t>(stream));
@@ -442,9 +440,6 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
   const bool sign = L->gate.format != MOE_FORMAT_TERNARY;  // sign codes or two-level scales
-  if (sign && prefill)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: sign-code and E16 layers take at most %d tokens",
-                kMaxDecodeTokens);
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total) return fail(MOE_ERR_WORKSPACE, "forward: workspace %zu < %zu bytes", ws_bytes, W.total);
   if ((rc = check_device())) return rc;
@@ -499,10 +494,6 @@ int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, co
   if ((rc = check_ptrs("forward_host", w_router, ws))) return rc;
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward_host: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
-  // refused before the copy of x is launched, as moe_forward would refuse it
-  if (prefill && L->gate.format != MOE_FORMAT_TERNARY)
-    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward_host: sign-code and E16 layers take at most %d tokens",
-                kMaxDecodeTokens);
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total)
     return fail(MOE_ERR_WORKSPACE, "forward_host: workspace %zu < %zu bytes", ws_bytes, W.total);

@@ -92,6 +92,7 @@ struct PrefillSmem {
   int abort;
   alignas(128) uint32_t w[kWStages][4][kBlockWords * kPanel];  // packed words, [panel][word][row]
   alignas(16) uint16_t wsc[kWStages][4][kPanel];                // fp16 block scales, [panel][row]
+  alignas(16) uint32_t wc[kWStages][4][kE16Words * kPanel];     // two-level scales: 4-bit codes, [panel][word][row]
   alignas(128) BStage st[kBStages];
   alignas(128) unsigned char neg1[kPM * 32];  // A operand of all -1 (s8): D = -sum(a) before the digits' MMA
   float xch[2][64][kPN + 1];  // the tile's gate and up results, [row][pair], for the epilogue
@@ -183,6 +184,12 @@ template <bool kGU>
 __device__ __forceinline__ const uint16_t* panel_scales(const DecodeParams& P, int p) {
   return kGU ? (p < 2 ? P.gate_scales : P.up_scales) : P.down_scales;
 }
+template <bool kGU>
+__device__ __forceinline__ const uint32_t* panel_codes(const DecodeParams& P, int p) {
+  return kGU ? (p < 2 ? P.gate_codes : P.up_codes) : P.down_codes;
+}
+// Packed words per 256-weight block of a 32-row panel, by weight format.
+__host__ __device__ constexpr int pf_words(int fmt) { return fmt == MOE_FORMAT_SIGN ? kSignWords : kBlockWords; }
 
 // The gate/up epilogue's output for pairs [n0, n0 + kNP) at ffn row f of a
 // tile: each lane (32 consecutive f, one 32-block) requantizes the SwiGLU
@@ -225,9 +232,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Pr
   return false;
 }
 
-// kDbg: the test hook's instantiation, which also writes the exact block sums.
-template <bool kGU, bool kDbg>
+// kFmt: the weights' format (MOE_FORMAT_*); kDbg: the test hook's
+// instantiation, which also writes the exact block sums.
+template <int kFmt, bool kGU, bool kDbg>
 __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
+  constexpr bool kE16 = kFmt == MOE_FORMAT_E16, kSgn = kFmt == MOE_FORMAT_SIGN;
+  constexpr int kWords = pf_words(kFmt);
   pdl_enter();
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(smem_raw);
@@ -280,19 +290,46 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       for (int b = 0; b < nb; ++b, ++wi) {
         const int ws = wi % kWStages, a = wi % kAStages;
         if (!wait_or_abort(&S.w_full[ws], (wi / kWStages) & 1u, S, P.status)) { ok = false; break; }
-        uint32_t w[kBlockWords];
+        uint32_t w[kWords], cw[kE16Words];
 #pragma unroll
-        for (int j = 0; j < kBlockWords; ++j) w[j] = S.w[ws][warp][j * kPanel + lane];
+        for (int j = 0; j < kWords; ++j) w[j] = S.w[ws][warp][j * kPanel + lane];
+        if (kE16) {
+#pragma unroll
+          for (int u = 0; u < kE16Words; ++u) cw[u] = S.wc[ws][warp][u * kPanel + lane];
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.w_empty[ws]);
         if (!wait_or_abort(&S.a_empty[a], ((wi / kAStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t w7[7], dg[32];
+          // digit word c (weights 4c..4c+3 of the block) into column 32h + c
+          uint32_t dg[32];
+          if (kSgn) {
+            // sign bits: word j holds weights 32j + 4i + l in bit 8l + i; the
+            // digit byte is 2t (t = the bit), so that with the -1 MMA the sum
+            // is sum((2t - 1) * a) = sum(q * a)
 #pragma unroll
-          for (int jj = 0; jj < 7; ++jj) w7[jj] = w[6 * h + jj];
-          if (h == 0) digit_half<0>(w7, dg);
-          else digit_half<1>(w7, dg);
+            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dg[8 * jj + i] = ((w[4 * h + jj] >> i) & 0x01010101u) << 1;
+          } else {
+            uint32_t w7[7];
+#pragma unroll
+            for (int jj = 0; jj < 7; ++jj) w7[jj] = w[6 * h + jj];
+            if (h == 0) digit_half<0>(w7, dg);
+            else digit_half<1>(w7, dg);
+            if (kE16) {
+              // two-level scales: the signed byte q * (c + 1) of the weight's
+              // 16-block (t * (c + 1) + 0x80 - (c + 1) stays in [0x70, 0x90]
+              // per byte, so no carry crosses a byte; the xor makes it s8)
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                const int hb = (32 * h + c) >> 2;
+                const uint32_t m1 = ((cw[hb >> 3] >> (4 * (hb & 7))) & 15u) + 1u;
+                dg[c] = (dg[c] * m1 + (0x80u - m1) * 0x01010101u) ^ 0x80808080u;
+              }
+            }
+          }
           tmem_st32(tlane + kAcol + 64 * a + 32 * h, dg);
         }
         tc_wait_st();
@@ -325,11 +362,16 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
       float y[kFixPairs];
 #pragma unroll
       for (int n = 0; n < kFixPairs; ++n) y[n] = 0.f;
+      // two-level scales: the row's anchor A / 16 takes the place of the
+      // block scale (y = sum over blocks of fma(A/16, inner, y))
+      const float a16 = kE16 ? __fmul_rn(f16_bits_to_f32(panel_scales<kGU>(P, q)[tile_panel_index<kGU>(P, T, q) *
+                                                                                kPanel + lane]), 0.0625f)
+                             : 0.f;
       for (int b = 0; b < nb && ok; ++b, ++bi) {
         // the row's block scale from the weight stage of this block
         const int ws = bi % kWStages;
         if (!wait_or_abort(&S.w_full[ws], (bi / kWStages) & 1u, S, P.status)) { ok = false; break; }
-        const float sw = f16_bits_to_f32(S.wsc[ws][q][lane]);
+        const float sw = kE16 ? a16 : f16_bits_to_f32(S.wsc[ws][q][lane]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.w_empty[ws]);
         const int bs = bi % kBStages;
@@ -443,22 +485,29 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
     TileInfo T;
     for (int t = blockIdx.x; ok && tile_info(P, t, m_tiles, T); t += gridDim.x) {
       if (T.it.expert < 0) continue;
+      // per block and panel: the packed words, then the fp16 block scales
+      // (two-level scales: the 4-bit code words; the anchors are per row)
+      constexpr uint32_t kWBytes = kWords * kPanel * 4;
+      constexpr uint32_t kSBytes = kE16 ? kE16Words * kPanel * 4 : kPanel * 2;
       const uint32_t* src[4];
-      const uint16_t* ssrc[4];
+      const void* ssrc[4];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        src[p] = panel_trits<kGU>(P, p) + tile_panel_index<kGU>(P, T, p) * nb * kBlockWords * kPanel;
-        ssrc[p] = panel_scales<kGU>(P, p) + tile_panel_index<kGU>(P, T, p) * nb * kPanel;
+        const size_t pi = tile_panel_index<kGU>(P, T, p);
+        src[p] = panel_trits<kGU>(P, p) + pi * nb * kWords * kPanel;
+        if (kE16) ssrc[p] = panel_codes<kGU>(P, p) + pi * nb * kE16Words * kPanel;
+        else ssrc[p] = panel_scales<kGU>(P, p) + pi * nb * kPanel;
       }
       for (int b = 0; b < nb; ++b, ++wi) {
         const int ws = wi % kWStages;
         if (!wait_or_abort(&S.w_empty[ws], ((wi / kWStages) & 1u) ^ 1u, S, P.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&S.w_full[ws], 4 * (kPanelBytes + kPanel * 2));
+        mbar_arrive_expect_tx(&S.w_full[ws], 4 * (kWBytes + kSBytes));
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          bulk_g2s(S.w[ws][p], src[p] + static_cast<size_t>(b) * kBlockWords * kPanel, kPanelBytes, &S.w_full[ws],
-                   pol);
-          bulk_g2s(S.wsc[ws][p], ssrc[p] + static_cast<size_t>(b) * kPanel, kPanel * 2, &S.w_full[ws], pol);
+          bulk_g2s(S.w[ws][p], src[p] + static_cast<size_t>(b) * kWords * kPanel, kWBytes, &S.w_full[ws], pol);
+          void* sdst = kE16 ? static_cast<void*>(S.wc[ws][p]) : static_cast<void*>(S.wsc[ws][p]);
+          bulk_g2s(sdst, static_cast<const unsigned char*>(ssrc[p]) + static_cast<size_t>(b) * kSBytes, kSBytes,
+                   &S.w_full[ws], pol);
         }
       }
     }
@@ -485,7 +534,7 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
   } else if (warp == kWMma && lane == 0) {
     // ------------------------------------------------ MMA issue
     const uint32_t idesc = idesc_i8(kPM, kPN);
-    const uint32_t idesc_neg = idesc_i8(kPM, kPN, true);
+    const uint32_t idesc_neg = idesc_i8(kPM, kPN, true);  // A signed
     const uint64_t ndesc = smem_desc(smem_u32(S.neg1), 128, 256);
     uint32_t bi = 0, si = 0;
     bool ok = true;
@@ -508,11 +557,17 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
 #pragma unroll
           for (int s2 = 0; s2 < kDSub; ++s2) {
             // onto the offset: -sum(a) (all -1 A operand), then sum(t * a)
+            // (sign codes: sum(2t * a)); two-level scales: the signed bytes
+            // q * (c + 1) in one MMA
             const int s = kDSub * h + s2;
             const uint32_t dcol = tbase + kDcol + kDSub * kPN * ds + kPN * s2;
             const uint64_t bsub = bdesc + static_cast<uint64_t>((s * kPN * 32) >> 4);
-            mma_i8_ss(dcol, ndesc, bsub, idesc_neg, true);
-            mma_i8_ts(dcol, tbase + kAcol + 64 * a + 8 * s, bsub, idesc, true);
+            if (kE16) {
+              mma_i8_ts(dcol, tbase + kAcol + 64 * a + 8 * s, bsub, idesc_neg, true);
+            } else {
+              mma_i8_ss(dcol, ndesc, bsub, idesc_neg, true);
+              mma_i8_ts(dcol, tbase + kAcol + 64 * a + 8 * s, bsub, idesc, true);
+            }
           }
           mma_commit(&S.d_full[ds]);
         }
@@ -563,35 +618,47 @@ static size_t prefill_smem() {
 
 size_t prefill_block_bytes() { return kBTile; }
 int prefill_group_pairs() { return kPN; }
-bool prefill_tc_supported(const DecodeParams& P) { return P.format == MOE_FORMAT_TERNARY; }
+bool prefill_tc_supported(const DecodeParams& P) {
+  return P.format == MOE_FORMAT_TERNARY || P.format == MOE_FORMAT_SIGN || P.format == MOE_FORMAT_E16;
+}
+
+// The gate/up and down GEMM launches of one weight format.
+template <int kFmt>
+static void launch_gemms(const DecodeParams& P, bool dbg, int dev, int n_sm, cudaStream_t stream) {
+  static std::atomic<bool> attrs_done[64];  // the attribute calls are idempotent
+  if (dev >= 0 && dev < 64 && !attrs_done[dev].load(std::memory_order_relaxed)) {
+    cudaFuncSetAttribute(k_prefill_mma<kFmt, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<kFmt, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<kFmt, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_prefill_mma<kFmt, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    attrs_done[dev].store(true, std::memory_order_relaxed);
+  }
+  const size_t smem = prefill_smem();
+  launch_k(dbg ? k_prefill_mma<kFmt, true, true> : k_prefill_mma<kFmt, true, false>, dim3(n_sm), dim3(kPThreads), smem,
+           stream, P);
+  note_launch(MOE_K_PREFILL_GATEUP, stream);
+  launch_k(dbg ? k_prefill_mma<kFmt, false, true> : k_prefill_mma<kFmt, false, false>, dim3(n_sm), dim3(kPThreads),
+           smem, stream, P);
+  note_launch(MOE_K_PREFILL_DOWN, stream);
+}
 
 int launch_prefill(const DecodeParams& P0, cudaStream_t stream) {
   DecodeParams P = P0;
   P.direct = 0;
   P.group_chunk = kPN;
+  if (!prefill_tc_supported(P)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "prefill: weight format %d", P.format);
   int rc = launch_group(P, stream);
   if (rc) return rc;
-  static std::atomic<bool> attrs_done[64];  // the attribute calls are idempotent
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attrs_done[dev].load(std::memory_order_relaxed)) {
-    cudaFuncSetAttribute(k_prefill_mma<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_prefill_mma<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_prefill_mma<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_prefill_mma<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    attrs_done[dev].store(true, std::memory_order_relaxed);
-  }
   int n_sm = 148;
   cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-  const size_t smem = prefill_smem();
   launch_k(k_prefill_gather, dim3(4 * n_sm), dim3(kPN * kSubPerBlock), 0, stream, P);
   note_launch(MOE_K_PREFILL_GATHER, stream);
   const bool dbg = P.dbg_isum_gu != nullptr;
-  launch_k(dbg ? k_prefill_mma<true, true> : k_prefill_mma<true, false>, dim3(n_sm), dim3(kPThreads), smem, stream, P);
-  note_launch(MOE_K_PREFILL_GATEUP, stream);
-  launch_k(dbg ? k_prefill_mma<false, true> : k_prefill_mma<false, false>, dim3(n_sm), dim3(kPThreads), smem, stream,
-           P);
-  note_launch(MOE_K_PREFILL_DOWN, stream);
+  if (P.format == MOE_FORMAT_SIGN) launch_gemms<MOE_FORMAT_SIGN>(P, dbg, dev, n_sm, stream);
+  else if (P.format == MOE_FORMAT_E16) launch_gemms<MOE_FORMAT_E16>(P, dbg, dev, n_sm, stream);
+  else launch_gemms<MOE_FORMAT_TERNARY>(P, dbg, dev, n_sm, stream);
   launch_k(k_combine, dim3(4 * n_sm), dim3(256), 0, stream, P);
   note_launch(MOE_K_COMBINE, stream);
   return check_launch("expert_ffn_prefill");

@@ -109,9 +109,10 @@ typedef struct {
  * (k = hidden) and rows [e*hidden, (e+1)*hidden) of down (k = ffn).  The
  * three matrices share one format.  Limits: hidden and ffn multiples of 256,
  * hidden <= 16384, ffn <= 8192, 1 <= top_k <= min(n_experts, 32),
- * n_experts <= 1024.  Sign-code and E16 layers run the decode path only: up
- * to 64 tokens per call (moe_expert_ffn_prefill, and moe_forward of more than
- * 64 tokens, return MOE_ERR_UNSUPPORTED_SHAPE for them).                   */
+ * n_experts <= 1024.  All three formats run the decode path (up to 64
+ * tokens) and the prefill GEMM (moe_expert_ffn_prefill, moe_forward of more
+ * than 64 tokens); the one-token fused step is ternary only (other formats
+ * take the four-kernel decode chain for one token).                       */
 typedef struct {
   int32_t hidden, ffn, n_experts, top_k;
   moe_tmat gate, up, down;
@@ -217,7 +218,8 @@ int moe_expert_ffn_decode_static(const moe_layer* layer, int32_t ntok, const int
  *      large batches take a GEMM path over the quantized tiles) -----------
  * Same result as moe_expert_ffn_decode for any ntok >= 1 (up to rounding
  * order), computed by grouping the (token, slot) pairs by expert and running
- * an int8 tensor-core grouped GEMM.  ntok <= 65536.                       */
+ * an int8 tensor-core grouped GEMM (exact int32 block sums; ternary, sign
+ * codes and two-level scales).  ntok <= 65536.                             */
 int moe_expert_ffn_prefill(const moe_layer* layer, int32_t ntok, const int8_t* xq,
                            const float* xd, const int32_t* idx, const float* wts, float* y,
                            void* ws, size_t ws_bytes, moe_stream_t stream);
@@ -306,9 +308,11 @@ int moe_debug_matvec(const moe_tmat* m, int32_t ntok, const int8_t* xq, const fl
  * README, "How it works": int8 x quantized-block products).  Runs the expert
  * FFN of moe_expert_ffn_decode (prefill == 0: the grouped tensor-core
  * mat-vecs, any ntok <= 64, ternary layers with hidden and ffn <= 4096) or of
- * moe_expert_ffn_prefill (prefill != 0: the grouped tensor-core GEMM) with
- * the same arguments, and also writes, for every (token, slot) pair
- * p = t * top_k + j, row and 32-value block s, the exact sum(q * a):
+ * moe_expert_ffn_prefill (prefill != 0: the grouped tensor-core GEMM, any of
+ * the three formats) with the same arguments, and also writes, for every
+ * (token, slot) pair p = t * top_k + j, row and 32-value block s, the exact
+ * sum(q * a) (two-level scales: sum over the block's two 16-weight halves h
+ * of (c_h + 1) * sum_{k in h} q * a):
  *   isum_gu [p][2][ffn][hidden/32]   gate (index 0) and up (index 1) rows
  *                                    against the pair's token's codes xq;
  *   isum_dn [p][hidden][ffn/32]      down rows against the pair's int8

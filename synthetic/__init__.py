@@ -95,6 +95,11 @@ WORKLOADS = {
     # prefill of 2048 tokens through the 30B-class layer
     "30b-prefill": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 2048, 0.02,
                             layers=1, prefill=True, seed=4),
+    # the same prefill on 1-bit sign codes and on two-level (E16) scales
+    "30b-sign-prefill": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 2048, 0.02,
+                                 layers=1, prefill=True, seed=9, fmt="sign"),
+    "30b-e16-prefill": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 2048, 0.02,
+                                layers=1, prefill=True, seed=10, fmt="e16"),
 }
 
 

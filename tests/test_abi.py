@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -100,7 +101,11 @@ def test_shared_expert_host_side_without_device():
     assert L.moe_quantize_weights_q8(p, 4, 48, p, p, None) == -2
 
 
-def test_forward_host_refuses_long_non_ternary_calls_before_any_launch():
+@pytest.mark.skipif(torch.cuda.is_available(), reason="would launch kernels on the placeholder pointers")
+def test_forward_host_long_sign_call_passes_the_format_checks():
+    """A 65-token call on a sign-code layer takes the prefill GEMM: its
+    arguments pass the host checks and the call stops only at the device
+    check (no CUDA device here), having launched nothing."""
     B, L = _lib()
     buf = (ctypes.c_uint8 * 64)()
     p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
@@ -110,5 +115,6 @@ def test_forward_host_refuses_long_non_ternary_calls_before_any_launch():
     lay = B.moe_layer(256, 256, 2, 1, tm(512, 256, 1), tm(512, 256, 1), tm(512, 256, 1))
     n0 = L.moe_launch_count()
     rc = L.moe_forward_host(ctypes.byref(lay), p, 65, p, p, p, 1 << 30, None)
-    assert rc == -2 and b"64 tokens" in L.moe_last_error()
+    assert rc in (-5, -8), L.moe_last_error()  # no usable device on this machine
+    assert b"64 tokens" not in L.moe_last_error()
     assert L.moe_launch_count() == n0

@@ -1,8 +1,8 @@
 """Parity of the 1-bit sign-code format (MOE_FORMAT_SIGN) on the CUDA path
 with the CPU oracle: packed codes and scales bit-exact, int32 block sums
 bit-exact, mat-vec outputs within 1e-5 of max(|ref|, RMS(ref)) elementwise,
-layer outputs within 2e-3 * RMS(ref); the shapes the format does not run
-(prefill) are refused before any launch."""
+layer outputs within 2e-3 * RMS(ref) (the prefill GEMM on this format:
+test_gpu_prefill_formats.py)."""
 import numpy as np
 import pytest
 import torch
@@ -121,10 +121,10 @@ def test_sign_batch_equals_single_tokens():
         assert np.array_equal(ys[0], yb[t])
 
 
-def test_sign_decode_entry_point_and_refusals(orc):
+def test_sign_decode_entry_point(orc):
     """moe_expert_ffn_decode on a sign-code layer (1 and 4 tokens) equals
-    moe_forward's routing of the same tokens; the prefill entry point and a
-    65-token forward are refused."""
+    moe_forward's routing of the same tokens (the prefill GEMM on this format
+    is tested in test_gpu_prefill_formats.py)."""
     B = bm()
     wl = synthetic.WORKLOADS["tiny"]
     layer, _ = gpu_layer(wl, fmt="sign")
@@ -138,15 +138,3 @@ def test_sign_decode_entry_point_and_refusals(orc):
         yd = B.moe_expert_ffn_decode(layer, xq, xd, idx, wts, ws).cpu().numpy()
         assert B.moe_check_status(ws) == 0
         assert np.array_equal(yf, yd)
-    x = synthetic.activations(wl, 35, ntok=65, device="cuda")
-    ws = B.Workspace.for_layer(layer, 65, prefill=True)
-    n0 = B.moe_launch_count()
-    with pytest.raises(B.MoEError):
-        B.moe_forward(layer, wr, x, ws)
-    assert B.moe_launch_count() == n0
-    xq, xd = B.moe_quant_act_q8(x)
-    idx, wts = B.moe_route_topk(x, wr, wl.top_k)
-    n1 = B.moe_launch_count()
-    with pytest.raises(B.MoEError):
-        B.moe_expert_ffn_prefill(layer, xq, xd, idx, wts, ws)
-    assert B.moe_launch_count() == n1
