@@ -545,12 +545,22 @@ def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do
                   "launches": len(v)} for n, v in per_kernel.items()}
     dom = max(shares, key=lambda n: shares[n]["share"])
     peak, peak_kind = measured_peaks()
-    avg_s = shares[dom]["avg_us"] / 1e6
+    eager_s = shares[dom]["avg_us"] / 1e6
+    if launches_per_step == 1 and len(shares) == 1:
+        # one kernel per step: its average launch duration is the timed
+        # region's time over its launches (the replayed launches overlap a
+        # launch's start with the previous one's end, which the eager,
+        # event-separated timing above does not)
+        avg_s, dur_src = ms / 1e3 / steps, "timed region / launches"
+    else:
+        avg_s, dur_src = eager_s, "events around each launch, launched back to back"
     achieved = kb.get(dom, 0) / avg_s / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
                 "algorithmic_bytes_per_launch": kb.get(dom, 0),
-                "traffic": ncu_traffic(dom, wl.describe())}
+                "traffic": ncu_traffic(dom, wl.describe()),
+                "launch_us": avg_s * 1e6, "launch_us_source": dur_src,
+                "achieved_event_timed": kb.get(dom, 0) / eager_s / 1e9}
     step_bytes = sum(kb[n] for n in kb if n in shares)
     step_s = ms / 1e3 / steps
     res = {"workload": wl.describe(), "tokens_per_step": T, "steps": steps, "warmup": warmup,
