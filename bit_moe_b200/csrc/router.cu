@@ -51,19 +51,18 @@ constexpr int kRtT = 16, kRtKC = 256;
 // 1024 wide (two stages of 80 KB) to cut the number of copy round trips.
 constexpr int kRtKCWide = 1024;
 
-// kWE warps along the experts (8 / kWE along the tokens); a lane holds a
-// micro-tile of kMT tokens x kME experts: the CTA tile is 16 tokens x
-// kWE*kME experts.
+// kW warps per CTA, kWE of them along the experts (kW / kWE along the
+// tokens); a lane holds a micro-tile of kMT tokens x kME experts: the CTA
+// tile is (kW / kWE) * kMT tokens x kWE * kME experts.
 // With xq non-null the CTAs also quantize x to int8 32-blocks, the blocks
 // dealt round-robin over all warps of the grid (as k_quant_act_q8 does).
-template <int kWE, int kMT, int kME, int kKC>
-__global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __restrict__ x,
-                                                             const float* __restrict__ wr, int ntok, int H,
-                                                             int E, float* __restrict__ logits,
-                                                             int8_t* __restrict__ xq, float* __restrict__ xd) {
+template <int kW, int kWE, int kMT, int kME, int kKC>
+__global__ void __launch_bounds__(kW * 32) k_router_logits_tiled(const float* __restrict__ x,
+                                                                 const float* __restrict__ wr, int ntok, int H,
+                                                                 int E, float* __restrict__ logits,
+                                                                 int8_t* __restrict__ xq, float* __restrict__ xd) {
   pdl_enter();
-  constexpr int kRtMT = kMT, kRtME = kME, kRtE = kWE * kME;
-  static_assert((8 / kWE) * kMT == kRtT, "16 tokens per tile");
+  constexpr int kRtMT = kMT, kRtME = kME, kRtE = kWE * kME, kRtT = (kW / kWE) * kMT;
   extern __shared__ __align__(16) float rsm[];
   float* xs = rsm;                        // [2][kRtT][kKC]
   float* ws = rsm + 2 * kRtT * kKC;     // [2][kRtE][kKC]
@@ -73,8 +72,8 @@ __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __rest
   const int we = (warp % kWE) * kRtME;    // warp's first expert in the tile
   const int nchunk = H / kKC;
   auto stage = [&](int ch, int buf) {
-    // (kRtT + kRtE) rows x 256 floats = 2048 chunks of 16 bytes, 8 per thread
-    for (int c = tid; c < (kRtT + kRtE) * (kKC / 4); c += 256) {
+    // (kRtT + kRtE) rows x kKC floats in chunks of 16 bytes
+    for (int c = tid; c < (kRtT + kRtE) * (kKC / 4); c += kW * 32) {
       const int row = c / (kKC / 4), q = c % (kKC / 4);
       const bool isx = row < kRtT;
       const int r = isx ? row : row - kRtT;
@@ -97,8 +96,8 @@ __global__ void __launch_bounds__(256) k_router_logits_tiled(const float* __rest
   stage(0, 0);
   if (xq) {
     const int64_t nblk = static_cast<int64_t>(ntok) * (H / kQBlock);
-    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * gridDim.y * 8;
-    for (int64_t blk = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * 8 + warp; blk < nblk;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * gridDim.y * kW;
+    for (int64_t blk = (static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x) * kW + warp; blk < nblk;
          blk += nwarps)
       quant_act_block(x, blk, lane, xq, xd);
   }
@@ -170,11 +169,12 @@ __global__ void k_topk_softmax(const float* __restrict__ logits, int ntok, int E
   }
 }
 
-template <int kWE, int kMT, int kME, int kKC = kRtKC>
+template <int kWE, int kMT, int kME, int kKC = kRtKC, int kW = 8>
 static void launch_tiled(const float* x, const float* wr, int ntok, int H, int E, float* logits,
                          cudaStream_t stream, int8_t* xq = nullptr, float* xd = nullptr) {
-  auto kern = k_router_logits_tiled<kWE, kMT, kME, kKC>;
-  const size_t smem = sizeof(float) * 2 * (kRtT + kWE * kME) * kKC;
+  auto kern = k_router_logits_tiled<kW, kWE, kMT, kME, kKC>;
+  constexpr int kT = (kW / kWE) * kMT;
+  const size_t smem = sizeof(float) * 2 * (kT + kWE * kME) * kKC;
   static std::atomic<bool> attr_done[64];  // the attribute call is idempotent
   int dev = 0;
   cudaGetDevice(&dev);
@@ -182,8 +182,8 @@ static void launch_tiled(const float* x, const float* wr, int ntok, int H, int E
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     attr_done[dev].store(true, std::memory_order_relaxed);
   }
-  const dim3 grid((ntok + kRtT - 1) / kRtT, (E + kWE * kME - 1) / (kWE * kME));
-  launch_k(kern, grid, dim3(256), smem, stream, x, wr, ntok, H, E, logits, xq, xd);
+  const dim3 grid((ntok + kT - 1) / kT, (E + kWE * kME - 1) / (kWE * kME));
+  launch_k(kern, grid, dim3(kW * 32), smem, stream, x, wr, ntok, H, E, logits, xq, xd);
 }
 
 int launch_router_logits(const float* x, const float* wr, int ntok, int H, int E, float* logits,
@@ -194,9 +194,10 @@ int launch_router_logits(const float* x, const float* wr, int ntok, int H, int E
     if (grid > 148 * 16) grid = 148 * 16;
     launch_k(k_router_logits, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream, x, wr, ntok, H, E, logits);
   } else if (ntok >= 4 * kRtT && E >= 64) {
-    // 16 tokens x 32 experts: an 8 x 8 micro-tile per lane, 16 shared-memory
-    // loads per 64 fused multiply-adds
-    launch_tiled<4, 8, 8>(x, wr, ntok, H, E, logits, stream);
+    // 32 tokens x 32 experts on 16 warps: an 8 x 8 micro-tile per lane (16
+    // shared-memory loads per 64 fused multiply-adds), each staged row used
+    // by 32 logits
+    launch_tiled<4, 8, 8, kRtKC, 16>(x, wr, ntok, H, E, logits, stream);
   } else if (ntok >= 4 * kRtT) {
     launch_tiled<4, 8, 4>(x, wr, ntok, H, E, logits, stream);  // 16 x 16 tiles
   } else if (H % kRtKCWide == 0) {

@@ -116,7 +116,7 @@ def test_matvec_extreme_codes(orc):
 # ------------------------------------------------------------------ S2 router
 @pytest.mark.parametrize("ntok,H,E,K", [(1, 256, 8, 2), (16, 2048, 128, 8), (200, 2048, 128, 8),
                                         (3, 4096, 256, 8), (4, 512, 32, 32), (5, 256, 64, 1),
-                                        (37, 512, 40, 4), (6, 256, 600, 8)])
+                                        (37, 512, 40, 4), (6, 256, 600, 8), (70, 256, 100, 4)])
 def test_router_exact_ids(orc, ntok, H, E, K):
     B = bm()
     g = np.random.default_rng(ntok * 1000 + E)
