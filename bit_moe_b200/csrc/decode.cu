@@ -46,7 +46,9 @@ size_t group_ws_layout(int E, int npairs, size_t off, GroupWs* G) {
 // ---------------------------------------------------------------------------
 constexpr int kGroupThreads = 1024;
 
-__device__ __forceinline__ void group_body(const DecodeParams& P) {
+// sidx: the pairs' expert ids in shared memory where the caller has them
+// (else they are read from P.idx).
+__device__ __forceinline__ void group_body(const DecodeParams& P, const int* sidx = nullptr) {
   using Scan = cub::BlockScan<int, kGroupThreads>;
   __shared__ typename Scan::TempStorage scan_tmp;
   __shared__ int cnt[kMaxExperts + 1];
@@ -56,7 +58,7 @@ __device__ __forceinline__ void group_body(const DecodeParams& P) {
   for (int e = tid; e <= E; e += kGroupThreads) { cnt[e] = 0; fill[e] = 0; }
   __syncthreads();
   for (int p = tid; p < npairs; p += kGroupThreads) {
-    int e = __ldcg(P.idx + p);
+    int e = sidx ? sidx[p] : __ldcg(P.idx + p);
     if (e < 0 || e >= E) { record_status(P.status, MOE_ERR_BAD_INDEX); e = E; }
     atomicAdd(&cnt[e], 1);
   }
@@ -92,7 +94,7 @@ __device__ __forceinline__ void group_body(const DecodeParams& P) {
   __syncthreads();
   int32_t* pairs = const_cast<int32_t*>(P.pairs);
   for (int p = tid; p < npairs; p += kGroupThreads) {
-    int e = __ldcg(P.idx + p);
+    int e = sidx ? sidx[p] : __ldcg(P.idx + p);
     if (e < 0 || e >= E) e = E;
     pairs[off[e] + atomicAdd(&fill[e], 1)] = p;
   }
@@ -110,6 +112,7 @@ template <int kPer>
 __global__ void __launch_bounds__(kGroupThreads) k_topk_group(DecodeParams P, const float* __restrict__ logits,
                                                               float* __restrict__ wts) {
   pdl_enter();
+  __shared__ int sidx[kMaxDecodeTokens * kMaxTopK];  // the ids again for the grouping
   const int lane = threadIdx.x & 31;
   const int E = P.n_experts, K = P.top_k;
   for (int t = threadIdx.x >> 5; t < P.ntok; t += kGroupThreads / 32) {
@@ -129,11 +132,12 @@ __global__ void __launch_bounds__(kGroupThreads) k_topk_group(DecodeParams P, co
     warp_topk_softmax<kPer>(key, need, K, lane, my_e, w);
     if (lane < K) {
       const_cast<int32_t*>(P.idx)[static_cast<int64_t>(t) * K + lane] = my_e;
+      sidx[t * K + lane] = my_e;
       wts[static_cast<int64_t>(t) * K + lane] = w;
     }
   }
   __syncthreads();
-  group_body(P);
+  group_body(P, sidx);
 }
 
 // ---------------------------------------------------------------------------
