@@ -105,11 +105,11 @@ def kernel_bytes(wl, unique_experts):
     # the tensor-core mat-vecs move the same bytes as the CUDA-core ones
     kb["tc_gateup"], kb["tc_down"] = kb["gateup"], kb["down"]
     if wl.shared_ffn:
-        # the shared expert's three kernels (gate/up, requantization, down with
-        # the add into y), per launch on average: 8-bit codes plus an fp16 scale
-        # per 32 weights, activations in and out
+        # the shared expert's two kernels (gate/up with the requantization,
+        # down with the add into y), per launch on average: 8-bit codes plus
+        # an fp16 scale per 32 weights, activations in and out
         Fs = wl.shared_ffn
-        kb["shared"] = (3 * H * Fs * 34 // 32 + T * H * 2 + T * Fs * 6 + T * H * 8) / 3
+        kb["shared"] = (3 * H * Fs * 34 // 32 + T * H * 5 // 4 + T * Fs * 5 // 2 + T * H * 8) / 2
     return kb
 
 
@@ -450,19 +450,17 @@ def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
     shared = build_shared(B, wl, L, dev, seed_off) if wl.shared_ffn else None
     if shared:
-        sxq = torch.empty((T, H), dtype=torch.int8, device=dev)
-        sxd = torch.empty((T, H // 32), dtype=torch.float32, device=dev)
+        # x's int8 codes and scales that moe_forward leaves in its workspace
+        sxq, sxd = ws.act(layers[0], T)
         sws = shared[0].workspace(T, dev)
     torch.cuda.synchronize()
 
     def step(j):
         B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
         if shared:
-            # the shared expert's FFN added to y: x^ again (the step's own copy
-            # stays inside the fused kernels), then the 8-bit gate/up, the
-            # requantization and the down mat-vec with the add
-            B.lib().moe_quant_act_q8(xs[j % NX].data_ptr(), T, H, sxq.data_ptr(), sxd.data_ptr(),
-                                     torch.cuda.current_stream().cuda_stream)
+            # the shared expert's FFN added to y, from the x^ of the step: the
+            # 8-bit gate/up with the requantization, then the down mat-vec
+            # with the add
             shared[j % L].add(sxq, sxd, y, ws=sws)
 
     for j in range(warmup):

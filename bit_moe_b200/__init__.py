@@ -37,7 +37,7 @@ EXPORTS = (
     "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
     "moe_sign_words", "moe_quantize_weights_sign", "moe_e16_code_words", "moe_quantize_weights_e16",
     "moe_quantize_weights_q8", "moe_shared_workspace_bytes", "moe_shared_ffn_add",
-    "moe_debug_ffn_blocksums", "moe_debug_wait_knob",
+    "moe_debug_ffn_blocksums", "moe_debug_wait_knob", "moe_workspace_act",
 )
 
 
@@ -119,6 +119,7 @@ def load_library(path):
         "moe_expert_ffn_decode_static": (ctypes.c_int, [p, i32, p, p, p, p, p, p]),
         "moe_debug_ffn_blocksums": (ctypes.c_int, [p, i32, p, p, p, p, p, p, sz, i32, p, p, p, p]),
         "moe_debug_wait_knob": (ctypes.c_int, [p, sz, i32, i32, p]),
+        "moe_workspace_act": (ctypes.c_int, [p, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -316,6 +317,18 @@ class Workspace:
 
     def ptr(self):
         return ctypes.c_void_p(self.buf.data_ptr())
+
+    def act(self, layer, ntok, prefill=None):
+        """Views of x's int8 codes [ntok][hidden] and fp32 scales
+        [ntok][hidden/32] that moe_forward left in this workspace."""
+        if prefill is None:
+            prefill = ntok > MAX_DECODE_TOKENS
+        oq, od = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        _check(lib().moe_workspace_act(layer.c_ref(), ntok, int(bool(prefill)), ctypes.byref(oq), ctypes.byref(od)))
+        H = layer.hidden
+        xq = self.buf[oq.value:oq.value + ntok * H].view(torch.int8).view(ntok, H)
+        xd = self.buf[od.value:od.value + ntok * (H // QBLOCK) * 4].view(torch.float32).view(ntok, H // QBLOCK)
+        return xq, xd
 
 
 # ---------------------------------------------------------------- the path

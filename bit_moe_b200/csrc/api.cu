@@ -318,6 +318,16 @@ size_t moe_workspace_bytes(const moe_layer* L, int32_t ntok, int32_t prefill) {
   return ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill != 0).total;
 }
 
+int moe_workspace_act(const moe_layer* L, int32_t ntok, int32_t prefill, size_t* xq_offset, size_t* xd_offset) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if (ntok <= 0 || !xq_offset || !xd_offset) return fail(MOE_ERR_INVALID_ARG, "workspace_act: ntok > 0, offsets");
+  const WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill != 0);
+  *xq_offset = W.xq;
+  *xd_offset = W.xd;
+  return MOE_OK;
+}
+
 size_t moe_route_workspace_bytes(int32_t ntok, int32_t n_experts) {
   if (ntok <= 0 || n_experts <= 0) return 0;
   return kWsHeaderBytes + align_up(sizeof(float) * static_cast<size_t>(ntok) * n_experts, 256);

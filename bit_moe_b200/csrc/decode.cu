@@ -183,7 +183,36 @@ __device__ __forceinline__ void gateup_run(const DecodeParams& P, const Item& it
     const uint32_t* const tc[2] = {P.gate_codes + pb0 * kE16Words * kPanel + lane,
                                    P.up_codes + pb0 * kE16Words * kPanel + lane};
     const float a16[2] = {f16_bits_to_f32(P.gate_scales[row]) * 0.0625f, f16_bits_to_f32(P.up_scales[row]) * 0.0625f};
-    panel_dot_e16<2, NT>(tw, tc, a16, warp, nb, kGateUpWarps, q4, d, out);
+    if constexpr (NT >= 4) {
+      // many vectors: gate, then up (each matrix's sums are independent, so
+      // the results are those of the joint pass, in fewer registers)
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t* const tw1[1] = {tw[m]};
+        const uint32_t* const tc1[1] = {tc[m]};
+        const float a1[1] = {a16[m]};
+        float o1[1][NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) o1[0][n] = 0.f;
+        panel_dot_e16<1, NT>(tw1, tc1, a1, warp, nb, kGateUpWarps, q4, d, o1);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) out[m][n] = o1[0][n];
+      }
+    } else {
+      panel_dot_e16<2, NT>(tw, tc, a16, warp, nb, kGateUpWarps, q4, d, out);
+    }
+  } else if constexpr (NT >= 4) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t* const tw1[1] = {tw[m]};
+      const uint16_t* const ts1[1] = {ts[m]};
+      float o1[1][NT];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) o1[0][n] = 0.f;
+      panel_dot<1, NT, kFmt == MOE_FORMAT_SIGN>(tw1, ts1, warp, nb, kGateUpWarps, q4, d, as, o1);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) out[m][n] = o1[0][n];
+    }
   } else {
     panel_dot<2, NT, kFmt == MOE_FORMAT_SIGN>(tw, ts, warp, nb, kGateUpWarps, q4, d, as, out);
   }

@@ -66,15 +66,23 @@ __device__ __forceinline__ float q8_row_dot(const int8_t* __restrict__ q, const 
   return acc;
 }
 
-// a[t][f] = silu(gate_f . x^_t) * (up_f . x^_t) for every token: one warp per
-// row f of the shared expert's ffn.
-__global__ void __launch_bounds__(kSharedWarps * 32) k_shared_gateup(SharedParams S, int ntok, const int8_t* __restrict__ xq,
-                                                                     const float* __restrict__ xd, float* __restrict__ a) {
+// a[t][f] = silu(gate_f . x^_t) * (up_f . x^_t) for every token and row f of
+// the shared ffn, requantized in the same kernel: a CTA of 32 warps takes one
+// 32-row block of the shared ffn (one row per warp), puts the block's a
+// values in shared memory, and one warp quantizes them (as the activation
+// quantization) into aq and ad, token by token.
+constexpr int kSharedBlockWarps = kQBlock;
+__global__ void __launch_bounds__(kSharedBlockWarps * 32) k_shared_gateup_q(SharedParams S, int ntok,
+                                                                            const int8_t* __restrict__ xq,
+                                                                            const float* __restrict__ xd,
+                                                                            int8_t* __restrict__ aq,
+                                                                            float* __restrict__ ad) {
   pdl_enter();
-  const int lane = threadIdx.x & 31;
+  __shared__ float sa[kQBlock];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int H = S.hidden, F = S.ffn;
-  const int nw = gridDim.x * kSharedWarps;
-  for (int f = blockIdx.x * kSharedWarps + (threadIdx.x >> 5); f < F; f += nw) {
+  for (int blk = blockIdx.x; blk < F / kQBlock; blk += gridDim.x) {
+    const int f = blk * kQBlock + warp;
     const int8_t* gq = S.gate_q + static_cast<size_t>(f) * H;
     const int8_t* uq = S.up_q + static_cast<size_t>(f) * H;
     const uint16_t* gd = S.gate_d + static_cast<size_t>(f) * (H / kQBlock);
@@ -84,20 +92,13 @@ __global__ void __launch_bounds__(kSharedWarps * 32) k_shared_gateup(SharedParam
       const float* dt = xd + static_cast<size_t>(t) * (H / kQBlock);
       const float g = q8_row_dot(gq, gd, H, xt, dt, lane);
       const float u = q8_row_dot(uq, ud, H, xt, dt, lane);
-      if (lane == 0) a[static_cast<size_t>(t) * F + f] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
+      if (lane == 0) sa[warp] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
+      __syncthreads();
+      if (warp == 0) quant_act_block(sa, 0, lane, aq + static_cast<size_t>(t) * F + blk * kQBlock,
+                                     ad + static_cast<size_t>(t) * (F / kQBlock) + blk);
+      __syncthreads();
     }
   }
-}
-
-// int8 32-blocks of a (as the activation quantization).
-__global__ void k_shared_quant(const float* __restrict__ a, int64_t nblk, int8_t* __restrict__ aq,
-                               float* __restrict__ ad) {
-  pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t blk = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); blk < nblk;
-       blk += nw)
-    quant_act_block(a, blk, lane, aq, ad);
 }
 
 // y[t][h] += down_h . a^_t: one warp per row h of hidden.
@@ -136,26 +137,18 @@ int launch_quantize_weights_q8(const float* w, int64_t rows, int64_t k, int8_t* 
 
 size_t shared_ws_bytes(int hidden, int ffn, int ntok) {
   (void)hidden;
-  const size_t a = align_up(sizeof(float) * static_cast<size_t>(ntok) * ffn, 256);
   const size_t aq = align_up(static_cast<size_t>(ntok) * ffn, 256);
   const size_t ad = align_up(sizeof(float) * static_cast<size_t>(ntok) * (ffn / kQBlock), 256);
-  return a + aq + ad;
+  return aq + ad;
 }
 
 int launch_shared_ffn_add(const SharedParams& S, int ntok, const int8_t* xq, const float* xd, float* y, void* ws,
                           cudaStream_t stream) {
   unsigned char* base = static_cast<unsigned char*>(ws);
-  float* a = reinterpret_cast<float*>(base);
-  int8_t* aq = reinterpret_cast<int8_t*>(base + align_up(sizeof(float) * static_cast<size_t>(ntok) * S.ffn, 256));
-  float* ad = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(aq) +
-                                       align_up(static_cast<size_t>(ntok) * S.ffn, 256));
-  launch_k(k_shared_gateup, dim3(rows_grid(S.ffn)), dim3(kSharedWarps * 32), 0, stream, S, ntok, xq, xd, a);
-  note_launch(MOE_K_SHARED, stream);
-  const int64_t nblk = static_cast<int64_t>(ntok) * (S.ffn / kQBlock);
-  int64_t g = (nblk + 7) / 8;
-  if (g > 148 * 8) g = 148 * 8;
-  launch_k(k_shared_quant, dim3(static_cast<unsigned>(g)), dim3(256), 0, stream, static_cast<const float*>(a), nblk,
-           aq, ad);
+  int8_t* aq = reinterpret_cast<int8_t*>(base);
+  float* ad = reinterpret_cast<float*>(base + align_up(static_cast<size_t>(ntok) * S.ffn, 256));
+  launch_k(k_shared_gateup_q, dim3(static_cast<unsigned>(S.ffn / kQBlock)), dim3(kSharedBlockWarps * 32), 0, stream,
+           S, ntok, xq, xd, aq, ad);
   note_launch(MOE_K_SHARED, stream);
   launch_k(k_shared_down_add, dim3(rows_grid(S.hidden)), dim3(kSharedWarps * 32), 0, stream, S, ntok,
            static_cast<const int8_t*>(aq), static_cast<const float*>(ad), y);

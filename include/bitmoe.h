@@ -126,6 +126,15 @@ size_t moe_scale_count(int64_t rows, int64_t k); /* rows*(k/256)    */
 /* Bytes of workspace a decode (prefill = 0) or prefill (prefill = 1) call
  * of `ntok` tokens, or moe_forward, needs.  0 on invalid arguments.        */
 size_t moe_workspace_bytes(const moe_layer* layer, int32_t ntok, int32_t prefill);
+/* Where a workspace of this layer (for `ntok` tokens, decode or prefill
+ * layout) holds the int8 codes [ntok][hidden] and fp32 scales
+ * [ntok][hidden/32] of x (S1, pxq_llama README, "PXQ vs MXFP4": one scale
+ * per 32-value block): byte offsets from the workspace's start.  Every
+ * moe_forward call writes them there (the same values moe_quant_act_q8
+ * gives), so a caller can hand them on, e.g. to moe_shared_ffn_add, without
+ * quantizing x again.  MOE_ERR_INVALID_ARG on a bad layer or ntok <= 0.    */
+int moe_workspace_act(const moe_layer* layer, int32_t ntok, int32_t prefill, size_t* xq_offset,
+                      size_t* xd_offset);
 /* Zero a workspace (status word and counters).  Every workspace must be
  * initialised once before its first use; calls leave it reusable.         */
 int moe_workspace_init(void* ws, size_t ws_bytes, moe_stream_t stream);

@@ -266,6 +266,23 @@ def test_batch_equals_single_tokens():
         assert np.array_equal(ys[0], yb[t])
 
 
+@pytest.mark.parametrize("fmt", ["ternary", "sign", "e16"])
+def test_full_items_equal_single_tokens(fmt):
+    """40 tokens through the tiny layer (8 experts, top-2): about 10 pairs per
+    expert, so the grouped mat-vecs run items of 8 vectors (gate and up in
+    two passes) beside the short ones; every token bit for bit equal to the
+    same token alone."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"]
+    layer, _ = gpu_layer(wl, fmt=fmt)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 19, ntok=40, device="cuda")
+    yb, _ = _run_forward(B, layer, wr, x)
+    for t in range(0, 40, 3):
+        ys, _ = _run_forward(B, layer, wr, x[t:t + 1].contiguous())
+        assert np.array_equal(ys[0], yb[t]), t
+
+
 def test_prefill_equals_decode():
     B = bm()
     wl = synthetic.WORKLOADS["30b"]

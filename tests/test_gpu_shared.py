@@ -70,3 +70,23 @@ def test_shared_expert_alone(orc):
     y = sh.add(xq, xd, torch.zeros((ntok, H), dtype=torch.float32, device="cuda")).cpu().numpy()
     ref = orc.SharedExpert(H, Fs, wg, wu, wd).add_to(np.zeros((ntok, H)), xq.cpu().numpy(), xd.cpu().numpy())
     assert rel_err_rms(y, ref) <= LAYER_TOL
+
+
+@pytest.mark.parametrize("wl_name,ntok", [("30b", 1), ("tiny", 1), ("30b", 5), ("tiny", 70)])
+def test_workspace_act_is_the_step_quantization(wl_name, ntok):
+    """moe_forward leaves x's int8 codes and scales in its workspace (the
+    one-token step, the batched decode and the prefill path each write them):
+    bit for bit those of moe_quant_act_q8, so the shared expert can take them
+    without quantizing x again."""
+    B = bm()
+    wl = synthetic.WORKLOADS[wl_name]
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 75 + ntok, ntok=ntok, device="cuda")
+    ws = B.Workspace.for_layer(layer, ntok)
+    B.moe_forward(layer, wr, x, ws)
+    assert B.moe_check_status(ws) == 0
+    wq, wd = ws.act(layer, ntok)
+    xq, xd = B.moe_quant_act_q8(x)
+    assert np.array_equal(wq.cpu().numpy(), xq.cpu().numpy())
+    assert np.array_equal(wd.cpu().numpy().view(np.uint32), xd.cpu().numpy().view(np.uint32))
