@@ -449,7 +449,10 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   if ((rc = check_ptrs("forward", w_router, x, y, ws))) return rc;
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
-  const bool sign = L->gate.format != MOE_FORMAT_TERNARY;  // sign codes or two-level scales
+  // layers whose one token does not take the fused one-token step: two-level
+  // scales, and sign codes of shapes the step does not fit (ternary layers
+  // of such shapes take the first-version one-token chain below)
+  bool chain1 = L->gate.format == MOE_FORMAT_E16;
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total) return fail(MOE_ERR_WORKSPACE, "forward: workspace %zu < %zu bytes", ws_bytes, W.total);
   if ((rc = check_device())) return rc;
@@ -461,8 +464,12 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   float* wts = reinterpret_cast<float*>(base + W.wts);
   float* logits = reinterpret_cast<float*>(base + W.logits);
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
-  if ((ntok > 1 || sign) && !prefill && router_quant_small_ok(ntok, L->hidden)) {
-    // few tokens (and one token of a sign-code or E16 layer): router logits with
+  if (ntok == 1 && L->gate.format == MOE_FORMAT_SIGN) {
+    size_t smem_s = 0;
+    chain1 = !step1_supported(P, sm_count(), &smem_s);
+  }
+  if ((ntok > 1 || chain1) && !prefill && router_quant_small_ok(ntok, L->hidden)) {
+    // few tokens (and one token of an E16 layer): router logits with
     // the activation quantization, then the top-k with the grouping, then
     // the grouped mat-vecs
     if ((rc = launch_router_quant_small(x, w_router, ntok, L->hidden, L->n_experts, logits, xq, xd, s)))
@@ -470,7 +477,7 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
     if ((rc = launch_topk_group(P, logits, wts, s))) return rc;
     return launch_ffn(P, s);
   }
-  if (ntok > 1 || sign) {
+  if (ntok > 1 || chain1) {
     if ((rc = launch_quant_act_q8(x, ntok, L->hidden, xq, xd, s))) return rc;
     if ((rc = launch_route_topk(x, w_router, ntok, L->hidden, L->n_experts, L->top_k, idx, wts, logits, s)))
       return rc;

@@ -225,6 +225,55 @@ __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc
   }
 }
 
+// The same for one vector over 1-bit sign codes (kSignWords words per
+// block, word j = activation block j, weight 32j + 4i + l in bit 8l + i):
+// per sub-block the exact sum(q * a) = 2 * sum(t * a) - sum(a), scaled and
+// accumulated in the order of the grouped sign-code kernels.  Matrix m's
+// words are at wsrc + m * mat_stride, its fp16 scales scale_off bytes further.
+template <int NM, bool kInner = false>
+__device__ __forceinline__ void block_dot_sign(const unsigned char* __restrict__ wsrc, int mat_stride, int scale_off,
+                                               const int* __restrict__ q4, const float* __restrict__ ds,
+                                               const int* __restrict__ as, int lane, float (&part)[NM][1],
+                                               float* sc_out = nullptr) {
+  uint32_t w[NM][kSignWords];
+  float sc[NM];
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const uint32_t* tw = reinterpret_cast<const uint32_t*>(wsrc + m * mat_stride);
+#pragma unroll
+    for (int j = 0; j < kSignWords; ++j) w[m][j] = tw[j * kPanel + lane];
+    sc[m] = f16_bits_to_f32(reinterpret_cast<const uint16_t*>(wsrc + m * mat_stride + scale_off)[lane]);
+  }
+  float inner[NM];
+#pragma unroll
+  for (int m = 0; m < NM; ++m) inner[m] = 0.f;
+#pragma unroll
+  for (int j = 0; j < kSignWords; ++j) {
+    int acc[NM];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) acc[m] = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int a = q4[8 * j + i];
+#pragma unroll
+      for (int m = 0; m < NM; ++m) acc[m] = __dp4a(static_cast<int>((w[m][j] >> i) & 0x01010101u), a, acc[m]);
+    }
+    const int an = as[j];
+    const float dn = ds[j];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) inner[m] = __fmaf_rn(dn, static_cast<float>(2 * acc[m] - an), inner[m]);
+  }
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    if constexpr (kInner) {
+      part[m][0] = inner[m];
+      sc_out[m] = sc[m];
+    } else {
+      part[m][0] = __fmaf_rn(sc[m], inner[m], part[m][0]);
+    }
+  }
+}
+
 // Dispatch on the number of pairs of the item (1, 2, 4 or 8 vectors).
 template <int NM, int NTMAX>
 __device__ __forceinline__ void block_dot_n(int count, const unsigned char* wsrc, const int* q4, int qs,

@@ -25,7 +25,11 @@
 // Parakon Runtime README, "How it works" (fused decode mat-vecs on the packed
 // blocks, int8 activations); llama-modchip page, "Key highlights" (all top-k
 // experts evaluated); pxq_llama README, "Updates -- 2026-07-28" (gate/up with
-// the SiLU unary).  The numerics are those of the decode kernels.
+// the SiLU unary).  The numerics are those of the decode kernels.  The same
+// kernel takes 1-bit sign codes (pxq_llama README, "What's PXQ?", the PXQ1
+// tier) with their block decode; two-level scales keep one fp32 chain over
+// every block of a down row, which phase C's split of the blocks over two
+// warps cannot reproduce, so they take the four-kernel chain.
 #include <atomic>
 #include "bitmoe.h"
 #include "common.cuh"
@@ -54,6 +58,11 @@ static_assert(kS1MaxK <= kNC, "phase C: one warp per slot");
 // and the int32 code sum.
 constexpr int kUnitWords = kPanel / 4 + 2;
 
+// Bytes of one 256-weight block of a 32-row panel: packed words, then the
+// 32 fp16 scales (base-3 digits, or 1-bit sign codes).
+__host__ __device__ constexpr int s1_word_bytes(bool sign) { return (sign ? kSignWords : kBlockWords) * kPanel * 4; }
+__host__ __device__ constexpr int s1_mat_bytes(bool sign) { return s1_word_bytes(sign) + kPanel * 2; }
+
 struct Step1Params {
   Decode2Params D;
   unsigned long long* ticket;  // launch ticket counter (only grows): generation = ticket / CTAs
@@ -70,7 +79,7 @@ struct Step1Layout {
 // activations alias the gate/up ring (which is used only between them); the
 // router rows alias the down prefetch area.  Three ring slots per warp where
 // they fit, else two.
-__host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) {
+__host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, bool sign) {
   Step1Layout L{};
   for (int sw = 3; sw >= 2; --sw) {
     L = Step1Layout{};
@@ -81,7 +90,7 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
       off = (off + bytes + 127) / 128 * 128;
       return o;
     };
-    size_t ring = static_cast<size_t>(kS1Warps) * sw * Slot<2, 1, true>::bytes;
+    size_t ring = static_cast<size_t>(kS1Warps) * sw * 2 * s1_mat_bytes(sign);
     const size_t xf = static_cast<size_t>(H) * 4;
     const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
     const size_t inner = static_cast<size_t>(2) * K * (F / kBlock) * kPanel * 4;
@@ -91,7 +100,7 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K) 
     L.act = L.ring;
     L.inner = L.ring + act;
     L.xf = L.ring;
-    const size_t pref = static_cast<size_t>(K) * (F / kBlock) * kMatBytes;
+    const size_t pref = static_cast<size_t>(K) * (F / kBlock) * s1_mat_bytes(sign);
     const size_t rows = static_cast<size_t>(2) * H * 4;  // at most two router rows per CTA
     L.pref = take(pref > rows ? pref : rows);
     L.xq4 = take(static_cast<size_t>(H));
@@ -128,7 +137,11 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// kSign: the weights are 1-bit sign codes (else base-3 digits).
+template <bool kSign>
 __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
+  constexpr int kWBytes = s1_word_bytes(kSign), kMat = s1_mat_bytes(kSign);
+  constexpr int kWords = kSign ? kSignWords : kBlockWords;
   extern __shared__ __align__(1024) unsigned char smem[];
   const Decode2Params& D = S1.D;
   const DecodeParams& P = D.P;
@@ -136,7 +149,7 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   const int nbH = H / kBlock, nbF = F / kBlock;
   const int C = gridDim.x, c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Step1Layout L = step1_layout(H, F, E, K);
+  const Step1Layout L = step1_layout(H, F, E, K, kSign);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L.flag);
   uint64_t* pbar = reinterpret_cast<uint64_t*>(smem + L.flag + 16);
   int* sq4 = reinterpret_cast<int*>(smem + L.xq4);
@@ -287,12 +300,12 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   const int panelH = c;  // C >= hidden/32: at most one panel per CTA
   const bool has_panel = panelH < H / kPanel;
   unsigned char* pref = smem + L.pref;
-  const size_t pref_slot = static_cast<size_t>(nbF) * kMatBytes;
+  const size_t pref_slot = static_cast<size_t>(nbF) * kMat;
   // gate/up: units (slot, 32-row panel of ffn); stream h of this CTA takes
   // every other unit of the CTA's list, the blocks of hidden of a unit split
   // over the stream's warps
   {
-    using SL = Slot<2, 1, true>;
+    constexpr int kSlotBytes = 2 * kMat;  // gate, then up: words and scales each
     const int SW = L.sw;
     const int panels = F / kPanel;
     const int64_t U = static_cast<int64_t>(K) * panels;
@@ -307,7 +320,7 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     int nmine = 0;
     while (unit_of(kS1Streams * nmine + h) < U) ++nmine;
     auto my_unit = [&](int i) { return unit_of(kS1Streams * i + h); };
-    unsigned char* myring = smem + L.ring + static_cast<size_t>(warp) * SW * SL::bytes;
+    unsigned char* myring = smem + L.ring + static_cast<size_t>(warp) * SW * kSlotBytes;
     float* rb = reinterpret_cast<float*>(smem + L.red) + h * (2 * kNC * 32);
     const int bar_done = 1 + h, bar_free = 1 + kS1Streams + h;
     const unsigned long long tag64 = static_cast<unsigned long long>(*sgen) << 32;
@@ -323,15 +336,15 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         if (lane == 0) {
           const int64_t iu = my_unit(im);
           const int e = sel_e[iu / panels];
-          unsigned char* dst = myring + slot * SL::bytes;
+          unsigned char* dst = myring + slot * kSlotBytes;
           if (e >= 0 && e < E) {
             const size_t pb = (static_cast<size_t>(e) * panels + static_cast<size_t>(iu % panels)) * nbH + ib;
-            const uint32_t tb = kBlockWords * kPanel * 4, sb = kPanel * 2;
+            const uint32_t tb = kWBytes, sb = kPanel * 2;
             mbar_arrive_expect_tx(mybar + slot, 2 * (tb + sb));
-            bulk_g2s(dst, P.gate_trits + pb * kBlockWords * kPanel, tb, mybar + slot, pol);
+            bulk_g2s(dst, P.gate_trits + pb * kWords * kPanel, tb, mybar + slot, pol);
             bulk_g2s(dst + tb, P.gate_scales + pb * kPanel, sb, mybar + slot, pol);
-            bulk_g2s(dst + kMatBytes, P.up_trits + pb * kBlockWords * kPanel, tb, mybar + slot, pol);
-            bulk_g2s(dst + kMatBytes + tb, P.up_scales + pb * kPanel, sb, mybar + slot, pol);
+            bulk_g2s(dst + kMat, P.up_trits + pb * kWords * kPanel, tb, mybar + slot, pol);
+            bulk_g2s(dst + kMat + tb, P.up_scales + pb * kPanel, sb, mybar + slot, pol);
           } else {
             mbar_arrive(mybar + slot);
           }
@@ -347,10 +360,10 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       const int j = warp;
       const size_t pb0 = (static_cast<size_t>(sel_e[j]) * (H / kPanel) + panelH) * nbF;
       unsigned char* dst = pref + j * pref_slot;
-      const uint32_t tb = static_cast<uint32_t>(nbF) * kBlockWords * kPanel * 4;
+      const uint32_t tb = static_cast<uint32_t>(nbF) * kWBytes;
       const uint32_t sb = static_cast<uint32_t>(nbF) * kPanel * 2;
       mbar_arrive_expect_tx(pbar, tb + sb);
-      bulk_g2s(dst, P.down_trits + pb0 * kBlockWords * kPanel, tb, pbar, policy_evict_first());
+      bulk_g2s(dst, P.down_trits + pb0 * kWords * kPanel, tb, pbar, policy_evict_first());
       bulk_g2s(dst + tb, P.down_scales + pb0 * kPanel, sb, pbar, policy_evict_first());
     }
     int s = 0;
@@ -364,8 +377,12 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
           record_status(P.status, MOE_ERR_TIMEOUT);
           *abort = 1;
         }
-        block_dot<2, 1, 1>(myring + slot * SL::bytes, sq4 + b * (kBlock / 4), 0, sxd + b * kSubPerBlock,
-                           sxas + b * kSubPerBlock, 0, lane, part);
+        if constexpr (kSign)
+          block_dot_sign<2>(myring + slot * kSlotBytes, kMat, kWBytes, sq4 + b * (kBlock / 4), sxd + b * kSubPerBlock,
+                            sxas + b * kSubPerBlock, lane, part);
+        else
+          block_dot<2, 1, 1>(myring + slot * kSlotBytes, sq4 + b * (kBlock / 4), 0, sxd + b * kSubPerBlock,
+                             sxas + b * kSubPerBlock, 0, lane, part);
         __syncwarp();
         issue_next(slot);
       }
@@ -472,13 +489,18 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         __syncwarp();
         const unsigned char* wj = pref + j * pref_slot;
         for (int b = bb; b < be; ++b) {
-          const int scale_off = nbF * kBlockWords * kPanel * 4 + b * kPanel * 2 - b * kBlockWords * kPanel * 4;
+          // block b's words, then (after every block's words) its scales
+          const int scale_off = nbF * kWBytes + b * kPanel * 2 - b * kWBytes;
           float inner[1][1];
           float sc[1];
-          block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kBlockWords * kPanel * 4,
-                                   aq4 + j * (F / 4) + b * (kBlock / 4), 0,
-                                   ad + j * (F / kQBlock) + b * kSubPerBlock,
-                                   aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
+          if constexpr (kSign)
+            block_dot_sign<1, true>(wj + static_cast<size_t>(b) * kWBytes, kMat, scale_off,
+                                    aq4 + j * (F / 4) + b * (kBlock / 4), ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                    aas + j * (F / kQBlock) + b * kSubPerBlock, lane, inner, sc);
+          else
+            block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kWBytes, aq4 + j * (F / 4) + b * (kBlock / 4), 0,
+                                     ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                     aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
           sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
           sscale[(j * nbF + b) * kPanel + lane] = sc[0];
         }
@@ -508,7 +530,8 @@ bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem) {
   if (P.hidden / kPanel > n_sm) return false;
   if (P.n_experts > 2 * n_sm) return false;  // at most two router rows per CTA
   if (P.n_experts > kS1MaxE) return false;
-  const Step1Layout L = step1_layout(P.hidden, P.ffn, P.n_experts, P.top_k);
+  if (P.format != MOE_FORMAT_TERNARY && P.format != MOE_FORMAT_SIGN) return false;
+  const Step1Layout L = step1_layout(P.hidden, P.ffn, P.n_experts, P.top_k, P.format == MOE_FORMAT_SIGN);
   *smem = L.total;
   return L.total <= static_cast<size_t>(kMaxDynSmem);
 }
@@ -519,7 +542,8 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !done[dev].load(std::memory_order_relaxed)) {
-    cudaFuncSetAttribute(k_step1, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_step1<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_step1<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     done[dev].store(true, std::memory_order_relaxed);
   }
   size_t smem = 0;
@@ -542,12 +566,13 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_ok[di] >= 0 ? 2 : 1;
-  cudaError_t err = cudaLaunchKernelEx(&cfg, k_step1, S);
+  auto kern = D.P.format == MOE_FORMAT_SIGN ? k_step1<true> : k_step1<false>;
+  cudaError_t err = cudaLaunchKernelEx(&cfg, kern, S);
   if (err != cudaSuccess && cfg.numAttrs == 2 && pdl_ok[di] == 0) {
     cudaGetLastError();
     pdl_ok[di] = -1;
     cfg.numAttrs = 1;
-    err = cudaLaunchKernelEx(&cfg, k_step1, S);
+    err = cudaLaunchKernelEx(&cfg, kern, S);
   } else if (err == cudaSuccess && cfg.numAttrs == 2) {
     pdl_ok[di] = 1;
   }

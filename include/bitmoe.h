@@ -111,8 +111,8 @@ typedef struct {
  * hidden <= 16384, ffn <= 8192, 1 <= top_k <= min(n_experts, 32),
  * n_experts <= 1024.  All three formats run the decode path (up to 64
  * tokens) and the prefill GEMM (moe_expert_ffn_prefill, moe_forward of more
- * than 64 tokens); the one-token fused step is ternary only (other formats
- * take the four-kernel decode chain for one token).                       */
+ * than 64 tokens); the one-token fused step takes ternary and sign-code
+ * layers (two-level scales take the four-kernel decode chain for one token). */
 typedef struct {
   int32_t hidden, ffn, n_experts, top_k;
   moe_tmat gate, up, down;

@@ -22,7 +22,9 @@ def _names(B, fn):
 @pytest.mark.parametrize("fmt,ntok,expect", [
     ("ternary", 1, ["step1"]),
     ("ternary", 16, ["router_quant", "topk_group", "gateup", "down"]),
-    ("sign", 1, ["router_quant", "topk_group", "gateup", "down"]),
+    ("sign", 1, ["step1"]),
+    ("sign", 3, ["router_quant", "topk_group", "gateup", "down"]),
+    ("e16", 1, ["router_quant", "topk_group", "gateup", "down"]),
     ("e16", 3, ["router_quant", "topk_group", "gateup", "down"]),
 ])
 def test_forward_kernels(fmt, ntok, expect):

@@ -100,11 +100,11 @@ def test_sign_layer_30b(orc, ntok):
     assert rel_err_rms(y, ref) <= LAYER_TOL
 
 
-@pytest.mark.parametrize("ntok", [8])
+@pytest.mark.parametrize("ntok", [1, 8])
 def test_sign_layer_large(orc, ntok):
-    """The large layer (hidden 4096, ffn 2048, 256 experts, top-8) at 8
-    tokens, the shape the benchmark times: every token, two at a time through
-    the oracle."""
+    """The large layer (hidden 4096, ffn 2048, 256 experts, top-8) at one
+    token (the fused one-token step) and at 8 tokens, the shape the benchmark
+    times: every token, two at a time through the oracle."""
     y, ref = _layer_parity(orc, synthetic.WORKLOADS["large"], ntok, 34, np.arange(ntok), chunk=2)
     assert rel_err_rms(y, ref) <= LAYER_TOL
 
