@@ -57,10 +57,23 @@ __device__ __forceinline__ void group_body(const DecodeParams& P, const int* sid
   const int E = P.n_experts, npairs = P.ntok * P.top_k, tid = threadIdx.x;
   for (int e = tid; e <= E; e += kGroupThreads) { cnt[e] = 0; fill[e] = 0; }
   __syncthreads();
-  for (int p = tid; p < npairs; p += kGroupThreads) {
-    int e = sidx ? sidx[p] : __ldcg(P.idx + p);
-    if (e < 0 || e >= E) { record_status(P.status, MOE_ERR_BAD_INDEX); e = E; }
-    atomicAdd(&cnt[e], 1);
+  // eight ids per thread in flight at a time (the counts' atomics would
+  // otherwise hold each load back)
+  constexpr int kU = 8;
+  for (int p0 = tid; p0 < npairs; p0 += kU * kGroupThreads) {
+    int ev[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int p = p0 + u * kGroupThreads;
+      ev[u] = p < npairs ? (sidx ? sidx[p] : __ldcg(P.idx + p)) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (p0 + u * kGroupThreads >= npairs) continue;
+      int e = ev[u];
+      if (e < 0 || e >= E) { record_status(P.status, MOE_ERR_BAD_INDEX); e = E; }
+      atomicAdd(&cnt[e], 1);
+    }
   }
   __syncthreads();
   // groups 0..E handled two per thread (E + 1 <= 2 * kGroupThreads)
@@ -93,10 +106,21 @@ __device__ __forceinline__ void group_body(const DecodeParams& P, const int* sid
   if (tid == 0) *const_cast<int32_t*>(P.n_items) = tot_i;
   __syncthreads();
   int32_t* pairs = const_cast<int32_t*>(P.pairs);
-  for (int p = tid; p < npairs; p += kGroupThreads) {
-    int e = sidx ? sidx[p] : __ldcg(P.idx + p);
-    if (e < 0 || e >= E) e = E;
-    pairs[off[e] + atomicAdd(&fill[e], 1)] = p;
+  for (int p0 = tid; p0 < npairs; p0 += kU * kGroupThreads) {
+    int ev[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int p = p0 + u * kGroupThreads;
+      ev[u] = p < npairs ? (sidx ? sidx[p] : __ldcg(P.idx + p)) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int p = p0 + u * kGroupThreads;
+      if (p >= npairs) continue;
+      int e = ev[u];
+      if (e < 0 || e >= E) e = E;
+      pairs[off[e] + atomicAdd(&fill[e], 1)] = p;
+    }
   }
 }
 

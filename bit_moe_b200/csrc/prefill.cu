@@ -586,26 +586,29 @@ __global__ void __launch_bounds__(kPThreads, 1) k_prefill_mma(DecodeParams P) {
 }
 
 // y[t] = sum_j wts[t][j] * ye[t][j], slots in order; four h per thread
-// (16-byte loads and stores; hidden is a multiple of 256).
+// (16-byte loads and stores; hidden is a multiple of 256): CTAs take tokens,
+// threads the token's float4 columns.
 __global__ void k_combine(DecodeParams P) {
   pdl_enter();
-  const int H = P.hidden, K = P.top_k, H4 = H / 4;
-  const int64_t total = static_cast<int64_t>(P.ntok) * H4;
+  const int H4 = P.hidden / 4, K = P.top_k;
   const float4* ye = reinterpret_cast<const float4*>(P.ye);
   float4* y = reinterpret_cast<float4*>(P.y);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t t = i / H4, h4 = i % H4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < K; ++j) {
-      const float w = P.wts[t * K + j];
-      const float4 v = __ldcs(ye + (t * K + j) * H4 + h4);
-      acc.x = __fmaf_rn(w, v.x, acc.x);
-      acc.y = __fmaf_rn(w, v.y, acc.y);
-      acc.z = __fmaf_rn(w, v.z, acc.z);
-      acc.w = __fmaf_rn(w, v.w, acc.w);
+  for (int t = blockIdx.x; t < P.ntok; t += gridDim.x) {
+    const float* wt = P.wts + static_cast<size_t>(t) * K;
+    const float4* src = ye + static_cast<size_t>(t) * K * H4;
+    for (int h4 = threadIdx.x; h4 < H4; h4 += blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int j = 0; j < K; ++j) {
+        const float w = wt[j];
+        const float4 v = __ldcs(src + static_cast<size_t>(j) * H4 + h4);
+        acc.x = __fmaf_rn(w, v.x, acc.x);
+        acc.y = __fmaf_rn(w, v.y, acc.y);
+        acc.z = __fmaf_rn(w, v.z, acc.z);
+        acc.w = __fmaf_rn(w, v.w, acc.w);
+      }
+      y[static_cast<size_t>(t) * H4 + h4] = acc;
     }
-    y[i] = acc;
   }
 }
 
