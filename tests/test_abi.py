@@ -118,3 +118,27 @@ def test_forward_host_long_sign_call_passes_the_format_checks():
     assert rc in (-5, -8), L.moe_last_error()  # no usable device on this machine
     assert b"64 tokens" not in L.moe_last_error()
     assert L.moe_launch_count() == n0
+
+
+def test_workspace_act_offsets():
+    """The offsets of x's int8 codes and scales in a workspace: 256-byte
+    aligned, past the header, inside the workspace, not overlapping; bad
+    arguments refused."""
+    B, L = _lib()
+    buf = (ctypes.c_uint8 * 64)()
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
+
+    def tm(rows, k):
+        return B.moe_tmat(rows, k, p.value, p.value, 0, None)
+    H, F, E, K = 2048, 768, 128, 8
+    lay = B.moe_layer(H, F, E, K, tm(E * F, H), tm(E * F, H), tm(E * H, F))
+    for ntok, prefill in ((1, 0), (16, 0), (2048, 1)):
+        oq, od = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        assert L.moe_workspace_act(ctypes.byref(lay), ntok, prefill, ctypes.byref(oq), ctypes.byref(od)) == 0
+        total = L.moe_workspace_bytes(ctypes.byref(lay), ntok, prefill)
+        assert oq.value % 256 == 0 and od.value % 256 == 0 and oq.value >= 256
+        assert oq.value + ntok * H <= od.value
+        assert od.value + ntok * (H // 32) * 4 <= total
+    oq, od = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert L.moe_workspace_act(ctypes.byref(lay), 0, 0, ctypes.byref(oq), ctypes.byref(od)) == -1
+    assert L.moe_workspace_act(ctypes.byref(lay), 1, 0, None, ctypes.byref(od)) == -1
