@@ -96,6 +96,7 @@ def kernel_bytes(wl, unique_experts):
         "topk_softmax": T * E * 4 + pairs * 8,
         "router_quant": E * H * 4 + T * H * 4 + T * E * 4 + T * H + T * H // 32 * 4,
         "topk_group": T * E * 4 + pairs * 8 + pairs * 4 * 3,
+        "route_group": E * H * 4 + T * H * 4 + 2 * T * E * 4 + T * H + T * H // 32 * 4 + pairs * 8 + pairs * 4 * 3,
         "group": pairs * 4 * 3,
         "gateup": unique_experts * 2 * wl.matrix_bytes(F, H) + T * H + T * H // 32 * 4
         + pairs * F + pairs * F // 32 * 4 + pairs * 8,

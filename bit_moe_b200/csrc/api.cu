@@ -468,10 +468,19 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
     size_t smem_s = 0;
     chain1 = !step1_supported(P, sm_count(), &smem_s);
   }
+  if ((ntok > 1 || chain1) && !prefill && route_group_ok(P, sm_count())) {
+    // few tokens (and one token of an E16 layer): router logits, activation
+    // quantization, top-k and grouping in one launch, then the grouped
+    // mat-vecs
+    WsHeader* hd = reinterpret_cast<WsHeader*>(ws);
+    if ((rc = launch_route_group(P, x, w_router, logits, wts, reinterpret_cast<uint32_t*>(&hd->pad[1]), sm_count(), s)))
+      return rc;
+    return launch_ffn(P, s);
+  }
   if ((ntok > 1 || chain1) && !prefill && router_quant_small_ok(ntok, L->hidden)) {
-    // few tokens (and one token of an E16 layer): router logits with
-    // the activation quantization, then the top-k with the grouping, then
-    // the grouped mat-vecs
+    // the same in two launches where no one-wave shape exists: router
+    // logits with the activation quantization, then the top-k with the
+    // grouping
     if ((rc = launch_router_quant_small(x, w_router, ntok, L->hidden, L->n_experts, logits, xq, xd, s)))
       return rc;
     if ((rc = launch_topk_group(P, logits, wts, s))) return rc;
@@ -617,7 +626,7 @@ const char* moe_kernel_name(int32_t id) {
   static const char* names[MOE_K_COUNT] = {
       "quantize_weights", "quant_act_q8", "router_logits", "topk_softmax", "group",
       "gateup", "down", "debug_matvec", "prefill_gateup", "prefill_down", "route", "combine", "step1", "prefill_gather", "copy",
-      "router_quant", "topk_group", "shared", "tc_gateup", "tc_down"};
+      "router_quant", "topk_group", "shared", "tc_gateup", "tc_down", "route_group"};
   return (id >= 0 && id < MOE_K_COUNT) ? names[id] : "";
 }
 

@@ -35,7 +35,8 @@ constexpr int kMaxDynSmem = 227 * 1024;  // opt-in dynamic shared memory per CTA
 // Workspace header: the first 256 bytes hold the device status word.
 struct WsHeader {
   int32_t status;    // first error code seen by a kernel (0 = ok)
-  int32_t pad[63];   // pad[0]: route counter; pad[3..4]: 64-bit one-token step tickets;
+  int32_t pad[63];   // pad[0]: route counter; pad[1]: route_group counter; pad[3..4]: 64-bit
+                     // one-token step tickets;
                      // pad[8..9]: the wait test knob (below)
 };
 // Test knob of the bounded device waits (moe_debug_wait_knob; zero in every

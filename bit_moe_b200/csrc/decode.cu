@@ -19,6 +19,8 @@
 #include "bitmoe.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
 #include "tcmv.cuh"
 #include "ternary_dot.cuh"
 #include "topk.cuh"
@@ -158,6 +160,127 @@ __global__ void __launch_bounds__(kGroupThreads) k_topk_group(DecodeParams P, co
       const_cast<int32_t*>(P.idx)[static_cast<int64_t>(t) * K + lane] = my_e;
       sidx[t * K + lane] = my_e;
       wts[static_cast<int64_t>(t) * K + lane] = w;
+    }
+  }
+  __syncthreads();
+  group_body(P, sidx);
+}
+
+// S1 + S2 + S6 of a decode batch in one launch.  CTA (i, c) copies router
+// rows [i*EW, (i+1)*EW) and tokens [c*TT, (c+1)*TT) of x into shared memory
+// (one bulk copy each, so the CTA pays one copy latency), computes those
+// logits with the fixed evaluation order of the router kernels (one warp per
+// logit: lane l's chain over k = l, l+32, ... ascending, then the xor
+// butterfly), and quantizes its share of the tile's 32-blocks of x.  The last
+// CTA to finish (a ticket counter that it resets) takes every token's top-k
+// and softmax (warp_topk_softmax, one warp per token) and groups the pairs
+// by expert (group_body).  No CTA waits for another.
+template <int kPer>
+__global__ void __launch_bounds__(kGroupThreads) k_route_group(DecodeParams P, const float* __restrict__ x,
+                                                               const float* __restrict__ wr,
+                                                               float* __restrict__ logits,
+                                                               float* __restrict__ wts, uint32_t* ticket,
+                                                               int EW, int TT) {
+  extern __shared__ __align__(128) unsigned char rsm[];
+  __shared__ int sidx[kMaxDecodeTokens * kMaxTopK];
+  const int H = P.hidden, E = P.n_experts, T = P.ntok, K = P.top_k;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarp = blockDim.x >> 5;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(rsm);
+  int* flag = reinterpret_cast<int*>(rsm + 8);
+  float* wsm = reinterpret_cast<float*>(rsm + 128);  // [EW][H]
+  float* xsm = wsm + static_cast<size_t>(EW) * H;    // [TT][H]
+  const int e0 = blockIdx.x * EW, ne = min(EW, E - e0);
+  const int t0 = blockIdx.y * TT, nt = min(TT, T - t0);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // the router rows are caller data that no kernel of this library writes:
+  // their copy starts before the dependency wait
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(ne + nt) * H * 4);
+    bulk_g2s(wsm, wr + static_cast<size_t>(e0) * H, static_cast<uint32_t>(ne) * H * 4, bar, policy_evict_first());
+  }
+  pdl_wait();
+  if (tid == 0)
+    bulk_g2s(xsm, x + static_cast<size_t>(t0) * H, static_cast<uint32_t>(nt) * H * 4, bar, policy_evict_last());
+  pdl_launch_dependents();
+  const bool ok = mbar_wait(bar, 0);
+  if (!ok) {
+    // the copies must land before the CTA exits; the counter still counts
+    // this CTA, and the status tells the caller that the step is void
+    if (tid == 0) record_status(P.status, MOE_ERR_TIMEOUT);
+    mbar_wait(bar, 0);
+  } else {
+    // micro-tiles of up to 2 tokens x 2 experts per warp: each value a lane
+    // loads from shared memory feeds two of the logits' chains (shared
+    // memory bandwidth, not the chains, bounds one logit per warp)
+    const int mtn = (nt + 1) / 2, men = (ne + 1) / 2;
+    for (int mt = warp; mt < mtn * men; mt += nwarp) {
+      const int ti = (mt / men) * 2, ei = (mt % men) * 2;
+      const bool t1 = ti + 1 < nt, e1 = ei + 1 < ne;
+      const float* w0 = wsm + static_cast<size_t>(ei) * H;
+      const float* w1 = e1 ? w0 + H : w0;
+      const float* x0 = xsm + static_cast<size_t>(ti) * H;
+      const float* x1 = t1 ? x0 + H : x0;
+      float p00 = 0.f, p01 = 0.f, p10 = 0.f, p11 = 0.f;
+#pragma unroll 4
+      for (int k = lane; k < H; k += 32) {
+        const float a0 = x0[k], a1 = x1[k], b0 = w0[k], b1 = w1[k];
+        p00 = __fmaf_rn(b0, a0, p00);
+        p01 = __fmaf_rn(b1, a0, p01);
+        p10 = __fmaf_rn(b0, a1, p10);
+        p11 = __fmaf_rn(b1, a1, p11);
+      }
+#pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) {
+        p00 = __fadd_rn(p00, __shfl_xor_sync(0xffffffffu, p00, m));
+        p01 = __fadd_rn(p01, __shfl_xor_sync(0xffffffffu, p01, m));
+        p10 = __fadd_rn(p10, __shfl_xor_sync(0xffffffffu, p10, m));
+        p11 = __fadd_rn(p11, __shfl_xor_sync(0xffffffffu, p11, m));
+      }
+      if (lane == 0) {
+        float* l0 = logits + static_cast<size_t>(t0 + ti) * E + e0 + ei;
+        l0[0] = p00;
+        if (e1) l0[1] = p01;
+        if (t1) l0[E] = p10;
+        if (t1 && e1) l0[E + 1] = p11;
+      }
+    }
+    // the tile's 32-blocks of x, dealt over the CTAs that hold it from the
+    // last warp down (the first warps take the logits)
+    const int nblk = nt * (H / kQBlock);
+    for (int blk = (nwarp - 1 - warp) * gridDim.x + blockIdx.x; blk < nblk; blk += gridDim.x * nwarp)
+      quant_act_block(xsm, blk, lane, const_cast<int8_t*>(P.xq) + static_cast<size_t>(t0) * H,
+                      const_cast<float*>(P.xd) + static_cast<size_t>(t0) * (H / kQBlock));
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) *flag = (atomicAdd(ticket, 1u) == gridDim.x * gridDim.y - 1) ? 1 : 0;
+  __syncthreads();
+  if (!*flag) return;
+  __threadfence();
+  if (tid == 0) atomicExch(ticket, 0u);  // every CTA has taken its ticket
+  for (int t = warp; t < T; t += nwarp) {
+    uint32_t key[kPer];
+    uint32_t need = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = 0u;
+      if (e < E) {
+        key[i] = f32_key(__ldcg(logits + static_cast<size_t>(t) * E + e));
+        need |= 1u << i;
+      }
+    }
+    int my_e;
+    float w;
+    warp_topk_softmax<kPer>(key, need, K, lane, my_e, w);
+    if (lane < K) {
+      const_cast<int32_t*>(P.idx)[static_cast<size_t>(t) * K + lane] = my_e;
+      sidx[t * K + lane] = my_e;
+      wts[static_cast<size_t>(t) * K + lane] = w;
     }
   }
   __syncthreads();
@@ -451,6 +574,82 @@ int launch_group(const DecodeParams& P, cudaStream_t stream) {
   launch_k(k_group, dim3(1), dim3(kGroupThreads), 0, stream, P);
   note_launch(MOE_K_GROUP, stream);
   return check_launch("group");
+}
+
+// Shape of k_route_group: EW experts and TT tokens per CTA with their rows
+// in shared memory, in one wave of at most n_sm CTAs, the fewest rows per
+// CTA first (the least copying per SM), then the most CTAs.  False if no
+// shape fits one wave.
+static bool route_group_shape(int H, int E, int T, int n_sm, size_t smem_cap, int* EW, int* TT) {
+  const size_t row = static_cast<size_t>(H) * 4;
+  int best_rows = 0, best_grid = 0;
+  for (int tt = T;; tt = (tt + 1) / 2) {
+    for (int ew = 1; ew <= E && ew <= 64; ++ew) {
+      const int64_t grid = static_cast<int64_t>((E + ew - 1) / ew) * ((T + tt - 1) / tt);
+      if (grid > n_sm || 128 + (ew + tt) * row > smem_cap) continue;
+      const int rows = ew + tt;
+      if (best_rows == 0 || rows < best_rows || (rows == best_rows && grid > best_grid)) {
+        best_rows = rows;
+        best_grid = static_cast<int>(grid);
+        *EW = ew;
+        *TT = tt;
+      }
+    }
+    if (tt == 1) break;
+  }
+  return best_rows > 0;
+}
+
+// Largest dynamic shared memory of k_route_group: the opt-in limit less its
+// static arrays.
+template <int kPer>
+static size_t route_group_cap() {
+  static std::atomic<size_t> cap{0};  // the same on every device of one architecture
+  size_t c = cap.load(std::memory_order_relaxed);
+  if (c == 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, k_route_group<kPer>) != cudaSuccess) return 0;
+    const size_t stat = fa.sharedSizeBytes + 1024;
+    c = stat < static_cast<size_t>(kMaxDynSmem) ? kMaxDynSmem - stat : 0;
+    cap.store(c, std::memory_order_relaxed);
+  }
+  return c;
+}
+
+bool route_group_ok(const DecodeParams& P, int n_sm) {
+  if (P.ntok < 1 || P.ntok > kMaxDecodeTokens || P.hidden % kQBlock) return false;
+  const size_t cap = P.n_experts <= 128 ? route_group_cap<4>()
+                     : P.n_experts <= 256 ? route_group_cap<8>() : route_group_cap<32>();
+  int ew = 0, tt = 0;
+  return route_group_shape(P.hidden, P.n_experts, P.ntok, n_sm, cap, &ew, &tt);
+}
+
+template <int kPer>
+static int launch_route_group_k(const DecodeParams& P, const float* x, const float* wr, float* logits,
+                                float* wts, uint32_t* ticket, int n_sm, cudaStream_t stream) {
+  const size_t cap = route_group_cap<kPer>();
+  int EW = 0, TT = 0;
+  if (!route_group_shape(P.hidden, P.n_experts, P.ntok, n_sm, cap, &EW, &TT))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "route_group: no one-wave shape");
+  const size_t smem = 128 + static_cast<size_t>(EW + TT) * P.hidden * 4;
+  static std::atomic<bool> done[64];  // the attribute call is idempotent
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !done[dev].load(std::memory_order_relaxed)) {
+    cudaFuncSetAttribute(k_route_group<kPer>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(cap));
+    done[dev].store(true, std::memory_order_relaxed);
+  }
+  const dim3 grid((P.n_experts + EW - 1) / EW, (P.ntok + TT - 1) / TT);
+  launch_k(k_route_group<kPer>, grid, dim3(kGroupThreads), smem, stream, P, x, wr, logits, wts, ticket, EW, TT);
+  note_launch(MOE_K_ROUTE_GROUP, stream);
+  return check_launch("route_group");
+}
+
+int launch_route_group(const DecodeParams& P, const float* x, const float* wr, float* logits, float* wts,
+                       uint32_t* ticket, int n_sm, cudaStream_t stream) {
+  if (P.n_experts <= 128) return launch_route_group_k<4>(P, x, wr, logits, wts, ticket, n_sm, stream);
+  if (P.n_experts <= 256) return launch_route_group_k<8>(P, x, wr, logits, wts, ticket, n_sm, stream);
+  return launch_route_group_k<32>(P, x, wr, logits, wts, ticket, n_sm, stream);
 }
 
 int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cudaStream_t stream) {

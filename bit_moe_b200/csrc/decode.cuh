@@ -114,6 +114,13 @@ int launch_group(const DecodeParams& P, cudaStream_t stream);
 // Top-k softmax of P.ntok <= 64 tokens' logits ([ntok][E] fp32) into P.idx
 // and wts, then the grouping of launch_group, in one single-CTA kernel.
 int launch_topk_group(const DecodeParams& P, const float* logits, float* wts, cudaStream_t stream);
+// Router logits, activation quantization, top-k and grouping of up to 64
+// tokens in one launch (k_route_group); route_group_ok tells whether a
+// one-wave shape exists.  ticket: a workspace counter that is zero between
+// launches.
+bool route_group_ok(const DecodeParams& P, int n_sm);
+int launch_route_group(const DecodeParams& P, const float* x, const float* wr, float* logits, float* wts,
+                       uint32_t* ticket, int n_sm, cudaStream_t stream);
 int launch_ffn(const DecodeParams& P, cudaStream_t stream);
 int launch_debug_matvec(const moe_tmat* m, int ntok, const int8_t* xq, const float* xd, float* out,
                         int32_t* isum, cudaStream_t stream);

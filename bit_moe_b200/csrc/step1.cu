@@ -137,8 +137,10 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// kSign: the weights are 1-bit sign codes (else base-3 digits).
-template <bool kSign>
+// kSign: the weights are 1-bit sign codes (else base-3 digits).  kSlotOrder:
+// the down items go to the warps in slot order (at most two items per warp),
+// else by halves of a slot.
+template <bool kSign, bool kSlotOrder>
 __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   constexpr int kWBytes = s1_word_bytes(kSign), kMat = s1_mat_bytes(kSign);
   constexpr int kWords = kSign ? kSignWords : kBlockWords;
@@ -433,53 +435,84 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     // the prefetch must land before this CTA reads it or exits
     bool ok = mbar_wait_sleep(pbar, 0);
     if (!ok) record_status(P.status, MOE_ERR_TIMEOUT);
-    // warp w takes slot w % kNC, the first (w < kNC) or second half of its
-    // blocks of ffn, as soon as the units of those blocks are published; each
-    // block's inner sum and weight scale go to shared memory, and one warp
-    // applies the scales and combines the slots in the order of the grouped
-    // down kernel
+    // the items (slot j, block b of ffn): each polls the tagged words of its
+    // 8 units, multiplies them with the prefetched down weights and leaves
+    // its inner sums and weight scales in shared memory; one warp per slot
+    // then applies the scales and warp 0 combines the slots, in the order of
+    // the grouped down kernel.  With at most two items per warp they go to
+    // the warps in slot order (item i to warp i % kS1Warps: the units of the
+    // lower slots are published first, so every warp starts at once);
+    // otherwise warp w takes slot w % kNC, the first (w < kNC) or second half
+    // of its blocks, so that the warps of the early slots finish early.
     const int panels = F / kPanel;
     int* aq4 = reinterpret_cast<int*>(smem + L.act);                       // [K][F/4]
     float* ad = reinterpret_cast<float*>(aq4 + K * (F / 4));                 // [K][F/32]
     int* aas = reinterpret_cast<int*>(ad + K * (F / kQBlock));              // [K][F/32]
     float* sinner = reinterpret_cast<float*>(smem + L.inner);               // [K][nbF][32]
     float* sscale = sinner + K * nbF * kPanel;                              // [K][nbF][32]
-    const int j = warp % kNC, half = warp / kNC;
-    const int nb0 = (nbF + 1) / 2;
-    const int bb = half ? nb0 : 0, be = half ? nbF : nb0;
-    if (j < K && ok && bb < be) {
-      // the tagged words of panels [8*bb, 8*be) of slot j, all loads of a
-      // round in flight at once
-      constexpr int kPerC = (kS1MaxF / kBlock + 1) / 2 * (kBlock / kPanel) * kUnitWords / 32;
-      const int nw = (be - bb) * (kBlock / kPanel) * kUnitWords;
-      const unsigned long long* src =
-          S1.units + (static_cast<size_t>(j) * panels + bb * (kBlock / kPanel)) * kUnitWords;
+    if constexpr (kSlotOrder) {
       const uint32_t tag = *sgen;
-      unsigned long long v[kPerC];
-      uint32_t ready = 0, need = 0;
+      const unsigned char* wbase = pref;
+      constexpr int kItemWords = (kBlock / kPanel) * kUnitWords;  // the 8 units of one block of ffn
+      constexpr int kPerI = (kItemWords + 31) / 32;
+      uint32_t need = 0;
 #pragma unroll
-      for (int i = 0; i < kPerC; ++i)
-        if (lane + 32 * i < nw) need |= 1u << i;
-      for (uint32_t polls = 0; ready != need; ++polls) {
-        if (polls > kSpinLimit) break;
+      for (int i = 0; i < kPerI; ++i)
+        if (lane + 32 * i < kItemWords) need |= 1u << i;
+      auto item_src = [&](int it) {
+        const int j = it / nbF, b = it % nbF;
+        return S1.units + (static_cast<size_t>(j) * panels + b * (kBlock / kPanel)) * kUnitWords;
+      };
+      const int nitems = warp < K * nbF ? (K * nbF - 1 - warp) / kS1Warps + 1 : 0;
+      auto item_at = [&](int q) { return warp + q * kS1Warps; };
+      // the loads of a warp's next item are in flight while it computes the
+      // current one
+      unsigned long long vn[kPerI];
+      if (nitems > 0) {
+        const unsigned long long* src = item_src(item_at(0));
 #pragma unroll
-        for (int i = 0; i < kPerC; ++i)
-          if ((need & ~ready) & (1u << i)) v[i] = ld_relaxed_u64(src + lane + 32 * i);
-#pragma unroll
-        for (int i = 0; i < kPerC; ++i)
-          if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+        for (int i = 0; i < kPerI; ++i)
+          if (need & (1u << i)) vn[i] = ld_relaxed_u64(src + lane + 32 * i);
       }
-      if (!__all_sync(0xffffffffu, ready == need)) {
-        if (lane == 0) {
-          record_status(P.status, MOE_ERR_TIMEOUT);
-          *abort = 1;
-        }
-      } else {
+      for (int q = 0; ok && q < nitems; ++q) {
+        if (*abort) break;
+        const int it = item_at(q);
+        const int j = it / nbF, b = it % nbF;
+        const unsigned long long* src = item_src(it);
+        unsigned long long v[kPerI];
+        uint32_t ready = 0;
 #pragma unroll
-        for (int i = 0; i < kPerC; ++i) {
+        for (int i = 0; i < kPerI; ++i) {
+          v[i] = vn[i];
+          if ((need & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+        }
+        if (q + 1 < nitems) {
+          const unsigned long long* nsrc = item_src(item_at(q + 1));
+#pragma unroll
+          for (int i = 0; i < kPerI; ++i)
+            if (need & (1u << i)) vn[i] = ld_relaxed_u64(nsrc + lane + 32 * i);
+        }
+        for (uint32_t polls = 0; ready != need; ++polls) {
+          if (polls > kSpinLimit) break;
+#pragma unroll
+          for (int i = 0; i < kPerI; ++i)
+            if ((need & ~ready) & (1u << i)) v[i] = ld_relaxed_u64(src + lane + 32 * i);
+#pragma unroll
+          for (int i = 0; i < kPerI; ++i)
+            if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+        }
+        if (!__all_sync(0xffffffffu, ready == need)) {
+          if (lane == 0) {
+            record_status(P.status, MOE_ERR_TIMEOUT);
+            *abort = 1;
+          }
+          break;
+        }
+#pragma unroll
+        for (int i = 0; i < kPerI; ++i) {
           const int w = lane + 32 * i;
-          if (w < nw) {
-            const int pl = bb * (kBlock / kPanel) + w / kUnitWords, k = w % kUnitWords;
+          if (w < kItemWords) {
+            const int pl = b * (kBlock / kPanel) + w / kUnitWords, k = w % kUnitWords;
             const uint32_t x32 = static_cast<uint32_t>(v[i]);
             if (k < kPanel / 4) aq4[j * (F / 4) + pl * (kPanel / 4) + k] = static_cast<int>(x32);
             else if (k == kPanel / 4) ad[j * (F / kQBlock) + pl] = __uint_as_float(x32);
@@ -487,22 +520,83 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
           }
         }
         __syncwarp();
-        const unsigned char* wj = pref + j * pref_slot;
-        for (int b = bb; b < be; ++b) {
-          // block b's words, then (after every block's words) its scales
-          const int scale_off = nbF * kWBytes + b * kPanel * 2 - b * kWBytes;
-          float inner[1][1];
-          float sc[1];
-          if constexpr (kSign)
-            block_dot_sign<1, true>(wj + static_cast<size_t>(b) * kWBytes, kMat, scale_off,
-                                    aq4 + j * (F / 4) + b * (kBlock / 4), ad + j * (F / kQBlock) + b * kSubPerBlock,
-                                    aas + j * (F / kQBlock) + b * kSubPerBlock, lane, inner, sc);
-          else
-            block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kWBytes, aq4 + j * (F / 4) + b * (kBlock / 4), 0,
-                                     ad + j * (F / kQBlock) + b * kSubPerBlock,
-                                     aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
-          sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
-          sscale[(j * nbF + b) * kPanel + lane] = sc[0];
+        const unsigned char* wj = wbase + j * pref_slot;
+        // block b's words, then (after every block's words) its scales
+        const int scale_off = nbF * kWBytes + b * kPanel * 2 - b * kWBytes;
+        float inner[1][1];
+        float sc[1];
+        if constexpr (kSign)
+          block_dot_sign<1, true>(wj + static_cast<size_t>(b) * kWBytes, kMat, scale_off,
+                                  aq4 + j * (F / 4) + b * (kBlock / 4), ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                  aas + j * (F / kQBlock) + b * kSubPerBlock, lane, inner, sc);
+        else
+          block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kWBytes, aq4 + j * (F / 4) + b * (kBlock / 4), 0,
+                                   ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                   aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
+        sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
+        sscale[(j * nbF + b) * kPanel + lane] = sc[0];
+      }
+    } else {
+      const int j = warp % kNC, half = warp / kNC;
+      const int nb0 = (nbF + 1) / 2;
+      const int bb = half ? nb0 : 0, be = half ? nbF : nb0;
+      if (j < K && ok && bb < be) {
+        // the tagged words of panels [8*bb, 8*be) of slot j, all loads of a
+        // round in flight at once
+        constexpr int kPerC = (kS1MaxF / kBlock + 1) / 2 * (kBlock / kPanel) * kUnitWords / 32;
+        const int nw = (be - bb) * (kBlock / kPanel) * kUnitWords;
+        const unsigned long long* src =
+            S1.units + (static_cast<size_t>(j) * panels + bb * (kBlock / kPanel)) * kUnitWords;
+        const uint32_t tag = *sgen;
+        unsigned long long v[kPerC];
+        uint32_t ready = 0, need = 0;
+#pragma unroll
+        for (int i = 0; i < kPerC; ++i)
+          if (lane + 32 * i < nw) need |= 1u << i;
+        for (uint32_t polls = 0; ready != need; ++polls) {
+          if (polls > kSpinLimit) break;
+#pragma unroll
+          for (int i = 0; i < kPerC; ++i)
+            if ((need & ~ready) & (1u << i)) v[i] = ld_relaxed_u64(src + lane + 32 * i);
+#pragma unroll
+          for (int i = 0; i < kPerC; ++i)
+            if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(v[i] >> 32) == tag) ready |= 1u << i;
+        }
+        if (!__all_sync(0xffffffffu, ready == need)) {
+          if (lane == 0) {
+            record_status(P.status, MOE_ERR_TIMEOUT);
+            *abort = 1;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kPerC; ++i) {
+            const int w = lane + 32 * i;
+            if (w < nw) {
+              const int pl = bb * (kBlock / kPanel) + w / kUnitWords, k = w % kUnitWords;
+              const uint32_t x32 = static_cast<uint32_t>(v[i]);
+              if (k < kPanel / 4) aq4[j * (F / 4) + pl * (kPanel / 4) + k] = static_cast<int>(x32);
+              else if (k == kPanel / 4) ad[j * (F / kQBlock) + pl] = __uint_as_float(x32);
+              else aas[j * (F / kQBlock) + pl] = static_cast<int>(x32);
+            }
+          }
+          __syncwarp();
+          const unsigned char* wj = pref + j * pref_slot;
+          for (int b = bb; b < be; ++b) {
+            // block b's words, then (after every block's words) its scales
+            const int scale_off = nbF * kWBytes + b * kPanel * 2 - b * kWBytes;
+            float inner[1][1];
+            float sc[1];
+            if constexpr (kSign)
+              block_dot_sign<1, true>(wj + static_cast<size_t>(b) * kWBytes, kMat, scale_off,
+                                      aq4 + j * (F / 4) + b * (kBlock / 4), ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                      aas + j * (F / kQBlock) + b * kSubPerBlock, lane, inner, sc);
+            else
+              block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kWBytes, aq4 + j * (F / 4) + b * (kBlock / 4), 0,
+                                       ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                       aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
+            sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
+            sscale[(j * nbF + b) * kPanel + lane] = sc[0];
+          }
         }
       }
     }
@@ -542,8 +636,10 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !done[dev].load(std::memory_order_relaxed)) {
-    cudaFuncSetAttribute(k_step1<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_step1<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_step1<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_step1<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_step1<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    cudaFuncSetAttribute(k_step1<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     done[dev].store(true, std::memory_order_relaxed);
   }
   size_t smem = 0;
@@ -566,7 +662,10 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_ok[di] >= 0 ? 2 : 1;
-  auto kern = D.P.format == MOE_FORMAT_SIGN ? k_step1<true> : k_step1<false>;
+  const bool sign = D.P.format == MOE_FORMAT_SIGN;
+  const bool slot_order = D.P.top_k * (D.P.ffn / kBlock) <= 2 * kS1Warps;
+  auto kern = sign ? (slot_order ? k_step1<true, true> : k_step1<true, false>)
+                   : (slot_order ? k_step1<false, true> : k_step1<false, false>);
   cudaError_t err = cudaLaunchKernelEx(&cfg, kern, S);
   if (err != cudaSuccess && cfg.numAttrs == 2 && pdl_ok[di] == 0) {
     cudaGetLastError();

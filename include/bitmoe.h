@@ -290,7 +290,7 @@ typedef enum {
   MOE_K_PREFILL_GATEUP = 8, MOE_K_PREFILL_DOWN = 9, MOE_K_ROUTE = 10, MOE_K_COMBINE = 11,
   MOE_K_STEP1 = 12, MOE_K_PREFILL_GATHER = 13, MOE_K_COPY = 14, MOE_K_ROUTER_QUANT = 15,
   MOE_K_TOPK_GROUP = 16, MOE_K_SHARED = 17, MOE_K_TC_GATEUP = 18, MOE_K_TC_DOWN = 19,
-  MOE_K_COUNT = 20
+  MOE_K_ROUTE_GROUP = 20, MOE_K_COUNT = 21
 } moe_kernel_id;
 /* Number of kernels this thread has launched through the library so far. */
 int64_t moe_launch_count(void);

@@ -21,11 +21,11 @@ def _names(B, fn):
 
 @pytest.mark.parametrize("fmt,ntok,expect", [
     ("ternary", 1, ["step1"]),
-    ("ternary", 16, ["router_quant", "topk_group", "gateup", "down"]),
+    ("ternary", 16, ["route_group", "gateup", "down"]),
     ("sign", 1, ["step1"]),
-    ("sign", 3, ["router_quant", "topk_group", "gateup", "down"]),
-    ("e16", 1, ["router_quant", "topk_group", "gateup", "down"]),
-    ("e16", 3, ["router_quant", "topk_group", "gateup", "down"]),
+    ("sign", 3, ["route_group", "gateup", "down"]),
+    ("e16", 1, ["route_group", "gateup", "down"]),
+    ("e16", 3, ["route_group", "gateup", "down"]),
 ])
 def test_forward_kernels(fmt, ntok, expect):
     B = bm()
@@ -35,6 +35,32 @@ def test_forward_kernels(fmt, ntok, expect):
     x = synthetic.activations(wl, 81, ntok=ntok, device="cuda")
     ws = B.Workspace.for_layer(layer, ntok)
     assert _names(B, lambda: B.moe_forward(layer, wr, x, ws)) == expect
+
+
+def test_routing_in_one_launch_and_in_two():
+    """A decode batch routes in one launch (k_route_group) where a one-wave
+    shape holds the router rows and tokens in shared memory, and in two
+    (router with quantization, then top-k with grouping) where none does:
+    64 tokens of hidden 4096 over 128 experts.  Both give the same outputs,
+    bit for bit (each token's result does not depend on its batch)."""
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"].with_(hidden=4096, ffn=256, n_experts=128, top_k=2, seed=85)
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 86, ntok=64, device="cuda")
+    ws = B.Workspace.for_layer(layer, 64)
+    y64 = torch.empty((64, wl.hidden), device="cuda")
+    assert _names(B, lambda: B.moe_forward(layer, wr, x, ws, y=y64)) == [
+        "router_quant", "topk_group", "gateup", "down"]
+    assert B.moe_check_status(ws) == 0
+    ws8 = B.Workspace.for_layer(layer, 8)
+    for c in range(8):
+        xc = x[8 * c:8 * (c + 1)].contiguous()
+        y8 = torch.empty((8, wl.hidden), device="cuda")
+        names = _names(B, lambda: B.moe_forward(layer, wr, xc, ws8, y=y8))
+        assert names == ["route_group", "gateup", "down"]
+        assert torch.equal(y8, y64[8 * c:8 * (c + 1)])
+    assert B.moe_check_status(ws8) == 0
 
 
 def test_forward_prefill_kernels():
