@@ -182,13 +182,42 @@ class ClockSampler:
 _CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/', re.S)
 
 
-def kernel_source_hash():
-    """Hash of the kernel sources' code: comments dropped and runs of white
-    space collapsed, so that counters taken on a source stay attributed to it
-    when only its comments change."""
+# The translation unit that defines each kernel of the kernel_bytes table.
+KERNEL_SOURCE = {
+    "step1": "step1.cu", "gateup": "decode.cu", "down": "decode.cu", "route_group": "decode.cu",
+    "topk_group": "decode.cu", "group": "decode.cu", "router_quant": "router.cu", "router_logits": "router.cu",
+    "topk_softmax": "router.cu", "prefill_gateup": "prefill.cu", "prefill_down": "prefill.cu",
+    "prefill_gather": "prefill.cu", "combine": "prefill.cu", "quant_act_q8": "quant.cu",
+    "shared_gateup": "shared.cu", "shared_down": "shared.cu", "shared": "shared.cu", "tc_gateup": "tcmv.cu",
+    "tc_down": "tcmv.cu", "route": "decode2.cu"}
+_INCLUDE = re.compile(r'^\s*#\s*include\s+"([^"]+)"', re.M)
+
+
+def _source_closure(name, csrc):
+    """name and the local headers it includes, transitively."""
+    seen, todo = set(), [name]
+    while todo:
+        n = todo.pop()
+        path = os.path.join(csrc, n)
+        if n in seen or not os.path.exists(path):
+            continue
+        seen.add(n)
+        with open(path, encoding="utf-8") as f:
+            todo.extend(_INCLUDE.findall(f.read()))
+    return sorted(seen)
+
+
+def kernel_source_hash(kernel=None):
+    """Hash of the code of the translation unit that defines `kernel` (and the
+    headers it includes), or of every kernel source without a kernel: comments
+    dropped and runs of white space collapsed, so that counters taken on a
+    kernel stay attributed to it while neither its code nor that of the
+    headers it includes changes."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_moe_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    tu = KERNEL_SOURCE.get(kernel) if kernel else None
+    names = _source_closure(tu, csrc) if tu else sorted(os.listdir(csrc))
+    for name in names:
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         code = _CODE_TOKENS.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
@@ -204,7 +233,7 @@ def ncu_traffic(kernel, workload):
         with open(path) as f:
             d = json.load(f)
         e = d[kernel][workload]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("source_hash") != kernel_source_hash(kernel):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:
@@ -219,7 +248,7 @@ def ncu_field(kernel, workload, field):
         with open(path) as f:
             d = json.load(f)
         e = d[kernel][workload]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("source_hash") != kernel_source_hash(kernel):
             return None
         return float(e[field])
     except Exception:

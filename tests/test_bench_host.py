@@ -40,6 +40,24 @@ def test_code_hash_ignores_comments(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() != h0
 
 
+def test_code_hash_per_kernel_follows_its_includes(tmp_path, monkeypatch):
+    """A kernel's hash covers its translation unit and the local headers it
+    includes, transitively, and nothing else."""
+    csrc = tmp_path / "bit_moe_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "step1.cu").write_text('#include "a.cuh"\n#include "bitmoe.h"\nint s = 1;\n')
+    (csrc / "a.cuh").write_text('#include "b.cuh"\nint a = 1;\n')
+    (csrc / "b.cuh").write_text("int b = 1;\n")
+    (csrc / "decode.cu").write_text("int d = 1;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0, d0, all0 = bench.kernel_source_hash("step1"), bench.kernel_source_hash("gateup"), bench.kernel_source_hash()
+    (csrc / "decode.cu").write_text("int d = 2;\n")
+    assert bench.kernel_source_hash("step1") == h0
+    assert bench.kernel_source_hash("gateup") != d0 and bench.kernel_source_hash() != all0
+    (csrc / "b.cuh").write_text("int b = 2;\n")
+    assert bench.kernel_source_hash("step1") != h0
+
+
 def test_cpu_baseline_reports_host_and_pinning():
     """The oracle's timed CPU baseline on the tiny layer: pinned to one core
     (the affinity is restored afterwards), median of 3 timings, and the host's
