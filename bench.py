@@ -111,6 +111,9 @@ def kernel_bytes(wl, unique_experts):
         # an fp16 scale per 32 weights, activations in and out
         Fs = wl.shared_ffn
         kb["shared"] = (3 * H * Fs * 34 // 32 + T * H * 5 // 4 + T * Fs * 5 // 2 + T * H * 8) / 2
+        # one token: the one-token step reads the shared expert's weights too
+        # (and publishes its blocks as tagged words)
+        kb["step1"] += 3 * H * Fs * 34 // 32 + Fs // 32 * 10 * 8 * 2
     return kb
 
 
@@ -480,18 +483,18 @@ def run_workload(B, wl, layers, routers, steps, warmup, dev, world, seed_off, do
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
     shared = build_shared(B, wl, L, dev, seed_off) if wl.shared_ffn else None
     if shared:
-        # x's int8 codes and scales that moe_forward leaves in its workspace
-        sxq, sxd = ws.act(layers[0], T)
         sws = shared[0].workspace(T, dev)
     torch.cuda.synchronize()
 
     def step(j):
-        B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
         if shared:
-            # the shared expert's FFN added to y, from the x^ of the step: the
-            # 8-bit gate/up with the requantization, then the down mat-vec
-            # with the add
-            shared[j % L].add(sxq, sxd, y, ws=sws)
+            # the routed experts and the shared expert's FFN: one launch for
+            # one token (the shared expert inside the one-token step), else
+            # the routed kernels, then the shared expert's gate/up with the
+            # requantization and its down mat-vec with the add into y
+            B.moe_forward_shared(layers[j % L], shared[j % L], routers[j % L], xs[j % NX], ws, sws, y=y)
+        else:
+            B.moe_forward(layers[j % L], routers[j % L], xs[j % NX], ws, y=y)
 
     for j in range(warmup):
         step(j)

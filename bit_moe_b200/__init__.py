@@ -36,7 +36,7 @@ EXPORTS = (
     "moe_check_status", "moe_last_error", "moe_debug_matvec", "moe_launch_count",
     "moe_trace_begin", "moe_trace_end", "moe_kernel_name", "moe_expert_ffn_decode_static",
     "moe_sign_words", "moe_quantize_weights_sign", "moe_e16_code_words", "moe_quantize_weights_e16",
-    "moe_quantize_weights_q8", "moe_shared_workspace_bytes", "moe_shared_ffn_add",
+    "moe_quantize_weights_q8", "moe_shared_workspace_bytes", "moe_shared_ffn_add", "moe_forward_shared",
     "moe_debug_ffn_blocksums", "moe_debug_wait_knob", "moe_workspace_act",
 )
 
@@ -102,6 +102,7 @@ def load_library(path):
         "moe_quantize_weights_q8": (ctypes.c_int, [p, i64, i64, p, p, p]),
         "moe_shared_workspace_bytes": (sz, [p, i32]),
         "moe_shared_ffn_add": (ctypes.c_int, [p, i32, p, p, p, p, sz, p]),
+        "moe_forward_shared": (ctypes.c_int, [p, p, p, i32, p, p, p, sz, p, sz, p]),
         "moe_quant_act_q8": (ctypes.c_int, [p, i32, i32, p, p, p]),
         "moe_route_topk": (ctypes.c_int, [p, p, i32, i32, i32, i32, p, p, p, sz, p]),
         "moe_route_workspace_bytes": (sz, [i32, i32]),
@@ -393,6 +394,20 @@ def moe_forward(layer, w_router, x, ws, y=None, stream=None):
     _check(lib().moe_forward(layer.c_ref(), _dev(w_router, torch.float32, "w_router"), ntok,
                              _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y"), ws.ptr(),
                              ws.nbytes, _stream(stream)))
+    return y
+
+
+def moe_forward_shared(layer, shared, w_router, x, ws, shared_ws=None, y=None, stream=None):
+    """y = the routed experts' sum plus the shared expert's FFN of x (one
+    launch for one token where the one-token step applies)."""
+    ntok = x.shape[0]
+    if y is None:
+        y = torch.empty((ntok, layer.hidden), dtype=torch.float32, device=x.device)
+    if shared_ws is None:
+        shared_ws = shared.workspace(ntok, x.device)
+    _check(lib().moe_forward_shared(layer.c_ref(), shared.c_ref(), _dev(w_router, torch.float32, "w_router"), ntok,
+                                    _dev(x, torch.float32, "x"), _dev(y, torch.float32, "y"), ws.ptr(), ws.nbytes,
+                                    ctypes.c_void_p(shared_ws.data_ptr()), shared_ws.numel(), _stream(stream)))
     return y
 
 

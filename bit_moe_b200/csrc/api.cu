@@ -71,6 +71,7 @@ int check_device() {
 struct WsLayout {
   size_t logits = 0, xq = 0, xd = 0, idx = 0, wts = 0, aq = 0, ad = 0, ye = 0, cnt = 0;
   size_t units = 0;       // tagged gate/up unit outputs of the one-token step
+  size_t sunits = 0;      // the same for a shared expert's blocks
   size_t xs = 0, ys = 0;  // device copies of x and y for the host-buffer entry point
   size_t bgu = 0, bdn = 0;  // prefill only
   GroupWs grp;
@@ -96,6 +97,7 @@ static WsLayout ws_layout(int H, int F, int E, int K, int T, bool prefill) {
   L.ye = take(sizeof(float) * T * static_cast<size_t>(K) * H);
   L.cnt = take(sizeof(int32_t) * T * static_cast<size_t>(H / kPanel));
   L.units = take(sizeof(unsigned long long) * K * static_cast<size_t>(F / kPanel) * (kPanel / 4 + 2));
+  L.sunits = take(sizeof(unsigned long long) * kMaxSharedUnits * (kPanel / 4 + 2));  // a shared expert's blocks
   L.xs = take(sizeof(float) * T * static_cast<size_t>(H));
   L.ys = take(sizeof(float) * T * static_cast<size_t>(H));
   off = group_ws_layout(E, T * K, off, &L.grp);
@@ -442,8 +444,13 @@ int moe_expert_ffn_prefill(const moe_layer* L, int32_t ntok, const int8_t* xq, c
   return launch_prefill(P, static_cast<cudaStream_t>(stream));
 }
 
-int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const float* x, float* y,
-                void* ws, size_t ws_bytes, moe_stream_t stream) {
+static int check_shared(const char* what, const moe_shared* S);
+
+// moe_forward, and with `shared` (one token, a shared expert the one-token
+// step takes) the shared expert in the same launch; *fused tells which.
+static int forward_impl(const moe_layer* L, const float* w_router, int32_t ntok, const float* x, float* y,
+                        void* ws, size_t ws_bytes, moe_stream_t stream, const SharedParams* shared, bool* fused) {
+  if (fused) *fused = false;
   int rc = check_layer(L);
   if (rc) return rc;
   if ((rc = check_ptrs("forward", w_router, x, y, ws))) return rc;
@@ -506,10 +513,44 @@ int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const f
   size_t smem1 = 0;
   if (step1_supported(P, D.n_sm, &smem1)) {
     WsHeader* hd = reinterpret_cast<WsHeader*>(ws);
+    if (shared && fused) *fused = true;
     return launch_step1(D, reinterpret_cast<unsigned long long*>(&hd->pad[3]),
-                        reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(ws) + W.units), s);
+                        reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(ws) + W.units), s,
+                        fused ? shared : nullptr,
+                        reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(ws) + W.sunits));
   }
   return launch_decode2(D, true, s);
+}
+
+int moe_forward(const moe_layer* L, const float* w_router, int32_t ntok, const float* x, float* y,
+                void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(L, w_router, ntok, x, y, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+int moe_forward_shared(const moe_layer* L, const moe_shared* S, const float* w_router, int32_t ntok,
+                       const float* x, float* y, void* ws, size_t ws_bytes, void* shared_ws,
+                       size_t sws_bytes, moe_stream_t stream) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if ((rc = check_shared("forward_shared", S))) return rc;
+  if ((rc = check_ptrs("forward_shared", w_router, x, y, ws, shared_ws))) return rc;
+  if (S->hidden != L->hidden)
+    return fail(MOE_ERR_INVALID_ARG, "forward_shared: shared expert hidden %d != layer hidden %d", S->hidden, L->hidden);
+  if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward_shared: 1 <= ntok <= 65536");
+  const size_t sneed = shared_ws_bytes(S->hidden, S->ffn, ntok);
+  if (sws_bytes < sneed)
+    return fail(MOE_ERR_WORKSPACE, "forward_shared: shared workspace %zu < %zu bytes", sws_bytes, sneed);
+  const SharedParams SP{S->hidden, S->ffn, S->gate_q, S->gate_d, S->up_q, S->up_d, S->down_q, S->down_d};
+  const bool fusable = ntok == 1 && S->ffn / kQBlock <= kMaxSharedUnits;
+  bool fused = false;
+  if ((rc = forward_impl(L, w_router, ntok, x, y, ws, ws_bytes, stream, fusable ? &SP : nullptr, &fused))) return rc;
+  if (fused) return MOE_OK;
+  // the shared expert's own kernels on the int8 x the step left in ws
+  const WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, ntok > kMaxDecodeTokens);
+  const unsigned char* base = static_cast<const unsigned char*>(ws);
+  return launch_shared_ffn_add(SP, ntok, reinterpret_cast<const int8_t*>(base + W.xq),
+                               reinterpret_cast<const float*>(base + W.xd), y, shared_ws,
+                               static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward_host(const moe_layer* L, const float* w_router, int32_t ntok, const float* x_host,

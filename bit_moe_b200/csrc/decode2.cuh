@@ -40,8 +40,12 @@ int launch_route_only(Decode2Params& D, cudaStream_t stream);
 bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem);
 // `ticket`: a 64-bit counter that only grows; `units`: top_k * (ffn / 32) * 10
 // 8-byte words for the tagged gate/up unit outputs; the logits area of D must
-// hold 128 bytes per expert (tagged logits).
+// hold 128 bytes per expert (tagged logits).  With `shared` (hidden equal to
+// the layer's, ffn a multiple of 32 of at most kMaxSharedUnits blocks) the
+// same launch adds the shared expert's FFN to y; `sunits` then holds
+// (ffn / 32) * 10 words for its tagged block outputs.
+struct SharedParams;
 int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned long long* units,
-                 cudaStream_t stream);
+                 cudaStream_t stream, const SharedParams* shared = nullptr, unsigned long long* sunits = nullptr);
 
 }  // namespace bitmoe

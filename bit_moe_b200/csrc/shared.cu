@@ -40,32 +40,6 @@ __global__ void k_quantize_weights_q8(const float* __restrict__ w, int64_t nblk,
   }
 }
 
-// Row r of an 8-bit matrix [rows][k] against activation codes xq [k] with
-// scales xd [k/32]: sum over blocks of d_w * d_a * (exact int32 block sum),
-// the same value in every lane.
-__device__ __forceinline__ float q8_row_dot(const int8_t* __restrict__ q, const uint16_t* __restrict__ d, int k,
-                                            const int8_t* __restrict__ xq, const float* __restrict__ xd, int lane) {
-  float acc = 0.f;
-  for (int j = lane; j < k / kQBlock; j += 32) {
-    const int4* wq = reinterpret_cast<const int4*>(q + static_cast<size_t>(j) * kQBlock);
-    const int4* aq = reinterpret_cast<const int4*>(xq + static_cast<size_t>(j) * kQBlock);
-    const int4 w0 = wq[0], w1 = wq[1], a0 = aq[0], a1 = aq[1];
-    int s = __dp4a(w0.x, a0.x, 0);
-    s = __dp4a(w0.y, a0.y, s);
-    s = __dp4a(w0.z, a0.z, s);
-    s = __dp4a(w0.w, a0.w, s);
-    s = __dp4a(w1.x, a1.x, s);
-    s = __dp4a(w1.y, a1.y, s);
-    s = __dp4a(w1.z, a1.z, s);
-    s = __dp4a(w1.w, a1.w, s);
-    const float sc = __fmul_rn(f16_bits_to_f32(d[j]), xd[j]);
-    acc = __fmaf_rn(sc, static_cast<float>(s), acc);
-  }
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, m));
-  return acc;
-}
-
 // a[t][f] = silu(gate_f . x^_t) * (up_f . x^_t) for every token and row f of
 // the shared ffn, requantized in the same kernel: a CTA of 32 warps takes one
 // 32-row block of the shared ffn (one row per warp), puts the block's a
@@ -90,8 +64,8 @@ __global__ void __launch_bounds__(kSharedBlockWarps * 32) k_shared_gateup_q(Shar
     for (int t = 0; t < ntok; ++t) {
       const int8_t* xt = xq + static_cast<size_t>(t) * H;
       const float* dt = xd + static_cast<size_t>(t) * (H / kQBlock);
-      const float g = q8_row_dot(gq, gd, H, xt, dt, lane);
-      const float u = q8_row_dot(uq, ud, H, xt, dt, lane);
+      float g, u;
+      q8_row_dot2(gq, gd, uq, ud, H, xt, dt, lane, g, u);
       if (lane == 0) sa[warp] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
       __syncthreads();
       if (warp == 0) quant_act_block(sa, 0, lane, aq + static_cast<size_t>(t) * F + blk * kQBlock,

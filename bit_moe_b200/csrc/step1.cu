@@ -36,6 +36,7 @@
 #include "decode2.cuh"
 #include "matvec.cuh"
 #include "ptx.cuh"
+#include "shared.cuh"
 #include "topk.cuh"
 
 namespace bitmoe {
@@ -68,10 +69,14 @@ struct Step1Params {
   unsigned long long* ticket;  // launch ticket counter (only grows): generation = ticket / CTAs
   unsigned long long* tagged;  // [E][kTagStride] logits as (generation + 1) << 32 | fp32 bits
   unsigned long long* units;   // [top_k][ffn/32][kUnitWords] unit outputs, tagged the same way
+  // the shared expert (kShared): its 32-row blocks of the shared ffn are
+  // units after the routed ones, published to sunits [ffn_s/32][kUnitWords]
+  SharedParams S;
+  unsigned long long* sunits;
 };
 
 struct Step1Layout {
-  size_t ring, pref, xq4, xd, xas, sel, red, flag, rbar, xf, act, inner, total;
+  size_t ring, pref, xq4, xd, xas, sel, red, flag, rbar, shr, xf, act, inner, total;
   int sw;  // ring slots per warp
 };
 
@@ -95,7 +100,10 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, 
     const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
     const size_t inner = static_cast<size_t>(2) * K * (F / kBlock) * kPanel * 4;
     if (ring < xf) ring = xf;
-    if (ring < act + inner) ring = act + inner;
+    // phase C also keeps a shared expert's block codes and scales after the
+    // inner sums
+    const size_t scodes = static_cast<size_t>(kMaxSharedUnits) * (kPanel / 4 + 1) * 4;
+    if (ring < act + inner + scodes) ring = act + inner + scodes;
     L.ring = take(ring);
     L.act = L.ring;
     L.inner = L.ring + act;
@@ -110,6 +118,7 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, 
     L.red = take(static_cast<size_t>(kS1Streams) * 2 * kNC * 32 * 4);
     L.flag = take(64);
     L.rbar = take(static_cast<size_t>(kS1Warps) * 3 * 8);
+    L.shr = take(static_cast<size_t>(kS1Streams + 1) * 32 * 4);  // shared expert: a of a block per stream, down rows
     L.total = off;
     if (L.total <= static_cast<size_t>(kMaxDynSmem)) break;
   }
@@ -127,6 +136,12 @@ __device__ __forceinline__ void stream_bar_arrive(int id) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "n"(kNC * 32) : "memory");
 }
 
+// Bring a range of global memory into L2 (16-byte aligned, a multiple of 16
+// bytes), without waiting for it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Bounded polls of values another CTA publishes.
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
   unsigned long long v;
@@ -139,8 +154,13 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
 
 // kSign: the weights are 1-bit sign codes (else base-3 digits).  kSlotOrder:
 // the down items go to the warps in slot order (at most two items per warp),
-// else by halves of a slot.
-template <bool kSign, bool kSlotOrder>
+// else by halves of a slot.  kShared: the layer's shared expert (8-bit
+// blocks) is computed in the same launch: its 32-row blocks of the shared
+// ffn are gate/up units after the routed ones (on the streams the routed
+// units leave idle), and the CTAs with a panel of hidden add the panel's
+// rows of its down projection to y after the routed combine, with the
+// arithmetic of the shared expert's own kernels.
+template <bool kSign, bool kSlotOrder, bool kShared>
 __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   constexpr int kWBytes = s1_word_bytes(kSign), kMat = s1_mat_bytes(kSign);
   constexpr int kWords = kSign ? kSignWords : kBlockWords;
@@ -184,6 +204,23 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     cp16(reinterpret_cast<unsigned char*>(rows) + q * 16,
          reinterpret_cast<const unsigned char*>(D.wr + static_cast<size_t>(e0) * H) + q * 16);
   cp_commit();
+  if constexpr (kShared) {
+    // the shared expert's gate/up blocks this CTA will compute: into L2 now
+    // (caller data, like the router rows)
+    if (tid == 0) {
+      const int64_t U = static_cast<int64_t>(K) * (F / kPanel), Us = S1.S.ffn / kQBlock;
+      for (int64_t q = 0;; ++q) {
+        const int64_t u = q == 0 ? static_cast<int64_t>(c) : q * C + (C - 1 - c);
+        if (u >= U + Us) break;
+        if (u < U) continue;
+        const int64_t f0 = (u - U) * kQBlock;
+        bulk_prefetch_l2(S1.S.gate_q + f0 * H, static_cast<uint32_t>(kQBlock * H));
+        bulk_prefetch_l2(S1.S.up_q + f0 * H, static_cast<uint32_t>(kQBlock * H));
+        bulk_prefetch_l2(S1.S.gate_d + f0 * (H / kQBlock), static_cast<uint32_t>(2 * H));
+        bulk_prefetch_l2(S1.S.up_d + f0 * (H / kQBlock), static_cast<uint32_t>(2 * H));
+      }
+    }
+  }
 
   // launched as a programmatic dependent: everything the kernels before it
   // wrote (x among them) is visible only past this wait
@@ -319,8 +356,11 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     auto unit_of = [&](int q) -> int64_t {
       return q == 0 ? static_cast<int64_t>(c) : static_cast<int64_t>(q) * C + (C - 1 - c);
     };
-    int nmine = 0;
+    int nmine = 0;  // routed units; the shared expert's units come after them
     while (unit_of(kS1Streams * nmine + h) < U) ++nmine;
+    int nshared = 0;
+    if constexpr (kShared)
+      while (unit_of(kS1Streams * (nmine + nshared) + h) < U + S1.S.ffn / kQBlock) ++nshared;
     auto my_unit = [&](int i) { return unit_of(kS1Streams * i + h); };
     unsigned char* myring = smem + L.ring + static_cast<size_t>(warp) * SW * kSlotBytes;
     float* rb = reinterpret_cast<float*>(smem + L.red) + h * (2 * kNC * 32);
@@ -367,6 +407,15 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       mbar_arrive_expect_tx(pbar, tb + sb);
       bulk_g2s(dst, P.down_trits + pb0 * kWords * kPanel, tb, pbar, policy_evict_first());
       bulk_g2s(dst + tb, P.down_scales + pb0 * kPanel, sb, pbar, policy_evict_first());
+    }
+    if constexpr (kShared) {
+      // this panel's rows of the shared expert's down projection, for phase C
+      if (has_panel && tid == 0) {
+        const int Fs = S1.S.ffn;
+        bulk_prefetch_l2(S1.S.down_q + static_cast<size_t>(panelH) * kPanel * Fs, static_cast<uint32_t>(kPanel * Fs));
+        bulk_prefetch_l2(S1.S.down_d + static_cast<size_t>(panelH) * kPanel * (Fs / kQBlock),
+                         static_cast<uint32_t>(2 * Fs));
+      }
     }
     int s = 0;
     for (int ui = 0; ui < nmine; ++ui) {
@@ -424,6 +473,43 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
                                  : lane == kPanel / 4 ? __float_as_uint(dd) : static_cast<uint32_t>(qs);
         if (lane < kUnitWords)
           st_relaxed_u64(S1.units + (static_cast<size_t>(j) * panels + p) * kUnitWords + lane, tag64 | payload);
+      }
+    }
+    if constexpr (kShared) {
+      // the shared expert's units of this stream: warp w8 takes rows w8,
+      // w8 + 8, ... of the 32-row block (one row per warp, as the shared
+      // expert's own gate/up kernel), then warp 0 of the stream requantizes
+      // the block and publishes it like a routed unit
+      float* ssa = reinterpret_cast<float*>(smem + L.shr) + h * kQBlock;
+      const int8_t* xq8 = reinterpret_cast<const int8_t*>(sq4);
+      const int bar_sh = 1 + 2 * kS1Streams + h;
+      for (int si = 0; si < nshared; ++si) {
+        const int64_t su = my_unit(nmine + si) - U;
+        for (int r = w8; r < kQBlock; r += kNC) {
+          const int64_t f = su * kQBlock + r;
+          float g, u;
+          q8_row_dot2(S1.S.gate_q + f * H, S1.S.gate_d + f * (H / kQBlock), S1.S.up_q + f * H,
+                      S1.S.up_d + f * (H / kQBlock), H, xq8, sxd, lane, g, u);
+          if (lane == 0) ssa[r] = __fmul_rn(__fdiv_rn(g, __fadd_rn(1.f, expf(-g))), u);
+        }
+        stream_bar_sync(bar_sh);
+        if (w8 == 0) {
+          const float a = ssa[lane];
+          const float amax = warp_max(fabsf(a));
+          const float dd = __fdiv_rn(amax, 127.f);
+          int q = 0;
+          if (dd != 0.f) q = max(-127, min(127, __float2int_rn(__fdiv_rn(a, dd))));
+          const int qs = __reduce_add_sync(0xffffffffu, q);
+          const uint32_t qb = static_cast<uint32_t>(q) & 0xffu;
+          const uint32_t w4 = qb | (__shfl_down_sync(0xffffffffu, qb, 1) << 8) |
+                              (__shfl_down_sync(0xffffffffu, qb, 2) << 16) |
+                              (__shfl_down_sync(0xffffffffu, qb, 3) << 24);
+          const uint32_t cw = __shfl_sync(0xffffffffu, w4, (4 * lane) & 31);
+          const uint32_t payload = lane < kPanel / 4 ? cw
+                                   : lane == kPanel / 4 ? __float_as_uint(dd) : static_cast<uint32_t>(qs);
+          if (lane < kUnitWords) st_relaxed_u64(S1.sunits + su * kUnitWords + lane, tag64 | payload);
+        }
+        stream_bar_sync(bar_sh);
       }
     }
     // every copy issued was consumed above: none is in flight here
@@ -600,6 +686,88 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         }
       }
     }
+    float* ssv = reinterpret_cast<float*>(smem + L.shr) + kS1Streams * kQBlock;  // [32] shared down rows
+    if constexpr (kShared) {
+      // the panel's 32 rows of the shared expert's down projection on warps
+      // kNC.. (four rows each), lane j taking the shared ffn's 32-blocks j,
+      // j + 32, ... as the shared expert's own down kernel does.  Block j's
+      // codes and scale are the tagged words of shared unit j; one warp polls
+      // them (a warp per CTA, not eight: the units are few lines of L2 that
+      // every CTA reads) into the ring area past the inner sums.  Warps kNC..
+      // start as soon as their down items are done (in slot order they hold
+      // fewer), before the CTA-wide barrier.
+      if (ok && warp >= kNC) {
+        const int Fs = S1.S.ffn, nbs = Fs / kQBlock;
+        int* saq = reinterpret_cast<int*>(smem + L.inner + static_cast<size_t>(2) * K * nbF * kPanel * 4);  // [nbs][8]
+        float* sad = reinterpret_cast<float*>(saq + kMaxSharedUnits * (kPanel / 4));                      // [nbs]
+        if (warp == kNC && !*abort) {
+          const uint32_t tag = *sgen;
+          for (int j0 = 0; j0 < nbs; j0 += 32) {
+            const int jb = j0 + lane;
+            const uint32_t need = jb < nbs ? (1u << (kPanel / 4 + 1)) - 1u : 0u;  // 8 code words and the scale
+            const unsigned long long* src = S1.sunits + static_cast<size_t>(jb) * kUnitWords;
+            unsigned long long wv[kPanel / 4 + 1];
+            uint32_t ready = 0;
+            for (uint32_t polls = 0;; ++polls) {
+#pragma unroll
+              for (int i = 0; i <= kPanel / 4; ++i)
+                if ((need & ~ready) & (1u << i)) wv[i] = ld_relaxed_u64(src + i);
+#pragma unroll
+              for (int i = 0; i <= kPanel / 4; ++i)
+                if (((need & ~ready) & (1u << i)) && static_cast<uint32_t>(wv[i] >> 32) == tag) ready |= 1u << i;
+              if (__all_sync(0xffffffffu, ready == need) || polls > kSpinLimit) break;
+            }
+            if (!__all_sync(0xffffffffu, ready == need)) {
+              if (lane == 0) {
+                record_status(P.status, MOE_ERR_TIMEOUT);
+                *abort = 1;
+              }
+              break;
+            }
+            if (jb < nbs) {
+#pragma unroll
+              for (int i = 0; i < kPanel / 4; ++i) saq[jb * (kPanel / 4) + i] = static_cast<int>(wv[i]);
+              sad[jb] = __uint_as_float(static_cast<uint32_t>(wv[kPanel / 4]));
+            }
+          }
+        }
+        stream_bar_sync(1 + 3 * kS1Streams);  // warps kNC.. (the shared codes are in place)
+        if (!*abort) {
+          constexpr int kRows = kPanel / (kS1Warps - kNC);
+          float acc[kRows];
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) acc[i] = 0.f;
+          for (int jb = lane; jb < nbs; jb += 32) {
+            const int4 a0 = reinterpret_cast<const int4*>(saq + jb * (kPanel / 4))[0];
+            const int4 a1 = reinterpret_cast<const int4*>(saq + jb * (kPanel / 4))[1];
+            const float ad = sad[jb];
+#pragma unroll
+            for (int i = 0; i < kRows; ++i) {
+              const size_t hrow = static_cast<size_t>(panelH) * kPanel + (warp - kNC) + (kS1Warps - kNC) * i;
+              const int4* wq = reinterpret_cast<const int4*>(S1.S.down_q + hrow * Fs + static_cast<size_t>(jb) * kQBlock);
+              const int4 w0 = wq[0], w1 = wq[1];
+              int sd = __dp4a(w0.x, a0.x, 0);
+              sd = __dp4a(w0.y, a0.y, sd);
+              sd = __dp4a(w0.z, a0.z, sd);
+              sd = __dp4a(w0.w, a0.w, sd);
+              sd = __dp4a(w1.x, a1.x, sd);
+              sd = __dp4a(w1.y, a1.y, sd);
+              sd = __dp4a(w1.z, a1.z, sd);
+              sd = __dp4a(w1.w, a1.w, sd);
+              const float sc = __fmul_rn(f16_bits_to_f32(S1.S.down_d[hrow * nbs + jb]), ad);
+              acc[i] = __fmaf_rn(sc, static_cast<float>(sd), acc[i]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < kRows; ++i) {
+            float v = acc[i];
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, m));
+            if (lane == 0) ssv[(warp - kNC) + (kS1Warps - kNC) * i] = v;
+          }
+        }
+      }
+    }
     __syncthreads();
     // warp j applies slot j's block scales in order, then warp 0 combines
     // the slots in order (the summation order of the grouped down kernel)
@@ -614,6 +782,7 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     if (!*abort && ok && warp == 0) {
       float y = 0.f;
       for (int jj = 0; jj < K; ++jj) y = __fmaf_rn(sel_w[jj], spart[jj * kPanel + lane], y);
+      if constexpr (kShared) y = __fadd_rn(y, ssv[lane]);  // after the routed combine, as the shared kernel adds it
       P.y[panelH * kPanel + lane] = y;
     }
   }
@@ -631,20 +800,29 @@ bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem) {
 }
 
 int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned long long* units,
-                 cudaStream_t stream) {
+                 cudaStream_t stream, const SharedParams* shared, unsigned long long* sunits) {
   static std::atomic<bool> done[64];  // the attribute call is idempotent
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !done[dev].load(std::memory_order_relaxed)) {
-    cudaFuncSetAttribute(k_step1<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_step1<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_step1<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-    cudaFuncSetAttribute(k_step1<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+    const void* ks[] = {reinterpret_cast<const void*>(&k_step1<false, false, false>),
+                        reinterpret_cast<const void*>(&k_step1<true, false, false>),
+                        reinterpret_cast<const void*>(&k_step1<false, true, false>),
+                        reinterpret_cast<const void*>(&k_step1<true, true, false>),
+                        reinterpret_cast<const void*>(&k_step1<false, false, true>),
+                        reinterpret_cast<const void*>(&k_step1<true, false, true>),
+                        reinterpret_cast<const void*>(&k_step1<false, true, true>),
+                        reinterpret_cast<const void*>(&k_step1<true, true, true>)};
+    for (const void* k : ks) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     done[dev].store(true, std::memory_order_relaxed);
   }
   size_t smem = 0;
   if (!step1_supported(D.P, D.n_sm, &smem)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "step1: unsupported shape");
-  Step1Params S{D, ticket, reinterpret_cast<unsigned long long*>(D.logits), units};
+  if (shared && (shared->hidden != D.P.hidden || shared->ffn <= 0 || shared->ffn % kQBlock ||
+                 shared->ffn / kQBlock > kMaxSharedUnits || !sunits))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "step1: unsupported shared expert");
+  Step1Params S{D, ticket, reinterpret_cast<unsigned long long*>(D.logits), units, SharedParams{}, sunits};
+  if (shared) S.S = *shared;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(D.n_sm);
   cfg.blockDim = dim3(kS1Warps * 32);
@@ -664,8 +842,10 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   cfg.numAttrs = pdl_ok[di] >= 0 ? 2 : 1;
   const bool sign = D.P.format == MOE_FORMAT_SIGN;
   const bool slot_order = D.P.top_k * (D.P.ffn / kBlock) <= 2 * kS1Warps;
-  auto kern = sign ? (slot_order ? k_step1<true, true> : k_step1<true, false>)
-                   : (slot_order ? k_step1<false, true> : k_step1<false, false>);
+  auto kern = shared ? (sign ? (slot_order ? k_step1<true, true, true> : k_step1<true, false, true>)
+                             : (slot_order ? k_step1<false, true, true> : k_step1<false, false, true>))
+                      : (sign ? (slot_order ? k_step1<true, true, false> : k_step1<true, false, false>)
+                              : (slot_order ? k_step1<false, true, false> : k_step1<false, false, false>));
   cudaError_t err = cudaLaunchKernelEx(&cfg, kern, S);
   if (err != cudaSuccess && cfg.numAttrs == 2 && pdl_ok[di] == 0) {
     cudaGetLastError();

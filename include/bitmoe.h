@@ -274,6 +274,24 @@ size_t moe_shared_workspace_bytes(const moe_shared* shared, int32_t ntok);
  * scratch of moe_shared_workspace_bytes bytes.                             */
 int moe_shared_ffn_add(const moe_shared* shared, int32_t ntok, const int8_t* xq, const float* xd,
                        float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
+/* y [ntok][hidden] = the routed experts' sum (moe_forward) plus the shared
+ * expert's FFN, bit for bit what moe_forward followed by moe_shared_ffn_add
+ * on the int8 x that moe_forward leaves in ws (moe_workspace_act) gives.
+ * One token of a layer whose one-token step applies (moe_forward launches
+ * k_step1) with a shared ffn of at most 64 blocks of 32 rows runs as that one
+ * launch: the shared expert's 32-row gate/up blocks are units after the
+ * routed ones (their weights prefetched into L2 at the start), published with
+ * the step's tagged words, and each CTA with a 32-row panel of hidden adds
+ * the panel's rows of the shared down projection to y after the routed
+ * combine.  Any other call runs moe_forward, then moe_shared_ffn_add's
+ * kernels.  ws: moe_workspace_bytes(layer, ntok) bytes; shared_ws:
+ * moe_shared_workspace_bytes(shared, ntok) bytes; shared->hidden must equal
+ * layer->hidden (MOE_ERR_INVALID_ARG otherwise).  Errors as moe_forward and
+ * moe_shared_ffn_add.  (llama-modchip page, "The interesting bit": the
+ * shared expert beside the routed ones.)                                   */
+int moe_forward_shared(const moe_layer* layer, const moe_shared* shared, const float* w_router,
+                       int32_t ntok, const float* x, float* y, void* ws, size_t ws_bytes,
+                       void* shared_ws, size_t shared_ws_bytes, moe_stream_t stream);
 
 /* ---- status ------------------------------------------------------------- */
 /* Synchronizes `stream`, returns the status recorded in the workspace by

@@ -90,3 +90,62 @@ def test_workspace_act_is_the_step_quantization(wl_name, ntok):
     xq, xd = B.moe_quant_act_q8(x)
     assert np.array_equal(wq.cpu().numpy(), xq.cpu().numpy())
     assert np.array_equal(wd.cpu().numpy().view(np.uint32), xd.cpu().numpy().view(np.uint32))
+
+
+def _names(B, fn):
+    tr = B.KernelTrace(capacity=64)
+    with tr:
+        fn()
+    torch.cuda.synchronize()
+    return [B.lib().moe_kernel_name(i).decode() for i in tr.ids]
+
+
+@pytest.mark.parametrize("wl_name,fmt,ntok,Fs", [
+    ("30b", "ternary", 1, 768),     # slot-order down items, 24 shared blocks
+    ("tiny", "ternary", 1, 256),
+    ("tiny", "sign", 1, 2048),      # the most shared blocks the step takes (64)
+    ("large", "ternary", 1, 1024),  # half-slot down items
+    ("30b", "sign", 1, 96),
+    ("30b", "ternary", 3, 768),     # more tokens: the routed kernels, then the shared expert's
+    ("tiny", "ternary", 1, 2080),   # more than 64 blocks: moe_forward, then the shared expert's
+])
+def test_forward_shared_equals_forward_then_shared_add(wl_name, fmt, ntok, Fs):
+    """moe_forward_shared gives, bit for bit, moe_forward followed by the
+    shared expert's add on the int8 x the step leaves in the workspace; one
+    token of a layer the one-token step takes is one launch."""
+    B = bm()
+    wl = synthetic.WORKLOADS[wl_name]
+    H = wl.hidden
+    layer, _ = gpu_layer(wl, fmt=fmt)
+    wr = synthetic.router(wl, 0, "cuda")
+    wg, wu, wd = _shared_weights(H, Fs, 91 + Fs)
+    sh = B.SharedExpert(torch.from_numpy(wg).cuda(), torch.from_numpy(wu).cuda(), torch.from_numpy(wd).cuda())
+    ws = B.Workspace.for_layer(layer, ntok)
+    ws2 = B.Workspace.for_layer(layer, ntok)
+    sws = sh.workspace(ntok)
+    fused = ntok == 1 and Fs // 32 <= 64
+    for seed in range(3):
+        x = synthetic.activations(wl, 300 + seed, ntok=ntok, device="cuda")
+        y1 = torch.empty((ntok, H), device="cuda")
+        names = _names(B, lambda: B.moe_forward_shared(layer, sh, wr, x, ws, sws, y=y1))
+        if fused:
+            assert names == ["step1"]
+        else:
+            assert names[-2:] == ["shared", "shared"]
+        y2 = B.moe_forward(layer, wr, x, ws2)
+        xq, xd = ws2.act(layer, ntok)
+        sh.add(xq, xd, y2)
+        assert B.moe_check_status(ws) == 0 and B.moe_check_status(ws2) == 0
+        assert torch.equal(y1, y2), (wl_name, fmt, ntok, Fs, seed)
+
+
+def test_forward_shared_refuses_a_hidden_mismatch():
+    B = bm()
+    wl = synthetic.WORKLOADS["tiny"]
+    layer, _ = gpu_layer(wl)
+    wr = synthetic.router(wl, 0, "cuda")
+    wg, wu, wd = _shared_weights(512, 64, 5)
+    sh = B.SharedExpert(torch.from_numpy(wg).cuda(), torch.from_numpy(wu).cuda(), torch.from_numpy(wd).cuda())
+    x = synthetic.activations(wl, 1, ntok=1, device="cuda")
+    with pytest.raises(RuntimeError):
+        B.moe_forward_shared(layer, sh, wr, x, B.Workspace.for_layer(layer, 1))
