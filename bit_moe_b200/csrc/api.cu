@@ -456,10 +456,10 @@ static int forward_impl(const moe_layer* L, const float* w_router, int32_t ntok,
   if ((rc = check_ptrs("forward", w_router, x, y, ws))) return rc;
   if (ntok <= 0 || ntok > 65536) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "forward: 1 <= ntok <= 65536");
   const bool prefill = ntok > kMaxDecodeTokens;
-  // layers whose one token does not take the fused one-token step: two-level
-  // scales, and sign codes of shapes the step does not fit (ternary layers
-  // of such shapes take the first-version one-token chain below)
-  bool chain1 = L->gate.format == MOE_FORMAT_E16;
+  // layers whose one token does not take the fused one-token step: sign
+  // codes and two-level scales of shapes the step does not fit (ternary
+  // layers of such shapes take the first-version one-token chain below)
+  bool chain1 = false;
   WsLayout W = ws_layout(L->hidden, L->ffn, L->n_experts, L->top_k, ntok, prefill);
   if (ws_bytes < W.total) return fail(MOE_ERR_WORKSPACE, "forward: workspace %zu < %zu bytes", ws_bytes, W.total);
   if ((rc = check_device())) return rc;
@@ -471,12 +471,12 @@ static int forward_impl(const moe_layer* L, const float* w_router, int32_t ntok,
   float* wts = reinterpret_cast<float*>(base + W.wts);
   float* logits = reinterpret_cast<float*>(base + W.logits);
   DecodeParams P = make_params(L, ntok, xq, xd, idx, wts, y, ws, W);
-  if (ntok == 1 && L->gate.format == MOE_FORMAT_SIGN) {
+  if (ntok == 1 && L->gate.format != MOE_FORMAT_TERNARY) {
     size_t smem_s = 0;
     chain1 = !step1_supported(P, sm_count(), &smem_s);
   }
   if ((ntok > 1 || chain1) && !prefill && route_group_ok(P, sm_count())) {
-    // few tokens (and one token of an E16 layer): router logits, activation
+    // few tokens (and one token the fused step does not take): router logits, activation
     // quantization, top-k and grouping in one launch, then the grouped
     // mat-vecs
     WsHeader* hd = reinterpret_cast<WsHeader*>(ws);

@@ -225,6 +225,77 @@ __device__ __forceinline__ void block_dot(const unsigned char* __restrict__ wsrc
   }
 }
 
+// Two-level scales (E16) of one block for one vector: NM matrices' base-3
+// words at wsrc + m * mat_stride and their 4-bit sub-scale code words
+// (kE16Words per row) code_off bytes after each matrix's words.  accw[m][s]
+// receives, per 32-weight sub-block s, the exact integer sum over its two
+// 16-weight halves h of (c_h + 1) * (sum(t * a) - sum(a)) -- the integer the
+// grouped E16 kernels multiply by the activation scale of sub-block s; the
+// caller chains those products in the kernels' order.
+template <int NM>
+__device__ __forceinline__ void block_isums_e16(const unsigned char* __restrict__ wsrc, int mat_stride,
+                                                int code_off, const int* __restrict__ q4, int lane,
+                                                int (&accw_out)[NM][kSubPerBlock]) {
+  uint32_t w[NM][kBlockWords];
+  uint32_t cw[NM][kE16Words];
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const uint32_t* tw = reinterpret_cast<const uint32_t*>(wsrc + m * mat_stride);
+    const uint32_t* tc = reinterpret_cast<const uint32_t*>(wsrc + m * mat_stride + code_off);
+#pragma unroll
+    for (int j = 0; j < kBlockWords; ++j) w[m][j] = tw[j * kPanel + lane];
+#pragma unroll
+    for (int u = 0; u < kE16Words; ++u) cw[m][u] = tc[u * kPanel + lane];
+  }
+  int acc[NM], accw[NM];
+  int as16 = 0;
+#pragma unroll
+  for (int m = 0; m < NM; ++m) { acc[m] = 0; accw[m] = 0; }
+#pragma unroll
+  for (int j = 0; j < kBlockWords; ++j) {
+    uint32_t lo[NM], hi[NM], hp[NM];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) {
+      lo[m] = w[m][j] & 0x00FF00FFu;
+      hi[m] = __byte_perm(w[m][j], 0u, 0x4341);  // bytes 1, 3 into 16-bit lanes
+      hp[m] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      if (j == kBlockWords - 1 && i == 4) break;  // pad digit of the last word
+      const int g = 5 * j + i;                    // group of 4 weights, 0..63
+      const int a = q4[g];
+      as16 = __dp4a(a, 0x01010101, as16);
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        lo[m] *= 3u;
+        hi[m] *= 3u;
+        const uint32_t hn = __byte_perm(lo[m], hi[m], 0x7351);
+        const int t = static_cast<int>(hn - 3u * hp[m]);
+        hp[m] = hn;
+        acc[m] = __dp4a(t, a, acc[m]);
+      }
+      if ((g & 3) == 3) {  // a 16-weight half is complete
+        const int h = g >> 2;
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+          const int cm = static_cast<int>((cw[m][h >> 3] >> (4 * (h & 7))) & 15u) + 1;
+          accw[m] += cm * (acc[m] - as16);
+          acc[m] = 0;
+        }
+        as16 = 0;
+      }
+      if ((g & 7) == 7) {  // a 32-weight sub-block is complete
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+          accw_out[m][g >> 3] = accw[m];
+          accw[m] = 0;
+        }
+      }
+    }
+  }
+}
+
 // The same for one vector over 1-bit sign codes (kSignWords words per
 // block, word j = activation block j, weight 32j + 4i + l in bit 8l + i):
 // per sub-block the exact sum(q * a) = 2 * sum(t * a) - sum(a), scaled and

@@ -27,9 +27,10 @@
 // experts evaluated); pxq_llama README, "Updates -- 2026-07-28" (gate/up with
 // the SiLU unary).  The numerics are those of the decode kernels.  The same
 // kernel takes 1-bit sign codes (pxq_llama README, "What's PXQ?", the PXQ1
-// tier) with their block decode; two-level scales keep one fp32 chain over
-// every block of a down row, which phase C's split of the blocks over two
-// warps cannot reproduce, so they take the four-kernel chain.
+// tier) with their block decode, and two-level scales (an fp16 anchor per row,
+// a 4-bit sub-scale per 16 weights): their down rows keep one fp32 chain over
+// every sub-block, so phase C's items leave the blocks' exact integer sums
+// and one warp per slot chains them in order.
 #include <atomic>
 #include "bitmoe.h"
 #include "common.cuh"
@@ -60,9 +61,19 @@ static_assert(kS1MaxK <= kNC, "phase C: one warp per slot");
 constexpr int kUnitWords = kPanel / 4 + 2;
 
 // Bytes of one 256-weight block of a 32-row panel: packed words, then the
-// 32 fp16 scales (base-3 digits, or 1-bit sign codes).
-__host__ __device__ constexpr int s1_word_bytes(bool sign) { return (sign ? kSignWords : kBlockWords) * kPanel * 4; }
-__host__ __device__ constexpr int s1_mat_bytes(bool sign) { return s1_word_bytes(sign) + kPanel * 2; }
+// 32 fp16 scales (base-3 digits, or 1-bit sign codes), or for two-level
+// scales the rows' 4-bit sub-scale code words (their per-row fp16 anchors
+// come once per panel).
+__host__ __device__ constexpr int s1_word_bytes(int fmt) {
+  return (fmt == MOE_FORMAT_SIGN ? kSignWords : kBlockWords) * kPanel * 4;
+}
+__host__ __device__ constexpr int s1_tail_bytes(int fmt) {
+  return fmt == MOE_FORMAT_E16 ? kE16Words * kPanel * 4 : kPanel * 2;
+}
+__host__ __device__ constexpr int s1_mat_bytes(int fmt) { return s1_word_bytes(fmt) + s1_tail_bytes(fmt); }
+// Per-block results phase C keeps in shared memory: the inner sum and the
+// weight scale, or for two-level scales the 8 sub-blocks' integer sums.
+__host__ __device__ constexpr int s1_item_words(int fmt) { return fmt == MOE_FORMAT_E16 ? kSubPerBlock : 2; }
 
 struct Step1Params {
   Decode2Params D;
@@ -84,7 +95,7 @@ struct Step1Layout {
 // activations alias the gate/up ring (which is used only between them); the
 // router rows alias the down prefetch area.  Three ring slots per warp where
 // they fit, else two.
-__host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, bool sign) {
+__host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, int fmt) {
   Step1Layout L{};
   for (int sw = 3; sw >= 2; --sw) {
     L = Step1Layout{};
@@ -95,10 +106,10 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, 
       off = (off + bytes + 127) / 128 * 128;
       return o;
     };
-    size_t ring = static_cast<size_t>(kS1Warps) * sw * 2 * s1_mat_bytes(sign);
+    size_t ring = static_cast<size_t>(kS1Warps) * sw * 2 * s1_mat_bytes(fmt);
     const size_t xf = static_cast<size_t>(H) * 4;
     const size_t act = static_cast<size_t>(K) * (F + 2 * (F / kQBlock) * 4);
-    const size_t inner = static_cast<size_t>(2) * K * (F / kBlock) * kPanel * 4;
+    const size_t inner = static_cast<size_t>(s1_item_words(fmt)) * K * (F / kBlock) * kPanel * 4;
     if (ring < xf) ring = xf;
     // phase C also keeps a shared expert's block codes and scales after the
     // inner sums
@@ -108,7 +119,7 @@ __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, 
     L.act = L.ring;
     L.inner = L.ring + act;
     L.xf = L.ring;
-    const size_t pref = static_cast<size_t>(K) * (F / kBlock) * s1_mat_bytes(sign);
+    const size_t pref = static_cast<size_t>(K) * ((F / kBlock) * s1_mat_bytes(fmt) + (fmt == MOE_FORMAT_E16 ? kPanel * 2 : 0));
     const size_t rows = static_cast<size_t>(2) * H * 4;  // at most two router rows per CTA
     L.pref = take(pref > rows ? pref : rows);
     L.xq4 = take(static_cast<size_t>(H));
@@ -152,7 +163,8 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// kSign: the weights are 1-bit sign codes (else base-3 digits).  kSlotOrder:
+// kFmt: the weights' format (base-3 digits, 1-bit sign codes or two-level
+// scales).  kSlotOrder:
 // the down items go to the warps in slot order (at most two items per warp),
 // else by halves of a slot.  kShared: the layer's shared expert (8-bit
 // blocks) is computed in the same launch: its 32-row blocks of the shared
@@ -160,9 +172,11 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
 // units leave idle), and the CTAs with a panel of hidden add the panel's
 // rows of its down projection to y after the routed combine, with the
 // arithmetic of the shared expert's own kernels.
-template <bool kSign, bool kSlotOrder, bool kShared>
+template <int kFmt, bool kSlotOrder, bool kShared>
 __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
-  constexpr int kWBytes = s1_word_bytes(kSign), kMat = s1_mat_bytes(kSign);
+  constexpr bool kSign = kFmt == MOE_FORMAT_SIGN, kE16 = kFmt == MOE_FORMAT_E16;
+  static_assert(!kE16 || kSlotOrder, "two-level scales take the down items in slot order");
+  constexpr int kWBytes = s1_word_bytes(kFmt), kMat = s1_mat_bytes(kFmt);
   constexpr int kWords = kSign ? kSignWords : kBlockWords;
   extern __shared__ __align__(1024) unsigned char smem[];
   const Decode2Params& D = S1.D;
@@ -171,7 +185,7 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   const int nbH = H / kBlock, nbF = F / kBlock;
   const int C = gridDim.x, c = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Step1Layout L = step1_layout(H, F, E, K, kSign);
+  const Step1Layout L = step1_layout(H, F, E, K, kFmt);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L.flag);
   uint64_t* pbar = reinterpret_cast<uint64_t*>(smem + L.flag + 16);
   int* sq4 = reinterpret_cast<int*>(smem + L.xq4);
@@ -339,7 +353,7 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
   const int panelH = c;  // C >= hidden/32: at most one panel per CTA
   const bool has_panel = panelH < H / kPanel;
   unsigned char* pref = smem + L.pref;
-  const size_t pref_slot = static_cast<size_t>(nbF) * kMat;
+  const size_t pref_slot = static_cast<size_t>(nbF) * kMat + (kE16 ? kPanel * 2 : 0);  // E16: + the rows' anchors
   // gate/up: units (slot, 32-row panel of ffn); stream h of this CTA takes
   // every other unit of the CTA's list, the blocks of hidden of a unit split
   // over the stream's warps
@@ -381,12 +395,17 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
           unsigned char* dst = myring + slot * kSlotBytes;
           if (e >= 0 && e < E) {
             const size_t pb = (static_cast<size_t>(e) * panels + static_cast<size_t>(iu % panels)) * nbH + ib;
-            const uint32_t tb = kWBytes, sb = kPanel * 2;
+            const uint32_t tb = kWBytes, sb = kMat - kWBytes;
+            // after the words: the block scales, or the sub-scale code words
+            const void* gtail = kE16 ? static_cast<const void*>(P.gate_codes + pb * kE16Words * kPanel)
+                                     : static_cast<const void*>(P.gate_scales + pb * kPanel);
+            const void* utail = kE16 ? static_cast<const void*>(P.up_codes + pb * kE16Words * kPanel)
+                                     : static_cast<const void*>(P.up_scales + pb * kPanel);
             mbar_arrive_expect_tx(mybar + slot, 2 * (tb + sb));
             bulk_g2s(dst, P.gate_trits + pb * kWords * kPanel, tb, mybar + slot, pol);
-            bulk_g2s(dst + tb, P.gate_scales + pb * kPanel, sb, mybar + slot, pol);
+            bulk_g2s(dst + tb, gtail, sb, mybar + slot, pol);
             bulk_g2s(dst + kMat, P.up_trits + pb * kWords * kPanel, tb, mybar + slot, pol);
-            bulk_g2s(dst + kMat + tb, P.up_scales + pb * kPanel, sb, mybar + slot, pol);
+            bulk_g2s(dst + kMat + tb, utail, sb, mybar + slot, pol);
           } else {
             mbar_arrive(mybar + slot);
           }
@@ -403,10 +422,19 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       const size_t pb0 = (static_cast<size_t>(sel_e[j]) * (H / kPanel) + panelH) * nbF;
       unsigned char* dst = pref + j * pref_slot;
       const uint32_t tb = static_cast<uint32_t>(nbF) * kWBytes;
-      const uint32_t sb = static_cast<uint32_t>(nbF) * kPanel * 2;
-      mbar_arrive_expect_tx(pbar, tb + sb);
-      bulk_g2s(dst, P.down_trits + pb0 * kWords * kPanel, tb, pbar, policy_evict_first());
-      bulk_g2s(dst + tb, P.down_scales + pb0 * kPanel, sb, pbar, policy_evict_first());
+      const uint32_t sb = static_cast<uint32_t>(nbF) * (kMat - kWBytes);
+      if constexpr (kE16) {
+        // words, sub-scale codes, then the panel rows' fp16 anchors
+        mbar_arrive_expect_tx(pbar, tb + sb + kPanel * 2);
+        bulk_g2s(dst, P.down_trits + pb0 * kWords * kPanel, tb, pbar, policy_evict_first());
+        bulk_g2s(dst + tb, P.down_codes + pb0 * kE16Words * kPanel, sb, pbar, policy_evict_first());
+        bulk_g2s(dst + tb + sb, P.down_scales + static_cast<size_t>(sel_e[j]) * H + static_cast<size_t>(panelH) * kPanel,
+                 kPanel * 2, pbar, policy_evict_first());
+      } else {
+        mbar_arrive_expect_tx(pbar, tb + sb);
+        bulk_g2s(dst, P.down_trits + pb0 * kWords * kPanel, tb, pbar, policy_evict_first());
+        bulk_g2s(dst + tb, P.down_scales + pb0 * kPanel, sb, pbar, policy_evict_first());
+      }
     }
     if constexpr (kShared) {
       // this panel's rows of the shared expert's down projection, for phase C
@@ -422,20 +450,46 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       const int64_t u = my_unit(ui);
       const int j = static_cast<int>(u / panels), p = static_cast<int>(u % panels);
       float part[2][1] = {{0.f}, {0.f}};
+      // two-level scales: the rows' anchors / 16 (loaded now, used at the
+      // unit's end) and one fp32 chain over the warp's blocks, as the grouped
+      // E16 gate/up kernel keeps
+      float a16[2] = {0.f, 0.f}, tot[2] = {0.f, 0.f};
+      if constexpr (kE16) {
+        const int e = sel_e[j];
+        if (e >= 0 && e < E) {
+          const size_t row = static_cast<size_t>(e) * F + static_cast<size_t>(p) * kPanel + lane;
+          a16[0] = f16_bits_to_f32(P.gate_scales[row]) * 0.0625f;
+          a16[1] = f16_bits_to_f32(P.up_scales[row]) * 0.0625f;
+        }
+      }
       for (int b = w8; b < nbH; b += kNC, ++s) {
         const int slot = s % SW;
         if (!mbar_wait_sleep(mybar + slot, static_cast<uint32_t>(s / SW) & 1u) && lane == 0) {
           record_status(P.status, MOE_ERR_TIMEOUT);
           *abort = 1;
         }
-        if constexpr (kSign)
+        if constexpr (kE16) {
+          int isum[2][kSubPerBlock];
+          block_isums_e16<2>(myring + slot * kSlotBytes, kMat, kWBytes, sq4 + b * (kBlock / 4), lane, isum);
+#pragma unroll
+          for (int sb = 0; sb < kSubPerBlock; ++sb) {
+            const float dn = sxd[b * kSubPerBlock + sb];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) tot[m] = __fmaf_rn(dn, static_cast<float>(isum[m][sb]), tot[m]);
+          }
+        } else if constexpr (kSign) {
           block_dot_sign<2>(myring + slot * kSlotBytes, kMat, kWBytes, sq4 + b * (kBlock / 4), sxd + b * kSubPerBlock,
                             sxas + b * kSubPerBlock, lane, part);
-        else
+        } else {
           block_dot<2, 1, 1>(myring + slot * kSlotBytes, sq4 + b * (kBlock / 4), 0, sxd + b * kSubPerBlock,
                              sxas + b * kSubPerBlock, 0, lane, part);
+        }
         __syncwarp();
         issue_next(slot);
+      }
+      if constexpr (kE16) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m) part[m][0] = __fmaf_rn(a16[m], tot[m], 0.f);
       }
       // unit ui's epilogue runs on warp ui % kNC of the stream, which waits
       // for the stream's sums; the other warps leave theirs and go on with
@@ -607,20 +661,31 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
         }
         __syncwarp();
         const unsigned char* wj = wbase + j * pref_slot;
-        // block b's words, then (after every block's words) its scales
-        const int scale_off = nbF * kWBytes + b * kPanel * 2 - b * kWBytes;
-        float inner[1][1];
-        float sc[1];
-        if constexpr (kSign)
-          block_dot_sign<1, true>(wj + static_cast<size_t>(b) * kWBytes, kMat, scale_off,
-                                  aq4 + j * (F / 4) + b * (kBlock / 4), ad + j * (F / kQBlock) + b * kSubPerBlock,
-                                  aas + j * (F / kQBlock) + b * kSubPerBlock, lane, inner, sc);
-        else
-          block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kWBytes, aq4 + j * (F / 4) + b * (kBlock / 4), 0,
-                                   ad + j * (F / kQBlock) + b * kSubPerBlock,
-                                   aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, scale_off, sc);
-        sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
-        sscale[(j * nbF + b) * kPanel + lane] = sc[0];
+        // block b's words, then (after every block's words) its scales or
+        // sub-scale code words
+        const int tail_off = nbF * kWBytes + b * (kMat - kWBytes) - b * kWBytes;
+        if constexpr (kE16) {
+          // the block's 8 integer sums; warp j chains them with the scales
+          int isum[1][kSubPerBlock];
+          block_isums_e16<1>(wj + static_cast<size_t>(b) * kWBytes, kMat, tail_off,
+                             aq4 + j * (F / 4) + b * (kBlock / 4), lane, isum);
+          int* sacc = reinterpret_cast<int*>(sinner);  // [K][nbF][8][32]
+#pragma unroll
+          for (int sb = 0; sb < kSubPerBlock; ++sb) sacc[((j * nbF + b) * kSubPerBlock + sb) * kPanel + lane] = isum[0][sb];
+        } else {
+          float inner[1][1];
+          float sc[1];
+          if constexpr (kSign)
+            block_dot_sign<1, true>(wj + static_cast<size_t>(b) * kWBytes, kMat, tail_off,
+                                    aq4 + j * (F / 4) + b * (kBlock / 4), ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                    aas + j * (F / kQBlock) + b * kSubPerBlock, lane, inner, sc);
+          else
+            block_dot<1, 1, 1, true>(wj + static_cast<size_t>(b) * kWBytes, aq4 + j * (F / 4) + b * (kBlock / 4), 0,
+                                     ad + j * (F / kQBlock) + b * kSubPerBlock,
+                                     aas + j * (F / kQBlock) + b * kSubPerBlock, 0, lane, inner, tail_off, sc);
+          sinner[(j * nbF + b) * kPanel + lane] = inner[0][0];
+          sscale[(j * nbF + b) * kPanel + lane] = sc[0];
+        }
       }
     } else {
       const int j = warp % kNC, half = warp / kNC;
@@ -698,7 +763,7 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
       // fewer), before the CTA-wide barrier.
       if (ok && warp >= kNC) {
         const int Fs = S1.S.ffn, nbs = Fs / kQBlock;
-        int* saq = reinterpret_cast<int*>(smem + L.inner + static_cast<size_t>(2) * K * nbF * kPanel * 4);  // [nbs][8]
+        int* saq = reinterpret_cast<int*>(smem + L.inner + static_cast<size_t>(s1_item_words(kFmt)) * K * nbF * kPanel * 4);  // [nbs][8]
         float* sad = reinterpret_cast<float*>(saq + kMaxSharedUnits * (kPanel / 4));                      // [nbs]
         if (warp == kNC && !*abort) {
           const uint32_t tag = *sgen;
@@ -774,8 +839,22 @@ __global__ void __launch_bounds__(kS1Warps * 32, 1) k_step1(Step1Params S1) {
     float* spart = reinterpret_cast<float*>(smem + L.red);  // [K][32]; the gate/up sums are done with it
     if (!*abort && ok && warp < K) {
       float part = 0.f;
-      for (int b = 0; b < nbF; ++b)
-        part = __fmaf_rn(sscale[(warp * nbF + b) * kPanel + lane], sinner[(warp * nbF + b) * kPanel + lane], part);
+      if constexpr (kE16) {
+        // one fp32 chain over every sub-block of the row, then the row's
+        // anchor / 16 (the grouped E16 down kernel's order)
+        const int* sacc = reinterpret_cast<const int*>(sinner);
+        float tot = 0.f;
+        for (int b = 0; b < nbF; ++b)
+#pragma unroll
+          for (int sb = 0; sb < kSubPerBlock; ++sb)
+            tot = __fmaf_rn(ad[warp * (F / kQBlock) + b * kSubPerBlock + sb],
+                            static_cast<float>(sacc[((warp * nbF + b) * kSubPerBlock + sb) * kPanel + lane]), tot);
+        const uint16_t* anc = reinterpret_cast<const uint16_t*>(pref + warp * pref_slot + static_cast<size_t>(nbF) * kMat);
+        part = __fmaf_rn(f16_bits_to_f32(anc[lane]) * 0.0625f, tot, 0.f);
+      } else {
+        for (int b = 0; b < nbF; ++b)
+          part = __fmaf_rn(sscale[(warp * nbF + b) * kPanel + lane], sinner[(warp * nbF + b) * kPanel + lane], part);
+      }
       spart[warp * kPanel + lane] = part;
     }
     __syncthreads();
@@ -793,8 +872,8 @@ bool step1_supported(const DecodeParams& P, int n_sm, size_t* smem) {
   if (P.hidden / kPanel > n_sm) return false;
   if (P.n_experts > 2 * n_sm) return false;  // at most two router rows per CTA
   if (P.n_experts > kS1MaxE) return false;
-  if (P.format != MOE_FORMAT_TERNARY && P.format != MOE_FORMAT_SIGN) return false;
-  const Step1Layout L = step1_layout(P.hidden, P.ffn, P.n_experts, P.top_k, P.format == MOE_FORMAT_SIGN);
+  if (P.format != MOE_FORMAT_TERNARY && P.format != MOE_FORMAT_SIGN && P.format != MOE_FORMAT_E16) return false;
+  const Step1Layout L = step1_layout(P.hidden, P.ffn, P.n_experts, P.top_k, P.format);
   *smem = L.total;
   return L.total <= static_cast<size_t>(kMaxDynSmem);
 }
@@ -805,14 +884,17 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !done[dev].load(std::memory_order_relaxed)) {
-    const void* ks[] = {reinterpret_cast<const void*>(&k_step1<false, false, false>),
-                        reinterpret_cast<const void*>(&k_step1<true, false, false>),
-                        reinterpret_cast<const void*>(&k_step1<false, true, false>),
-                        reinterpret_cast<const void*>(&k_step1<true, true, false>),
-                        reinterpret_cast<const void*>(&k_step1<false, false, true>),
-                        reinterpret_cast<const void*>(&k_step1<true, false, true>),
-                        reinterpret_cast<const void*>(&k_step1<false, true, true>),
-                        reinterpret_cast<const void*>(&k_step1<true, true, true>)};
+    constexpr int T = MOE_FORMAT_TERNARY, Sg = MOE_FORMAT_SIGN, E6 = MOE_FORMAT_E16;
+    const void* ks[] = {reinterpret_cast<const void*>(&k_step1<T, false, false>),
+                        reinterpret_cast<const void*>(&k_step1<Sg, false, false>),
+                        reinterpret_cast<const void*>(&k_step1<T, true, false>),
+                        reinterpret_cast<const void*>(&k_step1<Sg, true, false>),
+                        reinterpret_cast<const void*>(&k_step1<E6, true, false>),
+                        reinterpret_cast<const void*>(&k_step1<T, false, true>),
+                        reinterpret_cast<const void*>(&k_step1<Sg, false, true>),
+                        reinterpret_cast<const void*>(&k_step1<T, true, true>),
+                        reinterpret_cast<const void*>(&k_step1<Sg, true, true>),
+                        reinterpret_cast<const void*>(&k_step1<E6, true, true>)};
     for (const void* k : ks) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
     done[dev].store(true, std::memory_order_relaxed);
   }
@@ -840,12 +922,19 @@ int launch_step1(const Decode2Params& D, unsigned long long* ticket, unsigned lo
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_ok[di] >= 0 ? 2 : 1;
-  const bool sign = D.P.format == MOE_FORMAT_SIGN;
-  const bool slot_order = D.P.top_k * (D.P.ffn / kBlock) <= 2 * kS1Warps;
-  auto kern = shared ? (sign ? (slot_order ? k_step1<true, true, true> : k_step1<true, false, true>)
-                             : (slot_order ? k_step1<false, true, true> : k_step1<false, false, true>))
-                      : (sign ? (slot_order ? k_step1<true, true, false> : k_step1<true, false, false>)
-                              : (slot_order ? k_step1<false, true, false> : k_step1<false, false, false>));
+  // two-level scales always take the down items in slot order (their
+  // per-block results are integer sums that one warp per slot chains)
+  const int fmt = D.P.format;
+  const bool slot_order = fmt == MOE_FORMAT_E16 || D.P.top_k * (D.P.ffn / kBlock) <= 2 * kS1Warps;
+  constexpr int T = MOE_FORMAT_TERNARY, Sg = MOE_FORMAT_SIGN, E6 = MOE_FORMAT_E16;
+  void (*kern)(Step1Params) = nullptr;
+  if (fmt == E6) kern = shared ? k_step1<E6, true, true> : k_step1<E6, true, false>;
+  else if (fmt == Sg)
+    kern = shared ? (slot_order ? k_step1<Sg, true, true> : k_step1<Sg, false, true>)
+                  : (slot_order ? k_step1<Sg, true, false> : k_step1<Sg, false, false>);
+  else
+    kern = shared ? (slot_order ? k_step1<T, true, true> : k_step1<T, false, true>)
+                  : (slot_order ? k_step1<T, true, false> : k_step1<T, false, false>);
   cudaError_t err = cudaLaunchKernelEx(&cfg, kern, S);
   if (err != cudaSuccess && cfg.numAttrs == 2 && pdl_ok[di] == 0) {
     cudaGetLastError();

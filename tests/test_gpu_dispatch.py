@@ -24,7 +24,7 @@ def _names(B, fn):
     ("ternary", 16, ["route_group", "gateup", "down"]),
     ("sign", 1, ["step1"]),
     ("sign", 3, ["route_group", "gateup", "down"]),
-    ("e16", 1, ["route_group", "gateup", "down"]),
+    ("e16", 1, ["step1"]),
     ("e16", 3, ["route_group", "gateup", "down"]),
 ])
 def test_forward_kernels(fmt, ntok, expect):

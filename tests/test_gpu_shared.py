@@ -106,6 +106,7 @@ def _names(B, fn):
     ("tiny", "sign", 1, 2048),      # the most shared blocks the step takes (64)
     ("large", "ternary", 1, 1024),  # half-slot down items
     ("30b", "sign", 1, 96),
+    ("30b", "e16", 1, 768),        # two-level scales in the step
     ("30b", "ternary", 3, 768),     # more tokens: the routed kernels, then the shared expert's
     ("tiny", "ternary", 1, 2080),   # more than 64 blocks: moe_forward, then the shared expert's
 ])
