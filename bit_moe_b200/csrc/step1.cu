@@ -94,10 +94,10 @@ struct Step1Layout {
 // Shared-memory plan of one CTA.  x in fp32, the logits and the down
 // activations alias the gate/up ring (which is used only between them); the
 // router rows alias the down prefetch area.  Three ring slots per warp where
-// they fit, else two.
+// they fit, else two, else one (two-level scales at the largest shapes).
 __host__ __device__ inline Step1Layout step1_layout(int H, int F, int E, int K, int fmt) {
   Step1Layout L{};
-  for (int sw = 3; sw >= 2; --sw) {
+  for (int sw = 3; sw >= 1; --sw) {
     L = Step1Layout{};
     L.sw = sw;
     size_t off = 0;

@@ -89,6 +89,8 @@ WORKLOADS = {
                         fmt="e16"),
     "large-e16-b8": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 8, 0.015, layers=5,
                              seed=8, fmt="e16"),
+    "large-e16": Workload("moe-h4096-f2048-e256-k8", 4096, 2048, 256, 8, 1, 0.015, layers=6,
+                          seed=8, fmt="e16"),
     # the 30B-class layer with a shared expert (ffn 768, 8-bit blocks) beside the routed ones
     "30b-shared": Workload("moe-h2048-f768-e128-k8", 2048, 768, 128, 8, 1, 0.02, layers=4, seed=1,
                            shared_ffn=768),

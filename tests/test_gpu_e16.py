@@ -93,11 +93,11 @@ def test_e16_layer_30b(orc, ntok):
     assert rel_err_rms(y, ref) <= LAYER_TOL
 
 
-@pytest.mark.parametrize("ntok", [8])
+@pytest.mark.parametrize("ntok", [1, 8])
 def test_e16_layer_large(orc, ntok):
-    """The large layer (hidden 4096, ffn 2048, 256 experts, top-8) at 8
-    tokens, the shape the benchmark times: every token, two at a time through
-    the oracle."""
+    """The large layer (hidden 4096, ffn 2048, 256 experts, top-8) at 1 token
+    (the one-token step with one ring slot per warp) and 8 tokens, the shape
+    the benchmark times: every token, two at a time through the oracle."""
     y, ref = _layer_parity(orc, synthetic.WORKLOADS["large"], ntok, 54, np.arange(ntok), chunk=2)
     assert rel_err_rms(y, ref) <= LAYER_TOL
 
@@ -110,6 +110,20 @@ def test_e16_batch_equals_single_tokens():
     x = synthetic.activations(wl, 53, ntok=5, device="cuda")
     yb = B.moe_forward(layer, wr, x, B.Workspace.for_layer(layer, 5)).cpu().numpy()
     for t in range(5):
+        ys = B.moe_forward(layer, wr, x[t:t + 1].contiguous(), B.Workspace.for_layer(layer, 1)).cpu().numpy()
+        assert np.array_equal(ys[0], yb[t])
+
+
+def test_e16_large_batch_equals_single_tokens():
+    """The large layer: 3 tokens through the grouped kernels, each bit for bit
+    the same token alone through the one-token step."""
+    B = bm()
+    wl = synthetic.WORKLOADS["large"]
+    layer, _ = gpu_layer(wl, fmt="e16")
+    wr = synthetic.router(wl, 0, "cuda")
+    x = synthetic.activations(wl, 55, ntok=3, device="cuda")
+    yb = B.moe_forward(layer, wr, x, B.Workspace.for_layer(layer, 3)).cpu().numpy()
+    for t in range(3):
         ys = B.moe_forward(layer, wr, x[t:t + 1].contiguous(), B.Workspace.for_layer(layer, 1)).cpu().numpy()
         assert np.array_equal(ys[0], yb[t])
 
