@@ -111,8 +111,10 @@ typedef struct {
  * hidden <= 16384, ffn <= 8192, 1 <= top_k <= min(n_experts, 32),
  * n_experts <= 1024.  All three formats run the decode path (up to 64
  * tokens) and the prefill GEMM (moe_expert_ffn_prefill, moe_forward of more
- * than 64 tokens); the one-token fused step takes ternary and sign-code
- * layers (two-level scales take the four-kernel decode chain for one token). */
+ * than 64 tokens); the one-token fused step takes all three formats where
+ * its shared-memory plan fits one CTA (hidden <= 4096, ffn <= 2048, top_k <=
+ * 8, at most 2 experts per SM); other one-token shapes take the decode
+ * chains. */
 typedef struct {
   int32_t hidden, ffn, n_experts, top_k;
   moe_tmat gate, up, down;
@@ -235,9 +237,12 @@ int moe_expert_ffn_prefill(const moe_layer* layer, int32_t ntok, const int8_t* x
 
 /* ---- the whole step ------------------------------------------------------
  * S1 + S2 + (S3-S5 or S7): y [ntok][hidden] = MoE(x [ntok][hidden]).  Uses
- * the decode path for ntok <= 64 and the prefill path above.  x and y are
- * device pointers; the quantized x, the routing and the intermediates live
- * in the workspace.                                                        */
+ * the decode path for ntok <= 64 and the prefill path above: one token runs
+ * as one cooperative kernel (the one-token step) where the layer's shape
+ * allows, 2..64 tokens as three kernels (routing with the activation
+ * quantization and the grouping in one launch, then the grouped gate/up and
+ * down mat-vecs).  x and y are device pointers; the quantized x, the routing
+ * and the intermediates live in the workspace.                             */
 int moe_forward(const moe_layer* layer, const float* w_router, int32_t ntok, const float* x,
                 float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
 /* The same with x and y in HOST memory (pinned for asynchronous copies):
