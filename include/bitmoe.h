@@ -112,9 +112,9 @@ typedef struct {
  * n_experts <= 1024.  All three formats run the decode path (up to 64
  * tokens) and the prefill GEMM (moe_expert_ffn_prefill, moe_forward of more
  * than 64 tokens); the one-token fused step takes all three formats where
- * its shared-memory plan fits one CTA (hidden <= 4096, ffn <= 2048, top_k <=
- * 8, at most 2 experts per SM); other one-token shapes take the decode
- * chains. */
+ * its shared-memory plan fits one CTA (hidden <= 4096 and at most one
+ * 32-row panel of hidden per SM, ffn <= 2048, top_k <= 8, n_experts <= 256
+ * and at most two per SM); other one-token shapes take the decode chains. */
 typedef struct {
   int32_t hidden, ffn, n_experts, top_k;
   moe_tmat gate, up, down;
