@@ -26,6 +26,17 @@ def test_kernel_bytes_scale_with_unique_experts():
     assert b["down"] - a["down"] == 10 * wl.matrix_bytes(wl.hidden, wl.ffn)
 
 
+def test_kernel_bytes_of_the_step_with_a_shared_expert():
+    """One token with a shared expert runs as the one-token step alone, so its
+    algorithmic bytes are the routed step's plus the shared expert's 8-bit
+    weights (three matrices of hidden x ffn_s, 34 bytes per 32) and its
+    tagged block words (written and read)."""
+    plain, shared = synthetic.WORKLOADS["30b"], synthetic.WORKLOADS["30b-shared"]
+    a, b = bench.kernel_bytes(plain, 8.0), bench.kernel_bytes(shared, 8.0)
+    H, Fs = shared.hidden, shared.shared_ffn
+    assert b["step1"] - a["step1"] == 3 * H * Fs * 34 // 32 + Fs // 32 * 10 * 8 * 2
+
+
 def test_code_hash_ignores_comments(tmp_path, monkeypatch):
     csrc = tmp_path / "bit_moe_b200" / "csrc"
     csrc.mkdir(parents=True)
